@@ -1,0 +1,208 @@
+/*
+ * oracle.c -- plain, slow fp64 CPU oracle for blockwise softmax attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, includes or
+ * calls this file; only the test suite, the package smoke check and the CPU
+ * baseline leg of the benchmark load it (through oracle/__init__.py).  It shares
+ * no code, header, table or constant with the CUDA path.
+ *
+ * What it computes follows "上下文并行与 Ring Attention" (hs-black.github.io),
+ * section 分块注意力 (online softmax 与 log-sum-exp 合并):
+ *   - the attention output of one query against a key set is the plain softmax
+ *     average  o = sum_j softmax(x)_j v_j  with  x_j = q.k_j / sqrt(d_h)
+ *     (scale passed in by the caller);
+ *   - the per-block statistics m_b = max x_j, l_b = sum e^{x_j - m_b},
+ *     o_b = (1/l_b) sum e^{x_j - m_b} v_j, and lse_b = m_b + log l_b (natural log);
+ *   - the merge of two partials, in the stable form given right after the boxed
+ *     identity: M = max(lse_1, lse_2), lse = M + log(e^{lse_1-M} + e^{lse_2-M}),
+ *     o = e^{lse_1-lse} o_1 + e^{lse_2-lse} o_2.
+ * The causal mask is judged on original token positions (same page, sections
+ * 因果掩码带来的负载不均 and 重排 token 的代价): key t is visible to query p iff
+ * pos_k(t) <= pos_q(p).  The GQA head map is kv_head = q_head / (Hq / Hkv).
+ *
+ * Readings taken where the page is silent: a query that sees no key in the
+ * given set gets o = 0 and lse = -inf; merging two such partials gives (0, -inf).
+ *
+ * Everything is scalar fp64, sequential summation in key order, no blocking and
+ * no reordering; threads only split independent query rows.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* One query row against all keys of one kv head.
+ *   q      : d values of the query
+ *   k, v   : key/value rows; row t starts at k + t * kv_row_stride
+ *   pos_k  : original position of each key (NULL means t)
+ *   x      : caller scratch of sk doubles
+ * Writes d outputs to o and returns lse. */
+static double attend_row(const double *q, int64_t pos_q, const double *k, const double *v,
+                         const int64_t *pos_k, int64_t sk, int64_t kv_row_stride, int64_t d,
+                         int causal, double scale, double *x, double *o)
+{
+    double m = -INFINITY;
+    int64_t nvis = 0;
+    for (int64_t t = 0; t < sk; ++t) {
+        int64_t pk = pos_k ? pos_k[t] : t;
+        if (causal && pk > pos_q) { x[t] = NAN; continue; }
+        const double *kr = k + t * kv_row_stride;
+        double dot = 0.0;
+        for (int64_t e = 0; e < d; ++e) dot += q[e] * kr[e];
+        x[t] = scale * dot;
+        if (x[t] > m) m = x[t];
+        ++nvis;
+    }
+    for (int64_t e = 0; e < d; ++e) o[e] = 0.0;
+    if (nvis == 0) return -INFINITY;
+    double l = 0.0;
+    for (int64_t t = 0; t < sk; ++t) {
+        if (isnan(x[t])) continue;
+        double w = exp(x[t] - m);
+        l += w;
+        const double *vr = v + t * kv_row_stride;
+        for (int64_t e = 0; e < d; ++e) o[e] += w * vr[e];
+    }
+    for (int64_t e = 0; e < d; ++e) o[e] /= l;
+    return m + log(l);
+}
+
+/* ------------------------------------------------------------------ full problem */
+
+typedef struct {
+    const double *q, *k, *v;
+    const int64_t *pos_q, *pos_k;
+    int64_t b, sq, sk, hq, hkv, d;
+    int causal;
+    double scale;
+    double *o, *lse;
+    /* row selection (rows mode) */
+    const int64_t *sel;  /* [n][3] = (batch, q head, query index) */
+    const double *q_sel; /* [n][d] */
+    int64_t nsel;
+    /* work split */
+    int64_t begin, end;
+} job_t;
+
+static void *full_worker(void *arg)
+{
+    job_t *j = (job_t *)arg;
+    double *x = (double *)malloc(sizeof(double) * (size_t)(j->sk > 0 ? j->sk : 1));
+    int64_t g = j->hq / j->hkv;
+    for (int64_t r = j->begin; r < j->end; ++r) {
+        /* r enumerates (batch, q head, query index) */
+        int64_t s = r % j->sq;
+        int64_t h = (r / j->sq) % j->hq;
+        int64_t bb = r / (j->sq * j->hq);
+        int64_t hk = h / g;
+        const double *qr = j->q + ((bb * j->sq + s) * j->hq + h) * j->d;
+        const double *kb = j->k + (bb * j->sk * j->hkv + hk) * j->d;
+        const double *vb = j->v + (bb * j->sk * j->hkv + hk) * j->d;
+        int64_t pq = j->pos_q ? j->pos_q[s] : s;
+        double *orow = j->o + ((bb * j->sq + s) * j->hq + h) * j->d;
+        j->lse[(bb * j->hq + h) * j->sq + s] =
+            attend_row(qr, pq, kb, vb, j->pos_k, j->sk, j->hkv * j->d, j->d, j->causal,
+                       j->scale, x, orow);
+    }
+    free(x);
+    return NULL;
+}
+
+static void *rows_worker(void *arg)
+{
+    job_t *j = (job_t *)arg;
+    double *x = (double *)malloc(sizeof(double) * (size_t)(j->sk > 0 ? j->sk : 1));
+    int64_t g = j->hq / j->hkv;
+    for (int64_t r = j->begin; r < j->end; ++r) {
+        int64_t bb = j->sel[3 * r + 0], h = j->sel[3 * r + 1], pq = j->sel[3 * r + 2];
+        int64_t hk = h / g;
+        const double *kb = j->k + (bb * j->sk * j->hkv + hk) * j->d;
+        const double *vb = j->v + (bb * j->sk * j->hkv + hk) * j->d;
+        j->lse[r] = attend_row(j->q_sel + r * j->d, pq, kb, vb, j->pos_k, j->sk, j->hkv * j->d,
+                               j->d, j->causal, j->scale, x, j->o + r * j->d);
+    }
+    free(x);
+    return NULL;
+}
+
+static int run_jobs(job_t *proto, int64_t nrows, int nthreads, void *(*fn)(void *))
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 1024) nthreads = 1024;
+    if (nrows < nthreads) nthreads = nrows > 0 ? (int)nrows : 1;
+    pthread_t th[1024];
+    job_t jobs[1024];
+    int64_t per = (nrows + nthreads - 1) / nthreads;
+    int started = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t] = *proto;
+        jobs[t].begin = t * per < nrows ? t * per : nrows;
+        jobs[t].end = (t + 1) * per < nrows ? (t + 1) * per : nrows;
+        if (nthreads == 1) { fn(&jobs[t]); continue; }
+        if (pthread_create(&th[t], NULL, fn, &jobs[t]) != 0) return -1;
+        ++started;
+    }
+    for (int t = 0; t < started; ++t) pthread_join(th[t], NULL);
+    return 0;
+}
+
+/* Attention of every query row against every key.
+ *   q [b, sq, hq, d], k/v [b, sk, hkv, d], o [b, sq, hq, d], lse [b, hq, sq]
+ *   pos_q [sq] / pos_k [sk]: original token positions (NULL = identity).
+ * Returns 0, or -1 on bad sizes / thread failure. */
+int oracle_attention(const double *q, const double *k, const double *v, const int64_t *pos_q,
+                     const int64_t *pos_k, int64_t b, int64_t sq, int64_t sk, int64_t hq,
+                     int64_t hkv, int64_t d, int causal, double scale, double *o, double *lse,
+                     int nthreads)
+{
+    if (b < 0 || sq < 0 || sk < 0 || hq <= 0 || hkv <= 0 || d <= 0 || hq % hkv) return -1;
+    job_t j;
+    memset(&j, 0, sizeof j);
+    j.q = q; j.k = k; j.v = v; j.pos_q = pos_q; j.pos_k = pos_k;
+    j.b = b; j.sq = sq; j.sk = sk; j.hq = hq; j.hkv = hkv; j.d = d;
+    j.causal = causal; j.scale = scale; j.o = o; j.lse = lse;
+    return run_jobs(&j, b * hq * sq, nthreads, full_worker);
+}
+
+/* Attention of selected query rows only (for sampled checks at full size).
+ *   sel [n][3] = (batch, q head, original query position); q_sel [n][d]
+ *   k/v [b, sk, hkv, d] with original key positions pos_k (NULL = identity)
+ *   o_sel [n][d], lse_sel [n]. */
+int oracle_attention_rows(const double *q_sel, const int64_t *sel, int64_t n, const double *k,
+                          const double *v, const int64_t *pos_k, int64_t b, int64_t sk,
+                          int64_t hq, int64_t hkv, int64_t d, int causal, double scale,
+                          double *o_sel, double *lse_sel, int nthreads)
+{
+    if (n < 0 || b <= 0 || sk < 0 || hq <= 0 || hkv <= 0 || d <= 0 || hq % hkv) return -1;
+    for (int64_t r = 0; r < n; ++r)
+        if (sel[3 * r] < 0 || sel[3 * r] >= b || sel[3 * r + 1] < 0 || sel[3 * r + 1] >= hq)
+            return -1;
+    job_t j;
+    memset(&j, 0, sizeof j);
+    j.k = k; j.v = v; j.pos_k = pos_k;
+    j.b = b; j.sk = sk; j.hq = hq; j.hkv = hkv; j.d = d;
+    j.causal = causal; j.scale = scale; j.o = o_sel; j.lse = lse_sel;
+    j.sel = sel; j.q_sel = q_sel; j.nsel = n;
+    return run_jobs(&j, n, nthreads, rows_worker);
+}
+
+/* Merge of two partials (o_1, lse_1), (o_2, lse_2) for n rows of d values, stable form.
+ * Both partials empty (lse = -inf) gives o = 0, lse = -inf. */
+void oracle_lse_merge(int64_t n, int64_t d, const double *o1, const double *lse1, const double *o2,
+                      const double *lse2, double *o, double *lse)
+{
+    for (int64_t r = 0; r < n; ++r) {
+        double a = lse1[r], c = lse2[r];
+        double M = a > c ? a : c;
+        if (M == -INFINITY) {
+            lse[r] = -INFINITY;
+            for (int64_t e = 0; e < d; ++e) o[r * d + e] = 0.0;
+            continue;
+        }
+        double L = M + log(exp(a - M) + exp(c - M));
+        double w1 = exp(a - L), w2 = exp(c - L);
+        for (int64_t e = 0; e < d; ++e) o[r * d + e] = w1 * o1[r * d + e] + w2 * o2[r * d + e];
+        lse[r] = L;
+    }
+}
