@@ -1,0 +1,334 @@
+"""Benchmark: ring-attention forward TFLOP/s on effective (unmasked) FLOPs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--mode fused|stepwise]
+    python bench.py --impl reference ...     (the fp64 CPU oracle on a bounded row sample)
+
+One step = one cp_ring_attn_fwd over the whole workload (all N virtual ranks, all
+ring steps), inputs already permuted to rank-major order and resident in HBM.
+L2 is flushed (a 256 MiB write) before every timed step; each step is timed with
+CUDA events on the launching stream.  With --gpus N > 1 (torchrun) every rank
+runs its own instance of the workload (weak scaling, no collective on the data
+path); the time is the max over ranks.  Rank 0 prints one JSON line.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import cp_workloads as W  # noqa: E402
+
+METRIC = "ring-attn fwd TFLOP/s (causal, effective FLOPs) & % bf16 peak; merge GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_oracle_rate(w, seconds_target=12.0, seed=0):
+    """Times the fp64 oracle on a bounded sample of query rows of the workload.
+
+    Returns (TFLOP/s on effective FLOPs, description, threads used).  The rows are
+    exact answers (rows are independent), so the rate is the oracle's own."""
+    import numpy as np
+
+    import oracle
+    rng = np.random.default_rng(seed)
+    q, k, v = W.make_inputs(w)
+    k64 = k.float().numpy().astype(np.float64)
+    v64 = v.float().numpy().astype(np.float64)
+    threads = oracle.default_threads()
+
+    def run(n):
+        sel = np.stack([rng.integers(0, w.b, n), rng.integers(0, w.hq, n), rng.integers(0, w.S, n)], axis=1)
+        q_sel = np.stack([q[b, p, h].float().numpy() for b, h, p in sel]).astype(np.float64)
+        t0 = time.perf_counter()
+        oracle.attention_rows(q_sel, sel, k64, v64, w.causal, w.scale, w.hq, nthreads=threads)
+        dt = time.perf_counter() - t0
+        pairs = sum((int(p) + 1) if w.causal else w.S for _, _, p in sel)
+        return 4.0 * w.d * pairs / dt / 1e12, dt
+
+    _, dt = run(threads)
+    n = max(threads, int(threads * seconds_target / max(dt, 1e-3)))
+    n = min(n, 200000)
+    rate, dt = run(n)
+    return rate, "%d random query rows of %s (%.1f s of fp64 CPU work)" % (n, w.name, dt), threads
+
+
+def run_reference(args):
+    """The oracle as the reference arm, on the machine's host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = W.BY_NAME[args.workload]
+    per = []
+    desc = ""
+    threads = 0
+    for i in range(args.warmup + args.steps):
+        rate, desc, threads = cpu_oracle_rate(w, seconds_target=args.ref_seconds, seed=i)
+        if i >= args.warmup:
+            per.append(rate)
+    value = statistics.mean(per)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "ms_per_step": None,
+        "config": {"workload": w.name, "b": w.b, "S": w.S, "hq": w.hq, "hkv": w.hkv, "d": w.d,
+                   "layout": w.layout, "N": w.N, "causal": w.causal},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=W.BENCH_WORKLOAD, choices=sorted(W.BY_NAME))
+    ap.add_argument("--mode", default="fused", choices=["fused", "stepwise"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import context_attention_cp_b200 as cp
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    w = W.BY_NAME[args.workload]
+    peaks, peak_src = load_peaks()
+    q, k, v = W.make_inputs(w)
+    qd, kd, vd = (cp.layout_permute(t.to(dev), w.layout, w.N) for t in (q, k, v))
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.b, w.hq, w.S), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ws_bytes = cp.ring_workspace_bytes(w.layout, w.N, args.mode, 0 if w.dtype == "bf16" else 1,
+                                       w.b, w.S, w.hq, w.d)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        cp.ring_attn_fwd(qd, kd, vd, w.layout, w.N, w.causal, w.scale, o=o, lse=lse, mode=args.mode,
+                         workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    cp.stream_check()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    cp.stream_check()
+    times = [s.elapsed_time(e) for s, e in zip(starts, ends)]  # ms
+    total_ms = sum(times)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    flops = w.effective_flops()
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    launches_per_step = 1 if (args.mode == "fused" or w.N == 1) else (2 * w.N - 1)
+
+    # dominant kernel: the attention kernel (the whole fused ring is one launch)
+    per_launch_tflops = flops / (ms_per_step * 1e-3) / 1e12 if args.mode == "fused" else None
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+
+    # standalone merge bandwidth on this workload's partial size: (N-1) merges of
+    # [b, S, Hq, d] per ring, bytes per (row, head) = (8 + 2) * d + 12
+    merge = None
+    if w.dtype == "bf16" and rank == 0:
+        oa = torch.randn((w.b, w.S, w.hq, w.d), device=dev)
+        ob = torch.randn((w.b, w.S, w.hq, w.d), device=dev).to(torch.bfloat16)
+        la = torch.randn((w.b, w.hq, w.S), device=dev)
+        lb = torch.randn((w.b, w.hq, w.S), device=dev)
+        for _ in range(3):
+            cp.lse_merge(oa, la, ob, lb)
+        ms = []
+        for _ in range(10):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            cp.lse_merge(oa, la, ob, lb)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        rows = w.b * w.S * w.hq
+        mbytes = rows * ((8 + 2) * w.d + 12)
+        gbs = mbytes / (statistics.mean(ms) * 1e-3) / 1e9
+        merge = {"gbs": gbs, "frac_of_measured_hbm": gbs / peaks.get("hbm_gbs", 6650.0),
+                 "frac_of_8tbs": gbs / 8000.0, "bytes_per_launch": mbytes, "ms_per_launch": statistics.mean(ms)}
+        del oa, ob, la, lb
+
+    # end to end through the public API: host (pinned) -> device, permute, ring,
+    # unpermute, device -> host, every step
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    lh = torch.empty((w.b, w.hq, w.S), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        qg, kg, vg = (t.to(dev, non_blocking=True) for t in (qh, kh, vh))
+        qr, kr, vr = (cp.layout_permute(t, w.layout, w.N) for t in (qg, kg, vg))
+        og, lg = cp.ring_attn_fwd(qr, kr, vr, w.layout, w.N, w.causal, w.scale, mode=args.mode, workspace=ws)
+        og = cp.layout_permute(og, w.layout, w.N, inverse=True)
+        lg = cp.layout_permute(lg, w.layout, w.N, seq_axis=2, inverse=True)
+        oh.copy_(og, non_blocking=True)
+        lh.copy_(lg, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    e2e_value = world * flops * e_steps / (e_ms * 1e-3) / 1e12
+    es = 2 if w.dtype == "bf16" else 4
+    h2d = (q.numel() + k.numel() + v.numel()) * es
+    d2h = q.numel() * es + w.b * w.hq * w.S * 4
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc, threads = cpu_oracle_rate(w)
+        cpu = {"value": rate, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "b": w.b, "S": w.S, "hq": w.hq, "hkv": w.hkv, "d": w.d,
+                       "layout": w.layout, "N": w.N, "causal": w.causal, "mode": args.mode,
+                       "l2": "flushed before every timed step (256 MiB write)",
+                       "parallelism": "replicas x%d" % world},
+            "pct_bf16_peak": value / world / peak_tf,
+            "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel",
+                         "achieved": per_launch_tflops, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": (per_launch_tflops / peak_tf) if per_launch_tflops else None,
+                         "peak_source": peak_src + " bf16 burst", "traffic": None},
+            "merge": merge,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,21 @@
+"""Ring-scheduled blockwise softmax attention on one B200: Python binding of libcpattn.
+
+Argument marshalling only.  Every step of the path runs in the CUDA kernels of
+libcpattn.so (built in-tree by context_attention_cp_b200.build); if that library
+is missing the first call raises ImportError instead of computing anything.
+
+Entry points mirror include/cpattn.h:
+  block_attn_fwd(q, k, v, q_range, kv_range, causal, scale, o, lse, accumulate)
+  lse_merge(o_acc, lse_acc, o_b, lse_b, o_out=None)
+  ring_attn_fwd(q, k, v, layout, N, causal, scale, o=None, lse=None, mode="fused")
+  layout_permute(x, layout, N, seq_axis=1, inverse=False, out=None)
+  layout_range(layout, N, S, rank) -> (nseg, start, len, stride)
+  tile_classes(q_range, q_len, kv_range, kv_len, causal, tile_q, tile_k)
+  stream_check()
+Tensors are torch tensors on the current CUDA device; token tensors are
+[b, s, H, d] with d contiguous, lse tensors [b, H, s] fp32.
+"""
+from ._binding import (  # noqa: F401
+    CPError, LAYOUTS, MODES, block_attn_fwd, layout_permute, layout_range, lib, lib_path,
+    lse_merge, ring_attn_fwd, ring_workspace_bytes, stream_check, tile_classes,
+)

@@ -1,0 +1,202 @@
+"""ctypes marshalling between torch tensors and the libcpattn C ABI (include/cpattn.h)."""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libcpattn.so")
+
+CP_BF16, CP_FP32 = 0, 1
+LAYOUTS = {"contiguous": 0, "zigzag": 1, "striped": 2}
+MODES = {"fused": 0, "stepwise": 1}
+STATUS = {0: "CP_OK", 1: "CP_ERR_INVALID_ARG", 2: "CP_ERR_UNSUPPORTED", 3: "CP_ERR_SHAPE",
+          4: "CP_ERR_CUDA", 5: "CP_ERR_TIMEOUT"}
+
+
+class CPError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__("%s: %s" % (STATUS.get(code, code), msg))
+        self.code = code
+
+
+class CpTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+class CpRange(ctypes.Structure):
+    _fields_ = [("nseg", ctypes.c_int32), ("reserved", ctypes.c_int32), ("start", ctypes.c_int64 * 2),
+                ("len", ctypes.c_int64 * 2), ("stride", ctypes.c_int64)]
+
+
+_T = ctypes.POINTER(CpTensor)
+_R = ctypes.POINTER(CpRange)
+_i32, _i64, _vp, _f32, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
+
+_SIGNATURES = {
+    "cp_block_attn_fwd": (_i32, [_T, _T, _T, _R, _R, _i32, _f32, _T, _T, _i32, _vp]),
+    "cp_lse_merge": (_i32, [_T, _T, _T, _T, _T, _vp]),
+    "cp_ring_attn_fwd": (_i32, [_i32, _i32, _i32, _T, _T, _T, _f32, _T, _T, _i32, _vp, _sz, _vp]),
+    "cp_ring_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _i64]),
+    "cp_layout_permute": (_i32, [_i32, _i32, _i32, _T, _T, _i32, _vp]),
+    "cp_layout_range": (_i32, [_i32, _i32, _i64, _i32, _R]),
+    "cp_tile_classes": (_i32, [_R, _i64, _R, _i64, _i32, _i32, _i32, ctypes.POINTER(ctypes.c_int8)]),
+    "cp_stream_check": (_i32, [_vp]),
+    "cp_status_string": (ctypes.c_char_p, [_i32]),
+    "cp_last_error": (ctypes.c_char_p, []),
+    "cp_abi_version": (_i32, []),
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded libcpattn.so; raises ImportError if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(lib_path):
+            raise ImportError("libcpattn.so is not built; run python -m context_attention_cp_b200.build")
+        handle = ctypes.CDLL(lib_path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(code):
+    if code != 0:
+        msg = lib().cp_last_error().decode(errors="replace")
+        raise CPError(code, msg)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return CP_BF16
+    if t.dtype == torch.float32:
+        return CP_FP32
+    raise TypeError("unsupported dtype %s" % t.dtype)
+
+
+def _tensor(t, as4d=None):
+    """cp_tensor view of a CUDA tensor; 3-D lse tensors [b, H, s] become [b, H, s, 1]."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    shape, stride = list(t.shape), list(t.stride())
+    if t.dim() == 3:
+        shape, stride = shape + [1], stride + [1]
+    if len(shape) != 4:
+        raise ValueError("expected a 4-D token tensor or a 3-D lse tensor, got %s" % (tuple(t.shape),))
+    ct = CpTensor()
+    ct.data = t.data_ptr()
+    ct.dtype = _dtype_code(t)
+    for i in range(4):
+        ct.shape[i] = shape[i]
+        ct.stride[i] = stride[i]
+    return ct
+
+
+def _ref(x):
+    return ctypes.byref(x) if x is not None else None
+
+
+def _stream():
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _range(r):
+    """(starts, lens, stride) -> cp_range."""
+    starts, lens, stride = r
+    cr = CpRange()
+    cr.nseg = len(starts)
+    for i, (s, n) in enumerate(zip(starts, lens)):
+        cr.start[i] = s
+        cr.len[i] = n
+    cr.stride = stride
+    return cr
+
+
+def layout_range(layout, N, S, rank):
+    """Positions of rank `rank`'s tokens as (starts, lens, stride)."""
+    cr = CpRange()
+    _check(lib().cp_layout_range(LAYOUTS[layout], N, S, rank, ctypes.byref(cr)))
+    return tuple(cr.start[: cr.nseg]), tuple(cr.len[: cr.nseg]), cr.stride
+
+
+def tile_classes(q_range, q_len, kv_range, kv_len, causal, tile_q=128, tile_k=128):
+    """Per-tile classes (0 skip, 1 full, 2 partial) as a list of lists."""
+    n_qt = -(-q_len // tile_q)
+    n_kt = -(-kv_len // tile_k)
+    buf = (ctypes.c_int8 * max(1, n_qt * n_kt))()
+    qr, kr = _range(q_range), _range(kv_range)
+    _check(lib().cp_tile_classes(ctypes.byref(qr), q_len, ctypes.byref(kr), kv_len, int(bool(causal)),
+                                 tile_q, tile_k, buf))
+    return [[buf[i * n_kt + j] for j in range(n_kt)] for i in range(n_qt)]
+
+
+def block_attn_fwd(q, k, v, q_range, kv_range, causal, scale, o, lse, accumulate=False):
+    """One block partial (accumulate=False) or its fused merge into fp32 (o, lse)."""
+    qr, kr = _range(q_range), _range(kv_range)
+    tq, tk, tv, to, tl = _tensor(q), _tensor(k), _tensor(v), _tensor(o), _tensor(lse)
+    _check(lib().cp_block_attn_fwd(_ref(tq), _ref(tk), _ref(tv), ctypes.byref(qr), ctypes.byref(kr),
+                                   int(bool(causal)), float(scale), _ref(to), _ref(tl), int(bool(accumulate)),
+                                   _stream()))
+    return o, lse
+
+
+def lse_merge(o_acc, lse_acc, o_b, lse_b, o_out=None):
+    ta, tla, tb, tlb, tout = _tensor(o_acc), _tensor(lse_acc), _tensor(o_b), _tensor(lse_b), _tensor(o_out)
+    _check(lib().cp_lse_merge(_ref(ta), _ref(tla), _ref(tb), _ref(tlb), _ref(tout), _stream()))
+    return (o_out if o_out is not None else o_acc), lse_acc
+
+
+def ring_workspace_bytes(layout, N, mode, dtype_code, b, S, Hq, d):
+    return lib().cp_ring_workspace_bytes(LAYOUTS[layout], N, MODES[mode], dtype_code, b, S, Hq, d)
+
+
+def ring_attn_fwd(q, k, v, layout, N, causal, scale=None, o=None, lse=None, mode="fused", workspace=None):
+    """Ring attention over N virtual ranks; q/k/v/o/lse in rank-major order."""
+    import torch
+    b, S, Hq, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((b, Hq, S), dtype=torch.float32, device=q.device)
+    need = ring_workspace_bytes(layout, N, mode, _dtype_code(q), b, S, Hq, d)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = ctypes.c_void_p(workspace.data_ptr()) if (need and workspace is not None) else None
+    tq, tk, tv, to, tl = _tensor(q), _tensor(k), _tensor(v), _tensor(o), _tensor(lse)
+    _check(lib().cp_ring_attn_fwd(LAYOUTS[layout], N, int(bool(causal)), _ref(tq), _ref(tk), _ref(tv),
+                                  float(scale), _ref(to), _ref(tl), MODES[mode], ws_ptr, need, _stream()))
+    return o, lse
+
+
+def layout_permute(x, layout, N, seq_axis=1, inverse=False, out=None):
+    """Forward: rank-major copy of x.  Inverse: x is rank-major; returns original order."""
+    import torch
+    x = x.contiguous()
+    if out is None:
+        out = torch.empty_like(x)
+    if x.dim() == 3 and seq_axis == 2:
+        x4, o4 = x.unsqueeze(-1), out.unsqueeze(-1)
+    else:
+        x4, o4 = x, out
+    tx, to = _tensor(x4), _tensor(o4)
+    if inverse:
+        # the ABI writes the original-order tensor (its `x`) from the ranked one
+        _check(lib().cp_layout_permute(LAYOUTS[layout], N, seq_axis, _ref(to), _ref(tx), 1, _stream()))
+    else:
+        _check(lib().cp_layout_permute(LAYOUTS[layout], N, seq_axis, _ref(tx), _ref(to), 0, _stream()))
+    return out
+
+
+def stream_check():
+    """Synchronise the current stream and raise if a kernel reported a device-side error."""
+    _check(lib().cp_stream_check(_stream()))

@@ -1,0 +1,521 @@
+// abi.cu -- the C ABI of libcpattn (include/cpattn.h): argument checks, the ring
+// scheduler (work order and step launches) and dispatch to the kernels.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include "../../include/cpattn.h"
+#include "kernels.h"
+
+using namespace cpattn;
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+cp_status fail(cp_status s, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+cp_status cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(CP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int64_t elem_size(int32_t dt) { return dt == CP_BF16 ? 2 : (dt == CP_FP32 ? 4 : 0); }
+
+cp_status check_tensor(const cp_tensor *t, const char *name, bool need_data = true)
+{
+    if (!t) return fail(CP_ERR_INVALID_ARG, "%s is NULL", name);
+    if (need_data && !t->data) return fail(CP_ERR_INVALID_ARG, "%s->data is NULL", name);
+    if (t->dtype != CP_BF16 && t->dtype != CP_FP32) return fail(CP_ERR_INVALID_ARG, "%s has an unknown dtype", name);
+    for (int i = 0; i < 4; ++i)
+        if (t->shape[i] < 0 || t->stride[i] < 0) return fail(CP_ERR_INVALID_ARG, "%s has a negative size or stride", name);
+    if (t->stride[3] != 1 && t->shape[3] > 1) return fail(CP_ERR_INVALID_ARG, "%s: innermost stride must be 1", name);
+    return CP_OK;
+}
+
+// A token tensor [b, s, H, d] whose rows start on 16-byte boundaries.
+cp_status check_rows16(const cp_tensor *t, const char *name)
+{
+    const int64_t es = elem_size(t->dtype);
+    const int64_t per16 = 16 / es;
+    if (reinterpret_cast<uintptr_t>(t->data) % 16)
+        return fail(CP_ERR_INVALID_ARG, "%s->data must be 16-byte aligned", name);
+    for (int i = 0; i < 3; ++i)
+        if (t->shape[i] > 1 && t->stride[i] % per16)
+            return fail(CP_ERR_INVALID_ARG, "%s: stride[%d] must be a multiple of 16 bytes", name, i);
+    if ((t->shape[3] * es) % 16) return fail(CP_ERR_INVALID_ARG, "%s: rows must be a multiple of 16 bytes", name);
+    return CP_OK;
+}
+
+bool same_shape(const cp_tensor *a, const cp_tensor *b)
+{
+    for (int i = 0; i < 4; ++i)
+        if (a->shape[i] != b->shape[i]) return false;
+    return true;
+}
+
+Range to_range(const cp_range &r)
+{
+    Range x;
+    x.start0 = r.start[0];
+    x.len0 = r.len[0];
+    x.start1 = r.nseg == 2 ? r.start[1] : 0;
+    x.len1 = r.nseg == 2 ? r.len[1] : 0;
+    x.stride = r.stride;
+    return x;
+}
+
+cp_status check_range(const cp_range *r, int64_t len, const char *name)
+{
+    if (!r) return fail(CP_ERR_INVALID_ARG, "%s is NULL", name);
+    if (r->nseg != 1 && r->nseg != 2) return fail(CP_ERR_INVALID_ARG, "%s: nseg must be 1 or 2", name);
+    Range x = to_range(*r);
+    if (range_len(x) != len) return fail(CP_ERR_SHAPE, "%s covers %lld tokens, the tensor has %lld", name,
+                                         (long long)range_len(x), (long long)len);
+    if (!range_increasing(x) || x.start0 < 0)
+        return fail(CP_ERR_INVALID_ARG, "%s: positions must be >= 0 and increase with the local index", name);
+    return CP_OK;
+}
+
+void set_status_ptr(AttnParams &p)
+{
+    int *s = nullptr;
+    status_word(&s);
+    p.status = s;
+}
+
+void fill_inputs(AttnParams &p, const cp_tensor *q, const cp_tensor *k, const cp_tensor *v)
+{
+    p.q = q->data; p.k = k->data; p.v = v->data;
+    p.q_sb = q->stride[0]; p.q_ss = q->stride[1]; p.q_sh = q->stride[2];
+    p.k_sb = k->stride[0]; p.k_ss = k->stride[1]; p.k_sh = k->stride[2];
+    p.v_sb = v->stride[0]; p.v_ss = v->stride[1]; p.v_sh = v->stride[2];
+}
+
+void fill_outputs(AttnParams &p, int epi, const cp_tensor *o, const cp_tensor *lse)
+{
+    p.epi = epi;
+    p.o = o->data;
+    p.o_dtype = o->dtype;
+    p.o_sb = o->stride[0]; p.o_ss = o->stride[1]; p.o_sh = o->stride[2];
+    p.lse = static_cast<float *>(lse->data);
+    p.lse_sb = lse->stride[0]; p.lse_sh = lse->stride[1]; p.lse_ss = lse->stride[2];
+}
+
+cp_status launch_attn(const AttnParams &p, int32_t dtype, cudaStream_t stream)
+{
+    cudaError_t e = dtype == CP_BF16 ? launch_attn_tc(p, stream) : launch_attn_simt(p, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    return CP_OK;
+}
+
+// ---------------------------------------------------------------- ring scheduler
+
+// Work order for the ring: (rank, query tile) entries sorted by the number of key
+// tiles they visit over all steps, heaviest first, so the long causal rows start
+// early and the tail of the launch is made of short ones.
+struct OrderKey {
+    int layout, n, causal;
+    int64_t seq;
+    bool operator<(const OrderKey &o) const
+    {
+        return std::tie(layout, n, causal, seq) < std::tie(o.layout, o.n, o.causal, o.seq);
+    }
+};
+std::mutex g_order_mu;
+std::map<OrderKey, std::vector<uint32_t>> g_order_cache;
+
+const std::vector<uint32_t> &ring_order(int layout, int N, int64_t S, int causal)
+{
+    std::lock_guard<std::mutex> lk(g_order_mu);
+    OrderKey key{layout, N, causal, S};
+    auto it = g_order_cache.find(key);
+    if (it != g_order_cache.end()) return it->second;
+    const int64_t c = S / N;
+    const int n_qt = (int)((c + 127) / 128);
+    std::vector<std::pair<int64_t, uint32_t>> work;
+    work.reserve((size_t)N * n_qt);
+    for (int i = 0; i < N; ++i) {
+        Range qr = layout_range(layout, N, S, i);
+        for (int qt = 0; qt < n_qt; ++qt) {
+            int64_t tiles = 0;
+            for (int r = 0; r < N; ++r) {
+                Range kr = layout_range(layout, N, S, ((i - r) % N + N) % N);
+                int kf, ke;
+                kv_tile_bounds(qr, c, (int64_t)qt * 128, 128, kr, c, 128, causal != 0, &kf, &ke);
+                tiles += ke;
+            }
+            work.push_back({tiles, ((uint32_t)i << 16) | (uint32_t)qt});
+        }
+    }
+    std::stable_sort(work.begin(), work.end(),
+                     [](const std::pair<int64_t, uint32_t> &a, const std::pair<int64_t, uint32_t> &b) {
+                         return a.first > b.first;
+                     });
+    std::vector<uint32_t> out;
+    for (auto &w : work) out.push_back(w.second);
+    return g_order_cache.emplace(key, std::move(out)).first->second;
+}
+
+cp_status check_attn_dtypes(const cp_tensor *q, const cp_tensor *k, const cp_tensor *v)
+{
+    if (k->dtype != q->dtype || v->dtype != q->dtype)
+        return fail(CP_ERR_INVALID_ARG, "q, k and v must share one dtype");
+    const int64_t d = q->shape[3];
+    if (d != 64 && d != 128) return fail(CP_ERR_UNSUPPORTED, "head dim %lld is not supported (64 or 128)", (long long)d);
+    if (k->shape[3] != d || v->shape[3] != d) return fail(CP_ERR_SHAPE, "q, k, v head dims differ");
+    if (q->shape[0] != k->shape[0] || !same_shape(k, v)) return fail(CP_ERR_SHAPE, "q/k/v batch or k/v shapes differ");
+    if (q->shape[2] <= 0 || k->shape[2] <= 0 || q->shape[2] % k->shape[2])
+        return fail(CP_ERR_SHAPE, "query heads (%lld) must be a multiple of kv heads (%lld)", (long long)q->shape[2],
+                    (long long)k->shape[2]);
+    if (q->dtype == CP_BF16) {
+        cp_status s;
+        if ((s = check_rows16(q, "q")) != CP_OK || (s = check_rows16(k, "k")) != CP_OK ||
+            (s = check_rows16(v, "v")) != CP_OK)
+            return s;
+    }
+    return CP_OK;
+}
+
+cp_status check_out(const cp_tensor *o, const cp_tensor *lse, const cp_tensor *q, int64_t rows, bool need_fp32)
+{
+    cp_status s;
+    if ((s = check_tensor(o, "o")) != CP_OK || (s = check_tensor(lse, "lse")) != CP_OK) return s;
+    if (o->shape[0] != q->shape[0] || o->shape[1] != rows || o->shape[2] != q->shape[2] || o->shape[3] != q->shape[3])
+        return fail(CP_ERR_SHAPE, "o must be [b, s, Hq, d] like q");
+    if (need_fp32 && o->dtype != CP_FP32) return fail(CP_ERR_INVALID_ARG, "o must be fp32 when accumulating");
+    if (o->dtype != q->dtype && o->dtype != CP_FP32) return fail(CP_ERR_INVALID_ARG, "o must have q's dtype or fp32");
+    if (q->dtype == CP_FP32 && o->dtype != CP_FP32) return fail(CP_ERR_INVALID_ARG, "fp32 inputs give fp32 outputs");
+    if ((s = check_rows16(o, "o")) != CP_OK) return s;
+    if (lse->dtype != CP_FP32) return fail(CP_ERR_INVALID_ARG, "lse must be fp32");
+    if (lse->shape[0] != q->shape[0] || lse->shape[1] != q->shape[2] || lse->shape[2] != rows || lse->shape[3] != 1)
+        return fail(CP_ERR_SHAPE, "lse must be [b, Hq, s, 1]");
+    return CP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *cp_status_string(cp_status s)
+{
+    switch (s) {
+    case CP_OK: return "ok";
+    case CP_ERR_INVALID_ARG: return "invalid argument";
+    case CP_ERR_UNSUPPORTED: return "unsupported";
+    case CP_ERR_SHAPE: return "shape mismatch";
+    case CP_ERR_CUDA: return "CUDA error";
+    case CP_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+const char *cp_last_error(void) { return g_last_error; }
+
+int32_t cp_abi_version(void) { return 1; }
+
+cp_status cp_layout_range(int32_t layout, int32_t N, int64_t S, int32_t rank, cp_range *out)
+{
+    g_last_error[0] = 0;
+    if (!out) return fail(CP_ERR_INVALID_ARG, "out is NULL");
+    if (layout < 0 || layout > 2) return fail(CP_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (N < 1 || N > 65535 || S < 0 || S > INT32_MAX) return fail(CP_ERR_INVALID_ARG, "bad N or S");
+    if (S % N) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of N = %d", (long long)S, N);
+    if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N)) return fail(CP_ERR_SHAPE, "zig-zag needs S to be a multiple of 2N");
+    if (rank < 0 || rank >= N) return fail(CP_ERR_INVALID_ARG, "rank out of range");
+    Range r = layout_range(layout, N, S, rank);
+    out->nseg = r.len1 > 0 ? 2 : 1;
+    out->reserved = 0;
+    out->start[0] = r.start0;
+    out->start[1] = r.start1;
+    out->len[0] = r.len0;
+    out->len[1] = r.len1;
+    out->stride = r.stride;
+    return CP_OK;
+}
+
+cp_status cp_tile_classes(const cp_range *q_range, int64_t q_len, const cp_range *kv_range, int64_t kv_len,
+                          int32_t mask_mode, int32_t tile_q, int32_t tile_k, int8_t *out)
+{
+    g_last_error[0] = 0;
+    cp_status s;
+    if (!out) return fail(CP_ERR_INVALID_ARG, "out is NULL");
+    if (tile_q < 1 || tile_k < 1) return fail(CP_ERR_INVALID_ARG, "tile sizes must be positive");
+    if ((s = check_range(q_range, q_len, "q_range")) != CP_OK) return s;
+    if ((s = check_range(kv_range, kv_len, "kv_range")) != CP_OK) return s;
+    const Range qr = to_range(*q_range), kr = to_range(*kv_range);
+    const int64_t n_qt = (q_len + tile_q - 1) / tile_q, n_kt = (kv_len + tile_k - 1) / tile_k;
+    for (int64_t qt = 0; qt < n_qt; ++qt) {
+        int kf, ke;
+        kv_tile_bounds(qr, q_len, qt * tile_q, tile_q, kr, kv_len, tile_k, mask_mode == CP_MASK_CAUSAL, &kf, &ke);
+        for (int64_t kt = 0; kt < n_kt; ++kt)
+            out[qt * n_kt + kt] = (int8_t)(kt < kf ? TILE_FULL : (kt < ke ? TILE_PARTIAL : TILE_SKIP));
+    }
+    return CP_OK;
+}
+
+cp_status cp_block_attn_fwd(const cp_tensor *q, const cp_tensor *k, const cp_tensor *v, const cp_range *q_range,
+                            const cp_range *kv_range, int32_t mask_mode, float softmax_scale, cp_tensor *o,
+                            cp_tensor *lse, int32_t accumulate, void *stream)
+{
+    g_last_error[0] = 0;
+    cp_status s;
+    if ((s = check_tensor(q, "q")) != CP_OK || (s = check_tensor(k, "k")) != CP_OK ||
+        (s = check_tensor(v, "v")) != CP_OK)
+        return s;
+    if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
+    if (mask_mode != CP_MASK_NONE && mask_mode != CP_MASK_CAUSAL) return fail(CP_ERR_INVALID_ARG, "unknown mask mode");
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if (accumulate != 0 && accumulate != 1) return fail(CP_ERR_INVALID_ARG, "accumulate must be 0 or 1");
+    const int64_t sq = q->shape[1], sk = k->shape[1];
+    if (sq > INT32_MAX / 2 || sk > INT32_MAX / 2) return fail(CP_ERR_SHAPE, "sequence too long");
+    if ((s = check_out(o, lse, q, sq, accumulate == 1)) != CP_OK) return s;
+    if ((s = check_range(q_range, sq, "q_range")) != CP_OK) return s;
+    if ((s = check_range(kv_range, sk, "kv_range")) != CP_OK) return s;
+    if (q->shape[0] == 0 || sq == 0) return CP_OK;
+
+    thread_local AttnParams p;  // large (work-order table); built fresh below
+    std::memset(&p, 0, sizeof p);
+    p.b = (int)q->shape[0];
+    p.hq = (int)q->shape[2];
+    p.hkv = (int)k->shape[2];
+    p.group = p.hq / p.hkv;
+    p.d = (int)q->shape[3];
+    p.q_len = (int)sq;
+    p.kv_len = (int)sk;
+    p.n_ranks = 1;
+    p.step_begin = 0;
+    p.step_end = 1;
+    p.causal = mask_mode == CP_MASK_CAUSAL;
+    p.use_layout = 0;
+    p.q_range = to_range(*q_range);
+    p.kv_range = to_range(*kv_range);
+    p.scale = softmax_scale;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.n_qt = (int)((sq + 127) / 128);
+    if (p.n_qt > 65535) return fail(CP_ERR_SHAPE, "too many query tiles");
+    fill_inputs(p, q, k, v);
+    fill_outputs(p, accumulate ? EPI_MERGE : EPI_STORE, o, lse);
+    set_status_ptr(p);
+    return launch_attn(p, q->dtype, static_cast<cudaStream_t>(stream));
+}
+
+cp_status cp_lse_merge(cp_tensor *o_acc, cp_tensor *lse_acc, const cp_tensor *o_b, const cp_tensor *lse_b,
+                       cp_tensor *o_out, void *stream)
+{
+    g_last_error[0] = 0;
+    cp_status s;
+    if ((s = check_tensor(o_acc, "o_acc")) != CP_OK || (s = check_tensor(lse_acc, "lse_acc")) != CP_OK ||
+        (s = check_tensor(o_b, "o_b")) != CP_OK || (s = check_tensor(lse_b, "lse_b")) != CP_OK)
+        return s;
+    if (o_acc->dtype != CP_FP32) return fail(CP_ERR_INVALID_ARG, "o_acc must be fp32");
+    if (lse_acc->dtype != CP_FP32 || lse_b->dtype != CP_FP32) return fail(CP_ERR_INVALID_ARG, "lse must be fp32");
+    if (!same_shape(o_acc, o_b)) return fail(CP_ERR_SHAPE, "o_acc and o_b differ in shape");
+    const int64_t b = o_acc->shape[0], S = o_acc->shape[1], H = o_acc->shape[2], d = o_acc->shape[3];
+    if (!same_shape(lse_acc, lse_b) || lse_acc->shape[0] != b || lse_acc->shape[1] != H || lse_acc->shape[2] != S ||
+        lse_acc->shape[3] != 1)
+        return fail(CP_ERR_SHAPE, "lse tensors must be [b, H, s, 1]");
+    if (d % 8 || d > 256 || 32 % (d / 8))
+        return fail(CP_ERR_UNSUPPORTED, "d must be 8, 16, 32, 64, 128 or 256");
+    if ((s = check_rows16(o_acc, "o_acc")) != CP_OK || (s = check_rows16(o_b, "o_b")) != CP_OK) return s;
+    if (o_out) {
+        if ((s = check_tensor(o_out, "o_out")) != CP_OK) return s;
+        if (!same_shape(o_out, o_acc)) return fail(CP_ERR_SHAPE, "o_out differs in shape");
+        if ((s = check_rows16(o_out, "o_out")) != CP_OK) return s;
+    }
+    MergeParams p;
+    p.b = b; p.s = S; p.h = H; p.d = d;
+    p.o_acc = static_cast<float *>(o_acc->data);
+    p.oa_sb = o_acc->stride[0]; p.oa_ss = o_acc->stride[1]; p.oa_sh = o_acc->stride[2];
+    p.lse_acc = static_cast<float *>(lse_acc->data);
+    p.la_sb = lse_acc->stride[0]; p.la_sh = lse_acc->stride[1]; p.la_ss = lse_acc->stride[2];
+    p.o_b = o_b->data; p.ob_dtype = o_b->dtype;
+    p.ob_sb = o_b->stride[0]; p.ob_ss = o_b->stride[1]; p.ob_sh = o_b->stride[2];
+    p.lse_b = static_cast<const float *>(lse_b->data);
+    p.lb_sb = lse_b->stride[0]; p.lb_sh = lse_b->stride[1]; p.lb_ss = lse_b->stride[2];
+    p.o_out = o_out ? o_out->data : nullptr;
+    p.out_dtype = o_out ? o_out->dtype : CP_FP32;
+    p.out_sb = o_out ? o_out->stride[0] : 0; p.out_ss = o_out ? o_out->stride[1] : 0;
+    p.out_sh = o_out ? o_out->stride[2] : 0;
+    cudaError_t e = launch_lse_merge(p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+    return CP_OK;
+}
+
+size_t cp_ring_workspace_bytes(int32_t layout, int32_t N, int32_t mode, int32_t dtype, int64_t b, int64_t S,
+                               int64_t Hq, int64_t d)
+{
+    if (mode != CP_RING_STEPWISE) return 0;
+    if (layout < 0 || layout > 2 || N < 1 || b < 0 || S < 0 || Hq < 0 || d < 0) return 0;
+    if (N == 1) return 0;
+    const int64_t es = elem_size(dtype);
+    if (!es) return 0;
+    const int64_t rows = b * S * Hq;
+    // o_acc fp32, o_b in the input dtype, lse_b fp32; each region 256-byte aligned
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    return (size_t)(up(rows * d * 4) + up(rows * d * es) + up(rows * 4));
+}
+
+cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q, const cp_tensor *k,
+                           const cp_tensor *v, float softmax_scale, cp_tensor *o, cp_tensor *lse, int32_t mode,
+                           void *workspace, size_t workspace_bytes, void *stream)
+{
+    g_last_error[0] = 0;
+    cp_status s;
+    if (layout < 0 || layout > 2) return fail(CP_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (mode != CP_RING_FUSED && mode != CP_RING_STEPWISE) return fail(CP_ERR_INVALID_ARG, "unknown ring mode");
+    if (causal != 0 && causal != 1) return fail(CP_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if ((s = check_tensor(q, "q")) != CP_OK || (s = check_tensor(k, "k")) != CP_OK ||
+        (s = check_tensor(v, "v")) != CP_OK)
+        return s;
+    if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    const int64_t S = q->shape[1];
+    if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
+    if (N < 1 || N > 4096) return fail(CP_ERR_INVALID_ARG, "N must be in [1, 4096]");
+    if (S > INT32_MAX / 2) return fail(CP_ERR_SHAPE, "sequence too long");
+    if (S % N) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of N = %d", (long long)S, N);
+    if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N)) return fail(CP_ERR_SHAPE, "zig-zag needs S to be a multiple of 2N");
+    if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;
+    if (o->dtype != q->dtype) return fail(CP_ERR_INVALID_ARG, "o must have q's dtype");
+    const int64_t c = S / N;
+    if (q->shape[0] == 0 || S == 0) return CP_OK;
+    const int n_qt = (int)((c + 127) / 128);
+    if (n_qt > 65535) return fail(CP_ERR_SHAPE, "too many query tiles per rank");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    thread_local AttnParams p;
+    std::memset(&p, 0, sizeof p);
+    p.b = (int)q->shape[0];
+    p.hq = (int)q->shape[2];
+    p.hkv = (int)k->shape[2];
+    p.group = p.hq / p.hkv;
+    p.d = (int)q->shape[3];
+    p.q_len = (int)c;
+    p.kv_len = (int)c;
+    p.n_ranks = N;
+    p.causal = causal;
+    p.use_layout = 1;
+    p.layout = layout;
+    p.seq_len = S;
+    p.q_row_step = c;
+    p.kv_row_step = c;
+    p.scale = softmax_scale;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.n_qt = n_qt;
+    const std::vector<uint32_t> &ord = ring_order(layout, N, S, causal);
+    if ((int64_t)ord.size() <= kMaxOrder) {
+        p.order_len = (int)ord.size();
+        std::copy(ord.begin(), ord.end(), p.order);
+    }
+    fill_inputs(p, q, k, v);
+    set_status_ptr(p);
+
+    if (mode == CP_RING_FUSED || N == 1) {
+        p.step_begin = 0;
+        p.step_end = N;
+        fill_outputs(p, EPI_STORE, o, lse);
+        return launch_attn(p, q->dtype, st);
+    }
+
+    // STEPWISE: the ring as N block launches plus N-1 standalone merges
+    const size_t need = cp_ring_workspace_bytes(layout, N, mode, q->dtype, q->shape[0], S, q->shape[2], q->shape[3]);
+    if (!workspace || workspace_bytes < need)
+        return fail(CP_ERR_INVALID_ARG, "workspace of %zu bytes needed", need);
+    if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const int64_t b = q->shape[0], Hq = q->shape[2], d = q->shape[3], rows = b * S * Hq;
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    char *ws = static_cast<char *>(workspace);
+    cp_tensor o_acc{ws, CP_FP32, 0, {b, S, Hq, d}, {S * Hq * d, Hq * d, d, 1}};
+    cp_tensor o_b{ws + up(rows * d * 4), q->dtype, 0, {b, S, Hq, d}, {S * Hq * d, Hq * d, d, 1}};
+    cp_tensor lse_b{ws + up(rows * d * 4) + up(rows * d * elem_size(q->dtype)), CP_FP32, 0, {b, Hq, S, 1},
+                    {Hq * S, S, 1, 1}};
+    for (int r = 0; r < N; ++r) {
+        p.step_begin = r;
+        p.step_end = r + 1;
+        if (r == 0) fill_outputs(p, EPI_STORE, &o_acc, lse);  // first partial initialises the running result
+        else fill_outputs(p, EPI_STORE, &o_b, &lse_b);
+        if ((s = launch_attn(p, q->dtype, st)) != CP_OK) return s;
+        if (r > 0 && (s = cp_lse_merge(&o_acc, lse, &o_b, &lse_b, r == N - 1 ? o : nullptr, stream)) != CP_OK)
+            return s;
+    }
+    return CP_OK;
+}
+
+cp_status cp_layout_permute(int32_t layout, int32_t N, int32_t seq_axis, const cp_tensor *x, cp_tensor *x_ranked,
+                            int32_t inverse, void *stream)
+{
+    g_last_error[0] = 0;
+    cp_status s;
+    if ((s = check_tensor(x, "x")) != CP_OK || (s = check_tensor(x_ranked, "x_ranked")) != CP_OK) return s;
+    if (layout < 0 || layout > 2) return fail(CP_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (seq_axis < 0 || seq_axis > 3) return fail(CP_ERR_INVALID_ARG, "seq_axis must be 0..3");
+    if (inverse != 0 && inverse != 1) return fail(CP_ERR_INVALID_ARG, "inverse must be 0 or 1");
+    if (x->dtype != x_ranked->dtype || !same_shape(x, x_ranked)) return fail(CP_ERR_SHAPE, "x and x_ranked differ");
+    // both must be densely packed (row-major, no gaps)
+    const cp_tensor *pair[2] = {x, x_ranked};
+    for (const cp_tensor *t : pair) {
+        int64_t expect = 1;
+        for (int i = 3; i >= 0; --i) {
+            if (t->shape[i] > 1 && t->stride[i] != expect) return fail(CP_ERR_INVALID_ARG, "tensors must be contiguous");
+            expect *= t->shape[i];
+        }
+    }
+    const int64_t S = x->shape[seq_axis];
+    if (N < 1 || S % N) return fail(CP_ERR_SHAPE, "sequence axis length must be a multiple of N");
+    if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N)) return fail(CP_ERR_SHAPE, "zig-zag needs S to be a multiple of 2N");
+    PermuteParams p;
+    p.layout = layout;
+    p.n_ranks = N;
+    p.inverse = inverse;
+    p.outer = 1;
+    for (int i = 0; i < seq_axis; ++i) p.outer *= x->shape[i];
+    p.seq = S;
+    p.inner_bytes = elem_size(x->dtype);
+    for (int i = seq_axis + 1; i < 4; ++i) p.inner_bytes *= x->shape[i];
+    p.src = inverse ? x_ranked->data : x->data;
+    p.dst = inverse ? x->data : x_ranked->data;
+    if (p.outer * p.seq * p.inner_bytes == 0) return CP_OK;
+    const char *a = static_cast<const char *>(p.src), *bptr = static_cast<const char *>(p.dst);
+    const int64_t bytes = p.outer * p.seq * p.inner_bytes;
+    if (a < bptr + bytes && bptr < a + bytes) return fail(CP_ERR_INVALID_ARG, "x and x_ranked overlap");
+    cudaError_t e = launch_permute(p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+    return CP_OK;
+}
+
+cp_status cp_stream_check(void *stream)
+{
+    g_last_error[0] = 0;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    int *word = nullptr;
+    if ((e = status_word(&word)) != cudaSuccess) return cuda_fail(e, "status word");
+    int h[2] = {0, 0};
+    if ((e = cudaMemcpy(h, word, sizeof h, cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e, "status read");
+    if (h[0]) {
+        const int zero[2] = {0, 0};
+        cudaMemcpy(word, zero, sizeof zero, cudaMemcpyHostToDevice);
+        return fail(CP_ERR_TIMEOUT, "a device wait expired (status %d, first at wait tag %d)", h[0], h[1]);
+    }
+    return CP_OK;
+}
+
+}  // extern "C"

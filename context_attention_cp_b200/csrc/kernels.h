@@ -1,0 +1,85 @@
+// kernels.h -- internal launch interface between the C ABI (abi.cu) and the
+// CUDA kernels of libcpattn.  Not installed; the public ABI is include/cpattn.h.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "layout.h"
+
+namespace cpattn {
+
+enum { DT_BF16 = 0, DT_FP32 = 1 };
+enum { EPI_STORE = 0, EPI_MERGE = 1 };
+
+// Largest number of (rank, query tile) entries the work-order table in the kernel
+// parameters can hold; longer problems fall back to the natural order.
+constexpr int kMaxOrder = 2048;
+
+// One attention launch: for every (rank, query tile, batch, query head) work item,
+// walk ring steps [step_begin, step_end) (source rank (rank - step) mod n_ranks),
+// build each step's partial (o_b, lse_b) over the non-skipped key tiles, merge the
+// partials with the LSE formula, and finish with the epilogue:
+//   EPI_STORE: write (o, lse) of the merged result (o in o_dtype, lse fp32);
+//   EPI_MERGE: LSE-merge the result into the fp32 (o, lse) already in memory.
+// A block call is n_ranks = 1, one step, explicit ranges.
+struct AttnParams {
+    // sizes
+    int b, hq, hkv, group, d;
+    int q_len, kv_len;         // rows of one rank's query / key block
+    int n_ranks, step_begin, step_end;
+    int causal;
+    int use_layout;            // 1: ranges from (layout, n_ranks, seq_len); 0: explicit
+    int layout;
+    int64_t seq_len;
+    Range q_range, kv_range;   // explicit ranges (use_layout == 0)
+    int64_t q_row_step, kv_row_step;  // tensor row offset of rank i's block = i * step
+    float scale;               // softmax scale
+    float scale_log2;          // softmax scale * log2(e)
+    // inputs (fp32 SIMT kernel reads these; the tcgen05 kernel uses tensor maps)
+    const void *q, *k, *v;
+    int64_t q_sb, q_ss, q_sh, k_sb, k_ss, k_sh, v_sb, v_ss, v_sh;
+    // outputs
+    int epi;
+    void *o;
+    int o_dtype;
+    int64_t o_sb, o_ss, o_sh;
+    float *lse;
+    int64_t lse_sb, lse_sh, lse_ss;
+    int *status;
+    // work order: entry e -> (rank, query tile) = (order[e] >> 16, order[e] & 0xffff)
+    int n_qt;                  // query tiles per rank
+    int order_len;             // 0 = natural order
+    uint32_t order[kMaxOrder];
+};
+
+struct TensorMaps;  // defined in attn_tc.cu
+
+// bf16 tcgen05 path (d in {64, 128}).  q/k/v base pointers and strides in p are
+// used to build TMA tensor maps.  Returns a cudaError_t.
+cudaError_t launch_attn_tc(const AttnParams &p, cudaStream_t stream);
+
+// fp32 SIMT path (d in {64, 128}).
+cudaError_t launch_attn_simt(const AttnParams &p, cudaStream_t stream);
+
+struct MergeParams {
+    int64_t b, s, h, d;
+    float *o_acc;  int64_t oa_sb, oa_ss, oa_sh;
+    float *lse_acc; int64_t la_sb, la_sh, la_ss;
+    const void *o_b; int ob_dtype; int64_t ob_sb, ob_ss, ob_sh;
+    const float *lse_b; int64_t lb_sb, lb_sh, lb_ss;
+    void *o_out; int out_dtype; int64_t out_sb, out_ss, out_sh;  // o_out == nullptr: in place
+};
+cudaError_t launch_lse_merge(const MergeParams &p, cudaStream_t stream);
+
+struct PermuteParams {
+    int layout, n_ranks, inverse;
+    int64_t outer, seq, inner_bytes;  // contiguous [outer, seq, inner]
+    const void *src;
+    void *dst;
+};
+cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream);
+
+// Device status word of the current device (2 ints), from status.cu.
+cudaError_t status_word(int **ptr);
+
+}  // namespace cpattn

@@ -1,0 +1,183 @@
+/*
+ * cpattn.h -- C ABI of libcpattn: ring-scheduled blockwise softmax attention
+ * (context parallelism with N virtual ranks) on one NVIDIA B200 (sm_100a).
+ *
+ * The operations follow "上下文并行与 Ring Attention" (hs-black.github.io):
+ *   - section 分块注意力: block partial (o_b, lse_b) of a query set against one
+ *     key/value block, with m_b = max x_j, l_b = sum e^{x_j - m_b},
+ *     o_b = sum e^{x_j - m_b} v_j / l_b, lse_b = m_b + log l_b (natural log), and
+ *     the merge o = e^{lse_1-lse} o_1 + e^{lse_2-lse} o_2, lse = M + log(e^{lse_1-M}
+ *     + e^{lse_2-M}), M = max(lse_1, lse_2) (the boxed identity and its stable form);
+ *   - section Ring Attention: at ring step r rank i attends its local Q to the K/V
+ *     that rank (i - r) mod N started with, and merges the partial into its
+ *     running (o, lse); Q and O never move;
+ *   - sections 因果掩码带来的负载不均 / Zig-zag / Striped / 重排 token 的代价: the
+ *     causal mask is judged on original token positions, and the three token
+ *     layouts are permutations applied once at model entry.
+ *
+ * Conventions shared by every entry point
+ *   - Token tensors are [b, s, H, d] with d contiguous; lse tensors are
+ *     [b, H, s] fp32 holding natural-log values.  Strides are in elements.
+ *   - Ownership: the caller owns every buffer and the stream.  No entry point
+ *     allocates device memory; no pointer is kept after return, apart from work
+ *     already queued on `stream`.
+ *   - Errors: argument problems are reported synchronously through the return
+ *     value (and a message from cp_last_error()).  Device-side problems (a
+ *     bounded wait that ran out, a CUDA launch error) are reported by
+ *     cp_stream_check() or by the next call's return value.  Nothing throws.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - Thread-compatible: no global mutable state besides the per-device status
+ *     word read by cp_stream_check() and the per-thread last-error message.
+ */
+#ifndef CPATTN_H
+#define CPATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CP_OK = 0,
+    CP_ERR_INVALID_ARG = 1, /* null pointer, bad enum, bad dtype, bad stride */
+    CP_ERR_UNSUPPORTED = 2, /* valid request this build does not implement (e.g. d) */
+    CP_ERR_SHAPE = 3,       /* inconsistent or indivisible sizes */
+    CP_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+    CP_ERR_TIMEOUT = 5      /* a device-side bounded wait expired (see cp_stream_check) */
+} cp_status;
+
+typedef enum { CP_BF16 = 0, CP_FP32 = 1 } cp_dtype;
+
+/* CP_MASK_CAUSAL: key t is visible to query p iff pos_k(t) <= pos_q(p), positions
+ * taken from the cp_range arguments (original token positions). */
+typedef enum { CP_MASK_NONE = 0, CP_MASK_CAUSAL = 1 } cp_mask_mode;
+
+/* Token layouts over N ranks of c = S/N tokens each (section Zig-zag / Striped):
+ *   CONTIGUOUS: rank i holds positions [i*c, (i+1)*c)
+ *   ZIGZAG    : 2N chunks of c/2; rank i holds chunk i then chunk 2N-1-i
+ *   STRIPED   : rank i holds positions i, i+N, i+2N, ... (token p on rank p mod N) */
+typedef enum { CP_LAYOUT_CONTIGUOUS = 0, CP_LAYOUT_ZIGZAG = 1, CP_LAYOUT_STRIPED = 2 } cp_layout;
+
+/* How cp_ring_attn_fwd runs the N steps:
+ *   FUSED   : one launch; each CTA owns a 128-row query tile of one rank and walks
+ *             the ring steps in order, keeping each step's partial (o_b, lse_b) and
+ *             the running (o, lse) on chip and merging them with the LSE formula.
+ *   STEPWISE: N launches of the block kernel (all ranks per launch) writing
+ *             (o_b, lse_b) to the workspace, each followed by a standalone merge
+ *             launch; the last merge writes the output.  Needs a workspace. */
+typedef enum { CP_RING_FUSED = 0, CP_RING_STEPWISE = 1 } cp_ring_mode;
+
+/* A strided 4-D view.  Token tensors: [b, s, H, d]; lse tensors: [b, H, s, 1]
+ * (shape[3] = 1).  dtype is a cp_dtype.  Strides in elements; stride[3] must be 1. */
+typedef struct {
+    void *data;
+    int32_t dtype;
+    int32_t reserved;
+    int64_t shape[4];
+    int64_t stride[4];
+} cp_tensor;
+
+/* Original position of local token t (0 <= t < len[0] + len[1]):
+ *   t <  len[0]: start[0] + t * stride
+ *   t >= len[0]: start[1] + (t - len[0]) * stride      (only when nseg == 2)
+ * stride >= 1.  Contiguous rank i: {1, {i*c}, {c}, 1}; zig-zag rank i:
+ * {2, {i*c/2, (2N-1-i)*c/2}, {c/2, c/2}, 1}; striped rank i: {1, {i}, {c}, N}. */
+typedef struct {
+    int32_t nseg;
+    int32_t reserved;
+    int64_t start[2];
+    int64_t len[2];
+    int64_t stride;
+} cp_range;
+
+/* Block attention (section 分块注意力; the flash_attn call of section Ring Attention).
+ *   q [b, sq, Hq, d], k/v [b, sk, Hkv, d]: same dtype (CP_BF16 or CP_FP32),
+ *     Hq % Hkv == 0, query head h reads KV head h / (Hq/Hkv); d in {64, 128}.
+ *   q_range / kv_range: original positions of the sq query / sk key rows
+ *     (len[0] + len[1] must equal sq / sk).  Used only when mask_mode is causal.
+ *   softmax_scale: multiplies q.k (1/sqrt(d) for standard attention); > 0.
+ *   accumulate == 0: writes o_b into o ([b, sq, Hq, d], dtype = q's dtype or
+ *     CP_FP32) and lse_b into lse ([b, Hq, sq, 1] fp32).  Rows that see no key get
+ *     o = 0, lse = -inf.
+ *   accumulate == 1: o must be CP_FP32; (o, lse) hold a running partial and are
+ *     updated in place with the LSE merge of (o_b, lse_b) (fused epilogue).
+ * Fully masked key tiles are skipped whole.  Asynchronous on `stream`. */
+cp_status cp_block_attn_fwd(const cp_tensor *q, const cp_tensor *k, const cp_tensor *v,
+                            const cp_range *q_range, const cp_range *kv_range, int32_t mask_mode,
+                            float softmax_scale, cp_tensor *o, cp_tensor *lse, int32_t accumulate,
+                            void *stream);
+
+/* Standalone LSE merge (section 分块注意力, stable form), one HBM pass:
+ *   (o_acc, lse_acc) <- merge((o_acc, lse_acc), (o_b, lse_b))
+ *   o_acc [b, s, H, d] CP_FP32, o_b same shape CP_BF16 or CP_FP32,
+ *   lse_acc / lse_b [b, H, s, 1] CP_FP32.
+ * o_out: NULL to write the merged o back into o_acc; otherwise a [b, s, H, d]
+ *   tensor (CP_BF16 or CP_FP32) that receives the merged o (rounded to nearest
+ *   even for bf16) while o_acc is left unchanged; lse_acc is always updated.
+ * An empty side (lse = -inf) contributes nothing; two empty sides give (0, -inf).
+ * Rows are 16-byte aligned: d * sizeof(element) must be a multiple of 16. */
+cp_status cp_lse_merge(cp_tensor *o_acc, cp_tensor *lse_acc, const cp_tensor *o_b,
+                       const cp_tensor *lse_b, cp_tensor *o_out, void *stream);
+
+/* Ring attention forward over N virtual ranks on one GPU (section Ring Attention).
+ *   q [b, S, Hq, d], k/v [b, S, Hkv, d] in RANK-MAJOR order (as produced by
+ *   cp_layout_permute): rows [i*c, (i+1)*c) belong to rank i, c = S/N.
+ *   causal: 1 for the causal mask on original positions, 0 for none.
+ *   o [b, S, Hq, d] (q's dtype), lse [b, Hq, S, 1] fp32, both in rank-major order.
+ *   mode: cp_ring_mode.  workspace / workspace_bytes: device memory of at least
+ *   cp_ring_workspace_bytes(...) bytes (may be NULL/0 when that is 0); the
+ *   caller keeps it alive until the work on `stream` has finished.
+ * Requires S % N == 0, S % (2N) == 0 for zig-zag, Hq % Hkv == 0, d in {64, 128}. */
+cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q,
+                           const cp_tensor *k, const cp_tensor *v, float softmax_scale,
+                           cp_tensor *o, cp_tensor *lse, int32_t mode, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+/* Workspace bytes cp_ring_attn_fwd needs for this problem (0 for CP_RING_FUSED).
+ * Returns 0 as well for invalid arguments (cp_ring_attn_fwd then reports them). */
+size_t cp_ring_workspace_bytes(int32_t layout, int32_t N, int32_t mode, int32_t dtype, int64_t b,
+                               int64_t S, int64_t Hq, int64_t d);
+
+/* Token permutation into / out of rank-major order (section 重排 token 的代价).
+ *   x and x_ranked: same shape, dtype and contiguous layout; the sequence axis is
+ *   seq_axis (1 for [b, S, H, d], 2 for lse [b, H, S, 1]).
+ *   inverse == 0: x_ranked[.., i*c + t, ..] = x[.., pos(i, t), ..]
+ *   inverse == 1: x[.., pos(i, t), ..] = x_ranked[.., i*c + t, ..]
+ *     (here x_ranked is read and x is written).
+ * Bit-exact copy; x and x_ranked must not overlap. */
+cp_status cp_layout_permute(int32_t layout, int32_t N, int32_t seq_axis, const cp_tensor *x,
+                            cp_tensor *x_ranked, int32_t inverse, void *stream);
+
+/* Host only: the cp_range of rank `rank` for a sequence of S tokens. */
+cp_status cp_layout_range(int32_t layout, int32_t N, int64_t S, int32_t rank, cp_range *out);
+
+/* Host only: the tile classes the kernels use for a (query block, key block) pair.
+ * out[qt * n_kt + kt] = 0 (skip: no visible pair), 1 (full: every pair visible),
+ * 2 (partial: masked element by element), for tiles of tile_q x tile_k local
+ * rows; n_qt = ceil(q_len / tile_q), n_kt = ceil(kv_len / tile_k).  Rows past
+ * q_len / kv_len are not tokens (a tile holding them is partial in the key axis). */
+cp_status cp_tile_classes(const cp_range *q_range, int64_t q_len, const cp_range *kv_range,
+                          int64_t kv_len, int32_t mask_mode, int32_t tile_q, int32_t tile_k,
+                          int8_t *out);
+
+/* Synchronises `stream`, then reports (and clears) the device status word of the
+ * current device: CP_ERR_TIMEOUT if a kernel's bounded wait expired since the last
+ * check, CP_ERR_CUDA if the stream reported an error, else CP_OK. */
+cp_status cp_stream_check(void *stream);
+
+/* Static description of a status code. */
+const char *cp_status_string(cp_status s);
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char *cp_last_error(void);
+
+/* ABI version, bumped on incompatible changes. */
+int32_t cp_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CPATTN_H */

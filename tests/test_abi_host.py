@@ -1,0 +1,206 @@
+"""Host-side checks of libcpattn that need no GPU: the library loads, exports every
+entry point include/cpattn.h declares, computes layout ranges and tile classes
+that match the oracle's integer maps bit for bit, and rejects bad arguments
+synchronously (before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from oracle import layout as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def cp():
+    from context_attention_cp_b200 import build
+    build.build()
+    import context_attention_cp_b200 as m
+    m.lib()
+    return m
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "cpattn.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(cp_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(cp):
+    names = _declared_symbols()
+    assert len(names) >= 10
+    handle = ctypes.CDLL(cp.lib_path)
+    for n in names:
+        assert hasattr(handle, n), n
+    assert cp.lib().cp_abi_version() == 1
+
+
+def test_status_strings(cp):
+    for code in range(6):
+        assert cp.lib().cp_status_string(code)
+    assert cp.lib().cp_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("layout", L.LAYOUTS)
+@pytest.mark.parametrize("N,S", [(1, 16), (2, 16), (4, 64), (8, 256), (3, 24)])
+def test_layout_range_matches_oracle(cp, layout, N, S):
+    for rank in range(N):
+        starts, lens, stride = cp.layout_range(layout, N, S, rank)
+        pos = []
+        for s0, n in zip(starts, lens):
+            pos.extend(s0 + t * stride for t in range(n))
+        assert pos == L.rank_positions(layout, N, S, rank)
+
+
+def test_layout_range_rejects(cp):
+    with pytest.raises(cp.CPError) as e:
+        cp.layout_range("contiguous", 3, 10, 0)
+    assert e.value.code == 3
+    with pytest.raises(cp.CPError):
+        cp.layout_range("zigzag", 4, 12, 0)
+    with pytest.raises(cp.CPError):
+        cp.layout_range("striped", 4, 16, 4)
+
+
+def _brute_classes(pq, pk, causal, tq, tk):
+    out = []
+    for q0 in range(0, len(pq), tq):
+        row = []
+        qs = pq[q0:q0 + tq]
+        for k0 in range(0, len(pk), tk):
+            ks = pk[k0:k0 + tk]
+            vis = sum(1 for a in qs for b in ks if (not causal) or b <= a)
+            whole = len(ks) == tk
+            if vis == 0:
+                row.append(0)
+            elif vis == len(qs) * len(ks) and whole:
+                row.append(1)
+            else:
+                row.append(2)
+        out.append(row)
+    return out
+
+
+@pytest.mark.parametrize("layout", L.LAYOUTS)
+@pytest.mark.parametrize("N,S,tile", [(2, 64, 8), (4, 128, 8), (4, 96, 16), (3, 48, 5), (8, 256, 16)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_tile_classes_match_brute_force(cp, layout, N, S, tile, causal):
+    if layout == "zigzag" and S % (2 * N):
+        pytest.skip("zig-zag needs S % 2N == 0")
+    c = S // N
+    for i in range(N):
+        for j in range(N):
+            qr, kr = cp.layout_range(layout, N, S, i), cp.layout_range(layout, N, S, j)
+            got = cp.tile_classes(qr, c, kr, c, causal, tile, tile)
+            want = _brute_classes(L.rank_positions(layout, N, S, i), L.rank_positions(layout, N, S, j),
+                                  causal, tile, tile)
+            assert got == want, (i, j)
+
+
+def test_tile_classes_zigzag_rectangles(cp):
+    """Off-diagonal zig-zag steps need no mask: with tiles that divide c/2, no tile is
+    partial unless j == i (section Zig-zag, the remark after the case table)."""
+    N, S = 4, 512
+    c = S // N
+    for i in range(N):
+        for j in range(N):
+            cls = cp.tile_classes(cp.layout_range("zigzag", N, S, i), c, cp.layout_range("zigzag", N, S, j), c,
+                                  True, 16, 16)
+            partial = sum(x == 2 for row in cls for x in row)
+            assert (partial > 0) == (i == j)
+
+
+class _FakeTensor:
+    """Stands in for a CUDA tensor in argument-validation tests (never dereferenced)."""
+
+
+def _ct(cp, shape, dtype=0, data=0x10000, stride=None):
+    from context_attention_cp_b200._binding import CpTensor
+    t = CpTensor()
+    t.data = data
+    t.dtype = dtype
+    if stride is None:
+        stride = [0, 0, 0, 1]
+        acc = 1
+        for i in (3, 2, 1, 0):
+            stride[i] = acc
+            acc *= shape[i]
+    for i in range(4):
+        t.shape[i] = shape[i]
+        t.stride[i] = stride[i]
+    return t
+
+
+def _call_ring(cp, q, k, v, o, lse, layout=0, N=2, causal=1, scale=0.1, mode=0):
+    return cp.lib().cp_ring_attn_fwd(layout, N, causal, ctypes.byref(q), ctypes.byref(k), ctypes.byref(v),
+                                     ctypes.c_float(scale), ctypes.byref(o), ctypes.byref(lse), mode, None, 0, None)
+
+
+def test_ring_argument_errors_are_synchronous(cp):
+    q = _ct(cp, [1, 256, 4, 128])
+    k = _ct(cp, [1, 256, 2, 128])
+    v = _ct(cp, [1, 256, 2, 128])
+    o = _ct(cp, [1, 256, 4, 128])
+    lse = _ct(cp, [1, 4, 256, 1], dtype=1)
+    assert _call_ring(cp, q, k, v, o, lse, N=3) == 3            # S % N
+    assert _call_ring(cp, q, k, v, o, lse, layout=1, N=3) == 3  # S % 2N
+    assert _call_ring(cp, q, k, v, o, lse, layout=7) == 1       # layout
+    assert _call_ring(cp, q, k, v, o, lse, scale=-1.0) == 1     # scale
+    assert _call_ring(cp, q, k, v, o, lse, mode=5) == 1         # mode
+    k3 = _ct(cp, [1, 256, 3, 128])
+    assert _call_ring(cp, q, k3, k3, o, lse) == 3               # Hq % Hkv
+    q96 = _ct(cp, [1, 256, 4, 96])
+    assert _call_ring(cp, q96, k, v, o, lse) in (2, 3)          # head dim
+    kf = _ct(cp, [1, 256, 2, 128], dtype=1)
+    assert _call_ring(cp, q, kf, kf, o, lse) == 1               # mixed dtypes
+    bad = _ct(cp, [1, 256, 4, 128], data=0x10008)
+    assert _call_ring(cp, bad, k, v, o, lse) == 1               # alignment
+    lse_bad = _ct(cp, [1, 4, 255, 1], dtype=1)
+    assert _call_ring(cp, q, k, v, o, lse_bad) == 3             # lse shape
+    assert b"multiple" in cp.lib().cp_last_error() or cp.lib().cp_last_error()
+
+
+def test_block_argument_errors_are_synchronous(cp):
+    from context_attention_cp_b200._binding import CpRange
+    q = _ct(cp, [1, 128, 2, 64], dtype=1)
+    k = _ct(cp, [1, 100, 2, 64], dtype=1)
+    o = _ct(cp, [1, 128, 2, 64], dtype=1)
+    lse = _ct(cp, [1, 2, 128, 1], dtype=1)
+    qr, kr = CpRange(), CpRange()
+    qr.nseg, qr.start[0], qr.len[0], qr.stride = 1, 0, 128, 1
+    kr.nseg, kr.start[0], kr.len[0], kr.stride = 1, 0, 99, 1  # wrong length
+    f = cp.lib().cp_block_attn_fwd
+    assert f(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(qr), ctypes.byref(kr), 1,
+             ctypes.c_float(0.1), ctypes.byref(o), ctypes.byref(lse), 0, None) == 3
+    kr.len[0] = 100
+    kr.nseg, kr.start[1], kr.len[0], kr.len[1] = 2, 10, 50, 50  # second segment overlaps the first
+    assert f(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(qr), ctypes.byref(kr), 1,
+             ctypes.c_float(0.1), ctypes.byref(o), ctypes.byref(lse), 0, None) == 1
+    kr.nseg, kr.len[0] = 1, 100
+    o16 = _ct(cp, [1, 128, 2, 64], dtype=0)
+    assert f(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(qr), ctypes.byref(kr), 1,
+             ctypes.c_float(0.1), ctypes.byref(o16), ctypes.byref(lse), 0, None) == 1  # fp32 in -> fp32 out
+    assert f(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(qr), ctypes.byref(kr), 1,
+             ctypes.c_float(0.1), ctypes.byref(o16), ctypes.byref(lse), 1, None) == 1  # accumulate needs fp32
+
+
+def test_merge_and_permute_argument_errors(cp):
+    oa = _ct(cp, [1, 16, 2, 128], dtype=1)
+    ob = _ct(cp, [1, 16, 2, 128], dtype=0)
+    la = _ct(cp, [1, 2, 16, 1], dtype=1)
+    lb = _ct(cp, [1, 2, 16, 1], dtype=1)
+    f = cp.lib().cp_lse_merge
+    ob_bad = _ct(cp, [1, 16, 3, 128], dtype=0)
+    assert f(ctypes.byref(oa), ctypes.byref(la), ctypes.byref(ob_bad), ctypes.byref(lb), None, None) == 3
+    oa16 = _ct(cp, [1, 16, 2, 128], dtype=0)
+    assert f(ctypes.byref(oa16), ctypes.byref(la), ctypes.byref(ob), ctypes.byref(lb), None, None) == 1
+    x = _ct(cp, [1, 16, 2, 128], dtype=0)
+    y = _ct(cp, [1, 16, 2, 128], dtype=0, data=0x20000)
+    g = cp.lib().cp_layout_permute
+    assert g(1, 3, 1, ctypes.byref(x), ctypes.byref(y), 0, None) == 3       # 16 % 6
+    assert g(0, 2, 1, ctypes.byref(x), ctypes.byref(x), 0, None) == 1       # overlap
+    assert cp.lib().cp_ring_workspace_bytes(0, 4, 0, 0, 1, 256, 4, 128) == 0  # fused needs none
+    assert cp.lib().cp_ring_workspace_bytes(0, 4, 1, 0, 1, 256, 4, 128) >= 256 * 4 * 128 * 6
