@@ -41,6 +41,7 @@ _SIGNATURES = {
     "cp_layout_range": (_i32, [_i32, _i32, _i64, _i32, _R]),
     "cp_tile_classes": (_i32, [_R, _i64, _R, _i64, _i32, _i32, _i32, ctypes.POINTER(ctypes.c_int8)]),
     "cp_stream_check": (_i32, [_vp]),
+    "cp_ring_attn_fwd_static_scratch": (_i32, [_i32, _i32, _i32, _T, _T, _T, _f32, _T, _T, _vp]),
     "cp_status_string": (ctypes.c_char_p, [_i32]),
     "cp_last_error": (ctypes.c_char_p, []),
     "cp_abi_version": (_i32, []),
@@ -175,6 +176,15 @@ def ring_attn_fwd(q, k, v, layout, N, causal, scale=None, o=None, lse=None, mode
     tq, tk, tv, to, tl = _tensor(q), _tensor(k), _tensor(v), _tensor(o), _tensor(lse)
     _check(lib().cp_ring_attn_fwd(LAYOUTS[layout], N, int(bool(causal)), _ref(tq), _ref(tk), _ref(tv),
                                   float(scale), _ref(to), _ref(tl), MODES[mode], ws_ptr, need, _stream()))
+    return o, lse
+
+
+def ring_attn_fwd_static_scratch(q, k, v, layout, N, causal, scale, o, lse):
+    """Stepwise ring that takes its workspace from the library's static device
+    scratch, for callers that cannot allocate; o and lse are caller-allocated."""
+    tq, tk, tv, to, tl = _tensor(q), _tensor(k), _tensor(v), _tensor(o), _tensor(lse)
+    _check(lib().cp_ring_attn_fwd_static_scratch(LAYOUTS[layout], N, int(bool(causal)), _ref(tq), _ref(tk),
+                                                 _ref(tv), float(scale), _ref(to), _ref(tl), _stream()))
     return o, lse
 
 

@@ -210,6 +210,15 @@ cp_status check_out(const cp_tensor *o, const cp_tensor *lse, const cp_tensor *q
 
 }  // namespace
 
+cp_status cpattn::report_error(cp_status status, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return status;
+}
+
 extern "C" {
 
 const char *cp_status_string(cp_status s)

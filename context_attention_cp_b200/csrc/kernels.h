@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/cpattn.h"
 #include "layout.h"
 
 namespace cpattn {
@@ -81,5 +82,8 @@ cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream);
 
 // Device status word of the current device (2 ints), from status.cu.
 cudaError_t status_word(int **ptr);
+
+// Records a printf-style message for cp_last_error() and returns `status` (abi.cu).
+cp_status report_error(cp_status status, const char *fmt, ...);
 
 }  // namespace cpattn

@@ -176,6 +176,28 @@ const char *cp_last_error(void);
 /* ABI version, bumped on incompatible changes. */
 int32_t cp_abi_version(void);
 
+/* Bytes of device scratch the library reserves for cp_ring_attn_fwd_static_scratch. */
+#define CP_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/* Stepwise ring attention that allocates nothing, for callers that cannot call
+ * cudaMalloc (for example a plug-in whose host engine owns all device memory and
+ * passes it only input and output pointers, or a caller that must not take the
+ * synchronisation an allocation can cause).  The pages have no counterpart: this
+ * is a packaging variant of cp_ring_attn_fwd(..., CP_RING_STEPWISE, ...).
+ *   Arguments and results are those of cp_ring_attn_fwd; the caller still owns q,
+ *   k, v, o and lse.  The workspace comes from a static device array of
+ *   CP_STATIC_SCRATCH_BYTES that every GPU loading the library holds until exit.
+ *   Errors: CP_ERR_UNSUPPORTED (returned before any launch) when
+ *   cp_ring_workspace_bytes(layout, N, CP_RING_STEPWISE, ...) exceeds
+ *   CP_STATIC_SCRATCH_BYTES; otherwise as cp_ring_attn_fwd.
+ *   All calls on a device share the array and it keeps the last call's contents
+ *   (the ring writes everything it reads, so nothing needs clearing); calls whose
+ *   work overlaps on the GPU race on it.  The first call on each device looks up
+ *   the array's device address; make that first call before any stream capture. */
+cp_status cp_ring_attn_fwd_static_scratch(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q,
+                                          const cp_tensor *k, const cp_tensor *v, float softmax_scale,
+                                          cp_tensor *o, cp_tensor *lse, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
