@@ -126,41 +126,44 @@ cp_status launch_attn(const AttnParams &p, int32_t dtype, cudaStream_t stream)
 
 // ---------------------------------------------------------------- ring scheduler
 
-// Work order for the ring: (rank, query tile) entries sorted by the number of key
-// tiles they visit over all steps, heaviest first, so the long causal rows start
-// early and the tail of the launch is made of short ones.
+// Work order for the ring: (rank, row group) entries sorted by the number of key
+// tiles their 128-row query tiles visit over all steps, heaviest first, so the long
+// causal rows start early and the tail of the launch is made of short ones.
 struct OrderKey {
-    int layout, n, causal;
+    int layout, n, causal, rows;
     int64_t seq;
     bool operator<(const OrderKey &o) const
     {
-        return std::tie(layout, n, causal, seq) < std::tie(o.layout, o.n, o.causal, o.seq);
+        return std::tie(layout, n, causal, rows, seq) < std::tie(o.layout, o.n, o.causal, o.rows, o.seq);
     }
 };
 std::mutex g_order_mu;
 std::map<OrderKey, std::vector<uint32_t>> g_order_cache;
 
-const std::vector<uint32_t> &ring_order(int layout, int N, int64_t S, int causal)
+const std::vector<uint32_t> &ring_order(int layout, int N, int64_t S, int causal, int rows_per_cta)
 {
     std::lock_guard<std::mutex> lk(g_order_mu);
-    OrderKey key{layout, N, causal, S};
+    OrderKey key{layout, N, causal, rows_per_cta, S};
     auto it = g_order_cache.find(key);
     if (it != g_order_cache.end()) return it->second;
     const int64_t c = S / N;
-    const int n_qt = (int)((c + 127) / 128);
+    const int n_groups = (int)((c + rows_per_cta - 1) / rows_per_cta);
     std::vector<std::pair<int64_t, uint32_t>> work;
-    work.reserve((size_t)N * n_qt);
+    work.reserve((size_t)N * n_groups);
     for (int i = 0; i < N; ++i) {
         Range qr = layout_range(layout, N, S, i);
-        for (int qt = 0; qt < n_qt; ++qt) {
+        for (int g = 0; g < n_groups; ++g) {
             int64_t tiles = 0;
-            for (int r = 0; r < N; ++r) {
-                Range kr = layout_range(layout, N, S, ((i - r) % N + N) % N);
-                int kf, ke;
-                kv_tile_bounds(qr, c, (int64_t)qt * 128, 128, kr, c, 128, causal != 0, &kf, &ke);
-                tiles += ke;
+            for (int64_t q_lo = (int64_t)g * rows_per_cta; q_lo < std::min<int64_t>(c, (int64_t)(g + 1) * rows_per_cta);
+                 q_lo += 128) {
+                for (int r = 0; r < N; ++r) {
+                    Range kr = layout_range(layout, N, S, ((i - r) % N + N) % N);
+                    int kf, ke;
+                    kv_tile_bounds(qr, c, q_lo, 128, kr, c, 128, causal != 0, &kf, &ke);
+                    tiles += ke;
+                }
             }
-            work.push_back({tiles, ((uint32_t)i << 16) | (uint32_t)qt});
+            work.push_back({tiles, ((uint32_t)i << 16) | (uint32_t)g});
         }
     }
     std::stable_sort(work.begin(), work.end(),
@@ -171,6 +174,8 @@ const std::vector<uint32_t> &ring_order(int layout, int N, int64_t S, int causal
     for (auto &w : work) out.push_back(w.second);
     return g_order_cache.emplace(key, std::move(out)).first->second;
 }
+
+int rows_per_cta(int32_t dtype) { return dtype == CP_BF16 ? attn_tc_rows_per_cta() : 128; }
 
 cp_status check_attn_dtypes(const cp_tensor *q, const cp_tensor *k, const cp_tensor *v)
 {
@@ -317,7 +322,7 @@ cp_status cp_block_attn_fwd(const cp_tensor *q, const cp_tensor *k, const cp_ten
     p.kv_range = to_range(*kv_range);
     p.scale = softmax_scale;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
-    p.n_qt = (int)((sq + 127) / 128);
+    p.n_qt = (int)((sq + rows_per_cta(q->dtype) - 1) / rows_per_cta(q->dtype));
     if (p.n_qt > 65535) return fail(CP_ERR_SHAPE, "too many query tiles");
     fill_inputs(p, q, k, v);
     fill_outputs(p, accumulate ? EPI_MERGE : EPI_STORE, o, lse);
@@ -406,7 +411,8 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     if (o->dtype != q->dtype) return fail(CP_ERR_INVALID_ARG, "o must have q's dtype");
     const int64_t c = S / N;
     if (q->shape[0] == 0 || S == 0) return CP_OK;
-    const int n_qt = (int)((c + 127) / 128);
+    const int rows = rows_per_cta(q->dtype);
+    const int n_qt = (int)((c + rows - 1) / rows);
     if (n_qt > 65535) return fail(CP_ERR_SHAPE, "too many query tiles per rank");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
@@ -429,7 +435,7 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     p.scale = softmax_scale;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.n_qt = n_qt;
-    const std::vector<uint32_t> &ord = ring_order(layout, N, S, causal);
+    const std::vector<uint32_t> &ord = ring_order(layout, N, S, causal, rows);
     if ((int64_t)ord.size() <= kMaxOrder) {
         p.order_len = (int)ord.size();
         std::copy(ord.begin(), ord.end(), p.order);
@@ -449,12 +455,12 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     if (!workspace || workspace_bytes < need)
         return fail(CP_ERR_INVALID_ARG, "workspace of %zu bytes needed", need);
     if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-    const int64_t b = q->shape[0], Hq = q->shape[2], d = q->shape[3], rows = b * S * Hq;
+    const int64_t b = q->shape[0], Hq = q->shape[2], d = q->shape[3], nrows = b * S * Hq;
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
     char *ws = static_cast<char *>(workspace);
     cp_tensor o_acc{ws, CP_FP32, 0, {b, S, Hq, d}, {S * Hq * d, Hq * d, d, 1}};
-    cp_tensor o_b{ws + up(rows * d * 4), q->dtype, 0, {b, S, Hq, d}, {S * Hq * d, Hq * d, d, 1}};
-    cp_tensor lse_b{ws + up(rows * d * 4) + up(rows * d * elem_size(q->dtype)), CP_FP32, 0, {b, Hq, S, 1},
+    cp_tensor o_b{ws + up(nrows * d * 4), q->dtype, 0, {b, S, Hq, d}, {S * Hq * d, Hq * d, d, 1}};
+    cp_tensor lse_b{ws + up(nrows * d * 4) + up(nrows * d * elem_size(q->dtype)), CP_FP32, 0, {b, Hq, S, 1},
                     {Hq * S, S, 1, 1}};
     for (int r = 0; r < N; ++r) {
         p.step_begin = r;

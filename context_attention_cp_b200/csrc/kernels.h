@@ -47,8 +47,9 @@ struct AttnParams {
     float *lse;
     int64_t lse_sb, lse_sh, lse_ss;
     int *status;
-    // work order: entry e -> (rank, query tile) = (order[e] >> 16, order[e] & 0xffff)
-    int n_qt;                  // query tiles per rank
+    // work order: entry e -> (rank, row group) = (order[e] >> 16, order[e] & 0xffff);
+    // a row group is the query rows one CTA covers (256 tensor-core, 128 SIMT)
+    int n_qt;                  // row groups per rank
     int order_len;             // 0 = natural order
     uint32_t order[kMaxOrder];
 };
@@ -59,7 +60,10 @@ struct TensorMaps;  // defined in attn_tc.cu
 // used to build TMA tensor maps.  Returns a cudaError_t.
 cudaError_t launch_attn_tc(const AttnParams &p, cudaStream_t stream);
 
-// fp32 SIMT path (d in {64, 128}).
+// Query rows one CTA of the tensor-core kernel covers (the unit of the work order).
+int attn_tc_rows_per_cta();
+
+// fp32 SIMT path (d in {64, 128}); one CTA covers 128 query rows.
 cudaError_t launch_attn_simt(const AttnParams &p, cudaStream_t stream);
 
 struct MergeParams {

@@ -73,7 +73,7 @@ struct WaitCtx {
 
 // Waits until the phase with parity `parity` of `bar` completed.  Returns false if
 // the CTA was aborted or the wait expired (then STATUS_TIMEOUT is raised).
-static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx &w)
+static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx &w)
 {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = global_timer_ns();
@@ -214,6 +214,24 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64])
 }
 #undef CP_R8
 
+// Same, 64 columns straight into floats (no integer staging registers).
+#define CP_F8(b) "=f"(v[b + 0]), "=f"(v[b + 1]), "=f"(v[b + 2]), "=f"(v[b + 3]), \
+                 "=f"(v[b + 4]), "=f"(v[b + 5]), "=f"(v[b + 6]), "=f"(v[b + 7])
+__device__ __forceinline__ void tmem_ld64f(uint32_t taddr, float *v)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : CP_F8(0), CP_F8(8), CP_F8(16), CP_F8(24), CP_F8(32), CP_F8(40), CP_F8(48), CP_F8(56)
+        : "r"(taddr)
+        : "memory");
+}
+#undef CP_F8
+
 #define CP_W8(b) "r"(r[b + 0]), "r"(r[b + 1]), "r"(r[b + 2]), "r"(r[b + 3]), \
                  "r"(r[b + 4]), "r"(r[b + 5]), "r"(r[b + 6]), "r"(r[b + 7])
 // Registers -> TMEM, 32 columns (completion via tmem_wait_st()).
@@ -224,6 +242,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
         "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
         CP_W8(0), CP_W8(8), CP_W8(16), CP_W8(24)
+        : "memory");
+}
+// Registers -> TMEM, 16 columns.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        CP_W8(0), CP_W8(8)
         : "memory");
 }
 #undef CP_W8
