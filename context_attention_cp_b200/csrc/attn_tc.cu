@@ -36,6 +36,7 @@
 
 #include "kernels.h"
 #include "ptx.cuh"
+#include "exp2_poly.h"
 
 namespace cpattn {
 namespace {
@@ -51,6 +52,13 @@ constexpr int REGS_OTHER = 88;
 constexpr int WARP_LOAD = 8;
 constexpr int WARP_MMA = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// In tiles without masking, pair i of every 16 probability pairs is computed on
+// the FMA pipe (exp2_fma) when i % kEmuMod == kEmuMod - 1, the rest on the MUFU
+// pipe (ex2.approx); 0 disables.  Balances the two pipes.
+#ifndef CP_EXP2_EMU_MOD
+#define CP_EXP2_EMU_MOD 0
+#endif
+constexpr int kEmuMod = CP_EXP2_EMU_MOD;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
@@ -383,8 +391,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             tc_fence_after();
             float s[BN];
-            tmem_ld64f(s_tmem, s);
-            tmem_ld64f(s_tmem + 64, s + 64);
+            tmem_ld64f_nowait(s_tmem, s);
+            tmem_ld64f_nowait(s_tmem + 64, s + 64);
+            tmem_wait_ld_dep(s);
+            reg_dep64(s + 64);
             // ---- mask (partial tiles only).  Positions increase with the local key
             // index, so the keys this row may see form a prefix of the tile.
             if (seq.partial(j)) {
@@ -403,16 +413,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 for (int cc = 0; cc < BN; ++cc)
                     if (cc >= cnt) s[cc] = -INFINITY;
             }
-            // ---- row max
+            // ---- row max: four chains of 3-input max
             float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-            for (int cc = 4; cc < BN; cc += 4) {
-                mx0 = fmaxf(mx0, s[cc]);
-                mx1 = fmaxf(mx1, s[cc + 1]);
-                mx2 = fmaxf(mx2, s[cc + 2]);
-                mx3 = fmaxf(mx3, s[cc + 3]);
+            for (int cc = 4; cc < BN - 4; cc += 8) {
+                mx0 = fmax3(mx0, s[cc], s[cc + 1]);
+                mx1 = fmax3(mx1, s[cc + 2], s[cc + 3]);
+                mx2 = fmax3(mx2, s[cc + 4], s[cc + 5]);
+                mx3 = fmax3(mx3, s[cc + 6], s[cc + 7]);
             }
-            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+            mx0 = fmax3(mx0, s[BN - 4], s[BN - 3]);
+            mx1 = fmax3(mx1, s[BN - 2], s[BN - 1]);
+            const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
             // Raise the exponent's max only when it grew by more than the threshold;
             // then O and l are rescaled below (after P is out of the registers).
             float f_rescale = 1.f;
@@ -431,22 +443,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             const float mu = (m == -INFINITY) ? 0.f : m;
             // ---- probabilities, row sum, bf16 P into TMEM columns [0, 64) of S_j,
-            // 32 columns at a time so each chunk's scores die once packed
-            float sum0 = 0.f, sum1 = 0.f;
+            // 32 columns at a time so each chunk's scores die once packed.  The
+            // scale-subtract and the row sum run as packed fp32x2 instructions.
+            {
+                const uint64_t sl2x2 = f2_pack(sl2, sl2);
+                const uint64_t nmux2 = f2_pack(-mu, -mu);
+                uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = f2_pack(0.f, 0.f);
+                const bool emu = kEmuMod > 0 && !seq.partial(j);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint32_t pk[16];
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float e0 = ex2_approx(fmaf(s[32 * q4 + 2 * i], sl2, -mu));
-                    const float e1 = ex2_approx(fmaf(s[32 * q4 + 2 * i + 1], sl2, -mu));
-                    sum0 += e0;
-                    sum1 += e1;
-                    pk[i] = pack_bf16x2(e0, e1);
+                    for (int i = 0; i < 16; ++i) {
+                        float e0, e1;
+                        f2_unpack(f2_fma(f2_pack(s[32 * q4 + 2 * i], s[32 * q4 + 2 * i + 1]), sl2x2, nmux2), e0, e1);
+                        if (kEmuMod > 0 && (i % (kEmuMod > 0 ? kEmuMod : 1)) == kEmuMod - 1 && emu) {
+                            exp2_fma2(e0, e1);
+                        } else {
+                            e0 = ex2_approx(e0);
+                            e1 = ex2_approx(e1);
+                        }
+                        const uint64_t e01 = f2_pack(e0, e1);
+                        if (i & 1) acc1 = f2_add(acc1, e01); else acc0 = f2_add(acc0, e01);
+                        pk[i] = pack_bf16x2(e0, e1);
+                    }
+                    tmem_st16(s_tmem + 16 * q4, pk);
                 }
-                tmem_st16(s_tmem + 16 * q4, pk);
+                float a0, a1, a2, a3;
+                f2_unpack(acc0, a0, a1);
+                f2_unpack(acc1, a2, a3);
+                l += (a0 + a1) + (a2 + a3);
             }
-            l += sum0 + sum1;
             if (rescale) {
                 // O must hold every earlier tile's P V before it is rescaled
                 const bool okw = mbar_wait(bar(C::B_PV + j), (c - 1) & 1, w);

@@ -257,7 +257,76 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// TMEM -> registers without waiting: 64 columns into floats.  The values are
+// valid only after tmem_wait_ld_dep() names the same registers.
+#define CP_F8(b) "=f"(v[b + 0]), "=f"(v[b + 1]), "=f"(v[b + 2]), "=f"(v[b + 3]), \
+                 "=f"(v[b + 4]), "=f"(v[b + 5]), "=f"(v[b + 6]), "=f"(v[b + 7])
+__device__ __forceinline__ void tmem_ld64f_nowait(uint32_t taddr, float *v)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+        : CP_F8(0), CP_F8(8), CP_F8(16), CP_F8(24), CP_F8(32), CP_F8(40), CP_F8(48), CP_F8(56)
+        : "r"(taddr)
+        : "memory");
+}
+#undef CP_F8
+
+// Waits for this thread's outstanding TMEM loads and ties the 64 registers v[] to
+// the wait, so no use of them is scheduled before it.
+#define CP_D8(b) "+f"(v[b + 0]), "+f"(v[b + 1]), "+f"(v[b + 2]), "+f"(v[b + 3]), \
+                 "+f"(v[b + 4]), "+f"(v[b + 5]), "+f"(v[b + 6]), "+f"(v[b + 7])
+__device__ __forceinline__ void tmem_wait_ld_dep(float *v)
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : CP_D8(0), CP_D8(8), CP_D8(16), CP_D8(24), CP_D8(32), CP_D8(40), CP_D8(48), CP_D8(56)
+                 :
+                 : "memory");
+}
+// Compiler-only dependency on 64 more registers (after a tmem_wait_ld_dep()).
+__device__ __forceinline__ void reg_dep64(float *v)
+{
+    asm volatile(""
+                 : CP_D8(0), CP_D8(8), CP_D8(16), CP_D8(24), CP_D8(32), CP_D8(40), CP_D8(48), CP_D8(56));
+}
+#undef CP_D8
+
 // ------------------------------------------------------------------ math helpers
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Packed fp32 pair arithmetic (one instruction for two lanes of work).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
 
 __device__ __forceinline__ float ex2_approx(float x)
 {
