@@ -115,10 +115,12 @@ def cpu_oracle_rate(w, seconds_target=12.0, seed=0):
         pairs = sum((int(p) + 1) if w.causal else w.S for _, _, p in sel)
         return 4.0 * w.d * pairs / dt / 1e12, dt
 
-    _, dt = run(threads)
-    n = max(threads, int(threads * seconds_target / max(dt, 1e-3)))
-    n = min(n, 200000)
+    # grow the sample until one run takes about seconds_target
+    n = threads
     rate, dt = run(n)
+    while dt < 0.5 * seconds_target and n < 400000:
+        n = min(400000, int(n * min(8.0, max(1.5, seconds_target / max(dt, 1e-3)))))
+        rate, dt = run(n)
     return rate, "%d random query rows of %s (%.1f s of fp64 CPU work)" % (n, w.name, dt), threads
 
 
@@ -131,8 +133,10 @@ def run_reference(args):
     per = []
     desc = ""
     threads = 0
+    # keep the whole run to a few minutes
+    per_step = min(args.ref_seconds, 150.0 / (args.warmup + args.steps))
     for i in range(args.warmup + args.steps):
-        rate, desc, threads = cpu_oracle_rate(w, seconds_target=args.ref_seconds, seed=i)
+        rate, desc, threads = cpu_oracle_rate(w, seconds_target=per_step, seed=i)
         if i >= args.warmup:
             per.append(rate)
     value = statistics.mean(per)

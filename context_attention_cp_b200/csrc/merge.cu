@@ -7,11 +7,12 @@
 // A side with lse = -inf is empty and contributes nothing; two empty sides give
 // (0, -inf).
 //
-// Work split: a group of d/8 threads owns one (batch, token, head) row; each thread
-// moves 8 elements with 16-byte accesses (two float4 of the fp32 accumulator, one
-// 16-byte load of bf16 partials or two float4 of fp32 partials).  Rows are visited
-// in memory order of the [b, s, H, d] tensors, so consecutive groups touch
-// consecutive addresses.  Bytes per row: (8 + sizeof(o_b)) * d + 12.
+// Work split: one CTA per (batch, 8 consecutive positions); the LSE weights of
+// its (head, position) pairs are computed once into shared memory, then d/8
+// threads per (position, head) row move 8 elements each with 16-byte streaming
+// accesses (two float4 of the fp32 accumulator, one 16-byte load of bf16 partials
+// or two float4 of fp32 partials), consecutive threads on consecutive addresses.
+// Bytes per row: (8 + sizeof(o_b)) * d + 12.
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -55,54 +56,102 @@ __device__ __forceinline__ void store8(void *base, int dtype, int64_t off, const
     }
 }
 
-__global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ MergeParams p)
+constexpr int MT = 256;  // threads per CTA
+#ifndef CP_MERGE_TS
+#define CP_MERGE_TS 8
+#endif
+#ifndef CP_MERGE_U
+#define CP_MERGE_U 2
+#endif
+#ifndef CP_MERGE_CTAS_PER_SM
+#define CP_MERGE_CTAS_PER_SM 4
+#endif
+constexpr int TS = CP_MERGE_TS;  // sequence positions per work item
+
+// One CTA merges TS consecutive positions of one batch row, all heads.
+//   Phase 1: the LSE weights w_acc = e^{lse_acc - lse}, w_b = e^{lse_b - lse} and the
+//   new lse of every (head, position) go to shared memory (lse reads are coalesced
+//   along the sequence).  Phase 2: the o rows stream through with 16-byte accesses,
+//   thread t owning elements [8 (t % (D/8)), +8) of head h0 + t / (D/8).
+template <int D>
+__global__ void __launch_bounds__(MT, CP_MERGE_CTAS_PER_SM) lse_merge_kernel(const __grid_constant__ MergeParams p)
 {
-    const int gpr = (int)(p.d / 8);  // threads per row; divides 32, so a row never spans warps
-    const int64_t rows = p.b * p.s * p.h;
-    const int64_t total = rows * gpr;
-    const int lane = threadIdx.x & 31;
-    const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    // the loop bound is uniform per warp, so __syncwarp() below sees every lane
-    for (int64_t base = warp_id * 32; base < total; base += n_warps * 32) {
-        const int64_t idx = base + lane;
-        const bool active = idx < total;
-        const int64_t r = active ? idx / gpr : 0;
-        const int part = (int)(idx - r * gpr);
-        const int64_t hh = r % p.h;
-        const int64_t ss = (r / p.h) % p.s;
-        const int64_t bb = r / (p.h * p.s);
-        float *la_ptr = p.lse_acc + bb * p.la_sb + hh * p.la_sh + ss * p.la_ss;
-        float lse = -INFINITY;
-        if (active) {
-            const float la = *la_ptr;
-            const float lb = p.lse_b[bb * p.lb_sb + hh * p.lb_sh + ss * p.lb_ss];
-            const float M = fmaxf(la, lb);
-            float wa = 0.f, wb = 0.f;
-            if (M != -INFINITY) {
-                lse = M + logf(__expf(la - M) + __expf(lb - M));
-                wa = __expf(la - lse);
-                wb = __expf(lb - lse);
+    extern __shared__ float wsm[];  // [2][H][TS]
+    const int H = (int)p.h;
+    float *wa_s = wsm;
+    float *wb_s = wsm + H * TS;
+    const int tid = threadIdx.x;
+    const int64_t tiles_per_b = (p.s + TS - 1) / TS;
+    const int64_t n_work = tiles_per_b * p.b;
+    // persistent: the grid strides over (batch, position tile) work items
+    for (int64_t wk = blockIdx.x; wk < n_work; wk += gridDim.x) {
+    const int64_t bb = wk / tiles_per_b;
+    const int64_t s0 = (wk - bb * tiles_per_b) * TS;
+    const int ns = (int)min((int64_t)TS, p.s - s0);
+
+    for (int i = tid; i < H * TS; i += MT) {
+        const int hh = i / TS, t = i % TS;
+        if (t >= ns) continue;
+        float *la_ptr = p.lse_acc + bb * p.la_sb + hh * p.la_sh + (s0 + t) * p.la_ss;
+        const float la = *la_ptr;
+        const float lb = p.lse_b[bb * p.lb_sb + hh * p.lb_sh + (s0 + t) * p.lb_ss];
+        const float M = fmaxf(la, lb);
+        float wa = 0.f, wb = 0.f, lse = -INFINITY;
+        if (M != -INFINITY) {
+            lse = M + logf(__expf(la - M) + __expf(lb - M));
+            // an empty side may hold anything in o: its weight is exactly 0
+            wa = (la == -INFINITY) ? 0.f : __expf(la - lse);
+            wb = (lb == -INFINITY) ? 0.f : __expf(lb - lse);
+        }
+        wa_s[i] = wa;
+        wb_s[i] = wb;
+        *la_ptr = lse;
+    }
+    __syncthreads();
+
+    constexpr int TPR = D / 8;     // threads per (position, head) row
+    constexpr int HPB = MT / TPR;  // heads per pass
+    constexpr int U = CP_MERGE_U;  // rows in flight per thread
+    const int part = tid % TPR;
+    const int hl = tid / TPR;
+    const int passes = (H + HPB - 1) / HPB;
+    const int items = ns * passes;  // (position, head pass) pairs
+    for (int it0 = 0; it0 < items; it0 += U) {
+        float a[U][8], bv[U][8];
+        float wa[U], wb[U];
+        int64_t oa_off[U], out_off[U];
+        bool ok[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int it = it0 + u;
+            const int t = it / passes;
+            const int hh = (it - t * passes) * HPB + hl;
+            ok[u] = it < items && hh < H;
+            const int64_t ss = s0 + t;
+            wa[u] = ok[u] ? wa_s[hh * TS + t] : 0.f;
+            wb[u] = ok[u] ? wb_s[hh * TS + t] : 0.f;
+            oa_off[u] = bb * p.oa_sb + ss * p.oa_ss + (int64_t)hh * p.oa_sh + part * 8;
+            out_off[u] = p.o_out ? bb * p.out_sb + ss * p.out_ss + (int64_t)hh * p.out_sh + part * 8 : oa_off[u];
+            if (ok[u]) {
+                load8(p.o_b, p.ob_dtype, bb * p.ob_sb + ss * p.ob_ss + (int64_t)hh * p.ob_sh + part * 8, bv[u]);
+                if (wa[u] != 0.f) load8(p.o_acc, DT_FP32, oa_off[u], a[u]);
             }
-            const int64_t oa_off = bb * p.oa_sb + ss * p.oa_ss + hh * p.oa_sh + part * 8;
-            const int64_t ob_off = bb * p.ob_sb + ss * p.ob_ss + hh * p.ob_sh + part * 8;
-            float a[8], b[8], o[8];
-            load8(p.o_acc, DT_FP32, oa_off, a);
-            load8(p.o_b, p.ob_dtype, ob_off, b);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (!ok[u]) continue;
+            float o[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                // an empty side may hold anything; select instead of multiplying by 0
-                const float ta = (la == -INFINITY) ? 0.f : wa * a[i];
-                const float tb = (lb == -INFINITY) ? 0.f : wb * b[i];
+                const float ta = (wa[u] != 0.f) ? wa[u] * a[u][i] : 0.f;
+                const float tb = (wb[u] != 0.f) ? wb[u] * bv[u][i] : 0.f;
                 o[i] = ta + tb;
             }
-            if (p.o_out)
-                store8(p.o_out, p.out_dtype, bb * p.out_sb + ss * p.out_ss + hh * p.out_sh + part * 8, o);
-            else
-                store8(p.o_acc, DT_FP32, oa_off, o);
+            if (p.o_out) store8(p.o_out, p.out_dtype, out_off[u], o);
+            else store8(p.o_acc, DT_FP32, out_off[u], o);
         }
-        __syncwarp();  // every lane of the row has read lse_acc before it is replaced
-        if (active && part == 0) *la_ptr = lse;
+    }
+    __syncthreads();  // the weights of this item are consumed before the next item's
     }
 }
 
@@ -110,15 +159,24 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ 
 
 cudaError_t launch_lse_merge(const MergeParams &p, cudaStream_t stream)
 {
-    const int64_t total = p.b * p.s * p.h * (p.d / 8);
-    if (total == 0) return cudaSuccess;
+    if (p.b * p.s * p.h == 0) return cudaSuccess;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t blocks = (total + 255) / 256;
-    const int64_t cap = (int64_t)sms * 8;  // 8 resident 256-thread blocks per SM
-    if (blocks > cap) blocks = cap;
-    lse_merge_kernel<<<(unsigned)blocks, 256, 0, stream>>>(p);
+    const int64_t n_work = (p.s + TS - 1) / TS * p.b;
+    const int64_t cap = (int64_t)sms * CP_MERGE_CTAS_PER_SM;
+    const unsigned grid = (unsigned)(n_work < cap ? n_work : cap);
+    const size_t smem = 2 * (size_t)p.h * TS * sizeof(float);
+    if (smem > 48 * 1024) return cudaErrorInvalidValue;
+    switch (p.d) {
+    case 8: lse_merge_kernel<8><<<grid, MT, smem, stream>>>(p); break;
+    case 16: lse_merge_kernel<16><<<grid, MT, smem, stream>>>(p); break;
+    case 32: lse_merge_kernel<32><<<grid, MT, smem, stream>>>(p); break;
+    case 64: lse_merge_kernel<64><<<grid, MT, smem, stream>>>(p); break;
+    case 128: lse_merge_kernel<128><<<grid, MT, smem, stream>>>(p); break;
+    case 256: lse_merge_kernel<256><<<grid, MT, smem, stream>>>(p); break;
+    default: return cudaErrorInvalidValue;
+    }
     return cudaGetLastError();
 }
 
