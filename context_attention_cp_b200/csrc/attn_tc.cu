@@ -44,8 +44,14 @@ namespace {
 constexpr int BM = 128;  // query rows per tile (TMEM lanes)
 constexpr int BN = 128;  // keys per tile
 constexpr int NQ = 2;    // query tiles per CTA
-constexpr int NSK = 2;   // K stages
-constexpr int NSV = 2;   // V stages
+#ifndef CP_ATTN_NSK
+#define CP_ATTN_NSK 2
+#endif
+#ifndef CP_ATTN_NSV
+#define CP_ATTN_NSV 2
+#endif
+constexpr int NSK = CP_ATTN_NSK;  // K stages
+constexpr int NSV = CP_ATTN_NSV;  // V stages
 constexpr int NTHREADS = 384;
 constexpr int REGS_SOFTMAX = 208;
 constexpr int REGS_OTHER = 88;
@@ -84,6 +90,7 @@ struct Cfg {
     };
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 64 + 1024;  // + alignment slack
+    static_assert(SMEM <= 232448, "shared memory per CTA exceeds 227 KB");
     static constexpr int T_O = 256;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false);
@@ -202,7 +209,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int i = 0; i < NSV; ++i) { mbar_init(bar(C::B_VF + i), 1); mbar_init(bar(C::B_VE + i), 1); }
         for (int j = 0; j < NQ; ++j) {
             mbar_init(bar(C::B_SF + j), 1);
-            mbar_init(bar(C::B_PF + j), BM);
+            mbar_init(bar(C::B_PF + j), BM / 32);  // one arrival per softmax warp
             mbar_init(bar(C::B_PV + j), 1);
         }
         mbar_init(bar(C::B_DONE), 1);
@@ -490,7 +497,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(C::B_PF + j));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_PF + j));
             ++c;
         }
         aborted = __any_sync(0xffffffffu, aborted || (*abort_flag != 0));

@@ -50,9 +50,23 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
                  : "memory");
 }
 
+// One probe of the phase with parity `parity`.  try_wait may park the thread for
+// a short while until the phase completes; test_wait returns at once.
+#ifndef CP_MBAR_TEST_WAIT
+#define CP_MBAR_TEST_WAIT 0
+#endif
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
+#if CP_MBAR_TEST_WAIT
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -60,6 +74,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
         : "=r"(ok)
         : "r"(bar), "r"(parity)
         : "memory");
+#endif
     return ok != 0;
 }
 
