@@ -89,6 +89,9 @@ cp_status check_range(const cp_range *r, int64_t len, const char *name)
                                          (long long)range_len(x), (long long)len);
     if (!range_increasing(x) || x.start0 < 0)
         return fail(CP_ERR_INVALID_ARG, "%s: positions must be >= 0 and increase with the local index", name);
+    const int64_t last = len > 0 ? range_pos(x, len - 1) : 0;
+    if (last >= ((int64_t)1 << 30))
+        return fail(CP_ERR_UNSUPPORTED, "%s: positions must stay below 2^30", name);
     return CP_OK;
 }
 
@@ -404,7 +407,7 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     const int64_t S = q->shape[1];
     if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
     if (N < 1 || N > 4096) return fail(CP_ERR_INVALID_ARG, "N must be in [1, 4096]");
-    if (S > INT32_MAX / 2) return fail(CP_ERR_SHAPE, "sequence too long");
+    if (S >= ((int64_t)1 << 30)) return fail(CP_ERR_SHAPE, "sequence too long (S must be below 2^30)");
     if (S % N) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of N = %d", (long long)S, N);
     if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N)) return fail(CP_ERR_SHAPE, "zig-zag needs S to be a multiple of 2N");
     if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;

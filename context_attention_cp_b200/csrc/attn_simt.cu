@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(RM) attn_simt_kernel(const __grid_constant__ A
         const int src = ((rank - step) % N + N) % N;
         const Range kr = p.use_layout ? layout_range(p.layout, N, p.seq_len, src) : p.kv_range;
         int kt_full, kt_end;
-        kv_tile_bounds(qr, p.q_len, q_lo, RM, kr, p.kv_len, RN, p.causal != 0, &kt_full, &kt_end);
+        kv_tile_bounds<int64_t>(qr, p.q_len, q_lo, RM, kr, p.kv_len, RN, p.causal != 0, &kt_full, &kt_end);
         if (kt_end == 0) continue;
         any_key_tile = true;
         float m = -INFINITY, l = 0.f;

@@ -131,11 +131,11 @@ struct TileSeq {
             const int N = p->n_ranks;
             src = ((rank - step) % N + N) % N;
             kr = p->use_layout ? layout_range(p->layout, N, p->seq_len, src) : p->kv_range;
-            kv_tile_bounds(qr, p->q_len, q_lo0, BM, kr, p->kv_len, BN, p->causal != 0, &kt_full0, &kt_end0);
+            kv_tile_bounds<int64_t>(qr, p->q_len, q_lo0, BM, kr, p->kv_len, BN, p->causal != 0, &kt_full0, &kt_end0);
             kt_full1 = kt_end1 = 0;
             if (q_ok1)
-                kv_tile_bounds(qr, p->q_len, q_lo0 + BM, BM, kr, p->kv_len, BN, p->causal != 0, &kt_full1,
-                               &kt_end1);
+                kv_tile_bounds<int64_t>(qr, p->q_len, q_lo0 + BM, BM, kr, p->kv_len, BN, p->causal != 0, &kt_full1,
+                                        &kt_end1);
             kt_end_all = kt_end0 > kt_end1 ? kt_end0 : kt_end1;
             kt = 0;
         }

@@ -27,16 +27,32 @@ namespace cpattn {
 enum { LAYOUT_CONTIGUOUS = 0, LAYOUT_ZIGZAG = 1, LAYOUT_STRIPED = 2 };
 enum { TILE_SKIP = 0, TILE_FULL = 1, TILE_PARTIAL = 2 };
 
-// Position map of one rank's (or one block's) local tokens.
-struct Range {
-    int64_t start0, start1;  // first position of segment 0 / 1
-    int64_t len0, len1;      // tokens in segment 0 / 1 (len1 = 0 for one segment)
-    int64_t stride;          // position step between neighbouring local tokens
+// Position map of one rank's (or one block's) local tokens.  The host uses 64-bit
+// fields; the kernels use the 32-bit form (positions stay below 2^30, which the
+// ABI checks).
+template <typename I>
+struct RangeT {
+    I start0, start1;  // first position of segment 0 / 1
+    I len0, len1;      // tokens in segment 0 / 1 (len1 = 0 for one segment)
+    I stride;          // position step between neighbouring local tokens
 };
+using Range = RangeT<int64_t>;
+using Range32 = RangeT<int32_t>;
+
+template <typename I>
+CP_HD I range_pos(const RangeT<I> &r, I t)
+{
+    return t < r.len0 ? r.start0 + t * r.stride : r.start1 + (t - r.len0) * r.stride;
+}
 
 CP_HD int64_t range_pos(const Range &r, int64_t t)
 {
     return t < r.len0 ? r.start0 + t * r.stride : r.start1 + (t - r.len0) * r.stride;
+}
+
+CP_HD Range32 to_range32(const Range &r)
+{
+    return Range32{(int32_t)r.start0, (int32_t)r.start1, (int32_t)r.len0, (int32_t)r.len1, (int32_t)r.stride};
 }
 
 CP_HD int64_t range_len(const Range &r) { return r.len0 + r.len1; }
@@ -50,18 +66,19 @@ CP_HD bool range_increasing(const Range &r)
 }
 
 // Range of rank `rank` in a sequence of S tokens split over N ranks.
-CP_HD Range layout_range(int layout, int N, int64_t S, int rank)
+template <typename I>
+CP_HD RangeT<I> layout_range_t(int layout, int N, I S, int rank)
 {
-    Range r;
-    int64_t c = S / N;
+    RangeT<I> r;
+    I c = S / N;
     r.start1 = 0;
     r.len1 = 0;
     r.stride = 1;
     if (layout == LAYOUT_ZIGZAG) {
-        int64_t h = c / 2;
+        I h = c / 2;
         r.start0 = rank * h;
         r.len0 = h;
-        r.start1 = (int64_t)(2 * N - 1 - rank) * h;
+        r.start1 = (I)(2 * N - 1 - rank) * h;
         r.len1 = h;
     } else if (layout == LAYOUT_STRIPED) {
         r.start0 = rank;
@@ -74,11 +91,14 @@ CP_HD Range layout_range(int layout, int N, int64_t S, int rank)
     return r;
 }
 
+CP_HD Range layout_range(int layout, int N, int64_t S, int rank) { return layout_range_t<int64_t>(layout, N, S, rank); }
+
 // For query tile [q_lo, q_lo + tile_q) of a block of q_len rows (ranges q) against a
 // key block of kv_len rows (ranges k) cut into tiles of tile_k: key tiles
 // [0, *kt_full) are FULL, [*kt_full, *kt_end) PARTIAL, [*kt_end, n_kt) SKIP.
-CP_HD void kv_tile_bounds(const Range &q, int64_t q_len, int64_t q_lo, int tile_q, const Range &k,
-                          int64_t kv_len, int tile_k, bool causal, int *kt_full, int *kt_end)
+template <typename I>
+CP_HD void kv_tile_bounds(const RangeT<I> &q, I q_len, I q_lo, int tile_q, const RangeT<I> &k, I kv_len, int tile_k,
+                          bool causal, int *kt_full, int *kt_end)
 {
     int n_kt = (int)((kv_len + tile_k - 1) / tile_k);
     bool ragged = (kv_len % tile_k) != 0;
@@ -87,14 +107,14 @@ CP_HD void kv_tile_bounds(const Range &q, int64_t q_len, int64_t q_lo, int tile_
         *kt_full = ragged ? n_kt - 1 : n_kt;
         return;
     }
-    int64_t q_hi = q_lo + tile_q - 1;
+    I q_hi = q_lo + tile_q - 1;
     if (q_hi > q_len - 1) q_hi = q_len - 1;
-    int64_t qmin = range_pos(q, q_lo), qmax = range_pos(q, q_hi);
+    const I qmin = range_pos(q, q_lo), qmax = range_pos(q, q_hi);
     // kt_end: number of tiles whose first key is visible to the last query row.
     int lo = 0, hi = n_kt;  // answer in [lo, hi]
     while (lo < hi) {
         int mid = (lo + hi) / 2;
-        if (range_pos(k, (int64_t)mid * tile_k) <= qmax) lo = mid + 1; else hi = mid;
+        if (range_pos(k, (I)mid * tile_k) <= qmax) lo = mid + 1; else hi = mid;
     }
     *kt_end = lo;
     // kt_full: number of leading tiles that are whole (inside kv_len) and whose last
@@ -104,7 +124,7 @@ CP_HD void kv_tile_bounds(const Range &q, int64_t q_len, int64_t q_lo, int tile_
     if (hi > *kt_end) hi = *kt_end;
     while (lo < hi) {
         int mid = (lo + hi) / 2;
-        if (range_pos(k, (int64_t)mid * tile_k + tile_k - 1) <= qmin) lo = mid + 1; else hi = mid;
+        if (range_pos(k, (I)mid * tile_k + tile_k - 1) <= qmin) lo = mid + 1; else hi = mid;
     }
     *kt_full = lo;
 }
