@@ -92,6 +92,31 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+KERNEL_SOURCES = ["context_attention_cp_b200/csrc/attn_tc.cu", "context_attention_cp_b200/csrc/ptx.cuh",
+                  "context_attention_cp_b200/csrc/layout.h", "context_attention_cp_b200/csrc/kernels.h",
+                  "context_attention_cp_b200/csrc/exp2_poly.h"]
+
+
+def profiled_traffic(profile="profiles/attn_tc_kernel_llama3_8b_s8k_zigzag4.md"):
+    """DRAM bytes per launch from the committed ncu summary, or None when the kernel
+    sources changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, profile)) as f:
+            text = f.read()
+        h = hashlib.sha256()
+        for name in KERNEL_SOURCES:
+            with open(os.path.join(ROOT, name), "rb") as f:
+                h.update(f.read())
+    except OSError:
+        return None
+    rec = dict(ln.split(":", 1) for ln in text.splitlines() if ln.startswith(("traffic_bytes_per_launch:",
+                                                                              "source_sha256:")))
+    if rec.get("source_sha256", "").strip() != h.hexdigest():
+        return None
+    return int(rec["traffic_bytes_per_launch"].strip())
+
+
 def cpu_oracle_rate(w, seconds_target=12.0, seed=0):
     """Times the fp64 oracle on a bounded sample of query rows of the workload.
 
@@ -320,7 +345,8 @@ def main():
             "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel",
                          "achieved": per_launch_tflops, "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": (per_launch_tflops / peak_tf) if per_launch_tflops else None,
-                         "peak_source": peak_src + " bf16 burst", "traffic": None},
+                         "peak_source": peak_src + " bf16 burst",
+                         "traffic": profiled_traffic() if w.name == W.BENCH_WORKLOAD else None},
             "merge": merge,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

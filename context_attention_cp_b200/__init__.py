@@ -17,6 +17,6 @@ Tensors are torch tensors on the current CUDA device; token tensors are
 """
 from ._binding import (  # noqa: F401
     CPError, LAYOUTS, MODES, block_attn_fwd, layout_permute, layout_range, lib, lib_path,
-    lse_merge, ring_attn_fwd, ring_attn_fwd_static_scratch, ring_workspace_bytes, stream_check,
-    tile_classes,
+    lse_merge, ring_attn_fwd, ring_attn_fwd_static_scratch, ring_workspace_bytes, selftest_wait_timeout,
+    stream_check, tile_classes,
 )

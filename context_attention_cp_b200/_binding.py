@@ -41,6 +41,7 @@ _SIGNATURES = {
     "cp_layout_range": (_i32, [_i32, _i32, _i64, _i32, _R]),
     "cp_tile_classes": (_i32, [_R, _i64, _R, _i64, _i32, _i32, _i32, ctypes.POINTER(ctypes.c_int8)]),
     "cp_stream_check": (_i32, [_vp]),
+    "cp_selftest_wait_timeout": (_i32, [ctypes.c_uint64, _vp]),
     "cp_ring_attn_fwd_static_scratch": (_i32, [_i32, _i32, _i32, _T, _T, _T, _f32, _T, _T, _vp]),
     "cp_status_string": (ctypes.c_char_p, [_i32]),
     "cp_last_error": (ctypes.c_char_p, []),
@@ -205,6 +206,11 @@ def layout_permute(x, layout, N, seq_axis=1, inverse=False, out=None):
     else:
         _check(lib().cp_layout_permute(LAYOUTS[layout], N, seq_axis, _ref(tx), _ref(to), 0, _stream()))
     return out
+
+
+def selftest_wait_timeout(limit_ns=20_000_000):
+    """Launch the bounded-wait self-test kernel (its wait is made to expire)."""
+    _check(lib().cp_selftest_wait_timeout(int(limit_ns), _stream()))
 
 
 def stream_check():

@@ -519,6 +519,16 @@ cp_status cp_layout_permute(int32_t layout, int32_t N, int32_t seq_axis, const c
     return CP_OK;
 }
 
+cp_status cp_selftest_wait_timeout(uint64_t limit_ns, void *stream)
+{
+    g_last_error[0] = 0;
+    if (limit_ns < 1000000ull || limit_ns > 1000000000ull)
+        return fail(CP_ERR_INVALID_ARG, "limit_ns must be in [1 ms, 1 s]");
+    cudaError_t e = launch_wait_timeout_selftest(limit_ns, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+    return CP_OK;
+}
+
 cp_status cp_stream_check(void *stream)
 {
     g_last_error[0] = 0;

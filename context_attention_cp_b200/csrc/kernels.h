@@ -87,6 +87,10 @@ cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream);
 // Device status word of the current device (2 ints), from status.cu.
 cudaError_t status_word(int **ptr);
 
+// Launches a one-warp kernel whose bounded mbarrier wait is made to expire after
+// limit_ns (nothing arrives), raising the timeout bit of the status word.
+cudaError_t launch_wait_timeout_selftest(uint64_t limit_ns, cudaStream_t stream);
+
 // Records a printf-style message for cp_last_error() and returns `status` (abi.cu).
 cp_status report_error(cp_status status, const char *fmt, ...);
 

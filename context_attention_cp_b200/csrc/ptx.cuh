@@ -86,9 +86,11 @@ struct WaitCtx {
     int where;            // tag stored on expiry
 };
 
-// Waits until the phase with parity `parity` of `bar` completed.  Returns false if
-// the CTA was aborted or the wait expired (then STATUS_TIMEOUT is raised).
-static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx &w)
+// Waits until the phase with parity `parity` of `bar` completed, for at most
+// limit_ns.  Returns false if the CTA was aborted or the wait expired (then
+// STATUS_TIMEOUT is raised in the device status word and the CTA's abort flag set).
+static __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, const WaitCtx &w,
+                                                      uint64_t limit_ns)
 {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = global_timer_ns();
@@ -97,7 +99,7 @@ static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, 
         if ((i & 63) == 0) {
             if (*w.abort) return false;
             if (*(volatile int *)w.status & STATUS_TIMEOUT) { *w.abort = 1; return false; }
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 atomicOr(w.status, STATUS_TIMEOUT);
                 atomicCAS(w.status + 1, 0, w.where);
                 *w.abort = 1;
@@ -105,6 +107,11 @@ static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, 
             }
         }
     }
+}
+
+static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx &w)
+{
+    return mbar_wait_limit(bar, parity, w, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------ TMA

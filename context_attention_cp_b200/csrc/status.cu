@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace cpattn {
 
@@ -26,6 +27,39 @@ cudaError_t status_word(int **ptr)
     if (dev >= 0 && dev < kMaxDevices) cached[dev] = static_cast<int *>(addr);
     *ptr = static_cast<int *>(addr);
     return cudaSuccess;
+}
+
+namespace {
+
+// One warp waits on an mbarrier that nothing ever arrives at; the bounded wait runs
+// out after limit_ns and reports through the status word, the way every wait in the
+// attention kernels does.  The kernel then returns normally.
+__global__ void wait_timeout_kernel(int *status, uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&mbar), 1);
+        abort_flag = 0;
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        WaitCtx w{&abort_flag, status, 99};
+        mbar_wait_limit(smem_u32(&mbar), 0, w, limit_ns);
+    }
+    __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_wait_timeout_selftest(uint64_t limit_ns, cudaStream_t stream)
+{
+    int *word = nullptr;
+    cudaError_t e = status_word(&word);
+    if (e != cudaSuccess) return e;
+    wait_timeout_kernel<<<1, 32, 0, stream>>>(word, limit_ns);
+    return cudaGetLastError();
 }
 
 }  // namespace cpattn

@@ -167,6 +167,15 @@ cp_status cp_tile_classes(const cp_range *q_range, int64_t q_len, const cp_range
  * check, CP_ERR_CUDA if the stream reported an error, else CP_OK. */
 cp_status cp_stream_check(void *stream);
 
+/* Failure-detection self-test: launches on `stream` a one-warp kernel that waits on
+ * a barrier nothing ever completes, with the same bounded wait every kernel of this
+ * library uses, cut to limit_ns (1 ms .. 1 s).  The wait expires, the kernel sets the
+ * device status word and returns normally; the next cp_stream_check(stream) then
+ * reports CP_ERR_TIMEOUT (and clears the word).  The context stays usable.
+ * Returns CP_ERR_INVALID_ARG for a limit outside the range.  No counterpart on the
+ * pages: it exercises this library's own fault reporting. */
+cp_status cp_selftest_wait_timeout(uint64_t limit_ns, void *stream);
+
 /* Static description of a status code. */
 const char *cp_status_string(cp_status s);
 

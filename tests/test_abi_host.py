@@ -204,3 +204,9 @@ def test_merge_and_permute_argument_errors(cp):
     assert g(0, 2, 1, ctypes.byref(x), ctypes.byref(x), 0, None) == 1       # overlap
     assert cp.lib().cp_ring_workspace_bytes(0, 4, 0, 0, 1, 256, 4, 128) == 0  # fused needs none
     assert cp.lib().cp_ring_workspace_bytes(0, 4, 1, 0, 1, 256, 4, 128) >= 256 * 4 * 128 * 6
+
+
+def test_selftest_limit_is_checked_before_any_launch(cp):
+    f = cp.lib().cp_selftest_wait_timeout
+    assert f(10, None) == 1             # below 1 ms
+    assert f(5_000_000_000, None) == 1  # above 1 s
