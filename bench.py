@@ -117,6 +117,17 @@ def profiled_traffic(profile="profiles/attn_tc_kernel_llama3_8b_s8k_zigzag4.md")
     return int(rec["traffic_bytes_per_launch"].strip())
 
 
+def reduce_max(value, world, device):
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def cpu_oracle_rate(w, seconds_target=12.0, seed=0):
     """Times the fp64 oracle on a bounded sample of query rows of the workload.
 
@@ -249,11 +260,7 @@ def main():
     clk = clocks.stop() if clocks else None
     cp.stream_check()
     times = [s.elapsed_time(e) for s, e in zip(starts, ends)]  # ms
-    total_ms = sum(times)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(sum(times), world, dev)
     ms_per_step = total_ms / args.steps
     flops = w.effective_flops()
     value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
@@ -317,11 +324,7 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms = reduce_max(e0.elapsed_time(e1), world, dev)
     e2e_value = world * flops * e_steps / (e_ms * 1e-3) / 1e12
     es = 2 if w.dtype == "bf16" else 4
     h2d = (q.numel() + k.numel() + v.numel()) * es
