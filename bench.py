@@ -270,60 +270,92 @@ def main():
     per_launch_tflops = flops / (ms_per_step * 1e-3) / 1e12 if args.mode == "fused" else None
     peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
 
-    # standalone merge bandwidth on this workload's partial size: (N-1) merges of
-    # [b, S, Hq, d] per ring, bytes per (row, head) = (8 + 2) * d + 12
-    merge = None
-    if w.dtype == "bf16" and rank == 0:
-        oa = torch.randn((w.b, w.S, w.hq, w.d), device=dev)
-        ob = torch.randn((w.b, w.S, w.hq, w.d), device=dev).to(torch.bfloat16)
-        la = torch.randn((w.b, w.hq, w.S), device=dev)
-        lb = torch.randn((w.b, w.hq, w.S), device=dev)
+    # standalone merge bandwidth: one merge of a [b, S, Hq, d] fp32 accumulator with a
+    # bf16 partial, bytes per (row, head) = (8 + 2) * d + 12; measured at this
+    # workload's partial size and at the non-causal 64K workload's (16 heads), the
+    # case with 31 merges per rank
+    def merge_gbs(b, S, H, d):
+        oa = torch.randn((b, S, H, d), device=dev)
+        ob = torch.randn((b, S, H, d), device=dev).to(torch.bfloat16)
+        la = torch.randn((b, H, S), device=dev)
+        lb = torch.randn((b, H, S), device=dev)
         for _ in range(3):
             cp.lse_merge(oa, la, ob, lb)
         ms = []
         for _ in range(10):
             flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
+            m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            m0.record(stream)
             cp.lse_merge(oa, la, ob, lb)
-            e1.record(stream)
+            m1.record(stream)
             torch.cuda.synchronize()
-            ms.append(e0.elapsed_time(e1))
-        rows = w.b * w.S * w.hq
-        mbytes = rows * ((8 + 2) * w.d + 12)
-        gbs = mbytes / (statistics.mean(ms) * 1e-3) / 1e9
-        merge = {"gbs": gbs, "frac_of_measured_hbm": gbs / peaks.get("hbm_gbs", 6650.0),
-                 "frac_of_8tbs": gbs / 8000.0, "bytes_per_launch": mbytes, "ms_per_launch": statistics.mean(ms)}
+            ms.append(m0.elapsed_time(m1))
+        mbytes = b * S * H * ((8 + 2) * d + 12)
+        t = statistics.mean(ms)
+        gbs = mbytes / (t * 1e-3) / 1e9
         del oa, ob, la, lb
+        return {"shape": [b, S, H, d], "gbs": gbs, "frac_of_measured_hbm": gbs / peaks.get("hbm_gbs", 6650.0),
+                "frac_of_8tbs": gbs / 8000.0, "bytes_per_launch": mbytes, "ms_per_launch": t}
 
-    # end to end through the public API: host (pinned) -> device, permute, ring,
-    # unpermute, device -> host, every step
+    merge = None
+    if w.dtype == "bf16" and rank == 0:
+        merge = merge_gbs(w.b, w.S, w.hq, w.d)
+        w5 = W.BY_NAME["noncausal_s64k_contig32"]
+        merge["noncausal_s64k_contig32"] = merge_gbs(w5.b, w5.S, w5.hq, w5.d)
+        torch.cuda.empty_cache()
+
+    # end to end through the public API, every step: pinned host -> device copy of
+    # q/k/v, permute to rank-major order, ring attention, unpermute, device -> host
+    # copy of o and lse.  Consecutive steps are pipelined on three streams (copy-in,
+    # compute, copy-out) with double-buffered device tensors, as a serving loop would
+    # run them; the time runs from the first copy-in to the last copy-out.
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
     oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     lh = torch.empty((w.b, w.hq, w.S), dtype=torch.float32).pin_memory()
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    buf_in = [[torch.empty_like(t, device=dev) for t in (q, k, v)] for _ in range(2)]
+    buf_out = [(torch.empty(q.shape, dtype=q.dtype, device=dev),
+                torch.empty((w.b, w.hq, w.S), dtype=torch.float32, device=dev)) for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        qg, kg, vg = (t.to(dev, non_blocking=True) for t in (qh, kh, vh))
-        qr, kr, vr = (cp.layout_permute(t, w.layout, w.N) for t in (qg, kg, vg))
-        og, lg = cp.ring_attn_fwd(qr, kr, vr, w.layout, w.N, w.causal, w.scale, mode=args.mode, workspace=ws)
-        og = cp.layout_permute(og, w.layout, w.N, inverse=True)
-        lg = cp.layout_permute(lg, w.layout, w.N, seq_axis=2, inverse=True)
-        oh.copy_(og, non_blocking=True)
-        lh.copy_(lg, non_blocking=True)
+    def e2e_step(i):
+        sl = i % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_cmp[sl])  # step i-2 finished reading these inputs
+            for src, dst in zip((qh, kh, vh), buf_in[sl]):
+                dst.copy_(src, non_blocking=True)
+            ev_in[sl].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[sl])
+            s_cmp.wait_event(ev_out[sl])  # step i-2's outputs have left the device
+            qr, kr, vr = (cp.layout_permute(t, w.layout, w.N) for t in buf_in[sl])
+            og, lg = cp.ring_attn_fwd(qr, kr, vr, w.layout, w.N, w.causal, w.scale, mode=args.mode, workspace=ws)
+            cp.layout_permute(og, w.layout, w.N, inverse=True, out=buf_out[sl][0])
+            cp.layout_permute(lg, w.layout, w.N, seq_axis=2, inverse=True, out=buf_out[sl][1])
+            ev_cmp[sl].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[sl])
+            oh.copy_(buf_out[sl][0], non_blocking=True)
+            lh.copy_(buf_out[sl][1], non_blocking=True)
+            ev_out[sl].record(s_out)
 
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     e_steps = max(3, min(args.steps, 10))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(e_steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(e_steps):
+        e2e_step(i)
+    s_in.wait_stream(s_out)
+    e1.record(s_in)
     torch.cuda.synchronize()
+    cp.stream_check()
     e_ms = reduce_max(e0.elapsed_time(e1), world, dev)
     e2e_value = world * flops * e_steps / (e_ms * 1e-3) / 1e12
     es = 2 if w.dtype == "bf16" else 4
@@ -352,7 +384,8 @@ def main():
                          "traffic": profiled_traffic() if w.name == W.BENCH_WORKLOAD else None},
             "merge": merge,
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e_ms / e_steps, "pipelined": "copy-in / compute / copy-out on 3 streams"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
         }
