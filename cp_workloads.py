@@ -8,6 +8,8 @@ Recipe: a CPU torch.Generator seeded with 1000 + workload index draws fp32
 standard normals for Q, then K, then V, each of shape [b, S, H, d]; bf16
 workloads cast them with round-to-nearest-even; the striped 32K workload then
 multiplies K by 4 (a power of two, so exact in bf16) to widen the lse range.
+The backward's output gradient dO comes from a second generator seeded with
+2000 + that seed, the same way.
 Head shapes follow the Llama-3 GQA table (8B: 32 query / 8 KV heads, 70B: 64 / 8).
 """
 from dataclasses import dataclass, field, asdict
@@ -89,3 +91,14 @@ def random_qkv(b, S, hq, hkv, d, dtype="bf16", seed=0, k_scale=1.0, q_zero=False
 
 def make_inputs(w: Workload):
     return random_qkv(w.b, w.S, w.hq, w.hkv, w.d, w.dtype, w.seed, w.k_scale)
+
+
+def random_do(b, S, hq, d, dtype="bf16", seed=0):
+    """Output gradient dO [b, S, hq, d] on the CPU in original token order: fp32
+    standard normals from a CPU generator seeded with 2000 + seed, cast like Q."""
+    g = torch.Generator().manual_seed(2000 + seed)
+    return torch.randn((b, S, hq, d), generator=g, dtype=torch.float32).to(torch_dtype(dtype))
+
+
+def make_do(w: Workload):
+    return random_do(w.b, w.S, w.hq, w.d, w.dtype, w.seed)

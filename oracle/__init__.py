@@ -6,7 +6,8 @@ imports nor links it, and it shares no code with the CUDA path.
 
 What it computes is the plain definition of softmax attention and of the
 log-sum-exp merge from "上下文并行与 Ring Attention" (hs-black.github.io),
-section 分块注意力: see oracle.c for the formulas and layout.py for the token
+section 分块注意力, and of its gradients (the same section's paragraph on the
+backward pass): see oracle.c for the formulas and layout.py for the token
 layouts (sections Ring Attention, Zig-zag, Striped, 重排 token 的代价).
 
 Inputs are numpy arrays; they are upcast to float64 before the C code sees
@@ -37,6 +38,7 @@ def _load():
             [ctypes.c_int64] * 5 + [ctypes.c_int, ctypes.c_double, _F64P, _F64P, ctypes.c_int]
         lib.oracle_lse_merge.restype = None
         lib.oracle_lse_merge.argtypes = [ctypes.c_int64, ctypes.c_int64] + [_F64P] * 6
+        _bwd_sigs(lib)
         _lib = lib
     return _lib
 
@@ -129,3 +131,123 @@ def ring_attention(q, k, v, layout_name, n_ranks, causal, scale, nthreads=None):
     """
     layout.tokens_per_rank(layout_name, n_ranks, q.shape[1])
     return attention(q, k, v, causal, scale, nthreads=nthreads)
+
+
+def _bwd_sigs(lib):
+    lib.oracle_attention_bwd.restype = ctypes.c_int
+    lib.oracle_attention_bwd.argtypes = [_F64P] * 4 + [_I64P] * 2 + [ctypes.c_int64] * 6 + \
+        [ctypes.c_int, ctypes.c_double] + [_F64P] * 7 + [ctypes.c_int]
+    lib.oracle_attention_bwd_sel.restype = ctypes.c_int
+    lib.oracle_attention_bwd_sel.argtypes = [_F64P] * 4 + [_I64P] * 2 + [ctypes.c_int64] * 6 + \
+        [ctypes.c_int, ctypes.c_double, _I64P, ctypes.c_int64, _F64P, _I64P, ctypes.c_int64, _F64P, _F64P,
+         ctypes.c_int]
+
+
+def _opt_pos(pos, n, what):
+    if pos is None:
+        return None
+    a = np.ascontiguousarray(pos, dtype=np.int64)
+    if a.shape != (n,):
+        raise ValueError(what + " shape")
+    return a
+
+
+def attention_bwd(q, k, v, do, causal, scale, pos_q=None, pos_k=None, lse=None, delta=None, nthreads=None):
+    """Gradients of softmax attention (section 分块注意力, backward paragraph).
+
+    q, do [b, sq, hq, d]; k, v [b, sk, hkv, d].  With lse = delta = None the
+    row statistics (lse, D = do . o) come from the definition over these keys;
+    otherwise lse, delta [b, hq, sq] are the rows' GLOBAL statistics and the
+    result is this key block's share of the gradients.  Returns
+    (dq, dk, dv, lse, delta) in float64.
+    """
+    lib = _load()
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    b, sq, hq, d = q.shape
+    bk, sk, hkv, dk_ = k.shape
+    if bk != b or dk_ != d or v.shape != k.shape or do.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if (lse is None) != (delta is None):
+        raise ValueError("give both lse and delta, or neither")
+    lse_in = None if lse is None else _f64(lse).reshape(b, hq, sq)
+    delta_in = None if delta is None else _f64(delta).reshape(b, hq, sq)
+    pq, pk = _opt_pos(pos_q, sq, "pos_q"), _opt_pos(pos_k, sk, "pos_k")
+    dq = np.empty_like(q)
+    dkk = np.empty_like(k)
+    dv = np.empty_like(v)
+    lse_out = np.empty((b, hq, sq), np.float64)
+    delta_out = np.empty((b, hq, sq), np.float64)
+    rc = lib.oracle_attention_bwd(_ptr(q, _F64P), _ptr(k, _F64P), _ptr(v, _F64P), _ptr(do, _F64P),
+                                  _ptr(pq, _I64P), _ptr(pk, _I64P), b, sq, sk, hq, hkv, d, int(bool(causal)),
+                                  float(scale), _ptr(lse_in, _F64P), _ptr(delta_in, _F64P), _ptr(dq, _F64P),
+                                  _ptr(dkk, _F64P), _ptr(dv, _F64P), _ptr(lse_out, _F64P),
+                                  _ptr(delta_out, _F64P), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_attention_bwd rejected its arguments")
+    return dq, dkk, dv, lse_out, delta_out
+
+
+def attention_bwd_sel(q, k, v, do, causal, scale, sel_q, sel_k, pos_q=None, pos_k=None, nthreads=None):
+    """Gradients at selected rows: sel_q [n, 3] = (batch, q head, query index) gives
+    dq [n, d]; sel_k [m, 3] = (batch, kv head, key index) gives dk, dv [m, d]."""
+    lib = _load()
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    b, sq, hq, d = q.shape
+    _, sk, hkv, _ = k.shape
+    sq_sel = np.ascontiguousarray(np.asarray(sel_q, dtype=np.int64).reshape(-1, 3))
+    sk_sel = np.ascontiguousarray(np.asarray(sel_k, dtype=np.int64).reshape(-1, 3))
+    pq, pk = _opt_pos(pos_q, sq, "pos_q"), _opt_pos(pos_k, sk, "pos_k")
+    dq = np.empty((sq_sel.shape[0], d), np.float64)
+    dkk = np.empty((sk_sel.shape[0], d), np.float64)
+    dv = np.empty((sk_sel.shape[0], d), np.float64)
+    rc = lib.oracle_attention_bwd_sel(_ptr(q, _F64P), _ptr(k, _F64P), _ptr(v, _F64P), _ptr(do, _F64P),
+                                      _ptr(pq, _I64P), _ptr(pk, _I64P), b, sq, sk, hq, hkv, d,
+                                      int(bool(causal)), float(scale), _ptr(sq_sel, _I64P), sq_sel.shape[0],
+                                      _ptr(dq, _F64P), _ptr(sk_sel, _I64P), sk_sel.shape[0], _ptr(dkk, _F64P),
+                                      _ptr(dv, _F64P), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_attention_bwd_sel rejected its arguments")
+    return dq, dkk, dv
+
+
+def ring_attention_bwd(q, k, v, do, layout_name, n_ranks, causal, scale, nthreads=None):
+    """Reference gradients of ring attention on original-order tensors.
+
+    The ring reaches the plain definition's gradients exactly (section 分块注意力,
+    backward paragraph: each block's share uses the global statistics), so this
+    is the definition over the whole sequence; layout and N only permute tokens.
+    Returns (dq, dk, dv) in ORIGINAL token order.
+    """
+    layout.tokens_per_rank(layout_name, n_ranks, q.shape[1])
+    dq, dk, dv, _, _ = attention_bwd(q, k, v, do, causal, scale, nthreads=nthreads)
+    return dq, dk, dv
+
+
+def ring_attention_bwd_steps(q, k, v, do, layout_name, n_ranks, causal, scale, nthreads=None):
+    """The ring's backward walked step by step, in the page's order.
+
+    The forward's global (lse, D) of every query row come first.  Then at step r
+    rank i holds the K/V block of rank (i - r) mod N together with that block's
+    travelling dK, dV accumulators (section Ring Attention); it adds the block's
+    share to its local dQ and to the travelling dK, dV.  After N steps every
+    accumulator holds the full sum.  Returns (dq, dk, dv) in ORIGINAL token order.
+    """
+    S = q.shape[1]
+    layout.tokens_per_rank(layout_name, n_ranks, S)
+    o, lse = attention(q, k, v, causal, scale, nthreads=nthreads)
+    delta = np.einsum("bshd,bshd->bhs", _f64(do), o)
+    pos = [np.asarray(layout.rank_positions(layout_name, n_ranks, S, i), dtype=np.int64) for i in range(n_ranks)]
+    dq = np.zeros(_f64(q).shape)
+    dk = np.zeros(_f64(k).shape)
+    dv = np.zeros(_f64(v).shape)
+    for r in range(n_ranks):
+        for i in range(n_ranks):
+            src = (i - r) % n_ranks
+            pi, pj = pos[i], pos[src]
+            gq, gk, gv, _, _ = attention_bwd(q[:, pi], k[:, pj], v[:, pj], do[:, pi], causal, scale,
+                                             pos_q=pi, pos_k=pj, lse=lse[:, :, pi], delta=delta[:, :, pi],
+                                             nthreads=nthreads)
+            dq[:, pi] += gq
+            dk[:, pj] += gk
+            dv[:, pj] += gv
+    return dq, dk, dv

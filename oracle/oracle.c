@@ -24,7 +24,8 @@
  * given set gets o = 0 and lse = -inf; merging two such partials gives (0, -inf).
  *
  * Everything is scalar fp64, sequential summation in key order, no blocking and
- * no reordering; threads only split independent query rows.
+ * no reordering; threads only split independent output rows.  The gradients of
+ * the same section's backward paragraph follow at the end of the file.
  */
 #include <math.h>
 #include <pthread.h>
@@ -205,4 +206,267 @@ void oracle_lse_merge(int64_t n, int64_t d, const double *o1, const double *lse1
         for (int64_t e = 0; e < d; ++e) o[r * d + e] = w1 * o1[r * d + e] + w2 * o2[r * d + e];
         lse[r] = L;
     }
+}
+
+/* ------------------------------------------------------------------ backward
+ *
+ * Same page, last paragraph of section 分块注意力 (the backward pass needs only
+ * the lse): with the GLOBAL lse of a query row, the softmax probability of a
+ * visible key is p_j = e^{x_j - lse}, whichever block the key sits in, so every
+ * key block yields its exact share of the gradients on its own:
+ *   dv_j += p_j do,    dx_j = p_j (do . v_j - D),    D = do . o (one scalar per
+ *   query row, also global),
+ * and through x_j = scale q . k_j (chain rule):
+ *   dq += scale dx_j k_j,    dk_j += scale dx_j q.
+ * The statistics (lse, D) of each query row are either computed here from the
+ * definition over the keys given (whole problem) or passed in (a block of keys
+ * against the global statistics: one ring step's contribution).
+ *
+ * Rows with no visible key (lse = -inf) contribute nothing.  Sums run
+ * sequentially: over keys in key order for dq, over (query head, query) in that
+ * order for dk and dv; threads split independent output rows only.
+ */
+
+typedef struct {
+    const double *q, *k, *v, *dout;
+    const int64_t *pos_q, *pos_k;
+    int64_t b, sq, sk, hq, hkv, d;
+    int causal;
+    double scale;
+    const double *lse_in, *delta_in; /* [b, hq, sq] or NULL (compute them) */
+    double *lse, *delta;             /* [b, hq, sq] statistics in use */
+    const unsigned char *head_mask;  /* [b * hq]: rows of unmarked heads skipped; NULL = all */
+    const int64_t *sel;              /* [n][3] selected rows, or NULL = every row */
+    double *dq;                      /* query pass: [b, sq, hq, d] or [n][d]; NULL = stats only */
+    double *dk, *dv;                 /* key pass: [b, sk, hkv, d] or [n][d] */
+    int64_t begin, end;
+} bwd_job_t;
+
+static double dotd(const double *a, const double *b, int64_t d)
+{
+    double s = 0.0;
+    for (int64_t e = 0; e < d; ++e) s += a[e] * b[e];
+    return s;
+}
+
+static const double *qrow_of(const bwd_job_t *j, const double *base, int64_t bb, int64_t i, int64_t h)
+{
+    return base + ((bb * j->sq + i) * j->hq + h) * j->d;
+}
+
+static const double *krow_of(const bwd_job_t *j, const double *base, int64_t bb, int64_t t, int64_t hk)
+{
+    return base + ((bb * j->sk + t) * j->hkv + hk) * j->d;
+}
+
+/* Query pass: statistics of the row, then (optionally) its dq. */
+static void *bwd_query_worker(void *arg)
+{
+    bwd_job_t *j = (bwd_job_t *)arg;
+    const int64_t d = j->d, g = j->hq / j->hkv;
+    double *x = (double *)malloc(sizeof(double) * (size_t)(j->sk > 0 ? j->sk : 1));
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+    for (int64_t r = j->begin; r < j->end; ++r) {
+        int64_t bb, h, i;
+        if (j->sel) {
+            bb = j->sel[3 * r + 0]; h = j->sel[3 * r + 1]; i = j->sel[3 * r + 2];
+        } else {
+            i = r % j->sq; h = (r / j->sq) % j->hq; bb = r / (j->sq * j->hq);
+        }
+        if (j->head_mask && !j->head_mask[bb * j->hq + h]) continue;
+        const int64_t hk = h / g;
+        const int64_t pq = j->pos_q ? j->pos_q[i] : i;
+        const double *qi = qrow_of(j, j->q, bb, i, h);
+        const double *doi = qrow_of(j, j->dout, bb, i, h);
+        const int64_t srow = (bb * j->hq + h) * j->sq + i;
+        double lse, D;
+        if (j->lse_in) {
+            lse = j->lse_in[srow];
+            D = j->delta_in[srow];
+        } else {
+            lse = attend_row(qi, pq, krow_of(j, j->k, bb, 0, hk), krow_of(j, j->v, bb, 0, hk), j->pos_k,
+                             j->sk, j->hkv * d, d, j->causal, j->scale, x, o);
+            D = dotd(doi, o, d);
+        }
+        if (j->lse) { j->lse[srow] = lse; j->delta[srow] = D; }
+        if (!j->dq) continue;
+        double *dqi = j->sel ? j->dq + r * d : j->dq + ((bb * j->sq + i) * j->hq + h) * d;
+        for (int64_t e = 0; e < d; ++e) dqi[e] = 0.0;
+        if (lse == -INFINITY) continue;
+        for (int64_t t = 0; t < j->sk; ++t) {
+            const int64_t pk = j->pos_k ? j->pos_k[t] : t;
+            if (j->causal && pk > pq) continue;
+            const double *kt = krow_of(j, j->k, bb, t, hk);
+            const double *vt = krow_of(j, j->v, bb, t, hk);
+            const double p = exp(j->scale * dotd(qi, kt, d) - lse);
+            const double dx = p * (dotd(doi, vt, d) - D);
+            for (int64_t e = 0; e < d; ++e) dqi[e] += j->scale * dx * kt[e];
+        }
+    }
+    free(o);
+    free(x);
+    return NULL;
+}
+
+/* Key pass: dk and dv of one key row, summed over the query heads of its group
+ * and over every query row that sees it. */
+static void *bwd_key_worker(void *arg)
+{
+    bwd_job_t *j = (bwd_job_t *)arg;
+    const int64_t d = j->d, g = j->hq / j->hkv;
+    for (int64_t r = j->begin; r < j->end; ++r) {
+        int64_t bb, hk, t;
+        if (j->sel) {
+            bb = j->sel[3 * r + 0]; hk = j->sel[3 * r + 1]; t = j->sel[3 * r + 2];
+        } else {
+            t = r % j->sk; hk = (r / j->sk) % j->hkv; bb = r / (j->sk * j->hkv);
+        }
+        double *dkt = j->sel ? j->dk + r * d : j->dk + ((bb * j->sk + t) * j->hkv + hk) * d;
+        double *dvt = j->sel ? j->dv + r * d : j->dv + ((bb * j->sk + t) * j->hkv + hk) * d;
+        for (int64_t e = 0; e < d; ++e) { dkt[e] = 0.0; dvt[e] = 0.0; }
+        const int64_t pk = j->pos_k ? j->pos_k[t] : t;
+        const double *kt = krow_of(j, j->k, bb, t, hk);
+        const double *vt = krow_of(j, j->v, bb, t, hk);
+        for (int64_t h = hk * g; h < (hk + 1) * g; ++h) {
+            for (int64_t i = 0; i < j->sq; ++i) {
+                const int64_t pq = j->pos_q ? j->pos_q[i] : i;
+                if (j->causal && pk > pq) continue;
+                const int64_t srow = (bb * j->hq + h) * j->sq + i;
+                const double lse = j->lse[srow], D = j->delta[srow];
+                if (lse == -INFINITY) continue;
+                const double *qi = qrow_of(j, j->q, bb, i, h);
+                const double *doi = qrow_of(j, j->dout, bb, i, h);
+                const double p = exp(j->scale * dotd(qi, kt, d) - lse);
+                const double dx = p * (dotd(doi, vt, d) - D);
+                for (int64_t e = 0; e < d; ++e) {
+                    dvt[e] += p * doi[e];
+                    dkt[e] += j->scale * dx * qi[e];
+                }
+            }
+        }
+    }
+    return NULL;
+}
+
+static int run_bwd_jobs(const bwd_job_t *proto, int64_t nrows, int nthreads, void *(*fn)(void *))
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 1024) nthreads = 1024;
+    if (nrows < nthreads) nthreads = nrows > 0 ? (int)nrows : 1;
+    pthread_t th[1024];
+    bwd_job_t *jobs = (bwd_job_t *)malloc(sizeof(bwd_job_t) * (size_t)nthreads);
+    if (!jobs) return -1;
+    int64_t per = (nrows + nthreads - 1) / nthreads;
+    int started = 0, rc = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t] = *proto;
+        jobs[t].begin = t * per < nrows ? t * per : nrows;
+        jobs[t].end = (t + 1) * per < nrows ? (t + 1) * per : nrows;
+        if (nthreads == 1) { fn(&jobs[t]); continue; }
+        if (pthread_create(&th[t], NULL, fn, &jobs[t]) != 0) { rc = -1; break; }
+        ++started;
+    }
+    for (int t = 0; t < started; ++t) pthread_join(th[t], NULL);
+    free(jobs);
+    return rc;
+}
+
+static int bwd_dims_ok(int64_t b, int64_t sq, int64_t sk, int64_t hq, int64_t hkv, int64_t d)
+{
+    return b >= 0 && sq >= 0 && sk >= 0 && hq > 0 && hkv > 0 && d > 0 && hq % hkv == 0;
+}
+
+/* Gradients of every input.
+ *   q, dout [b, sq, hq, d]; k, v [b, sk, hkv, d]; pos_q [sq] / pos_k [sk] (NULL = identity)
+ *   lse_in, delta_in [b, hq, sq]: the rows' global statistics, or both NULL to
+ *     compute them from the definition over these keys;
+ *   dq [b, sq, hq, d], dk, dv [b, sk, hkv, d] are overwritten;
+ *   lse_out, delta_out [b, hq, sq] (may be NULL) receive the statistics used.
+ * Returns 0, or -1 on bad sizes / allocation or thread failure. */
+int oracle_attention_bwd(const double *q, const double *k, const double *v, const double *dout,
+                         const int64_t *pos_q, const int64_t *pos_k, int64_t b, int64_t sq, int64_t sk,
+                         int64_t hq, int64_t hkv, int64_t d, int causal, double scale,
+                         const double *lse_in, const double *delta_in, double *dq, double *dk,
+                         double *dv, double *lse_out, double *delta_out, int nthreads)
+{
+    if (!bwd_dims_ok(b, sq, sk, hq, hkv, d) || (!lse_in) != (!delta_in)) return -1;
+    const int64_t nstat = b * hq * sq;
+    double *lse = lse_out, *delta = delta_out, *own = NULL;
+    if (!lse || !delta) {
+        own = (double *)malloc(sizeof(double) * (size_t)(2 * nstat + 1));
+        if (!own) return -1;
+        lse = own;
+        delta = own + nstat;
+    }
+    bwd_job_t j;
+    memset(&j, 0, sizeof j);
+    j.q = q; j.k = k; j.v = v; j.dout = dout; j.pos_q = pos_q; j.pos_k = pos_k;
+    j.b = b; j.sq = sq; j.sk = sk; j.hq = hq; j.hkv = hkv; j.d = d;
+    j.causal = causal; j.scale = scale; j.lse_in = lse_in; j.delta_in = delta_in;
+    j.lse = lse; j.delta = delta; j.dq = dq; j.dk = dk; j.dv = dv;
+    int rc = run_bwd_jobs(&j, nstat, nthreads, bwd_query_worker);
+    if (rc == 0) rc = run_bwd_jobs(&j, b * hkv * sk, nthreads, bwd_key_worker);
+    free(own);
+    return rc;
+}
+
+/* Gradients at selected rows only (for sampled checks at full size).
+ *   sel_q [nq][3] = (batch, q head, query index) -> dq_sel [nq][d]
+ *   sel_k [nk][3] = (batch, kv head, key index)  -> dk_sel, dv_sel [nk][d]
+ * The statistics are computed from the definition: per selected query row, and
+ * for every query row of the heads that a selected key row serves. */
+int oracle_attention_bwd_sel(const double *q, const double *k, const double *v, const double *dout,
+                             const int64_t *pos_q, const int64_t *pos_k, int64_t b, int64_t sq,
+                             int64_t sk, int64_t hq, int64_t hkv, int64_t d, int causal, double scale,
+                             const int64_t *sel_q, int64_t nq, double *dq_sel, const int64_t *sel_k,
+                             int64_t nk, double *dk_sel, double *dv_sel, int nthreads)
+{
+    if (!bwd_dims_ok(b, sq, sk, hq, hkv, d) || nq < 0 || nk < 0) return -1;
+    const int64_t g = hq / hkv;
+    for (int64_t r = 0; r < nq; ++r)
+        if (sel_q[3 * r] < 0 || sel_q[3 * r] >= b || sel_q[3 * r + 1] < 0 || sel_q[3 * r + 1] >= hq ||
+            sel_q[3 * r + 2] < 0 || sel_q[3 * r + 2] >= sq)
+            return -1;
+    for (int64_t r = 0; r < nk; ++r)
+        if (sel_k[3 * r] < 0 || sel_k[3 * r] >= b || sel_k[3 * r + 1] < 0 || sel_k[3 * r + 1] >= hkv ||
+            sel_k[3 * r + 2] < 0 || sel_k[3 * r + 2] >= sk)
+            return -1;
+    bwd_job_t j;
+    memset(&j, 0, sizeof j);
+    j.q = q; j.k = k; j.v = v; j.dout = dout; j.pos_q = pos_q; j.pos_k = pos_k;
+    j.b = b; j.sq = sq; j.sk = sk; j.hq = hq; j.hkv = hkv; j.d = d;
+    j.causal = causal; j.scale = scale;
+    int rc = 0;
+    if (nq > 0) {
+        bwd_job_t jq = j;
+        jq.sel = sel_q;
+        jq.dq = dq_sel;
+        rc = run_bwd_jobs(&jq, nq, nthreads, bwd_query_worker);
+    }
+    if (rc == 0 && nk > 0) {
+        const int64_t nstat = b * hq * sq;
+        double *stats = (double *)malloc(sizeof(double) * (size_t)(2 * nstat + 1));
+        unsigned char *mask = (unsigned char *)calloc((size_t)(b * hq + 1), 1);
+        if (!stats || !mask) { free(stats); free(mask); return -1; }
+        for (int64_t r = 0; r < nk; ++r)
+            for (int64_t h = sel_k[3 * r + 1] * g; h < (sel_k[3 * r + 1] + 1) * g; ++h)
+                mask[sel_k[3 * r] * hq + h] = 1;
+        bwd_job_t js = j;
+        js.lse = stats;
+        js.delta = stats + nstat;
+        js.head_mask = mask;
+        rc = run_bwd_jobs(&js, nstat, nthreads, bwd_query_worker);
+        if (rc == 0) {
+            bwd_job_t jk = j;
+            jk.lse = stats;
+            jk.delta = stats + nstat;
+            jk.sel = sel_k;
+            jk.dk = dk_sel;
+            jk.dv = dv_sel;
+            rc = run_bwd_jobs(&jk, nk, nthreads, bwd_key_worker);
+        }
+        free(mask);
+        free(stats);
+    }
+    return rc;
 }
