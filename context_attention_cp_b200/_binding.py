@@ -37,6 +37,8 @@ _SIGNATURES = {
     "cp_lse_merge": (_i32, [_T, _T, _T, _T, _T, _vp]),
     "cp_ring_attn_fwd": (_i32, [_i32, _i32, _i32, _T, _T, _T, _f32, _T, _T, _i32, _vp, _sz, _vp]),
     "cp_ring_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _i64]),
+    "cp_ring_attn_bwd": (_i32, [_i32, _i32, _i32, _T, _T, _T, _T, _T, _T, _f32, _T, _T, _T, _vp, _sz, _vp]),
+    "cp_ring_bwd_workspace_bytes": (_sz, [_i32, _i32, _i32, _i64, _i64, _i64, _i64]),
     "cp_layout_permute": (_i32, [_i32, _i32, _i32, _T, _T, _i32, _vp]),
     "cp_layout_range": (_i32, [_i32, _i32, _i64, _i32, _R]),
     "cp_tile_classes": (_i32, [_R, _i64, _R, _i64, _i32, _i32, _i32, ctypes.POINTER(ctypes.c_int8)]),
@@ -178,6 +180,30 @@ def ring_attn_fwd(q, k, v, layout, N, causal, scale=None, o=None, lse=None, mode
     _check(lib().cp_ring_attn_fwd(LAYOUTS[layout], N, int(bool(causal)), _ref(tq), _ref(tk), _ref(tv),
                                   float(scale), _ref(to), _ref(tl), MODES[mode], ws_ptr, need, _stream()))
     return o, lse
+
+
+def ring_bwd_workspace_bytes(layout, N, dtype_code, b, S, Hq, d):
+    return lib().cp_ring_bwd_workspace_bytes(LAYOUTS[layout], N, dtype_code, b, S, Hq, d)
+
+
+def ring_attn_bwd(q, k, v, o, lse, do, layout, N, causal, scale=None, dq=None, dk=None, dv=None, workspace=None):
+    """Gradients (dq, dk, dv) of ring attention; every tensor in rank-major order,
+    o and lse the forward's results for the same arguments."""
+    import torch
+    b, S, Hq, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = ring_bwd_workspace_bytes(layout, N, _dtype_code(q), b, S, Hq, d)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ts = [_tensor(t) for t in (q, k, v, o, lse, do, dq, dk, dv)]
+    _check(lib().cp_ring_attn_bwd(LAYOUTS[layout], N, int(bool(causal)), *[_ref(t) for t in ts[:6]], float(scale),
+                                  *[_ref(t) for t in ts[6:]], ctypes.c_void_p(workspace.data_ptr()), need,
+                                  _stream()))
+    return dq, dk, dv
 
 
 def ring_attn_fwd_static_scratch(q, k, v, layout, N, causal, scale, o, lse):

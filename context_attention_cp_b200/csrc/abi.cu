@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "../../include/cpattn.h"
+#include "bwd.h"
 #include "kernels.h"
 
 using namespace cpattn;
@@ -179,6 +180,60 @@ const std::vector<uint32_t> &ring_order(int layout, int N, int64_t S, int causal
 }
 
 int rows_per_cta(int32_t dtype) { return dtype == CP_BF16 ? attn_tc_rows_per_cta() : 128; }
+
+// Work order of the backward: (key rank, key tile) entries sorted by the number of
+// query tiles that see the key tile over all steps, heaviest first.
+std::map<std::tuple<int, int, int, int64_t>, std::vector<uint32_t>> g_bwd_order_cache;
+
+const std::vector<uint32_t> &bwd_order(int layout, int N, int64_t S, int causal)
+{
+    std::lock_guard<std::mutex> lk(g_order_mu);
+    const auto key = std::make_tuple(layout, N, causal, S);
+    auto it = g_bwd_order_cache.find(key);
+    if (it != g_bwd_order_cache.end()) return it->second;
+    const int64_t c = S / N;
+    const int n_kt = (int)((c + kBwdKeyTile - 1) / kBwdKeyTile);
+    const int n_qt = (int)((c + kBwdQueryTile - 1) / kBwdQueryTile);
+    std::vector<std::pair<int64_t, uint32_t>> work;
+    work.reserve((size_t)N * n_kt);
+    for (int jr = 0; jr < N; ++jr) {
+        Range kr = layout_range(layout, N, S, jr);
+        for (int kt = 0; kt < n_kt; ++kt) {
+            int64_t tiles = 0;
+            for (int r = 0; r < N; ++r) {
+                Range qr = layout_range(layout, N, S, (jr + r) % N);
+                int qb, qf;
+                q_tile_bounds<int64_t>(qr, c, kBwdQueryTile, kr, c, (int64_t)kt * kBwdKeyTile, kBwdKeyTile,
+                                       causal != 0, &qb, &qf);
+                tiles += n_qt - qb;
+            }
+            work.push_back({tiles, ((uint32_t)jr << 16) | (uint32_t)kt});
+        }
+    }
+    std::stable_sort(work.begin(), work.end(),
+                     [](const std::pair<int64_t, uint32_t> &a, const std::pair<int64_t, uint32_t> &b) {
+                         return a.first > b.first;
+                     });
+    std::vector<uint32_t> out;
+    for (auto &w : work) out.push_back(w.second);
+    return g_bwd_order_cache.emplace(key, std::move(out)).first->second;
+}
+
+// Workspace regions of the backward: statistics [b][Hq][N][lpad] float2, then the
+// fp32 dQ accumulator [b, S, Hq, d]; each 256-byte aligned.
+struct BwdWorkspace {
+    int64_t lpad, stats_bytes, acc_bytes;
+};
+BwdWorkspace bwd_workspace(int32_t N, int64_t b, int64_t S, int64_t Hq, int64_t d)
+{
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    BwdWorkspace w;
+    const int64_t c = S / N;
+    w.lpad = (c + kBwdQueryTile - 1) / kBwdQueryTile * kBwdQueryTile;
+    w.stats_bytes = up(b * Hq * N * w.lpad * 8);
+    w.acc_bytes = up(b * S * Hq * d * 4);
+    return w;
+}
 
 cp_status check_attn_dtypes(const cp_tensor *q, const cp_tensor *k, const cp_tensor *v)
 {
@@ -474,6 +529,111 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
         if (r > 0 && (s = cp_lse_merge(&o_acc, lse, &o_b, &lse_b, r == N - 1 ? o : nullptr, stream)) != CP_OK)
             return s;
     }
+    return CP_OK;
+}
+
+size_t cp_ring_bwd_workspace_bytes(int32_t layout, int32_t N, int32_t dtype, int64_t b, int64_t S, int64_t Hq,
+                                   int64_t d)
+{
+    if (layout < 0 || layout > 2 || N < 1 || b < 0 || S < 0 || Hq < 0 || d < 0 || !elem_size(dtype)) return 0;
+    if (S % N) return 0;
+    const BwdWorkspace w = bwd_workspace(N, b, S, Hq, d);
+    return (size_t)(w.stats_bytes + w.acc_bytes);
+}
+
+cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q, const cp_tensor *k,
+                           const cp_tensor *v, const cp_tensor *o, const cp_tensor *lse, const cp_tensor *dout,
+                           float softmax_scale, cp_tensor *dq, cp_tensor *dk, cp_tensor *dv, void *workspace,
+                           size_t workspace_bytes, void *stream)
+{
+    g_last_error[0] = 0;
+    cp_status s;
+    if (layout < 0 || layout > 2) return fail(CP_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (causal != 0 && causal != 1) return fail(CP_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if ((s = check_tensor(q, "q")) != CP_OK || (s = check_tensor(k, "k")) != CP_OK ||
+        (s = check_tensor(v, "v")) != CP_OK || (s = check_tensor(dout, "dout")) != CP_OK ||
+        (s = check_tensor(dq, "dq")) != CP_OK || (s = check_tensor(dk, "dk")) != CP_OK ||
+        (s = check_tensor(dv, "dv")) != CP_OK)
+        return s;
+    if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
+    if (q->dtype != CP_BF16) return fail(CP_ERR_UNSUPPORTED, "the backward takes bf16 tensors");
+    if (q->shape[3] != 128) return fail(CP_ERR_UNSUPPORTED, "the backward supports d = 128");
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    const int64_t S = q->shape[1];
+    if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
+    if (N < 1 || N > 4096) return fail(CP_ERR_INVALID_ARG, "N must be in [1, 4096]");
+    if (S >= ((int64_t)1 << 30)) return fail(CP_ERR_SHAPE, "sequence too long (S must be below 2^30)");
+    if (S % N) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of N = %d", (long long)S, N);
+    if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N)) return fail(CP_ERR_SHAPE, "zig-zag needs S to be a multiple of 2N");
+    if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;
+    if (o->dtype != CP_BF16) return fail(CP_ERR_INVALID_ARG, "o must be bf16");
+    const cp_tensor *like_q[2] = {dout, dq};
+    for (const cp_tensor *t : like_q) {
+        if (!same_shape(t, q) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "dout and dq must be bf16 shaped like q");
+        if ((s = check_rows16(t, t == dq ? "dq" : "dout")) != CP_OK) return s;
+    }
+    const cp_tensor *like_k[2] = {dk, dv};
+    for (const cp_tensor *t : like_k) {
+        if (!same_shape(t, k) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "dk and dv must be bf16 shaped like k");
+        if ((s = check_rows16(t, t == dk ? "dk" : "dv")) != CP_OK) return s;
+    }
+    const int64_t c = S / N;
+    const int64_t b = q->shape[0], Hq = q->shape[2], d = q->shape[3];
+    const int64_t n_kt = (c + kBwdKeyTile - 1) / kBwdKeyTile;
+    if (n_kt > 65535) return fail(CP_ERR_SHAPE, "too many key tiles per rank");
+    const size_t need = cp_ring_bwd_workspace_bytes(layout, N, q->dtype, b, S, Hq, d);
+    if (!workspace || workspace_bytes < need) return fail(CP_ERR_INVALID_ARG, "workspace of %zu bytes needed", need);
+    if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (b == 0 || S == 0) return CP_OK;
+
+    thread_local BwdParams p;
+    std::memset(&p, 0, sizeof p);
+    p.b = (int)b;
+    p.hq = (int)Hq;
+    p.hkv = (int)k->shape[2];
+    p.group = p.hq / p.hkv;
+    p.d = (int)d;
+    p.q_len = (int)c;
+    p.kv_len = (int)c;
+    p.n_ranks = N;
+    p.step_begin = 0;
+    p.step_end = N;
+    p.causal = causal;
+    p.use_layout = 1;
+    p.layout = layout;
+    p.seq_len = S;
+    p.q_row_step = c;
+    p.kv_row_step = c;
+    p.scale = softmax_scale;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.q = q->data; p.k = k->data; p.v = v->data; p.o = o->data; p.dout = dout->data;
+    p.q_sb = q->stride[0]; p.q_ss = q->stride[1]; p.q_sh = q->stride[2];
+    p.k_sb = k->stride[0]; p.k_ss = k->stride[1]; p.k_sh = k->stride[2];
+    p.v_sb = v->stride[0]; p.v_ss = v->stride[1]; p.v_sh = v->stride[2];
+    p.o_sb = o->stride[0]; p.o_ss = o->stride[1]; p.o_sh = o->stride[2];
+    p.do_sb = dout->stride[0]; p.do_ss = dout->stride[1]; p.do_sh = dout->stride[2];
+    p.lse = static_cast<const float *>(lse->data);
+    p.lse_sb = lse->stride[0]; p.lse_sh = lse->stride[1]; p.lse_ss = lse->stride[2];
+    const BwdWorkspace w = bwd_workspace(N, b, S, Hq, d);
+    p.stats = static_cast<float2 *>(workspace);
+    p.lpad = (int)w.lpad;
+    p.dq_acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.stats_bytes);
+    p.dq = dq->data; p.dk = dk->data; p.dv = dv->data;
+    p.dq_sb = dq->stride[0]; p.dq_ss = dq->stride[1]; p.dq_sh = dq->stride[2];
+    p.dk_sb = dk->stride[0]; p.dk_ss = dk->stride[1]; p.dk_sh = dk->stride[2];
+    p.dv_sb = dv->stride[0]; p.dv_ss = dv->stride[1]; p.dv_sh = dv->stride[2];
+    int *word = nullptr;
+    status_word(&word);
+    p.status = word;
+    p.n_kt = (int)n_kt;
+    const std::vector<uint32_t> &ord = bwd_order(layout, N, S, causal);
+    if ((int64_t)ord.size() <= kMaxOrder) {
+        p.order_len = (int)ord.size();
+        std::copy(ord.begin(), ord.end(), p.order);
+    }
+    cudaError_t e = launch_attn_bwd(p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return CP_OK;
 }
 

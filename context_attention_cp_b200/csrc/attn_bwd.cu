@@ -1,0 +1,699 @@
+// attn_bwd.cu -- bf16 attention backward on sm_100a tensor cores (tcgen05 + TMEM +
+// TMA), the whole ring's backward in one launch.
+//
+// What it computes ("上下文并行与 Ring Attention", hs-black.github.io, section
+// 分块注意力, paragraph on the backward pass; section Ring Attention for the
+// schedule): with the forward's GLOBAL lse and D = do . o of every query row,
+//   p = e^{x - lse},  dv_j += p do,  dx = p (do . v_j - D),
+//   dq += scale dx k_j,  dk_j += scale dx q.
+// In the ring, K/V block j visits rank (j + r) mod N at step r; dK_j, dV_j travel
+// with it and dQ stays home.  On one device the travelling accumulators become
+// TMEM-resident: one CTA keeps a 128-key tile of block j (K, V in shared memory,
+// dK, dV in TMEM) and walks every (query head of its group, ring step, 64-row
+// query tile) that sees the tile.  dQ shares leave through bulk-tensor reductions
+// (fp32 add) into an accumulator in HBM.
+//
+// Per query tile, in the transposed form that puts keys on TMEM lanes:
+//   S^T  = K Q^T        (M 128 keys, N 64 queries, K = d)   -> TMEM
+//   dP^T = V dO^T       (same shapes)                        -> TMEM
+//   P^T  = exp2(S^T scale log2e - lse log2e), dS^T = P^T (dP^T - D)  (softmax warps,
+//          bf16 to shared memory, 128-byte swizzled, K-major)
+//   dV  += P^T dO       (M 128 keys, N = d, K 64 queries)    TMEM accumulator
+//   dK  += dS^T Q       (same)                               TMEM accumulator
+//   dQ^T = K^T dS^T     (M = d, N 64 queries, K 128 keys)    -> TMEM -> fp32 staging
+//                                                              -> bulk reduce-add
+// Roles (448 threads):
+//   warps 0-3  / 4-7  P and dS of query columns [0, 32) / [32, 64), one key row per
+//                     thread; afterwards the dK (warps 0-3) and dV (4-7) epilogue
+//   warps 8-11 dQ^T out of TMEM, scaled, staged, reduced into the accumulator
+//   warp 12    TMA producer (K, V once; Q, dO and row statistics per query tile)
+//   warp 13    TMEM owner and single-thread MMA issuer
+// TMEM columns: S^T double buffer [0, 128), dP^T [128, 192), dQ^T [192, 256),
+// dV [256, 384), dK [384, 512).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "bwd.h"
+#include "ptx.cuh"
+
+namespace cpattn {
+namespace {
+
+constexpr int BK = kBwdKeyTile;    // keys per CTA
+constexpr int BQ = kBwdQueryTile;  // queries per step
+constexpr int HD = 128;            // head dim
+constexpr int NS = 2;              // Q / dO stages
+constexpr int NTHREADS = 448;
+constexpr int WARP_DQ0 = 8;
+constexpr int WARP_LOAD = 12;
+constexpr int WARP_MMA = 13;
+constexpr float kLog2eB = 1.44269504088896340736f;
+
+struct BCfg {
+    static constexpr int KV_SUB = BK * 128;  // 128 rows x 64 bf16 (one swizzle column block)
+    static constexpr int Q_SUB = BQ * 128;   // 64 rows x 64 bf16
+    static constexpr int KV_TILE = 2 * KV_SUB;
+    static constexpr int Q_TILE = 2 * Q_SUB;
+    static constexpr int STAGE = 2 * Q_TILE;  // Q then dO
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + KV_TILE;
+    static constexpr int OFF_Q = OFF_V + KV_TILE;
+    static constexpr int OFF_P = OFF_Q + NS * STAGE;  // P^T  [128 keys][64 queries] bf16
+    static constexpr int OFF_DS = OFF_P + BK * 128;   // dS^T [128 keys][64 queries] bf16
+    static constexpr int OFF_DQ = OFF_DS + BK * 128;  // dQ staging [64 queries][128] fp32
+    static constexpr int OFF_ST = OFF_DQ + BQ * HD * 4;  // per stage: 64 x (lse log2e, D)
+    static constexpr int OFF_BAR = OFF_ST + NS * BQ * 8;
+    enum {
+        B_KV = 0,
+        B_QF = 1,
+        B_QE = B_QF + NS,
+        B_SF = B_QE + NS,
+        B_SE = B_SF + 2,
+        B_DPF = B_SE + 2,
+        B_PR,
+        B_PE,
+        B_DSR,
+        B_DSE,
+        B_DQF,
+        B_DQE,
+        B_DONE,
+        NBAR
+    };
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 64 + 1024;
+    static_assert(SMEM <= 232448, "shared memory per CTA exceeds 227 KB");
+    static constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 192, T_DV = 256, T_DK = 384, TMEM_COLS = 512;
+};
+
+// kind::f16 instruction descriptor with both operand majors selectable:
+// bit 15 A MN-major, bit 16 B MN-major (other fields as idesc_bf16_f32).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+constexpr uint32_t IDESC_S = idesc_bf16(BK, BQ, false, false);   // K Q^T, V dO^T
+constexpr uint32_t IDESC_KV = idesc_bf16(BK, HD, false, true);   // P^T dO, dS^T Q
+constexpr uint32_t IDESC_DQ = idesc_bf16(HD, BQ, true, true);    // K^T dS^T
+
+// ---- bulk copies and reductions (no multicast)
+
+// Contiguous global -> shared copy, completion counted on `bar` (bytes).
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Element-wise fp32 add of a shared-memory box into the global tensor of `map`.
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2, int c3)
+{
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Makes this thread's generic-proxy shared-memory writes visible to the async proxy
+// (tensor cores, bulk copies).
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// OR of `pred` over the `nthreads` threads of named barrier `id` (all must call).
+__device__ __forceinline__ bool bar_any(uint32_t id, uint32_t nthreads, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
+// Query-tile sequence of one CTA: (query head of the group, ring step, query tile)
+// with the tile seeing at least one key of the CTA's key tile.  Every role walks it.
+struct QSeq {
+    const BwdParams *p;
+    int j, k_lo, h0, n_qt;
+    Range kr;
+    int hi, r, qt, qt_full, i, h;
+    Range qr;
+
+    __device__ void init(const BwdParams &pp, int jj, int klo, const Range &k, int hq0)
+    {
+        p = &pp;
+        j = jj;
+        k_lo = klo;
+        kr = k;
+        h0 = hq0;
+        n_qt = (pp.q_len + BQ - 1) / BQ;
+        hi = 0;
+        r = pp.step_begin - 1;
+        qt = n_qt - 1;
+        qt_full = 0;
+        i = 0;
+        h = hq0;
+    }
+    __device__ bool next()
+    {
+        ++qt;
+        while (qt >= n_qt) {
+            ++r;
+            if (r >= p->step_end) {
+                r = p->step_begin;
+                if (++hi >= p->group) return false;
+            }
+            const int N = p->n_ranks;
+            i = (j + r) % N;
+            qr = p->use_layout ? layout_range(p->layout, N, p->seq_len, i) : p->q_range;
+            int qb;
+            q_tile_bounds<int64_t>(qr, p->q_len, BQ, kr, p->kv_len, k_lo, BK, p->causal != 0, &qb, &qt_full);
+            qt = qb;
+        }
+        h = h0 + hi;
+        return true;
+    }
+    __device__ bool partial() const { return qt < qt_full; }
+    __device__ int q_row() const { return (int)(i * p->q_row_step) + qt * BQ; }
+};
+
+// 32 consecutive bf16 of one row (64 bytes) from fp32 values.
+__device__ __forceinline__ void store_bf16x32(void *dst, const float *v)
+{
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+        w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+        w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+        w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+        d4[i] = w;
+    }
+}
+
+// 32 bf16 (packed in 16 words) into row `row` of a [128 rows x 64] bf16 K-major
+// tile with 128-byte swizzle, columns [32 half, 32 half + 32).
+__device__ __forceinline__ void st_sw128_half(uint8_t *tile, int row, int half, const uint32_t *w)
+{
+    uint8_t *rowp = tile + row * 128;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int ch = (half * 4 + t) ^ (row & 7);
+        *reinterpret_cast<uint4 *>(rowp + ch * 16) = make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
+    }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    attn_bwd_kernel(const __grid_constant__ BwdParams p, const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_dq)
+{
+    using C = BCfg;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t bar0 = s_base + C::OFF_BAR;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    // ---- work item: (key rank, key tile) from the order table, then (batch, kv head)
+    const int bkh = p.b * p.hkv;
+    const int e = blockIdx.x / bkh;
+    const int bh = blockIdx.x % bkh;
+    int j, kt;
+    if (p.order_len) {
+        j = (int)(p.order[e] >> 16);
+        kt = (int)(p.order[e] & 0xffffu);
+    } else {
+        j = e / p.n_kt;
+        kt = e % p.n_kt;
+    }
+    const int hk = bh % p.hkv;
+    const int bb = bh / p.hkv;
+    const int k_lo = kt * BK;
+    const Range kr = p.use_layout ? layout_range(p.layout, p.n_ranks, p.seq_len, j) : p.kv_range;
+
+    if (tid == 0) {
+        mbar_init(bar(C::B_KV), 1);
+        for (int s = 0; s < NS; ++s) { mbar_init(bar(C::B_QF + s), 1); mbar_init(bar(C::B_QE + s), 1); }
+        for (int b2 = 0; b2 < 2; ++b2) { mbar_init(bar(C::B_SF + b2), 1); mbar_init(bar(C::B_SE + b2), 8); }
+        mbar_init(bar(C::B_DPF), 1);
+        mbar_init(bar(C::B_PR), 8);
+        mbar_init(bar(C::B_PE), 1);
+        mbar_init(bar(C::B_DSR), 8);
+        mbar_init(bar(C::B_DSE), 1);
+        mbar_init(bar(C::B_DQF), 1);
+        mbar_init(bar(C::B_DQE), 4);
+        mbar_init(bar(C::B_DONE), 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+
+    QSeq seq;
+    seq.init(p, j, k_lo, kr, hk * p.group);
+
+    if (warp == WARP_LOAD) {
+        // ================================================================ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_do);
+            WaitCtx w{abort_flag, p.status, 41};
+            const int kv_row = (int)(j * p.kv_row_step) + k_lo;
+            mbar_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
+            for (int kb = 0; kb < 2; ++kb) {
+                tma_load_4d(s_base + C::OFF_K + kb * C::KV_SUB, &tm_k, bar(C::B_KV), kb * 64, hk, kv_row, bb);
+                tma_load_4d(s_base + C::OFF_V + kb * C::KV_SUB, &tm_v, bar(C::B_KV), kb * 64, hk, kv_row, bb);
+            }
+            int n = 0;
+            while (seq.next()) {
+                const int s = n % NS;
+                if (!mbar_wait(bar(C::B_QE + s), ((n / NS) & 1) ^ 1, w)) break;
+                mbar_expect_tx(bar(C::B_QF + s), C::STAGE + BQ * 8);
+                const int q_row = seq.q_row();
+                const uint32_t st = s_base + C::OFF_Q + s * C::STAGE;
+                for (int kb = 0; kb < 2; ++kb) {
+                    tma_load_4d(st + kb * C::Q_SUB, &tm_q, bar(C::B_QF + s), kb * 64, seq.h, q_row, bb);
+                    tma_load_4d(st + C::Q_TILE + kb * C::Q_SUB, &tm_do, bar(C::B_QF + s), kb * 64, seq.h, q_row, bb);
+                }
+                const float2 *src =
+                    p.stats + (((int64_t)bb * p.hq + seq.h) * p.n_ranks + seq.i) * p.lpad + (int64_t)seq.qt * BQ;
+                bulk_g2s(s_base + C::OFF_ST + s * BQ * 8, src, BQ * 8, bar(C::B_QF + s));
+                ++n;
+            }
+            if (*abort_flag) {
+                // let the copies already issued land before the CTA leaves
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(bar(C::B_KV), 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
+                for (int i = (n > NS ? n - NS : 0); i < n; ++i) {
+                    const uint64_t t1 = global_timer_ns();
+                    while (!mbar_try_wait(bar(C::B_QF + i % NS), (i / NS) & 1) && global_timer_ns() - t1 < kWaitLimitNs) {}
+                }
+            }
+        }
+    } else if (warp == WARP_MMA) {
+        // ================================================================ MMA issuer
+        if (lane == 0) {
+            WaitCtx w{abort_flag, p.status, 43};
+            const uint32_t ka = s_base + C::OFF_K, va = s_base + C::OFF_V;
+            // S^T(n) = K Q(n)^T into S buffer n & 1
+            auto issue_s = [&](int n) {
+                const uint32_t qa = s_base + C::OFF_Q + (n % NS) * C::STAGE;
+                const uint32_t d_t = tbase + C::T_S + (uint32_t)((n & 1) * BQ);
+#pragma unroll
+                for (int k = 0; k < HD / 16; ++k)
+                    mma_ss(d_t, smem_desc_sw128(ka + (k >> 2) * C::KV_SUB + (k & 3) * 32, 16, 1024),
+                           smem_desc_sw128(qa + (k >> 2) * C::Q_SUB + (k & 3) * 32, 16, 1024), IDESC_S, k > 0 ? 1u : 0u);
+                tc_commit(bar(C::B_SF + (n & 1)));
+            };
+            // dP^T(n) = V dO(n)^T
+            auto issue_dp = [&](int n) {
+                const uint32_t da = s_base + C::OFF_Q + (n % NS) * C::STAGE + C::Q_TILE;
+#pragma unroll
+                for (int k = 0; k < HD / 16; ++k)
+                    mma_ss(tbase + C::T_DP, smem_desc_sw128(va + (k >> 2) * C::KV_SUB + (k & 3) * 32, 16, 1024),
+                           smem_desc_sw128(da + (k >> 2) * C::Q_SUB + (k & 3) * 32, 16, 1024), IDESC_S, k > 0 ? 1u : 0u);
+                tc_commit(bar(C::B_DPF));
+            };
+            bool have = seq.next();
+            bool ok = mbar_wait(bar(C::B_KV), 0, w);
+            if (have && ok) {
+                ok = mbar_wait(bar(C::B_QF + 0), 0, w);
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(0);
+                    issue_dp(0);
+                }
+            }
+            int n = 0;
+            while (have && ok) {
+                const int s = n % NS;
+                const bool have_next = seq.next();
+                if (have_next) {
+                    const int m = n + 1;
+                    if (!mbar_wait(bar(C::B_QF + m % NS), (m / NS) & 1, w)) break;
+                    if (m >= 2 && !mbar_wait(bar(C::B_SE + (m & 1)), ((m >> 1) - 1) & 1, w)) break;
+                    tc_fence_after();
+                    issue_s(m);
+                }
+                const uint32_t qa = s_base + C::OFF_Q + s * C::STAGE;
+                // dV += P^T dO
+                if (!mbar_wait(bar(C::B_PR), n & 1, w)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < BQ / 16; ++k)
+                    mma_ss(tbase + C::T_DV, smem_desc_sw128(s_base + C::OFF_P + k * 32, 16, 1024),
+                           smem_desc_sw128(qa + C::Q_TILE + k * 2048, C::Q_SUB, 1024), IDESC_KV,
+                           (n > 0 || k > 0) ? 1u : 0u);
+                tc_commit(bar(C::B_PE));
+                // dS^T ready: next dP first (the softmax waits on it), then dK and dQ^T
+                if (!mbar_wait(bar(C::B_DSR), n & 1, w)) break;
+                tc_fence_after();
+                if (have_next) issue_dp(n + 1);
+#pragma unroll
+                for (int k = 0; k < BQ / 16; ++k)
+                    mma_ss(tbase + C::T_DK, smem_desc_sw128(s_base + C::OFF_DS + k * 32, 16, 1024),
+                           smem_desc_sw128(qa + k * 2048, C::Q_SUB, 1024), IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+                if (n > 0 && !mbar_wait(bar(C::B_DQE), (n - 1) & 1, w)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)
+                    mma_ss(tbase + C::T_DQ, smem_desc_sw128(ka + k * 2048, C::KV_SUB, 1024),
+                           smem_desc_sw128(s_base + C::OFF_DS + k * 2048, C::KV_SUB, 1024), IDESC_DQ, k > 0 ? 1u : 0u);
+                tc_commit(bar(C::B_DQF));
+                tc_commit(bar(C::B_DSE));
+                tc_commit(bar(C::B_QE + s));
+                ++n;
+                have = have_next;
+            }
+            // drain: every MMA issued above has finished before the epilogue and teardown
+            tc_commit(bar(C::B_DONE));
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bar(C::B_DONE), 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
+        }
+    } else if (warp >= WARP_DQ0) {
+        // ================================================================ dQ warps 8-11
+        const int wq = warp - WARP_DQ0;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const bool leader = (wq == 0 && lane == 0);
+        WaitCtx w{abort_flag, p.status, 45};
+        float *stg = reinterpret_cast<float *>(smem + C::OFF_DQ);
+        const int dcol = wq * 32 + lane;
+        const float scale = p.scale;
+        int n = 0;
+        while (seq.next()) {
+            const bool okw = mbar_wait(bar(C::B_DQF), n & 1, w);
+            if (leader) bulk_wait_read_all();  // the staging buffer is free again
+            if (bar_any(2, 128, !okw)) break;
+            tc_fence_after();
+            uint32_t r0[32], r1[32];
+            tmem_ld32(tbase + lane_off + C::T_DQ, r0);
+            tmem_ld32(tbase + lane_off + C::T_DQ + 32, r1);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_DQE));
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                stg[c * HD + dcol] = __uint_as_float(r0[c]) * scale;
+                stg[(32 + c) * HD + dcol] = __uint_as_float(r1[c]) * scale;
+            }
+            fence_async_smem();
+            asm volatile("barrier.sync 2, 128;" ::: "memory");
+            if (leader) {
+                tma_reduce_add_4d(&tm_dq, s_base + C::OFF_DQ, 0, seq.h, seq.q_row(), bb);
+                bulk_commit();
+            }
+            ++n;
+        }
+        if (leader) bulk_wait_all();
+    } else {
+        // ================================================================ P / dS warps 0-7
+        const int half = warp >> 2;
+        const int wl = warp & 3;
+        const int krow = wl * 32 + lane;  // key row of the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
+        WaitCtx w{abort_flag, p.status, 47 + half};
+        const int key = k_lo + krow;
+        const bool key_ok = key < p.kv_len;
+        const int64_t pk = range_pos(kr, (int64_t)(key_ok ? key : (p.kv_len > 0 ? p.kv_len - 1 : 0)));
+        const float sl2 = p.scale_log2;
+        bool aborted = false;
+        int n = 0;
+        while (seq.next()) {
+            const int s = n % NS;
+            // columns [0, c_first) of this row are masked (keys past the block end,
+            // or queries that precede the key)
+            int c_first = 0;
+            if (seq.partial()) {
+                if (!key_ok) {
+                    c_first = BQ;
+                } else if (p.causal) {
+                    // rows past the block end are clamped to its last row: a range
+                    // gives positions only for its own rows, and the search needs
+                    // them non-decreasing (those rows carry no probability anyway)
+                    int lo = 0, hi = BQ;
+                    const int64_t row0 = (int64_t)seq.qt * BQ, last = p.q_len - 1;
+                    while (lo < hi) {
+                        const int mid = (lo + hi) >> 1;
+                        const int64_t row = row0 + mid < last ? row0 + mid : last;
+                        if (range_pos(seq.qr, row) < pk) lo = mid + 1; else hi = mid;
+                    }
+                    c_first = lo;
+                }
+            }
+            c_first -= half * 32;
+            {
+                const bool okw = mbar_wait(bar(C::B_SF + (n & 1)), (n >> 1) & 1, w) &&
+                                 mbar_wait(bar(C::B_QF + s), (n / NS) & 1, w);
+                if (__any_sync(0xffffffffu, !okw)) { aborted = true; break; }
+            }
+            tc_fence_after();
+            uint32_t sv[32];
+            tmem_ld32(tbase + lane_off + C::T_S + (uint32_t)((n & 1) * BQ + half * 32), sv);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_SE + (n & 1)));
+            const float2 *stat = reinterpret_cast<const float2 *>(smem + C::OFF_ST + s * BQ * 8) + half * 32;
+            float pv[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                const float x = fmaf(__uint_as_float(sv[c]), sl2, -stat[c].x);
+                pv[c] = (c < c_first) ? 0.f : ex2_approx(x);
+            }
+            uint32_t pk16[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pk16[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
+            if (n > 0) {
+                const bool okw = mbar_wait(bar(C::B_PE), (n - 1) & 1, w);
+                if (__any_sync(0xffffffffu, !okw)) { aborted = true; break; }
+            }
+            st_sw128_half(smem + C::OFF_P, krow, half, pk16);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_PR));
+            {
+                const bool okw = mbar_wait(bar(C::B_DPF), n & 1, w);
+                if (__any_sync(0xffffffffu, !okw)) { aborted = true; break; }
+            }
+            tc_fence_after();
+            uint32_t dv[32];
+            tmem_ld32(tbase + lane_off + C::T_DP + (uint32_t)(half * 32), dv);
+            tc_fence_before();
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const float d0 = pv[2 * c] * (__uint_as_float(dv[2 * c]) - stat[2 * c].y);
+                const float d1 = pv[2 * c + 1] * (__uint_as_float(dv[2 * c + 1]) - stat[2 * c + 1].y);
+                pk16[c] = pack_bf16x2(d0, d1);
+            }
+            if (n > 0) {
+                const bool okw = mbar_wait(bar(C::B_DSE), (n - 1) & 1, w);
+                if (__any_sync(0xffffffffu, !okw)) { aborted = true; break; }
+            }
+            st_sw128_half(smem + C::OFF_DS, krow, half, pk16);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_DSR));
+            ++n;
+        }
+        aborted = __any_sync(0xffffffffu, aborted || (*abort_flag != 0));
+
+        // ================================================================ dK / dV epilogue
+        if (!aborted) {
+            const bool okw = mbar_wait(bar(C::B_DONE), 0, w);
+            aborted = __any_sync(0xffffffffu, !okw);
+            if (!aborted) tc_fence_after();
+        }
+        if (!aborted) {
+            const uint32_t t_acc = half == 0 ? C::T_DK : C::T_DV;
+            const float f = half == 0 ? p.scale : 1.f;
+            void *out = half == 0 ? p.dk : p.dv;
+            const int64_t sb = half == 0 ? p.dk_sb : p.dv_sb, ss = half == 0 ? p.dk_ss : p.dv_ss,
+                          sh = half == 0 ? p.dk_sh : p.dv_sh;
+            const int64_t orow = (int64_t)j * p.kv_row_step + key;
+            uint16_t *dst = reinterpret_cast<uint16_t *>(out) + (int64_t)bb * sb + orow * ss + (int64_t)hk * sh;
+#pragma unroll
+            for (int c0 = 0; c0 < HD; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tbase + lane_off + t_acc + (uint32_t)c0, r);
+                float v[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) v[c] = n > 0 ? __uint_as_float(r[c]) * f : 0.f;
+                if (key_ok) store_bf16x32(dst + c0, v);
+            }
+        }
+    }
+
+    // ---- teardown: all TMEM traffic done, CTA-wide barrier, owner frees TMEM
+    __syncwarp();
+    tc_fence_before();
+    asm volatile("barrier.sync 1, %0;" ::"n"(NTHREADS) : "memory");
+    if (warp == WARP_MMA) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tbase, C::TMEM_COLS);
+    }
+}
+
+// Per query row: (lse log2 e, D = do . o) into the statistics table (padding rows
+// get (+inf, 0), which makes their probabilities 0), and a zeroed dQ accumulator row.
+// One warp per (batch, head, rank, padded row).
+__global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __grid_constant__ BwdParams p, int64_t acc_rows)
+{
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t total = (int64_t)p.b * p.hq * p.n_ranks * p.lpad;
+    if (gw >= total) return;
+    const int t = (int)(gw % p.lpad);
+    int64_t rest = gw / p.lpad;
+    const int i = (int)(rest % p.n_ranks);
+    rest /= p.n_ranks;
+    const int h = (int)(rest % p.hq);
+    const int bb = (int)(rest / p.hq);
+    float2 st = make_float2(INFINITY, 0.f);
+    if (t < p.q_len) {
+        const int64_t row = (int64_t)i * p.q_row_step + t;
+        const uint2 ov = *reinterpret_cast<const uint2 *>(reinterpret_cast<const uint16_t *>(p.o) + bb * p.o_sb +
+                                                          row * p.o_ss + h * p.o_sh + lane * 4);
+        const uint2 gv = *reinterpret_cast<const uint2 *>(reinterpret_cast<const uint16_t *>(p.dout) + bb * p.do_sb +
+                                                          row * p.do_ss + h * p.do_sh + lane * 4);
+        auto lo = [](uint32_t x) { return __uint_as_float(x << 16); };
+        auto hi = [](uint32_t x) { return __uint_as_float(x & 0xffff0000u); };
+        float acc = lo(ov.x) * lo(gv.x);
+        acc = fmaf(hi(ov.x), hi(gv.x), acc);
+        acc = fmaf(lo(ov.y), lo(gv.y), acc);
+        acc = fmaf(hi(ov.y), hi(gv.y), acc);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        const float lse = p.lse[bb * p.lse_sb + h * p.lse_sh + row * p.lse_ss];
+        st.x = (lse == -INFINITY) ? INFINITY : lse * kLog2eB;
+        st.y = acc;
+        float4 *dq = reinterpret_cast<float4 *>(p.dq_acc + (((int64_t)bb * acc_rows + row) * p.hq + h) * HD) + lane;
+        *dq = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (lane == 0) p.stats[gw] = st;
+}
+
+// dq = dq_acc (already scaled) in bf16; 8 values per thread.
+__global__ void __launch_bounds__(256) attn_bwd_post_kernel(const __grid_constant__ BwdParams p, int64_t acc_rows)
+{
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t per_row = HD / 8;
+    const int64_t total = (int64_t)p.b * p.n_ranks * p.q_len * p.hq * per_row;
+    if (idx >= total) return;
+    const int c8 = (int)(idx % per_row);
+    int64_t rest = idx / per_row;
+    const int h = (int)(rest % p.hq);
+    rest /= p.hq;
+    const int64_t t = rest % ((int64_t)p.n_ranks * p.q_len);
+    const int bb = (int)(rest / ((int64_t)p.n_ranks * p.q_len));
+    const int64_t row = (t / p.q_len) * p.q_row_step + t % p.q_len;
+    const float4 *src = reinterpret_cast<const float4 *>(p.dq_acc + (((int64_t)bb * acc_rows + row) * p.hq + h) * HD) +
+                        c8 * 2;
+    const float4 a = src[0], b = src[1];
+    uint4 w;
+    w.x = pack_bf16x2(a.x, a.y);
+    w.y = pack_bf16x2(a.z, a.w);
+    w.z = pack_bf16x2(b.x, b.y);
+    w.w = pack_bf16x2(b.z, b.w);
+    *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.dq) + bb * p.dq_sb + row * p.dq_ss + h * p.dq_sh +
+                               c8 * 8) = w;
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFnB)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFnB encode_fn_b()
+{
+    static EncodeTiledFnB fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFnB>(ptr);
+    }
+    return fn;
+}
+
+// [b, s, H, d] tensor with element strides (sb, ss, sh, 1) -> 4-D map {d, H, s, b}.
+bool make_map_b(CUtensorMap *m, CUtensorMapDataType dt, int es, const void *base, int64_t b, int64_t s, int64_t H,
+                int64_t d, int64_t sb, int64_t ss, int64_t sh, uint32_t box_d, uint32_t box_s, CUtensorMapSwizzle sw)
+{
+    EncodeTiledFnB fn = encode_fn_b();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)s, (cuuint64_t)b};
+    cuuint64_t strides[3] = {(cuuint64_t)(sh * es), (cuuint64_t)(ss * es), (cuuint64_t)(sb * es)};
+    cuuint32_t box[4] = {box_d, 1, box_s, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream)
+{
+    if (p.d != HD) return cudaErrorInvalidValue;
+    const int64_t q_rows = (int64_t)p.n_ranks * p.q_row_step;
+    const int64_t kv_rows = (int64_t)p.n_ranks * p.kv_row_step;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+    CUtensorMap tq, tk, tv, tdo, tdq;
+    if (!make_map_b(&tq, BF, 2, p.q, p.b, q_rows, p.hq, HD, p.q_sb, p.q_ss, p.q_sh, 64, BQ, SW) ||
+        !make_map_b(&tdo, BF, 2, p.dout, p.b, q_rows, p.hq, HD, p.do_sb, p.do_ss, p.do_sh, 64, BQ, SW) ||
+        !make_map_b(&tk, BF, 2, p.k, p.b, kv_rows, p.hkv, HD, p.k_sb, p.k_ss, p.k_sh, 64, BK, SW) ||
+        !make_map_b(&tv, BF, 2, p.v, p.b, kv_rows, p.hkv, HD, p.v_sb, p.v_ss, p.v_sh, 64, BK, SW) ||
+        !make_map_b(&tdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.dq_acc, p.b, q_rows, p.hq, HD, q_rows * p.hq * HD,
+                    (int64_t)p.hq * HD, HD, HD, BQ, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BCfg::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int64_t warps = (int64_t)p.b * p.hq * p.n_ranks * p.lpad;
+    if (warps == 0) return cudaSuccess;
+    attn_bwd_pre_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, stream>>>(p, q_rows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t items = (int64_t)(p.order_len ? p.order_len : p.n_ranks * p.n_kt) * p.b * p.hkv;
+    if (items > 0) {
+        attn_bwd_kernel<<<(unsigned)items, NTHREADS, BCfg::SMEM, stream>>>(p, tq, tk, tv, tdo, tdq);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    const int64_t threads = (int64_t)p.b * p.n_ranks * p.q_len * p.hq * (HD / 8);
+    attn_bwd_post_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(p, q_rows);
+    return cudaGetLastError();
+}
+
+}  // namespace cpattn

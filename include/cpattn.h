@@ -13,7 +13,9 @@
  *     running (o, lse); Q and O never move;
  *   - sections 因果掩码带来的负载不均 / Zig-zag / Striped / 重排 token 的代价: the
  *     causal mask is judged on original token positions, and the three token
- *     layouts are permutations applied once at model entry.
+ *     layouts are permutations applied once at model entry;
+ *   - section 分块注意力, paragraph on the backward pass: with the global lse any
+ *     key block alone gives its exact share of dq, dk, dv.
  *
  * Conventions shared by every entry point
  *   - Token tensors are [b, s, H, d] with d contiguous; lse tensors are
@@ -139,6 +141,36 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
  * Returns 0 as well for invalid arguments (cp_ring_attn_fwd then reports them). */
 size_t cp_ring_workspace_bytes(int32_t layout, int32_t N, int32_t mode, int32_t dtype, int64_t b,
                                int64_t S, int64_t Hq, int64_t d);
+
+/* Ring attention backward over N virtual ranks on one GPU (section 分块注意力,
+ * paragraph on the backward pass; section Ring Attention for the schedule).
+ * With the forward's GLOBAL o and lse of every query row and the output gradient
+ * dout, computes the gradients of L with dL/do = dout:
+ *   p = e^{x - lse},  dv_j = sum_q p dout,  dx = p (dout . v_j - D),  D = dout . o,
+ *   dq = scale sum_j dx k_j,  dk_j = scale sum_q dx q      (x = scale q . k).
+ * The K/V blocks walk the ring once more; dK, dV travel with their block and dQ
+ * accumulates on its rank.  One launch covers all N steps (like CP_RING_FUSED),
+ * between a statistics pass (D and zeroed accumulators) and the dq conversion.
+ *   q, o, dout [b, S, Hq, d]; k, v [b, S, Hkv, d]; lse [b, Hq, S, 1] fp32; all in
+ *   rank-major order, as cp_ring_attn_fwd takes and returns them (o and lse are its
+ *   results for the same q, k, v, layout, N, causal and softmax_scale).
+ *   dq [b, S, Hq, d], dk / dv [b, S, Hkv, d]: outputs (bf16, rank-major), overwritten.
+ *   workspace: device memory of at least cp_ring_bwd_workspace_bytes(...) bytes,
+ *   256-byte aligned (row statistics and the fp32 dQ accumulator); the caller keeps
+ *   it alive until the work on `stream` has finished.
+ * Requires bf16 tensors and d = 128 (CP_ERR_UNSUPPORTED otherwise) besides the
+ * conditions of cp_ring_attn_fwd.  Rows whose lse is -inf contribute nothing.
+ * dq sums its shares with fp32 atomic reductions, so its rounding can differ from
+ * run to run; dk and dv are summed in a fixed order. */
+cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q,
+                           const cp_tensor *k, const cp_tensor *v, const cp_tensor *o,
+                           const cp_tensor *lse, const cp_tensor *dout, float softmax_scale,
+                           cp_tensor *dq, cp_tensor *dk, cp_tensor *dv, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+/* Workspace bytes cp_ring_attn_bwd needs (0 for invalid arguments). */
+size_t cp_ring_bwd_workspace_bytes(int32_t layout, int32_t N, int32_t dtype, int64_t b, int64_t S,
+                                   int64_t Hq, int64_t d);
 
 /* Token permutation into / out of rank-major order (section 重排 token 的代价).
  *   x and x_ranked: same shape, dtype and contiguous layout; the sequence axis is

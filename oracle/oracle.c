@@ -235,7 +235,9 @@ typedef struct {
     double scale;
     const double *lse_in, *delta_in; /* [b, hq, sq] or NULL (compute them) */
     double *lse, *delta;             /* [b, hq, sq] statistics in use */
-    const unsigned char *head_mask;  /* [b * hq]: rows of unmarked heads skipped; NULL = all */
+    const int64_t *min_pos;          /* [b * hq]: with the causal mask only rows at positions
+                                        >= min_pos are needed, without it only heads whose
+                                        entry is not INT64_MAX; NULL = every row */
     const int64_t *sel;              /* [n][3] selected rows, or NULL = every row */
     double *dq;                      /* query pass: [b, sq, hq, d] or [n][d]; NULL = stats only */
     double *dk, *dv;                 /* key pass: [b, sk, hkv, d] or [n][d] */
@@ -273,9 +275,12 @@ static void *bwd_query_worker(void *arg)
         } else {
             i = r % j->sq; h = (r / j->sq) % j->hq; bb = r / (j->sq * j->hq);
         }
-        if (j->head_mask && !j->head_mask[bb * j->hq + h]) continue;
         const int64_t hk = h / g;
         const int64_t pq = j->pos_q ? j->pos_q[i] : i;
+        if (j->min_pos) {
+            const int64_t mp = j->min_pos[bb * j->hq + h];
+            if (mp == INT64_MAX || (j->causal && pq < mp)) continue;
+        }
         const double *qi = qrow_of(j, j->q, bb, i, h);
         const double *doi = qrow_of(j, j->dout, bb, i, h);
         const int64_t srow = (bb * j->hq + h) * j->sq + i;
@@ -414,7 +419,8 @@ int oracle_attention_bwd(const double *q, const double *k, const double *v, cons
  *   sel_q [nq][3] = (batch, q head, query index) -> dq_sel [nq][d]
  *   sel_k [nk][3] = (batch, kv head, key index)  -> dk_sel, dv_sel [nk][d]
  * The statistics are computed from the definition: per selected query row, and
- * for every query row of the heads that a selected key row serves. */
+ * for every query row that may see a selected key row (same batch, a query head
+ * of the key's group, and with the causal mask a position at or after the key). */
 int oracle_attention_bwd_sel(const double *q, const double *k, const double *v, const double *dout,
                              const int64_t *pos_q, const int64_t *pos_k, int64_t b, int64_t sq,
                              int64_t sk, int64_t hq, int64_t hkv, int64_t d, int causal, double scale,
@@ -446,15 +452,19 @@ int oracle_attention_bwd_sel(const double *q, const double *k, const double *v, 
     if (rc == 0 && nk > 0) {
         const int64_t nstat = b * hq * sq;
         double *stats = (double *)malloc(sizeof(double) * (size_t)(2 * nstat + 1));
-        unsigned char *mask = (unsigned char *)calloc((size_t)(b * hq + 1), 1);
-        if (!stats || !mask) { free(stats); free(mask); return -1; }
-        for (int64_t r = 0; r < nk; ++r)
+        int64_t *minp = (int64_t *)malloc(sizeof(int64_t) * (size_t)(b * hq + 1));
+        if (!stats || !minp) { free(stats); free(minp); return -1; }
+        for (int64_t x = 0; x < b * hq; ++x) minp[x] = INT64_MAX;
+        for (int64_t r = 0; r < nk; ++r) {
+            const int64_t t = sel_k[3 * r + 2];
+            const int64_t pk = pos_k ? pos_k[t] : t;
             for (int64_t h = sel_k[3 * r + 1] * g; h < (sel_k[3 * r + 1] + 1) * g; ++h)
-                mask[sel_k[3 * r] * hq + h] = 1;
+                if (pk < minp[sel_k[3 * r] * hq + h]) minp[sel_k[3 * r] * hq + h] = pk;
+        }
         bwd_job_t js = j;
         js.lse = stats;
         js.delta = stats + nstat;
-        js.head_mask = mask;
+        js.min_pos = minp;
         rc = run_bwd_jobs(&js, nstat, nthreads, bwd_query_worker);
         if (rc == 0) {
             bwd_job_t jk = j;
@@ -465,7 +475,7 @@ int oracle_attention_bwd_sel(const double *q, const double *k, const double *v, 
             jk.dv = dv_sel;
             rc = run_bwd_jobs(&jk, nk, nthreads, bwd_key_worker);
         }
-        free(mask);
+        free(minp);
         free(stats);
     }
     return rc;

@@ -1,0 +1,182 @@
+"""GPU parity of the ring backward (cp_ring_attn_bwd through the C ABI) against the
+fp64 oracle's gradients (section 分块注意力, paragraph on the backward pass).
+
+Tolerance, from the arithmetic of the bf16 path: Q, K, V, dO enter exactly; P and
+dS are rounded to bf16 before the tensor-core products (relative error u = 2^-8
+at most each), products accumulate in fp32, D = dO . o uses the forward's bf16 o,
+and the results are rounded to bf16 once more (u / 2).  Each gradient element is
+a sum whose terms carry a relative error of at most about 2u, so the error is
+bounded by a small multiple of u times the size of the summands; against the
+largest reference element that gives the bar used here,
+    max |got - ref| <= 2e-2 * max |ref|     (per gradient tensor),
+about five bf16 ulps of the largest element.  dK and dV are summed in a fixed
+order and must be bit-identical across runs; dQ sums with atomic reductions.
+"""
+import numpy as np
+import pytest
+import torch
+
+import cp_workloads as W
+import oracle
+from gpu_helpers import np64
+
+pytestmark = pytest.mark.gpu
+
+TOL_REL = 2e-2
+
+
+@pytest.fixture(scope="module")
+def cp():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import context_attention_cp_b200 as m
+    m.lib()
+    return m
+
+
+def _fwd_bwd(cp, q, k, v, do, layout, N, causal, scale):
+    """Original-order CPU inputs -> rank-major device tensors -> ring forward and
+    backward -> gradients back in original order (device tensors)."""
+    qr, kr, vr, dor = (cp.layout_permute(t.cuda(), layout, N) for t in (q, k, v, do))
+    o, lse = cp.ring_attn_fwd(qr, kr, vr, layout, N, causal, scale)
+    dq, dk, dv = cp.ring_attn_bwd(qr, kr, vr, o, lse, dor, layout, N, causal, scale)
+    cp.stream_check()
+    return tuple(cp.layout_permute(t, layout, N, inverse=True) for t in (dq, dk, dv))
+
+
+def _assert_grad(got, want, what):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    ref = np.max(np.abs(want)) if want.size else 0.0
+    err = np.max(np.abs(got - want)) if want.size else 0.0
+    assert err <= TOL_REL * ref, "%s: max abs err %.3g > %.3g (max |ref| %.3g)" % (what, err, TOL_REL * ref, ref)
+    return err / ref if ref else 0.0
+
+
+BWD_CASES = [
+    # layout, N, S, causal, b, hq, hkv
+    ("contiguous", 2, 512, True, 1, 4, 2),
+    ("zigzag", 4, 1024, True, 1, 4, 1),
+    ("zigzag", 2, 424, True, 2, 2, 2),       # c = 212: ragged query and key tiles
+    ("striped", 4, 1024, True, 1, 4, 2),
+    ("striped", 3, 390, True, 1, 2, 1),      # c = 130: a key tile of two keys
+    ("contiguous", 4, 1024, False, 1, 2, 2),
+    ("contiguous", 1, 320, True, 2, 2, 1),
+    ("contiguous", 3, 96, True, 1, 2, 2),    # c = 32, less than one query tile
+    ("zigzag", 8, 2048, True, 1, 8, 2),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_ring_bwd_matches_oracle(cp, case):
+    layout, N, S, causal, b, hq, hkv = case
+    d = 128
+    q, k, v = W.random_qkv(b, S, hq, hkv, d, "bf16", seed=S + 3 * N)
+    do = W.random_do(b, S, hq, d, "bf16", seed=S + 3 * N)
+    dq, dk, dv = _fwd_bwd(cp, q, k, v, do, layout, N, causal, d ** -0.5)
+    want = oracle.ring_attention_bwd(np64(q), np64(k), np64(v), np64(do), layout, N, causal, d ** -0.5)
+    for name, g, w in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
+        _assert_grad(np64(g), w, name)
+
+
+def test_ring_bwd_dkdv_deterministic(cp):
+    q, k, v = W.random_qkv(1, 2048, 8, 2, 128, "bf16", seed=77)
+    do = W.random_do(1, 2048, 8, 128, "bf16", seed=77)
+    a = _fwd_bwd(cp, q, k, v, do, "zigzag", 4, True, 128 ** -0.5)
+    b_ = _fwd_bwd(cp, q, k, v, do, "zigzag", 4, True, 128 ** -0.5)
+    assert torch.equal(a[1].view(torch.int16), b_[1].view(torch.int16))
+    assert torch.equal(a[2].view(torch.int16), b_[2].view(torch.int16))
+    assert (a[0].float() - b_[0].float()).abs().max().item() <= TOL_REL * a[0].float().abs().max().item()
+
+
+def test_ring_bwd_layouts_agree(cp):
+    """Permutation equivariance: the three layouts give the same gradients."""
+    q, k, v = W.random_qkv(1, 1024, 4, 2, 128, "bf16", seed=31)
+    do = W.random_do(1, 1024, 4, 128, "bf16", seed=31)
+    res = [_fwd_bwd(cp, q, k, v, do, lay, 4, True, 128 ** -0.5) for lay in ("contiguous", "zigzag", "striped")]
+    for r in res[1:]:
+        for g, g0 in zip(r, res[0]):
+            assert (g.float() - g0.float()).abs().max().item() <= TOL_REL * g0.float().abs().max().item()
+
+
+def test_ring_bwd_argument_errors(cp):
+    q, k, v = (t.cuda() for t in W.random_qkv(1, 256, 4, 2, 128, "bf16", seed=1))
+    o = torch.empty_like(q)
+    lse = torch.empty((1, 4, 256), dtype=torch.float32, device="cuda")
+    with pytest.raises(cp.CPError) as e:
+        cp.ring_attn_bwd(q, k, v, o, lse, q, "zigzag", 3, True)
+    assert e.value.code == 3
+    q64 = torch.zeros((1, 256, 4, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(cp.CPError) as e:
+        cp.ring_attn_bwd(q64, q64[:, :, :2], q64[:, :, :2], q64, lse, q64, "zigzag", 2, True)
+    assert e.value.code == 2
+    with pytest.raises(cp.CPError):
+        cp.ring_attn_bwd(q, k, v, o, lse[:, :, :128], q, "zigzag", 2, True)
+
+
+# ------------------------------------------------------------------ full sizes
+
+def _key_samples(w, rng):
+    """(batch, kv head, original key position): the last keys of the sequence, whose
+    gradients the oracle reaches through few query rows, plus early keys when the
+    sequence is short enough for the oracle to walk every query row."""
+    pos = {w.S - 1, w.S - 2, w.S - 64, w.S - 129}
+    pos.update(int(x) for x in rng.integers(w.S - 256, w.S, 4))
+    if w.S <= 8192:
+        pos.update({0, 1, 127, 128, w.S // 2, w.S // 4 - 1})
+    sel = []
+    for n, p in enumerate(sorted(pos)):
+        sel.append((n % w.b, (5 * n) % w.hkv, p))
+    return np.array(sel, dtype=np.int64)
+
+
+def _query_samples(w, rng):
+    pos = {0, 1, w.S - 1, w.S // 2, w.S // w.N, w.S // w.N - 1}
+    pos.update(int(x) for x in rng.integers(0, w.S, 8))
+    sel = []
+    for n, p in enumerate(sorted(pos)):
+        sel.append((n % w.b, (7 * n) % w.hq, p))
+    return np.array(sel, dtype=np.int64)
+
+
+BF16_WORKLOADS = [w.name for w in W.WORKLOADS if w.dtype == "bf16"]
+
+
+@pytest.mark.parametrize("name", BF16_WORKLOADS)
+def test_full_size_bwd_sampled(cp, name):
+    """Every bf16 workload at full size through the same launch as the bench:
+    sampled dq rows and dk, dv rows against the oracle, plus the row-sum identities
+    sum_j dk_j = 0 and sum_j dv_j = sum of dO over the group's rows."""
+    w = W.BY_NAME[name]
+    q, k, v = W.make_inputs(w)
+    do = W.make_do(w)
+    dq, dk, dv = _fwd_bwd(cp, q, k, v, do, w.layout, w.N, w.causal, w.scale)
+    rng = np.random.default_rng(w.seed)
+    sel_q = _query_samples(w, rng)
+    sel_k = _key_samples(w, rng) if w.causal else np.zeros((0, 3), np.int64)
+    # the oracle sees only the query rows it needs: the sampled ones and (causal)
+    # every row at or after the first sampled key
+    need = set(int(x) for x in sel_q[:, 2])
+    if len(sel_k):
+        need.update(range(int(sel_k[:, 2].min()), w.S))
+    rows = np.array(sorted(need), dtype=np.int64)
+    where = {int(r): n for n, r in enumerate(rows)}
+    sq = sel_q.copy()
+    sq[:, 2] = [where[int(x)] for x in sel_q[:, 2]]
+    ridx = torch.from_numpy(rows)
+    gq, gk, gv = oracle.attention_bwd_sel(np64(q[:, ridx]), np64(k), np64(v), np64(do[:, ridx]), w.causal, w.scale,
+                                          sq, sel_k, pos_q=rows)
+    got_q = np.stack([np64(dq[b_, p, h]) for b_, h, p in sel_q])
+    _assert_grad(got_q, gq, name + " dq")
+    if len(sel_k):
+        got_k = np.stack([np64(dk[b_, p, h]) for b_, h, p in sel_k])
+        got_v = np.stack([np64(dv[b_, p, h]) for b_, h, p in sel_k])
+        _assert_grad(got_k, gk, name + " dk")
+        _assert_grad(got_v, gv, name + " dv")
+    # identities at every size: the probabilities of a row sum to one
+    u = 2.0 ** -8
+    dk64, dv64 = dk.double(), dv.double()
+    assert torch.all(dk64.sum(1).abs() <= u * dk64.abs().sum(1) + 1e-30)
+    g = w.hq // w.hkv
+    do_sum = do.cuda().double().sum(1).view(w.b, w.hkv, g, w.d).sum(2)
+    assert torch.all((dv64.sum(1) - do_sum).abs() <= 2 * u * dv64.abs().sum(1))

@@ -170,15 +170,16 @@ def test_key_shift_leaves_gradients_unchanged():
         assert np.max(np.abs(x - y)) <= 1e-12
 
 
-def test_selected_rows_match_full():
+@pytest.mark.parametrize("causal", [True, False])
+def test_selected_rows_match_full(causal):
     b, S, hq, hkv, d = 2, 20, 4, 2, 6
     q, k, v, do = _inputs(55, b, S, S, hq, hkv, d)
     pos = np.asarray(L.rank_positions("striped", 4, S, 2) + L.rank_positions("striped", 4, S, 0)
                      + L.rank_positions("striped", 4, S, 3) + L.rank_positions("striped", 4, S, 1))
-    dq, dk, dv, _, _ = oracle.attention_bwd(q, k, v, do, True, 0.3, pos_q=pos, pos_k=pos)
+    dq, dk, dv, _, _ = oracle.attention_bwd(q, k, v, do, causal, 0.3, pos_q=pos, pos_k=pos)
     sel_q = np.array([[0, 0, 0], [1, 3, 19], [0, 2, 7], [1, 1, 11]])
     sel_k = np.array([[0, 0, 0], [1, 1, 19], [0, 1, 5], [1, 0, 12]])
-    gq, gk, gv = oracle.attention_bwd_sel(q, k, v, do, True, 0.3, sel_q, sel_k, pos_q=pos, pos_k=pos)
+    gq, gk, gv = oracle.attention_bwd_sel(q, k, v, do, causal, 0.3, sel_q, sel_k, pos_q=pos, pos_k=pos)
     for r, (bb, h, i) in enumerate(sel_q):
         assert np.max(np.abs(gq[r] - dq[bb, i, h])) <= 1e-14
     for r, (bb, hk, t) in enumerate(sel_k):
