@@ -632,7 +632,13 @@ cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_t
         p.order_len = (int)ord.size();
         std::copy(ord.begin(), ord.end(), p.order);
     }
-    cudaError_t e = launch_attn_bwd(p, static_cast<cudaStream_t>(stream));
+    // head-major grid once one head's work items fill a wave of the device
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    p.head_major = (int64_t)N * n_kt >= (int64_t)sms;
+    e = launch_attn_bwd(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return CP_OK;
 }

@@ -16,8 +16,8 @@
 // Per query tile, in the transposed form that puts keys on TMEM lanes:
 //   S^T  = K Q^T        (M 128 keys, N 64 queries, K = d)   -> TMEM
 //   dP^T = V dO^T       (same shapes)                        -> TMEM
-//   P^T  = exp2(S^T scale log2e - lse log2e), dS^T = P^T (dP^T - D)  (softmax warps,
-//          bf16 to shared memory, 128-byte swizzled, K-major)
+//   P^T  = exp2(S^T scale log2e - lse log2e), dS^T = P^T (dP^T - D)  (softmax warps;
+//          P^T bf16 back into TMEM, dS^T bf16 to shared memory, 128-byte swizzled)
 //   dV  += P^T dO       (M 128 keys, N = d, K 64 queries)    TMEM accumulator
 //   dK  += dS^T Q       (same)                               TMEM accumulator
 //   dQ^T = K^T dS^T     (M = d, N 64 queries, K 128 keys)    -> TMEM -> fp32 staging
@@ -29,7 +29,10 @@
 //   warp 12    TMA producer (K, V once; Q, dO and row statistics per query tile)
 //   warp 13    TMEM owner and single-thread MMA issuer
 // TMEM columns: S^T double buffer [0, 128), dP^T [128, 192), dQ^T [192, 256),
-// dV [256, 384), dK [384, 512).
+// dV [256, 384), dK [384, 512).  The softmax warps overwrite part of their own S^T
+// columns with bf16 P^T, which the dV MMA reads straight from TMEM; dS^T has two
+// shared-memory buffers, so tile n + 1 is written while the MMAs of tile n still
+// read tile n.  Three Q/dO stages keep the next loads in flight.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -43,7 +46,7 @@ namespace {
 constexpr int BK = kBwdKeyTile;    // keys per CTA
 constexpr int BQ = kBwdQueryTile;  // queries per step
 constexpr int HD = 128;            // head dim
-constexpr int NS = 2;              // Q / dO stages
+constexpr int NS = 3;              // Q / dO stages
 constexpr int NTHREADS = 448;
 constexpr int WARP_DQ0 = 8;
 constexpr int WARP_LOAD = 12;
@@ -59,9 +62,9 @@ struct BCfg {
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + KV_TILE;
     static constexpr int OFF_Q = OFF_V + KV_TILE;
-    static constexpr int OFF_P = OFF_Q + NS * STAGE;  // P^T  [128 keys][64 queries] bf16
-    static constexpr int OFF_DS = OFF_P + BK * 128;   // dS^T [128 keys][64 queries] bf16
-    static constexpr int OFF_DQ = OFF_DS + BK * 128;  // dQ staging [64 queries][128] fp32
+    static constexpr int PBUF = BK * 128;              // one [128 keys][64 queries] bf16 tile
+    static constexpr int OFF_DS = OFF_Q + NS * STAGE;  // dS^T, two buffers
+    static constexpr int OFF_DQ = OFF_DS + 2 * PBUF;   // dQ staging [64 queries][128] fp32
     static constexpr int OFF_ST = OFF_DQ + BQ * HD * 4;  // per stage: 64 x (lse log2e, D)
     static constexpr int OFF_BAR = OFF_ST + NS * BQ * 8;
     enum {
@@ -69,13 +72,11 @@ struct BCfg {
         B_QF = 1,
         B_QE = B_QF + NS,
         B_SF = B_QE + NS,
-        B_SE = B_SF + 2,
-        B_DPF = B_SE + 2,
-        B_PR,
-        B_PE,
-        B_DSR,
-        B_DSE,
-        B_DQF,
+        B_DPF = B_SF + 2,
+        B_PR,             // per tile parity: P^T in TMEM / dS^T in shared memory ready
+        B_DSR = B_PR + 2, // (8 warp arrivals); dS^T buffer free (MMA commit)
+        B_DSE = B_DSR + 2,
+        B_DQF = B_DSE + 2,
         B_DQE,
         B_DONE,
         NBAR
@@ -140,23 +141,29 @@ __device__ __forceinline__ bool bar_any(uint32_t id, uint32_t nthreads, bool pre
 
 // Query-tile sequence of one CTA: (query head of the group, ring step, query tile)
 // with the tile seeing at least one key of the CTA's key tile.  Every role walks it.
+// With the head-major grid, the steps of a head start at a rotation that depends on
+// the key tile, so CTAs of one key block reduce into different dQ rows at any one
+// time.
 struct QSeq {
     const BwdParams *p;
-    int j, k_lo, h0, n_qt;
+    int j, k_lo, h0, n_qt, nsteps, rot;
     Range kr;
-    int hi, r, qt, qt_full, i, h;
+    int hi, sc, r, qt, qt_full, i, h;
     Range qr;
 
-    __device__ void init(const BwdParams &pp, int jj, int klo, const Range &k, int hq0)
+    __device__ void init(const BwdParams &pp, int jj, int kt, const Range &k, int hq0)
     {
         p = &pp;
         j = jj;
-        k_lo = klo;
+        k_lo = kt * BK;
         kr = k;
         h0 = hq0;
         n_qt = (pp.q_len + BQ - 1) / BQ;
+        nsteps = pp.step_end - pp.step_begin;
+        rot = (nsteps > 0 && pp.head_major) ? kt % nsteps : 0;
         hi = 0;
-        r = pp.step_begin - 1;
+        sc = -1;
+        r = pp.step_begin;
         qt = n_qt - 1;
         qt_full = 0;
         i = 0;
@@ -164,13 +171,14 @@ struct QSeq {
     }
     __device__ bool next()
     {
+        if (nsteps <= 0) return false;
         ++qt;
         while (qt >= n_qt) {
-            ++r;
-            if (r >= p->step_end) {
-                r = p->step_begin;
+            if (++sc >= nsteps) {
+                sc = 0;
                 if (++hi >= p->group) return false;
             }
+            r = p->step_begin + (sc + rot) % nsteps;
             const int N = p->n_ranks;
             i = (j + r) % N;
             qr = p->use_layout ? layout_range(p->layout, N, p->seq_len, i) : p->q_range;
@@ -231,9 +239,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int lane = tid & 31;
 
     // ---- work item: (key rank, key tile) from the order table, then (batch, kv head)
+    // head_major: (batch, kv head) outermost, so the CTAs resident at one time share a
+    // few heads' dQ rows and the accumulator they reduce into stays in L2; otherwise
+    // the work order outermost (heaviest key tiles of every head first)
+    const int n_items = p.order_len ? p.order_len : p.n_ranks * p.n_kt;
     const int bkh = p.b * p.hkv;
-    const int e = blockIdx.x / bkh;
-    const int bh = blockIdx.x % bkh;
+    const int bh = p.head_major ? (int)(blockIdx.x / n_items) : (int)(blockIdx.x % bkh);
+    const int e = p.head_major ? (int)(blockIdx.x % n_items) : (int)(blockIdx.x / bkh);
     int j, kt;
     if (p.order_len) {
         j = (int)(p.order[e] >> 16);
@@ -250,12 +262,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (tid == 0) {
         mbar_init(bar(C::B_KV), 1);
         for (int s = 0; s < NS; ++s) { mbar_init(bar(C::B_QF + s), 1); mbar_init(bar(C::B_QE + s), 1); }
-        for (int b2 = 0; b2 < 2; ++b2) { mbar_init(bar(C::B_SF + b2), 1); mbar_init(bar(C::B_SE + b2), 8); }
+        for (int b2 = 0; b2 < 2; ++b2) mbar_init(bar(C::B_SF + b2), 1);
         mbar_init(bar(C::B_DPF), 1);
-        mbar_init(bar(C::B_PR), 8);
-        mbar_init(bar(C::B_PE), 1);
-        mbar_init(bar(C::B_DSR), 8);
-        mbar_init(bar(C::B_DSE), 1);
+        for (int b2 = 0; b2 < 2; ++b2) {
+            mbar_init(bar(C::B_PR + b2), 8);
+            mbar_init(bar(C::B_DSR + b2), 8);
+            mbar_init(bar(C::B_DSE + b2), 1);
+        }
         mbar_init(bar(C::B_DQF), 1);
         mbar_init(bar(C::B_DQE), 4);
         mbar_init(bar(C::B_DONE), 1);
@@ -272,7 +285,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tbase = *tmem_slot;
 
     QSeq seq;
-    seq.init(p, j, k_lo, kr, hk * p.group);
+    seq.init(p, j, kt, kr, hk * p.group);
 
     if (warp == WARP_LOAD) {
         // ================================================================ producer
@@ -354,38 +367,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const bool have_next = seq.next();
                 if (have_next) {
                     const int m = n + 1;
+                    // S buffer m & 1 last held S^T / P^T of tile m - 2, whose dV MMA was
+                    // issued earlier by this thread (MMAs run in issue order)
                     if (!mbar_wait(bar(C::B_QF + m % NS), (m / NS) & 1, w)) break;
-                    if (m >= 2 && !mbar_wait(bar(C::B_SE + (m & 1)), ((m >> 1) - 1) & 1, w)) break;
                     tc_fence_after();
                     issue_s(m);
                 }
                 const uint32_t qa = s_base + C::OFF_Q + s * C::STAGE;
-                // dV += P^T dO
-                if (!mbar_wait(bar(C::B_PR), n & 1, w)) break;
+                const int pb = n & 1;  // P^T / dS^T buffer of this tile
+                const uint32_t dsa = s_base + C::OFF_DS + pb * C::PBUF;
+                // dV += P^T dO, P^T (bf16) from TMEM: queries [0, 32) in columns [0, 16) of
+                // S buffer pb, queries [32, 64) in columns [32, 48)
+                if (!mbar_wait(bar(C::B_PR + pb), (n >> 1) & 1, w)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < BQ / 16; ++k)
-                    mma_ss(tbase + C::T_DV, smem_desc_sw128(s_base + C::OFF_P + k * 32, 16, 1024),
+                    mma_ts(tbase + C::T_DV, tbase + C::T_S + (uint32_t)(pb * BQ + (k >> 1) * 32 + (k & 1) * 8),
                            smem_desc_sw128(qa + C::Q_TILE + k * 2048, C::Q_SUB, 1024), IDESC_KV,
                            (n > 0 || k > 0) ? 1u : 0u);
-                tc_commit(bar(C::B_PE));
                 // dS^T ready: next dP first (the softmax waits on it), then dK and dQ^T
-                if (!mbar_wait(bar(C::B_DSR), n & 1, w)) break;
+                if (!mbar_wait(bar(C::B_DSR + pb), (n >> 1) & 1, w)) break;
                 tc_fence_after();
                 if (have_next) issue_dp(n + 1);
 #pragma unroll
                 for (int k = 0; k < BQ / 16; ++k)
-                    mma_ss(tbase + C::T_DK, smem_desc_sw128(s_base + C::OFF_DS + k * 32, 16, 1024),
+                    mma_ss(tbase + C::T_DK, smem_desc_sw128(dsa + k * 32, 16, 1024),
                            smem_desc_sw128(qa + k * 2048, C::Q_SUB, 1024), IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+                tc_commit(bar(C::B_QE + s));  // the last reader of this Q / dO stage
                 if (n > 0 && !mbar_wait(bar(C::B_DQE), (n - 1) & 1, w)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < BK / 16; ++k)
                     mma_ss(tbase + C::T_DQ, smem_desc_sw128(ka + k * 2048, C::KV_SUB, 1024),
-                           smem_desc_sw128(s_base + C::OFF_DS + k * 2048, C::KV_SUB, 1024), IDESC_DQ, k > 0 ? 1u : 0u);
+                           smem_desc_sw128(dsa + k * 2048, C::KV_SUB, 1024), IDESC_DQ, k > 0 ? 1u : 0u);
                 tc_commit(bar(C::B_DQF));
-                tc_commit(bar(C::B_DSE));
-                tc_commit(bar(C::B_QE + s));
+                tc_commit(bar(C::B_DSE + pb));
                 ++n;
                 have = have_next;
             }
@@ -472,28 +488,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             tc_fence_after();
             uint32_t sv[32];
-            tmem_ld32(tbase + lane_off + C::T_S + (uint32_t)((n & 1) * BQ + half * 32), sv);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_SE + (n & 1)));
-            const float2 *stat = reinterpret_cast<const float2 *>(smem + C::OFF_ST + s * BQ * 8) + half * 32;
+            const uint32_t s_cols = tbase + lane_off + C::T_S + (uint32_t)((n & 1) * BQ + half * 32);
+            tmem_ld32(s_cols, sv);
+            // (lse log2 e, D) of two query columns per 16-byte load
+            const float4 *stat = reinterpret_cast<const float4 *>(smem + C::OFF_ST + s * BQ * 8) + half * 16;
             float pv[32];
+            const uint64_t sl2x2 = f2_pack(sl2, sl2);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float x = fmaf(__uint_as_float(sv[c]), sl2, -stat[c].x);
-                pv[c] = (c < c_first) ? 0.f : ex2_approx(x);
+            for (int c = 0; c < 16; ++c) {
+                const float4 st = stat[c];
+                float x0, x1;
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), sl2x2,
+                                 f2_pack(-st.x, -st.z)),
+                          x0, x1);
+                pv[2 * c] = (2 * c < c_first) ? 0.f : ex2_approx(x0);
+                pv[2 * c + 1] = (2 * c + 1 < c_first) ? 0.f : ex2_approx(x1);
             }
             uint32_t pk16[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c) pk16[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
-            if (n > 0) {
-                const bool okw = mbar_wait(bar(C::B_PE), (n - 1) & 1, w);
-                if (__any_sync(0xffffffffu, !okw)) { aborted = true; break; }
-            }
-            st_sw128_half(smem + C::OFF_P, krow, half, pk16);
-            fence_async_smem();
+            // bf16 P^T over the first 16 of this warp's own 32 score columns (no other
+            // warp reads them), the A operand of the dV MMA
+            const int pb = n & 1;
+            tmem_st16(s_cols, pk16);
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_PR));
+            if (lane == 0) mbar_arrive(bar(C::B_PR + pb));
             {
                 const bool okw = mbar_wait(bar(C::B_DPF), n & 1, w);
                 if (__any_sync(0xffffffffu, !okw)) { aborted = true; break; }
@@ -504,18 +525,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc_fence_before();
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-                const float d0 = pv[2 * c] * (__uint_as_float(dv[2 * c]) - stat[2 * c].y);
-                const float d1 = pv[2 * c + 1] * (__uint_as_float(dv[2 * c + 1]) - stat[2 * c + 1].y);
+                const float4 st = stat[c];
+                const uint64_t t = f2_add(f2_pack(__uint_as_float(dv[2 * c]), __uint_as_float(dv[2 * c + 1])),
+                                          f2_pack(-st.y, -st.w));
+                float d0, d1;
+                f2_unpack(f2_fma(f2_pack(pv[2 * c], pv[2 * c + 1]), t, f2_pack(0.f, 0.f)), d0, d1);
                 pk16[c] = pack_bf16x2(d0, d1);
             }
-            if (n > 0) {
-                const bool okw = mbar_wait(bar(C::B_DSE), (n - 1) & 1, w);
+            if (n >= 2) {
+                const bool okw = mbar_wait(bar(C::B_DSE + pb), ((n >> 1) - 1) & 1, w);
                 if (__any_sync(0xffffffffu, !okw)) { aborted = true; break; }
             }
-            st_sw128_half(smem + C::OFF_DS, krow, half, pk16);
+            st_sw128_half(smem + C::OFF_DS + pb * C::PBUF, krow, half, pk16);
             fence_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_DSR));
+            if (lane == 0) mbar_arrive(bar(C::B_DSR + pb));
             ++n;
         }
         aborted = __any_sync(0xffffffffu, aborted || (*abort_flag != 0));

@@ -84,7 +84,9 @@ struct BwdParams {
     void *dq, *dk, *dv;
     int64_t dq_sb, dq_ss, dq_sh, dk_sb, dk_ss, dk_sh, dv_sb, dv_ss, dv_sh;
     int *status;
-    // work order: entry e -> (key rank, key tile) = (order[e] >> 16, order[e] & 0xffff)
+    // work order: entry e -> (key rank, key tile) = (order[e] >> 16, order[e] & 0xffff);
+    // head_major puts (batch, kv head) outside the order in the grid
+    int head_major;
     int n_kt;
     int order_len;
     uint32_t order[kMaxOrder];
