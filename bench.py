@@ -5,6 +5,8 @@
 
 One step = one cp_ring_attn_fwd over the whole workload (all N virtual ranks, all
 ring steps), inputs already permuted to rank-major order and resident in HBM.
+The line also carries the standalone merge bandwidth and the backward
+(cp_ring_attn_bwd) of the same workload, each timed on its own.
 L2 is flushed (a 256 MiB write) before every timed step; each step is timed with
 CUDA events on the launching stream.  With --gpus N > 1 (torchrun) every rank
 runs its own instance of the workload (weak scaling, no collective on the data
@@ -304,6 +306,48 @@ def main():
         merge["noncausal_s64k_contig32"] = merge_gbs(w5.b, w5.S, w5.hq, w5.d)
         torch.cuda.empty_cache()
 
+    # backward of the same workload (cp_ring_attn_bwd: statistics pass, the tcgen05
+    # kernel, dq conversion), inputs resident, L2 flushed before every timed call;
+    # effective FLOPs = 2.5x the forward's (five 2*d-flop products per visible pair)
+    def bwd_leg():
+        do = W.make_do(w).to(dev)
+        dor = cp.layout_permute(do, w.layout, w.N)
+        del do
+        step()
+        wsb = torch.empty(cp.ring_bwd_workspace_bytes(w.layout, w.N, 0, w.b, w.S, w.hq, w.d), dtype=torch.uint8,
+                          device=dev)
+        dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+
+        def bstep():
+            cp.ring_attn_bwd(qd, kd, vd, o, lse, dor, w.layout, w.N, w.causal, w.scale, dq, dk, dv, wsb)
+
+        for _ in range(3):
+            bstep()
+        ms = []
+        for _ in range(max(3, min(args.steps, 10))):
+            flush.zero_()
+            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b0.record(stream)
+            bstep()
+            b1.record(stream)
+            torch.cuda.synchronize()
+            ms.append(b0.elapsed_time(b1))
+        cp.stream_check()
+        t = statistics.mean(ms)
+        tf = 2.5 * flops / (t * 1e-3) / 1e12
+        del dor, wsb, dq, dk, dv
+        torch.cuda.empty_cache()
+        return {"metric": "ring-attn bwd TFLOP/s (effective: 5 products of 2*d flops per visible pair)",
+                "value": tf, "unit": "TFLOP/s", "ms_per_step": t, "steps": len(ms), "launches_per_step": 3,
+                "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel", "achieved": tf, "peak": peak_tf,
+                             "unit": "TFLOP/s", "frac": tf / peak_tf, "peak_source": peak_src + " bf16 burst",
+                             "timed": "whole call: statistics + attn_bwd_kernel + dq conversion",
+                             "traffic": None}}
+
+    backward = None
+    if w.dtype == "bf16" and w.d == 128 and rank == 0:
+        backward = bwd_leg()
+
     # end to end through the public API, every step: pinned host -> device copy of
     # q/k/v, permute to rank-major order, ring attention, unpermute, device -> host
     # copy of o and lse.  Consecutive steps are pipelined on three streams (copy-in,
@@ -383,6 +427,7 @@ def main():
                          "peak_source": peak_src + " bf16 burst",
                          "traffic": profiled_traffic() if w.name == W.BENCH_WORKLOAD else None},
             "merge": merge,
+            "backward": backward,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e_ms / e_steps, "pipelined": "copy-in / compute / copy-out on 3 streams"},
