@@ -14,7 +14,7 @@
 // (fp32 add) into an accumulator in HBM.
 //
 // Per query tile, in the transposed form that puts keys on TMEM lanes:
-//   S^T  = K Q^T        (M 128 keys, N 64 queries, K = d)   -> TMEM (K from TMEM)
+//   S^T  = K Q^T        (M 128 keys, N 64 queries, K = d)   -> TMEM
 //   dP^T = V dO^T       (same shapes)                        -> TMEM
 //   P^T  = exp2(S^T scale log2e - lse log2e), dS^T = P^T (dP^T - D)  (softmax warps;
 //          P^T bf16 back into TMEM, dS^T bf16 to shared memory, 128-byte swizzled)
@@ -28,13 +28,11 @@
 //   warps 8-11 dQ^T out of TMEM, scaled, staged, reduced into the accumulator
 //   warp 12    TMA producer (K, V once; Q, dO and row statistics per query tile)
 //   warp 13    TMEM owner and single-thread MMA issuer
-// TMEM columns: K (bf16, copied once) [0, 64), S^T [64, 128), dP^T [128, 192),
-// dQ^T [192, 256), dV [256, 384), dK [384, 512).  K as a TMEM operand spares the
-// S^T products half their shared-memory reads.  The softmax warps overwrite part
-// of their own S^T columns with bf16 P^T, which the dV MMA reads from TMEM; the
-// MMA warp issues S^T(n + 1) right after dV(n).  dS^T has two shared-memory
-// buffers, so tile n + 1 is written while the MMAs of tile n still read tile n.
-// Three Q/dO stages keep the next loads in flight.
+// TMEM columns: S^T double buffer [0, 128), dP^T [128, 192), dQ^T [192, 256),
+// dV [256, 384), dK [384, 512).  The softmax warps overwrite part of their own S^T
+// columns with bf16 P^T, which the dV MMA reads straight from TMEM; dS^T has two
+// shared-memory buffers, so tile n + 1 is written while the MMAs of tile n still
+// read tile n.  Three Q/dO stages keep the next loads in flight.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -74,10 +72,9 @@ struct BCfg {
         B_QF = 1,
         B_QE = B_QF + NS,
         B_SF = B_QE + NS,
-        B_KT,             // K copied into TMEM (8 warp arrivals)
-        B_DPF,
-        B_PR,             // P^T in TMEM ready (8 warp arrivals)
-        B_DSR,            // per dS^T buffer: ready (8 warp arrivals), free (MMA commit)
+        B_DPF = B_SF + 2,
+        B_PR,             // per tile parity: P^T in TMEM / dS^T in shared memory ready
+        B_DSR = B_PR + 2, // (8 warp arrivals); dS^T buffer free (MMA commit)
         B_DSE = B_DSR + 2,
         B_DQF = B_DSE + 2,
         B_DQE,
@@ -87,7 +84,7 @@ struct BCfg {
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 64 + 1024;
     static_assert(SMEM <= 232448, "shared memory per CTA exceeds 227 KB");
-    static constexpr uint32_t T_K = 0, T_S = 64, T_DP = 128, T_DQ = 192, T_DV = 256, T_DK = 384, TMEM_COLS = 512;
+    static constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 192, T_DV = 256, T_DK = 384, TMEM_COLS = 512;
 };
 
 // kind::f16 instruction descriptor with both operand majors selectable:
@@ -265,11 +262,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (tid == 0) {
         mbar_init(bar(C::B_KV), 1);
         for (int s = 0; s < NS; ++s) { mbar_init(bar(C::B_QF + s), 1); mbar_init(bar(C::B_QE + s), 1); }
-        mbar_init(bar(C::B_SF), 1);
-        mbar_init(bar(C::B_KT), 8);
-        mbar_init(bar(C::B_PR), 8);
+        for (int b2 = 0; b2 < 2; ++b2) mbar_init(bar(C::B_SF + b2), 1);
         mbar_init(bar(C::B_DPF), 1);
         for (int b2 = 0; b2 < 2; ++b2) {
+            mbar_init(bar(C::B_PR + b2), 8);
             mbar_init(bar(C::B_DSR + b2), 8);
             mbar_init(bar(C::B_DSE + b2), 1);
         }
@@ -336,14 +332,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) {
             WaitCtx w{abort_flag, p.status, 43};
             const uint32_t ka = s_base + C::OFF_K, va = s_base + C::OFF_V;
-            // S^T(n) = K Q(n)^T, K (bf16) as the A operand from TMEM
+            // S^T(n) = K Q(n)^T into S buffer n & 1
             auto issue_s = [&](int n) {
                 const uint32_t qa = s_base + C::OFF_Q + (n % NS) * C::STAGE;
+                const uint32_t d_t = tbase + C::T_S + (uint32_t)((n & 1) * BQ);
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k)
-                    mma_ts(tbase + C::T_S, tbase + C::T_K + (uint32_t)(k * 8),
+                    mma_ss(d_t, smem_desc_sw128(ka + (k >> 2) * C::KV_SUB + (k & 3) * 32, 16, 1024),
                            smem_desc_sw128(qa + (k >> 2) * C::Q_SUB + (k & 3) * 32, 16, 1024), IDESC_S, k > 0 ? 1u : 0u);
-                tc_commit(bar(C::B_SF));
+                tc_commit(bar(C::B_SF + (n & 1)));
             };
             // dP^T(n) = V dO(n)^T
             auto issue_dp = [&](int n) {
@@ -355,7 +352,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc_commit(bar(C::B_DPF));
             };
             bool have = seq.next();
-            bool ok = mbar_wait(bar(C::B_KV), 0, w) && mbar_wait(bar(C::B_KT), 0, w);
+            bool ok = mbar_wait(bar(C::B_KV), 0, w);
             if (have && ok) {
                 ok = mbar_wait(bar(C::B_QF + 0), 0, w);
                 if (ok) {
@@ -368,26 +365,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             while (have && ok) {
                 const int s = n % NS;
                 const bool have_next = seq.next();
-                const uint32_t qa = s_base + C::OFF_Q + s * C::STAGE;
-                const int pb = n & 1;  // dS^T buffer of this tile
-                const uint32_t dsa = s_base + C::OFF_DS + pb * C::PBUF;
-                // dV += P^T dO, P^T (bf16) from TMEM: queries [0, 32) in columns [0, 16) of
-                // the S buffer, queries [32, 64) in columns [32, 48)
-                if (!mbar_wait(bar(C::B_PR), n & 1, w)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < BQ / 16; ++k)
-                    mma_ts(tbase + C::T_DV, tbase + C::T_S + (uint32_t)((k >> 1) * 32 + (k & 1) * 8),
-                           smem_desc_sw128(qa + C::Q_TILE + k * 2048, C::Q_SUB, 1024), IDESC_KV,
-                           (n > 0 || k > 0) ? 1u : 0u);
-                // the next S^T overwrites the S buffer after that dV MMA (MMAs run in
-                // issue order); the softmax warps finished reading S^T(n) before P^T(n)
                 if (have_next) {
                     const int m = n + 1;
+                    // S buffer m & 1 last held S^T / P^T of tile m - 2, whose dV MMA was
+                    // issued earlier by this thread (MMAs run in issue order)
                     if (!mbar_wait(bar(C::B_QF + m % NS), (m / NS) & 1, w)) break;
                     tc_fence_after();
                     issue_s(m);
                 }
+                const uint32_t qa = s_base + C::OFF_Q + s * C::STAGE;
+                const int pb = n & 1;  // P^T / dS^T buffer of this tile
+                const uint32_t dsa = s_base + C::OFF_DS + pb * C::PBUF;
+                // dV += P^T dO, P^T (bf16) from TMEM: queries [0, 32) in columns [0, 16) of
+                // S buffer pb, queries [32, 64) in columns [32, 48)
+                if (!mbar_wait(bar(C::B_PR + pb), (n >> 1) & 1, w)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < BQ / 16; ++k)
+                    mma_ts(tbase + C::T_DV, tbase + C::T_S + (uint32_t)(pb * BQ + (k >> 1) * 32 + (k & 1) * 8),
+                           smem_desc_sw128(qa + C::Q_TILE + k * 2048, C::Q_SUB, 1024), IDESC_KV,
+                           (n > 0 || k > 0) ? 1u : 0u);
                 // dS^T ready: next dP first (the softmax waits on it), then dK and dQ^T
                 if (!mbar_wait(bar(C::B_DSR + pb), (n >> 1) & 1, w)) break;
                 tc_fence_after();
@@ -461,30 +458,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float sl2 = p.scale_log2;
         bool aborted = false;
         int n = 0;
-        // K into TMEM once (the A operand of every S^T MMA): this thread's key row,
-        // columns [64 half, 64 half + 64) of the head dim, out of the swizzled tile
-        {
-            const bool okw = mbar_wait(bar(C::B_KV), 0, w);
-            aborted = __any_sync(0xffffffffu, !okw);
-        }
-        if (!aborted) {
-            uint32_t kw[32];
-            const uint8_t *krow_p = smem + C::OFF_K + half * C::KV_SUB + krow * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v4 = *reinterpret_cast<const uint4 *>(krow_p + ((c ^ (krow & 7)) << 4));
-                kw[4 * c + 0] = v4.x;
-                kw[4 * c + 1] = v4.y;
-                kw[4 * c + 2] = v4.z;
-                kw[4 * c + 3] = v4.w;
-            }
-            tmem_st32(tbase + lane_off + C::T_K + (uint32_t)(half * 32), kw);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_KT));
-        }
-        while (!aborted && seq.next()) {
+        while (seq.next()) {
             const int s = n % NS;
             // columns [0, c_first) of this row are masked (keys past the block end,
             // or queries that precede the key)
@@ -508,13 +482,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             c_first -= half * 32;
             {
-                const bool okw = mbar_wait(bar(C::B_SF), n & 1, w) &&
+                const bool okw = mbar_wait(bar(C::B_SF + (n & 1)), (n >> 1) & 1, w) &&
                                  mbar_wait(bar(C::B_QF + s), (n / NS) & 1, w);
                 if (__any_sync(0xffffffffu, !okw)) { aborted = true; break; }
             }
             tc_fence_after();
             uint32_t sv[32];
-            const uint32_t s_cols = tbase + lane_off + C::T_S + (uint32_t)(half * 32);
+            const uint32_t s_cols = tbase + lane_off + C::T_S + (uint32_t)((n & 1) * BQ + half * 32);
             tmem_ld32(s_cols, sv);
             // (lse log2 e, D) of two query columns per 16-byte load
             const float4 *stat = reinterpret_cast<const float4 *>(smem + C::OFF_ST + s * BQ * 8) + half * 16;
@@ -540,7 +514,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_PR));
+            if (lane == 0) mbar_arrive(bar(C::B_PR + pb));
             {
                 const bool okw = mbar_wait(bar(C::B_DPF), n & 1, w);
                 if (__any_sync(0xffffffffu, !okw)) { aborted = true; break; }
