@@ -210,3 +210,32 @@ def test_selftest_limit_is_checked_before_any_launch(cp):
     f = cp.lib().cp_selftest_wait_timeout
     assert f(10, None) == 1             # below 1 ms
     assert f(5_000_000_000, None) == 1  # above 1 s
+
+
+def test_ring_bwd_argument_errors_are_synchronous(cp):
+    q = _ct(cp, [1, 256, 4, 128])
+    k = _ct(cp, [1, 256, 2, 128])
+    o = _ct(cp, [1, 256, 4, 128])
+    lse = _ct(cp, [1, 4, 256, 1], dtype=1)
+    dq = _ct(cp, [1, 256, 4, 128])
+    dk = _ct(cp, [1, 256, 2, 128])
+    f = cp.lib().cp_ring_attn_bwd
+    need = cp.lib().cp_ring_bwd_workspace_bytes(1, 2, 0, 1, 256, 4, 128)
+    assert need >= 256 * 4 * 128 * 4      # the fp32 dQ accumulator at least
+
+    def call(layout=1, N=2, causal=1, q_=q, k_=k, o_=o, lse_=lse, do_=q, dq_=dq, dk_=dk, ws=0x100000, wsb=None):
+        return f(layout, N, causal, ctypes.byref(q_), ctypes.byref(k_), ctypes.byref(k_), ctypes.byref(o_),
+                 ctypes.byref(lse_), ctypes.byref(do_), ctypes.c_float(0.088), ctypes.byref(dq_), ctypes.byref(dk_),
+                 ctypes.byref(dk_), ctypes.c_void_p(ws), need if wsb is None else wsb, None)
+
+    assert call(N=3) == 3                                  # S % 2N
+    assert call(layout=9) == 1                             # layout
+    assert call(causal=2) == 1                             # causal flag
+    assert call(wsb=16) == 1                               # workspace too small
+    assert call(ws=0x100010) == 1                          # workspace alignment
+    assert call(q_=_ct(cp, [1, 256, 4, 64]), k_=_ct(cp, [1, 256, 2, 64])) == 2  # d = 64 unsupported
+    qf = _ct(cp, [1, 256, 4, 128], dtype=1)
+    assert call(q_=qf, k_=_ct(cp, [1, 256, 2, 128], dtype=1)) == 2             # fp32 unsupported
+    assert call(dk_=_ct(cp, [1, 256, 4, 128])) == 3        # dk shaped like q
+    assert call(lse_=_ct(cp, [1, 4, 255, 1], dtype=1)) == 3
+    assert cp.lib().cp_ring_bwd_workspace_bytes(1, 3, 0, 1, 256, 4, 128) == 0  # S % N
