@@ -39,6 +39,12 @@ def _load():
         lib.oracle_lse_merge.restype = None
         lib.oracle_lse_merge.argtypes = [ctypes.c_int64, ctypes.c_int64] + [_F64P] * 6
         _bwd_sigs(lib)
+        lib.oracle_attention_doc.restype = ctypes.c_int
+        lib.oracle_attention_doc.argtypes = [_F64P, _F64P, _F64P, _I64P, _I64P] + [ctypes.c_int64] * 6 + \
+            [ctypes.c_int, _I64P, ctypes.c_int64, ctypes.c_double, _F64P, _F64P, ctypes.c_int]
+        lib.oracle_attention_rows_doc.restype = ctypes.c_int
+        lib.oracle_attention_rows_doc.argtypes = [_F64P, _I64P, ctypes.c_int64, _F64P, _F64P, _I64P] + \
+            [ctypes.c_int64] * 5 + [ctypes.c_int, _I64P, ctypes.c_int64, ctypes.c_double, _F64P, _F64P, ctypes.c_int]
         _lib = lib
     return _lib
 
@@ -251,3 +257,77 @@ def ring_attention_bwd_steps(q, k, v, do, layout_name, n_ranks, causal, scale, n
             dk[:, pj] += gk
             dv[:, pj] += gv
     return dq, dk, dv
+
+
+def _docs(doc_starts):
+    d = np.ascontiguousarray(doc_starts, dtype=np.int64)
+    if d.ndim != 1 or d.size < 1 or d[0] != 0 or np.any(np.diff(d) <= 0):
+        raise ValueError("doc_starts must be strictly increasing and start at 0")
+    return d
+
+
+def attention_doc(q, k, v, causal, scale, doc_starts, pos_q=None, pos_k=None, nthreads=None):
+    """Attention with a document mask (section All-Gather 式 CP: documents packed
+    into one sequence do not see each other).  doc_starts: sorted first positions
+    of the documents, starting with 0.  Otherwise as attention()."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    b, sq, hq, d = q.shape
+    bk, sk, hkv, dk = k.shape
+    if bk != b or dk != d or v.shape != k.shape:
+        raise ValueError("shape mismatch")
+    pq, pk = _opt_pos(pos_q, sq, "pos_q"), _opt_pos(pos_k, sk, "pos_k")
+    docs = _docs(doc_starts)
+    o = np.empty((b, sq, hq, d), np.float64)
+    lse = np.empty((b, hq, sq), np.float64)
+    rc = _load().oracle_attention_doc(_ptr(q, _F64P), _ptr(k, _F64P), _ptr(v, _F64P), _ptr(pq, _I64P),
+                                      _ptr(pk, _I64P), b, sq, sk, hq, hkv, d, int(bool(causal)), _ptr(docs, _I64P),
+                                      docs.size, float(scale), _ptr(o, _F64P), _ptr(lse, _F64P),
+                                      nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_attention_doc rejected its arguments")
+    return o, lse
+
+
+def attention_rows_doc(q_sel, sel, k, v, causal, scale, hq, doc_starts, pos_k=None, nthreads=None):
+    """attention_rows() with the document mask."""
+    q_sel = _f64(q_sel)
+    sel = np.ascontiguousarray(sel, dtype=np.int64)
+    k, v = _f64(k), _f64(v)
+    b, sk, hkv, d = k.shape
+    n = sel.shape[0]
+    pk = _opt_pos(pos_k, sk, "pos_k")
+    docs = _docs(doc_starts)
+    o = np.empty((n, d), np.float64)
+    lse = np.empty((n,), np.float64)
+    rc = _load().oracle_attention_rows_doc(_ptr(q_sel, _F64P), _ptr(sel, _I64P), n, _ptr(k, _F64P),
+                                           _ptr(v, _F64P), _ptr(pk, _I64P), b, sk, hq, hkv, d, int(bool(causal)),
+                                           _ptr(docs, _I64P), docs.size, float(scale), _ptr(o, _F64P),
+                                           _ptr(lse, _F64P), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_attention_rows_doc rejected its arguments")
+    return o, lse
+
+
+def allgather_attention(q, k, v, layout_name, n_ranks, causal, scale, doc_starts, nthreads=None):
+    """Reference result of All-Gather context parallelism (section All-Gather 式 CP)
+    on original-order tensors: every rank sees the whole K/V, so the result is the
+    plain definition with the document mask over the whole sequence.  Returns
+    (o, lse) in ORIGINAL token order."""
+    layout.tokens_per_rank(layout_name, n_ranks, q.shape[1])
+    return attention_doc(q, k, v, causal, scale, doc_starts, nthreads=nthreads)
+
+
+def allgather_attention_steps(q, k, v, layout_name, n_ranks, causal, scale, doc_starts, nthreads=None):
+    """The All-Gather schedule written out: K and V gathered into one original-order
+    copy, then each rank's queries (its layout positions) attend to all of it."""
+    S = q.shape[1]
+    layout.tokens_per_rank(layout_name, n_ranks, S)
+    q64 = _f64(q)
+    o = np.zeros(q64.shape)
+    lse = np.zeros((q64.shape[0], q64.shape[2], S))
+    for i in range(n_ranks):
+        pos = np.asarray(layout.rank_positions(layout_name, n_ranks, S, i), dtype=np.int64)
+        oi, li = attention_doc(q64[:, pos], k, v, causal, scale, doc_starts, pos_q=pos, nthreads=nthreads)
+        o[:, pos] = oi
+        lse[:, :, pos] = li
+    return o, lse

@@ -33,21 +33,40 @@
 #include <stdlib.h>
 #include <string.h>
 
+/* Document of a position: the index of the last document start <= pos, with
+ * doc_starts sorted ascending (section All-Gather 式 CP: several documents packed
+ * into one sequence, keys of another document are invisible).  -1 before the
+ * first start. */
+static int64_t doc_of(const int64_t *doc_starts, int64_t n_docs, int64_t pos)
+{
+    int64_t lo = 0, hi = n_docs; /* first start > pos */
+    while (lo < hi) {
+        int64_t mid = (lo + hi) / 2;
+        if (doc_starts[mid] <= pos) lo = mid + 1; else hi = mid;
+    }
+    return lo - 1;
+}
+
 /* One query row against all keys of one kv head.
  *   q      : d values of the query
  *   k, v   : key/value rows; row t starts at k + t * kv_row_stride
  *   pos_k  : original position of each key (NULL means t)
+ *   docs   : document starts (NULL = one document); a key of another document is
+ *            invisible
  *   x      : caller scratch of sk doubles
  * Writes d outputs to o and returns lse. */
 static double attend_row(const double *q, int64_t pos_q, const double *k, const double *v,
                          const int64_t *pos_k, int64_t sk, int64_t kv_row_stride, int64_t d,
-                         int causal, double scale, double *x, double *o)
+                         int causal, const int64_t *docs, int64_t n_docs, double scale, double *x,
+                         double *o)
 {
     double m = -INFINITY;
     int64_t nvis = 0;
+    const int64_t dq = docs ? doc_of(docs, n_docs, pos_q) : 0;
     for (int64_t t = 0; t < sk; ++t) {
         int64_t pk = pos_k ? pos_k[t] : t;
         if (causal && pk > pos_q) { x[t] = NAN; continue; }
+        if (docs && doc_of(docs, n_docs, pk) != dq) { x[t] = NAN; continue; }
         const double *kr = k + t * kv_row_stride;
         double dot = 0.0;
         for (int64_t e = 0; e < d; ++e) dot += q[e] * kr[e];
@@ -76,6 +95,8 @@ typedef struct {
     const int64_t *pos_q, *pos_k;
     int64_t b, sq, sk, hq, hkv, d;
     int causal;
+    const int64_t *docs;
+    int64_t n_docs;
     double scale;
     double *o, *lse;
     /* row selection (rows mode) */
@@ -103,8 +124,8 @@ static void *full_worker(void *arg)
         int64_t pq = j->pos_q ? j->pos_q[s] : s;
         double *orow = j->o + ((bb * j->sq + s) * j->hq + h) * j->d;
         j->lse[(bb * j->hq + h) * j->sq + s] =
-            attend_row(qr, pq, kb, vb, j->pos_k, j->sk, j->hkv * j->d, j->d, j->causal,
-                       j->scale, x, orow);
+            attend_row(qr, pq, kb, vb, j->pos_k, j->sk, j->hkv * j->d, j->d, j->causal, j->docs,
+                       j->n_docs, j->scale, x, orow);
     }
     free(x);
     return NULL;
@@ -121,7 +142,7 @@ static void *rows_worker(void *arg)
         const double *kb = j->k + (bb * j->sk * j->hkv + hk) * j->d;
         const double *vb = j->v + (bb * j->sk * j->hkv + hk) * j->d;
         j->lse[r] = attend_row(j->q_sel + r * j->d, pq, kb, vb, j->pos_k, j->sk, j->hkv * j->d,
-                               j->d, j->causal, j->scale, x, j->o + r * j->d);
+                               j->d, j->causal, j->docs, j->n_docs, j->scale, x, j->o + r * j->d);
     }
     free(x);
     return NULL;
@@ -184,6 +205,49 @@ int oracle_attention_rows(const double *q_sel, const int64_t *sel, int64_t n, co
     j.k = k; j.v = v; j.pos_k = pos_k;
     j.b = b; j.sk = sk; j.hq = hq; j.hkv = hkv; j.d = d;
     j.causal = causal; j.scale = scale; j.o = o_sel; j.lse = lse_sel;
+    j.sel = sel; j.q_sel = q_sel; j.nsel = n;
+    return run_jobs(&j, n, nthreads, rows_worker);
+}
+
+/* Attention with a document mask as well (section All-Gather 式 CP): doc_starts
+ * [n_docs] sorted ascending, first entry 0; key t is visible to query p only if
+ * both positions fall in the same document (and, causal, pos_k <= pos_q).
+ * Otherwise as oracle_attention. */
+int oracle_attention_doc(const double *q, const double *k, const double *v, const int64_t *pos_q,
+                         const int64_t *pos_k, int64_t b, int64_t sq, int64_t sk, int64_t hq,
+                         int64_t hkv, int64_t d, int causal, const int64_t *doc_starts,
+                         int64_t n_docs, double scale, double *o, double *lse, int nthreads)
+{
+    if (b < 0 || sq < 0 || sk < 0 || hq <= 0 || hkv <= 0 || d <= 0 || hq % hkv) return -1;
+    if (n_docs < 1 || !doc_starts || doc_starts[0] != 0) return -1;
+    for (int64_t i = 1; i < n_docs; ++i)
+        if (doc_starts[i] <= doc_starts[i - 1]) return -1;
+    job_t j;
+    memset(&j, 0, sizeof j);
+    j.q = q; j.k = k; j.v = v; j.pos_q = pos_q; j.pos_k = pos_k;
+    j.b = b; j.sq = sq; j.sk = sk; j.hq = hq; j.hkv = hkv; j.d = d;
+    j.causal = causal; j.docs = doc_starts; j.n_docs = n_docs; j.scale = scale; j.o = o; j.lse = lse;
+    return run_jobs(&j, b * hq * sq, nthreads, full_worker);
+}
+
+/* Selected rows with the document mask (see oracle_attention_rows). */
+int oracle_attention_rows_doc(const double *q_sel, const int64_t *sel, int64_t n, const double *k,
+                              const double *v, const int64_t *pos_k, int64_t b, int64_t sk,
+                              int64_t hq, int64_t hkv, int64_t d, int causal,
+                              const int64_t *doc_starts, int64_t n_docs, double scale,
+                              double *o_sel, double *lse_sel, int nthreads)
+{
+    if (n < 0 || b <= 0 || sk < 0 || hq <= 0 || hkv <= 0 || d <= 0 || hq % hkv) return -1;
+    if (n_docs < 1 || !doc_starts || doc_starts[0] != 0) return -1;
+    for (int64_t r = 0; r < n; ++r)
+        if (sel[3 * r] < 0 || sel[3 * r] >= b || sel[3 * r + 1] < 0 || sel[3 * r + 1] >= hq)
+            return -1;
+    job_t j;
+    memset(&j, 0, sizeof j);
+    j.k = k; j.v = v; j.pos_k = pos_k;
+    j.b = b; j.sk = sk; j.hq = hq; j.hkv = hkv; j.d = d;
+    j.causal = causal; j.docs = doc_starts; j.n_docs = n_docs; j.scale = scale;
+    j.o = o_sel; j.lse = lse_sel;
     j.sel = sel; j.q_sel = q_sel; j.nsel = n;
     return run_jobs(&j, n, nthreads, rows_worker);
 }
@@ -290,7 +354,7 @@ static void *bwd_query_worker(void *arg)
             D = j->delta_in[srow];
         } else {
             lse = attend_row(qi, pq, krow_of(j, j->k, bb, 0, hk), krow_of(j, j->v, bb, 0, hk), j->pos_k,
-                             j->sk, j->hkv * d, d, j->causal, j->scale, x, o);
+                             j->sk, j->hkv * d, d, j->causal, NULL, 0, j->scale, x, o);
             D = dotd(doi, o, d);
         }
         if (j->lse) { j->lse[srow] = lse; j->delta[srow] = D; }
