@@ -9,6 +9,7 @@ Entry points mirror include/cpattn.h:
   lse_merge(o_acc, lse_acc, o_b, lse_b, o_out=None)
   ring_attn_fwd(q, k, v, layout, N, causal, scale, o=None, lse=None, mode="fused")
   ring_attn_bwd(q, k, v, o, lse, do, layout, N, causal, scale) -> (dq, dk, dv)
+  allgather_attn_fwd(q, k, v, layout, N, causal, doc_starts=None, scale=None)
   layout_permute(x, layout, N, seq_axis=1, inverse=False, out=None)
   layout_range(layout, N, S, rank) -> (nseg, start, len, stride)
   tile_classes(q_range, q_len, kv_range, kv_len, causal, tile_q, tile_k)
@@ -17,7 +18,8 @@ Tensors are torch tensors on the current CUDA device; token tensors are
 [b, s, H, d] with d contiguous, lse tensors [b, H, s] fp32.
 """
 from ._binding import (  # noqa: F401
-    CPError, LAYOUTS, MODES, block_attn_fwd, layout_permute, layout_range, lib, lib_path,
+    CPError, LAYOUTS, MODES, allgather_attn_fwd, allgather_workspace_bytes, block_attn_fwd, layout_permute,
+    layout_range, lib, lib_path,
     lse_merge, ring_attn_bwd, ring_attn_fwd, ring_attn_fwd_static_scratch, ring_bwd_workspace_bytes,
     ring_workspace_bytes, selftest_wait_timeout, stream_check, tile_classes,
 )

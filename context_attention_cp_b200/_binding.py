@@ -39,6 +39,9 @@ _SIGNATURES = {
     "cp_ring_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _i64]),
     "cp_ring_attn_bwd": (_i32, [_i32, _i32, _i32, _T, _T, _T, _T, _T, _T, _f32, _T, _T, _T, _vp, _sz, _vp]),
     "cp_ring_bwd_workspace_bytes": (_sz, [_i32, _i32, _i32, _i64, _i64, _i64, _i64]),
+    "cp_allgather_attn_fwd": (_i32, [_i32, _i32, _i32, _T, _T, _T, ctypes.POINTER(ctypes.c_int64), _i32, _f32, _T, _T,
+                                     _vp, _sz, _vp]),
+    "cp_allgather_workspace_bytes": (_sz, [_i32, _i32, _i64, _i64, _i64, _i64, _i32]),
     "cp_layout_permute": (_i32, [_i32, _i32, _i32, _T, _T, _i32, _vp]),
     "cp_layout_range": (_i32, [_i32, _i32, _i64, _i32, _R]),
     "cp_tile_classes": (_i32, [_R, _i64, _R, _i64, _i32, _i32, _i32, ctypes.POINTER(ctypes.c_int8)]),
@@ -204,6 +207,34 @@ def ring_attn_bwd(q, k, v, o, lse, do, layout, N, causal, scale=None, dq=None, d
                                   *[_ref(t) for t in ts[6:]], ctypes.c_void_p(workspace.data_ptr()), need,
                                   _stream()))
     return dq, dk, dv
+
+
+def allgather_workspace_bytes(N, dtype_code, b, S, Hkv, d, n_docs):
+    return lib().cp_allgather_workspace_bytes(N, dtype_code, b, S, Hkv, d, n_docs)
+
+
+def allgather_attn_fwd(q, k, v, layout, N, causal, doc_starts=None, scale=None, o=None, lse=None, workspace=None):
+    """All-Gather context parallelism: every rank's Q against the gathered K/V, with an
+    optional document mask (doc_starts: first positions, starting with 0).  q/k/v/o/lse
+    in rank-major order."""
+    import torch
+    b, S, Hq, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    docs = [0] if doc_starts is None else [int(x) for x in doc_starts]
+    arr = (ctypes.c_int64 * len(docs))(*docs)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((b, Hq, S), dtype=torch.float32, device=q.device)
+    need = allgather_workspace_bytes(N, _dtype_code(q), b, S, k.shape[2], d, len(docs))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    tq, tk, tv, to, tl = _tensor(q), _tensor(k), _tensor(v), _tensor(o), _tensor(lse)
+    _check(lib().cp_allgather_attn_fwd(LAYOUTS[layout], N, int(bool(causal)), _ref(tq), _ref(tk), _ref(tv), arr,
+                                       len(docs), float(scale), _ref(to), _ref(tl),
+                                       ctypes.c_void_p(workspace.data_ptr()), need, _stream()))
+    return o, lse
 
 
 def ring_attn_fwd_static_scratch(q, k, v, layout, N, causal, scale, o, lse):

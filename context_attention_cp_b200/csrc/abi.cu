@@ -532,6 +532,120 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     return CP_OK;
 }
 
+size_t cp_allgather_workspace_bytes(int32_t N, int32_t dtype, int64_t b, int64_t S, int64_t Hkv, int64_t d,
+                                    int32_t n_docs)
+{
+    if (N < 1 || b < 0 || S < 0 || Hkv < 0 || d < 0 || n_docs < 1 || !elem_size(dtype)) return 0;
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    // gathered K and V in original token order, then the document starts (int32)
+    return (size_t)(2 * up(b * S * Hkv * d * elem_size(dtype)) + up((int64_t)n_docs * 4));
+}
+
+cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q, const cp_tensor *k,
+                                const cp_tensor *v, const int64_t *doc_starts, int32_t n_docs, float softmax_scale,
+                                cp_tensor *o, cp_tensor *lse, void *workspace, size_t workspace_bytes, void *stream)
+{
+    g_last_error[0] = 0;
+    cp_status s;
+    if (layout < 0 || layout > 2) return fail(CP_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (causal != 0 && causal != 1) return fail(CP_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if ((s = check_tensor(q, "q")) != CP_OK || (s = check_tensor(k, "k")) != CP_OK ||
+        (s = check_tensor(v, "v")) != CP_OK)
+        return s;
+    if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
+    if (q->dtype != CP_BF16) return fail(CP_ERR_UNSUPPORTED, "the All-Gather path takes bf16 tensors");
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    const int64_t S = q->shape[1];
+    if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
+    if (N < 1 || N > 4096) return fail(CP_ERR_INVALID_ARG, "N must be in [1, 4096]");
+    if (S >= ((int64_t)1 << 30)) return fail(CP_ERR_SHAPE, "sequence too long (S must be below 2^30)");
+    if (S % N) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of N = %d", (long long)S, N);
+    if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N)) return fail(CP_ERR_SHAPE, "zig-zag needs S to be a multiple of 2N");
+    if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;
+    if (o->dtype != q->dtype) return fail(CP_ERR_INVALID_ARG, "o must have q's dtype");
+    if (n_docs < 1 || !doc_starts) return fail(CP_ERR_INVALID_ARG, "doc_starts must hold at least one start");
+    if (doc_starts[0] != 0) return fail(CP_ERR_INVALID_ARG, "the first document must start at 0");
+    for (int32_t i = 1; i < n_docs; ++i)
+        if (doc_starts[i] <= doc_starts[i - 1] || doc_starts[i] >= S)
+            return fail(CP_ERR_INVALID_ARG, "document starts must increase and stay below S");
+    if (n_docs > 1 && !causal) return fail(CP_ERR_UNSUPPORTED, "the document mask is defined with the causal mask");
+    for (const cp_tensor *t : {k, v}) {
+        int64_t expect = 1;
+        for (int i = 3; i >= 0; --i) {
+            if (t->shape[i] > 1 && t->stride[i] != expect)
+                return fail(CP_ERR_INVALID_ARG, "k and v must be contiguous for the gather");
+            expect *= t->shape[i];
+        }
+    }
+    const int64_t b = q->shape[0], Hkv = k->shape[2], d = q->shape[3];
+    const size_t need = cp_allgather_workspace_bytes(N, q->dtype, b, S, Hkv, d, n_docs);
+    if (!workspace || workspace_bytes < need) return fail(CP_ERR_INVALID_ARG, "workspace of %zu bytes needed", need);
+    if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const int64_t c = S / N;
+    if (b == 0 || S == 0) return CP_OK;
+    const int rows = rows_per_cta(q->dtype);
+    const int n_qt = (int)((c + rows - 1) / rows);
+    if (n_qt > 65535) return fail(CP_ERR_SHAPE, "too many query tiles per rank");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // the all-gather: every rank's K/V block back into one original-order copy
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    char *ws = static_cast<char *>(workspace);
+    const int64_t kv_bytes = up(b * S * Hkv * d * elem_size(q->dtype));
+    cp_tensor kg{ws, q->dtype, 0, {b, S, Hkv, d}, {S * Hkv * d, Hkv * d, d, 1}};
+    cp_tensor vg{ws + kv_bytes, q->dtype, 0, {b, S, Hkv, d}, {S * Hkv * d, Hkv * d, d, 1}};
+    int *docs_dev = reinterpret_cast<int *>(ws + 2 * kv_bytes);
+    if ((s = cp_layout_permute(layout, N, 1, &kg, const_cast<cp_tensor *>(k), 1, stream)) != CP_OK) return s;
+    if ((s = cp_layout_permute(layout, N, 1, &vg, const_cast<cp_tensor *>(v), 1, stream)) != CP_OK) return s;
+    int32_t docs32[1024];
+    std::vector<int32_t> docs_big;
+    int32_t *docs_h = docs32;
+    if (n_docs > 1024) {
+        docs_big.resize((size_t)n_docs);
+        docs_h = docs_big.data();
+    }
+    for (int32_t i = 0; i < n_docs; ++i) docs_h[i] = (int32_t)doc_starts[i];
+    // pageable source: the copy is staged before the call returns
+    cudaError_t e = cudaMemcpyAsync(docs_dev, docs_h, sizeof(int32_t) * (size_t)n_docs, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "document table copy");
+
+    thread_local AttnParams p;
+    std::memset(&p, 0, sizeof p);
+    p.b = (int)b;
+    p.hq = (int)q->shape[2];
+    p.hkv = (int)Hkv;
+    p.group = p.hq / p.hkv;
+    p.d = (int)d;
+    p.q_len = (int)c;
+    p.kv_len = (int)S;
+    p.n_ranks = N;
+    p.step_begin = 0;
+    p.step_end = 1;
+    p.causal = causal;
+    p.use_layout = 1;
+    p.layout = layout;
+    p.seq_len = S;
+    p.kv_explicit = 1;
+    p.kv_range = Range{0, 0, S, 0, 1};
+    p.q_row_step = c;
+    p.kv_row_step = 0;
+    p.scale = softmax_scale;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.n_qt = n_qt;
+    p.doc_starts = n_docs > 1 ? docs_dev : nullptr;
+    p.n_docs = n_docs > 1 ? n_docs : 0;
+    const std::vector<uint32_t> &ord = ring_order(layout, N, S, causal, rows);
+    if ((int64_t)ord.size() <= kMaxOrder) {
+        p.order_len = (int)ord.size();
+        std::copy(ord.begin(), ord.end(), p.order);
+    }
+    fill_inputs(p, q, &kg, &vg);
+    fill_outputs(p, EPI_STORE, o, lse);
+    set_status_ptr(p);
+    return launch_attn(p, q->dtype, st);
+}
+
 size_t cp_ring_bwd_workspace_bytes(int32_t layout, int32_t N, int32_t dtype, int64_t b, int64_t S, int64_t Hq,
                                    int64_t d)
 {

@@ -97,9 +97,41 @@ struct Cfg {
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
 };
 
+// Document start of position pos: the last entry of the sorted starts <= pos.
+__device__ __forceinline__ int64_t doc_start_of(const int *starts, int n, int64_t pos)
+{
+    int lo = 0, hi = n;  // first start > pos
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if ((int64_t)__ldg(starts + mid) <= pos) lo = mid + 1; else hi = mid;
+    }
+    return lo > 0 ? (int64_t)__ldg(starts + lo - 1) : 0;
+}
+
+// First key tile t of a block (kv_len keys, ranges k, tiles of BN) whose key at
+// index min(t * BN + off, kv_len - 1) has a position >= x.
+__device__ __forceinline__ int first_tile_from(const Range &k, int64_t kv_len, int off, int64_t x)
+{
+    const int n_kt = (int)((kv_len + BN - 1) / BN);
+    int lo = 0, hi = n_kt;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        int64_t t = (int64_t)mid * BN + off;
+        if (t > kv_len - 1) t = kv_len - 1;
+        if (range_pos(k, t) < x) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+}
+
 // Key-tile sequence of one CTA: every (ring step, key tile) that at least one of the
 // two query tiles must visit, in order.  All roles walk the same sequence; tile n is
-// visited by query tile j iff kt < end[j] of its step.
+// visited by query tile j iff kt_beg[j] <= kt < kt_end[j] of its step, and needs the
+// element mask unless kt_fb[j] <= kt < kt_full[j].  Without documents kt_beg = kt_fb
+// = 0.  With the document mask the keys a query tile sees span from the document
+// start of its first row to its last row, and every row sees the keys from the
+// document start of its last row to its first row (positions increase with the
+// local index, so both are runs of whole tiles).
+template <bool DOC>
 struct TileSeq {
     const AttnParams *p;
     Range qr;
@@ -108,6 +140,8 @@ struct TileSeq {
     bool q_ok1;  // query tile 1 holds rows (tile 0 always does)
     int step, kt, kt_end_all;
     int kt_full0, kt_full1, kt_end0, kt_end1;
+    int kt_beg0, kt_beg1, kt_fb0, kt_fb1, kt_beg_all;
+    int64_t ds_min0, ds_max0, ds_min1, ds_max1;  // document starts of the tiles' first / last rows
     int src;
     Range kr;
 
@@ -121,28 +155,67 @@ struct TileSeq {
         step = pp.step_begin - 1;
         kt = 0;
         kt_end_all = 0;
+        kt_beg0 = kt_beg1 = kt_fb0 = kt_fb1 = kt_beg_all = 0;
+        ds_min0 = ds_max0 = ds_min1 = ds_max1 = 0;
+        if (DOC) {
+            const int64_t last = pp.q_len - 1;
+            ds_min0 = doc_start_of(pp.doc_starts, pp.n_docs, range_pos(q, (int64_t)qlo0));
+            ds_max0 = doc_start_of(pp.doc_starts, pp.n_docs, range_pos(q, (int64_t)(qlo0 + BM - 1 < last ? qlo0 + BM - 1 : last)));
+            if (q_ok1) {
+                ds_min1 = doc_start_of(pp.doc_starts, pp.n_docs, range_pos(q, (int64_t)(qlo0 + BM)));
+                ds_max1 = doc_start_of(pp.doc_starts, pp.n_docs,
+                                       range_pos(q, (int64_t)(qlo0 + 2 * BM - 1 < last ? qlo0 + 2 * BM - 1 : last)));
+            }
+        }
+    }
+    // With documents the two query tiles (far apart in position under the zig-zag
+    // layout) can need two disjoint runs of key tiles; tiles in between, needed by
+    // neither, are skipped, so every tile of the sequence has a reader (the K/V stage
+    // bookkeeping of the producer and the MMA warp relies on it).
+    __device__ void skip_gap()
+    {
+        if (!DOC || need(0) || need(1)) return;
+        int nk = kt_end_all;
+        if (kt < kt_beg0 && kt_beg0 < kt_end0 && kt_beg0 < nk) nk = kt_beg0;
+        if (q_ok1 && kt < kt_beg1 && kt_beg1 < kt_end1 && kt_beg1 < nk) nk = kt_beg1;
+        kt = nk;
     }
     __device__ bool next()
     {
         ++kt;
+        skip_gap();
         while (kt >= kt_end_all) {
             ++step;
             if (step >= p->step_end) return false;
             const int N = p->n_ranks;
             src = ((rank - step) % N + N) % N;
-            kr = p->use_layout ? layout_range(p->layout, N, p->seq_len, src) : p->kv_range;
+            kr = (p->use_layout && !p->kv_explicit) ? layout_range(p->layout, N, p->seq_len, src) : p->kv_range;
             kv_tile_bounds<int64_t>(qr, p->q_len, q_lo0, BM, kr, p->kv_len, BN, p->causal != 0, &kt_full0, &kt_end0);
             kt_full1 = kt_end1 = 0;
             if (q_ok1)
                 kv_tile_bounds<int64_t>(qr, p->q_len, q_lo0 + BM, BM, kr, p->kv_len, BN, p->causal != 0, &kt_full1,
                                         &kt_end1);
+            if (DOC) {
+                kt_beg0 = first_tile_from(kr, p->kv_len, BN - 1, ds_min0);
+                kt_fb0 = first_tile_from(kr, p->kv_len, 0, ds_max0);
+                kt_beg1 = q_ok1 ? first_tile_from(kr, p->kv_len, BN - 1, ds_min1) : kt_end1;
+                kt_fb1 = q_ok1 ? first_tile_from(kr, p->kv_len, 0, ds_max1) : kt_end1;
+                kt_beg_all = kt_beg0 < kt_beg1 ? kt_beg0 : kt_beg1;
+            }
             kt_end_all = kt_end0 > kt_end1 ? kt_end0 : kt_end1;
-            kt = 0;
+            kt = kt_beg_all;
+            skip_gap();
         }
         return true;
     }
-    __device__ bool need(int j) const { return kt < (j ? kt_end1 : kt_end0); }
-    __device__ bool partial(int j) const { return kt >= (j ? kt_full1 : kt_full0); }
+    __device__ bool need(int j) const
+    {
+        return kt < (j ? kt_end1 : kt_end0) && (!DOC || kt >= (j ? kt_beg1 : kt_beg0));
+    }
+    __device__ bool partial(int j) const
+    {
+        return kt >= (j ? kt_full1 : kt_full0) || (DOC && kt < (j ? kt_fb1 : kt_fb0));
+    }
 };
 
 __device__ __forceinline__ void store_row_chunk(void *o, int dtype, int64_t off, const float *v)
@@ -166,7 +239,7 @@ __device__ __forceinline__ void store_row_chunk(void *o, int dtype, int64_t off,
     }
 }
 
-template <int D>
+template <int D, bool DOC>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v)
@@ -248,7 +321,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             WaitCtx w{abort_flag, p.status, 1};
-            TileSeq seq;
+            TileSeq<DOC> seq;
             seq.init(p, qr, rank, q_lo0);
             int n = 0;
             const int q_row = (int)(rank * p.q_row_step) + q_lo0;
@@ -295,7 +368,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // ================================================================ MMA issuer
         if (lane == 0) {
             WaitCtx w{abort_flag, p.status, 3};
-            TileSeq seq;
+            TileSeq<DOC> seq;
             seq.init(p, qr, rank, q_lo0);
             int pc0 = 0, pc1 = 0;  // PV MMAs issued per query tile
             auto issue_s = [&](int j, int m) {
@@ -378,6 +451,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int row = q_lo0 + j * BM + r_in;  // local query index in the rank's block
         const bool row_ok = row < p.q_len;
         const int64_t pos_q = range_pos(qr, row_ok ? row : (p.q_len > 0 ? p.q_len - 1 : 0));
+        const int64_t ds_row = DOC ? doc_start_of(p.doc_starts, p.n_docs, pos_q) : 0;
         const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
         const uint32_t s_tmem = tbase + lane_off + (uint32_t)(j * 128);
         const uint32_t o_tmem = tbase + lane_off + C::T_O + (uint32_t)(j * D);
@@ -388,7 +462,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int c = 0;            // tiles processed by this query tile
         bool aborted = false;
 
-        TileSeq seq;
+        TileSeq<DOC> seq;
         seq.init(p, qr, rank, q_lo0);
         while (seq.next()) {
             if (!seq.need(j)) continue;
@@ -416,9 +490,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     cnt = lo;
                 }
+                int beg = 0;  // keys before this row's document start are invisible
+                if (DOC) {
+                    int lo = 0, hi = cnt;
+                    while (lo < hi) {
+                        const int mid = (lo + hi) >> 1;
+                        if (range_pos(seq.kr, k0 + mid) < ds_row) lo = mid + 1; else hi = mid;
+                    }
+                    beg = lo;
+                }
 #pragma unroll
                 for (int cc = 0; cc < BN; ++cc)
-                    if (cc >= cnt) s[cc] = -INFINITY;
+                    if (cc >= cnt || (DOC && cc < beg)) s[cc] = -INFINITY;
             }
             // ---- row max: four chains of 3-input max
             float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
@@ -607,6 +690,23 @@ bool make_map(CUtensorMap *m, const void *base, int64_t b, int64_t s, int64_t H,
     return r == CUDA_SUCCESS;
 }
 
+template <int D, bool DOC>
+cudaError_t launch_dd(const AttnParams &p, cudaStream_t stream, const CUtensorMap &tq, const CUtensorMap &tk,
+                      const CUtensorMap &tv)
+{
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e =
+            cudaFuncSetAttribute(attn_tc_kernel<D, DOC>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int64_t items = (int64_t)p.n_ranks * p.n_qt * p.b * p.hq;
+    if (items == 0) return cudaSuccess;
+    attn_tc_kernel<D, DOC><<<(unsigned)items, NTHREADS, Cfg<D>::SMEM, stream>>>(p, tq, tk, tv);
+    return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_d(const AttnParams &p, cudaStream_t stream, int64_t q_rows, int64_t kv_rows)
 {
@@ -615,18 +715,7 @@ cudaError_t launch_d(const AttnParams &p, cudaStream_t stream, int64_t q_rows, i
         !make_map(&tk, p.k, p.b, kv_rows, p.hkv, D, p.k_sb, p.k_ss, p.k_sh) ||
         !make_map(&tv, p.v, p.b, kv_rows, p.hkv, D, p.v_sb, p.v_ss, p.v_sh))
         return cudaErrorInvalidValue;
-    static bool attr_set[2] = {false, false};
-    const int slot = D == 128 ? 1 : 0;
-    if (!attr_set[slot]) {
-        cudaError_t e =
-            cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set[slot] = true;
-    }
-    const int64_t items = (int64_t)p.n_ranks * p.n_qt * p.b * p.hq;
-    if (items == 0) return cudaSuccess;
-    attn_tc_kernel<D><<<(unsigned)items, NTHREADS, Cfg<D>::SMEM, stream>>>(p, tq, tk, tv);
-    return cudaGetLastError();
+    return p.n_docs > 0 ? launch_dd<D, true>(p, stream, tq, tk, tv) : launch_dd<D, false>(p, stream, tq, tk, tv);
 }
 
 }  // namespace

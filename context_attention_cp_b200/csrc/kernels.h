@@ -47,6 +47,13 @@ struct AttnParams {
     float *lse;
     int64_t lse_sb, lse_sh, lse_ss;
     int *status;
+    // All-Gather form: kv_explicit = 1 takes kv_range for every rank and step (one
+    // gathered key block, kv_row_step = 0).  Document mask (bf16 path): doc_starts
+    // [n_docs] device array, sorted, first 0; a key in another document than the
+    // query is invisible; n_docs = 0 means none.
+    int kv_explicit;
+    const int *doc_starts;
+    int n_docs;
     // work order: entry e -> (rank, row group) = (order[e] >> 16, order[e] & 0xffff);
     // a row group is the query rows one CTA covers (256 tensor-core, 128 SIMT)
     int n_qt;                  // row groups per rank

@@ -15,7 +15,9 @@
  *     causal mask is judged on original token positions, and the three token
  *     layouts are permutations applied once at model entry;
  *   - section 分块注意力, paragraph on the backward pass: with the global lse any
- *     key block alone gives its exact share of dq, dk, dv.
+ *     key block alone gives its exact share of dq, dk, dv;
+ *   - section All-Gather 式 CP: K/V gathered once per layer, any attention mask
+ *     (documents) applied in one local pass.
  *
  * Conventions shared by every entry point
  *   - Token tensors are [b, s, H, d] with d contiguous; lse tensors are
@@ -141,6 +143,32 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
  * Returns 0 as well for invalid arguments (cp_ring_attn_fwd then reports them). */
 size_t cp_ring_workspace_bytes(int32_t layout, int32_t N, int32_t mode, int32_t dtype, int64_t b,
                                int64_t S, int64_t Hq, int64_t d);
+
+/* All-Gather context parallelism over N virtual ranks on one GPU (section
+ * All-Gather 式 CP): before attention the K/V blocks of all ranks are gathered into
+ * one copy of the whole sequence, then every rank's local Q attends to it in one
+ * pass, with an optional document mask (documents packed into one sequence do not
+ * see each other) -- the mask the page gives as the reason to gather instead of
+ * ringing.
+ *   q [b, S, Hq, d], k / v [b, S, Hkv, d]: bf16, rank-major (as for
+ *   cp_ring_attn_fwd); k and v contiguous.  o [b, S, Hq, d] bf16 and lse
+ *   [b, Hq, S, 1] fp32 come out rank-major.
+ *   doc_starts: HOST array of n_docs first positions (original order), strictly
+ *   increasing, doc_starts[0] = 0, all < S; n_docs = 1 means no document mask.
+ *   Key t is visible to query p iff pos_k(t) <= pos_q(p) (causal) and both lie in
+ *   the same document; n_docs > 1 requires causal = 1.
+ *   workspace: at least cp_allgather_workspace_bytes(...) bytes, 256-byte aligned
+ *   (the gathered K and V and the document table); kept alive by the caller until
+ *   the work on `stream` has finished.
+ * The result equals the ring's when n_docs = 1 (same FLOPs, one step). */
+cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q,
+                                const cp_tensor *k, const cp_tensor *v, const int64_t *doc_starts,
+                                int32_t n_docs, float softmax_scale, cp_tensor *o, cp_tensor *lse,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes cp_allgather_attn_fwd needs (0 for invalid arguments). */
+size_t cp_allgather_workspace_bytes(int32_t N, int32_t dtype, int64_t b, int64_t S, int64_t Hkv,
+                                    int64_t d, int32_t n_docs);
 
 /* Ring attention backward over N virtual ranks on one GPU (section 分块注意力,
  * paragraph on the backward pass; section Ring Attention for the schedule).
