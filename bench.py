@@ -5,8 +5,9 @@
 
 One step = one cp_ring_attn_fwd over the whole workload (all N virtual ranks, all
 ring steps), inputs already permuted to rank-major order and resident in HBM.
-The line also carries the standalone merge bandwidth and the backward
-(cp_ring_attn_bwd) of the same workload, each timed on its own.
+The line also carries the standalone merge bandwidth, the backward
+(cp_ring_attn_bwd) of the same workload and the All-Gather forward with a document
+mask (cp_allgather_attn_fwd) on its 8-document variant, each timed on its own.
 L2 is flushed (a 256 MiB write) before every timed step; each step is timed with
 CUDA events on the launching stream.  With --gpus N > 1 (torchrun) every rank
 runs its own instance of the workload (weak scaling, no collective on the data
@@ -197,7 +198,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=W.BENCH_WORKLOAD, choices=sorted(W.BY_NAME))
+    ap.add_argument("--workload", default=W.BENCH_WORKLOAD,
+                    choices=sorted(n for n, x in W.BY_NAME.items() if x.n_docs == 1))
     ap.add_argument("--mode", default="fused", choices=["fused", "stepwise"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -348,6 +350,50 @@ def main():
     if w.dtype == "bf16" and w.d == 128 and rank == 0:
         backward = bwd_leg()
 
+    # All-Gather CP with a document mask (cp_allgather_attn_fwd: K and V gathered
+    # into original order by two permute launches, then one document-masked pass),
+    # on the 8-document variant of the 8B workload; effective FLOPs count only the
+    # pairs the causal document mask leaves visible
+    def allgather_leg():
+        wd = W.BY_NAME["llama3_8b_s8k_zigzag4_docs8"]
+        docs = wd.doc_starts()
+        qa, ka, va = (cp.layout_permute(t.to(dev), wd.layout, wd.N) for t in W.make_inputs(wd))
+        oa = torch.empty_like(qa)
+        la = torch.empty((wd.b, wd.hq, wd.S), dtype=torch.float32, device=dev)
+        wsa = torch.empty(cp.allgather_workspace_bytes(wd.N, 0, wd.b, wd.S, wd.hkv, wd.d, len(docs)),
+                          dtype=torch.uint8, device=dev)
+
+        def astep():
+            cp.allgather_attn_fwd(qa, ka, va, wd.layout, wd.N, wd.causal, docs, wd.scale, oa, la, wsa)
+
+        for _ in range(3):
+            astep()
+        ms = []
+        for _ in range(max(3, min(args.steps, 10))):
+            flush.zero_()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            astep()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            ms.append(a0.elapsed_time(a1))
+        cp.stream_check()
+        t = statistics.mean(ms)
+        tf = wd.effective_flops() / (t * 1e-3) / 1e12
+        del qa, ka, va, oa, la, wsa
+        torch.cuda.empty_cache()
+        return {"metric": "all-gather CP fwd TFLOP/s (causal document mask, effective FLOPs)", "workload": wd.name,
+                "n_docs": len(docs), "value": tf, "unit": "TFLOP/s", "ms_per_step": t, "steps": len(ms),
+                "launches_per_step": 3,
+                "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (document variant)", "achieved": tf,
+                             "peak": peak_tf, "unit": "TFLOP/s", "frac": tf / peak_tf,
+                             "peak_source": peak_src + " bf16 burst",
+                             "timed": "whole call: K and V gather + document-masked attention", "traffic": None}}
+
+    allgather = None
+    if w.dtype == "bf16" and w.d == 128 and rank == 0:
+        allgather = allgather_leg()
+
     # end to end through the public API, every step: pinned host -> device copy of
     # q/k/v, permute to rank-major order, ring attention, unpermute, device -> host
     # copy of o and lse.  Consecutive steps are pipelined on three streams (copy-in,
@@ -428,6 +474,7 @@ def main():
                          "traffic": profiled_traffic() if w.name == W.BENCH_WORKLOAD else None},
             "merge": merge,
             "backward": backward,
+            "allgather": allgather,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e_ms / e_steps, "pipelined": "copy-in / compute / copy-out on 3 streams"},

@@ -239,3 +239,30 @@ def test_ring_bwd_argument_errors_are_synchronous(cp):
     assert call(dk_=_ct(cp, [1, 256, 4, 128])) == 3        # dk shaped like q
     assert call(lse_=_ct(cp, [1, 4, 255, 1], dtype=1)) == 3
     assert cp.lib().cp_ring_bwd_workspace_bytes(1, 3, 0, 1, 256, 4, 128) == 0  # S % N
+
+
+def test_allgather_argument_errors_are_synchronous(cp):
+    q = _ct(cp, [1, 256, 4, 128])
+    k = _ct(cp, [1, 256, 2, 128])
+    o = _ct(cp, [1, 256, 4, 128])
+    lse = _ct(cp, [1, 4, 256, 1], dtype=1)
+    f = cp.lib().cp_allgather_attn_fwd
+    need = cp.lib().cp_allgather_workspace_bytes(2, 0, 1, 256, 2, 128, 3)
+    assert need >= 2 * 256 * 2 * 128 * 2
+
+    def call(docs, layout=1, N=2, causal=1, q_=q, k_=k, ws=0x100000, wsb=None):
+        arr = (ctypes.c_int64 * len(docs))(*docs)
+        return f(layout, N, causal, ctypes.byref(q_), ctypes.byref(k_), ctypes.byref(k_), arr, len(docs),
+                 ctypes.c_float(0.088), ctypes.byref(o), ctypes.byref(lse), ctypes.c_void_p(ws),
+                 need if wsb is None else wsb, None)
+
+    assert call([1, 10]) == 1                    # first document must start at 0
+    assert call([0, 10, 10]) == 1                # strictly increasing
+    assert call([0, 256]) == 1                   # below S
+    assert call([0, 100], causal=0) == 2         # document mask needs the causal mask
+    assert call([0, 100], N=3) == 3              # S % 2N
+    assert call([0, 100], wsb=64) == 1           # workspace too small
+    assert call([0, 100], ws=0x100040) == 1      # workspace alignment
+    qf, kf = _ct(cp, [1, 256, 4, 128], dtype=1), _ct(cp, [1, 256, 2, 128], dtype=1)
+    assert call([0], q_=qf, k_=kf) == 2          # bf16 only
+    assert cp.lib().cp_allgather_workspace_bytes(2, 0, 1, 256, 2, 128, 0) == 0
