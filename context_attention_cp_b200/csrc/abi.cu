@@ -635,10 +635,38 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
     p.n_qt = n_qt;
     p.doc_starts = n_docs > 1 ? docs_dev : nullptr;
     p.n_docs = n_docs > 1 ? n_docs : 0;
-    const std::vector<uint32_t> &ord = ring_order(layout, N, S, causal, rows);
-    if ((int64_t)ord.size() <= kMaxOrder) {
-        p.order_len = (int)ord.size();
-        std::copy(ord.begin(), ord.end(), p.order);
+    // work order, heaviest (rank, row group) first: the key tiles each 128-row query
+    // tile of the group walks, from the document start of its first row to its last
+    // row (the document mask's bounds on the gathered block)
+    {
+        std::vector<std::pair<int64_t, uint32_t>> work;
+        const int n_groups = (int)((c + rows - 1) / rows);
+        auto doc_start = [&](int64_t pos) {
+            int64_t ds = 0;
+            for (int32_t i2 = 0; i2 < n_docs && doc_starts[i2] <= pos; ++i2) ds = doc_starts[i2];
+            return ds;
+        };
+        for (int i2 = 0; i2 < N; ++i2) {
+            const Range qr = layout_range(layout, N, S, i2);
+            for (int g = 0; g < n_groups; ++g) {
+                int64_t tiles = 0;
+                for (int64_t q_lo = (int64_t)g * rows; q_lo < std::min<int64_t>(c, (int64_t)(g + 1) * rows); q_lo += 128) {
+                    const int64_t q_hi = std::min<int64_t>(q_lo + 127, c - 1);
+                    const int64_t first = range_pos(qr, q_lo), last = range_pos(qr, q_hi);
+                    const int64_t lo = causal ? doc_start(first) : 0, hi = causal ? last : S - 1;
+                    tiles += hi / 128 - lo / 128 + 1;
+                }
+                work.push_back({tiles, ((uint32_t)i2 << 16) | (uint32_t)g});
+            }
+        }
+        std::stable_sort(work.begin(), work.end(),
+                         [](const std::pair<int64_t, uint32_t> &x, const std::pair<int64_t, uint32_t> &y) {
+                             return x.first > y.first;
+                         });
+        if ((int64_t)work.size() <= kMaxOrder) {
+            p.order_len = (int)work.size();
+            for (size_t e2 = 0; e2 < work.size(); ++e2) p.order[e2] = work[e2].second;
+        }
     }
     fill_inputs(p, q, &kg, &vg);
     fill_outputs(p, EPI_STORE, o, lse);
