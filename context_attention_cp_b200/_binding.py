@@ -42,6 +42,9 @@ _SIGNATURES = {
     "cp_allgather_attn_fwd": (_i32, [_i32, _i32, _i32, _T, _T, _T, ctypes.POINTER(ctypes.c_int64), _i32, _f32, _T, _T,
                                      _vp, _sz, _vp]),
     "cp_allgather_workspace_bytes": (_sz, [_i32, _i32, _i64, _i64, _i64, _i64, _i32]),
+    "cp_ulysses_all_to_all": (_i32, [_i32, _i32, _T, _T, _vp]),
+    "cp_ulysses_attn_fwd": (_i32, [_i32, _i32, _T, _T, _T, _f32, _T, _T, _vp, _sz, _vp]),
+    "cp_ulysses_workspace_bytes": (_sz, [_i32, _i32, _i64, _i64, _i64, _i64, _i64]),
     "cp_layout_permute": (_i32, [_i32, _i32, _i32, _T, _T, _i32, _vp]),
     "cp_layout_range": (_i32, [_i32, _i32, _i64, _i32, _R]),
     "cp_tile_classes": (_i32, [_R, _i64, _R, _i64, _i32, _i32, _i32, ctypes.POINTER(ctypes.c_int8)]),
@@ -234,6 +237,42 @@ def allgather_attn_fwd(q, k, v, layout, N, causal, doc_starts=None, scale=None, 
     _check(lib().cp_allgather_attn_fwd(LAYOUTS[layout], N, int(bool(causal)), _ref(tq), _ref(tk), _ref(tv), arr,
                                        len(docs), float(scale), _ref(to), _ref(tl),
                                        ctypes.c_void_p(workspace.data_ptr()), need, _stream()))
+    return o, lse
+
+
+def ulysses_all_to_all(x, P, inverse=False, out=None):
+    """Sequence-sharded [b, S, H, d] -> head-sharded [P*b, S, H/P, d] (inverse: back)."""
+    import torch
+    x = x.contiguous()
+    if inverse:
+        Pb, S, hp, d = x.shape
+        out = torch.empty((Pb // P, S, hp * P, d), dtype=x.dtype, device=x.device) if out is None else out
+        _check(lib().cp_ulysses_all_to_all(P, 1, _ref(_tensor(out)), _ref(_tensor(x)), _stream()))
+    else:
+        b, S, H, d = x.shape
+        out = torch.empty((P * b, S, H // P, d), dtype=x.dtype, device=x.device) if out is None else out
+        _check(lib().cp_ulysses_all_to_all(P, 0, _ref(_tensor(x)), _ref(_tensor(out)), _stream()))
+    return out
+
+
+def ulysses_workspace_bytes(P, dtype_code, b, S, Hq, Hkv, d):
+    return lib().cp_ulysses_workspace_bytes(P, dtype_code, b, S, Hq, Hkv, d)
+
+
+def ulysses_attn_fwd(q, k, v, P, causal, scale=None, o=None, lse=None, workspace=None):
+    """Ulysses attention over P virtual ranks; q/k/v/o in original order."""
+    import torch
+    b, S, Hq, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((b, Hq, S), dtype=torch.float32, device=q.device) if lse is None else lse
+    need = ulysses_workspace_bytes(P, _dtype_code(q), b, S, Hq, k.shape[2], d)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ts = [_tensor(t) for t in (q, k, v, o, lse)]
+    _check(lib().cp_ulysses_attn_fwd(P, int(bool(causal)), _ref(ts[0]), _ref(ts[1]), _ref(ts[2]), float(scale),
+                                     _ref(ts[3]), _ref(ts[4]), ctypes.c_void_p(workspace.data_ptr()), need, _stream()))
     return o, lse
 
 

@@ -15,6 +15,7 @@
 #include "../../include/cpattn.h"
 #include "bwd.h"
 #include "kernels.h"
+#include "ulysses.h"
 
 using namespace cpattn;
 
@@ -529,6 +530,107 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
         if (r > 0 && (s = cp_lse_merge(&o_acc, lse, &o_b, &lse_b, r == N - 1 ? o : nullptr, stream)) != CP_OK)
             return s;
     }
+    return CP_OK;
+}
+
+cp_status cp_ulysses_all_to_all(int32_t P, int32_t direction, const cp_tensor *x_seq, cp_tensor *y_head, void *stream)
+{
+    g_last_error[0] = 0;
+    cp_status s;
+    if ((s = check_tensor(x_seq, "x_seq")) != CP_OK || (s = check_tensor(y_head, "y_head")) != CP_OK) return s;
+    if (direction != 0 && direction != 1) return fail(CP_ERR_INVALID_ARG, "direction must be 0 or 1");
+    if (P < 1) return fail(CP_ERR_INVALID_ARG, "P must be >= 1");
+    if (x_seq->dtype != y_head->dtype) return fail(CP_ERR_INVALID_ARG, "x_seq and y_head differ in dtype");
+    const int64_t b = x_seq->shape[0], S = x_seq->shape[1], H = x_seq->shape[2], d = x_seq->shape[3];
+    if (H % P || S % P) return fail(CP_ERR_SHAPE, "P must divide the heads (%lld) and the sequence (%lld)",
+                                    (long long)H, (long long)S);
+    if (y_head->shape[0] != P * b || y_head->shape[1] != S || y_head->shape[2] != H / P || y_head->shape[3] != d)
+        return fail(CP_ERR_SHAPE, "y_head must be [P*b, S, H/P, d]");
+    for (const cp_tensor *t : {x_seq, static_cast<const cp_tensor *>(y_head)}) {
+        int64_t expect = 1;
+        for (int i = 3; i >= 0; --i) {
+            if (t->shape[i] > 1 && t->stride[i] != expect) return fail(CP_ERR_INVALID_ARG, "tensors must be contiguous");
+            expect *= t->shape[i];
+        }
+    }
+    const int64_t bytes = b * S * H * d * elem_size(x_seq->dtype);
+    const char *a = static_cast<const char *>(x_seq->data), *bp = static_cast<const char *>(y_head->data);
+    if (bytes && a < bp + bytes && bp < a + bytes) return fail(CP_ERR_INVALID_ARG, "x_seq and y_head overlap");
+    ShardParams sp{P, b, S, (H / P) * d * elem_size(x_seq->dtype), direction, direction ? y_head->data : x_seq->data,
+                   direction ? const_cast<void *>(x_seq->data) : y_head->data};
+    cudaError_t e = launch_shard_transpose(sp, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "all-to-all launch");
+    return CP_OK;
+}
+
+size_t cp_ulysses_workspace_bytes(int32_t P, int32_t dtype, int64_t b, int64_t S, int64_t Hq, int64_t Hkv, int64_t d)
+{
+    if (P < 1 || b < 0 || S < 0 || Hq < 0 || Hkv < 0 || d < 0 || !elem_size(dtype)) return 0;
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    const int64_t es = elem_size(dtype);
+    // head-sharded q, k, v, o and lse
+    return (size_t)(2 * up(b * S * Hq * d * es) + 2 * up(b * S * Hkv * d * es) + up(b * Hq * S * 4));
+}
+
+cp_status cp_ulysses_attn_fwd(int32_t P, int32_t causal, const cp_tensor *q, const cp_tensor *k, const cp_tensor *v,
+                              float softmax_scale, cp_tensor *o, cp_tensor *lse, void *workspace,
+                              size_t workspace_bytes, void *stream)
+{
+    g_last_error[0] = 0;
+    cp_status s;
+    if (causal != 0 && causal != 1) return fail(CP_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if ((s = check_tensor(q, "q")) != CP_OK || (s = check_tensor(k, "k")) != CP_OK ||
+        (s = check_tensor(v, "v")) != CP_OK)
+        return s;
+    if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    const int64_t b = q->shape[0], S = q->shape[1], Hq = q->shape[2], Hkv = k->shape[2], d = q->shape[3];
+    if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
+    if (P < 1) return fail(CP_ERR_INVALID_ARG, "P must be >= 1");
+    if (Hq % P || Hkv % P)
+        return fail(CP_ERR_SHAPE, "P must divide the query heads (%lld) and the kv heads (%lld)", (long long)Hq,
+                    (long long)Hkv);
+    if (S % P) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of P = %d", (long long)S, P);
+    if (S % 4) return fail(CP_ERR_SHAPE, "S must be a multiple of 4");
+    if (S >= ((int64_t)1 << 30)) return fail(CP_ERR_SHAPE, "sequence too long (S must be below 2^30)");
+    if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;
+    if (o->dtype != q->dtype) return fail(CP_ERR_INVALID_ARG, "o must have q's dtype");
+    for (const cp_tensor *t : {q, k, v, static_cast<const cp_tensor *>(o)}) {
+        int64_t expect = 1;
+        for (int i = 3; i >= 0; --i) {
+            if (t->shape[i] > 1 && t->stride[i] != expect) return fail(CP_ERR_INVALID_ARG, "tensors must be contiguous");
+            expect *= t->shape[i];
+        }
+    }
+    if (!(lse->stride[2] == 1 && lse->stride[1] == S && (b <= 1 || lse->stride[0] == Hq * S)))
+        return fail(CP_ERR_INVALID_ARG, "lse must be contiguous");
+    const size_t need = cp_ulysses_workspace_bytes(P, q->dtype, b, S, Hq, Hkv, d);
+    if (!workspace || workspace_bytes < need) return fail(CP_ERR_INVALID_ARG, "workspace of %zu bytes needed", need);
+    if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (b == 0 || S == 0) return CP_OK;
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    const int64_t es = elem_size(q->dtype), hp = Hq / P, hkp = Hkv / P;
+    char *ws = static_cast<char *>(workspace);
+    const int64_t qb = up(b * S * Hq * d * es), kb = up(b * S * Hkv * d * es);
+    cp_tensor qh{ws, q->dtype, 0, {P * b, S, hp, d}, {S * hp * d, hp * d, d, 1}};
+    cp_tensor kh{ws + qb, q->dtype, 0, {P * b, S, hkp, d}, {S * hkp * d, hkp * d, d, 1}};
+    cp_tensor vh{ws + qb + kb, q->dtype, 0, {P * b, S, hkp, d}, {S * hkp * d, hkp * d, d, 1}};
+    cp_tensor oh{ws + qb + 2 * kb, q->dtype, 0, {P * b, S, hp, d}, {S * hp * d, hp * d, d, 1}};
+    cp_tensor lh{ws + 2 * qb + 2 * kb, CP_FP32, 0, {P * b, hp, S, 1}, {hp * S, S, 1, 1}};
+    // all-to-all: sequence-sharded -> head-sharded
+    if ((s = cp_ulysses_all_to_all(P, 0, q, &qh, stream)) != CP_OK) return s;
+    if ((s = cp_ulysses_all_to_all(P, 0, k, &kh, stream)) != CP_OK) return s;
+    if ((s = cp_ulysses_all_to_all(P, 0, v, &vh, stream)) != CP_OK) return s;
+    // every rank's heads over the whole sequence: one launch, the ranks as batch entries
+    if ((s = cp_ring_attn_fwd(CP_LAYOUT_CONTIGUOUS, 1, causal, &qh, &kh, &vh, softmax_scale, &oh, &lh, CP_RING_FUSED,
+                              nullptr, 0, stream)) != CP_OK)
+        return s;
+    // and back: o [P*b, S, hp, d] -> [b, S, Hq, d]; lse [P][b][hp * S] -> [b][P][hp * S]
+    if ((s = cp_ulysses_all_to_all(P, 1, o, &oh, stream)) != CP_OK) return s;
+    ShardParams sp{P, b, 1, hp * S * 4, 1, lh.data, lse->data};
+    cudaError_t e = launch_shard_transpose(sp, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "all-to-all launch");
     return CP_OK;
 }
 

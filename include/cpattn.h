@@ -17,7 +17,9 @@
  *   - section 分块注意力, paragraph on the backward pass: with the global lse any
  *     key block alone gives its exact share of dq, dk, dv;
  *   - section All-Gather 式 CP: K/V gathered once per layer, any attention mask
- *     (documents) applied in one local pass.
+ *     (documents) applied in one local pass;
+ *   - section DeepSpeed-Ulysses: an all-to-all switches the sharded dimension from
+ *     the sequence to the heads, attention runs per head group, and back.
  *
  * Conventions shared by every entry point
  *   - Token tensors are [b, s, H, d] with d contiguous; lse tensors are
@@ -169,6 +171,36 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
 /* Workspace bytes cp_allgather_attn_fwd needs (0 for invalid arguments). */
 size_t cp_allgather_workspace_bytes(int32_t N, int32_t dtype, int64_t b, int64_t S, int64_t Hkv,
                                     int64_t d, int32_t n_docs);
+
+/* DeepSpeed-Ulysses all-to-all on one GPU (section DeepSpeed-Ulysses): the
+ * exchange that moves block (s_i, h_j) -- the i-th sequence shard's j-th head
+ * group -- from rank i to rank j.
+ *   x_seq [b, S, H, d]: sequence-sharded, rank i holds tokens [i S/P, (i+1) S/P)
+ *     (the original order, contiguous split);
+ *   y_head [P * b, S, H/P, d]: head-sharded, entry r * b + bb holds every token of
+ *     heads [r H/P, (r+1) H/P) of batch bb.
+ *   direction 0 writes y_head from x_seq, 1 writes x_seq from y_head.  Both
+ *   contiguous, same dtype, not overlapping; P must divide H and S.  Bit-exact. */
+cp_status cp_ulysses_all_to_all(int32_t P, int32_t direction, const cp_tensor *x_seq, cp_tensor *y_head,
+                                void *stream);
+
+/* Ulysses attention over P virtual ranks on one GPU: all-to-all of q, k, v to the
+ * head-sharded layout, each rank's n_h/P heads attend over the whole sequence (one
+ * launch of the tensor-core kernel, bf16, or the FFMA kernel, fp32), all-to-all of o
+ * and lse back.
+ *   q [b, S, Hq, d], k / v [b, S, Hkv, d], o [b, S, Hq, d] in original order (the
+ *   sequence-sharded layout), contiguous; lse [b, Hq, S, 1] fp32 contiguous.
+ *   P must divide Hq and Hkv (a rank owns whole KV groups; with GQA, P <= Hkv) and
+ *   S; S % 4 == 0.  causal: the causal mask on positions.
+ *   workspace: cp_ulysses_workspace_bytes(...) bytes, 256-byte aligned (the
+ *   head-sharded q, k, v, o, lse). */
+cp_status cp_ulysses_attn_fwd(int32_t P, int32_t causal, const cp_tensor *q, const cp_tensor *k,
+                              const cp_tensor *v, float softmax_scale, cp_tensor *o, cp_tensor *lse,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes cp_ulysses_attn_fwd needs (0 for invalid arguments). */
+size_t cp_ulysses_workspace_bytes(int32_t P, int32_t dtype, int64_t b, int64_t S, int64_t Hq,
+                                  int64_t Hkv, int64_t d);
 
 /* Ring attention backward over N virtual ranks on one GPU (section 分块注意力,
  * paragraph on the backward pass; section Ring Attention for the schedule).

@@ -331,3 +331,50 @@ def allgather_attention_steps(q, k, v, layout_name, n_ranks, causal, scale, doc_
         o[:, pos] = oi
         lse[:, :, pos] = li
     return o, lse
+
+
+def ulysses_all_to_all(x, n_ranks, inverse=False):
+    """The Ulysses exchange written out (section DeepSpeed-Ulysses): block (s_i, h_j)
+    moves from rank i to rank j.  Forward: x [b, S, H, d] with rank i holding tokens
+    [i S/P, (i+1) S/P) -> [P, b, S, H/P, d] (rank j: all tokens, heads
+    [j H/P, (j+1) H/P)).  Inverse: the reverse.  A pure index map in numpy."""
+    P = n_ranks
+    if not inverse:
+        b, S, H, d = x.shape
+        c, hp = S // P, H // P
+        out = np.empty((P, b, S, hp, d), dtype=x.dtype)
+        for i in range(P):          # source rank: sequence shard i
+            for j in range(P):      # destination rank: head group j
+                out[j, :, i * c:(i + 1) * c] = x[:, i * c:(i + 1) * c, j * hp:(j + 1) * hp]
+        return out
+    P_, b, S, hp, d = x.shape
+    c = S // P
+    out = np.empty((b, S, hp * P, d), dtype=x.dtype)
+    for j in range(P):
+        for i in range(P):
+            out[:, i * c:(i + 1) * c, j * hp:(j + 1) * hp] = x[j, :, i * c:(i + 1) * c]
+    return out
+
+
+def ulysses_attention(q, k, v, n_ranks, causal, scale, nthreads=None):
+    """Reference result of Ulysses attention: heads are independent, so the exchange
+    around per-head-group attention reproduces plain attention exactly."""
+    if q.shape[2] % n_ranks or k.shape[2] % n_ranks or q.shape[1] % n_ranks:
+        raise ValueError("P must divide the heads and the sequence")
+    return attention(q, k, v, causal, scale, nthreads=nthreads)
+
+
+def ulysses_attention_steps(q, k, v, n_ranks, causal, scale, nthreads=None):
+    """The four steps of the page: all-to-all of q, k, v, each rank's attention over
+    its n_h/P heads and the whole sequence, all-to-all of o (and lse) back."""
+    P = n_ranks
+    qh, kh, vh = (ulysses_all_to_all(_f64(t), P) for t in (q, k, v))
+    b, S, Hq, d = _f64(q).shape
+    hp = Hq // P
+    oh = np.empty_like(qh)
+    lh = np.empty((P, b, hp, S))
+    for j in range(P):
+        oh[j], lh[j] = attention(qh[j], kh[j], vh[j], causal, scale, nthreads=nthreads)
+    o = ulysses_all_to_all(oh, P, inverse=True)
+    lse = np.concatenate([lh[j] for j in range(P)], axis=1)  # [b, Hq, S], head group j at j*hp
+    return o, lse

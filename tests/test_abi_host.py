@@ -266,3 +266,25 @@ def test_allgather_argument_errors_are_synchronous(cp):
     qf, kf = _ct(cp, [1, 256, 4, 128], dtype=1), _ct(cp, [1, 256, 2, 128], dtype=1)
     assert call([0], q_=qf, k_=kf) == 2          # bf16 only
     assert cp.lib().cp_allgather_workspace_bytes(2, 0, 1, 256, 2, 128, 0) == 0
+
+
+def test_ulysses_argument_errors_are_synchronous(cp):
+    x = _ct(cp, [1, 64, 8, 128])
+    y = _ct(cp, [4, 64, 2, 128], data=0x200000)
+    g = cp.lib().cp_ulysses_all_to_all
+    assert g(4, 2, ctypes.byref(x), ctypes.byref(y), None) == 1      # direction
+    assert g(3, 0, ctypes.byref(x), ctypes.byref(y), None) == 3      # P divides H
+    y_bad = _ct(cp, [4, 64, 4, 128], data=0x200000)
+    assert g(4, 0, ctypes.byref(x), ctypes.byref(y_bad), None) == 3  # y shape
+    y_ov = _ct(cp, [4, 64, 2, 128], data=0x10000)
+    assert g(4, 0, ctypes.byref(x), ctypes.byref(y_ov), None) == 1   # overlap
+    q = _ct(cp, [1, 64, 8, 128])
+    k = _ct(cp, [1, 64, 2, 128])
+    o = _ct(cp, [1, 64, 8, 128])
+    lse = _ct(cp, [1, 8, 64, 1], dtype=1)
+    f = cp.lib().cp_ulysses_attn_fwd
+    assert f(4, 1, ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.c_float(0.1), ctypes.byref(o),
+             ctypes.byref(lse), ctypes.c_void_p(0x100000), 1 << 30, None) == 3   # P must divide Hkv = 2
+    assert f(2, 1, ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.c_float(0.1), ctypes.byref(o),
+             ctypes.byref(lse), ctypes.c_void_p(0x100000), 16, None) == 1        # workspace too small
+    assert cp.lib().cp_ulysses_workspace_bytes(0, 0, 1, 64, 8, 2, 128) == 0
