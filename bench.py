@@ -7,7 +7,8 @@ One step = one cp_ring_attn_fwd over the whole workload (all N virtual ranks, al
 ring steps), inputs already permuted to rank-major order and resident in HBM.
 The line also carries the standalone merge bandwidth, the backward
 (cp_ring_attn_bwd) of the same workload and the All-Gather forward with a document
-mask (cp_allgather_attn_fwd) on its 8-document variant, each timed on its own.
+mask (cp_allgather_attn_fwd) on its 8-document variant and Ulysses
+(cp_ulysses_attn_fwd, P = 4) on its shape, each timed on its own.
 L2 is flushed (a 256 MiB write) before every timed step; each step is timed with
 CUDA events on the launching stream.  With --gpus N > 1 (torchrun) every rank
 runs its own instance of the workload (weak scaling, no collective on the data
@@ -394,6 +395,44 @@ def main():
     if w.dtype == "bf16" and w.d == 128 and rank == 0:
         allgather = allgather_leg()
 
+    # Ulysses over P = 4 virtual ranks on this workload's shape (original order):
+    # all-to-all of q, k, v, one attention launch over the head groups, all-to-all
+    # of o and lse back (5 + 1 launches)
+    def ulysses_leg(P=4):
+        qu, ku, vu = (t.to(dev) for t in W.make_inputs(w))
+        ou = torch.empty_like(qu)
+        lu = torch.empty((w.b, w.hq, w.S), dtype=torch.float32, device=dev)
+        wsu = torch.empty(cp.ulysses_workspace_bytes(P, 0, w.b, w.S, w.hq, w.hkv, w.d), dtype=torch.uint8, device=dev)
+
+        def ustep():
+            cp.ulysses_attn_fwd(qu, ku, vu, P, w.causal, w.scale, ou, lu, wsu)
+
+        for _ in range(3):
+            ustep()
+        ms = []
+        for _ in range(max(3, min(args.steps, 10))):
+            flush.zero_()
+            u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            u0.record(stream)
+            ustep()
+            u1.record(stream)
+            torch.cuda.synchronize()
+            ms.append(u0.elapsed_time(u1))
+        cp.stream_check()
+        t = statistics.mean(ms)
+        tf = flops / (t * 1e-3) / 1e12
+        del qu, ku, vu, ou, lu, wsu
+        torch.cuda.empty_cache()
+        return {"metric": "Ulysses fwd TFLOP/s (causal, effective FLOPs)", "P": P, "value": tf, "unit": "TFLOP/s",
+                "ms_per_step": t, "steps": len(ms), "launches_per_step": 6,
+                "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": tf, "peak": peak_tf,
+                             "unit": "TFLOP/s", "frac": tf / peak_tf, "peak_source": peak_src + " bf16 burst",
+                             "timed": "whole call: 5 all-to-all launches + attention", "traffic": None}}
+
+    ulysses = None
+    if w.dtype == "bf16" and w.hkv % 4 == 0 and w.hq % 4 == 0 and w.S % 4 == 0 and rank == 0:
+        ulysses = ulysses_leg()
+
     # end to end through the public API, every step: pinned host -> device copy of
     # q/k/v, permute to rank-major order, ring attention, unpermute, device -> host
     # copy of o and lse.  Consecutive steps are pipelined on three streams (copy-in,
@@ -475,6 +514,7 @@ def main():
             "merge": merge,
             "backward": backward,
             "allgather": allgather,
+            "ulysses": ulysses,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e_ms / e_steps, "pipelined": "copy-in / compute / copy-out on 3 streams"},
