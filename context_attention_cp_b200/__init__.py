@@ -11,6 +11,7 @@ Entry points mirror include/cpattn.h:
   ring_attn_bwd(q, k, v, o, lse, do, layout, N, causal, scale) -> (dq, dk, dv)
   allgather_attn_fwd(q, k, v, layout, N, causal, doc_starts=None, scale=None)
   ulysses_attn_fwd(q, k, v, P, causal, scale=None); ulysses_all_to_all(x, P, inverse=False)
+  ulysses_attn_bwd(q, k, v, o, lse, do, P, causal, scale=None) -> (dq, dk, dv)
   layout_permute(x, layout, N, seq_axis=1, inverse=False, out=None)
   layout_range(layout, N, S, rank) -> (nseg, start, len, stride)
   tile_classes(q_range, q_len, kv_range, kv_len, causal, tile_q, tile_k)
@@ -22,6 +23,6 @@ from ._binding import (  # noqa: F401
     CPError, LAYOUTS, MODES, allgather_attn_fwd, allgather_workspace_bytes, block_attn_fwd, layout_permute,
     layout_range, lib, lib_path,
     lse_merge, ring_attn_bwd, ring_attn_fwd, ring_attn_fwd_static_scratch, ring_bwd_workspace_bytes,
-    ring_workspace_bytes, selftest_wait_timeout, stream_check, tile_classes, ulysses_all_to_all, ulysses_attn_fwd,
+    ring_workspace_bytes, selftest_wait_timeout, stream_check, tile_classes, ulysses_all_to_all, ulysses_attn_bwd, ulysses_attn_fwd,
     ulysses_workspace_bytes,
 )

@@ -634,6 +634,93 @@ cp_status cp_ulysses_attn_fwd(int32_t P, int32_t causal, const cp_tensor *q, con
     return CP_OK;
 }
 
+size_t cp_ulysses_bwd_workspace_bytes(int32_t P, int32_t dtype, int64_t b, int64_t S, int64_t Hq, int64_t Hkv,
+                                      int64_t d)
+{
+    if (P < 1 || b < 0 || S < 0 || Hq < 0 || Hkv < 0 || d < 0 || !elem_size(dtype) || Hq % P) return 0;
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    const int64_t es = elem_size(dtype);
+    const int64_t qb = up(b * S * Hq * d * es), kb = up(b * S * Hkv * d * es), lb = up(b * Hq * S * 4);
+    // head-sharded q, o, dout, dq; k, v, dk, dv; lse; then the ring backward's own
+    return (size_t)(4 * qb + 4 * kb + lb) +
+           cp_ring_bwd_workspace_bytes(CP_LAYOUT_CONTIGUOUS, 1, dtype, P * b, S, Hq / P, d);
+}
+
+cp_status cp_ulysses_attn_bwd(int32_t P, int32_t causal, const cp_tensor *q, const cp_tensor *k, const cp_tensor *v,
+                              const cp_tensor *o, const cp_tensor *lse, const cp_tensor *dout, float softmax_scale,
+                              cp_tensor *dq, cp_tensor *dk, cp_tensor *dv, void *workspace, size_t workspace_bytes,
+                              void *stream)
+{
+    g_last_error[0] = 0;
+    cp_status s;
+    if (causal != 0 && causal != 1) return fail(CP_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if ((s = check_tensor(q, "q")) != CP_OK || (s = check_tensor(k, "k")) != CP_OK ||
+        (s = check_tensor(v, "v")) != CP_OK || (s = check_tensor(dout, "dout")) != CP_OK ||
+        (s = check_tensor(dq, "dq")) != CP_OK || (s = check_tensor(dk, "dk")) != CP_OK ||
+        (s = check_tensor(dv, "dv")) != CP_OK)
+        return s;
+    if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
+    if (q->dtype != CP_BF16) return fail(CP_ERR_UNSUPPORTED, "the backward takes bf16 tensors");
+    if (q->shape[3] != 128) return fail(CP_ERR_UNSUPPORTED, "the backward supports d = 128");
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    const int64_t b = q->shape[0], S = q->shape[1], Hq = q->shape[2], Hkv = k->shape[2], d = q->shape[3];
+    if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
+    if (P < 1) return fail(CP_ERR_INVALID_ARG, "P must be >= 1");
+    if (Hq % P || Hkv % P)
+        return fail(CP_ERR_SHAPE, "P must divide the query heads (%lld) and the kv heads (%lld)", (long long)Hq,
+                    (long long)Hkv);
+    if (S % P) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of P = %d", (long long)S, P);
+    if (S % 4) return fail(CP_ERR_SHAPE, "S must be a multiple of 4");
+    if (S >= ((int64_t)1 << 30)) return fail(CP_ERR_SHAPE, "sequence too long (S must be below 2^30)");
+    if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;
+    if (o->dtype != CP_BF16) return fail(CP_ERR_INVALID_ARG, "o must be bf16");
+    const cp_tensor *like_q[3] = {o, dout, dq};
+    for (const cp_tensor *t : like_q)
+        if (!same_shape(t, q) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "o, dout and dq must be bf16 shaped like q");
+    const cp_tensor *like_k[2] = {dk, dv};
+    for (const cp_tensor *t : like_k)
+        if (!same_shape(t, k) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "dk and dv must be bf16 shaped like k");
+    if (!(lse->stride[2] == 1 && lse->stride[1] == S && (b <= 1 || lse->stride[0] == Hq * S)))
+        return fail(CP_ERR_INVALID_ARG, "lse must be contiguous");
+    const size_t need = cp_ulysses_bwd_workspace_bytes(P, q->dtype, b, S, Hq, Hkv, d);
+    if (!workspace || workspace_bytes < need) return fail(CP_ERR_INVALID_ARG, "workspace of %zu bytes needed", need);
+    if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (b == 0 || S == 0) return CP_OK;
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    const int64_t hp = Hq / P, hkp = Hkv / P;
+    const int64_t qb = up(b * S * Hq * d * 2), kb = up(b * S * Hkv * d * 2), lb = up(b * Hq * S * 4);
+    char *ws = static_cast<char *>(workspace);
+    auto qt = [&](int i) {
+        return cp_tensor{ws + i * qb, CP_BF16, 0, {P * b, S, hp, d}, {S * hp * d, hp * d, d, 1}};
+    };
+    auto kt = [&](int i) {
+        return cp_tensor{ws + 4 * qb + i * kb, CP_BF16, 0, {P * b, S, hkp, d}, {S * hkp * d, hkp * d, d, 1}};
+    };
+    cp_tensor qh = qt(0), oh = qt(1), doh = qt(2), dqh = qt(3);
+    cp_tensor kh = kt(0), vh = kt(1), dkh = kt(2), dvh = kt(3);
+    cp_tensor lh{ws + 4 * qb + 4 * kb, CP_FP32, 0, {P * b, hp, S, 1}, {hp * S, S, 1, 1}};
+    char *ws_ring = ws + 4 * qb + 4 * kb + lb;
+    const size_t ring_need = cp_ring_bwd_workspace_bytes(CP_LAYOUT_CONTIGUOUS, 1, CP_BF16, P * b, S, hp, d);
+    // exchange in: q, k, v, o, dout and lse to the head-sharded layout
+    const cp_tensor *ins[5] = {q, k, v, o, dout};
+    cp_tensor *outs[5] = {&qh, &kh, &vh, &oh, &doh};
+    for (int i = 0; i < 5; ++i)
+        if ((s = cp_ulysses_all_to_all(P, 0, ins[i], outs[i], stream)) != CP_OK) return s;
+    ShardParams sp{P, b, 1, hp * S * 4, 0, lse->data, lh.data};
+    cudaError_t e = launch_shard_transpose(sp, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "all-to-all launch");
+    // each rank's head group over the whole sequence
+    if ((s = cp_ring_attn_bwd(CP_LAYOUT_CONTIGUOUS, 1, causal, &qh, &kh, &vh, &oh, &lh, &doh, softmax_scale, &dqh, &dkh,
+                              &dvh, ws_ring, ring_need, stream)) != CP_OK)
+        return s;
+    // exchange out: the gradients back to the sequence-sharded layout
+    if ((s = cp_ulysses_all_to_all(P, 1, dq, &dqh, stream)) != CP_OK) return s;
+    if ((s = cp_ulysses_all_to_all(P, 1, dk, &dkh, stream)) != CP_OK) return s;
+    if ((s = cp_ulysses_all_to_all(P, 1, dv, &dvh, stream)) != CP_OK) return s;
+    return CP_OK;
+}
+
 size_t cp_allgather_workspace_bytes(int32_t N, int32_t dtype, int64_t b, int64_t S, int64_t Hkv, int64_t d,
                                     int32_t n_docs)
 {

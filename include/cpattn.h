@@ -202,6 +202,22 @@ cp_status cp_ulysses_attn_fwd(int32_t P, int32_t causal, const cp_tensor *q, con
 size_t cp_ulysses_workspace_bytes(int32_t P, int32_t dtype, int64_t b, int64_t S, int64_t Hq,
                                   int64_t Hkv, int64_t d);
 
+/* Ulysses backward: the exchange of q, k, v, o, dout and lse to the head-sharded
+ * layout, the ring backward with N = 1 over every rank's head group (the same
+ * kernels as cp_ring_attn_bwd), and the exchange of dq, dk, dv back.
+ *   Tensors in original order as for cp_ulysses_attn_fwd (o and lse its results);
+ *   dq [b, S, Hq, d], dk / dv [b, S, Hkv, d] bf16 outputs; all contiguous.
+ *   Requires bf16, d = 128 and the conditions of cp_ulysses_attn_fwd.
+ *   workspace: cp_ulysses_bwd_workspace_bytes(...) bytes, 256-byte aligned. */
+cp_status cp_ulysses_attn_bwd(int32_t P, int32_t causal, const cp_tensor *q, const cp_tensor *k,
+                              const cp_tensor *v, const cp_tensor *o, const cp_tensor *lse,
+                              const cp_tensor *dout, float softmax_scale, cp_tensor *dq, cp_tensor *dk,
+                              cp_tensor *dv, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes cp_ulysses_attn_bwd needs (0 for invalid arguments). */
+size_t cp_ulysses_bwd_workspace_bytes(int32_t P, int32_t dtype, int64_t b, int64_t S, int64_t Hq,
+                                      int64_t Hkv, int64_t d);
+
 /* Ring attention backward over N virtual ranks on one GPU (section 分块注意力,
  * paragraph on the backward pass; section Ring Attention for the schedule).
  * With the forward's GLOBAL o and lse of every query row and the output gradient

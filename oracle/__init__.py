@@ -378,3 +378,21 @@ def ulysses_attention_steps(q, k, v, n_ranks, causal, scale, nthreads=None):
     o = ulysses_all_to_all(oh, P, inverse=True)
     lse = np.concatenate([lh[j] for j in range(P)], axis=1)  # [b, Hq, S], head group j at j*hp
     return o, lse
+
+
+def ulysses_attention_bwd(q, k, v, do, n_ranks, causal, scale, nthreads=None):
+    """Reference gradients of Ulysses attention: the plain definition (heads are
+    independent).  Returns (dq, dk, dv) in original order."""
+    if q.shape[2] % n_ranks or k.shape[2] % n_ranks or q.shape[1] % n_ranks:
+        raise ValueError("P must divide the heads and the sequence")
+    dq, dk, dv, _, _ = attention_bwd(q, k, v, do, causal, scale, nthreads=nthreads)
+    return dq, dk, dv
+
+
+def ulysses_attention_bwd_steps(q, k, v, do, n_ranks, causal, scale, nthreads=None):
+    """Exchange of q, k, v, dO; each rank's head-group gradients over the whole
+    sequence; exchange of dq, dk, dv back."""
+    P = n_ranks
+    qh, kh, vh, doh = (ulysses_all_to_all(_f64(t), P) for t in (q, k, v, do))
+    g = [attention_bwd(qh[j], kh[j], vh[j], doh[j], causal, scale, nthreads=nthreads)[:3] for j in range(P)]
+    return tuple(ulysses_all_to_all(np.stack([g[j][n] for j in range(P)]), P, inverse=True) for n in range(3))

@@ -79,3 +79,19 @@ def test_full_size_ulysses_sampled(cp):
     tol_o, tol_l = TOL["bf16"]
     assert_close_lse(got_l, rl, tol_l)
     assert_close_o(got_o, ro, tol_o)
+
+
+@pytest.mark.parametrize("P,b,S,hq,hkv,causal", [(4, 1, 1024, 8, 4, True), (2, 2, 600, 4, 2, True),
+                                                 (8, 1, 512, 8, 8, False), (1, 1, 256, 4, 1, True)])
+def test_ulysses_bwd_matches_oracle(cp, P, b, S, hq, hkv, causal):
+    d = 128
+    q, k, v = W.random_qkv(b, S, hq, hkv, d, "bf16", seed=S + 2 * P)
+    do = W.random_do(b, S, hq, d, "bf16", seed=S + 2 * P)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = cp.ulysses_attn_fwd(qd, kd, vd, P, causal)
+    dq, dk, dv = cp.ulysses_attn_bwd(qd, kd, vd, o, lse, dod, P, causal)
+    cp.stream_check()
+    want = oracle.ulysses_attention_bwd(np64(q), np64(k), np64(v), np64(do), P, causal, d ** -0.5)
+    for name, g, w in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
+        err = np.max(np.abs(np64(g) - w))
+        assert err <= 2e-2 * np.max(np.abs(w)), (name, err)

@@ -34,3 +34,14 @@ def test_p_must_divide_heads():
     x = np.zeros((1, 8, 6, 2))
     with pytest.raises(ValueError):
         oracle.ulysses_attention(x, x[:, :, :3], x[:, :, :3], 4, True, 0.5)
+
+
+@pytest.mark.parametrize("P", [1, 2, 4])
+def test_backward_steps_equal_plain_gradients(P):
+    r = np.random.default_rng(10 + P)
+    b, S, hq, hkv, d = 1, 12, 8, 4, 3
+    q, k, v, do = (r.standard_normal(s) for s in ((b, S, hq, d), (b, S, hkv, d), (b, S, hkv, d), (b, S, hq, d)))
+    got = oracle.ulysses_attention_bwd_steps(q, k, v, do, P, True, 0.6)
+    want = oracle.ulysses_attention_bwd(q, k, v, do, P, True, 0.6)
+    for g, w in zip(got, want):
+        assert np.max(np.abs(g - w)) <= 1e-13
