@@ -39,6 +39,9 @@ def _load():
         lib.oracle_lse_merge.restype = None
         lib.oracle_lse_merge.argtypes = [ctypes.c_int64, ctypes.c_int64] + [_F64P] * 6
         _bwd_sigs(lib)
+        lib.oracle_attention_bwd_doc.restype = ctypes.c_int
+        lib.oracle_attention_bwd_doc.argtypes = [_F64P] * 4 + [_I64P] * 2 + [ctypes.c_int64] * 6 + \
+            [ctypes.c_int, _I64P, ctypes.c_int64, ctypes.c_double] + [_F64P] * 3 + [ctypes.c_int]
         lib.oracle_attention_doc.restype = ctypes.c_int
         lib.oracle_attention_doc.argtypes = [_F64P, _F64P, _F64P, _I64P, _I64P] + [ctypes.c_int64] * 6 + \
             [ctypes.c_int, _I64P, ctypes.c_int64, ctypes.c_double, _F64P, _F64P, ctypes.c_int]
@@ -396,3 +399,79 @@ def ulysses_attention_bwd_steps(q, k, v, do, n_ranks, causal, scale, nthreads=No
     qh, kh, vh, doh = (ulysses_all_to_all(_f64(t), P) for t in (q, k, v, do))
     g = [attention_bwd(qh[j], kh[j], vh[j], doh[j], causal, scale, nthreads=nthreads)[:3] for j in range(P)]
     return tuple(ulysses_all_to_all(np.stack([g[j][n] for j in range(P)]), P, inverse=True) for n in range(3))
+
+
+def attention_bwd_doc(q, k, v, do, causal, scale, doc_starts, pos_q=None, pos_k=None, nthreads=None):
+    """Gradients of attention_doc (the document mask of section All-Gather 式 CP).
+    Returns (dq, dk, dv) in float64."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    b, sq, hq, d = q.shape
+    _, sk, hkv, _ = k.shape
+    if do.shape != q.shape or v.shape != k.shape:
+        raise ValueError("shape mismatch")
+    pq, pk = _opt_pos(pos_q, sq, "pos_q"), _opt_pos(pos_k, sk, "pos_k")
+    docs = _docs(doc_starts)
+    dq, dkk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    rc = _load().oracle_attention_bwd_doc(_ptr(q, _F64P), _ptr(k, _F64P), _ptr(v, _F64P), _ptr(do, _F64P),
+                                          _ptr(pq, _I64P), _ptr(pk, _I64P), b, sq, sk, hq, hkv, d, int(bool(causal)),
+                                          _ptr(docs, _I64P), docs.size, float(scale), _ptr(dq, _F64P),
+                                          _ptr(dkk, _F64P), _ptr(dv, _F64P), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_attention_bwd_doc rejected its arguments")
+    return dq, dkk, dv
+
+
+def allgather_attention_bwd(q, k, v, do, layout_name, n_ranks, causal, scale, doc_starts, nthreads=None):
+    """Reference gradients of All-Gather CP (gathered K/V, document mask; the dK, dV
+    reduce-scatter sums every rank's share): the definition over the whole sequence.
+    Returns (dq, dk, dv) in ORIGINAL token order."""
+    layout.tokens_per_rank(layout_name, n_ranks, q.shape[1])
+    return attention_bwd_doc(q, k, v, do, causal, scale, doc_starts, nthreads=nthreads)
+
+
+def allgather_attention_bwd_steps(q, k, v, do, layout_name, n_ranks, causal, scale, doc_starts, nthreads=None):
+    """The All-Gather backward written out: each rank's queries against the gathered
+    K/V give its dq and a full-length share of dK, dV; the reduce-scatter sums the
+    shares and hands each rank its own block (returned here in original order)."""
+    S = q.shape[1]
+    layout.tokens_per_rank(layout_name, n_ranks, S)
+    q64, do64 = _f64(q), _f64(do)
+    o, lse = attention_doc(q, k, v, causal, scale, doc_starts, nthreads=nthreads)
+    delta = np.einsum("bshd,bshd->bhs", do64, o)
+    dq = np.zeros(q64.shape)
+    dk_sum = np.zeros(_f64(k).shape)
+    dv_sum = np.zeros(_f64(v).shape)
+    docs = _docs(doc_starts)
+    for i in range(n_ranks):
+        pos = np.asarray(layout.rank_positions(layout_name, n_ranks, S, i), dtype=np.int64)
+        # the rank's own share, with the global statistics of its rows: dq rows and a
+        # full-length dK, dV contribution (keys of other documents masked)
+        q_i, do_i = q64[:, pos], do64[:, pos]
+        share = _share_doc(q_i, k, v, do_i, causal, scale, docs, pos, lse[:, :, pos], delta[:, :, pos], nthreads)
+        dq[:, pos] = share[0]
+        dk_sum += share[1]
+        dv_sum += share[2]
+    return dq, dk_sum, dv_sum
+
+
+def _share_doc(q_i, k, v, do_i, causal, scale, docs, pos, lse_i, delta_i, nthreads):
+    """One rank's share under the document mask, as a block with global statistics:
+    documents cut the keys into independent groups, so the share is summed document
+    by document with oracle_attention_bwd's block mode."""
+    S = k.shape[1]
+    bounds = list(docs) + [S]
+    dq = np.zeros(q_i.shape)
+    dk = np.zeros(_f64(k).shape)
+    dv = np.zeros(_f64(v).shape)
+    for a, e in zip(bounds[:-1], bounds[1:]):
+        rows = np.nonzero((pos >= a) & (pos < e))[0]
+        if rows.size == 0:
+            continue
+        keys = np.arange(a, e)
+        gq, gk, gv, _, _ = attention_bwd(q_i[:, rows], _f64(k)[:, keys], _f64(v)[:, keys], do_i[:, rows], causal,
+                                         scale, pos_q=pos[rows], pos_k=keys, lse=lse_i[:, :, rows],
+                                         delta=delta_i[:, :, rows], nthreads=nthreads)
+        dq[:, rows] = gq
+        dk[:, keys] += gk
+        dv[:, keys] += gv
+    return dq, dk, dv

@@ -303,6 +303,8 @@ typedef struct {
                                         >= min_pos are needed, without it only heads whose
                                         entry is not INT64_MAX; NULL = every row */
     const int64_t *sel;              /* [n][3] selected rows, or NULL = every row */
+    const int64_t *docs;             /* document starts (NULL = one document) */
+    int64_t n_docs;
     double *dq;                      /* query pass: [b, sq, hq, d] or [n][d]; NULL = stats only */
     double *dk, *dv;                 /* key pass: [b, sk, hkv, d] or [n][d] */
     int64_t begin, end;
@@ -354,7 +356,7 @@ static void *bwd_query_worker(void *arg)
             D = j->delta_in[srow];
         } else {
             lse = attend_row(qi, pq, krow_of(j, j->k, bb, 0, hk), krow_of(j, j->v, bb, 0, hk), j->pos_k,
-                             j->sk, j->hkv * d, d, j->causal, NULL, 0, j->scale, x, o);
+                             j->sk, j->hkv * d, d, j->causal, j->docs, j->n_docs, j->scale, x, o);
             D = dotd(doi, o, d);
         }
         if (j->lse) { j->lse[srow] = lse; j->delta[srow] = D; }
@@ -362,9 +364,11 @@ static void *bwd_query_worker(void *arg)
         double *dqi = j->sel ? j->dq + r * d : j->dq + ((bb * j->sq + i) * j->hq + h) * d;
         for (int64_t e = 0; e < d; ++e) dqi[e] = 0.0;
         if (lse == -INFINITY) continue;
+        const int64_t dq_doc = j->docs ? doc_of(j->docs, j->n_docs, pq) : 0;
         for (int64_t t = 0; t < j->sk; ++t) {
             const int64_t pk = j->pos_k ? j->pos_k[t] : t;
             if (j->causal && pk > pq) continue;
+            if (j->docs && doc_of(j->docs, j->n_docs, pk) != dq_doc) continue;
             const double *kt = krow_of(j, j->k, bb, t, hk);
             const double *vt = krow_of(j, j->v, bb, t, hk);
             const double p = exp(j->scale * dotd(qi, kt, d) - lse);
@@ -394,12 +398,14 @@ static void *bwd_key_worker(void *arg)
         double *dvt = j->sel ? j->dv + r * d : j->dv + ((bb * j->sk + t) * j->hkv + hk) * d;
         for (int64_t e = 0; e < d; ++e) { dkt[e] = 0.0; dvt[e] = 0.0; }
         const int64_t pk = j->pos_k ? j->pos_k[t] : t;
+        const int64_t dk_doc = j->docs ? doc_of(j->docs, j->n_docs, pk) : 0;
         const double *kt = krow_of(j, j->k, bb, t, hk);
         const double *vt = krow_of(j, j->v, bb, t, hk);
         for (int64_t h = hk * g; h < (hk + 1) * g; ++h) {
             for (int64_t i = 0; i < j->sq; ++i) {
                 const int64_t pq = j->pos_q ? j->pos_q[i] : i;
                 if (j->causal && pk > pq) continue;
+                if (j->docs && doc_of(j->docs, j->n_docs, pq) != dk_doc) continue;
                 const int64_t srow = (bb * j->hq + h) * j->sq + i;
                 const double lse = j->lse[srow], D = j->delta[srow];
                 if (lse == -INFINITY) continue;
@@ -452,11 +458,12 @@ static int bwd_dims_ok(int64_t b, int64_t sq, int64_t sk, int64_t hq, int64_t hk
  *   dq [b, sq, hq, d], dk, dv [b, sk, hkv, d] are overwritten;
  *   lse_out, delta_out [b, hq, sq] (may be NULL) receive the statistics used.
  * Returns 0, or -1 on bad sizes / allocation or thread failure. */
-int oracle_attention_bwd(const double *q, const double *k, const double *v, const double *dout,
-                         const int64_t *pos_q, const int64_t *pos_k, int64_t b, int64_t sq, int64_t sk,
-                         int64_t hq, int64_t hkv, int64_t d, int causal, double scale,
-                         const double *lse_in, const double *delta_in, double *dq, double *dk,
-                         double *dv, double *lse_out, double *delta_out, int nthreads)
+static int attention_bwd_impl(const double *q, const double *k, const double *v, const double *dout,
+                              const int64_t *pos_q, const int64_t *pos_k, int64_t b, int64_t sq, int64_t sk,
+                              int64_t hq, int64_t hkv, int64_t d, int causal, const int64_t *docs,
+                              int64_t n_docs, double scale, const double *lse_in, const double *delta_in,
+                              double *dq, double *dk, double *dv, double *lse_out, double *delta_out,
+                              int nthreads)
 {
     if (!bwd_dims_ok(b, sq, sk, hq, hkv, d) || (!lse_in) != (!delta_in)) return -1;
     const int64_t nstat = b * hq * sq;
@@ -472,11 +479,36 @@ int oracle_attention_bwd(const double *q, const double *k, const double *v, cons
     j.q = q; j.k = k; j.v = v; j.dout = dout; j.pos_q = pos_q; j.pos_k = pos_k;
     j.b = b; j.sq = sq; j.sk = sk; j.hq = hq; j.hkv = hkv; j.d = d;
     j.causal = causal; j.scale = scale; j.lse_in = lse_in; j.delta_in = delta_in;
+    j.docs = docs; j.n_docs = n_docs;
     j.lse = lse; j.delta = delta; j.dq = dq; j.dk = dk; j.dv = dv;
     int rc = run_bwd_jobs(&j, nstat, nthreads, bwd_query_worker);
     if (rc == 0) rc = run_bwd_jobs(&j, b * hkv * sk, nthreads, bwd_key_worker);
     free(own);
     return rc;
+}
+
+int oracle_attention_bwd(const double *q, const double *k, const double *v, const double *dout,
+                         const int64_t *pos_q, const int64_t *pos_k, int64_t b, int64_t sq, int64_t sk,
+                         int64_t hq, int64_t hkv, int64_t d, int causal, double scale,
+                         const double *lse_in, const double *delta_in, double *dq, double *dk,
+                         double *dv, double *lse_out, double *delta_out, int nthreads)
+{
+    return attention_bwd_impl(q, k, v, dout, pos_q, pos_k, b, sq, sk, hq, hkv, d, causal, NULL, 0, scale,
+                              lse_in, delta_in, dq, dk, dv, lse_out, delta_out, nthreads);
+}
+
+/* oracle_attention_bwd with the document mask of oracle_attention_doc (section
+ * All-Gather 式 CP): a key of another document than the query contributes nothing. */
+int oracle_attention_bwd_doc(const double *q, const double *k, const double *v, const double *dout,
+                             const int64_t *pos_q, const int64_t *pos_k, int64_t b, int64_t sq, int64_t sk,
+                             int64_t hq, int64_t hkv, int64_t d, int causal, const int64_t *doc_starts,
+                             int64_t n_docs, double scale, double *dq, double *dk, double *dv, int nthreads)
+{
+    if (n_docs < 1 || !doc_starts || doc_starts[0] != 0) return -1;
+    for (int64_t i = 1; i < n_docs; ++i)
+        if (doc_starts[i] <= doc_starts[i - 1]) return -1;
+    return attention_bwd_impl(q, k, v, dout, pos_q, pos_k, b, sq, sk, hq, hkv, d, causal, doc_starts, n_docs,
+                              scale, NULL, NULL, dq, dk, dv, NULL, NULL, nthreads);
 }
 
 /* Gradients at selected rows only (for sampled checks at full size).

@@ -101,3 +101,58 @@ def test_doc_starts_are_checked():
     for bad in ([1, 4], [0, 4, 4], [0, 5, 3]):
         with pytest.raises(ValueError):
             oracle.attention_doc(q, k, v, True, 0.5, bad)
+
+
+# ------------------------------------------------------------------ backward
+
+def _loss_doc(q, k, v, do, causal, scale, starts, pos):
+    o, _ = oracle.attention_doc(q, k, v, causal, scale, starts, pos_q=pos, pos_k=pos, nthreads=1)
+    return float(np.sum(o * do))
+
+
+def test_doc_gradients_match_finite_differences():
+    b, S, hq, hkv, d = 1, 9, 2, 1, 3
+    q, k, v = _inputs(12, b, S, hq, hkv, d)
+    do = np.random.default_rng(13).standard_normal(q.shape)
+    pos = np.array(L.rank_positions("zigzag", 3, 18, 1) + L.rank_positions("zigzag", 3, 18, 2)[:3])
+    starts = [0, 4, 11, 15]
+    dq, dk, dv = oracle.attention_bwd_doc(q, k, v, do, True, 0.9, starts, pos_q=pos, pos_k=pos)
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = x[idx]
+            x[idx] = old + 1e-5
+            fp = _loss_doc(q, k, v, do, True, 0.9, starts, pos)
+            x[idx] = old - 1e-5
+            fm = _loss_doc(q, k, v, do, True, 0.9, starts, pos)
+            x[idx] = old
+            num[idx] = (fp - fm) / 2e-5
+        assert np.max(np.abs(num - g)) <= 1e-7
+
+
+def test_doc_gradients_are_per_document():
+    b, S, hq, hkv, d = 2, 30, 4, 2, 4
+    q, k, v = _inputs(14, b, S, hq, hkv, d)
+    do = np.random.default_rng(15).standard_normal(q.shape)
+    starts = [0, 9, 10, 22]
+    dq, dk, dv = oracle.attention_bwd_doc(q, k, v, do, True, 0.5, starts)
+    bounds = starts + [S]
+    for a, e in zip(bounds[:-1], bounds[1:]):
+        gq, gk, gv, _, _ = oracle.attention_bwd(q[:, a:e], k[:, a:e], v[:, a:e], do[:, a:e], True, 0.5)
+        assert np.max(np.abs(dq[:, a:e] - gq)) <= 1e-13
+        assert np.max(np.abs(dk[:, a:e] - gk)) <= 1e-13
+        assert np.max(np.abs(dv[:, a:e] - gv)) <= 1e-13
+
+
+@pytest.mark.parametrize("layout", L.LAYOUTS)
+def test_allgather_backward_steps_equal_whole(layout):
+    S, N = 32, 4
+    q, k, v = _inputs(16 + len(layout), 1, S, 4, 2, 3)
+    do = np.random.default_rng(17).standard_normal(q.shape)
+    starts = [0, 5, 6, 19, 31]
+    got = oracle.allgather_attention_bwd_steps(q, k, v, do, layout, N, True, 0.4, starts)
+    want = oracle.allgather_attention_bwd(q, k, v, do, layout, N, True, 0.4, starts)
+    for g, w in zip(got, want):
+        assert np.max(np.abs(g - w)) <= 1e-12
