@@ -10,6 +10,7 @@ Entry points mirror include/cpattn.h:
   ring_attn_fwd(q, k, v, layout, N, causal, scale, o=None, lse=None, mode="fused")
   ring_attn_bwd(q, k, v, o, lse, do, layout, N, causal, scale) -> (dq, dk, dv)
   allgather_attn_fwd(q, k, v, layout, N, causal, doc_starts=None, scale=None)
+  allgather_attn_bwd(q, k, v, o, lse, do, layout, N, causal, doc_starts=None) -> (dq, dk, dv)
   ulysses_attn_fwd(q, k, v, P, causal, scale=None); ulysses_all_to_all(x, P, inverse=False)
   ulysses_attn_bwd(q, k, v, o, lse, do, P, causal, scale=None) -> (dq, dk, dv)
   layout_permute(x, layout, N, seq_axis=1, inverse=False, out=None)
@@ -20,7 +21,7 @@ Tensors are torch tensors on the current CUDA device; token tensors are
 [b, s, H, d] with d contiguous, lse tensors [b, H, s] fp32.
 """
 from ._binding import (  # noqa: F401
-    CPError, LAYOUTS, MODES, allgather_attn_fwd, allgather_workspace_bytes, block_attn_fwd, layout_permute,
+    CPError, LAYOUTS, MODES, allgather_attn_bwd, allgather_attn_fwd, allgather_workspace_bytes, block_attn_fwd, layout_permute,
     layout_range, lib, lib_path,
     lse_merge, ring_attn_bwd, ring_attn_fwd, ring_attn_fwd_static_scratch, ring_bwd_workspace_bytes,
     ring_workspace_bytes, selftest_wait_timeout, stream_check, tile_classes, ulysses_all_to_all, ulysses_attn_bwd, ulysses_attn_fwd,

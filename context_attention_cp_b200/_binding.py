@@ -43,6 +43,9 @@ _SIGNATURES = {
                                      _vp, _sz, _vp]),
     "cp_allgather_workspace_bytes": (_sz, [_i32, _i32, _i64, _i64, _i64, _i64, _i32]),
     "cp_ulysses_all_to_all": (_i32, [_i32, _i32, _T, _T, _vp]),
+    "cp_allgather_attn_bwd": (_i32, [_i32, _i32, _i32, _T, _T, _T, _T, _T, _T, ctypes.POINTER(ctypes.c_int64), _i32,
+                                     _f32, _T, _T, _T, _vp, _sz, _vp]),
+    "cp_allgather_bwd_workspace_bytes": (_sz, [_i32, _i32, _i64, _i64, _i64, _i64, _i64, _i32]),
     "cp_ulysses_attn_fwd": (_i32, [_i32, _i32, _T, _T, _T, _f32, _T, _T, _vp, _sz, _vp]),
     "cp_ulysses_workspace_bytes": (_sz, [_i32, _i32, _i64, _i64, _i64, _i64, _i64]),
     "cp_ulysses_attn_bwd": (_i32, [_i32, _i32, _T, _T, _T, _T, _T, _T, _f32, _T, _T, _T, _vp, _sz, _vp]),
@@ -240,6 +243,28 @@ def allgather_attn_fwd(q, k, v, layout, N, causal, doc_starts=None, scale=None, 
                                        len(docs), float(scale), _ref(to), _ref(tl),
                                        ctypes.c_void_p(workspace.data_ptr()), need, _stream()))
     return o, lse
+
+
+def allgather_attn_bwd(q, k, v, o, lse, do, layout, N, causal, doc_starts=None, scale=None, dq=None, dk=None, dv=None,
+                       workspace=None):
+    """Gradients of All-Gather CP with the document mask; rank-major tensors."""
+    import torch
+    b, S, Hq, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    docs = [0] if doc_starts is None else [int(x) for x in doc_starts]
+    arr = (ctypes.c_int64 * len(docs))(*docs)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = lib().cp_allgather_bwd_workspace_bytes(N, _dtype_code(q), b, S, Hq, k.shape[2], d, len(docs))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ts = [_tensor(t) for t in (q, k, v, o, lse, do, dq, dk, dv)]
+    _check(lib().cp_allgather_attn_bwd(LAYOUTS[layout], N, int(bool(causal)), *[_ref(t) for t in ts[:6]], arr,
+                                       len(docs), float(scale), *[_ref(t) for t in ts[6:]],
+                                       ctypes.c_void_p(workspace.data_ptr()), need, _stream()))
+    return dq, dk, dv
 
 
 def ulysses_all_to_all(x, P, inverse=False, out=None):

@@ -634,6 +634,154 @@ cp_status cp_ulysses_attn_fwd(int32_t P, int32_t causal, const cp_tensor *q, con
     return CP_OK;
 }
 
+size_t cp_allgather_bwd_workspace_bytes(int32_t N, int32_t dtype, int64_t b, int64_t S, int64_t Hq, int64_t Hkv,
+                                        int64_t d, int32_t n_docs)
+{
+    if (N < 1 || b < 0 || S < 0 || Hq < 0 || Hkv < 0 || d < 0 || n_docs < 1 || !elem_size(dtype) || S % N) return 0;
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    const int64_t kb = up(b * S * Hkv * d * elem_size(dtype));
+    // gathered K, V, dK, dV; the document table; the statistics and the dQ accumulator
+    return (size_t)(4 * kb + up((int64_t)n_docs * 4)) +
+           cp_ring_bwd_workspace_bytes(CP_LAYOUT_CONTIGUOUS, N, dtype, b, S, Hq, d);
+}
+
+cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q, const cp_tensor *k,
+                                const cp_tensor *v, const cp_tensor *o, const cp_tensor *lse, const cp_tensor *dout,
+                                const int64_t *doc_starts, int32_t n_docs, float softmax_scale, cp_tensor *dq,
+                                cp_tensor *dk, cp_tensor *dv, void *workspace, size_t workspace_bytes, void *stream)
+{
+    g_last_error[0] = 0;
+    cp_status s;
+    if (layout < 0 || layout > 2) return fail(CP_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (causal != 0 && causal != 1) return fail(CP_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if ((s = check_tensor(q, "q")) != CP_OK || (s = check_tensor(k, "k")) != CP_OK ||
+        (s = check_tensor(v, "v")) != CP_OK || (s = check_tensor(dout, "dout")) != CP_OK ||
+        (s = check_tensor(dq, "dq")) != CP_OK || (s = check_tensor(dk, "dk")) != CP_OK ||
+        (s = check_tensor(dv, "dv")) != CP_OK)
+        return s;
+    if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
+    if (q->dtype != CP_BF16) return fail(CP_ERR_UNSUPPORTED, "the backward takes bf16 tensors");
+    if (q->shape[3] != 128) return fail(CP_ERR_UNSUPPORTED, "the backward supports d = 128");
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    const int64_t S = q->shape[1];
+    if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
+    if (N < 1 || N > 4096) return fail(CP_ERR_INVALID_ARG, "N must be in [1, 4096]");
+    if (S >= ((int64_t)1 << 30)) return fail(CP_ERR_SHAPE, "sequence too long (S must be below 2^30)");
+    if (S % N) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of N = %d", (long long)S, N);
+    if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N)) return fail(CP_ERR_SHAPE, "zig-zag needs S to be a multiple of 2N");
+    if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;
+    if (o->dtype != CP_BF16) return fail(CP_ERR_INVALID_ARG, "o must be bf16");
+    const cp_tensor *like_q[2] = {dout, dq};
+    for (const cp_tensor *t : like_q) {
+        if (!same_shape(t, q) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "dout and dq must be bf16 shaped like q");
+        if ((s = check_rows16(t, t == dq ? "dq" : "dout")) != CP_OK) return s;
+    }
+    const cp_tensor *like_k[4] = {k, v, dk, dv};
+    for (const cp_tensor *t : like_k) {
+        if (!same_shape(t, k) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "dk and dv must be bf16 shaped like k");
+        int64_t expect = 1;
+        for (int i = 3; i >= 0; --i) {
+            if (t->shape[i] > 1 && t->stride[i] != expect)
+                return fail(CP_ERR_INVALID_ARG, "k, v, dk and dv must be contiguous");
+            expect *= t->shape[i];
+        }
+    }
+    if (n_docs < 1 || !doc_starts) return fail(CP_ERR_INVALID_ARG, "doc_starts must hold at least one start");
+    if (doc_starts[0] != 0) return fail(CP_ERR_INVALID_ARG, "the first document must start at 0");
+    for (int32_t i = 1; i < n_docs; ++i)
+        if (doc_starts[i] <= doc_starts[i - 1] || doc_starts[i] >= S)
+            return fail(CP_ERR_INVALID_ARG, "document starts must increase and stay below S");
+    if (n_docs > 1 && !causal) return fail(CP_ERR_UNSUPPORTED, "the document mask is defined with the causal mask");
+    const int64_t b = q->shape[0], Hq = q->shape[2], Hkv = k->shape[2], d = q->shape[3];
+    const int64_t c = S / N;
+    const int64_t n_kt = (S + kBwdKeyTile - 1) / kBwdKeyTile;
+    if (n_kt > 65535) return fail(CP_ERR_SHAPE, "too many key tiles");
+    const size_t need = cp_allgather_bwd_workspace_bytes(N, q->dtype, b, S, Hq, Hkv, d, n_docs);
+    if (!workspace || workspace_bytes < need) return fail(CP_ERR_INVALID_ARG, "workspace of %zu bytes needed", need);
+    if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (b == 0 || S == 0) return CP_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    char *ws = static_cast<char *>(workspace);
+    const int64_t kb = up(b * S * Hkv * d * 2);
+    auto kv_t = [&](int i) {
+        return cp_tensor{ws + i * kb, CP_BF16, 0, {b, S, Hkv, d}, {S * Hkv * d, Hkv * d, d, 1}};
+    };
+    cp_tensor kg = kv_t(0), vg = kv_t(1), dkg = kv_t(2), dvg = kv_t(3);
+    int *docs_dev = reinterpret_cast<int *>(ws + 4 * kb);
+    char *ws_q = ws + 4 * kb + up((int64_t)n_docs * 4);
+    // the gather of K and V into original order (as in the forward)
+    if ((s = cp_layout_permute(layout, N, 1, &kg, const_cast<cp_tensor *>(k), 1, stream)) != CP_OK) return s;
+    if ((s = cp_layout_permute(layout, N, 1, &vg, const_cast<cp_tensor *>(v), 1, stream)) != CP_OK) return s;
+    std::vector<int32_t> docs_h((size_t)n_docs);
+    for (int32_t i = 0; i < n_docs; ++i) docs_h[i] = (int32_t)doc_starts[i];
+    cudaError_t e = cudaMemcpyAsync(docs_dev, docs_h.data(), sizeof(int32_t) * (size_t)n_docs, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "document table copy");
+
+    thread_local BwdParams p;
+    std::memset(&p, 0, sizeof p);
+    p.b = (int)b;
+    p.hq = (int)Hq;
+    p.hkv = (int)Hkv;
+    p.group = p.hq / p.hkv;
+    p.d = (int)d;
+    p.q_len = (int)c;
+    p.kv_len = (int)S;
+    p.n_ranks = N;
+    p.step_begin = 0;
+    p.step_end = N;  // key block 0 meets query rank r at step r
+    p.causal = causal;
+    p.use_layout = 1;
+    p.layout = layout;
+    p.seq_len = S;
+    p.kv_explicit = 1;
+    p.kv_range = Range{0, 0, S, 0, 1};
+    p.n_kv_blocks = 1;
+    p.q_row_step = c;
+    p.kv_row_step = 0;
+    p.scale = softmax_scale;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.q = q->data; p.k = kg.data; p.v = vg.data; p.o = o->data; p.dout = dout->data;
+    p.q_sb = q->stride[0]; p.q_ss = q->stride[1]; p.q_sh = q->stride[2];
+    p.k_sb = kg.stride[0]; p.k_ss = kg.stride[1]; p.k_sh = kg.stride[2];
+    p.v_sb = vg.stride[0]; p.v_ss = vg.stride[1]; p.v_sh = vg.stride[2];
+    p.o_sb = o->stride[0]; p.o_ss = o->stride[1]; p.o_sh = o->stride[2];
+    p.do_sb = dout->stride[0]; p.do_ss = dout->stride[1]; p.do_sh = dout->stride[2];
+    p.lse = static_cast<const float *>(lse->data);
+    p.lse_sb = lse->stride[0]; p.lse_sh = lse->stride[1]; p.lse_ss = lse->stride[2];
+    const BwdWorkspace w = bwd_workspace(N, b, S, Hq, d);
+    p.stats = reinterpret_cast<float2 *>(ws_q);
+    p.lpad = (int)w.lpad;
+    p.dq_acc = reinterpret_cast<float *>(ws_q + w.stats_bytes);
+    p.dq = dq->data; p.dk = dkg.data; p.dv = dvg.data;
+    p.dq_sb = dq->stride[0]; p.dq_ss = dq->stride[1]; p.dq_sh = dq->stride[2];
+    p.dk_sb = dkg.stride[0]; p.dk_ss = dkg.stride[1]; p.dk_sh = dkg.stride[2];
+    p.dv_sb = dvg.stride[0]; p.dv_ss = dvg.stride[1]; p.dv_sh = dvg.stride[2];
+    p.doc_starts = n_docs > 1 ? docs_dev : nullptr;
+    p.n_docs = n_docs > 1 ? n_docs : 0;
+    int *word = nullptr;
+    status_word(&word);
+    p.status = word;
+    p.n_kt = (int)n_kt;
+    // work order: the key tiles of the gathered block, earliest (most queries) first
+    if (n_kt <= kMaxOrder) {
+        p.order_len = (int)n_kt;
+        for (int kt = 0; kt < (int)n_kt; ++kt) p.order[kt] = (uint32_t)kt;
+    }
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    p.head_major = n_kt >= (int64_t)sms;
+    e = launch_attn_bwd(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    // the reduce-scatter: the summed dK, dV of the gathered block back to each rank
+    if ((s = cp_layout_permute(layout, N, 1, &dkg, dk, 0, stream)) != CP_OK) return s;
+    if ((s = cp_layout_permute(layout, N, 1, &dvg, dv, 0, stream)) != CP_OK) return s;
+    return CP_OK;
+}
+
 size_t cp_ulysses_bwd_workspace_bytes(int32_t P, int32_t dtype, int64_t b, int64_t S, int64_t Hq, int64_t Hkv,
                                       int64_t d)
 {
@@ -958,6 +1106,7 @@ cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     status_word(&word);
     p.status = word;
     p.n_kt = (int)n_kt;
+    p.n_kv_blocks = N;
     const std::vector<uint32_t> &ord = bwd_order(layout, N, S, causal);
     if ((int64_t)ord.size() <= kMaxOrder) {
         p.order_len = (int)ord.size();

@@ -141,6 +141,33 @@ __device__ __forceinline__ bool bar_any(uint32_t id, uint32_t nthreads, bool pre
 
 // Query-tile sequence of one CTA: (query head of the group, ring step, query tile)
 // with the tile seeing at least one key of the CTA's key tile.  Every role walks it.
+// End of the document that holds position pos: the first document start > pos
+// (INT32_MAX past the last document).
+__device__ __forceinline__ int64_t doc_end_of(const int *starts, int n, int64_t pos)
+{
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if ((int64_t)__ldg(starts + mid) <= pos) lo = mid + 1; else hi = mid;
+    }
+    return lo < n ? (int64_t)__ldg(starts + lo) : (int64_t)INT32_MAX;
+}
+
+// First query tile (of BQ rows, q_len rows, ranges q) whose row at offset off
+// (clamped to the block) has a position >= x.
+__device__ __forceinline__ int first_qtile_from(const Range &q, int q_len, int off, int64_t x)
+{
+    const int n_qt = (q_len + BQ - 1) / BQ;
+    int lo = 0, hi = n_qt;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        int64_t r = (int64_t)mid * BQ + off;
+        if (r > q_len - 1) r = q_len - 1;
+        if (range_pos(q, r) < x) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+}
+
 // With the head-major grid, the steps of a head start at a rotation that depends on
 // the key tile, so CTAs of one key block reduce into different dQ rows at any one
 // time.
@@ -149,6 +176,8 @@ struct QSeq {
     int j, k_lo, h0, n_qt, nsteps, rot;
     Range kr;
     int hi, sc, r, qt, qt_full, i, h;
+    int qt_stop, qt_fend;          // query tiles [qt_stop, ...) see nothing; [qt_full, qt_fend) are full
+    int64_t de_first, de_last;     // document ends of the tile's first / last key (document mask)
     Range qr;
 
     __device__ void init(const BwdParams &pp, int jj, int kt, const Range &k, int hq0)
@@ -166,6 +195,14 @@ struct QSeq {
         r = pp.step_begin;
         qt = n_qt - 1;
         qt_full = 0;
+        qt_stop = n_qt;
+        qt_fend = n_qt;
+        de_first = de_last = INT32_MAX;
+        if (pp.n_docs > 0 && pp.kv_len > 0) {
+            const int64_t k_hi = k_lo + BK - 1 < pp.kv_len - 1 ? k_lo + BK - 1 : pp.kv_len - 1;
+            de_first = doc_end_of(pp.doc_starts, pp.n_docs, range_pos(k, (int64_t)k_lo));
+            de_last = doc_end_of(pp.doc_starts, pp.n_docs, range_pos(k, k_hi));
+        }
         i = 0;
         h = hq0;
     }
@@ -173,7 +210,7 @@ struct QSeq {
     {
         if (nsteps <= 0) return false;
         ++qt;
-        while (qt >= n_qt) {
+        while (qt >= qt_stop) {
             if (++sc >= nsteps) {
                 sc = 0;
                 if (++hi >= p->group) return false;
@@ -182,14 +219,28 @@ struct QSeq {
             const int N = p->n_ranks;
             i = (j + r) % N;
             qr = p->use_layout ? layout_range(p->layout, N, p->seq_len, i) : p->q_range;
+            if (p->n_docs > 0 && p->kv_len > 0 && p->q_len > 0 &&
+                range_pos(qr, (int64_t)0) >= de_last) {  // the whole rank lies after the tile's documents
+                qt = n_qt;
+                qt_stop = n_qt;
+                continue;
+            }
             int qb;
             q_tile_bounds<int64_t>(qr, p->q_len, BQ, kr, p->kv_len, k_lo, BK, p->causal != 0, &qb, &qt_full);
+            qt_stop = n_qt;
+            qt_fend = n_qt;
+            if (p->n_docs > 0) {
+                // rows at or past the end of the last key's document see none of the
+                // tile; rows must end before the first key's document ends to see all
+                qt_stop = first_qtile_from(qr, p->q_len, 0, de_last);
+                qt_fend = first_qtile_from(qr, p->q_len, BQ - 1, de_first);
+            }
             qt = qb;
         }
         h = h0 + hi;
         return true;
     }
-    __device__ bool partial() const { return qt < qt_full; }
+    __device__ bool partial() const { return qt < qt_full || qt >= qt_fend; }
     __device__ int q_row() const { return (int)(i * p->q_row_step) + qt * BQ; }
 };
 
@@ -242,7 +293,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // head_major: (batch, kv head) outermost, so the CTAs resident at one time share a
     // few heads' dQ rows and the accumulator they reduce into stays in L2; otherwise
     // the work order outermost (heaviest key tiles of every head first)
-    const int n_items = p.order_len ? p.order_len : p.n_ranks * p.n_kt;
+    const int n_items = p.order_len ? p.order_len : p.n_kv_blocks * p.n_kt;
     const int bkh = p.b * p.hkv;
     const int bh = p.head_major ? (int)(blockIdx.x / n_items) : (int)(blockIdx.x % bkh);
     const int e = p.head_major ? (int)(blockIdx.x % n_items) : (int)(blockIdx.x / bkh);
@@ -257,7 +308,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int hk = bh % p.hkv;
     const int bb = bh / p.hkv;
     const int k_lo = kt * BK;
-    const Range kr = p.use_layout ? layout_range(p.layout, p.n_ranks, p.seq_len, j) : p.kv_range;
+    const Range kr = (p.use_layout && !p.kv_explicit) ? layout_range(p.layout, p.n_ranks, p.seq_len, j) : p.kv_range;
 
     if (tid == 0) {
         mbar_init(bar(C::B_KV), 1);
@@ -455,6 +506,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int key = k_lo + krow;
         const bool key_ok = key < p.kv_len;
         const int64_t pk = range_pos(kr, (int64_t)(key_ok ? key : (p.kv_len > 0 ? p.kv_len - 1 : 0)));
+        const int64_t de_key = p.n_docs > 0 ? doc_end_of(p.doc_starts, p.n_docs, pk) : (int64_t)INT32_MAX;
         const float sl2 = p.scale_log2;
         bool aborted = false;
         int n = 0;
@@ -462,7 +514,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int s = n % NS;
             // columns [0, c_first) of this row are masked (keys past the block end,
             // or queries that precede the key)
-            int c_first = 0;
+            int c_first = 0, c_last = BQ;
             if (seq.partial()) {
                 if (!key_ok) {
                     c_first = BQ;
@@ -479,8 +531,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     c_first = lo;
                 }
+                if (key_ok && p.n_docs > 0 && de_key < (int64_t)INT32_MAX) {
+                    // queries at or past the end of the key's document do not see it
+                    int lo = 0, hi = BQ;
+                    const int64_t row0 = (int64_t)seq.qt * BQ, last = p.q_len - 1;
+                    while (lo < hi) {
+                        const int mid = (lo + hi) >> 1;
+                        const int64_t row = row0 + mid < last ? row0 + mid : last;
+                        if (range_pos(seq.qr, row) < de_key) lo = mid + 1; else hi = mid;
+                    }
+                    c_last = lo;
+                }
             }
             c_first -= half * 32;
+            c_last -= half * 32;
             {
                 const bool okw = mbar_wait(bar(C::B_SF + (n & 1)), (n >> 1) & 1, w) &&
                                  mbar_wait(bar(C::B_QF + s), (n / NS) & 1, w);
@@ -501,8 +565,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), sl2x2,
                                  f2_pack(-st.x, -st.z)),
                           x0, x1);
-                pv[2 * c] = (2 * c < c_first) ? 0.f : ex2_approx(x0);
-                pv[2 * c + 1] = (2 * c + 1 < c_first) ? 0.f : ex2_approx(x1);
+                pv[2 * c] = (2 * c < c_first || 2 * c >= c_last) ? 0.f : ex2_approx(x0);
+                pv[2 * c + 1] = (2 * c + 1 < c_first || 2 * c + 1 >= c_last) ? 0.f : ex2_approx(x1);
             }
             uint32_t pk16[16];
 #pragma unroll
@@ -688,7 +752,7 @@ cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream)
 {
     if (p.d != HD) return cudaErrorInvalidValue;
     const int64_t q_rows = (int64_t)p.n_ranks * p.q_row_step;
-    const int64_t kv_rows = (int64_t)p.n_ranks * p.kv_row_step;
+    const int64_t kv_rows = p.kv_row_step ? (int64_t)p.n_ranks * p.kv_row_step : p.kv_len;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
     CUtensorMap tq, tk, tv, tdo, tdq;
@@ -710,7 +774,7 @@ cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream)
     attn_bwd_pre_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, stream>>>(p, q_rows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int64_t items = (int64_t)(p.order_len ? p.order_len : p.n_ranks * p.n_kt) * p.b * p.hkv;
+    const int64_t items = (int64_t)(p.order_len ? p.order_len : p.n_kv_blocks * p.n_kt) * p.b * p.hkv;
     if (items > 0) {
         attn_bwd_kernel<<<(unsigned)items, NTHREADS, BCfg::SMEM, stream>>>(p, tq, tk, tv, tdo, tdq);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -84,7 +84,15 @@ struct BwdParams {
     void *dq, *dk, *dv;
     int64_t dq_sb, dq_ss, dq_sh, dk_sb, dk_ss, dk_sh, dv_sb, dv_ss, dv_sh;
     int *status;
-    // work order: entry e -> (key rank, key tile) = (order[e] >> 16, order[e] & 0xffff);
+    // All-Gather form: kv_explicit = 1 takes kv_range as the one key block (the
+    // gathered sequence, kv_row_step = 0); n_kv_blocks counts the key blocks (the
+    // ring: n_ranks; the gathered form: 1).  Document mask: doc_starts [n_docs]
+    // device array, sorted, first 0 (n_docs = 0: none); a query sees a key only
+    // inside its own document.
+    int kv_explicit, n_kv_blocks;
+    const int *doc_starts;
+    int n_docs;
+    // work order: entry e -> (key block, key tile) = (order[e] >> 16, order[e] & 0xffff);
     // head_major puts (batch, kv head) outside the order in the grid
     int head_major;
     int n_kt;

@@ -168,6 +168,23 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
                                 int32_t n_docs, float softmax_scale, cp_tensor *o, cp_tensor *lse,
                                 void *workspace, size_t workspace_bytes, void *stream);
 
+/* All-Gather backward (section All-Gather 式 CP: the reduce-scatter of dK, dV in
+ * the backward): K and V gathered again, every rank's queries against the whole
+ * sequence with the same document mask, the summed dK, dV handed back to each
+ * rank's block.  Arguments as cp_allgather_attn_fwd (o and lse its results) plus
+ * dout [b, S, Hq, d]; dq [b, S, Hq, d], dk / dv [b, S, Hkv, d] bf16 outputs, all
+ * rank-major; k, v, dk, dv contiguous.  Requires bf16 and d = 128.
+ *   workspace: cp_allgather_bwd_workspace_bytes(...) bytes, 256-byte aligned. */
+cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q,
+                                const cp_tensor *k, const cp_tensor *v, const cp_tensor *o,
+                                const cp_tensor *lse, const cp_tensor *dout, const int64_t *doc_starts,
+                                int32_t n_docs, float softmax_scale, cp_tensor *dq, cp_tensor *dk,
+                                cp_tensor *dv, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes cp_allgather_attn_bwd needs (0 for invalid arguments). */
+size_t cp_allgather_bwd_workspace_bytes(int32_t N, int32_t dtype, int64_t b, int64_t S, int64_t Hq,
+                                        int64_t Hkv, int64_t d, int32_t n_docs);
+
 /* Workspace bytes cp_allgather_attn_fwd needs (0 for invalid arguments). */
 size_t cp_allgather_workspace_bytes(int32_t N, int32_t dtype, int64_t b, int64_t S, int64_t Hkv,
                                     int64_t d, int32_t n_docs);

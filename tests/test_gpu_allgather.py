@@ -114,3 +114,32 @@ def test_full_size_documents_sampled(cp):
     tol_o, tol_l = TOL["bf16"]
     assert_close_lse(got_l, rl, tol_l)
     assert_close_o(got_o, ro, tol_o)
+
+
+# ------------------------------------------------------------------ backward
+
+BWD_CASES = [
+    ("zigzag", 4, 1024, 1, 4, 2, [0, 100, 101, 400, 777]),
+    ("zigzag", 2, 424, 2, 2, 2, [0, 5, 211, 212, 300]),
+    ("striped", 4, 1024, 1, 4, 1, [0, 128, 255, 256, 1000]),
+    ("contiguous", 3, 390, 1, 2, 1, [0, 129, 130, 389]),
+    ("zigzag", 8, 2048, 1, 8, 2, list(range(0, 2048, 97))),
+    ("zigzag", 4, 1024, 1, 4, 2, [0]),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: "-".join(str(x) for x in c[:6]) + "-d%d" % len(c[6]))
+def test_allgather_bwd_matches_oracle(cp, case):
+    layout, N, S, b, hq, hkv, docs = case
+    d = 128
+    q, k, v = W.random_qkv(b, S, hq, hkv, d, "bf16", seed=2 * S + N)
+    do = W.random_do(b, S, hq, d, "bf16", seed=2 * S + N)
+    qr, kr, vr, dor = (cp.layout_permute(t.cuda(), layout, N) for t in (q, k, v, do))
+    o, lse = cp.allgather_attn_fwd(qr, kr, vr, layout, N, True, docs)
+    grads = cp.allgather_attn_bwd(qr, kr, vr, o, lse, dor, layout, N, True, docs)
+    grads = [cp.layout_permute(g, layout, N, inverse=True) for g in grads]
+    cp.stream_check()
+    want = oracle.allgather_attention_bwd(np64(q), np64(k), np64(v), np64(do), layout, N, True, d ** -0.5, docs)
+    for name, g, w in zip(("dq", "dk", "dv"), grads, want):
+        err = np.max(np.abs(np64(g) - w))
+        assert err <= 2e-2 * np.max(np.abs(w)), (name, err, np.max(np.abs(w)))
