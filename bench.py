@@ -381,9 +381,35 @@ def main():
         cp.stream_check()
         t = statistics.mean(ms)
         tf = wd.effective_flops() / (t * 1e-3) / 1e12
-        del qa, ka, va, oa, la, wsa
+        # its backward (gather, document-masked backward, dK/dV back to the ranks)
+        doa = cp.layout_permute(W.random_do(wd.b, wd.S, wd.hq, wd.d, wd.dtype, wd.seed).to(dev), wd.layout, wd.N)
+        gq, gk, gv = torch.empty_like(qa), torch.empty_like(ka), torch.empty_like(va)
+        wsb = torch.empty(cp.lib().cp_allgather_bwd_workspace_bytes(wd.N, 0, wd.b, wd.S, wd.hq, wd.hkv, wd.d, len(docs)),
+                          dtype=torch.uint8, device=dev)
+
+        def bstep():
+            cp.allgather_attn_bwd(qa, ka, va, oa, la, doa, wd.layout, wd.N, wd.causal, docs, wd.scale, gq, gk, gv, wsb)
+
+        for _ in range(3):
+            bstep()
+        bms = []
+        for _ in range(max(3, min(args.steps, 10))):
+            flush.zero_()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            bstep()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            bms.append(a0.elapsed_time(a1))
+        cp.stream_check()
+        tb = statistics.mean(bms)
+        tfb = 2.5 * wd.effective_flops() / (tb * 1e-3) / 1e12
+        del qa, ka, va, oa, la, wsa, doa, gq, gk, gv, wsb
         torch.cuda.empty_cache()
         return {"metric": "all-gather CP fwd TFLOP/s (causal document mask, effective FLOPs)", "workload": wd.name,
+                "backward": {"value": tfb, "unit": "TFLOP/s", "ms_per_step": tb, "frac": tfb / peak_tf,
+                             "launches_per_step": 7,
+                             "timed": "K, V gather + statistics + backward kernel + dq conversion + dK, dV scatter"},
                 "n_docs": len(docs), "value": tf, "unit": "TFLOP/s", "ms_per_step": t, "steps": len(ms),
                 "launches_per_step": 3,
                 "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (document variant)", "achieved": tf,
