@@ -558,15 +558,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float4 *stat = reinterpret_cast<const float4 *>(smem + C::OFF_ST + s * BQ * 8) + half * 16;
             float pv[32];
             const uint64_t sl2x2 = f2_pack(sl2, sl2);
+            if (seq.partial()) {  // warp-uniform: the element mask only where a tile needs it
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const float4 st = stat[c];
-                float x0, x1;
-                f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), sl2x2,
-                                 f2_pack(-st.x, -st.z)),
-                          x0, x1);
-                pv[2 * c] = (2 * c < c_first || 2 * c >= c_last) ? 0.f : ex2_approx(x0);
-                pv[2 * c + 1] = (2 * c + 1 < c_first || 2 * c + 1 >= c_last) ? 0.f : ex2_approx(x1);
+                for (int c = 0; c < 16; ++c) {
+                    const float4 st = stat[c];
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), sl2x2,
+                                     f2_pack(-st.x, -st.z)),
+                              x0, x1);
+                    pv[2 * c] = (2 * c < c_first || 2 * c >= c_last) ? 0.f : ex2_approx(x0);
+                    pv[2 * c + 1] = (2 * c + 1 < c_first || 2 * c + 1 >= c_last) ? 0.f : ex2_approx(x1);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const float4 st = stat[c];
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), sl2x2,
+                                     f2_pack(-st.x, -st.z)),
+                              x0, x1);
+                    pv[2 * c] = ex2_approx(x0);
+                    pv[2 * c + 1] = ex2_approx(x1);
+                }
             }
             uint32_t pk16[16];
 #pragma unroll
