@@ -17,6 +17,8 @@ Entry points mirror include/cpattn.h:
   layout_range(layout, N, S, rank) -> (nseg, start, len, stride)
   tile_classes(q_range, q_len, kv_range, kv_len, causal, tile_q, tile_k)
   stream_check()
+The real-rank ring (one process per GPU, K/V passed with torch.distributed
+point-to-point transfers) lives in context_attention_cp_b200.ring_dist.
 Tensors are torch tensors on the current CUDA device; token tensors are
 [b, s, H, d] with d contiguous, lse tensors [b, H, s] fp32.
 """

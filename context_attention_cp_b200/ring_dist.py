@@ -1,0 +1,66 @@
+"""Ring attention across real ranks: one process per GPU, K/V blocks passed around
+the ring with torch.distributed point-to-point transfers.
+
+"上下文并行与 Ring Attention" (hs-black.github.io), section Ring Attention: N
+devices form a ring; device i starts with Q_i, K_i, V_i; at step r it attends its
+Q to the K/V block it holds (the block of rank (i - r) mod N), merges the partial
+into its running (o, lse), and passes the block on to device i + 1 while it
+receives the next one from device i - 1, so the transfer hides behind the
+computation.  Q and O never move.
+
+Each rank holds its c = S / N tokens in the layout's order (rank-major local
+blocks, as cp_layout_permute produces them on one device).  The step's compute is
+cp_block_attn_fwd with the rank ranges of the layout: the first step writes the
+fp32 (o, lse), later steps merge into them with the kernel's fused epilogue.  The
+exchange of the next block is posted before the compute and waited for after it.
+
+The compute step can be replaced (`compute=`), which is how the schedule is tested
+on CPU ranks (gloo) without a GPU.
+"""
+import torch
+import torch.distributed as dist
+
+from . import _binding as B
+
+
+def block_compute(q, k, v, q_range, kv_range, causal, scale, o, lse, accumulate):
+    """The default step: the tensor-core (bf16) or FFMA (fp32) block kernel."""
+    B.block_attn_fwd(q, k, v, q_range, kv_range, causal, scale, o, lse, accumulate=accumulate)
+
+
+def ring_attn_fwd_dist(q, k, v, layout, causal, scale=None, group=None, compute=block_compute):
+    """This rank's share of ring attention.
+
+    q [b, c, Hq, d], k / v [b, c, Hkv, d]: this rank's local blocks (its layout
+    positions, in order).  Returns (o [b, c, Hq, d] in q's dtype, lse [b, Hq, c]
+    fp32) for the local queries.  All ranks of `group` call it together.
+    """
+    rank = dist.get_rank(group)
+    N = dist.get_world_size(group)
+    b, c, Hq, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    S = c * N
+    q_range = B.layout_range(layout, N, S, rank)
+    nxt, prv = (rank + 1) % N, (rank - 1) % N
+    to_global = (lambda r: dist.get_global_rank(group, r)) if group is not None else (lambda r: r)
+    o = torch.empty((b, c, Hq, d), dtype=torch.float32, device=q.device)
+    lse = torch.empty((b, Hq, c), dtype=torch.float32, device=q.device)
+    cur_k, cur_v = k.contiguous(), v.contiguous()
+    buf_k, buf_v = torch.empty_like(cur_k), torch.empty_like(cur_v)
+    for r in range(N):
+        src = (rank - r) % N                      # the block this rank holds at step r
+        reqs = []
+        if r + 1 < N:                             # pass the block on, take the next one
+            ops = [dist.P2POp(dist.isend, cur_k, to_global(nxt), group),
+                   dist.P2POp(dist.isend, cur_v, to_global(nxt), group),
+                   dist.P2POp(dist.irecv, buf_k, to_global(prv), group),
+                   dist.P2POp(dist.irecv, buf_v, to_global(prv), group)]
+            reqs = dist.batch_isend_irecv(ops)
+        compute(q, cur_k, cur_v, q_range, B.layout_range(layout, N, S, src), causal, scale, o, lse, r > 0)
+        for req in reqs:
+            req.wait()
+        if r + 1 < N:
+            cur_k, buf_k = buf_k, cur_k
+            cur_v, buf_v = buf_v, cur_v
+    return o.to(q.dtype), lse

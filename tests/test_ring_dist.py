@@ -1,0 +1,78 @@
+"""The real-rank ring (context_attention_cp_b200.ring_dist) on CPU: 2, 3 and 4 gloo
+ranks, each holding only its own layout block, pass K/V around the ring
+(section Ring Attention).  The block step is injected: here the fp64 oracle's block
+attention and LSE merge, so the test checks the schedule (which block each rank
+holds at each step, the exchange, the buffer swap) and the step-by-step merge
+against the oracle's whole-sequence attention."""
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _positions(rng_tuple):
+    starts, lens, stride = rng_tuple
+    out = []
+    for s0, n in zip(starts, lens):
+        out.extend(s0 + t * stride for t in range(n))
+    return np.array(out, dtype=np.int64)
+
+
+def _worker(rank, world, port, layout, S, out):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import oracle
+    from context_attention_cp_b200 import ring_dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        r = np.random.default_rng(7)
+        b, hq, hkv, d = 1, 4, 2, 8
+        q = r.standard_normal((b, S, hq, d))
+        k = r.standard_normal((b, S, hkv, d))
+        v = r.standard_normal((b, S, hkv, d))
+        pos = np.array(oracle.layout.rank_positions(layout, world, S, rank))
+        ql, kl, vl = (torch.from_numpy(np.ascontiguousarray(t[:, pos])) for t in (q, k, v))
+        seen = []
+
+        def oracle_step(qq, kk, vv, q_range, kv_range, causal, scale, o, lse, accumulate):
+            pk = _positions(kv_range)
+            seen.append(int(pk[0]))
+            ob, lb = oracle.attention(qq.numpy(), kk.numpy(), vv.numpy(), causal, scale,
+                                      pos_q=_positions(q_range), pos_k=pk, nthreads=1)
+            if accumulate:
+                om, lm = oracle.lse_merge(o.numpy().transpose(0, 2, 1, 3), lse.numpy(), ob.transpose(0, 2, 1, 3), lb)
+                ob, lb = om.transpose(0, 2, 1, 3), lm
+            o.copy_(torch.from_numpy(np.ascontiguousarray(ob)))
+            lse.copy_(torch.from_numpy(np.ascontiguousarray(lb)))
+
+        o, lse = ring_dist.ring_attn_fwd_dist(ql, kl, vl, layout, True, 0.35, compute=oracle_step)
+        want_o, want_l = oracle.ring_attention(q, k, v, layout, world, True, 0.35, nthreads=1)
+        out[rank] = (float(np.max(np.abs(o.numpy() - want_o[:, pos]))),
+                     float(np.max(np.abs(lse.numpy() - want_l[:, :, pos]))),
+                     seen,
+                     [int(oracle.layout.rank_positions(layout, world, S, (rank - s) % world)[0]) for s in range(world)])
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 32), ("striped", 4, 32), ("contiguous", 3, 24),
+                                            ("zigzag", 4, 64)])
+def test_ring_over_gloo_ranks(layout, world, S):
+    port = 29600 + (os.getpid() + world * 7 + len(layout)) % 900
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_worker, args=(world, port, layout, S, out), nprocs=world, start_method="spawn", join=True)
+    assert sorted(out.keys()) == list(range(world))
+    for rank, (err_o, err_l, seen, want_seen) in out.items():
+        assert err_o <= 1e-6 and err_l <= 1e-6, (rank, err_o, err_l)
+        assert seen == want_seen, (rank, seen, want_seen)   # step r holds rank (i - r) mod N's block
