@@ -7,8 +7,9 @@ One step = one cp_ring_attn_fwd over the whole workload (all N virtual ranks, al
 ring steps), inputs already permuted to rank-major order and resident in HBM.
 The line also carries the standalone merge bandwidth, the backward
 (cp_ring_attn_bwd) of the same workload and the All-Gather forward with a document
-mask (cp_allgather_attn_fwd) on its 8-document variant and Ulysses
-(cp_ulysses_attn_fwd, P = 4) on its shape, each timed on its own.
+mask (cp_allgather_attn_fwd) on its 8-document variant, Ulysses
+(cp_ulysses_attn_fwd, P = 4) on its shape and USP (cp_usp_attn_fwd: Ulysses groups
+of 2 inside the workload's ring), each timed on its own.
 L2 is flushed (a 256 MiB write) before every timed step; each step is timed with
 CUDA events on the launching stream.  With --gpus N > 1 (torchrun) every rank
 runs its own instance of the workload (weak scaling, no collective on the data
@@ -424,14 +425,21 @@ def main():
     # Ulysses over P = 4 virtual ranks on this workload's shape (original order):
     # all-to-all of q, k, v, one attention launch over the head groups, all-to-all
     # of o and lse back (5 + 1 launches)
-    def ulysses_leg(P=4):
+    def ulysses_leg(P=4, usp=False):
+        # usp: Ulysses groups of P inside each of the workload's N ring groups (the
+        # inputs in the ring's rank-major order, permuted before the timed region)
         qu, ku, vu = (t.to(dev) for t in W.make_inputs(w))
+        if usp:
+            qu, ku, vu = (cp.layout_permute(t, w.layout, w.N) for t in (qu, ku, vu))
         ou = torch.empty_like(qu)
         lu = torch.empty((w.b, w.hq, w.S), dtype=torch.float32, device=dev)
         wsu = torch.empty(cp.ulysses_workspace_bytes(P, 0, w.b, w.S, w.hq, w.hkv, w.d), dtype=torch.uint8, device=dev)
 
         def ustep():
-            cp.ulysses_attn_fwd(qu, ku, vu, P, w.causal, w.scale, ou, lu, wsu)
+            if usp:
+                cp.usp_attn_fwd(qu, ku, vu, w.layout, w.N, P, w.causal, w.scale, ou, lu, wsu)
+            else:
+                cp.ulysses_attn_fwd(qu, ku, vu, P, w.causal, w.scale, ou, lu, wsu)
 
         for _ in range(3):
             ustep()
@@ -449,7 +457,8 @@ def main():
         tf = flops / (t * 1e-3) / 1e12
         del qu, ku, vu, ou, lu, wsu
         torch.cuda.empty_cache()
-        return {"metric": "Ulysses fwd TFLOP/s (causal, effective FLOPs)", "P": P, "value": tf, "unit": "TFLOP/s",
+        return {"metric": ("USP" if usp else "Ulysses") + " fwd TFLOP/s (causal, effective FLOPs)", "P": P,
+                "ring": {"layout": w.layout, "N": w.N} if usp else None, "value": tf, "unit": "TFLOP/s",
                 "ms_per_step": t, "steps": len(ms), "launches_per_step": 6,
                 "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": tf, "peak": peak_tf,
                              "unit": "TFLOP/s", "frac": tf / peak_tf, "peak_source": peak_src + " bf16 burst",
@@ -458,6 +467,8 @@ def main():
     ulysses = None
     if w.dtype == "bf16" and w.hkv % 4 == 0 and w.hq % 4 == 0 and w.S % 4 == 0 and rank == 0:
         ulysses = ulysses_leg()
+        if w.hkv % 2 == 0 and w.S % (2 * w.N) == 0:
+            ulysses["usp"] = ulysses_leg(P=2, usp=True)
 
     # end to end through the public API, every step: pinned host -> device copy of
     # q/k/v, permute to rank-major order, ring attention, unpermute, device -> host

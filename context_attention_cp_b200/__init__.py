@@ -13,6 +13,8 @@ Entry points mirror include/cpattn.h:
   allgather_attn_bwd(q, k, v, o, lse, do, layout, N, causal, doc_starts=None) -> (dq, dk, dv)
   ulysses_attn_fwd(q, k, v, P, causal, scale=None); ulysses_all_to_all(x, P, inverse=False)
   ulysses_attn_bwd(q, k, v, o, lse, do, P, causal, scale=None) -> (dq, dk, dv)
+  usp_attn_fwd(q, k, v, layout, N, P, causal, scale=None)     (Ulysses x ring)
+  usp_attn_bwd(q, k, v, o, lse, do, layout, N, P, causal, scale=None) -> (dq, dk, dv)
   layout_permute(x, layout, N, seq_axis=1, inverse=False, out=None)
   layout_range(layout, N, S, rank) -> (nseg, start, len, stride)
   tile_classes(q_range, q_len, kv_range, kv_len, causal, tile_q, tile_k)
@@ -27,5 +29,5 @@ from ._binding import (  # noqa: F401
     layout_range, lib, lib_path,
     lse_merge, ring_attn_bwd, ring_attn_fwd, ring_attn_fwd_static_scratch, ring_bwd_workspace_bytes,
     ring_workspace_bytes, selftest_wait_timeout, stream_check, tile_classes, ulysses_all_to_all, ulysses_attn_bwd, ulysses_attn_fwd,
-    ulysses_workspace_bytes,
+    ulysses_workspace_bytes, usp_attn_bwd, usp_attn_fwd, usp_workspace_bytes,
 )

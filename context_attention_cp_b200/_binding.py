@@ -50,6 +50,10 @@ _SIGNATURES = {
     "cp_ulysses_workspace_bytes": (_sz, [_i32, _i32, _i64, _i64, _i64, _i64, _i64]),
     "cp_ulysses_attn_bwd": (_i32, [_i32, _i32, _T, _T, _T, _T, _T, _T, _f32, _T, _T, _T, _vp, _sz, _vp]),
     "cp_ulysses_bwd_workspace_bytes": (_sz, [_i32, _i32, _i64, _i64, _i64, _i64, _i64]),
+    "cp_usp_attn_fwd": (_i32, [_i32, _i32, _i32, _i32, _T, _T, _T, _f32, _T, _T, _vp, _sz, _vp]),
+    "cp_usp_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _i64, _i64]),
+    "cp_usp_attn_bwd": (_i32, [_i32, _i32, _i32, _i32, _T, _T, _T, _T, _T, _T, _f32, _T, _T, _T, _vp, _sz, _vp]),
+    "cp_usp_bwd_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _i64, _i64]),
     "cp_layout_permute": (_i32, [_i32, _i32, _i32, _T, _T, _i32, _vp]),
     "cp_layout_range": (_i32, [_i32, _i32, _i64, _i32, _R]),
     "cp_tile_classes": (_i32, [_R, _i64, _R, _i64, _i32, _i32, _i32, ctypes.POINTER(ctypes.c_int8)]),
@@ -319,6 +323,47 @@ def ulysses_attn_bwd(q, k, v, o, lse, do, P, causal, scale=None, dq=None, dk=Non
     _check(lib().cp_ulysses_attn_bwd(P, int(bool(causal)), *[_ref(t) for t in ts[:6]], float(scale),
                                      *[_ref(t) for t in ts[6:]], ctypes.c_void_p(workspace.data_ptr()), need,
                                      _stream()))
+    return dq, dk, dv
+
+
+def usp_workspace_bytes(layout, N, P, dtype_code, b, S, Hq, Hkv, d):
+    return lib().cp_usp_workspace_bytes(LAYOUTS[layout], N, P, dtype_code, b, S, Hq, Hkv, d)
+
+
+def usp_attn_fwd(q, k, v, layout, N, P, causal, scale=None, o=None, lse=None, workspace=None):
+    """USP: Ulysses over P inside each of N ring groups, the ring across them; q/k/v/o
+    in the ring's rank-major order for (layout, N)."""
+    import torch
+    b, S, Hq, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((b, Hq, S), dtype=torch.float32, device=q.device) if lse is None else lse
+    need = usp_workspace_bytes(layout, N, P, _dtype_code(q), b, S, Hq, k.shape[2], d)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ts = [_tensor(t) for t in (q, k, v, o, lse)]
+    _check(lib().cp_usp_attn_fwd(LAYOUTS[layout], N, P, int(bool(causal)), _ref(ts[0]), _ref(ts[1]), _ref(ts[2]),
+                                 float(scale), _ref(ts[3]), _ref(ts[4]), ctypes.c_void_p(workspace.data_ptr()), need,
+                                 _stream()))
+    return o, lse
+
+
+def usp_attn_bwd(q, k, v, o, lse, do, layout, N, P, causal, scale=None, dq=None, dk=None, dv=None, workspace=None):
+    """Gradients of USP attention; every tensor in the ring's rank-major order."""
+    import torch
+    b, S, Hq, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = lib().cp_usp_bwd_workspace_bytes(LAYOUTS[layout], N, P, _dtype_code(q), b, S, Hq, k.shape[2], d)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ts = [_tensor(t) for t in (q, k, v, o, lse, do, dq, dk, dv)]
+    _check(lib().cp_usp_attn_bwd(LAYOUTS[layout], N, P, int(bool(causal)), *[_ref(t) for t in ts[:6]], float(scale),
+                                 *[_ref(t) for t in ts[6:]], ctypes.c_void_p(workspace.data_ptr()), need, _stream()))
     return dq, dk, dv
 
 

@@ -572,12 +572,18 @@ size_t cp_ulysses_workspace_bytes(int32_t P, int32_t dtype, int64_t b, int64_t S
     return (size_t)(2 * up(b * S * Hq * d * es) + 2 * up(b * S * Hkv * d * es) + up(b * Hq * S * 4));
 }
 
-cp_status cp_ulysses_attn_fwd(int32_t P, int32_t causal, const cp_tensor *q, const cp_tensor *k, const cp_tensor *v,
-                              float softmax_scale, cp_tensor *o, cp_tensor *lse, void *workspace,
-                              size_t workspace_bytes, void *stream)
+// Ulysses exchange around a ring: the head-sharded tensors [P*b, S, H/P, d] keep
+// the sequence axis as it came in, so with N = 1 this is plain Ulysses and with a
+// rank-major sequence of N ring groups it is the Ulysses x ring hybrid (every
+// ring group's exchange moves tokens only inside the group's block).
+static cp_status uly_ring_fwd(int32_t layout, int32_t N, int32_t P, int32_t causal, const cp_tensor *q,
+                              const cp_tensor *k, const cp_tensor *v, float softmax_scale, cp_tensor *o, cp_tensor *lse,
+                              void *workspace, size_t workspace_bytes, void *stream)
 {
     g_last_error[0] = 0;
     cp_status s;
+    if (layout < 0 || layout > 2) return fail(CP_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (N < 1 || N > 4096) return fail(CP_ERR_INVALID_ARG, "N must be in [1, 4096]");
     if (causal != 0 && causal != 1) return fail(CP_ERR_INVALID_ARG, "causal must be 0 or 1");
     if ((s = check_tensor(q, "q")) != CP_OK || (s = check_tensor(k, "k")) != CP_OK ||
         (s = check_tensor(v, "v")) != CP_OK)
@@ -591,7 +597,9 @@ cp_status cp_ulysses_attn_fwd(int32_t P, int32_t causal, const cp_tensor *q, con
     if (Hq % P || Hkv % P)
         return fail(CP_ERR_SHAPE, "P must divide the query heads (%lld) and the kv heads (%lld)", (long long)Hq,
                     (long long)Hkv);
-    if (S % P) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of P = %d", (long long)S, P);
+    if (S % ((int64_t)N * P))
+        return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of N * P = %d * %d", (long long)S, N, P);
+    if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N)) return fail(CP_ERR_SHAPE, "zig-zag needs S to be a multiple of 2N");
     if (S % 4) return fail(CP_ERR_SHAPE, "S must be a multiple of 4");
     if (S >= ((int64_t)1 << 30)) return fail(CP_ERR_SHAPE, "sequence too long (S must be below 2^30)");
     if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;
@@ -622,9 +630,10 @@ cp_status cp_ulysses_attn_fwd(int32_t P, int32_t causal, const cp_tensor *q, con
     if ((s = cp_ulysses_all_to_all(P, 0, q, &qh, stream)) != CP_OK) return s;
     if ((s = cp_ulysses_all_to_all(P, 0, k, &kh, stream)) != CP_OK) return s;
     if ((s = cp_ulysses_all_to_all(P, 0, v, &vh, stream)) != CP_OK) return s;
-    // every rank's heads over the whole sequence: one launch, the ranks as batch entries
-    if ((s = cp_ring_attn_fwd(CP_LAYOUT_CONTIGUOUS, 1, causal, &qh, &kh, &vh, softmax_scale, &oh, &lh, CP_RING_FUSED,
-                              nullptr, 0, stream)) != CP_OK)
+    // every rank's heads over the whole sequence (with N > 1: the ring over the
+    // groups' blocks): one launch, the head groups as batch entries
+    if ((s = cp_ring_attn_fwd(layout, N, causal, &qh, &kh, &vh, softmax_scale, &oh, &lh, CP_RING_FUSED, nullptr, 0,
+                              stream)) != CP_OK)
         return s;
     // and back: o [P*b, S, hp, d] -> [b, S, Hq, d]; lse [P][b][hp * S] -> [b][P][hp * S]
     if ((s = cp_ulysses_all_to_all(P, 1, o, &oh, stream)) != CP_OK) return s;
@@ -632,6 +641,28 @@ cp_status cp_ulysses_attn_fwd(int32_t P, int32_t causal, const cp_tensor *q, con
     cudaError_t e = launch_shard_transpose(sp, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "all-to-all launch");
     return CP_OK;
+}
+
+cp_status cp_ulysses_attn_fwd(int32_t P, int32_t causal, const cp_tensor *q, const cp_tensor *k, const cp_tensor *v,
+                              float softmax_scale, cp_tensor *o, cp_tensor *lse, void *workspace,
+                              size_t workspace_bytes, void *stream)
+{
+    return uly_ring_fwd(CP_LAYOUT_CONTIGUOUS, 1, P, causal, q, k, v, softmax_scale, o, lse, workspace, workspace_bytes,
+                        stream);
+}
+
+size_t cp_usp_workspace_bytes(int32_t layout, int32_t N, int32_t P, int32_t dtype, int64_t b, int64_t S, int64_t Hq,
+                              int64_t Hkv, int64_t d)
+{
+    if (layout < 0 || layout > 2 || N < 1) return 0;
+    return cp_ulysses_workspace_bytes(P, dtype, b, S, Hq, Hkv, d);
+}
+
+cp_status cp_usp_attn_fwd(int32_t layout, int32_t N, int32_t P, int32_t causal, const cp_tensor *q, const cp_tensor *k,
+                          const cp_tensor *v, float softmax_scale, cp_tensor *o, cp_tensor *lse, void *workspace,
+                          size_t workspace_bytes, void *stream)
+{
+    return uly_ring_fwd(layout, N, P, causal, q, k, v, softmax_scale, o, lse, workspace, workspace_bytes, stream);
 }
 
 size_t cp_allgather_bwd_workspace_bytes(int32_t N, int32_t dtype, int64_t b, int64_t S, int64_t Hq, int64_t Hkv,
@@ -782,25 +813,40 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     return CP_OK;
 }
 
-size_t cp_ulysses_bwd_workspace_bytes(int32_t P, int32_t dtype, int64_t b, int64_t S, int64_t Hq, int64_t Hkv,
-                                      int64_t d)
+static size_t uly_ring_bwd_ws(int32_t layout, int32_t N, int32_t P, int32_t dtype, int64_t b, int64_t S, int64_t Hq,
+                              int64_t Hkv, int64_t d)
 {
-    if (P < 1 || b < 0 || S < 0 || Hq < 0 || Hkv < 0 || d < 0 || !elem_size(dtype) || Hq % P) return 0;
+    if (layout < 0 || layout > 2 || N < 1 || P < 1 || b < 0 || S < 0 || Hq < 0 || Hkv < 0 || d < 0 ||
+        !elem_size(dtype) || Hq % P || S % N)
+        return 0;
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
     const int64_t es = elem_size(dtype);
     const int64_t qb = up(b * S * Hq * d * es), kb = up(b * S * Hkv * d * es), lb = up(b * Hq * S * 4);
     // head-sharded q, o, dout, dq; k, v, dk, dv; lse; then the ring backward's own
-    return (size_t)(4 * qb + 4 * kb + lb) +
-           cp_ring_bwd_workspace_bytes(CP_LAYOUT_CONTIGUOUS, 1, dtype, P * b, S, Hq / P, d);
+    return (size_t)(4 * qb + 4 * kb + lb) + cp_ring_bwd_workspace_bytes(layout, N, dtype, P * b, S, Hq / P, d);
 }
 
-cp_status cp_ulysses_attn_bwd(int32_t P, int32_t causal, const cp_tensor *q, const cp_tensor *k, const cp_tensor *v,
-                              const cp_tensor *o, const cp_tensor *lse, const cp_tensor *dout, float softmax_scale,
-                              cp_tensor *dq, cp_tensor *dk, cp_tensor *dv, void *workspace, size_t workspace_bytes,
-                              void *stream)
+size_t cp_ulysses_bwd_workspace_bytes(int32_t P, int32_t dtype, int64_t b, int64_t S, int64_t Hq, int64_t Hkv,
+                                      int64_t d)
+{
+    return uly_ring_bwd_ws(CP_LAYOUT_CONTIGUOUS, 1, P, dtype, b, S, Hq, Hkv, d);
+}
+
+size_t cp_usp_bwd_workspace_bytes(int32_t layout, int32_t N, int32_t P, int32_t dtype, int64_t b, int64_t S,
+                                  int64_t Hq, int64_t Hkv, int64_t d)
+{
+    return uly_ring_bwd_ws(layout, N, P, dtype, b, S, Hq, Hkv, d);
+}
+
+static cp_status uly_ring_bwd(int32_t layout, int32_t N, int32_t P, int32_t causal, const cp_tensor *q,
+                              const cp_tensor *k, const cp_tensor *v, const cp_tensor *o, const cp_tensor *lse,
+                              const cp_tensor *dout, float softmax_scale, cp_tensor *dq, cp_tensor *dk, cp_tensor *dv,
+                              void *workspace, size_t workspace_bytes, void *stream)
 {
     g_last_error[0] = 0;
     cp_status s;
+    if (layout < 0 || layout > 2) return fail(CP_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (N < 1 || N > 4096) return fail(CP_ERR_INVALID_ARG, "N must be in [1, 4096]");
     if (causal != 0 && causal != 1) return fail(CP_ERR_INVALID_ARG, "causal must be 0 or 1");
     if ((s = check_tensor(q, "q")) != CP_OK || (s = check_tensor(k, "k")) != CP_OK ||
         (s = check_tensor(v, "v")) != CP_OK || (s = check_tensor(dout, "dout")) != CP_OK ||
@@ -818,7 +864,9 @@ cp_status cp_ulysses_attn_bwd(int32_t P, int32_t causal, const cp_tensor *q, con
     if (Hq % P || Hkv % P)
         return fail(CP_ERR_SHAPE, "P must divide the query heads (%lld) and the kv heads (%lld)", (long long)Hq,
                     (long long)Hkv);
-    if (S % P) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of P = %d", (long long)S, P);
+    if (S % ((int64_t)N * P))
+        return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of N * P = %d * %d", (long long)S, N, P);
+    if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N)) return fail(CP_ERR_SHAPE, "zig-zag needs S to be a multiple of 2N");
     if (S % 4) return fail(CP_ERR_SHAPE, "S must be a multiple of 4");
     if (S >= ((int64_t)1 << 30)) return fail(CP_ERR_SHAPE, "sequence too long (S must be below 2^30)");
     if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;
@@ -831,7 +879,7 @@ cp_status cp_ulysses_attn_bwd(int32_t P, int32_t causal, const cp_tensor *q, con
         if (!same_shape(t, k) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "dk and dv must be bf16 shaped like k");
     if (!(lse->stride[2] == 1 && lse->stride[1] == S && (b <= 1 || lse->stride[0] == Hq * S)))
         return fail(CP_ERR_INVALID_ARG, "lse must be contiguous");
-    const size_t need = cp_ulysses_bwd_workspace_bytes(P, q->dtype, b, S, Hq, Hkv, d);
+    const size_t need = uly_ring_bwd_ws(layout, N, P, q->dtype, b, S, Hq, Hkv, d);
     if (!workspace || workspace_bytes < need) return fail(CP_ERR_INVALID_ARG, "workspace of %zu bytes needed", need);
     if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     if (b == 0 || S == 0) return CP_OK;
@@ -849,7 +897,7 @@ cp_status cp_ulysses_attn_bwd(int32_t P, int32_t causal, const cp_tensor *q, con
     cp_tensor kh = kt(0), vh = kt(1), dkh = kt(2), dvh = kt(3);
     cp_tensor lh{ws + 4 * qb + 4 * kb, CP_FP32, 0, {P * b, hp, S, 1}, {hp * S, S, 1, 1}};
     char *ws_ring = ws + 4 * qb + 4 * kb + lb;
-    const size_t ring_need = cp_ring_bwd_workspace_bytes(CP_LAYOUT_CONTIGUOUS, 1, CP_BF16, P * b, S, hp, d);
+    const size_t ring_need = cp_ring_bwd_workspace_bytes(layout, N, CP_BF16, P * b, S, hp, d);
     // exchange in: q, k, v, o, dout and lse to the head-sharded layout
     const cp_tensor *ins[5] = {q, k, v, o, dout};
     cp_tensor *outs[5] = {&qh, &kh, &vh, &oh, &doh};
@@ -858,15 +906,34 @@ cp_status cp_ulysses_attn_bwd(int32_t P, int32_t causal, const cp_tensor *q, con
     ShardParams sp{P, b, 1, hp * S * 4, 0, lse->data, lh.data};
     cudaError_t e = launch_shard_transpose(sp, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "all-to-all launch");
-    // each rank's head group over the whole sequence
-    if ((s = cp_ring_attn_bwd(CP_LAYOUT_CONTIGUOUS, 1, causal, &qh, &kh, &vh, &oh, &lh, &doh, softmax_scale, &dqh, &dkh,
-                              &dvh, ws_ring, ring_need, stream)) != CP_OK)
+    // each rank's head group over the whole sequence (with N > 1: the ring backward
+    // over the groups' blocks, dK and dV travelling with their block)
+    if ((s = cp_ring_attn_bwd(layout, N, causal, &qh, &kh, &vh, &oh, &lh, &doh, softmax_scale, &dqh, &dkh, &dvh,
+                              ws_ring, ring_need, stream)) != CP_OK)
         return s;
     // exchange out: the gradients back to the sequence-sharded layout
     if ((s = cp_ulysses_all_to_all(P, 1, dq, &dqh, stream)) != CP_OK) return s;
     if ((s = cp_ulysses_all_to_all(P, 1, dk, &dkh, stream)) != CP_OK) return s;
     if ((s = cp_ulysses_all_to_all(P, 1, dv, &dvh, stream)) != CP_OK) return s;
     return CP_OK;
+}
+
+cp_status cp_ulysses_attn_bwd(int32_t P, int32_t causal, const cp_tensor *q, const cp_tensor *k, const cp_tensor *v,
+                              const cp_tensor *o, const cp_tensor *lse, const cp_tensor *dout, float softmax_scale,
+                              cp_tensor *dq, cp_tensor *dk, cp_tensor *dv, void *workspace, size_t workspace_bytes,
+                              void *stream)
+{
+    return uly_ring_bwd(CP_LAYOUT_CONTIGUOUS, 1, P, causal, q, k, v, o, lse, dout, softmax_scale, dq, dk, dv, workspace,
+                        workspace_bytes, stream);
+}
+
+cp_status cp_usp_attn_bwd(int32_t layout, int32_t N, int32_t P, int32_t causal, const cp_tensor *q, const cp_tensor *k,
+                          const cp_tensor *v, const cp_tensor *o, const cp_tensor *lse, const cp_tensor *dout,
+                          float softmax_scale, cp_tensor *dq, cp_tensor *dk, cp_tensor *dv, void *workspace,
+                          size_t workspace_bytes, void *stream)
+{
+    return uly_ring_bwd(layout, N, P, causal, q, k, v, o, lse, dout, softmax_scale, dq, dk, dv, workspace,
+                        workspace_bytes, stream);
 }
 
 size_t cp_allgather_workspace_bytes(int32_t N, int32_t dtype, int64_t b, int64_t S, int64_t Hkv, int64_t d,

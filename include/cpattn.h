@@ -235,6 +235,48 @@ cp_status cp_ulysses_attn_bwd(int32_t P, int32_t causal, const cp_tensor *q, con
 size_t cp_ulysses_bwd_workspace_bytes(int32_t P, int32_t dtype, int64_t b, int64_t S, int64_t Hq,
                                       int64_t Hkv, int64_t d);
 
+/* USP, Ulysses inside a group and the ring across groups, on one GPU ("DeepSpeed-
+ * Ulysses" page, section on USP; hs-black.github.io context-parallel post, end of
+ * section DeepSpeed-Ulysses).  N ring groups of P Ulysses ranks each (N * P virtual
+ * ranks): ring group g holds the layout's block g (the ring layout over N, as
+ * cp_layout_permute(layout, N) orders it), and Ulysses rank u of that group holds
+ * the contiguous u-th of the block's P slices, all heads.  The exchange inside every
+ * group gives rank (g, u) the group's whole block for heads [u Hq/P, (u+1) Hq/P)
+ * (KV heads likewise); the ring attention over the N groups runs for every head
+ * group (one fused launch, the head groups as batch entries); the exchange back
+ * returns o and lse to the sequence-sharded ranks.
+ *   q [b, S, Hq, d], k / v [b, S, Hkv, d], o [b, S, Hq, d]: the S axis in the
+ *   ring's rank-major order for (layout, N), contiguous; lse [b, Hq, S, 1] fp32
+ *   contiguous, same order.  P must divide Hq and Hkv; S % (N P) == 0, and
+ *   S % 2N == 0 under zig-zag; S % 4 == 0.  N = 1 is cp_ulysses_attn_fwd, P = 1
+ *   the fused ring.
+ *   workspace: cp_usp_workspace_bytes(...) bytes, 256-byte aligned (the head-
+ *   sharded q, k, v, o, lse).  Argument errors return synchronously; device
+ *   errors surface through cp_stream_check. */
+cp_status cp_usp_attn_fwd(int32_t layout, int32_t N, int32_t P, int32_t causal, const cp_tensor *q,
+                          const cp_tensor *k, const cp_tensor *v, float softmax_scale, cp_tensor *o,
+                          cp_tensor *lse, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes cp_usp_attn_fwd needs (0 for invalid arguments). */
+size_t cp_usp_workspace_bytes(int32_t layout, int32_t N, int32_t P, int32_t dtype, int64_t b, int64_t S,
+                              int64_t Hq, int64_t Hkv, int64_t d);
+
+/* USP backward: the exchange of q, k, v, o, dout and lse inside every group, the
+ * ring backward over the N groups for every head group (the kernels of
+ * cp_ring_attn_bwd; dK, dV travel with their block), the exchange of dq, dk, dv
+ * back.  Tensors as for cp_usp_attn_fwd (o and lse its results); dq [b, S, Hq, d],
+ * dk / dv [b, S, Hkv, d] bf16 outputs in the same order; all contiguous.  Requires
+ * bf16, d = 128 and the conditions of cp_usp_attn_fwd.
+ *   workspace: cp_usp_bwd_workspace_bytes(...) bytes, 256-byte aligned. */
+cp_status cp_usp_attn_bwd(int32_t layout, int32_t N, int32_t P, int32_t causal, const cp_tensor *q,
+                          const cp_tensor *k, const cp_tensor *v, const cp_tensor *o, const cp_tensor *lse,
+                          const cp_tensor *dout, float softmax_scale, cp_tensor *dq, cp_tensor *dk,
+                          cp_tensor *dv, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes cp_usp_attn_bwd needs (0 for invalid arguments). */
+size_t cp_usp_bwd_workspace_bytes(int32_t layout, int32_t N, int32_t P, int32_t dtype, int64_t b,
+                                  int64_t S, int64_t Hq, int64_t Hkv, int64_t d);
+
 /* Ring attention backward over N virtual ranks on one GPU (section 分块注意力,
  * paragraph on the backward pass; section Ring Attention for the schedule).
  * With the forward's GLOBAL o and lse of every query row and the output gradient

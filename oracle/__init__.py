@@ -401,6 +401,132 @@ def ulysses_attention_bwd_steps(q, k, v, do, n_ranks, causal, scale, nthreads=No
     return tuple(ulysses_all_to_all(np.stack([g[j][n] for j in range(P)]), P, inverse=True) for n in range(3))
 
 
+def _usp_positions(layout_name, n_ring, n_uly, S):
+    """Original positions held by rank (g, u) before the USP exchange: ring group g
+    holds the ring layout's block g, its Ulysses rank u the u-th contiguous slice."""
+    c = layout.tokens_per_rank(layout_name, n_ring, S)
+    if c % n_uly:
+        raise ValueError("the ring block must split into n_uly slices")
+    cs = c // n_uly
+    blocks = [np.asarray(layout.rank_positions(layout_name, n_ring, S, g), dtype=np.int64) for g in range(n_ring)]
+    return blocks, {(g, u): blocks[g][u * cs:(u + 1) * cs] for g in range(n_ring) for u in range(n_uly)}
+
+
+def usp_exchange(x, layout_name, n_ring, n_uly):
+    """The USP exchange written out ("DeepSpeed-Ulysses" page, section on USP: the
+    Ulysses all-to-all inside each group of the ring).  x [b, S, H, d] in original
+    order.  Rank (g, u) starts with its slice of group g's block (all heads); inside
+    the group, rank (g, u') sends the head group u of its slice to rank (g, u).
+    Returns a dict (g, u) -> [b, c, H/P, d]: group g's block in layout order, head
+    group u.  A pure index map."""
+    S, H = x.shape[1], x.shape[2]
+    P = n_uly
+    if H % P:
+        raise ValueError("n_uly must divide the heads")
+    hp = H // P
+    _, held = _usp_positions(layout_name, n_ring, n_uly, S)
+    out = {}
+    for g in range(n_ring):
+        for u in range(P):      # destination rank (g, u)
+            parts = [x[:, held[(g, u2)], u * hp:(u + 1) * hp] for u2 in range(P)]   # from (g, u2), in u2 order
+            out[(g, u)] = np.concatenate(parts, axis=1)
+    return out
+
+
+def usp_attention(q, k, v, layout_name, n_ring, n_uly, causal, scale, nthreads=None):
+    """Reference result of USP: heads are independent and the ring reaches full
+    attention, so the hybrid reproduces the plain definition exactly.  Original
+    order in and out."""
+    if q.shape[2] % n_uly or k.shape[2] % n_uly:
+        raise ValueError("n_uly must divide the heads")
+    _usp_positions(layout_name, n_ring, n_uly, q.shape[1])
+    return attention(q, k, v, causal, scale, nthreads=nthreads)
+
+
+def usp_attention_steps(q, k, v, layout_name, n_ring, n_uly, causal, scale, nthreads=None):
+    """USP step by step: the exchange inside every group, then for every head group
+    the ring over the N groups (at step r rank (g, u) holds the K/V block of rank
+    ((g - r) mod N, u), attends its queries to it and merges the partial into its
+    running (o, lse); section Ring Attention), then the exchange back.  Returns
+    (o [b, S, Hq, d], lse [b, Hq, S]) in original order."""
+    q64, k64, v64 = _f64(q), _f64(k), _f64(v)
+    b, S, Hq, d = q64.shape
+    N, P = n_ring, n_uly
+    hp = Hq // P
+    blocks, held = _usp_positions(layout_name, N, P, S)
+    qx, kx, vx = (usp_exchange(t, layout_name, N, P) for t in (q64, k64, v64))
+    o = np.zeros(q64.shape)
+    lse = np.zeros((b, Hq, S))
+    for g in range(N):
+        for u in range(P):
+            acc_o = np.zeros((b, hp, blocks[g].size, d))
+            acc_l = np.full((b, hp, blocks[g].size), -np.inf)
+            for r in range(N):
+                src = (g - r) % N
+                ob, lb = attention(qx[(g, u)], kx[(src, u)], vx[(src, u)], causal, scale, pos_q=blocks[g],
+                                   pos_k=blocks[src], nthreads=nthreads)
+                acc_o, acc_l = lse_merge(acc_o, acc_l, ob.transpose(0, 2, 1, 3), lb)
+            # exchange back: rank (g, u) returns slice u2 of its rows to rank (g, u2)
+            cs = blocks[g].size // P
+            for u2 in range(P):
+                rows = slice(u2 * cs, (u2 + 1) * cs)
+                o[:, held[(g, u2)], u * hp:(u + 1) * hp] = acc_o[:, :, rows].transpose(0, 2, 1, 3)
+                lse[:, u * hp:(u + 1) * hp, held[(g, u2)]] = acc_l[:, :, rows]
+    return o, lse
+
+
+def usp_attention_bwd(q, k, v, do, layout_name, n_ring, n_uly, causal, scale, nthreads=None):
+    """Reference gradients of USP: the plain definition's.  Original order."""
+    if q.shape[2] % n_uly or k.shape[2] % n_uly:
+        raise ValueError("n_uly must divide the heads")
+    _usp_positions(layout_name, n_ring, n_uly, q.shape[1])
+    dq, dk, dv, _, _ = attention_bwd(q, k, v, do, causal, scale, nthreads=nthreads)
+    return dq, dk, dv
+
+
+def usp_attention_bwd_steps(q, k, v, do, layout_name, n_ring, n_uly, causal, scale, nthreads=None):
+    """USP backward step by step: the exchange of q, k, v, dO inside every group; per
+    head group the global statistics of every row, then the ring over the groups
+    with dK, dV travelling with their block (the block shares of section 分块注意力's
+    backward paragraph); the exchange of dq, dk, dv back.  Original order."""
+    q64, k64, v64, do64 = _f64(q), _f64(k), _f64(v), _f64(do)
+    S, Hq, Hkv = q64.shape[1], q64.shape[2], k64.shape[2]
+    N, P = n_ring, n_uly
+    hp, hkp = Hq // P, Hkv // P
+    blocks, held = _usp_positions(layout_name, N, P, S)
+    qx, kx, vx, dox = (usp_exchange(t, layout_name, N, P) for t in (q64, k64, v64, do64))
+    dq, dk, dv = np.zeros(q64.shape), np.zeros(k64.shape), np.zeros(v64.shape)
+    for u in range(P):
+        # global statistics of every row of head group u (the forward's lse, D = dO . o)
+        stats = {}
+        for g in range(N):
+            kk = np.concatenate([kx[(j, u)] for j in range(N)], axis=1)
+            vv = np.concatenate([vx[(j, u)] for j in range(N)], axis=1)
+            pk = np.concatenate([blocks[j] for j in range(N)])
+            og, lg = attention(qx[(g, u)], kk, vv, causal, scale, pos_q=blocks[g], pos_k=pk, nthreads=nthreads)
+            stats[g] = (lg, np.einsum("bshd,bshd->bhs", dox[(g, u)], og))
+        gq = {g: np.zeros(qx[(g, u)].shape) for g in range(N)}
+        gk = {j: np.zeros(kx[(j, u)].shape) for j in range(N)}
+        gv = {j: np.zeros(vx[(j, u)].shape) for j in range(N)}
+        for r in range(N):
+            for g in range(N):
+                src = (g - r) % N
+                a, bk, bv, _, _ = attention_bwd(qx[(g, u)], kx[(src, u)], vx[(src, u)], dox[(g, u)], causal, scale,
+                                                pos_q=blocks[g], pos_k=blocks[src], lse=stats[g][0],
+                                                delta=stats[g][1], nthreads=nthreads)
+                gq[g] += a
+                gk[src] += bk
+                gv[src] += bv
+        for g in range(N):
+            cs = blocks[g].size // P
+            for u2 in range(P):
+                rows = slice(u2 * cs, (u2 + 1) * cs)
+                dq[:, held[(g, u2)], u * hp:(u + 1) * hp] = gq[g][:, rows]
+                dk[:, held[(g, u2)], u * hkp:(u + 1) * hkp] = gk[g][:, rows]
+                dv[:, held[(g, u2)], u * hkp:(u + 1) * hkp] = gv[g][:, rows]
+    return dq, dk, dv
+
+
 def attention_bwd_doc(q, k, v, do, causal, scale, doc_starts, pos_q=None, pos_k=None, nthreads=None):
     """Gradients of attention_doc (the document mask of section All-Gather 式 CP).
     Returns (dq, dk, dv) in float64."""

@@ -288,3 +288,32 @@ def test_ulysses_argument_errors_are_synchronous(cp):
     assert f(2, 1, ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.c_float(0.1), ctypes.byref(o),
              ctypes.byref(lse), ctypes.c_void_p(0x100000), 16, None) == 1        # workspace too small
     assert cp.lib().cp_ulysses_workspace_bytes(0, 0, 1, 64, 8, 2, 128) == 0
+
+
+def test_usp_argument_errors_are_synchronous(cp):
+    q = _ct(cp, [1, 64, 8, 128])
+    k = _ct(cp, [1, 64, 2, 128])
+    o = _ct(cp, [1, 64, 8, 128])
+    lse = _ct(cp, [1, 8, 64, 1], dtype=1)
+    f = cp.lib().cp_usp_attn_fwd
+
+    def call(layout, N, P, q_=q, k_=k, o_=o, lse_=lse, wsb=1 << 30):
+        return f(layout, N, P, 1, ctypes.byref(q_), ctypes.byref(k_), ctypes.byref(k_), ctypes.c_float(0.1),
+                 ctypes.byref(o_), ctypes.byref(lse_), ctypes.c_void_p(0x100000), wsb, None)
+
+    assert call(7, 2, 2) == 1                 # layout
+    assert call(1, 0, 2) == 1                 # N >= 1
+    assert call(1, 2, 4) == 3                 # P must divide Hkv = 2
+    assert call(0, 3, 2) == 3                 # S % (N P)
+    assert call(1, 2, 2, wsb=16) == 1         # workspace too small
+    q12, k12 = _ct(cp, [1, 12, 8, 128]), _ct(cp, [1, 12, 2, 128])
+    o12, l12 = _ct(cp, [1, 12, 8, 128]), _ct(cp, [1, 8, 12, 1], dtype=1)
+    assert call(1, 4, 1, q12, k12, o12, l12) == 3    # zig-zag: S % 2N
+    assert cp.lib().cp_usp_workspace_bytes(5, 2, 2, 0, 1, 64, 8, 2, 128) == 0
+    assert cp.lib().cp_usp_bwd_workspace_bytes(0, 3, 2, 0, 1, 64, 8, 2, 128) == 0   # S % N
+    assert cp.lib().cp_usp_bwd_workspace_bytes(0, 2, 2, 0, 1, 64, 8, 2, 128) > 0
+    g = cp.lib().cp_usp_attn_bwd
+    qf, kf = _ct(cp, [1, 64, 8, 128], dtype=1), _ct(cp, [1, 64, 2, 128], dtype=1)
+    of = _ct(cp, [1, 64, 8, 128], dtype=1)
+    assert g(1, 2, 2, 1, *[ctypes.byref(t) for t in (qf, kf, kf, of, lse, of)], ctypes.c_float(0.1),
+             *[ctypes.byref(t) for t in (of, kf, kf)], ctypes.c_void_p(0x100000), 1 << 30, None) == 2  # bf16 only
