@@ -854,8 +854,6 @@ static cp_status uly_ring_bwd(int32_t layout, int32_t N, int32_t P, int32_t caus
         (s = check_tensor(dv, "dv")) != CP_OK)
         return s;
     if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
-    if (q->dtype != CP_BF16) return fail(CP_ERR_UNSUPPORTED, "the backward takes bf16 tensors");
-    if (q->shape[3] != 128) return fail(CP_ERR_UNSUPPORTED, "the backward supports d = 128");
     if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
         return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
     const int64_t b = q->shape[0], S = q->shape[1], Hq = q->shape[2], Hkv = k->shape[2], d = q->shape[3];
@@ -870,13 +868,13 @@ static cp_status uly_ring_bwd(int32_t layout, int32_t N, int32_t P, int32_t caus
     if (S % 4) return fail(CP_ERR_SHAPE, "S must be a multiple of 4");
     if (S >= ((int64_t)1 << 30)) return fail(CP_ERR_SHAPE, "sequence too long (S must be below 2^30)");
     if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;
-    if (o->dtype != CP_BF16) return fail(CP_ERR_INVALID_ARG, "o must be bf16");
+    const int32_t dt = q->dtype;
     const cp_tensor *like_q[3] = {o, dout, dq};
     for (const cp_tensor *t : like_q)
-        if (!same_shape(t, q) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "o, dout and dq must be bf16 shaped like q");
+        if (!same_shape(t, q) || t->dtype != dt) return fail(CP_ERR_SHAPE, "o, dout and dq must be shaped like q, same dtype");
     const cp_tensor *like_k[2] = {dk, dv};
     for (const cp_tensor *t : like_k)
-        if (!same_shape(t, k) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "dk and dv must be bf16 shaped like k");
+        if (!same_shape(t, k) || t->dtype != dt) return fail(CP_ERR_SHAPE, "dk and dv must be shaped like k, same dtype");
     if (!(lse->stride[2] == 1 && lse->stride[1] == S && (b <= 1 || lse->stride[0] == Hq * S)))
         return fail(CP_ERR_INVALID_ARG, "lse must be contiguous");
     const size_t need = uly_ring_bwd_ws(layout, N, P, q->dtype, b, S, Hq, Hkv, d);
@@ -885,19 +883,20 @@ static cp_status uly_ring_bwd(int32_t layout, int32_t N, int32_t P, int32_t caus
     if (b == 0 || S == 0) return CP_OK;
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
     const int64_t hp = Hq / P, hkp = Hkv / P;
-    const int64_t qb = up(b * S * Hq * d * 2), kb = up(b * S * Hkv * d * 2), lb = up(b * Hq * S * 4);
+    const int64_t es = elem_size(dt);
+    const int64_t qb = up(b * S * Hq * d * es), kb = up(b * S * Hkv * d * es), lb = up(b * Hq * S * 4);
     char *ws = static_cast<char *>(workspace);
     auto qt = [&](int i) {
-        return cp_tensor{ws + i * qb, CP_BF16, 0, {P * b, S, hp, d}, {S * hp * d, hp * d, d, 1}};
+        return cp_tensor{ws + i * qb, dt, 0, {P * b, S, hp, d}, {S * hp * d, hp * d, d, 1}};
     };
     auto kt = [&](int i) {
-        return cp_tensor{ws + 4 * qb + i * kb, CP_BF16, 0, {P * b, S, hkp, d}, {S * hkp * d, hkp * d, d, 1}};
+        return cp_tensor{ws + 4 * qb + i * kb, dt, 0, {P * b, S, hkp, d}, {S * hkp * d, hkp * d, d, 1}};
     };
     cp_tensor qh = qt(0), oh = qt(1), doh = qt(2), dqh = qt(3);
     cp_tensor kh = kt(0), vh = kt(1), dkh = kt(2), dvh = kt(3);
     cp_tensor lh{ws + 4 * qb + 4 * kb, CP_FP32, 0, {P * b, hp, S, 1}, {hp * S, S, 1, 1}};
     char *ws_ring = ws + 4 * qb + 4 * kb + lb;
-    const size_t ring_need = cp_ring_bwd_workspace_bytes(layout, N, CP_BF16, P * b, S, hp, d);
+    const size_t ring_need = cp_ring_bwd_workspace_bytes(layout, N, dt, P * b, S, hp, d);
     // exchange in: q, k, v, o, dout and lse to the head-sharded layout
     const cp_tensor *ins[5] = {q, k, v, o, dout};
     cp_tensor *outs[5] = {&qh, &kh, &vh, &oh, &doh};
@@ -1102,8 +1101,10 @@ cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_t
         (s = check_tensor(dv, "dv")) != CP_OK)
         return s;
     if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
-    if (q->dtype != CP_BF16) return fail(CP_ERR_UNSUPPORTED, "the backward takes bf16 tensors");
-    if (q->shape[3] != 128) return fail(CP_ERR_UNSUPPORTED, "the backward supports d = 128");
+    // bf16 with d = 128 runs on the tensor cores; fp32 (d 64 or 128) and bf16 with
+    // d = 64 on the FFMA backward
+    const cp_dtype dt = static_cast<cp_dtype>(q->dtype);
+    const bool tc_path = dt == CP_BF16 && q->shape[3] == 128;
     if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
         return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
     const int64_t S = q->shape[1];
@@ -1113,15 +1114,15 @@ cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     if (S % N) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of N = %d", (long long)S, N);
     if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N)) return fail(CP_ERR_SHAPE, "zig-zag needs S to be a multiple of 2N");
     if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;
-    if (o->dtype != CP_BF16) return fail(CP_ERR_INVALID_ARG, "o must be bf16");
+    if (o->dtype != dt) return fail(CP_ERR_INVALID_ARG, "o must have q's dtype");
     const cp_tensor *like_q[2] = {dout, dq};
     for (const cp_tensor *t : like_q) {
-        if (!same_shape(t, q) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "dout and dq must be bf16 shaped like q");
+        if (!same_shape(t, q) || t->dtype != dt) return fail(CP_ERR_SHAPE, "dout and dq must be shaped like q, same dtype");
         if ((s = check_rows16(t, t == dq ? "dq" : "dout")) != CP_OK) return s;
     }
     const cp_tensor *like_k[2] = {dk, dv};
     for (const cp_tensor *t : like_k) {
-        if (!same_shape(t, k) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "dk and dv must be bf16 shaped like k");
+        if (!same_shape(t, k) || t->dtype != dt) return fail(CP_ERR_SHAPE, "dk and dv must be shaped like k, same dtype");
         if ((s = check_rows16(t, t == dk ? "dk" : "dv")) != CP_OK) return s;
     }
     const int64_t c = S / N;
@@ -1174,6 +1175,11 @@ cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     p.status = word;
     p.n_kt = (int)n_kt;
     p.n_kv_blocks = N;
+    if (!tc_path) {
+        cudaError_t e = launch_attn_bwd_simt(p, dt == CP_FP32, static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+        return CP_OK;
+    }
     const std::vector<uint32_t> &ord = bwd_order(layout, N, S, causal);
     if ((int64_t)ord.size() <= kMaxOrder) {
         p.order_len = (int)ord.size();

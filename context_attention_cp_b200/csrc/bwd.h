@@ -103,4 +103,9 @@ struct BwdParams {
 // Statistics + dq_acc zeroing, the main tcgen05 kernel, then dq_acc -> dq.
 cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream);
 
+// The FFMA backward (attn_simt_bwd.cu) for fp32 inputs or bf16 with d = 64: the ring
+// layout only (use_layout = 1, kv_explicit = 0, no documents); uses p.stats as its
+// (lse, D) table and leaves dq_acc untouched.
+cudaError_t launch_attn_bwd_simt(const BwdParams &p, bool fp32, cudaStream_t stream);
+
 }  // namespace cpattn

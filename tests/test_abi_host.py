@@ -233,9 +233,11 @@ def test_ring_bwd_argument_errors_are_synchronous(cp):
     assert call(causal=2) == 1                             # causal flag
     assert call(wsb=16) == 1                               # workspace too small
     assert call(ws=0x100010) == 1                          # workspace alignment
-    assert call(q_=_ct(cp, [1, 256, 4, 64]), k_=_ct(cp, [1, 256, 2, 64])) == 2  # d = 64 unsupported
+    assert call(q_=_ct(cp, [1, 256, 4, 256]), k_=_ct(cp, [1, 256, 2, 256])) == 2  # d = 256 unsupported
     qf = _ct(cp, [1, 256, 4, 128], dtype=1)
-    assert call(q_=qf, k_=_ct(cp, [1, 256, 2, 128], dtype=1)) == 2             # fp32 unsupported
+    assert call(q_=qf, k_=_ct(cp, [1, 256, 2, 128], dtype=1)) == 1             # fp32 q with a bf16 o
+    assert call(q_=qf, k_=_ct(cp, [1, 256, 2, 128], dtype=1), o_=_ct(cp, [1, 256, 4, 128], dtype=1),
+                do_=qf) == 3                                                    # bf16 dq for fp32 q
     assert call(dk_=_ct(cp, [1, 256, 4, 128])) == 3        # dk shaped like q
     assert call(lse_=_ct(cp, [1, 4, 255, 1], dtype=1)) == 3
     assert cp.lib().cp_ring_bwd_workspace_bytes(1, 3, 0, 1, 256, 4, 128) == 0  # S % N
@@ -316,4 +318,4 @@ def test_usp_argument_errors_are_synchronous(cp):
     qf, kf = _ct(cp, [1, 64, 8, 128], dtype=1), _ct(cp, [1, 64, 2, 128], dtype=1)
     of = _ct(cp, [1, 64, 8, 128], dtype=1)
     assert g(1, 2, 2, 1, *[ctypes.byref(t) for t in (qf, kf, kf, of, lse, of)], ctypes.c_float(0.1),
-             *[ctypes.byref(t) for t in (of, kf, kf)], ctypes.c_void_p(0x100000), 1 << 30, None) == 2  # bf16 only
+             *[ctypes.byref(t) for t in (q, kf, kf)], ctypes.c_void_p(0x100000), 1 << 30, None) == 3  # dq dtype

@@ -79,6 +79,51 @@ def test_ring_bwd_matches_oracle(cp, case):
         _assert_grad(np64(g), w, name)
 
 
+# The FFMA backward: fp32 inputs (d 64 and 128) and bf16 with d = 64.  fp32 bar: the
+# forward's o and lse enter with at most 1e-4 / 1e-5 absolute error (the forward's
+# fp32 bar), which reaches p = e^{x - lse} and D = dO . o as relative errors of that
+# size; every product and sum is fp32 (unit roundoff 2^-24, at most S terms per
+# sum).  So  max |got - ref| <= 1e-4 * max |ref|  per gradient tensor.  bf16 with
+# d = 64 computes in fp32 and rounds once to bf16: the bf16 bar above.
+TOL_REL_FP32 = 1e-4
+
+FFMA_CASES = [
+    # layout, N, S, causal, b, hq, hkv, d, dtype
+    ("contiguous", 2, 256, True, 1, 2, 2, 64, "fp32"),
+    ("zigzag", 4, 512, True, 2, 4, 2, 128, "fp32"),
+    ("striped", 3, 390, True, 1, 4, 1, 64, "fp32"),     # c = 130: ragged tiles
+    ("contiguous", 2, 256, False, 1, 2, 2, 64, "fp32"),
+    ("zigzag", 2, 424, True, 1, 4, 2, 64, "bf16"),
+    ("contiguous", 1, 200, True, 1, 2, 1, 64, "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", FFMA_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_ring_bwd_ffma_matches_oracle(cp, case):
+    layout, N, S, causal, b, hq, hkv, d, dt = case
+    q, k, v = W.random_qkv(b, S, hq, hkv, d, dt, seed=S + 7 * N + d)
+    do = W.random_do(b, S, hq, d, dt, seed=S + 7 * N + d)
+    dq, dk, dv = _fwd_bwd(cp, q, k, v, do, layout, N, causal, d ** -0.5)
+    want = oracle.ring_attention_bwd(np64(q), np64(k), np64(v), np64(do), layout, N, causal, d ** -0.5)
+    tol = TOL_REL_FP32 if dt == "fp32" else TOL_REL
+    for name, g, w in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
+        assert g.dtype == q.dtype
+        err = np.max(np.abs(np64(g) - w))
+        assert err <= tol * np.max(np.abs(w)), (name, err, np.max(np.abs(w)))
+
+
+def test_fp32_workload_bwd_element_by_element(cp):
+    """The fp32 workload (S = 256, contiguous N = 2, d = 64) at its full size."""
+    w = W.BY_NAME["fp32_s256_contig2"]
+    q, k, v = W.make_inputs(w)
+    do = W.make_do(w)
+    dq, dk, dv = _fwd_bwd(cp, q, k, v, do, w.layout, w.N, w.causal, w.scale)
+    want = oracle.ring_attention_bwd(np64(q), np64(k), np64(v), np64(do), w.layout, w.N, w.causal, w.scale)
+    for name, g, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
+        err = np.max(np.abs(np64(g) - ref))
+        assert err <= TOL_REL_FP32 * np.max(np.abs(ref)), (name, err)
+
+
 def test_ring_bwd_dkdv_deterministic(cp):
     q, k, v = W.random_qkv(1, 2048, 8, 2, 128, "bf16", seed=77)
     do = W.random_do(1, 2048, 8, 128, "bf16", seed=77)
@@ -106,9 +151,10 @@ def test_ring_bwd_argument_errors(cp):
     with pytest.raises(cp.CPError) as e:
         cp.ring_attn_bwd(q, k, v, o, lse, q, "zigzag", 3, True)
     assert e.value.code == 3
-    q64 = torch.zeros((1, 256, 4, 64), dtype=torch.bfloat16, device="cuda")
+    q256 = torch.zeros((1, 256, 4, 256), dtype=torch.bfloat16, device="cuda")
+    k256 = torch.zeros((1, 256, 2, 256), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(cp.CPError) as e:
-        cp.ring_attn_bwd(q64, q64[:, :, :2], q64[:, :, :2], q64, lse, q64, "zigzag", 2, True)
+        cp.ring_attn_bwd(q256, k256, k256, q256, lse, q256, "zigzag", 2, True)   # head dim 256
     assert e.value.code == 2
     with pytest.raises(cp.CPError):
         cp.ring_attn_bwd(q, k, v, o, lse[:, :, :128], q, "zigzag", 2, True)

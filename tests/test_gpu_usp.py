@@ -92,6 +92,23 @@ def test_usp_bwd_matches_oracle(cp, layout, N, P, b, S, hq, hkv, causal):
         assert err <= 2e-2 * np.max(np.abs(w)), (name, err, np.max(np.abs(w)))
 
 
+@pytest.mark.parametrize("layout,N,P,d", [("zigzag", 2, 2, 64), ("contiguous", 1, 2, 128)])
+def test_usp_bwd_fp32_matches_oracle(cp, layout, N, P, d):
+    """fp32 through the FFMA backward (N = 1: plain Ulysses), 1e-4 x max |ref|."""
+    b, S, hq, hkv = 1, 256, 4, 2
+    q, k, v = W.random_qkv(b, S, hq, hkv, d, "fp32", seed=S + N + d)
+    do = W.random_do(b, S, hq, d, "fp32", seed=S + N + d)
+    qr, kr, vr, dor = (cp.layout_permute(t.cuda(), layout, N) for t in (q, k, v, do))
+    o, lse = cp.usp_attn_fwd(qr, kr, vr, layout, N, P, True)
+    grads = cp.usp_attn_bwd(qr, kr, vr, o, lse, dor, layout, N, P, True)
+    grads = [cp.layout_permute(g, layout, N, inverse=True) for g in grads]
+    cp.stream_check()
+    want = oracle.usp_attention_bwd(np64(q), np64(k), np64(v), np64(do), layout, N, P, True, d ** -0.5)
+    for name, g, w in zip(("dq", "dk", "dv"), grads, want):
+        err = np.max(np.abs(np64(g) - w))
+        assert err <= 1e-4 * np.max(np.abs(w)), (name, err, np.max(np.abs(w)))
+
+
 def test_usp_argument_errors(cp):
     q, k, v = (t.cuda() for t in W.random_qkv(1, 256, 8, 2, 128, "bf16", seed=2))
     with pytest.raises(cp.CPError) as e:
@@ -100,11 +117,10 @@ def test_usp_argument_errors(cp):
     with pytest.raises(cp.CPError) as e:
         cp.usp_attn_fwd(q, k, v, "zigzag", 3, 2, True)    # 256 % (3 * 2)
     assert e.value.code == 3
-    qf, kf, vf = (t.cuda() for t in W.random_qkv(1, 256, 4, 2, 128, "fp32", seed=2))
-    o, lse = cp.usp_attn_fwd(qf, kf, vf, "zigzag", 2, 2, True)
+    o, lse = cp.usp_attn_fwd(q, k, v, "zigzag", 2, 2, True)
     with pytest.raises(cp.CPError) as e:
-        cp.usp_attn_bwd(qf, kf, vf, o, lse, qf, "zigzag", 2, 2, True)   # the backward is bf16 only
-    assert e.value.code == 2
+        cp.usp_attn_bwd(q, k, v, o.float(), lse, q, "zigzag", 2, 2, True)   # o in another dtype
+    assert e.value.code == 3
     cp.stream_check()
 
 
