@@ -223,8 +223,9 @@ size_t cp_ulysses_workspace_bytes(int32_t P, int32_t dtype, int64_t b, int64_t S
  * layout, the ring backward with N = 1 over every rank's head group (the same
  * kernels as cp_ring_attn_bwd), and the exchange of dq, dk, dv back.
  *   Tensors in original order as for cp_ulysses_attn_fwd (o and lse its results);
- *   dq [b, S, Hq, d], dk / dv [b, S, Hkv, d] bf16 outputs; all contiguous.
- *   Requires bf16, d = 128 and the conditions of cp_ulysses_attn_fwd.
+ *   dq [b, S, Hq, d], dk / dv [b, S, Hkv, d] outputs in q's dtype; all contiguous.
+ *   The dtypes and head dims of cp_ring_attn_bwd and the conditions of
+ *   cp_ulysses_attn_fwd.
  *   workspace: cp_ulysses_bwd_workspace_bytes(...) bytes, 256-byte aligned. */
 cp_status cp_ulysses_attn_bwd(int32_t P, int32_t causal, const cp_tensor *q, const cp_tensor *k,
                               const cp_tensor *v, const cp_tensor *o, const cp_tensor *lse,
@@ -265,8 +266,9 @@ size_t cp_usp_workspace_bytes(int32_t layout, int32_t N, int32_t P, int32_t dtyp
  * ring backward over the N groups for every head group (the kernels of
  * cp_ring_attn_bwd; dK, dV travel with their block), the exchange of dq, dk, dv
  * back.  Tensors as for cp_usp_attn_fwd (o and lse its results); dq [b, S, Hq, d],
- * dk / dv [b, S, Hkv, d] bf16 outputs in the same order; all contiguous.  Requires
- * bf16, d = 128 and the conditions of cp_usp_attn_fwd.
+ * dk / dv [b, S, Hkv, d] outputs in q's dtype and the same order; all contiguous.
+ * The dtypes and head dims of cp_ring_attn_bwd and the conditions of
+ * cp_usp_attn_fwd.
  *   workspace: cp_usp_bwd_workspace_bytes(...) bytes, 256-byte aligned. */
 cp_status cp_usp_attn_bwd(int32_t layout, int32_t N, int32_t P, int32_t causal, const cp_tensor *q,
                           const cp_tensor *k, const cp_tensor *v, const cp_tensor *o, const cp_tensor *lse,
@@ -289,14 +291,17 @@ size_t cp_usp_bwd_workspace_bytes(int32_t layout, int32_t N, int32_t P, int32_t 
  *   q, o, dout [b, S, Hq, d]; k, v [b, S, Hkv, d]; lse [b, Hq, S, 1] fp32; all in
  *   rank-major order, as cp_ring_attn_fwd takes and returns them (o and lse are its
  *   results for the same q, k, v, layout, N, causal and softmax_scale).
- *   dq [b, S, Hq, d], dk / dv [b, S, Hkv, d]: outputs (bf16, rank-major), overwritten.
+ *   dq [b, S, Hq, d], dk / dv [b, S, Hkv, d]: outputs (q's dtype, rank-major), overwritten.
  *   workspace: device memory of at least cp_ring_bwd_workspace_bytes(...) bytes,
  *   256-byte aligned (row statistics and the fp32 dQ accumulator); the caller keeps
  *   it alive until the work on `stream` has finished.
- * Requires bf16 tensors and d = 128 (CP_ERR_UNSUPPORTED otherwise) besides the
- * conditions of cp_ring_attn_fwd.  Rows whose lse is -inf contribute nothing.
- * dq sums its shares with fp32 atomic reductions, so its rounding can differ from
- * run to run; dk and dv are summed in a fixed order. */
+ * All tensors but lse share q's dtype.  bf16 with d = 128 runs the tensor-core
+ * kernel; fp32 (d = 64 or 128) and bf16 with d = 64 run FFMA kernels (fp32
+ * arithmetic, results rounded once to the dtype).  Besides that the conditions of
+ * cp_ring_attn_fwd.  Rows whose lse is -inf contribute nothing.  On the tensor-core
+ * path dq sums its shares with fp32 atomic reductions, so its rounding can differ
+ * from run to run; dk and dv are summed in a fixed order (every output of the FFMA
+ * path is). */
 cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q,
                            const cp_tensor *k, const cp_tensor *v, const cp_tensor *o,
                            const cp_tensor *lse, const cp_tensor *dout, float softmax_scale,
