@@ -319,3 +319,31 @@ def test_usp_argument_errors_are_synchronous(cp):
     of = _ct(cp, [1, 64, 8, 128], dtype=1)
     assert g(1, 2, 2, 1, *[ctypes.byref(t) for t in (qf, kf, kf, of, lse, of)], ctypes.c_float(0.1),
              *[ctypes.byref(t) for t in (q, kf, kf)], ctypes.c_void_p(0x100000), 1 << 30, None) == 3  # dq dtype
+
+
+@pytest.mark.parametrize("b,S", [(0, 256), (1, 0)])
+def test_empty_inputs_return_ok_without_device_work(cp, b, S):
+    """Empty batches or sequences are valid and launch nothing: on this host (no
+    device) any launch or device query would come back as CP_ERR_CUDA."""
+    L = cp.lib()
+    q = _ct(cp, [b, S, 4, 128])
+    k = _ct(cp, [b, S, 2, 128], data=0x20000)
+    o = _ct(cp, [b, S, 4, 128], data=0x30000)
+    lse = _ct(cp, [b, 4, S, 1], dtype=1, data=0x40000)
+    ws = ctypes.c_void_p(0x100000)
+    r = lambda *ts: [ctypes.byref(t) for t in ts]  # noqa: E731
+    sc = ctypes.c_float(0.1)
+    docs = (ctypes.c_int64 * 1)(0)
+    calls = {
+        "ring_fwd": L.cp_ring_attn_fwd(1, 2, 1, *r(q, k, k), sc, *r(o, lse), 0, ws, 1 << 30, None),
+        "ring_bwd": L.cp_ring_attn_bwd(1, 2, 1, *r(q, k, k, o, lse, q), sc, *r(o, k, k), ws, 1 << 30, None),
+        "allgather_fwd": L.cp_allgather_attn_fwd(1, 2, 1, *r(q, k, k), docs, 1, sc, *r(o, lse), ws, 1 << 30, None),
+        "allgather_bwd": L.cp_allgather_attn_bwd(1, 2, 1, *r(q, k, k, o, lse, q), docs, 1, sc, *r(o, k, k), ws,
+                                                 1 << 30, None),
+        "ulysses_fwd": L.cp_ulysses_attn_fwd(2, 1, *r(q, k, k), sc, *r(o, lse), ws, 1 << 30, None),
+        "ulysses_bwd": L.cp_ulysses_attn_bwd(2, 1, *r(q, k, k, o, lse, q), sc, *r(o, k, k), ws, 1 << 30, None),
+        "usp_fwd": L.cp_usp_attn_fwd(1, 2, 2, 1, *r(q, k, k), sc, *r(o, lse), ws, 1 << 30, None),
+        "usp_bwd": L.cp_usp_attn_bwd(1, 2, 2, 1, *r(q, k, k, o, lse, q), sc, *r(o, k, k), ws, 1 << 30, None),
+        "permute": L.cp_layout_permute(1, 2, 1, *r(q, o), 0, None),
+    }
+    assert all(v == 0 for v in calls.values()), calls
