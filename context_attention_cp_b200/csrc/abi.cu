@@ -691,8 +691,9 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
         (s = check_tensor(dv, "dv")) != CP_OK)
         return s;
     if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
-    if (q->dtype != CP_BF16) return fail(CP_ERR_UNSUPPORTED, "the backward takes bf16 tensors");
-    if (q->shape[3] != 128) return fail(CP_ERR_UNSUPPORTED, "the backward supports d = 128");
+    // bf16 with d = 128 on the tensor cores, fp32 and bf16 d = 64 on the FFMA kernels
+    const int32_t dt = q->dtype;
+    const bool tc_path = dt == CP_BF16 && q->shape[3] == 128;
     if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
         return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
     const int64_t S = q->shape[1];
@@ -702,15 +703,15 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     if (S % N) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of N = %d", (long long)S, N);
     if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N)) return fail(CP_ERR_SHAPE, "zig-zag needs S to be a multiple of 2N");
     if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;
-    if (o->dtype != CP_BF16) return fail(CP_ERR_INVALID_ARG, "o must be bf16");
+    if (o->dtype != dt) return fail(CP_ERR_INVALID_ARG, "o must have q's dtype");
     const cp_tensor *like_q[2] = {dout, dq};
     for (const cp_tensor *t : like_q) {
-        if (!same_shape(t, q) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "dout and dq must be bf16 shaped like q");
+        if (!same_shape(t, q) || t->dtype != dt) return fail(CP_ERR_SHAPE, "dout and dq must be shaped like q, same dtype");
         if ((s = check_rows16(t, t == dq ? "dq" : "dout")) != CP_OK) return s;
     }
     const cp_tensor *like_k[4] = {k, v, dk, dv};
     for (const cp_tensor *t : like_k) {
-        if (!same_shape(t, k) || t->dtype != CP_BF16) return fail(CP_ERR_SHAPE, "dk and dv must be bf16 shaped like k");
+        if (!same_shape(t, k) || t->dtype != dt) return fail(CP_ERR_SHAPE, "dk and dv must be shaped like k, same dtype");
         int64_t expect = 1;
         for (int i = 3; i >= 0; --i) {
             if (t->shape[i] > 1 && t->stride[i] != expect)
@@ -735,9 +736,9 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
     char *ws = static_cast<char *>(workspace);
-    const int64_t kb = up(b * S * Hkv * d * 2);
+    const int64_t kb = up(b * S * Hkv * d * elem_size(dt));
     auto kv_t = [&](int i) {
-        return cp_tensor{ws + i * kb, CP_BF16, 0, {b, S, Hkv, d}, {S * Hkv * d, Hkv * d, d, 1}};
+        return cp_tensor{ws + i * kb, dt, 0, {b, S, Hkv, d}, {S * Hkv * d, Hkv * d, d, 1}};
     };
     cp_tensor kg = kv_t(0), vg = kv_t(1), dkg = kv_t(2), dvg = kv_t(3);
     int *docs_dev = reinterpret_cast<int *>(ws + 4 * kb);
@@ -795,6 +796,13 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     status_word(&word);
     p.status = word;
     p.n_kt = (int)n_kt;
+    if (!tc_path) {
+        e = launch_attn_bwd_simt(p, dt == CP_FP32, st);
+        if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+        if ((s = cp_layout_permute(layout, N, 1, &dkg, dk, 0, stream)) != CP_OK) return s;
+        if ((s = cp_layout_permute(layout, N, 1, &dvg, dv, 0, stream)) != CP_OK) return s;
+        return CP_OK;
+    }
     // work order: the key tiles of the gathered block, earliest (most queries) first
     if (n_kt <= kMaxOrder) {
         p.order_len = (int)n_kt;
@@ -956,7 +964,6 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
         (s = check_tensor(v, "v")) != CP_OK)
         return s;
     if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
-    if (q->dtype != CP_BF16) return fail(CP_ERR_UNSUPPORTED, "the All-Gather path takes bf16 tensors");
     if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
         return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
     const int64_t S = q->shape[1];

@@ -9,6 +9,9 @@
 // the running (m, l, O) into the step partial o_b = O / l, lse_b = m + log l, and
 // merges it into the running result with the LSE merge.  Fully masked key tiles
 // are skipped; partial tiles are masked key by key on original positions.
+// The All-Gather form (kv_explicit: one gathered key block in original order) and
+// its document mask (section All-Gather 式 CP: a query sees only keys of its own
+// document) are honoured key by key.
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -20,6 +23,17 @@ namespace {
 
 constexpr int RM = 128;  // query rows per CTA
 constexpr int RN = 32;   // keys per shared-memory tile
+
+// Document start of position pos: the last of the sorted starts that is <= pos.
+__device__ __forceinline__ int64_t simt_doc_start(const int *starts, int n, int64_t pos)
+{
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if ((int64_t)starts[mid] <= pos) lo = mid + 1; else hi = mid;
+    }
+    return lo > 0 ? (int64_t)starts[lo - 1] : 0;
+}
 
 template <int D>
 struct SimtCfg {
@@ -60,6 +74,7 @@ __global__ void __launch_bounds__(RM) attn_simt_kernel(const __grid_constant__ A
     const bool row_ok = row < p.q_len;
     const Range qr = p.use_layout ? layout_range(p.layout, p.n_ranks, p.seq_len, rank) : p.q_range;
     const int64_t pos_q = range_pos(qr, row_ok ? row : p.q_len - 1);
+    const int64_t ds_q = p.n_docs > 0 ? simt_doc_start(p.doc_starts, p.n_docs, pos_q) : 0;
 
     const float *Q = reinterpret_cast<const float *>(p.q);
     const float *K = reinterpret_cast<const float *>(p.k);
@@ -80,7 +95,7 @@ __global__ void __launch_bounds__(RM) attn_simt_kernel(const __grid_constant__ A
     for (int step = p.step_begin; step < p.step_end; ++step) {
         const int N = p.n_ranks;
         const int src = ((rank - step) % N + N) % N;
-        const Range kr = p.use_layout ? layout_range(p.layout, N, p.seq_len, src) : p.kv_range;
+        const Range kr = (p.use_layout && !p.kv_explicit) ? layout_range(p.layout, N, p.seq_len, src) : p.kv_range;
         int kt_full, kt_end;
         kv_tile_bounds<int64_t>(qr, p.q_len, q_lo, RM, kr, p.kv_len, RN, p.causal != 0, &kt_full, &kt_end);
         if (kt_end == 0) continue;
@@ -109,6 +124,7 @@ __global__ void __launch_bounds__(RM) attn_simt_kernel(const __grid_constant__ A
                 const int key = k0 + j;
                 if (key >= p.kv_len) break;
                 if (p.causal && kt >= kt_full && range_pos(kr, key) > pos_q) continue;
+                if (p.n_docs > 0 && range_pos(kr, key) < ds_q) continue;
                 float x = 0.f;
 #pragma unroll 16
                 for (int i = 0; i < D; ++i) x = fmaf(q_s[tid * C::LD + i], k_s[j * D + i], x);

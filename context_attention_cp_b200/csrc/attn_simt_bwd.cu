@@ -21,6 +21,9 @@
 //      key row; every query head of the group and every query rank's rows that see
 //      the tile stream through shared memory 32 rows at a time.  One pass per
 //      gradient keeps a single d-vector accumulator in registers.
+// The All-Gather form (kv_explicit: one gathered key block in original order, met
+// by every query rank) and its document mask (a query sees only keys of its own
+// document; section All-Gather 式 CP) are honoured key by key.
 // Nothing waits on another CTA, so there is no bounded wait to report.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -50,6 +53,19 @@ struct SbCfg {
     static constexpr int FLOATS = OFF_ST + 2 * SRN;
     static constexpr int SMEM = FLOATS * 4;
 };
+
+// Document of position pos: [start, end) from the sorted starts (end = seq_len for
+// the last document).
+__device__ __forceinline__ void doc_bounds(const BwdParams &p, int64_t pos, int64_t *start, int64_t *end)
+{
+    int lo = 0, hi = p.n_docs;  // first start > pos
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if ((int64_t)p.doc_starts[mid] <= pos) lo = mid + 1; else hi = mid;
+    }
+    *start = lo > 0 ? (int64_t)p.doc_starts[lo - 1] : 0;
+    *end = lo < p.n_docs ? (int64_t)p.doc_starts[lo] : p.seq_len;
+}
 
 __device__ __forceinline__ int64_t stat_index(const BwdParams &p, int bb, int h, int rank, int t)
 {
@@ -96,6 +112,8 @@ __global__ void __launch_bounds__(SRM) simt_bwd_dq_kernel(const __grid_constant_
     const Range qr = layout_range(p.layout, p.n_ranks, p.seq_len, rank);
     const int64_t pos_q = range_pos(qr, (int64_t)(row_ok ? row : p.q_len - 1));
     const int64_t grow = (int64_t)rank * p.q_row_step + (row_ok ? row : 0);
+    int64_t ds_q = 0, de_q = 0;
+    if (p.n_docs > 0) doc_bounds(p, pos_q, &ds_q, &de_q);
 
     {
         const T *qs = static_cast<const T *>(p.q) + bb * p.q_sb + grow * p.q_ss + (int64_t)h * p.q_sh;
@@ -115,10 +133,12 @@ __global__ void __launch_bounds__(SRM) simt_bwd_dq_kernel(const __grid_constant_
 #pragma unroll
     for (int i = 0; i < D; ++i) dq[i] = 0.f;
 
-    for (int step = 0; step < p.n_ranks; ++step) {
+    // the ring: every step's block; the All-Gather form: the one gathered block
+    const int n_steps = p.kv_explicit ? 1 : p.n_ranks;
+    for (int step = 0; step < n_steps; ++step) {
         const int N = p.n_ranks;
-        const int src = ((rank - step) % N + N) % N;
-        const Range kr = layout_range(p.layout, N, p.seq_len, src);
+        const int src = p.kv_explicit ? 0 : ((rank - step) % N + N) % N;
+        const Range kr = p.kv_explicit ? p.kv_range : layout_range(p.layout, N, p.seq_len, src);
         int kt_full, kt_end;
         kv_tile_bounds<int64_t>(qr, p.q_len, q_lo, SRM, kr, p.kv_len, SRN, p.causal != 0, &kt_full, &kt_end);
         for (int kt = 0; kt < kt_end; ++kt) {
@@ -142,6 +162,7 @@ __global__ void __launch_bounds__(SRM) simt_bwd_dq_kernel(const __grid_constant_
                 const int key = k0 + j;
                 if (key >= p.kv_len) break;
                 if (p.causal && kt >= kt_full && range_pos(kr, (int64_t)key) > pos_q) continue;
+                if (p.n_docs > 0 && range_pos(kr, (int64_t)key) < ds_q) continue;
                 float x = 0.f, dp = 0.f;
 #pragma unroll 16
                 for (int i = 0; i < D; ++i) {
@@ -180,9 +201,11 @@ __global__ void __launch_bounds__(SRM) simt_bwd_dkv_kernel(const __grid_constant
     const int key = k_lo + tid;
     const bool key_ok = key < p.kv_len;
     const int N = p.n_ranks;
-    const Range kr = layout_range(p.layout, N, p.seq_len, j);
+    const Range kr = p.kv_explicit ? p.kv_range : layout_range(p.layout, N, p.seq_len, j);
     const int64_t pos_k = range_pos(kr, (int64_t)(key_ok ? key : p.kv_len - 1));
     const int64_t krow = (int64_t)j * p.kv_row_step + (key_ok ? key : 0);
+    int64_t ds_k = 0, de_k = INT64_MAX;  // queries at or past de_k lie in a later document
+    if (p.n_docs > 0) doc_bounds(p, pos_k, &ds_k, &de_k);
 
     {
         const T *ks = static_cast<const T *>(p.k) + bb * p.k_sb + krow * p.k_ss + (int64_t)hk * p.k_sh;
@@ -235,6 +258,7 @@ __global__ void __launch_bounds__(SRM) simt_bwd_dkv_kernel(const __grid_constant
                     const float2 st = st_s[i];
                     if (st.x == -INFINITY) continue;
                     if (p.causal && qt < qt_full && pos_k > range_pos(qr, (int64_t)row)) continue;
+                    if (p.n_docs > 0 && range_pos(qr, (int64_t)row) >= de_k) continue;
                     float x = 0.f, dp = 0.f;
 #pragma unroll 16
                     for (int c = 0; c < D; ++c) {
@@ -284,7 +308,7 @@ cudaError_t launch_simt_bwd_t(const BwdParams &p, cudaStream_t st)
     simt_bwd_stats_kernel<T, D><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(p);
     const int64_t n_qt = (p.q_len + SRM - 1) / SRM, n_kt = (p.kv_len + SRM - 1) / SRM;
     simt_bwd_dq_kernel<T, D><<<(unsigned)(p.n_ranks * n_qt * p.b * p.hq), SRM, C::SMEM, st>>>(p);
-    const unsigned kv_items = (unsigned)(p.n_ranks * n_kt * p.b * p.hkv);
+    const unsigned kv_items = (unsigned)(p.n_kv_blocks * n_kt * p.b * p.hkv);
     simt_bwd_dkv_kernel<T, D, false><<<kv_items, SRM, C::SMEM, st>>>(p);
     simt_bwd_dkv_kernel<T, D, true><<<kv_items, SRM, C::SMEM, st>>>(p);
     return cudaGetLastError();

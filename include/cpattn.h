@@ -152,9 +152,9 @@ size_t cp_ring_workspace_bytes(int32_t layout, int32_t N, int32_t mode, int32_t 
  * pass, with an optional document mask (documents packed into one sequence do not
  * see each other) -- the mask the page gives as the reason to gather instead of
  * ringing.
- *   q [b, S, Hq, d], k / v [b, S, Hkv, d]: bf16, rank-major (as for
- *   cp_ring_attn_fwd); k and v contiguous.  o [b, S, Hq, d] bf16 and lse
- *   [b, Hq, S, 1] fp32 come out rank-major.
+ *   q [b, S, Hq, d], k / v [b, S, Hkv, d]: bf16 (tensor cores) or fp32 (FFMA),
+ *   d = 64 or 128, rank-major (as for cp_ring_attn_fwd); k and v contiguous.
+ *   o [b, S, Hq, d] in q's dtype and lse [b, Hq, S, 1] fp32 come out rank-major.
  *   doc_starts: HOST array of n_docs first positions (original order), strictly
  *   increasing, doc_starts[0] = 0, all < S; n_docs = 1 means no document mask.
  *   Key t is visible to query p iff pos_k(t) <= pos_q(p) (causal) and both lie in
@@ -172,8 +172,9 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
  * the backward): K and V gathered again, every rank's queries against the whole
  * sequence with the same document mask, the summed dK, dV handed back to each
  * rank's block.  Arguments as cp_allgather_attn_fwd (o and lse its results) plus
- * dout [b, S, Hq, d]; dq [b, S, Hq, d], dk / dv [b, S, Hkv, d] bf16 outputs, all
- * rank-major; k, v, dk, dv contiguous.  Requires bf16 and d = 128.
+ * dout [b, S, Hq, d]; dq [b, S, Hq, d], dk / dv [b, S, Hkv, d] outputs in q's
+ * dtype, all rank-major; k, v, dk, dv contiguous.  The dtypes and head dims of
+ * cp_ring_attn_bwd (bf16 d = 128 on the tensor cores, the rest on FFMA kernels).
  *   workspace: cp_allgather_bwd_workspace_bytes(...) bytes, 256-byte aligned. */
 cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q,
                                 const cp_tensor *k, const cp_tensor *v, const cp_tensor *o,

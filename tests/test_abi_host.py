@@ -266,7 +266,9 @@ def test_allgather_argument_errors_are_synchronous(cp):
     assert call([0, 100], wsb=64) == 1           # workspace too small
     assert call([0, 100], ws=0x100040) == 1      # workspace alignment
     qf, kf = _ct(cp, [1, 256, 4, 128], dtype=1), _ct(cp, [1, 256, 2, 128], dtype=1)
-    assert call([0], q_=qf, k_=kf) == 2          # bf16 only
+    assert call([0], q_=qf, k_=kf) == 1          # fp32 q with a bf16 o
+    q256, k256 = _ct(cp, [1, 256, 4, 256]), _ct(cp, [1, 256, 2, 256])
+    assert call([0], q_=q256, k_=k256) == 2      # head dim 256
     assert cp.lib().cp_allgather_workspace_bytes(2, 0, 1, 256, 2, 128, 0) == 0
 
 

@@ -54,6 +54,28 @@ def test_allgather_matches_oracle(cp, case):
     assert_close_o(np64(o), ro, tol_o)
 
 
+OTHER_CASES = [
+    # layout, N, S, b, hq, hkv, d, dtype, document starts: the FFMA kernels (fp32) and
+    # the tensor-core kernel's d = 64 instantiation
+    ("zigzag", 4, 512, 1, 4, 2, 64, "fp32", [0, 100, 101, 400]),
+    ("striped", 2, 260, 2, 2, 1, 128, "fp32", [0, 7, 130]),
+    ("contiguous", 3, 390, 1, 2, 2, 64, "fp32", [0]),
+    ("zigzag", 2, 424, 1, 4, 2, 64, "bf16", [0, 5, 211, 212, 300]),
+]
+
+
+@pytest.mark.parametrize("case", OTHER_CASES, ids=lambda c: "-".join(str(x) for x in c[:8]) + "-d%d" % len(c[8]))
+def test_allgather_fp32_and_d64_match_oracle(cp, case):
+    layout, N, S, b, hq, hkv, d, dt, docs = case
+    q, k, v = W.random_qkv(b, S, hq, hkv, d, dt, seed=S + N + d)
+    o, lse = _allgather(cp, q, k, v, layout, N, True, docs)
+    assert o.dtype == q.dtype
+    ro, rl = oracle.allgather_attention(np64(q), np64(k), np64(v), layout, N, True, d ** -0.5, docs)
+    tol_o, tol_l = TOL[dt]
+    assert_close_lse(np64(lse), rl, tol_l)
+    assert_close_o(np64(o), ro, tol_o)
+
+
 def test_allgather_without_documents_matches_ring(cp):
     q, k, v = W.random_qkv(1, 2048, 8, 2, 128, "bf16", seed=5)
     o1, l1 = _allgather(cp, q, k, v, "zigzag", 4, True, None)
@@ -87,9 +109,10 @@ def test_allgather_argument_errors(cp):
     with pytest.raises(cp.CPError) as e:
         cp.allgather_attn_fwd(q, k, v, "zigzag", 2, False, [0, 100])
     assert e.value.code == 2
-    qf, kf, vf = (t.cuda() for t in W.random_qkv(1, 256, 4, 2, 128, "fp32", seed=1))
+    q256 = torch.zeros((1, 256, 4, 256), dtype=torch.bfloat16, device="cuda")
+    k256 = torch.zeros((1, 256, 2, 256), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(cp.CPError) as e:
-        cp.allgather_attn_fwd(qf, kf, vf, "zigzag", 2, True, None)
+        cp.allgather_attn_fwd(q256, k256, k256, "zigzag", 2, True, None)   # head dim 256
     assert e.value.code == 2
 
 
@@ -143,3 +166,23 @@ def test_allgather_bwd_matches_oracle(cp, case):
     for name, g, w in zip(("dq", "dk", "dv"), grads, want):
         err = np.max(np.abs(np64(g) - w))
         assert err <= 2e-2 * np.max(np.abs(w)), (name, err, np.max(np.abs(w)))
+
+
+@pytest.mark.parametrize("case", OTHER_CASES, ids=lambda c: "-".join(str(x) for x in c[:8]) + "-d%d" % len(c[8]))
+def test_allgather_bwd_fp32_and_d64_match_oracle(cp, case):
+    """The FFMA backward in its All-Gather form (one gathered key block, documents):
+    fp32 within 1e-4 x max |reference|, bf16 within 2e-2 x max |reference|."""
+    layout, N, S, b, hq, hkv, d, dt, docs = case
+    q, k, v = W.random_qkv(b, S, hq, hkv, d, dt, seed=3 * S + N + d)
+    do = W.random_do(b, S, hq, d, dt, seed=3 * S + N + d)
+    qr, kr, vr, dor = (cp.layout_permute(t.cuda(), layout, N) for t in (q, k, v, do))
+    o, lse = cp.allgather_attn_fwd(qr, kr, vr, layout, N, True, docs)
+    grads = cp.allgather_attn_bwd(qr, kr, vr, o, lse, dor, layout, N, True, docs)
+    grads = [cp.layout_permute(g, layout, N, inverse=True) for g in grads]
+    cp.stream_check()
+    want = oracle.allgather_attention_bwd(np64(q), np64(k), np64(v), np64(do), layout, N, True, d ** -0.5, docs)
+    tol = 1e-4 if dt == "fp32" else 2e-2
+    for name, g, w in zip(("dq", "dk", "dv"), grads, want):
+        assert g.dtype == q.dtype
+        err = np.max(np.abs(np64(g) - w))
+        assert err <= tol * np.max(np.abs(w)), (name, err, np.max(np.abs(w)))
