@@ -29,7 +29,7 @@ def test_usp_exchange_is_bit_exact(cp, layout, N, P, b, S, H):
     """Rank-major input (the ring layout over N) through the Ulysses exchange with P:
     entry u, rows [g c, (g+1) c) must hold the oracle's rank (g, u) buffer."""
     d = 128
-    x = torch.randn((b, S, H, d)).to(torch.bfloat16)
+    x = torch.randn((b, S, H, d), generator=torch.Generator().manual_seed(S + N + P)).to(torch.bfloat16)
     xr = cp.layout_permute(x.cuda(), layout, N)
     y = cp.ulysses_all_to_all(xr, P)
     got = y.cpu().view(torch.int16).numpy().reshape(P, b, S, H // P, d)
