@@ -803,10 +803,39 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
         if ((s = cp_layout_permute(layout, N, 1, &dvg, dv, 0, stream)) != CP_OK) return s;
         return CP_OK;
     }
-    // work order: the key tiles of the gathered block, earliest (most queries) first
+    // work order, heaviest first: a key tile of the gathered block costs the query
+    // tiles of every rank it meets, from the first that sees its first key (causal)
+    // to the last that starts before the end of its last key's document
     if (n_kt <= kMaxOrder) {
+        const int n_qt = (int)((c + kBwdQueryTile - 1) / kBwdQueryTile);
+        std::vector<std::pair<int64_t, uint32_t>> work;
+        work.reserve((size_t)n_kt);
+        const Range kr{0, 0, S, 0, 1};
+        for (int kt = 0; kt < (int)n_kt; ++kt) {
+            const int64_t k_hi = std::min<int64_t>((int64_t)kt * kBwdKeyTile + kBwdKeyTile - 1, S - 1);
+            const int64_t *next_doc = std::upper_bound(doc_starts, doc_starts + n_docs, k_hi);
+            const int64_t de = next_doc == doc_starts + n_docs ? S : *next_doc;  // end of the last key's document
+            int64_t tiles = 0;
+            for (int r = 0; r < N; ++r) {
+                const Range qr = layout_range(layout, N, S, r);
+                int qb, qf;
+                q_tile_bounds<int64_t>(qr, c, kBwdQueryTile, kr, S, (int64_t)kt * kBwdKeyTile, kBwdKeyTile,
+                                       causal != 0, &qb, &qf);
+                int lo = qb, hi = n_qt;  // first tile whose first row lies at or past de
+                while (lo < hi) {
+                    const int mid = (lo + hi) / 2;
+                    if (range_pos(qr, (int64_t)mid * kBwdQueryTile) < de) lo = mid + 1; else hi = mid;
+                }
+                tiles += lo - qb;
+            }
+            work.push_back({tiles, (uint32_t)kt});
+        }
+        std::stable_sort(work.begin(), work.end(),
+                         [](const std::pair<int64_t, uint32_t> &x, const std::pair<int64_t, uint32_t> &y) {
+                             return x.first > y.first;
+                         });
         p.order_len = (int)n_kt;
-        for (int kt = 0; kt < (int)n_kt; ++kt) p.order[kt] = (uint32_t)kt;
+        for (int64_t i = 0; i < n_kt; ++i) p.order[i] = work[(size_t)i].second;
     }
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
