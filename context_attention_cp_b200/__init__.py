@@ -6,6 +6,7 @@ is missing the first call raises ImportError instead of computing anything.
 
 Entry points mirror include/cpattn.h:
   block_attn_fwd(q, k, v, q_range, kv_range, causal, scale, o, lse, accumulate)
+  block_attn_bwd(q, k, v, o, lse, do, q_range, kv_range, causal, scale, dq_acc, dk_acc, dv_acc)
   lse_merge(o_acc, lse_acc, o_b, lse_b, o_out=None)
   ring_attn_fwd(q, k, v, layout, N, causal, scale, o=None, lse=None, mode="fused")
   ring_attn_bwd(q, k, v, o, lse, do, layout, N, causal, scale) -> (dq, dk, dv)
@@ -25,7 +26,7 @@ Tensors are torch tensors on the current CUDA device; token tensors are
 [b, s, H, d] with d contiguous, lse tensors [b, H, s] fp32.
 """
 from ._binding import (  # noqa: F401
-    CPError, LAYOUTS, MODES, allgather_attn_bwd, allgather_attn_fwd, allgather_workspace_bytes, block_attn_fwd, layout_permute,
+    CPError, LAYOUTS, MODES, allgather_attn_bwd, allgather_attn_fwd, allgather_workspace_bytes, block_attn_bwd, block_attn_fwd, layout_permute,
     layout_range, lib, lib_path,
     lse_merge, ring_attn_bwd, ring_attn_fwd, ring_attn_fwd_static_scratch, ring_bwd_workspace_bytes,
     ring_workspace_bytes, selftest_wait_timeout, stream_check, tile_classes, ulysses_all_to_all, ulysses_attn_bwd, ulysses_attn_fwd,

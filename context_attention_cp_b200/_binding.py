@@ -35,6 +35,8 @@ _i32, _i64, _vp, _f32, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ct
 _SIGNATURES = {
     "cp_block_attn_fwd": (_i32, [_T, _T, _T, _R, _R, _i32, _f32, _T, _T, _i32, _vp]),
     "cp_lse_merge": (_i32, [_T, _T, _T, _T, _T, _vp]),
+    "cp_block_attn_bwd": (_i32, [_T, _T, _T, _T, _T, _T, _R, _R, _i32, _f32, _T, _T, _T, _vp, _sz, _vp]),
+    "cp_block_bwd_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "cp_ring_attn_fwd": (_i32, [_i32, _i32, _i32, _T, _T, _T, _f32, _T, _T, _i32, _vp, _sz, _vp]),
     "cp_ring_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _i64]),
     "cp_ring_attn_bwd": (_i32, [_i32, _i32, _i32, _T, _T, _T, _T, _T, _T, _f32, _T, _T, _T, _vp, _sz, _vp]),
@@ -165,6 +167,23 @@ def block_attn_fwd(q, k, v, q_range, kv_range, causal, scale, o, lse, accumulate
                                    int(bool(causal)), float(scale), _ref(to), _ref(tl), int(bool(accumulate)),
                                    _stream()))
     return o, lse
+
+
+def block_attn_bwd(q, k, v, o, lse, do, q_range, kv_range, causal, scale, dq_acc, dk_acc, dv_acc, workspace=None):
+    """Adds one (query block, key block) pair's gradient shares into the fp32
+    accumulators dq_acc, dk_acc, dv_acc; lse and o are the rows' global forward
+    results."""
+    import torch
+    b, sq, Hq, _ = q.shape
+    need = lib().cp_block_bwd_workspace_bytes(b, sq, Hq)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    qr, kr = _range(q_range), _range(kv_range)
+    ts = [_tensor(t) for t in (q, k, v, o, lse, do, dq_acc, dk_acc, dv_acc)]
+    _check(lib().cp_block_attn_bwd(*[_ref(t) for t in ts[:6]], ctypes.byref(qr), ctypes.byref(kr), int(bool(causal)),
+                                   float(scale), *[_ref(t) for t in ts[6:]], ctypes.c_void_p(workspace.data_ptr()), need,
+                                   _stream()))
+    return dq_acc, dk_acc, dv_acc
 
 
 def lse_merge(o_acc, lse_acc, o_b, lse_b, o_out=None):

@@ -1113,6 +1113,85 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
     return launch_attn(p, q->dtype, st);
 }
 
+size_t cp_block_bwd_workspace_bytes(int64_t b, int64_t sq, int64_t Hq)
+{
+    if (b < 0 || sq < 0 || Hq < 0) return 0;
+    return (size_t)((b * Hq * sq * 8 + 255) / 256 * 256);  // (lse, D) per query row
+}
+
+cp_status cp_block_attn_bwd(const cp_tensor *q, const cp_tensor *k, const cp_tensor *v, const cp_tensor *o,
+                            const cp_tensor *lse, const cp_tensor *dout, const cp_range *q_range,
+                            const cp_range *kv_range, int32_t mask_mode, float softmax_scale, cp_tensor *dq_acc,
+                            cp_tensor *dk_acc, cp_tensor *dv_acc, void *workspace, size_t workspace_bytes,
+                            void *stream)
+{
+    g_last_error[0] = 0;
+    cp_status s;
+    if ((s = check_tensor(q, "q")) != CP_OK || (s = check_tensor(k, "k")) != CP_OK ||
+        (s = check_tensor(v, "v")) != CP_OK || (s = check_tensor(o, "o")) != CP_OK ||
+        (s = check_tensor(dout, "dout")) != CP_OK || (s = check_tensor(dq_acc, "dq_acc")) != CP_OK ||
+        (s = check_tensor(dk_acc, "dk_acc")) != CP_OK || (s = check_tensor(dv_acc, "dv_acc")) != CP_OK)
+        return s;
+    if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
+    if (mask_mode != CP_MASK_NONE && mask_mode != CP_MASK_CAUSAL) return fail(CP_ERR_INVALID_ARG, "unknown mask mode");
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    const int64_t b = q->shape[0], sq = q->shape[1], sk = k->shape[1], Hq = q->shape[2];
+    if (sq > INT32_MAX / 2 || sk > INT32_MAX / 2) return fail(CP_ERR_SHAPE, "sequence too long");
+    if ((s = check_out(o, lse, q, sq, false)) != CP_OK) return s;
+    if (o->dtype != q->dtype || dout->dtype != q->dtype || !same_shape(o, q) || !same_shape(dout, q))
+        return fail(CP_ERR_SHAPE, "o and dout must be shaped like q, same dtype");
+    if (!same_shape(dq_acc, q) || dq_acc->dtype != CP_FP32) return fail(CP_ERR_SHAPE, "dq_acc must be fp32 shaped like q");
+    if (!same_shape(dk_acc, k) || dk_acc->dtype != CP_FP32 || !same_shape(dv_acc, k) || dv_acc->dtype != CP_FP32)
+        return fail(CP_ERR_SHAPE, "dk_acc and dv_acc must be fp32 shaped like k");
+    if ((s = check_range(q_range, sq, "q_range")) != CP_OK) return s;
+    if ((s = check_range(kv_range, sk, "kv_range")) != CP_OK) return s;
+    const size_t need = cp_block_bwd_workspace_bytes(b, sq, Hq);
+    if (!workspace || workspace_bytes < need) return fail(CP_ERR_INVALID_ARG, "workspace of %zu bytes needed", need);
+    if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (b == 0 || sq == 0 || sk == 0) return CP_OK;
+
+    thread_local BwdParams p;
+    std::memset(&p, 0, sizeof p);
+    p.b = (int)b;
+    p.hq = (int)Hq;
+    p.hkv = (int)k->shape[2];
+    p.group = p.hq / p.hkv;
+    p.d = (int)q->shape[3];
+    p.q_len = (int)sq;
+    p.kv_len = (int)sk;
+    p.n_ranks = 1;
+    p.step_begin = 0;
+    p.step_end = 1;
+    p.causal = mask_mode == CP_MASK_CAUSAL;
+    p.use_layout = 0;
+    p.seq_len = 0;
+    p.q_range = to_range(*q_range);
+    p.kv_range = to_range(*kv_range);
+    p.kv_explicit = 1;
+    p.n_kv_blocks = 1;
+    p.scale = softmax_scale;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.q = q->data; p.k = k->data; p.v = v->data; p.o = o->data; p.dout = dout->data;
+    p.q_sb = q->stride[0]; p.q_ss = q->stride[1]; p.q_sh = q->stride[2];
+    p.k_sb = k->stride[0]; p.k_ss = k->stride[1]; p.k_sh = k->stride[2];
+    p.v_sb = v->stride[0]; p.v_ss = v->stride[1]; p.v_sh = v->stride[2];
+    p.o_sb = o->stride[0]; p.o_ss = o->stride[1]; p.o_sh = o->stride[2];
+    p.do_sb = dout->stride[0]; p.do_ss = dout->stride[1]; p.do_sh = dout->stride[2];
+    p.lse = static_cast<const float *>(lse->data);
+    p.lse_sb = lse->stride[0]; p.lse_sh = lse->stride[1]; p.lse_ss = lse->stride[2];
+    p.stats = static_cast<float2 *>(workspace);
+    p.lpad = (int)sq;
+    p.dq = dq_acc->data; p.dk = dk_acc->data; p.dv = dv_acc->data;
+    p.dq_sb = dq_acc->stride[0]; p.dq_ss = dq_acc->stride[1]; p.dq_sh = dq_acc->stride[2];
+    p.dk_sb = dk_acc->stride[0]; p.dk_ss = dk_acc->stride[1]; p.dk_sh = dk_acc->stride[2];
+    p.dv_sb = dv_acc->stride[0]; p.dv_ss = dv_acc->stride[1]; p.dv_sh = dv_acc->stride[2];
+    p.accumulate = 1;
+    cudaError_t e = launch_attn_bwd_simt(p, q->dtype == CP_FP32, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    return CP_OK;
+}
+
 size_t cp_ring_bwd_workspace_bytes(int32_t layout, int32_t N, int32_t dtype, int64_t b, int64_t S, int64_t Hq,
                                    int64_t d)
 {

@@ -23,7 +23,10 @@
 //      gradient keeps a single d-vector accumulator in registers.
 // The All-Gather form (kv_explicit: one gathered key block in original order, met
 // by every query rank) and its document mask (a query sees only keys of its own
-// document; section All-Gather 式 CP) are honoured key by key.
+// document; section All-Gather 式 CP) are honoured key by key.  The block form
+// (use_layout = 0: one explicit query block against one explicit key block, the
+// step a rank of a real ring runs) adds its shares into fp32 dq, dk, dv
+// (accumulate = 1).
 // Nothing waits on another CTA, so there is no bounded wait to report.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -109,7 +112,7 @@ __global__ void __launch_bounds__(SRM) simt_bwd_dq_kernel(const __grid_constant_
     const int q_lo = qt * SRM;
     const int row = q_lo + tid;
     const bool row_ok = row < p.q_len;
-    const Range qr = layout_range(p.layout, p.n_ranks, p.seq_len, rank);
+    const Range qr = p.use_layout ? layout_range(p.layout, p.n_ranks, p.seq_len, rank) : p.q_range;
     const int64_t pos_q = range_pos(qr, (int64_t)(row_ok ? row : p.q_len - 1));
     const int64_t grow = (int64_t)rank * p.q_row_step + (row_ok ? row : 0);
     int64_t ds_q = 0, de_q = 0;
@@ -177,9 +180,16 @@ __global__ void __launch_bounds__(SRM) simt_bwd_dq_kernel(const __grid_constant_
         }
     }
     if (!row_ok) return;
-    T *out = static_cast<T *>(p.dq) + bb * p.dq_sb + grow * p.dq_ss + (int64_t)h * p.dq_sh;
+    const int64_t off = bb * p.dq_sb + grow * p.dq_ss + (int64_t)h * p.dq_sh;
+    if (p.accumulate) {
+        float *out = static_cast<float *>(p.dq) + off;  // one thread owns the row: plain add
 #pragma unroll
-    for (int i = 0; i < D; ++i) stf(out + i, dq[i] * scale);
+        for (int i = 0; i < D; ++i) out[i] += dq[i] * scale;
+    } else {
+        T *out = static_cast<T *>(p.dq) + off;
+#pragma unroll
+        for (int i = 0; i < D; ++i) stf(out + i, dq[i] * scale);
+    }
 }
 
 template <typename T, int D, bool DK>
@@ -228,7 +238,7 @@ __global__ void __launch_bounds__(SRM) simt_bwd_dkv_kernel(const __grid_constant
         const int h = hk * p.group + hh;
         for (int r = 0; r < N; ++r) {
             const int qrank = (j + r) % N;  // the rank that holds block j at ring step r
-            const Range qr = layout_range(p.layout, N, p.seq_len, qrank);
+            const Range qr = p.use_layout ? layout_range(p.layout, N, p.seq_len, qrank) : p.q_range;
             int qt_begin, qt_full;
             q_tile_bounds<int64_t>(qr, p.q_len, SRN, kr, p.kv_len, k_lo, SRM, p.causal != 0, &qt_begin, &qt_full);
             for (int qt = qt_begin; qt < n_qt; ++qt) {
@@ -279,10 +289,18 @@ __global__ void __launch_bounds__(SRM) simt_bwd_dkv_kernel(const __grid_constant
         }
     }
     if (!key_ok) return;
-    T *out = DK ? static_cast<T *>(p.dk) + bb * p.dk_sb + krow * p.dk_ss + (int64_t)hk * p.dk_sh
-                : static_cast<T *>(p.dv) + bb * p.dv_sb + krow * p.dv_ss + (int64_t)hk * p.dv_sh;
+    const int64_t off = DK ? bb * p.dk_sb + krow * p.dk_ss + (int64_t)hk * p.dk_sh
+                           : bb * p.dv_sb + krow * p.dv_ss + (int64_t)hk * p.dv_sh;
+    void *base = DK ? p.dk : p.dv;
+    if (p.accumulate) {
+        float *out = static_cast<float *>(base) + off;  // one thread owns the row: plain add
 #pragma unroll
-    for (int c = 0; c < D; ++c) stf(out + c, DK ? acc[c] * scale : acc[c]);
+        for (int c = 0; c < D; ++c) out[c] += DK ? acc[c] * scale : acc[c];
+    } else {
+        T *out = static_cast<T *>(base) + off;
+#pragma unroll
+        for (int c = 0; c < D; ++c) stf(out + c, DK ? acc[c] * scale : acc[c]);
+    }
 }
 
 template <typename K>

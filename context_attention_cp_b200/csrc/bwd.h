@@ -92,6 +92,9 @@ struct BwdParams {
     int kv_explicit, n_kv_blocks;
     const int *doc_starts;
     int n_docs;
+    // accumulate = 1 (the block form, FFMA kernels only): dq, dk, dv are fp32 and this
+    // call's shares are added to them; 0: they are written in the input dtype
+    int accumulate;
     // work order: entry e -> (key block, key tile) = (order[e] >> 16, order[e] & 0xffff);
     // head_major puts (batch, kv head) outside the order in the grid
     int head_major;
@@ -103,9 +106,11 @@ struct BwdParams {
 // Statistics + dq_acc zeroing, the main tcgen05 kernel, then dq_acc -> dq.
 cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream);
 
-// The FFMA backward (attn_simt_bwd.cu) for fp32 inputs or bf16 with d = 64: the ring
-// layout only (use_layout = 1, kv_explicit = 0, no documents); uses p.stats as its
-// (lse, D) table and leaves dq_acc untouched.
+// The FFMA backward (attn_simt_bwd.cu) for fp32 inputs or bf16 with d = 64, and for
+// the block form: the ring layout (use_layout = 1), the gathered block (kv_explicit)
+// with documents, or one explicit query block against one key block (use_layout =
+// 0, kv_explicit = 1, n_ranks = 1); uses p.stats as its (lse, D) table and leaves
+// dq_acc untouched.
 cudaError_t launch_attn_bwd_simt(const BwdParams &p, bool fp32, cudaStream_t stream);
 
 }  // namespace cpattn

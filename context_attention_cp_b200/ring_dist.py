@@ -14,8 +14,17 @@ cp_block_attn_fwd with the rank ranges of the layout: the first step writes the
 fp32 (o, lse), later steps merge into them with the kernel's fused epilogue.  The
 exchange of the next block is posted before the compute and waited for after it.
 
-The compute step can be replaced (`compute=`), which is how the schedule is tested
-on CPU ranks (gloo) without a GPU.
+The backward (ring_attn_bwd_dist) walks the same ring once more (section 分块注意力,
+paragraph on the backward pass): at step r rank i holds block (i - r) mod N together
+with that block's travelling fp32 dK, dV accumulators, adds its queries' shares to
+its own dQ and to the travelling dK, dV (cp_block_attn_bwd, with the rows' global
+lse and o from the forward), and passes block and accumulators on.  The next K/V
+block is posted before the compute; the accumulators can only leave after it.
+After the last step every accumulator is one hop from its owner, and one more
+exchange brings it home.
+
+The compute steps can be replaced (`compute=`), which is how the schedules are
+tested on CPU ranks (gloo) without a GPU.
 """
 import torch
 import torch.distributed as dist
@@ -64,3 +73,56 @@ def ring_attn_fwd_dist(q, k, v, layout, causal, scale=None, group=None, compute=
             cur_k, buf_k = buf_k, cur_k
             cur_v, buf_v = buf_v, cur_v
     return o.to(q.dtype), lse
+
+
+def block_bwd_compute(q, k, v, o, lse, do, q_range, kv_range, causal, scale, dq_acc, dk_acc, dv_acc):
+    """The default backward step: the block backward, adding into fp32 accumulators."""
+    B.block_attn_bwd(q, k, v, o, lse, do, q_range, kv_range, causal, scale, dq_acc, dk_acc, dv_acc)
+
+
+def ring_attn_bwd_dist(q, k, v, o, lse, do, layout, causal, scale=None, group=None, compute=block_bwd_compute):
+    """This rank's gradients of ring attention.
+
+    q, o, do [b, c, Hq, d], k / v [b, c, Hkv, d]: this rank's local blocks; o and lse
+    [b, Hq, c] are this rank's results of the whole-sequence forward (for example
+    ring_attn_fwd_dist).  Returns (dq, dk, dv) in q's dtype for the local blocks.
+    All ranks of `group` call it together.
+    """
+    import torch
+    rank = dist.get_rank(group)
+    N = dist.get_world_size(group)
+    b, c, Hq, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    S = c * N
+    q_range = B.layout_range(layout, N, S, rank)
+    nxt, prv = (rank + 1) % N, (rank - 1) % N
+    to_global = (lambda r: dist.get_global_rank(group, r)) if group is not None else (lambda r: r)
+
+    def exchange(send, recv):
+        ops = [dist.P2POp(dist.isend, t, to_global(nxt), group) for t in send]
+        ops += [dist.P2POp(dist.irecv, t, to_global(prv), group) for t in recv]
+        return dist.batch_isend_irecv(ops)
+
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.zeros(q.shape, **f32)
+    cur_k, cur_v = k.contiguous(), v.contiguous()
+    buf_k, buf_v = torch.empty_like(cur_k), torch.empty_like(cur_v)
+    cur_dk, cur_dv = torch.zeros(k.shape, **f32), torch.zeros(v.shape, **f32)
+    buf_dk, buf_dv = torch.empty_like(cur_dk), torch.empty_like(cur_dv)
+    for r in range(N):
+        src = (rank - r) % N                      # the block this rank holds at step r
+        kv_reqs = exchange([cur_k, cur_v], [buf_k, buf_v]) if r + 1 < N else []
+        compute(q, cur_k, cur_v, o, lse, do, q_range, B.layout_range(layout, N, S, src), causal, scale, dq,
+                cur_dk, cur_dv)
+        # the block's accumulators follow it; after the last step they go home
+        acc_reqs = exchange([cur_dk, cur_dv], [buf_dk, buf_dv]) if N > 1 else []
+        for req in kv_reqs + acc_reqs:
+            req.wait()
+        if N > 1:
+            cur_dk, buf_dk = buf_dk, cur_dk
+            cur_dv, buf_dv = buf_dv, cur_dv
+            if r + 1 < N:
+                cur_k, buf_k = buf_k, cur_k
+                cur_v, buf_v = buf_v, cur_v
+    return dq.to(q.dtype), cur_dk.to(k.dtype), cur_dv.to(v.dtype)

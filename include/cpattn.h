@@ -309,6 +309,33 @@ cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_t
                            cp_tensor *dq, cp_tensor *dk, cp_tensor *dv, void *workspace,
                            size_t workspace_bytes, void *stream);
 
+/* Block backward ("上下文并行与 Ring Attention", section 分块注意力, paragraph on the
+ * backward pass): one query block against one key block with the query rows' GLOBAL
+ * statistics, the step one rank of a real ring runs per held K/V block.  With
+ * p_j = e^{x_j - lse} (lse of the whole sequence), D = dout . o (o of the whole
+ * sequence) and x_j = scale q . k_j, this call ADDS its shares
+ *   dq_acc += scale sum_j p_j (dout . v_j - D) k_j,
+ *   dk_acc_j += scale sum_q p_j (dout . v_j - D) q,   dv_acc_j += sum_q p_j dout
+ * over the visible (query, key) pairs of the two blocks.
+ *   q, o, dout [b, sq, Hq, d] and k, v [b, sk, Hkv, d]: bf16 or fp32 (one dtype),
+ *   d = 64 or 128; lse [b, Hq, sq, 1] fp32: the forward's GLOBAL lse of these rows;
+ *   q_range / kv_range: original positions of the rows (as cp_block_attn_fwd);
+ *   mask_mode: CP_MASK_CAUSAL or CP_MASK_NONE.
+ *   dq_acc [b, sq, Hq, d], dk_acc / dv_acc [b, sk, Hkv, d]: fp32 accumulators the
+ *   shares are added to (the caller zeroes them once).
+ *   workspace: cp_block_bwd_workspace_bytes(b, sq, Hq) bytes, 256-byte aligned (the
+ *   rows' lse and D).
+ * Runs the FFMA backward kernels (fp32 arithmetic).  Rows whose lse is -inf add
+ * nothing.  Argument errors return synchronously. */
+cp_status cp_block_attn_bwd(const cp_tensor *q, const cp_tensor *k, const cp_tensor *v,
+                            const cp_tensor *o, const cp_tensor *lse, const cp_tensor *dout,
+                            const cp_range *q_range, const cp_range *kv_range, int32_t mask_mode,
+                            float softmax_scale, cp_tensor *dq_acc, cp_tensor *dk_acc, cp_tensor *dv_acc,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes cp_block_attn_bwd needs. */
+size_t cp_block_bwd_workspace_bytes(int64_t b, int64_t sq, int64_t Hq);
+
 /* Workspace bytes cp_ring_attn_bwd needs (0 for invalid arguments). */
 size_t cp_ring_bwd_workspace_bytes(int32_t layout, int32_t N, int32_t dtype, int64_t b, int64_t S,
                                    int64_t Hq, int64_t d);

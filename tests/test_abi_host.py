@@ -349,3 +349,29 @@ def test_empty_inputs_return_ok_without_device_work(cp, b, S):
         "permute": L.cp_layout_permute(1, 2, 1, *r(q, o), 0, None),
     }
     assert all(v == 0 for v in calls.values()), calls
+
+
+def test_block_bwd_argument_errors_are_synchronous(cp):
+    from context_attention_cp_b200._binding import _range
+    L = cp.lib()
+    q, o, do = _ct(cp, [1, 128, 4, 64]), _ct(cp, [1, 128, 4, 64], data=0x30000), _ct(cp, [1, 128, 4, 64], data=0x50000)
+    k = _ct(cp, [1, 96, 2, 64], data=0x20000)
+    lse = _ct(cp, [1, 4, 128, 1], dtype=1, data=0x40000)
+    dq = _ct(cp, [1, 128, 4, 64], dtype=1, data=0x60000)
+    dk = _ct(cp, [1, 96, 2, 64], dtype=1, data=0x70000)
+    qr, kr = _range(((0,), (128,), 1)), _range(((0,), (96,), 1))
+    need = L.cp_block_bwd_workspace_bytes(1, 128, 4)
+    assert need >= 128 * 4 * 8
+
+    def call(mask=1, dq_=dq, dk_=dk, wsb=None, ws=0x100000, kr_=kr):
+        return L.cp_block_attn_bwd(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(o), ctypes.byref(lse),
+                                   ctypes.byref(do), ctypes.byref(qr), ctypes.byref(kr_), mask, ctypes.c_float(0.125),
+                                   ctypes.byref(dq_), ctypes.byref(dk_), ctypes.byref(dk_), ctypes.c_void_p(ws),
+                                   need if wsb is None else wsb, None)
+
+    assert call(mask=3) == 1                                   # mask mode
+    assert call(dq_=_ct(cp, [1, 128, 4, 64], data=0x60000)) == 3   # bf16 accumulator
+    assert call(dk_=_ct(cp, [1, 96, 4, 64], dtype=1, data=0x70000)) == 3   # dk shaped like q
+    assert call(wsb=8) == 1                                    # workspace too small
+    assert call(ws=0x100008) == 1                              # workspace alignment
+    assert call(kr_=_range(((0,), (95,), 1))) != 0             # range length differs from the key block

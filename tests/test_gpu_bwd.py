@@ -18,7 +18,7 @@ import torch
 
 import cp_workloads as W
 import oracle
-from gpu_helpers import np64
+from gpu_helpers import np64, positions
 
 pytestmark = pytest.mark.gpu
 
@@ -122,6 +122,37 @@ def test_fp32_workload_bwd_element_by_element(cp):
     for name, g, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
         err = np.max(np.abs(np64(g) - ref))
         assert err <= TOL_REL_FP32 * np.max(np.abs(ref)), (name, err)
+
+
+@pytest.mark.parametrize("dt,d,kind", [("bf16", 128, "zigzag"), ("fp32", 64, "zigzag"), ("bf16", 64, "striped"),
+                                       ("fp32", 128, "later_q")])
+def test_block_bwd_adds_the_block_share(cp, dt, d, kind):
+    """cp_block_attn_bwd: one query block against one key block with the rows' global
+    statistics; the shares are ADDED to fp32 accumulators (pre-filled here)."""
+    from context_attention_cp_b200 import layout_range
+    S, N = 512, 2
+    q, k, v = W.random_qkv(1, S, 4, 2, d, dt, seed=S + d)
+    do = W.random_do(1, S, 4, d, dt, seed=S + d)
+    o_full, lse_full = oracle.attention(np64(q), np64(k), np64(v), True, d ** -0.5)
+    if kind == "later_q":   # query block after the key block: every pair visible
+        qr, kr = ((256,), (256,), 1), ((0,), (256,), 1)
+    else:
+        qr, kr = layout_range(kind, N, S, 1), layout_range(kind, N, S, 0)
+    pq, pk = positions(qr), positions(kr)
+    qi, ki = torch.from_numpy(pq), torch.from_numpy(pk)
+    qb, kb, vb, dob = (t[:, idx].contiguous() for t, idx in ((q, qi), (k, ki), (v, ki), (do, qi)))
+    ob = torch.from_numpy(o_full[:, pq]).to(q.dtype)   # the global forward's o of these rows
+    lb = torch.from_numpy(np.ascontiguousarray(lse_full[:, :, pq])).float()
+    pre = 0.25
+    acc = [torch.full(t.shape, pre, dtype=torch.float32, device="cuda") for t in (qb, kb, vb)]
+    cp.block_attn_bwd(*(t.cuda() for t in (qb, kb, vb, ob, lb, dob)), qr, kr, True, d ** -0.5, *acc)
+    cp.stream_check()
+    delta = np.einsum("bshd,bshd->bhs", np64(dob), np64(ob))
+    want = oracle.attention_bwd(np64(qb), np64(kb), np64(vb), np64(dob), True, d ** -0.5, pos_q=pq, pos_k=pk,
+                                lse=np64(lb), delta=delta)[:3]
+    for name, g, w in zip(("dq", "dk", "dv"), acc, want):
+        err = np.max(np.abs(np64(g) - pre - w))
+        assert err <= 1e-4 * max(np.max(np.abs(w)), 1e-30) + 1e-6, (name, err, np.max(np.abs(w)))
 
 
 def test_ring_bwd_dkdv_deterministic(cp):

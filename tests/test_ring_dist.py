@@ -76,3 +76,63 @@ def test_ring_over_gloo_ranks(layout, world, S):
     for rank, (err_o, err_l, seen, want_seen) in out.items():
         assert err_o <= 1e-6 and err_l <= 1e-6, (rank, err_o, err_l)
         assert seen == want_seen, (rank, seen, want_seen)   # step r holds rank (i - r) mod N's block
+
+
+def _bwd_worker(rank, world, port, layout, S, out):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import oracle
+    from context_attention_cp_b200 import ring_dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        r = np.random.default_rng(11)
+        b, hq, hkv, d = 1, 4, 2, 8
+        q = r.standard_normal((b, S, hq, d))
+        k = r.standard_normal((b, S, hkv, d))
+        v = r.standard_normal((b, S, hkv, d))
+        do = r.standard_normal((b, S, hq, d))
+        o_full, lse_full = oracle.attention(q, k, v, True, 0.35, nthreads=1)
+        pos = np.array(oracle.layout.rank_positions(layout, world, S, rank))
+        loc = lambda t: torch.from_numpy(np.ascontiguousarray(t[:, pos]))  # noqa: E731
+        ql, kl, vl, dol, ol = (loc(t) for t in (q, k, v, do, o_full))
+        lsel = torch.from_numpy(np.ascontiguousarray(lse_full[:, :, pos]))
+        seen = []
+
+        def oracle_step(qq, kk, vv, oo, ll, gg, q_range, kv_range, causal, scale, dq, dk, dv):
+            pk = _positions(kv_range)
+            seen.append(int(pk[0]))
+            delta = np.einsum("bshd,bshd->bhs", gg.numpy(), oo.numpy())
+            a, bk, bv, _, _ = oracle.attention_bwd(qq.numpy(), kk.numpy(), vv.numpy(), gg.numpy(), causal, scale,
+                                                   pos_q=_positions(q_range), pos_k=pk, lse=ll.numpy(), delta=delta,
+                                                   nthreads=1)
+            dq += torch.from_numpy(a)
+            dk += torch.from_numpy(bk)
+            dv += torch.from_numpy(bv)
+
+        dq, dk, dv = ring_dist.ring_attn_bwd_dist(ql, kl, vl, ol, lsel, dol, layout, True, 0.35, compute=oracle_step)
+        want = oracle.attention_bwd(q, k, v, do, True, 0.35, nthreads=1)[:3]
+        errs = [float(np.max(np.abs(g.numpy() - w[:, pos]))) for g, w in zip((dq, dk, dv), want)]
+        out[rank] = (errs, seen,
+                     [int(oracle.layout.rank_positions(layout, world, S, (rank - s) % world)[0]) for s in range(world)])
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 32), ("striped", 4, 32), ("contiguous", 3, 24),
+                                            ("zigzag", 1, 16)])
+def test_ring_bwd_over_gloo_ranks(layout, world, S):
+    """Every rank ends with the whole-sequence gradients of its own rows and keys:
+    dQ accumulated locally, dK and dV carried around the ring with their block and
+    brought home after the last step."""
+    port = 29600 + (os.getpid() + world * 13 + len(layout) + 450) % 900
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_bwd_worker, args=(world, port, layout, S, out), nprocs=world, start_method="spawn", join=True)
+    assert sorted(out.keys()) == list(range(world))
+    for rank, (errs, seen, want_seen) in out.items():
+        assert max(errs) <= 1e-6, (rank, errs)   # the driver's accumulators are fp32
+        assert seen == want_seen, (rank, seen, want_seen)
