@@ -78,7 +78,7 @@ def test_ring_over_gloo_ranks(layout, world, S):
         assert seen == want_seen, (rank, seen, want_seen)   # step r holds rank (i - r) mod N's block
 
 
-def _bwd_worker(rank, world, port, layout, S, out):
+def _bwd_worker(rank, world, port, layout, S, causal, out):
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
@@ -94,7 +94,7 @@ def _bwd_worker(rank, world, port, layout, S, out):
         k = r.standard_normal((b, S, hkv, d))
         v = r.standard_normal((b, S, hkv, d))
         do = r.standard_normal((b, S, hq, d))
-        o_full, lse_full = oracle.attention(q, k, v, True, 0.35, nthreads=1)
+        o_full, lse_full = oracle.attention(q, k, v, causal, 0.35, nthreads=1)
         pos = np.array(oracle.layout.rank_positions(layout, world, S, rank))
         loc = lambda t: torch.from_numpy(np.ascontiguousarray(t[:, pos]))  # noqa: E731
         ql, kl, vl, dol, ol = (loc(t) for t in (q, k, v, do, o_full))
@@ -112,8 +112,8 @@ def _bwd_worker(rank, world, port, layout, S, out):
             dk += torch.from_numpy(bk)
             dv += torch.from_numpy(bv)
 
-        dq, dk, dv = ring_dist.ring_attn_bwd_dist(ql, kl, vl, ol, lsel, dol, layout, True, 0.35, compute=oracle_step)
-        want = oracle.attention_bwd(q, k, v, do, True, 0.35, nthreads=1)[:3]
+        dq, dk, dv = ring_dist.ring_attn_bwd_dist(ql, kl, vl, ol, lsel, dol, layout, causal, 0.35, compute=oracle_step)
+        want = oracle.attention_bwd(q, k, v, do, causal, 0.35, nthreads=1)[:3]
         errs = [float(np.max(np.abs(g.numpy() - w[:, pos]))) for g, w in zip((dq, dk, dv), want)]
         out[rank] = (errs, seen,
                      [int(oracle.layout.rank_positions(layout, world, S, (rank - s) % world)[0]) for s in range(world)])
@@ -122,17 +122,81 @@ def _bwd_worker(rank, world, port, layout, S, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 32), ("striped", 4, 32), ("contiguous", 3, 24),
-                                            ("zigzag", 1, 16)])
-def test_ring_bwd_over_gloo_ranks(layout, world, S):
+@pytest.mark.parametrize("layout,world,S,causal", [("zigzag", 2, 32, True), ("striped", 4, 32, True),
+                                                   ("contiguous", 3, 24, True), ("zigzag", 1, 16, True),
+                                                   ("contiguous", 2, 16, False)])
+def test_ring_bwd_over_gloo_ranks(layout, world, S, causal):
     """Every rank ends with the whole-sequence gradients of its own rows and keys:
     dQ accumulated locally, dK and dV carried around the ring with their block and
     brought home after the last step."""
-    port = 29600 + (os.getpid() + world * 13 + len(layout) + 450) % 900
+    port = 29600 + (os.getpid() + world * 13 + len(layout) + 450 + 7 * causal) % 900
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.start_processes(_bwd_worker, args=(world, port, layout, S, out), nprocs=world, start_method="spawn", join=True)
+    mp.start_processes(_bwd_worker, args=(world, port, layout, S, causal, out), nprocs=world, start_method="spawn",
+                       join=True)
     assert sorted(out.keys()) == list(range(world))
     for rank, (errs, seen, want_seen) in out.items():
         assert max(errs) <= 1e-6, (rank, errs)   # the driver's accumulators are fp32
         assert seen == want_seen, (rank, seen, want_seen)
+
+
+def _group_worker(rank, world, port, out):
+    """Ranks 1 and 3 of 4 form a sub-group and run the ring (forward and backward)
+    inside it: the driver must address its neighbours by their global ranks."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import oracle
+    from context_attention_cp_b200 import ring_dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        sub = dist.new_group([1, 3])
+        if rank in (1, 3):
+            me, n = [1, 3].index(rank), 2
+            S, layout = 16, "zigzag"
+            r = np.random.default_rng(5)
+            q, k, v, do = (r.standard_normal(s) for s in ((1, S, 2, 4), (1, S, 1, 4), (1, S, 1, 4), (1, S, 2, 4)))
+            pos = np.array(oracle.layout.rank_positions(layout, n, S, me))
+            loc = lambda t: torch.from_numpy(np.ascontiguousarray(t[:, pos]))  # noqa: E731
+
+            def fwd_step(qq, kk, vv, q_range, kv_range, causal, scale, o, lse, accumulate):
+                ob, lb = oracle.attention(qq.numpy(), kk.numpy(), vv.numpy(), causal, scale,
+                                          pos_q=_positions(q_range), pos_k=_positions(kv_range), nthreads=1)
+                if accumulate:
+                    om, lm = oracle.lse_merge(o.numpy().transpose(0, 2, 1, 3), lse.numpy(), ob.transpose(0, 2, 1, 3), lb)
+                    ob, lb = om.transpose(0, 2, 1, 3), lm
+                o.copy_(torch.from_numpy(np.ascontiguousarray(ob)))
+                lse.copy_(torch.from_numpy(np.ascontiguousarray(lb)))
+
+            def bwd_step(qq, kk, vv, oo, ll, gg, q_range, kv_range, causal, scale, dq, dk, dv):
+                delta = np.einsum("bshd,bshd->bhs", gg.numpy(), oo.numpy())
+                a, bk, bv, _, _ = oracle.attention_bwd(qq.numpy(), kk.numpy(), vv.numpy(), gg.numpy(), causal, scale,
+                                                       pos_q=_positions(q_range), pos_k=_positions(kv_range),
+                                                       lse=ll.numpy(), delta=delta, nthreads=1)
+                dq += torch.from_numpy(a)
+                dk += torch.from_numpy(bk)
+                dv += torch.from_numpy(bv)
+
+            o, lse = ring_dist.ring_attn_fwd_dist(loc(q), loc(k), loc(v), layout, True, 0.5, group=sub,
+                                                  compute=fwd_step)
+            grads = ring_dist.ring_attn_bwd_dist(loc(q), loc(k), loc(v), o, lse, loc(do), layout, True, 0.5,
+                                                 group=sub, compute=bwd_step)
+            wo, wl = oracle.attention(q, k, v, True, 0.5, nthreads=1)
+            wg = oracle.attention_bwd(q, k, v, do, True, 0.5, nthreads=1)[:3]
+            errs = [float(np.max(np.abs(o.numpy() - wo[:, pos]))), float(np.max(np.abs(lse.numpy() - wl[:, :, pos])))]
+            errs += [float(np.max(np.abs(g.numpy() - w[:, pos]))) for g, w in zip(grads, wg)]
+            out[rank] = errs
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ring_in_a_sub_group():
+    port = 29600 + (os.getpid() + 777) % 900
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_group_worker, args=(4, port, out), nprocs=4, start_method="spawn", join=True)
+    assert sorted(out.keys()) == [1, 3]
+    for rank, errs in out.items():
+        assert max(errs) <= 1e-6, (rank, errs)
