@@ -48,7 +48,7 @@ extern "C" {
 typedef enum {
     CP_OK = 0,
     CP_ERR_INVALID_ARG = 1, /* null pointer, bad enum, bad dtype, bad stride */
-    CP_ERR_UNSUPPORTED = 2, /* valid request this build does not implement (e.g. d) */
+    CP_ERR_UNSUPPORTED = 2, /* valid request the library does not implement (e.g. d) */
     CP_ERR_SHAPE = 3,       /* inconsistent or indivisible sizes */
     CP_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
     CP_ERR_TIMEOUT = 5      /* a device-side bounded wait expired (see cp_stream_check) */
