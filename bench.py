@@ -1,21 +1,39 @@
 """Benchmark: ring-attention forward TFLOP/s on effective (unmasked) FLOPs.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--mode fused|stepwise]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--mode M] [--legs L]
     python bench.py --impl reference ...     (the fp64 CPU oracle on a bounded row sample)
 
-One step = one cp_ring_attn_fwd over the whole workload (all N virtual ranks, all
-ring steps), inputs already permuted to rank-major order and resident in HBM.
-The line also carries the standalone merge bandwidth, the backward
-(cp_ring_attn_bwd) of the same workload and the All-Gather forward with a document
-mask (cp_allgather_attn_fwd) on its 8-document variant, Ulysses
-(cp_ulysses_attn_fwd, P = 4) on its shape and USP (cp_usp_attn_fwd: Ulysses groups
-of 2 inside the workload's ring), each timed on its own.
-L2 is flushed (a 256 MiB write) before every timed step; each step is timed with
-CUDA events on the launching stream.  With --gpus N > 1 (torchrun) every rank
-runs its own instance of the workload (weak scaling, no collective on the data
-path); the time is the max over ranks.  Rank 0 prints one JSON line.
+Headline (one GPU): one step = one cp_ring_attn_fwd over the whole workload (all N
+virtual ranks, all ring steps), inputs already permuted to rank-major order and
+resident in HBM.  The default workload is the largest one that fits one GPU: the
+Llama-3-70B head shape (64 query / 8 KV heads, d = 128) at S = 131072, causal,
+zig-zag over N = 8 virtual ranks.
+
+The same line carries, each timed on its own (CUDA events on the launching stream,
+L2 flushed before every timed call):
+  configs   : the other bf16 workloads (fused ring), and the two stepwise forms of
+              the ring (block launches + standalone merges, the page's loop as
+              written; block launches merging in their epilogue) on the 8B and the
+              non-causal 64K workloads, with the standalone merge's share;
+  merge     : the standalone LSE merge's HBM bandwidth at two partial sizes;
+  backward  : cp_ring_attn_bwd on the headline workload and the 8B one;
+  allgather : All-Gather CP with a document mask (8 and 32 documents), forward and
+              backward;
+  ulysses   : Ulysses (P = 4) and USP (Ulysses groups of 2 inside the ring);
+  e2e       : the headline through the public API with host buffers (pinned
+              host -> device copies of q, k, v, permute, ring, unpermute, device ->
+              host copies of o and lse), pipelined on three streams;
+  cpu_baseline : the fp64 oracle on the host cores, on a bounded row sample.
+
+With --gpus N > 1 (torchrun, one process per GPU) the ring runs across the N real
+ranks instead (context_attention_cp_b200.ring_dist): each rank holds its layout
+block of the workload (c = S / N tokens) and passes K/V blocks to its neighbour
+with NCCL point-to-point transfers while its block kernel runs.  The total work is
+the workload's, whatever N (strong scaling); the time is the max over ranks.
+Rank 0 prints one JSON line.
 """
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -32,6 +50,8 @@ import cp_workloads as W  # noqa: E402
 
 METRIC = "ring-attn fwd TFLOP/s (causal, effective FLOPs) & % bf16 peak; merge GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+VENDOR_BF16_DENSE_TFLOPS = 2250.0   # B200 dense bf16 (the 2:4-sparse figure halved)
+L2_FLUSH_BYTES = 256 << 20
 
 
 def load_peaks():
@@ -102,22 +122,27 @@ KERNEL_SOURCES = ["context_attention_cp_b200/csrc/attn_tc.cu", "context_attentio
                   "context_attention_cp_b200/csrc/exp2_poly.h"]
 
 
-def profiled_traffic(profile="profiles/attn_tc_kernel_llama3_8b_s8k_zigzag4.md"):
-    """DRAM bytes per launch from the committed ncu summary, or None when the kernel
-    sources changed since the counters were taken."""
-    import hashlib
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the forward kernel on `workload`, from the committed
+    ncu summary profiles/attn_tc_kernel_<workload>.md; None when there is none or
+    when the kernel sources changed since its counters were taken."""
     try:
-        with open(os.path.join(ROOT, profile)) as f:
+        with open(os.path.join(ROOT, "profiles", "attn_tc_kernel_%s.md" % workload)) as f:
             text = f.read()
-        h = hashlib.sha256()
-        for name in KERNEL_SOURCES:
-            with open(os.path.join(ROOT, name), "rb") as f:
-                h.update(f.read())
+        sha = kernel_source_sha()
     except OSError:
         return None
     rec = dict(ln.split(":", 1) for ln in text.splitlines() if ln.startswith(("traffic_bytes_per_launch:",
                                                                               "source_sha256:")))
-    if rec.get("source_sha256", "").strip() != h.hexdigest():
+    if rec.get("source_sha256", "").strip() != sha or "traffic_bytes_per_launch" not in rec:
         return None
     return int(rec["traffic_bytes_per_launch"].strip())
 
@@ -133,7 +158,7 @@ def reduce_max(value, world, device):
     return float(t.item())
 
 
-def cpu_oracle_rate(w, seconds_target=12.0, seed=0):
+def cpu_oracle_rate(w, seconds_target=12.0, seed=0, threads=None, inputs=None):
     """Times the fp64 oracle on a bounded sample of query rows of the workload.
 
     Returns (TFLOP/s on effective FLOPs, description, threads used).  The rows are
@@ -142,10 +167,11 @@ def cpu_oracle_rate(w, seconds_target=12.0, seed=0):
 
     import oracle
     rng = np.random.default_rng(seed)
-    q, k, v = W.make_inputs(w)
+    q, k, v = inputs if inputs is not None else W.make_inputs(w)
     k64 = k.float().numpy().astype(np.float64)
     v64 = v.float().numpy().astype(np.float64)
-    threads = oracle.default_threads()
+    if threads is None:
+        threads = oracle.default_threads()
 
     def run(n):
         sel = np.stack([rng.integers(0, w.b, n), rng.integers(0, w.hq, n), rng.integers(0, w.S, n)], axis=1)
@@ -176,14 +202,16 @@ def run_reference(args):
     threads = 0
     # keep the whole run to a few minutes
     per_step = min(args.ref_seconds, 150.0 / (args.warmup + args.steps))
+    inputs = W.make_inputs(w)
     for i in range(args.warmup + args.steps):
-        rate, desc, threads = cpu_oracle_rate(w, seconds_target=per_step, seed=i)
+        rate, desc, threads = cpu_oracle_rate(w, seconds_target=per_step, seed=i, inputs=inputs)
         if i >= args.warmup:
             per.append(rate)
     value = statistics.mean(per)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+        "scaling": "strong" if args.gpus > 1 else "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "ms_per_step": None,
         "config": {"workload": w.name, "b": w.b, "S": w.S, "hq": w.hq, "hkv": w.hkv, "d": w.d,
@@ -195,51 +223,229 @@ def run_reference(args):
     return 0
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=W.BENCH_WORKLOAD,
-                    choices=sorted(n for n, x in W.BY_NAME.items() if x.n_docs == 1))
-    ap.add_argument("--mode", default="fused", choices=["fused", "stepwise"])
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-seconds", type=float, default=12.0)
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
-    if args.impl == "reference":
-        return run_reference(args)
+class Timer:
+    """CUDA-event timing of calls on the current stream, L2 flushed before each."""
 
+    def __init__(self, torch, flush):
+        self.torch = torch
+        self.flush = flush
+
+    def __call__(self, fn, steps, warmup=3):
+        torch = self.torch
+        stream = torch.cuda.current_stream()
+        for _ in range(warmup):
+            fn()
+        ms = []
+        for _ in range(steps):
+            self.flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        return statistics.mean(ms), ms
+
+
+def tflops_entry(flops, ms, peak_tf, peak_src, **extra):
+    tf = flops / (ms * 1e-3) / 1e12
+    d = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms, "frac": tf / peak_tf,
+         "frac_of": "%s bf16 burst %.1f TFLOP/s" % (peak_src, peak_tf)}
+    d.update(extra)
+    return d
+
+
+def run_legs(cp, torch, dev, w, qd, kd, vd, o, lse, timer, peaks, peak_src, args, legs):
+    """The sub-results of the one-GPU line (see the module docstring)."""
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    steps = max(3, min(args.steps, 10))
+    out = {}
+
+    def merge_gbs(b, S, H, d):
+        oa = torch.randn((b, S, H, d), device=dev)
+        ob = torch.randn((b, S, H, d), device=dev).to(torch.bfloat16)
+        la = torch.randn((b, H, S), device=dev)
+        lb = torch.randn((b, H, S), device=dev)
+        t, _ = timer(lambda: cp.lse_merge(oa, la, ob, lb), steps)
+        mbytes = b * S * H * ((8 + 2) * d + 12)
+        gbs = mbytes / (t * 1e-3) / 1e9
+        del oa, ob, la, lb
+        torch.cuda.empty_cache()
+        return {"shape": [b, S, H, d], "gbs": gbs, "frac_of_measured_hbm": gbs / hbm, "frac_of_8tbs": gbs / 8000.0,
+                "bytes_per_launch": mbytes, "ms_per_launch": t}
+
+    if "merge" in legs:
+        w2, w5 = W.BY_NAME["llama3_8b_s8k_zigzag4"], W.BY_NAME["noncausal_s64k_contig32"]
+        out["merge"] = {w2.name: merge_gbs(w2.b, w2.S, w2.hq, w2.d), w5.name: merge_gbs(w5.b, w5.S, w5.hq, w5.d)}
+
+    if "configs" in legs:
+        cfgs = {}
+        for wx in W.WORKLOADS:
+            if wx.dtype != "bf16" or wx.n_docs != 1:
+                continue
+            same = wx.name == w.name
+            if same:
+                qx, kx, vx, ox, lx = qd, kd, vd, o, lse
+            else:
+                qx, kx, vx = (cp.layout_permute(t.to(dev), wx.layout, wx.N) for t in W.make_inputs(wx))
+                ox = torch.empty_like(qx)
+                lx = torch.empty((wx.b, wx.hq, wx.S), dtype=torch.float32, device=dev)
+            flops = wx.effective_flops()
+            ent = {}
+            modes = ["fused"] if not same else []
+            if wx.name in ("llama3_8b_s8k_zigzag4", "noncausal_s64k_contig32") or same:
+                modes += ["stepwise", "stepwise_epi"]
+            for mode in modes:
+                need = cp.ring_workspace_bytes(wx.layout, wx.N, mode, 0, wx.b, wx.S, wx.hq, wx.d)
+                ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+                st = 3 if same else steps
+                t, _ = timer(lambda: cp.ring_attn_fwd(qx, kx, vx, wx.layout, wx.N, wx.causal, o=ox, lse=lx, mode=mode,
+                                                      workspace=ws), st)
+                e = tflops_entry(flops, t, peak_tf, peak_src,
+                                 launches_per_step=1 if mode == "fused" else (wx.N if mode == "stepwise_epi"
+                                                                              else 2 * wx.N - 1))
+                if mode == "stepwise":
+                    # share of the N - 1 standalone merges, from one merge timed alone at this size
+                    oa = torch.empty((wx.b, wx.S, wx.hq, wx.d), dtype=torch.float32, device=dev)
+                    ob = torch.empty((wx.b, wx.S, wx.hq, wx.d), dtype=torch.bfloat16, device=dev)
+                    la = torch.zeros((wx.b, wx.hq, wx.S), dtype=torch.float32, device=dev)
+                    lb = torch.zeros((wx.b, wx.hq, wx.S), dtype=torch.float32, device=dev)
+                    tm, _ = timer(lambda: cp.lse_merge(oa, la, ob, lb), steps)
+                    mb = wx.b * wx.S * wx.hq * ((8 + 2) * wx.d + 12)
+                    e["merge"] = {"ms_per_merge": tm, "merges_per_step": wx.N - 1,
+                                  "share_of_step": (wx.N - 1) * tm / t, "gbs": mb / (tm * 1e-3) / 1e9,
+                                  "how": "one standalone merge of this size timed alone, times N - 1"}
+                    del oa, ob, la, lb
+                ent[mode] = e
+                del ws
+            cfgs[wx.name] = ent
+            if not same:
+                del qx, kx, vx, ox, lx
+            torch.cuda.empty_cache()
+        out["configs"] = cfgs
+
+    def bwd(wx, qx, kx, vx, ox, lx, n_steps):
+        dor = cp.layout_permute(W.make_do(wx).to(dev), wx.layout, wx.N)
+        cp.ring_attn_fwd(qx, kx, vx, wx.layout, wx.N, wx.causal, o=ox, lse=lx)
+        wsb = torch.empty(cp.ring_bwd_workspace_bytes(wx.layout, wx.N, 0, wx.b, wx.S, wx.hq, wx.d),
+                          dtype=torch.uint8, device=dev)
+        dq, dk, dv = torch.empty_like(qx), torch.empty_like(kx), torch.empty_like(vx)
+        t, _ = timer(lambda: cp.ring_attn_bwd(qx, kx, vx, ox, lx, dor, wx.layout, wx.N, wx.causal, None, dq, dk, dv,
+                                              wsb), n_steps)
+        cp.stream_check()
+        del dor, wsb, dq, dk, dv
+        torch.cuda.empty_cache()
+        return tflops_entry(2.5 * wx.effective_flops(), t, peak_tf, peak_src, launches_per_step=3,
+                            kernel="attn_bwd_kernel",
+                            timed="whole call: statistics + attn_bwd_kernel + dq conversion")
+
+    if "backward" in legs and w.dtype == "bf16" and w.d == 128:
+        b = {"metric": "ring-attn bwd TFLOP/s (effective: 5 products of 2*d flops per visible pair)"}
+        b[w.name] = bwd(w, qd, kd, vd, o, lse, 3)
+        w2 = W.BY_NAME["llama3_8b_s8k_zigzag4"]
+        if w2.name != w.name:
+            q2, k2, v2 = (cp.layout_permute(t.to(dev), w2.layout, w2.N) for t in W.make_inputs(w2))
+            o2, l2 = torch.empty_like(q2), torch.empty((w2.b, w2.hq, w2.S), dtype=torch.float32, device=dev)
+            b[w2.name] = bwd(w2, q2, k2, v2, o2, l2, steps)
+            del q2, k2, v2, o2, l2
+            torch.cuda.empty_cache()
+        out["backward"] = b
+
+    if "allgather" in legs:
+        ag = {"metric": "all-gather CP TFLOP/s (causal document mask, effective FLOPs)"}
+        for name in ("llama3_8b_s8k_zigzag4_docs8", "llama3_8b_s8k_zigzag4_docs32"):
+            wd = W.BY_NAME[name]
+            docs = wd.doc_starts()
+            qa, ka, va = (cp.layout_permute(t.to(dev), wd.layout, wd.N) for t in W.make_inputs(wd))
+            oa = torch.empty_like(qa)
+            la = torch.empty((wd.b, wd.hq, wd.S), dtype=torch.float32, device=dev)
+            wsa = torch.empty(cp.allgather_workspace_bytes(wd.N, 0, wd.b, wd.S, wd.hkv, wd.d, len(docs)),
+                              dtype=torch.uint8, device=dev)
+            t, _ = timer(lambda: cp.allgather_attn_fwd(qa, ka, va, wd.layout, wd.N, wd.causal, docs, None, oa, la,
+                                                       wsa), steps)
+            cp.stream_check()
+            e = {"n_docs": len(docs),
+                 "forward": tflops_entry(wd.effective_flops(), t, peak_tf, peak_src, launches_per_step=3,
+                                         kernel="attn_tc_kernel (document variant)",
+                                         timed="whole call: K and V gather + document-masked attention")}
+            doa = cp.layout_permute(W.make_do(wd).to(dev), wd.layout, wd.N)
+            gq, gk, gv = torch.empty_like(qa), torch.empty_like(ka), torch.empty_like(va)
+            wsb = torch.empty(cp.lib().cp_allgather_bwd_workspace_bytes(wd.N, 0, wd.b, wd.S, wd.hq, wd.hkv, wd.d,
+                                                                        len(docs)), dtype=torch.uint8, device=dev)
+            tb, _ = timer(lambda: cp.allgather_attn_bwd(qa, ka, va, oa, la, doa, wd.layout, wd.N, wd.causal, docs,
+                                                        None, gq, gk, gv, wsb), steps)
+            cp.stream_check()
+            e["backward"] = tflops_entry(2.5 * wd.effective_flops(), tb, peak_tf, peak_src, launches_per_step=7,
+                                         timed="K, V gather + statistics + backward kernel + dq conversion"
+                                               " + dK, dV scatter")
+            ag[name] = e
+            del qa, ka, va, oa, la, wsa, doa, gq, gk, gv, wsb
+            torch.cuda.empty_cache()
+        out["allgather"] = ag
+
+    if "ulysses" in legs:
+        w2 = W.BY_NAME["llama3_8b_s8k_zigzag4"]
+
+        def uly(P, usp):
+            qu, ku, vu = (t.to(dev) for t in W.make_inputs(w2))
+            if usp:
+                qu, ku, vu = (cp.layout_permute(t, w2.layout, w2.N) for t in (qu, ku, vu))
+            ou = torch.empty_like(qu)
+            lu = torch.empty((w2.b, w2.hq, w2.S), dtype=torch.float32, device=dev)
+            wsu = torch.empty(cp.ulysses_workspace_bytes(P, 0, w2.b, w2.S, w2.hq, w2.hkv, w2.d), dtype=torch.uint8,
+                              device=dev)
+            if usp:
+                fn = lambda: cp.usp_attn_fwd(qu, ku, vu, w2.layout, w2.N, P, w2.causal, None, ou, lu, wsu)  # noqa
+            else:
+                fn = lambda: cp.ulysses_attn_fwd(qu, ku, vu, P, w2.causal, None, ou, lu, wsu)  # noqa
+            t, _ = timer(fn, steps)
+            cp.stream_check()
+            del qu, ku, vu, ou, lu, wsu
+            torch.cuda.empty_cache()
+            return tflops_entry(w2.effective_flops(), t, peak_tf, peak_src, P=P, launches_per_step=6,
+                                ring={"layout": w2.layout, "N": w2.N} if usp else None,
+                                timed="whole call: 5 all-to-all launches + attention")
+
+        out["ulysses"] = {"workload": w2.name, "ulysses_P4": uly(4, False), "usp_P2": uly(2, True)}
+    return out
+
+
+def cpu_baseline(w, inputs):
+    """The oracle on all host threads and on one, with the full run extrapolated."""
+    import oracle
+    rate, desc, threads = cpu_oracle_rate(w, inputs=inputs)
+    rate1, desc1, _ = cpu_oracle_rate(w, seconds_target=8.0, seed=1, threads=1, inputs=inputs)
+    full = w.effective_flops()
+    return {"value": rate, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+            "single_thread": {"value": rate1, "unit": "TFLOP/s", "cores": 1, "sample": desc1},
+            "full_run_s_extrapolated": {"all_threads": full / (rate * 1e12), "single_thread": full / (rate1 * 1e12),
+                                        "how": "extrapolated: the workload's effective FLOPs / the sampled rate"},
+            "host_threads_available": len(os.sched_getaffinity(0)), "oracle_default_threads": oracle.default_threads()}
+
+
+def run_one_gpu(args):
     import torch
-    import torch.distributed as dist
 
     import context_attention_cp_b200 as cp
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
     w = W.BY_NAME[args.workload]
     peaks, peak_src = load_peaks()
-    q, k, v = W.make_inputs(w)
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    inputs = W.make_inputs(w)
+    q, k, v = inputs
     qd, kd, vd = (cp.layout_permute(t.to(dev), w.layout, w.N) for t in (q, k, v))
     o = torch.empty_like(qd)
     lse = torch.empty((w.b, w.hq, w.S), dtype=torch.float32, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    ws_bytes = cp.ring_workspace_bytes(w.layout, w.N, args.mode, 0 if w.dtype == "bf16" else 1,
-                                       w.b, w.S, w.hq, w.d)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ws_bytes = cp.ring_workspace_bytes(w.layout, w.N, args.mode, 0 if w.dtype == "bf16" else 1, w.b, w.S, w.hq, w.d)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
-        cp.ring_attn_fwd(qd, kd, vd, w.layout, w.N, w.causal, w.scale, o=o, lse=lse, mode=args.mode,
-                         workspace=ws)
+        cp.ring_attn_fwd(qd, kd, vd, w.layout, w.N, w.causal, o=o, lse=lse, mode=args.mode, workspace=ws)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -248,12 +454,9 @@ def main():
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
-    if clocks:
-        clocks.start()
-        time.sleep(0.3)
-    if world > 1:
-        dist.barrier()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
     torch.cuda.synchronize()
     for i in range(args.steps):
         flush.zero_()
@@ -261,220 +464,27 @@ def main():
         step()
         ends[i].record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop() if clocks else None
+    clk = clocks.stop()
     cp.stream_check()
     times = [s.elapsed_time(e) for s, e in zip(starts, ends)]  # ms
-    total_ms = reduce_max(sum(times), world, dev)
+    total_ms = sum(times)
     ms_per_step = total_ms / args.steps
     flops = w.effective_flops()
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
-    launches_per_step = 1 if (args.mode == "fused" or w.N == 1) else (2 * w.N - 1)
+    value = flops * args.steps / (total_ms * 1e-3) / 1e12
+    launches_per_step = {"fused": 1, "stepwise": 2 * w.N - 1, "stepwise_epi": w.N}[args.mode] if w.N > 1 else 1
 
-    # dominant kernel: the attention kernel (the whole fused ring is one launch)
-    per_launch_tflops = flops / (ms_per_step * 1e-3) / 1e12 if args.mode == "fused" else None
-    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-
-    # standalone merge bandwidth: one merge of a [b, S, Hq, d] fp32 accumulator with a
-    # bf16 partial, bytes per (row, head) = (8 + 2) * d + 12; measured at this
-    # workload's partial size and at the non-causal 64K workload's (16 heads), the
-    # case with 31 merges per rank
-    def merge_gbs(b, S, H, d):
-        oa = torch.randn((b, S, H, d), device=dev)
-        ob = torch.randn((b, S, H, d), device=dev).to(torch.bfloat16)
-        la = torch.randn((b, H, S), device=dev)
-        lb = torch.randn((b, H, S), device=dev)
-        for _ in range(3):
-            cp.lse_merge(oa, la, ob, lb)
-        ms = []
-        for _ in range(10):
-            flush.zero_()
-            m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            m0.record(stream)
-            cp.lse_merge(oa, la, ob, lb)
-            m1.record(stream)
-            torch.cuda.synchronize()
-            ms.append(m0.elapsed_time(m1))
-        mbytes = b * S * H * ((8 + 2) * d + 12)
-        t = statistics.mean(ms)
-        gbs = mbytes / (t * 1e-3) / 1e9
-        del oa, ob, la, lb
-        return {"shape": [b, S, H, d], "gbs": gbs, "frac_of_measured_hbm": gbs / peaks.get("hbm_gbs", 6650.0),
-                "frac_of_8tbs": gbs / 8000.0, "bytes_per_launch": mbytes, "ms_per_launch": t}
-
-    merge = None
-    if w.dtype == "bf16" and rank == 0:
-        merge = merge_gbs(w.b, w.S, w.hq, w.d)
-        w5 = W.BY_NAME["noncausal_s64k_contig32"]
-        merge["noncausal_s64k_contig32"] = merge_gbs(w5.b, w5.S, w5.hq, w5.d)
-        torch.cuda.empty_cache()
-
-    # backward of the same workload (cp_ring_attn_bwd: statistics pass, the tcgen05
-    # kernel, dq conversion), inputs resident, L2 flushed before every timed call;
-    # effective FLOPs = 2.5x the forward's (five 2*d-flop products per visible pair)
-    def bwd_leg():
-        do = W.make_do(w).to(dev)
-        dor = cp.layout_permute(do, w.layout, w.N)
-        del do
-        step()
-        wsb = torch.empty(cp.ring_bwd_workspace_bytes(w.layout, w.N, 0, w.b, w.S, w.hq, w.d), dtype=torch.uint8,
-                          device=dev)
-        dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
-
-        def bstep():
-            cp.ring_attn_bwd(qd, kd, vd, o, lse, dor, w.layout, w.N, w.causal, w.scale, dq, dk, dv, wsb)
-
-        for _ in range(3):
-            bstep()
-        ms = []
-        for _ in range(max(3, min(args.steps, 10))):
-            flush.zero_()
-            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            b0.record(stream)
-            bstep()
-            b1.record(stream)
-            torch.cuda.synchronize()
-            ms.append(b0.elapsed_time(b1))
-        cp.stream_check()
-        t = statistics.mean(ms)
-        tf = 2.5 * flops / (t * 1e-3) / 1e12
-        del dor, wsb, dq, dk, dv
-        torch.cuda.empty_cache()
-        return {"metric": "ring-attn bwd TFLOP/s (effective: 5 products of 2*d flops per visible pair)",
-                "value": tf, "unit": "TFLOP/s", "ms_per_step": t, "steps": len(ms), "launches_per_step": 3,
-                "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel", "achieved": tf, "peak": peak_tf,
-                             "unit": "TFLOP/s", "frac": tf / peak_tf, "peak_source": peak_src + " bf16 burst",
-                             "timed": "whole call: statistics + attn_bwd_kernel + dq conversion",
-                             "traffic": None}}
-
-    backward = None
-    if w.dtype == "bf16" and w.d == 128 and rank == 0:
-        backward = bwd_leg()
-
-    # All-Gather CP with a document mask (cp_allgather_attn_fwd: K and V gathered
-    # into original order by two permute launches, then one document-masked pass),
-    # on the 8-document variant of the 8B workload; effective FLOPs count only the
-    # pairs the causal document mask leaves visible
-    def allgather_leg():
-        wd = W.BY_NAME["llama3_8b_s8k_zigzag4_docs8"]
-        docs = wd.doc_starts()
-        qa, ka, va = (cp.layout_permute(t.to(dev), wd.layout, wd.N) for t in W.make_inputs(wd))
-        oa = torch.empty_like(qa)
-        la = torch.empty((wd.b, wd.hq, wd.S), dtype=torch.float32, device=dev)
-        wsa = torch.empty(cp.allgather_workspace_bytes(wd.N, 0, wd.b, wd.S, wd.hkv, wd.d, len(docs)),
-                          dtype=torch.uint8, device=dev)
-
-        def astep():
-            cp.allgather_attn_fwd(qa, ka, va, wd.layout, wd.N, wd.causal, docs, wd.scale, oa, la, wsa)
-
-        for _ in range(3):
-            astep()
-        ms = []
-        for _ in range(max(3, min(args.steps, 10))):
-            flush.zero_()
-            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            astep()
-            a1.record(stream)
-            torch.cuda.synchronize()
-            ms.append(a0.elapsed_time(a1))
-        cp.stream_check()
-        t = statistics.mean(ms)
-        tf = wd.effective_flops() / (t * 1e-3) / 1e12
-        # its backward (gather, document-masked backward, dK/dV back to the ranks)
-        doa = cp.layout_permute(W.random_do(wd.b, wd.S, wd.hq, wd.d, wd.dtype, wd.seed).to(dev), wd.layout, wd.N)
-        gq, gk, gv = torch.empty_like(qa), torch.empty_like(ka), torch.empty_like(va)
-        wsb = torch.empty(cp.lib().cp_allgather_bwd_workspace_bytes(wd.N, 0, wd.b, wd.S, wd.hq, wd.hkv, wd.d, len(docs)),
-                          dtype=torch.uint8, device=dev)
-
-        def bstep():
-            cp.allgather_attn_bwd(qa, ka, va, oa, la, doa, wd.layout, wd.N, wd.causal, docs, wd.scale, gq, gk, gv, wsb)
-
-        for _ in range(3):
-            bstep()
-        bms = []
-        for _ in range(max(3, min(args.steps, 10))):
-            flush.zero_()
-            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            bstep()
-            a1.record(stream)
-            torch.cuda.synchronize()
-            bms.append(a0.elapsed_time(a1))
-        cp.stream_check()
-        tb = statistics.mean(bms)
-        tfb = 2.5 * wd.effective_flops() / (tb * 1e-3) / 1e12
-        del qa, ka, va, oa, la, wsa, doa, gq, gk, gv, wsb
-        torch.cuda.empty_cache()
-        return {"metric": "all-gather CP fwd TFLOP/s (causal document mask, effective FLOPs)", "workload": wd.name,
-                "backward": {"value": tfb, "unit": "TFLOP/s", "ms_per_step": tb, "frac": tfb / peak_tf,
-                             "launches_per_step": 7,
-                             "timed": "K, V gather + statistics + backward kernel + dq conversion + dK, dV scatter"},
-                "n_docs": len(docs), "value": tf, "unit": "TFLOP/s", "ms_per_step": t, "steps": len(ms),
-                "launches_per_step": 3,
-                "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (document variant)", "achieved": tf,
-                             "peak": peak_tf, "unit": "TFLOP/s", "frac": tf / peak_tf,
-                             "peak_source": peak_src + " bf16 burst",
-                             "timed": "whole call: K and V gather + document-masked attention", "traffic": None}}
-
-    allgather = None
-    if w.dtype == "bf16" and w.d == 128 and rank == 0:
-        allgather = allgather_leg()
-
-    # Ulysses over P = 4 virtual ranks on this workload's shape (original order):
-    # all-to-all of q, k, v, one attention launch over the head groups, all-to-all
-    # of o and lse back (5 + 1 launches)
-    def ulysses_leg(P=4, usp=False):
-        # usp: Ulysses groups of P inside each of the workload's N ring groups (the
-        # inputs in the ring's rank-major order, permuted before the timed region)
-        qu, ku, vu = (t.to(dev) for t in W.make_inputs(w))
-        if usp:
-            qu, ku, vu = (cp.layout_permute(t, w.layout, w.N) for t in (qu, ku, vu))
-        ou = torch.empty_like(qu)
-        lu = torch.empty((w.b, w.hq, w.S), dtype=torch.float32, device=dev)
-        wsu = torch.empty(cp.ulysses_workspace_bytes(P, 0, w.b, w.S, w.hq, w.hkv, w.d), dtype=torch.uint8, device=dev)
-
-        def ustep():
-            if usp:
-                cp.usp_attn_fwd(qu, ku, vu, w.layout, w.N, P, w.causal, w.scale, ou, lu, wsu)
-            else:
-                cp.ulysses_attn_fwd(qu, ku, vu, P, w.causal, w.scale, ou, lu, wsu)
-
-        for _ in range(3):
-            ustep()
-        ms = []
-        for _ in range(max(3, min(args.steps, 10))):
-            flush.zero_()
-            u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            u0.record(stream)
-            ustep()
-            u1.record(stream)
-            torch.cuda.synchronize()
-            ms.append(u0.elapsed_time(u1))
-        cp.stream_check()
-        t = statistics.mean(ms)
-        tf = flops / (t * 1e-3) / 1e12
-        del qu, ku, vu, ou, lu, wsu
-        torch.cuda.empty_cache()
-        return {"metric": ("USP" if usp else "Ulysses") + " fwd TFLOP/s (causal, effective FLOPs)", "P": P,
-                "ring": {"layout": w.layout, "N": w.N} if usp else None, "value": tf, "unit": "TFLOP/s",
-                "ms_per_step": t, "steps": len(ms), "launches_per_step": 6,
-                "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": tf, "peak": peak_tf,
-                             "unit": "TFLOP/s", "frac": tf / peak_tf, "peak_source": peak_src + " bf16 burst",
-                             "timed": "whole call: 5 all-to-all launches + attention", "traffic": None}}
-
-    ulysses = None
-    if w.dtype == "bf16" and w.hkv % 4 == 0 and w.hq % 4 == 0 and w.S % 4 == 0 and rank == 0:
-        ulysses = ulysses_leg()
-        if w.hkv % 2 == 0 and w.S % (2 * w.N) == 0:
-            ulysses["usp"] = ulysses_leg(P=2, usp=True)
+    legs = set(args.legs.split(",")) if args.legs not in ("all", "none") else (
+        {"merge", "configs", "backward", "allgather", "ulysses"} if args.legs == "all" else set())
+    timer = Timer(torch, flush)
+    extra = run_legs(cp, torch, dev, w, qd, kd, vd, o, lse, timer, peaks, peak_src, args, legs) if legs else {}
 
     # end to end through the public API, every step: pinned host -> device copy of
     # q/k/v, permute to rank-major order, ring attention, unpermute, device -> host
     # copy of o and lse.  Consecutive steps are pipelined on three streams (copy-in,
     # compute, copy-out) with double-buffered device tensors, as a serving loop would
     # run them; the time runs from the first copy-in to the last copy-out.
+    del flush
+    torch.cuda.empty_cache()
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
     oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     lh = torch.empty((w.b, w.hq, w.S), dtype=torch.float32).pin_memory()
@@ -497,7 +507,7 @@ def main():
             s_cmp.wait_event(ev_in[sl])
             s_cmp.wait_event(ev_out[sl])  # step i-2's outputs have left the device
             qr, kr, vr = (cp.layout_permute(t, w.layout, w.N) for t in buf_in[sl])
-            og, lg = cp.ring_attn_fwd(qr, kr, vr, w.layout, w.N, w.causal, w.scale, mode=args.mode, workspace=ws)
+            og, lg = cp.ring_attn_fwd(qr, kr, vr, w.layout, w.N, w.causal, mode=args.mode, workspace=ws)
             cp.layout_permute(og, w.layout, w.N, inverse=True, out=buf_out[sl][0])
             cp.layout_permute(lg, w.layout, w.N, seq_axis=2, inverse=True, out=buf_out[sl][1])
             ev_cmp[sl].record(s_cmp)
@@ -512,8 +522,6 @@ def main():
     torch.cuda.synchronize()
     e_steps = max(3, min(args.steps, 10))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
     torch.cuda.synchronize()
     e0.record(s_in)
     for i in range(e_steps):
@@ -522,47 +530,206 @@ def main():
     e1.record(s_in)
     torch.cuda.synchronize()
     cp.stream_check()
-    e_ms = reduce_max(e0.elapsed_time(e1), world, dev)
-    e2e_value = world * flops * e_steps / (e_ms * 1e-3) / 1e12
+    e_ms = e0.elapsed_time(e1)
+    e2e_value = flops * e_steps / (e_ms * 1e-3) / 1e12
     es = 2 if w.dtype == "bf16" else 4
     h2d = (q.numel() + k.numel() + v.numel()) * es
     d2h = q.numel() * es + w.b * w.hq * w.S * 4
+    del buf_in, buf_out, qh, kh, vh, oh, lh
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, desc, threads = cpu_oracle_rate(w)
-        cpu = {"value": rate, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+    cpu = None if args.no_cpu_baseline else cpu_baseline(w, inputs)
+    achieved = flops / (ms_per_step * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "b": w.b, "S": w.S, "hq": w.hq, "hkv": w.hkv, "d": w.d,
+                   "layout": w.layout, "N": w.N, "causal": w.causal, "mode": args.mode,
+                   "l2": "flushed before every timed step (256 MiB write); inputs also exceed L2",
+                   "parallelism": "one GPU, %d virtual ranks" % w.N},
+        "pct_bf16_peak": value / peak_tf,
+        "pct_vendor_bf16_dense": value / VENDOR_BF16_DENSE_TFLOPS,
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel" if args.mode == "fused" or w.dtype == "bf16"
+                     else "attn_simt_kernel",
+                     "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
+                     "peak_source": peak_src + " bf16 burst",
+                     "secondary": {"peak": VENDOR_BF16_DENSE_TFLOPS, "frac": achieved / VENDOR_BF16_DENSE_TFLOPS,
+                                   "source": "vendor dense bf16 (2:4-sparse figure halved)"},
+                     "sustained": {"peak": peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]),
+                                   "frac": achieved / peaks.get("bf16_tflops_sustained",
+                                                                FALLBACK_PEAKS["bf16_tflops_sustained"]),
+                                   "source": peak_src + " bf16 sustained (seconds of back-to-back GEMMs under the power"
+                                             " cap)", "timed_region_s": total_ms / 1e3,
+                                   "power_capped": bool(clk and "sw_power_cap" in clk.get("reasons", []))},
+                     "timed": "whole call (one launch in fused mode), CUDA events on the launching stream",
+                     "traffic": profiled_traffic(w.name) if args.mode == "fused" else None},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e_ms / e_steps, "pipelined": "copy-in / compute / copy-out on 3 streams"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    line.update(extra)
+    print(json.dumps(line), flush=True)
+    return 0
 
+
+def dist_inputs(w, rank, world, dev, torch):
+    """This rank's layout block of the workload (c = S / world tokens), drawn on the
+    device from a generator seeded with the workload's seed and the rank (every
+    rank draws only its own tokens)."""
+    c = w.S // world
+    g = torch.Generator(device=dev).manual_seed(w.seed * 1000 + rank)
+    td = W.torch_dtype(w.dtype)
+    q = torch.randn((w.b, c, w.hq, w.d), generator=g, device=dev, dtype=torch.float32).to(td)
+    k = torch.randn((w.b, c, w.hkv, w.d), generator=g, device=dev, dtype=torch.float32).to(td)
+    v = torch.randn((w.b, c, w.hkv, w.d), generator=g, device=dev, dtype=torch.float32).to(td)
+    if w.k_scale != 1.0:
+        k = k * w.k_scale
+    return q, k, v
+
+
+def run_dist(args, ring_kw=None, device=None, backend="nccl"):
+    """The ring across real ranks: one process per GPU (see the module docstring).
+
+    ring_kw / device / backend exist for the CPU test of this plumbing (gloo ranks,
+    injected block and merge steps); the bench itself uses the defaults."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from context_attention_cp_b200 import ring_dist
+
+    world = int(os.environ["WORLD_SIZE"])
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    if device is None:
+        torch.cuda.set_device(local)
+        device = torch.device("cuda", local)
+    cuda = device.type == "cuda"
+    w = W.BY_NAME[args.workload]
+    if w.S % world or (w.layout == "zigzag" and w.S % (2 * world)):
+        raise SystemExit("the workload's S does not split over %d ranks" % world)
+    peaks, peak_src = load_peaks()
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    q, k, v = dist_inputs(w, rank, world, device, torch)
+    kw = dict(ring_kw or {})
+
+    def step():
+        return ring_dist.ring_attn_fwd_dist(q, k, v, w.layout, w.causal, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    if cuda:
+        torch.cuda.synchronize()
+    dist.barrier()
+    clocks = ClockSampler(local) if (cuda and rank == 0) else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    if cuda:
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    if cuda:
+        e1.record()
+        torch.cuda.synchronize()
+        my_ms = e0.elapsed_time(e1)
+    else:
+        my_ms = (time.perf_counter() - t0) * 1e3
+    dist.barrier()
+    clk = clocks.stop() if clocks else None
+    total_ms = reduce_max(my_ms, world, device)
+    ms_per_step = total_ms / args.steps
+    flops = w.effective_flops()
+    value = flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    # end to end: this rank's inputs from pinned host memory, the ring, o and lse back
+    qh, kh, vh = (t.cpu() for t in (q, k, v))
+    if cuda:
+        qh, kh, vh = (t.pin_memory() for t in (qh, kh, vh))
+    e_steps = max(3, min(args.steps, 5))
+    dist.barrier()
+    t1 = time.perf_counter()
+    if cuda:
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record()
+    for _ in range(e_steps):
+        qx, kx, vx = (t.to(device, non_blocking=True) for t in (qh, kh, vh))
+        ox, lx = ring_dist.ring_attn_fwd_dist(qx, kx, vx, w.layout, w.causal, **kw)
+        ox.cpu(), lx.cpu()
+    if cuda:
+        f1.record()
+        torch.cuda.synchronize()
+        e_my = f0.elapsed_time(f1)
+    else:
+        e_my = (time.perf_counter() - t1) * 1e3
+    e_ms = reduce_max(e_my, world, device)
+    es = 2 if w.dtype == "bf16" else 4
+    h2d = world * (q.numel() + k.numel() + v.numel()) * es
+    d2h = world * (q.numel() * es + w.b * w.hq * (w.S // world) * 4)
+    dist.barrier()
     if rank == 0:
+        per_gpu = value / world
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (per-rank device generator)",
             "config": {"workload": w.name, "b": w.b, "S": w.S, "hq": w.hq, "hkv": w.hkv, "d": w.d,
-                       "layout": w.layout, "N": w.N, "causal": w.causal, "mode": args.mode,
-                       "l2": "flushed before every timed step (256 MiB write)",
-                       "parallelism": "replicas x%d" % world},
-            "pct_bf16_peak": value / world / peak_tf,
-            "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel",
-                         "achieved": per_launch_tflops, "peak": peak_tf, "unit": "TFLOP/s",
-                         "frac": (per_launch_tflops / peak_tf) if per_launch_tflops else None,
-                         "peak_source": peak_src + " bf16 burst",
-                         "traffic": profiled_traffic() if w.name == W.BENCH_WORKLOAD else None},
-            "merge": merge,
-            "backward": backward,
-            "allgather": allgather,
-            "ulysses": ulysses,
-            "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e_ms / e_steps, "pipelined": "copy-in / compute / copy-out on 3 streams"},
-            "gpu_launches": launches_per_step * args.steps,
+                       "layout": w.layout, "N": world, "causal": w.causal,
+                       "l2": "inputs exceed L2 (no flush between steps)",
+                       "parallelism": "ring over %d real ranks (K/V blocks passed with NCCL point-to-point)" % world},
+            "pct_bf16_peak": per_gpu / peak_tf,
+            "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (block form, one launch per ring step)",
+                         "achieved": per_gpu, "peak": peak_tf, "unit": "TFLOP/s", "frac": per_gpu / peak_tf,
+                         "peak_source": peak_src + " bf16 burst", "timed": "whole ring per rank, max over ranks",
+                         "traffic": None},
+            "cpu_baseline": None,
+            "e2e": {"value": flops * e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / e_steps},
+            "gpu_launches": world * args.steps * (w_launches_dist(world)),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    dist.barrier()
+    dist.destroy_process_group()
     return 0
+
+
+def w_launches_dist(world):
+    """Kernels of this library one rank launches per ring: a block launch per step
+    plus, on the last step, the block launch into a partial and the merge that
+    writes the output (see ring_dist.ring_attn_fwd_dist)."""
+    return world + 1 if world > 1 else 1
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=W.BENCH_WORKLOAD,
+                    choices=sorted(n for n, x in W.BY_NAME.items() if x.n_docs == 1))
+    ap.add_argument("--mode", default="fused", choices=["fused", "stepwise", "stepwise_epi"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--legs", default="all",
+                    help="comma list of merge,configs,backward,allgather,ulysses; 'all' or 'none'")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        return run_dist(args)
+    return run_one_gpu(args)
 
 
 if __name__ == "__main__":

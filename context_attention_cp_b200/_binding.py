@@ -3,13 +3,17 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-lib_path = os.path.join(_HERE, "libcpattn.so")
+# CP_LIBRARY=debug selects the bounds-checking build (libcpattn_debug.so); a path
+# selects a variant built with `build --define ... --out PATH`
+_choice = os.environ.get("CP_LIBRARY", "")
+lib_path = (os.path.join(_HERE, "libcpattn_debug.so") if _choice == "debug"
+            else os.path.abspath(_choice) if _choice else os.path.join(_HERE, "libcpattn.so"))
 
 CP_BF16, CP_FP32 = 0, 1
 LAYOUTS = {"contiguous": 0, "zigzag": 1, "striped": 2}
-MODES = {"fused": 0, "stepwise": 1}
+MODES = {"fused": 0, "stepwise": 1, "stepwise_epi": 2}
 STATUS = {0: "CP_OK", 1: "CP_ERR_INVALID_ARG", 2: "CP_ERR_UNSUPPORTED", 3: "CP_ERR_SHAPE",
-          4: "CP_ERR_CUDA", 5: "CP_ERR_TIMEOUT"}
+          4: "CP_ERR_CUDA", 5: "CP_ERR_TIMEOUT", 6: "CP_ERR_BOUNDS"}
 
 
 class CPError(RuntimeError):
@@ -129,6 +133,11 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
+def _scale(scale):
+    """The softmax scale for the C ABI: None asks the library for 1/sqrt(d) (0.0)."""
+    return 0.0 if scale is None else float(scale)
+
+
 def _range(r):
     """(starts, lens, stride) -> cp_range."""
     starts, lens, stride = r
@@ -164,7 +173,7 @@ def block_attn_fwd(q, k, v, q_range, kv_range, causal, scale, o, lse, accumulate
     qr, kr = _range(q_range), _range(kv_range)
     tq, tk, tv, to, tl = _tensor(q), _tensor(k), _tensor(v), _tensor(o), _tensor(lse)
     _check(lib().cp_block_attn_fwd(_ref(tq), _ref(tk), _ref(tv), ctypes.byref(qr), ctypes.byref(kr),
-                                   int(bool(causal)), float(scale), _ref(to), _ref(tl), int(bool(accumulate)),
+                                   int(bool(causal)), _scale(scale), _ref(to), _ref(tl), int(bool(accumulate)),
                                    _stream()))
     return o, lse
 
@@ -181,7 +190,7 @@ def block_attn_bwd(q, k, v, o, lse, do, q_range, kv_range, causal, scale, dq_acc
     qr, kr = _range(q_range), _range(kv_range)
     ts = [_tensor(t) for t in (q, k, v, o, lse, do, dq_acc, dk_acc, dv_acc)]
     _check(lib().cp_block_attn_bwd(*[_ref(t) for t in ts[:6]], ctypes.byref(qr), ctypes.byref(kr), int(bool(causal)),
-                                   float(scale), *[_ref(t) for t in ts[6:]], ctypes.c_void_p(workspace.data_ptr()), need,
+                                   _scale(scale), *[_ref(t) for t in ts[6:]], ctypes.c_void_p(workspace.data_ptr()), need,
                                    _stream()))
     return dq_acc, dk_acc, dv_acc
 
@@ -201,7 +210,7 @@ def ring_attn_fwd(q, k, v, layout, N, causal, scale=None, o=None, lse=None, mode
     import torch
     b, S, Hq, d = q.shape
     if scale is None:
-        scale = d ** -0.5
+        scale = 0.0  # the library's default: 1/sqrt(d)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
@@ -212,7 +221,7 @@ def ring_attn_fwd(q, k, v, layout, N, causal, scale=None, o=None, lse=None, mode
     ws_ptr = ctypes.c_void_p(workspace.data_ptr()) if (need and workspace is not None) else None
     tq, tk, tv, to, tl = _tensor(q), _tensor(k), _tensor(v), _tensor(o), _tensor(lse)
     _check(lib().cp_ring_attn_fwd(LAYOUTS[layout], N, int(bool(causal)), _ref(tq), _ref(tk), _ref(tv),
-                                  float(scale), _ref(to), _ref(tl), MODES[mode], ws_ptr, need, _stream()))
+                                  _scale(scale), _ref(to), _ref(tl), MODES[mode], ws_ptr, need, _stream()))
     return o, lse
 
 
@@ -226,7 +235,7 @@ def ring_attn_bwd(q, k, v, o, lse, do, layout, N, causal, scale=None, dq=None, d
     import torch
     b, S, Hq, d = q.shape
     if scale is None:
-        scale = d ** -0.5
+        scale = 0.0  # the library's default: 1/sqrt(d)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -234,7 +243,7 @@ def ring_attn_bwd(q, k, v, o, lse, do, layout, N, causal, scale=None, dq=None, d
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     ts = [_tensor(t) for t in (q, k, v, o, lse, do, dq, dk, dv)]
-    _check(lib().cp_ring_attn_bwd(LAYOUTS[layout], N, int(bool(causal)), *[_ref(t) for t in ts[:6]], float(scale),
+    _check(lib().cp_ring_attn_bwd(LAYOUTS[layout], N, int(bool(causal)), *[_ref(t) for t in ts[:6]], _scale(scale),
                                   *[_ref(t) for t in ts[6:]], ctypes.c_void_p(workspace.data_ptr()), need,
                                   _stream()))
     return dq, dk, dv
@@ -251,7 +260,7 @@ def allgather_attn_fwd(q, k, v, layout, N, causal, doc_starts=None, scale=None, 
     import torch
     b, S, Hq, d = q.shape
     if scale is None:
-        scale = d ** -0.5
+        scale = 0.0  # the library's default: 1/sqrt(d)
     docs = [0] if doc_starts is None else [int(x) for x in doc_starts]
     arr = (ctypes.c_int64 * len(docs))(*docs)
     if o is None:
@@ -263,7 +272,7 @@ def allgather_attn_fwd(q, k, v, layout, N, causal, doc_starts=None, scale=None, 
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     tq, tk, tv, to, tl = _tensor(q), _tensor(k), _tensor(v), _tensor(o), _tensor(lse)
     _check(lib().cp_allgather_attn_fwd(LAYOUTS[layout], N, int(bool(causal)), _ref(tq), _ref(tk), _ref(tv), arr,
-                                       len(docs), float(scale), _ref(to), _ref(tl),
+                                       len(docs), _scale(scale), _ref(to), _ref(tl),
                                        ctypes.c_void_p(workspace.data_ptr()), need, _stream()))
     return o, lse
 
@@ -274,7 +283,7 @@ def allgather_attn_bwd(q, k, v, o, lse, do, layout, N, causal, doc_starts=None, 
     import torch
     b, S, Hq, d = q.shape
     if scale is None:
-        scale = d ** -0.5
+        scale = 0.0  # the library's default: 1/sqrt(d)
     docs = [0] if doc_starts is None else [int(x) for x in doc_starts]
     arr = (ctypes.c_int64 * len(docs))(*docs)
     dq = torch.empty_like(q) if dq is None else dq
@@ -285,7 +294,7 @@ def allgather_attn_bwd(q, k, v, o, lse, do, layout, N, causal, doc_starts=None, 
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     ts = [_tensor(t) for t in (q, k, v, o, lse, do, dq, dk, dv)]
     _check(lib().cp_allgather_attn_bwd(LAYOUTS[layout], N, int(bool(causal)), *[_ref(t) for t in ts[:6]], arr,
-                                       len(docs), float(scale), *[_ref(t) for t in ts[6:]],
+                                       len(docs), _scale(scale), *[_ref(t) for t in ts[6:]],
                                        ctypes.c_void_p(workspace.data_ptr()), need, _stream()))
     return dq, dk, dv
 
@@ -314,14 +323,14 @@ def ulysses_attn_fwd(q, k, v, P, causal, scale=None, o=None, lse=None, workspace
     import torch
     b, S, Hq, d = q.shape
     if scale is None:
-        scale = d ** -0.5
+        scale = 0.0  # the library's default: 1/sqrt(d)
     o = torch.empty_like(q) if o is None else o
     lse = torch.empty((b, Hq, S), dtype=torch.float32, device=q.device) if lse is None else lse
     need = ulysses_workspace_bytes(P, _dtype_code(q), b, S, Hq, k.shape[2], d)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     ts = [_tensor(t) for t in (q, k, v, o, lse)]
-    _check(lib().cp_ulysses_attn_fwd(P, int(bool(causal)), _ref(ts[0]), _ref(ts[1]), _ref(ts[2]), float(scale),
+    _check(lib().cp_ulysses_attn_fwd(P, int(bool(causal)), _ref(ts[0]), _ref(ts[1]), _ref(ts[2]), _scale(scale),
                                      _ref(ts[3]), _ref(ts[4]), ctypes.c_void_p(workspace.data_ptr()), need, _stream()))
     return o, lse
 
@@ -331,7 +340,7 @@ def ulysses_attn_bwd(q, k, v, o, lse, do, P, causal, scale=None, dq=None, dk=Non
     import torch
     b, S, Hq, d = q.shape
     if scale is None:
-        scale = d ** -0.5
+        scale = 0.0  # the library's default: 1/sqrt(d)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -339,7 +348,7 @@ def ulysses_attn_bwd(q, k, v, o, lse, do, P, causal, scale=None, dq=None, dk=Non
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     ts = [_tensor(t) for t in (q, k, v, o, lse, do, dq, dk, dv)]
-    _check(lib().cp_ulysses_attn_bwd(P, int(bool(causal)), *[_ref(t) for t in ts[:6]], float(scale),
+    _check(lib().cp_ulysses_attn_bwd(P, int(bool(causal)), *[_ref(t) for t in ts[:6]], _scale(scale),
                                      *[_ref(t) for t in ts[6:]], ctypes.c_void_p(workspace.data_ptr()), need,
                                      _stream()))
     return dq, dk, dv
@@ -355,7 +364,7 @@ def usp_attn_fwd(q, k, v, layout, N, P, causal, scale=None, o=None, lse=None, wo
     import torch
     b, S, Hq, d = q.shape
     if scale is None:
-        scale = d ** -0.5
+        scale = 0.0  # the library's default: 1/sqrt(d)
     o = torch.empty_like(q) if o is None else o
     lse = torch.empty((b, Hq, S), dtype=torch.float32, device=q.device) if lse is None else lse
     need = usp_workspace_bytes(layout, N, P, _dtype_code(q), b, S, Hq, k.shape[2], d)
@@ -363,7 +372,7 @@ def usp_attn_fwd(q, k, v, layout, N, P, causal, scale=None, o=None, lse=None, wo
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     ts = [_tensor(t) for t in (q, k, v, o, lse)]
     _check(lib().cp_usp_attn_fwd(LAYOUTS[layout], N, P, int(bool(causal)), _ref(ts[0]), _ref(ts[1]), _ref(ts[2]),
-                                 float(scale), _ref(ts[3]), _ref(ts[4]), ctypes.c_void_p(workspace.data_ptr()), need,
+                                 _scale(scale), _ref(ts[3]), _ref(ts[4]), ctypes.c_void_p(workspace.data_ptr()), need,
                                  _stream()))
     return o, lse
 
@@ -373,7 +382,7 @@ def usp_attn_bwd(q, k, v, o, lse, do, layout, N, P, causal, scale=None, dq=None,
     import torch
     b, S, Hq, d = q.shape
     if scale is None:
-        scale = d ** -0.5
+        scale = 0.0  # the library's default: 1/sqrt(d)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -381,7 +390,7 @@ def usp_attn_bwd(q, k, v, o, lse, do, layout, N, P, causal, scale=None, dq=None,
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     ts = [_tensor(t) for t in (q, k, v, o, lse, do, dq, dk, dv)]
-    _check(lib().cp_usp_attn_bwd(LAYOUTS[layout], N, P, int(bool(causal)), *[_ref(t) for t in ts[:6]], float(scale),
+    _check(lib().cp_usp_attn_bwd(LAYOUTS[layout], N, P, int(bool(causal)), *[_ref(t) for t in ts[:6]], _scale(scale),
                                  *[_ref(t) for t in ts[6:]], ctypes.c_void_p(workspace.data_ptr()), need, _stream()))
     return dq, dk, dv
 
@@ -391,7 +400,7 @@ def ring_attn_fwd_static_scratch(q, k, v, layout, N, causal, scale, o, lse):
     scratch, for callers that cannot allocate; o and lse are caller-allocated."""
     tq, tk, tv, to, tl = _tensor(q), _tensor(k), _tensor(v), _tensor(o), _tensor(lse)
     _check(lib().cp_ring_attn_fwd_static_scratch(LAYOUTS[layout], N, int(bool(causal)), _ref(tq), _ref(tk),
-                                                 _ref(tv), float(scale), _ref(to), _ref(tl), _stream()))
+                                                 _ref(tv), _scale(scale), _ref(to), _ref(tl), _stream()))
     return o, lse
 
 

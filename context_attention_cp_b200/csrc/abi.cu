@@ -12,6 +12,8 @@
 #include <tuple>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/cpattn.h"
 #include "bwd.h"
 #include "kernels.h"
@@ -20,6 +22,21 @@
 using namespace cpattn;
 
 namespace {
+
+// NVTX range for profilers (a no-op unless a tool is attached): the entry points and,
+// in the stepwise ring modes, every ring step.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    NvtxRange(const char *fmt, int a, int b)
+    {
+        char buf[64];
+        snprintf(buf, sizeof buf, fmt, a, b);
+        nvtxRangePushA(buf);
+    }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 thread_local char g_last_error[512] = "";
 
@@ -97,6 +114,21 @@ cp_status check_range(const cp_range *r, int64_t len, const char *name)
     return CP_OK;
 }
 
+// The softmax scale: 0 asks for the standard 1 / sqrt(d) ("上下文并行与 Ring
+// Attention", section 分块注意力: x_j = q . k_j / sqrt(d_h)); any other value must be
+// finite and > 0 and is taken as given.
+cp_status resolve_scale(float *scale, int64_t d)
+{
+    if (*scale == 0.f) {
+        if (d <= 0) return fail(CP_ERR_SHAPE, "head dim must be > 0");
+        *scale = (float)(1.0 / std::sqrt((double)d));
+        return CP_OK;
+    }
+    if (!(*scale > 0.f) || !std::isfinite(*scale))
+        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be 0 (1/sqrt(d)) or finite and > 0");
+    return CP_OK;
+}
+
 void set_status_ptr(AttnParams &p)
 {
     int *s = nullptr;
@@ -145,12 +177,16 @@ struct OrderKey {
 std::mutex g_order_mu;
 std::map<OrderKey, std::vector<uint32_t>> g_order_cache;
 
-const std::vector<uint32_t> &ring_order(int layout, int N, int64_t S, int causal, int rows_per_cta)
+// The caches keep at most this many shapes each; a new shape beyond that empties
+// the cache first (orders are copied out under the lock, so nothing refers into it).
+constexpr size_t kOrderCacheMax = 64;
+
+const std::vector<uint32_t> &ring_order_locked(int layout, int N, int64_t S, int causal, int rows_per_cta)
 {
-    std::lock_guard<std::mutex> lk(g_order_mu);
     OrderKey key{layout, N, causal, rows_per_cta, S};
     auto it = g_order_cache.find(key);
     if (it != g_order_cache.end()) return it->second;
+    if (g_order_cache.size() >= kOrderCacheMax) g_order_cache.clear();
     const int64_t c = S / N;
     const int n_groups = (int)((c + rows_per_cta - 1) / rows_per_cta);
     std::vector<std::pair<int64_t, uint32_t>> work;
@@ -186,12 +222,12 @@ int rows_per_cta(int32_t dtype) { return dtype == CP_BF16 ? attn_tc_rows_per_cta
 // query tiles that see the key tile over all steps, heaviest first.
 std::map<std::tuple<int, int, int, int64_t>, std::vector<uint32_t>> g_bwd_order_cache;
 
-const std::vector<uint32_t> &bwd_order(int layout, int N, int64_t S, int causal)
+const std::vector<uint32_t> &bwd_order_locked(int layout, int N, int64_t S, int causal)
 {
-    std::lock_guard<std::mutex> lk(g_order_mu);
     const auto key = std::make_tuple(layout, N, causal, S);
     auto it = g_bwd_order_cache.find(key);
     if (it != g_bwd_order_cache.end()) return it->second;
+    if (g_bwd_order_cache.size() >= kOrderCacheMax) g_bwd_order_cache.clear();
     const int64_t c = S / N;
     const int n_kt = (int)((c + kBwdKeyTile - 1) / kBwdKeyTile);
     const int n_qt = (int)((c + kBwdQueryTile - 1) / kBwdQueryTile);
@@ -218,6 +254,31 @@ const std::vector<uint32_t> &bwd_order(int layout, int N, int64_t S, int causal)
     std::vector<uint32_t> out;
     for (auto &w : work) out.push_back(w.second);
     return g_bwd_order_cache.emplace(key, std::move(out)).first->second;
+}
+
+// Copies the work order into p.order (natural order, order_len = 0, when it does
+// not fit the table), holding the cache lock throughout.
+void set_ring_order(AttnParams &p, int layout, int N, int64_t S, int causal, int rows_per_cta)
+{
+    std::lock_guard<std::mutex> lk(g_order_mu);
+    const std::vector<uint32_t> &ord = ring_order_locked(layout, N, S, causal, rows_per_cta);
+    p.order_len = 0;
+    if ((int64_t)ord.size() <= kMaxOrder) {
+        p.order_len = (int)ord.size();
+        std::copy(ord.begin(), ord.end(), p.order);
+    }
+}
+
+template <typename P>
+void set_bwd_order(P &p, int layout, int N, int64_t S, int causal)
+{
+    std::lock_guard<std::mutex> lk(g_order_mu);
+    const std::vector<uint32_t> &ord = bwd_order_locked(layout, N, S, causal);
+    p.order_len = 0;
+    if ((int64_t)ord.size() <= kMaxOrder) {
+        p.order_len = (int)ord.size();
+        std::copy(ord.begin(), ord.end(), p.order);
+    }
 }
 
 // Workspace regions of the backward: statistics [b][Hq][N][lpad] float2, then the
@@ -294,6 +355,7 @@ const char *cp_status_string(cp_status s)
     case CP_ERR_SHAPE: return "shape mismatch";
     case CP_ERR_CUDA: return "CUDA error";
     case CP_ERR_TIMEOUT: return "device wait timed out";
+    case CP_ERR_BOUNDS: return "bounds check failed (debug build)";
     }
     return "unknown status";
 }
@@ -353,8 +415,7 @@ cp_status cp_block_attn_fwd(const cp_tensor *q, const cp_tensor *k, const cp_ten
         return s;
     if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
     if (mask_mode != CP_MASK_NONE && mask_mode != CP_MASK_CAUSAL) return fail(CP_ERR_INVALID_ARG, "unknown mask mode");
-    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
-        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if ((s = resolve_scale(&softmax_scale, q->shape[3])) != CP_OK) return s;
     if (accumulate != 0 && accumulate != 1) return fail(CP_ERR_INVALID_ARG, "accumulate must be 0 or 1");
     const int64_t sq = q->shape[1], sk = k->shape[1];
     if (sq > INT32_MAX / 2 || sk > INT32_MAX / 2) return fail(CP_ERR_SHAPE, "sequence too long");
@@ -434,14 +495,16 @@ cp_status cp_lse_merge(cp_tensor *o_acc, cp_tensor *lse_acc, const cp_tensor *o_
 size_t cp_ring_workspace_bytes(int32_t layout, int32_t N, int32_t mode, int32_t dtype, int64_t b, int64_t S,
                                int64_t Hq, int64_t d)
 {
-    if (mode != CP_RING_STEPWISE) return 0;
+    if (mode != CP_RING_STEPWISE && mode != CP_RING_STEPWISE_EPI) return 0;
     if (layout < 0 || layout > 2 || N < 1 || b < 0 || S < 0 || Hq < 0 || d < 0) return 0;
     if (N == 1) return 0;
     const int64_t es = elem_size(dtype);
     if (!es) return 0;
     const int64_t rows = b * S * Hq;
-    // o_acc fp32, o_b in the input dtype, lse_b fp32; each region 256-byte aligned
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    // STEPWISE_EPI: the fp32 running o (an fp32 output is its own accumulator)
+    if (mode == CP_RING_STEPWISE_EPI) return dtype == CP_FP32 ? 0 : (size_t)up(rows * d * 4);
+    // STEPWISE: o_acc fp32, o_b in the input dtype, lse_b fp32; each region 256-byte aligned
     return (size_t)(up(rows * d * 4) + up(rows * d * es) + up(rows * 4));
 }
 
@@ -452,14 +515,14 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     g_last_error[0] = 0;
     cp_status s;
     if (layout < 0 || layout > 2) return fail(CP_ERR_INVALID_ARG, "unknown layout %d", layout);
-    if (mode != CP_RING_FUSED && mode != CP_RING_STEPWISE) return fail(CP_ERR_INVALID_ARG, "unknown ring mode");
+    if (mode != CP_RING_FUSED && mode != CP_RING_STEPWISE && mode != CP_RING_STEPWISE_EPI)
+        return fail(CP_ERR_INVALID_ARG, "unknown ring mode");
     if (causal != 0 && causal != 1) return fail(CP_ERR_INVALID_ARG, "causal must be 0 or 1");
     if ((s = check_tensor(q, "q")) != CP_OK || (s = check_tensor(k, "k")) != CP_OK ||
         (s = check_tensor(v, "v")) != CP_OK)
         return s;
     if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
-    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
-        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if ((s = resolve_scale(&softmax_scale, q->shape[3])) != CP_OK) return s;
     const int64_t S = q->shape[1];
     if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
     if (N < 1 || N > 4096) return fail(CP_ERR_INVALID_ARG, "N must be in [1, 4096]");
@@ -474,6 +537,7 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     const int n_qt = (int)((c + rows - 1) / rows);
     if (n_qt > 65535) return fail(CP_ERR_SHAPE, "too many query tiles per rank");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    NvtxRange call_range(mode == CP_RING_FUSED ? "cp_ring_attn_fwd fused" : "cp_ring_attn_fwd stepwise");
 
     thread_local AttnParams p;
     std::memset(&p, 0, sizeof p);
@@ -494,11 +558,7 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     p.scale = softmax_scale;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.n_qt = n_qt;
-    const std::vector<uint32_t> &ord = ring_order(layout, N, S, causal, rows);
-    if ((int64_t)ord.size() <= kMaxOrder) {
-        p.order_len = (int)ord.size();
-        std::copy(ord.begin(), ord.end(), p.order);
-    }
+    set_ring_order(p, layout, N, S, causal, rows);
     fill_inputs(p, q, k, v);
     set_status_ptr(p);
 
@@ -509,19 +569,42 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
         return launch_attn(p, q->dtype, st);
     }
 
-    // STEPWISE: the ring as N block launches plus N-1 standalone merges
     const size_t need = cp_ring_workspace_bytes(layout, N, mode, q->dtype, q->shape[0], S, q->shape[2], q->shape[3]);
-    if (!workspace || workspace_bytes < need)
+    if (need && (!workspace || workspace_bytes < need))
         return fail(CP_ERR_INVALID_ARG, "workspace of %zu bytes needed", need);
     if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     const int64_t b = q->shape[0], Hq = q->shape[2], d = q->shape[3], nrows = b * S * Hq;
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
     char *ws = static_cast<char *>(workspace);
     cp_tensor o_acc{ws, CP_FP32, 0, {b, S, Hq, d}, {S * Hq * d, Hq * d, d, 1}};
+
+    if (mode == CP_RING_STEPWISE_EPI) {
+        // N launches, one ring step each; step 0 stores the running (o, lse) in fp32,
+        // every later step LSE-merges its partial into them in the block epilogue,
+        // and the last one writes the merged o in the output dtype.  An fp32 output
+        // is the running o itself.
+        const cp_tensor *acc = q->dtype == CP_FP32 ? o : &o_acc;
+        for (int r = 0; r < N; ++r) {
+            NvtxRange step_range("cp ring step %d of %d", r, N);
+            p.step_begin = r;
+            p.step_end = r + 1;
+            fill_outputs(p, r == 0 ? EPI_STORE : EPI_MERGE, acc, lse);
+            if (r == N - 1 && acc != o) {
+                p.o_out = o->data;
+                p.o_out_dtype = o->dtype;
+                p.oo_sb = o->stride[0]; p.oo_ss = o->stride[1]; p.oo_sh = o->stride[2];
+            }
+            if ((s = launch_attn(p, q->dtype, st)) != CP_OK) return s;
+        }
+        return CP_OK;
+    }
+
+    // STEPWISE: the ring as N block launches plus N-1 standalone merges
     cp_tensor o_b{ws + up(nrows * d * 4), q->dtype, 0, {b, S, Hq, d}, {S * Hq * d, Hq * d, d, 1}};
     cp_tensor lse_b{ws + up(nrows * d * 4) + up(nrows * d * elem_size(q->dtype)), CP_FP32, 0, {b, Hq, S, 1},
                     {Hq * S, S, 1, 1}};
     for (int r = 0; r < N; ++r) {
+        NvtxRange step_range("cp ring step %d of %d", r, N);
         p.step_begin = r;
         p.step_end = r + 1;
         if (r == 0) fill_outputs(p, EPI_STORE, &o_acc, lse);  // first partial initialises the running result
@@ -589,8 +672,7 @@ static cp_status uly_ring_fwd(int32_t layout, int32_t N, int32_t P, int32_t caus
         (s = check_tensor(v, "v")) != CP_OK)
         return s;
     if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
-    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
-        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if ((s = resolve_scale(&softmax_scale, q->shape[3])) != CP_OK) return s;
     const int64_t b = q->shape[0], S = q->shape[1], Hq = q->shape[2], Hkv = k->shape[2], d = q->shape[3];
     if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
     if (P < 1) return fail(CP_ERR_INVALID_ARG, "P must be >= 1");
@@ -671,8 +753,9 @@ size_t cp_allgather_bwd_workspace_bytes(int32_t N, int32_t dtype, int64_t b, int
     if (N < 1 || b < 0 || S < 0 || Hq < 0 || Hkv < 0 || d < 0 || n_docs < 1 || !elem_size(dtype) || S % N) return 0;
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
     const int64_t kb = up(b * S * Hkv * d * elem_size(dtype));
-    // gathered K, V, dK, dV; the document table; the statistics and the dQ accumulator
-    return (size_t)(4 * kb + up((int64_t)n_docs * 4)) +
+    // gathered K, V, dK, dV; the document starts and the per-position document
+    // bounds; the statistics and the dQ accumulator
+    return (size_t)(4 * kb + up((int64_t)n_docs * 4) + 2 * up(S * 4)) +
            cp_ring_bwd_workspace_bytes(CP_LAYOUT_CONTIGUOUS, N, dtype, b, S, Hq, d);
 }
 
@@ -694,8 +777,7 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     // bf16 with d = 128 on the tensor cores, fp32 and bf16 d = 64 on the FFMA kernels
     const int32_t dt = q->dtype;
     const bool tc_path = dt == CP_BF16 && q->shape[3] == 128;
-    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
-        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if ((s = resolve_scale(&softmax_scale, q->shape[3])) != CP_OK) return s;
     const int64_t S = q->shape[1];
     if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
     if (N < 1 || N > 4096) return fail(CP_ERR_INVALID_ARG, "N must be in [1, 4096]");
@@ -734,6 +816,7 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     if (b == 0 || S == 0) return CP_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    NvtxRange call_range("cp_allgather_attn_bwd");
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
     char *ws = static_cast<char *>(workspace);
     const int64_t kb = up(b * S * Hkv * d * elem_size(dt));
@@ -742,7 +825,9 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     };
     cp_tensor kg = kv_t(0), vg = kv_t(1), dkg = kv_t(2), dvg = kv_t(3);
     int *docs_dev = reinterpret_cast<int *>(ws + 4 * kb);
-    char *ws_q = ws + 4 * kb + up((int64_t)n_docs * 4);
+    int *doc_pos_start = reinterpret_cast<int *>(ws + 4 * kb + up((int64_t)n_docs * 4));
+    int *doc_pos_end = reinterpret_cast<int *>(ws + 4 * kb + up((int64_t)n_docs * 4) + up(S * 4));
+    char *ws_q = ws + 4 * kb + up((int64_t)n_docs * 4) + 2 * up(S * 4);
     // the gather of K and V into original order (as in the forward)
     if ((s = cp_layout_permute(layout, N, 1, &kg, const_cast<cp_tensor *>(k), 1, stream)) != CP_OK) return s;
     if ((s = cp_layout_permute(layout, N, 1, &vg, const_cast<cp_tensor *>(v), 1, stream)) != CP_OK) return s;
@@ -750,6 +835,10 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     for (int32_t i = 0; i < n_docs; ++i) docs_h[i] = (int32_t)doc_starts[i];
     cudaError_t e = cudaMemcpyAsync(docs_dev, docs_h.data(), sizeof(int32_t) * (size_t)n_docs, cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(e, "document table copy");
+    if (n_docs > 1 && tc_path) {
+        e = launch_doc_tables(docs_dev, n_docs, S, doc_pos_start, doc_pos_end, st);
+        if (e != cudaSuccess) return cuda_fail(e, "document bounds launch");
+    }
 
     thread_local BwdParams p;
     std::memset(&p, 0, sizeof p);
@@ -792,6 +881,7 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     p.dv_sb = dvg.stride[0]; p.dv_ss = dvg.stride[1]; p.dv_sh = dvg.stride[2];
     p.doc_starts = n_docs > 1 ? docs_dev : nullptr;
     p.n_docs = n_docs > 1 ? n_docs : 0;
+    p.doc_pos_end = doc_pos_end;
     int *word = nullptr;
     status_word(&word);
     p.status = word;
@@ -891,8 +981,7 @@ static cp_status uly_ring_bwd(int32_t layout, int32_t N, int32_t P, int32_t caus
         (s = check_tensor(dv, "dv")) != CP_OK)
         return s;
     if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
-    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
-        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if ((s = resolve_scale(&softmax_scale, q->shape[3])) != CP_OK) return s;
     const int64_t b = q->shape[0], S = q->shape[1], Hq = q->shape[2], Hkv = k->shape[2], d = q->shape[3];
     if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
     if (P < 1) return fail(CP_ERR_INVALID_ARG, "P must be >= 1");
@@ -977,8 +1066,9 @@ size_t cp_allgather_workspace_bytes(int32_t N, int32_t dtype, int64_t b, int64_t
 {
     if (N < 1 || b < 0 || S < 0 || Hkv < 0 || d < 0 || n_docs < 1 || !elem_size(dtype)) return 0;
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
-    // gathered K and V in original token order, then the document starts (int32)
-    return (size_t)(2 * up(b * S * Hkv * d * elem_size(dtype)) + up((int64_t)n_docs * 4));
+    // gathered K and V in original token order, then the document starts (int32) and
+    // the per-position document bounds (two int32 tables of S entries)
+    return (size_t)(2 * up(b * S * Hkv * d * elem_size(dtype)) + up((int64_t)n_docs * 4) + 2 * up(S * 4));
 }
 
 cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q, const cp_tensor *k,
@@ -993,8 +1083,7 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
         (s = check_tensor(v, "v")) != CP_OK)
         return s;
     if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
-    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
-        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if ((s = resolve_scale(&softmax_scale, q->shape[3])) != CP_OK) return s;
     const int64_t S = q->shape[1];
     if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
     if (N < 1 || N > 4096) return fail(CP_ERR_INVALID_ARG, "N must be in [1, 4096]");
@@ -1027,6 +1116,7 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
     const int n_qt = (int)((c + rows - 1) / rows);
     if (n_qt > 65535) return fail(CP_ERR_SHAPE, "too many query tiles per rank");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    NvtxRange call_range("cp_allgather_attn_fwd");
 
     // the all-gather: every rank's K/V block back into one original-order copy
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
@@ -1048,6 +1138,12 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
     // pageable source: the copy is staged before the call returns
     cudaError_t e = cudaMemcpyAsync(docs_dev, docs_h, sizeof(int32_t) * (size_t)n_docs, cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(e, "document table copy");
+    int *doc_pos_start = reinterpret_cast<int *>(ws + 2 * kv_bytes + up((int64_t)n_docs * 4));
+    int *doc_pos_end = doc_pos_start + up(S * 4) / 4;
+    if (n_docs > 1 && q->dtype == CP_BF16) {
+        e = launch_doc_tables(docs_dev, n_docs, S, doc_pos_start, doc_pos_end, st);
+        if (e != cudaSuccess) return cuda_fail(e, "document bounds launch");
+    }
 
     thread_local AttnParams p;
     std::memset(&p, 0, sizeof p);
@@ -1074,6 +1170,7 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
     p.n_qt = n_qt;
     p.doc_starts = n_docs > 1 ? docs_dev : nullptr;
     p.n_docs = n_docs > 1 ? n_docs : 0;
+    p.doc_pos_start = doc_pos_start;
     // work order, heaviest (rank, row group) first: the key tiles each 128-row query
     // tile of the group walks, from the document start of its first row to its last
     // row (the document mask's bounds on the gathered block)
@@ -1116,7 +1213,9 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
 size_t cp_block_bwd_workspace_bytes(int64_t b, int64_t sq, int64_t Hq)
 {
     if (b < 0 || sq < 0 || Hq < 0) return 0;
-    return (size_t)((b * Hq * sq * 8 + 255) / 256 * 256);  // (lse, D) per query row
+    // (lse, D) per query row, rows padded to the tensor-core kernel's query tile
+    const int64_t lpad = (sq + kBwdQueryTile - 1) / kBwdQueryTile * kBwdQueryTile;
+    return (size_t)((b * Hq * lpad * 8 + 255) / 256 * 256);
 }
 
 cp_status cp_block_attn_bwd(const cp_tensor *q, const cp_tensor *k, const cp_tensor *v, const cp_tensor *o,
@@ -1134,8 +1233,7 @@ cp_status cp_block_attn_bwd(const cp_tensor *q, const cp_tensor *k, const cp_ten
         return s;
     if ((s = check_attn_dtypes(q, k, v)) != CP_OK) return s;
     if (mask_mode != CP_MASK_NONE && mask_mode != CP_MASK_CAUSAL) return fail(CP_ERR_INVALID_ARG, "unknown mask mode");
-    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
-        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if ((s = resolve_scale(&softmax_scale, q->shape[3])) != CP_OK) return s;
     const int64_t b = q->shape[0], sq = q->shape[1], sk = k->shape[1], Hq = q->shape[2];
     if (sq > INT32_MAX / 2 || sk > INT32_MAX / 2) return fail(CP_ERR_SHAPE, "sequence too long");
     if ((s = check_out(o, lse, q, sq, false)) != CP_OK) return s;
@@ -1187,7 +1285,28 @@ cp_status cp_block_attn_bwd(const cp_tensor *q, const cp_tensor *k, const cp_ten
     p.dk_sb = dk_acc->stride[0]; p.dk_ss = dk_acc->stride[1]; p.dk_sh = dk_acc->stride[2];
     p.dv_sb = dv_acc->stride[0]; p.dv_ss = dv_acc->stride[1]; p.dv_sh = dv_acc->stride[2];
     p.accumulate = 1;
-    cudaError_t e = launch_attn_bwd_simt(p, q->dtype == CP_FP32, static_cast<cudaStream_t>(stream));
+    cudaError_t e;
+    if (q->dtype == CP_BF16 && q->shape[3] == 128) {
+        // tensor cores: one launch over the key tiles, dQ reduced into dq_acc
+        if ((s = check_rows16(dq_acc, "dq_acc")) != CP_OK || (s = check_rows16(dk_acc, "dk_acc")) != CP_OK ||
+            (s = check_rows16(dv_acc, "dv_acc")) != CP_OK)
+            return s;
+        if ((s = check_rows16(o, "o")) != CP_OK || (s = check_rows16(dout, "dout")) != CP_OK) return s;
+        const int64_t n_kt = (sk + kBwdKeyTile - 1) / kBwdKeyTile;
+        if (n_kt > 65535) return fail(CP_ERR_SHAPE, "too many key tiles");
+        p.lpad = (int)((sq + kBwdQueryTile - 1) / kBwdQueryTile * kBwdQueryTile);
+        p.q_row_step = sq;
+        p.kv_row_step = 0;
+        p.dq_acc = static_cast<float *>(dq_acc->data);
+        p.n_kt = (int)n_kt;
+        p.order_len = 0;
+        int *word = nullptr;
+        if ((e = status_word(&word)) != cudaSuccess) return cuda_fail(e, "status word");
+        p.status = word;
+        e = launch_attn_bwd(p, static_cast<cudaStream_t>(stream));
+    } else {
+        e = launch_attn_bwd_simt(p, q->dtype == CP_FP32, static_cast<cudaStream_t>(stream));
+    }
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return CP_OK;
 }
@@ -1220,14 +1339,14 @@ cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     // d = 64 on the FFMA backward
     const cp_dtype dt = static_cast<cp_dtype>(q->dtype);
     const bool tc_path = dt == CP_BF16 && q->shape[3] == 128;
-    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
-        return fail(CP_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if ((s = resolve_scale(&softmax_scale, q->shape[3])) != CP_OK) return s;
     const int64_t S = q->shape[1];
     if (k->shape[1] != S) return fail(CP_ERR_SHAPE, "q and k/v sequence lengths differ");
     if (N < 1 || N > 4096) return fail(CP_ERR_INVALID_ARG, "N must be in [1, 4096]");
     if (S >= ((int64_t)1 << 30)) return fail(CP_ERR_SHAPE, "sequence too long (S must be below 2^30)");
     if (S % N) return fail(CP_ERR_SHAPE, "S = %lld is not a multiple of N = %d", (long long)S, N);
     if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N)) return fail(CP_ERR_SHAPE, "zig-zag needs S to be a multiple of 2N");
+    NvtxRange call_range("cp_ring_attn_bwd");
     if ((s = check_out(o, lse, q, S, false)) != CP_OK) return s;
     if (o->dtype != dt) return fail(CP_ERR_INVALID_ARG, "o must have q's dtype");
     const cp_tensor *like_q[2] = {dout, dq};
@@ -1295,11 +1414,7 @@ cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_t
         if (e != cudaSuccess) return cuda_fail(e, "backward launch");
         return CP_OK;
     }
-    const std::vector<uint32_t> &ord = bwd_order(layout, N, S, causal);
-    if ((int64_t)ord.size() <= kMaxOrder) {
-        p.order_len = (int)ord.size();
-        std::copy(ord.begin(), ord.end(), p.order);
-    }
+    set_bwd_order(p, layout, N, S, causal);
     // head-major grid once one head's work items fill a wave of the device
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1375,6 +1490,9 @@ cp_status cp_stream_check(void *stream)
     if (h[0]) {
         const int zero[2] = {0, 0};
         cudaMemcpy(word, zero, sizeof zero, cudaMemcpyHostToDevice);
+        if (h[0] & 2)
+            return fail(CP_ERR_BOUNDS, "a bounds check of the debug build failed (status %d, first at check %d)", h[0],
+                        h[1]);
         return fail(CP_ERR_TIMEOUT, "a device wait expired (status %d, first at wait tag %d)", h[0], h[1]);
     }
     return CP_OK;

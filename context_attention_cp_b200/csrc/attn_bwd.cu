@@ -143,14 +143,10 @@ __device__ __forceinline__ bool bar_any(uint32_t id, uint32_t nthreads, bool pre
 // with the tile seeing at least one key of the CTA's key tile.  Every role walks it.
 // End of the document that holds position pos: the first document start > pos
 // (INT32_MAX past the last document).
-__device__ __forceinline__ int64_t doc_end_of(const int *starts, int n, int64_t pos)
+__device__ __forceinline__ int64_t doc_end_of(const BwdParams &p, int64_t pos)
 {
-    int lo = 0, hi = n;
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if ((int64_t)__ldg(starts + mid) <= pos) lo = mid + 1; else hi = mid;
-    }
-    return lo < n ? (int64_t)__ldg(starts + lo) : (int64_t)INT32_MAX;
+    if (!bounds_ok(pos >= 0 && pos < p.seq_len, p.status, 206)) return INT32_MAX;
+    return (int64_t)__ldg(p.doc_pos_end + pos);
 }
 
 // First query tile (of BQ rows, q_len rows, ranges q) whose row at offset off
@@ -200,8 +196,8 @@ struct QSeq {
         de_first = de_last = INT32_MAX;
         if (pp.n_docs > 0 && pp.kv_len > 0) {
             const int64_t k_hi = k_lo + BK - 1 < pp.kv_len - 1 ? k_lo + BK - 1 : pp.kv_len - 1;
-            de_first = doc_end_of(pp.doc_starts, pp.n_docs, range_pos(k, (int64_t)k_lo));
-            de_last = doc_end_of(pp.doc_starts, pp.n_docs, range_pos(k, k_hi));
+            de_first = doc_end_of(pp, range_pos(k, (int64_t)k_lo));
+            de_last = doc_end_of(pp, range_pos(k, k_hi));
         }
         i = 0;
         h = hq0;
@@ -308,6 +304,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int hk = bh % p.hkv;
     const int bb = bh / p.hkv;
     const int k_lo = kt * BK;
+    // tensor rows the maps and outputs cover (for the debug build's bounds checks)
+    const int64_t q_rows_all = (int64_t)p.n_ranks * p.q_row_step;
+    const int64_t kv_rows_all = p.kv_row_step ? (int64_t)p.n_ranks * p.kv_row_step : p.kv_len;
+    (void)q_rows_all;
+    (void)kv_rows_all;
     const Range kr = (p.use_layout && !p.kv_explicit) ? layout_range(p.layout, p.n_ranks, p.seq_len, j) : p.kv_range;
 
     if (tid == 0) {
@@ -348,7 +349,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             WaitCtx w{abort_flag, p.status, 41};
             const int kv_row = (int)(j * p.kv_row_step) + k_lo;
             mbar_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
-            for (int kb = 0; kb < 2; ++kb) {
+            const bool kv_ok = bounds_ok(kv_row >= 0 && kv_row < kv_rows_all && hk < p.hkv && bb < p.b, p.status, 201);
+            for (int kb = 0; kb < 2 && kv_ok; ++kb) {
                 tma_load_4d(s_base + C::OFF_K + kb * C::KV_SUB, &tm_k, bar(C::B_KV), kb * 64, hk, kv_row, bb);
                 tma_load_4d(s_base + C::OFF_V + kb * C::KV_SUB, &tm_v, bar(C::B_KV), kb * 64, hk, kv_row, bb);
             }
@@ -359,13 +361,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 mbar_expect_tx(bar(C::B_QF + s), C::STAGE + BQ * 8);
                 const int q_row = seq.q_row();
                 const uint32_t st = s_base + C::OFF_Q + s * C::STAGE;
-                for (int kb = 0; kb < 2; ++kb) {
+                const bool q_ok = bounds_ok(q_row >= 0 && q_row < q_rows_all && seq.h < p.hq && bb < p.b, p.status, 202);
+                for (int kb = 0; kb < 2 && q_ok; ++kb) {
                     tma_load_4d(st + kb * C::Q_SUB, &tm_q, bar(C::B_QF + s), kb * 64, seq.h, q_row, bb);
                     tma_load_4d(st + C::Q_TILE + kb * C::Q_SUB, &tm_do, bar(C::B_QF + s), kb * 64, seq.h, q_row, bb);
                 }
                 const float2 *src =
                     p.stats + (((int64_t)bb * p.hq + seq.h) * p.n_ranks + seq.i) * p.lpad + (int64_t)seq.qt * BQ;
-                bulk_g2s(s_base + C::OFF_ST + s * BQ * 8, src, BQ * 8, bar(C::B_QF + s));
+                if (bounds_ok(seq.i < p.n_ranks && (int64_t)seq.qt * BQ + BQ <= p.lpad, p.status, 203))
+                    bulk_g2s(s_base + C::OFF_ST + s * BQ * 8, src, BQ * 8, bar(C::B_QF + s));
                 ++n;
             }
             if (*abort_flag) {
@@ -490,7 +494,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             fence_async_smem();
             asm volatile("barrier.sync 2, 128;" ::: "memory");
             if (leader) {
-                tma_reduce_add_4d(&tm_dq, s_base + C::OFF_DQ, 0, seq.h, seq.q_row(), bb);
+                if (bounds_ok(seq.q_row() >= 0 && seq.q_row() < q_rows_all && seq.h < p.hq, p.status, 204))
+                    tma_reduce_add_4d(&tm_dq, s_base + C::OFF_DQ, 0, seq.h, seq.q_row(), bb);
                 bulk_commit();
             }
             ++n;
@@ -506,7 +511,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int key = k_lo + krow;
         const bool key_ok = key < p.kv_len;
         const int64_t pk = range_pos(kr, (int64_t)(key_ok ? key : (p.kv_len > 0 ? p.kv_len - 1 : 0)));
-        const int64_t de_key = p.n_docs > 0 ? doc_end_of(p.doc_starts, p.n_docs, pk) : (int64_t)INT32_MAX;
+        const int64_t de_key = p.n_docs > 0 ? doc_end_of(p, pk) : (int64_t)INT32_MAX;
         const float sl2 = p.scale_log2;
         bool aborted = false;
         int n = 0;
@@ -634,15 +639,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int64_t sb = half == 0 ? p.dk_sb : p.dv_sb, ss = half == 0 ? p.dk_ss : p.dv_ss,
                           sh = half == 0 ? p.dk_sh : p.dv_sh;
             const int64_t orow = (int64_t)j * p.kv_row_step + key;
-            uint16_t *dst = reinterpret_cast<uint16_t *>(out) + (int64_t)bb * sb + orow * ss + (int64_t)hk * sh;
+            const bool key_in = key_ok && bounds_ok(orow >= 0 && orow < kv_rows_all, p.status, 205);
+            if (p.accumulate) {
+                // block form: add this call's share into the caller's fp32 accumulator
+                // (each key row belongs to this CTA alone)
+                float *dst = reinterpret_cast<float *>(out) + (int64_t)bb * sb + orow * ss + (int64_t)hk * sh;
 #pragma unroll
-            for (int c0 = 0; c0 < HD; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(tbase + lane_off + t_acc + (uint32_t)c0, r);
-                float v[32];
+                for (int c0 = 0; c0 < HD; c0 += 32) {
+                    uint32_t r[32];
+                    if (n > 0) tmem_ld32(tbase + lane_off + t_acc + (uint32_t)c0, r);
+                    if (key_in && n > 0) {
+                        float4 *d4 = reinterpret_cast<float4 *>(dst + c0);
 #pragma unroll
-                for (int c = 0; c < 32; ++c) v[c] = n > 0 ? __uint_as_float(r[c]) * f : 0.f;
-                if (key_ok) store_bf16x32(dst + c0, v);
+                        for (int i = 0; i < 8; ++i) {
+                            float4 a = d4[i];
+                            a.x = fmaf(__uint_as_float(r[4 * i + 0]), f, a.x);
+                            a.y = fmaf(__uint_as_float(r[4 * i + 1]), f, a.y);
+                            a.z = fmaf(__uint_as_float(r[4 * i + 2]), f, a.z);
+                            a.w = fmaf(__uint_as_float(r[4 * i + 3]), f, a.w);
+                            d4[i] = a;
+                        }
+                    }
+                }
+            } else {
+                uint16_t *dst = reinterpret_cast<uint16_t *>(out) + (int64_t)bb * sb + orow * ss + (int64_t)hk * sh;
+#pragma unroll
+                for (int c0 = 0; c0 < HD; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + lane_off + t_acc + (uint32_t)c0, r);
+                    float v[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) v[c] = n > 0 ? __uint_as_float(r[c]) * f : 0.f;
+                    if (key_in) store_bf16x32(dst + c0, v);
+                }
             }
         }
     }
@@ -691,8 +720,10 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __grid_constant
         const float lse = p.lse[bb * p.lse_sb + h * p.lse_sh + row * p.lse_ss];
         st.x = (lse == -INFINITY) ? INFINITY : lse * kLog2eB;
         st.y = acc;
-        float4 *dq = reinterpret_cast<float4 *>(p.dq_acc + (((int64_t)bb * acc_rows + row) * p.hq + h) * HD) + lane;
-        *dq = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (!p.accumulate) {  // the block form adds into the caller's accumulator instead
+            float4 *dq = reinterpret_cast<float4 *>(p.dq_acc + (((int64_t)bb * acc_rows + row) * p.hq + h) * HD) + lane;
+            *dq = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     }
     if (lane == 0) p.stats[gw] = st;
 }
@@ -773,14 +804,15 @@ cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream)
         !make_map_b(&tdo, BF, 2, p.dout, p.b, q_rows, p.hq, HD, p.do_sb, p.do_ss, p.do_sh, 64, BQ, SW) ||
         !make_map_b(&tk, BF, 2, p.k, p.b, kv_rows, p.hkv, HD, p.k_sb, p.k_ss, p.k_sh, 64, BK, SW) ||
         !make_map_b(&tv, BF, 2, p.v, p.b, kv_rows, p.hkv, HD, p.v_sb, p.v_ss, p.v_sh, 64, BK, SW) ||
-        !make_map_b(&tdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.dq_acc, p.b, q_rows, p.hq, HD, q_rows * p.hq * HD,
-                    (int64_t)p.hq * HD, HD, HD, BQ, CU_TENSOR_MAP_SWIZZLE_NONE))
+        !(p.accumulate ? make_map_b(&tdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.dq_acc, p.b, q_rows, p.hq, HD, p.dq_sb,
+                                    p.dq_ss, p.dq_sh, HD, BQ, CU_TENSOR_MAP_SWIZZLE_NONE)
+                       : make_map_b(&tdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.dq_acc, p.b, q_rows, p.hq, HD,
+                                    q_rows * p.hq * HD, (int64_t)p.hq * HD, HD, HD, BQ, CU_TENSOR_MAP_SWIZZLE_NONE)))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BCfg::SMEM);
+    static unsigned long long attr_done = 0;
+    {
+        cudaError_t e = set_smem_per_device((const void *)attn_bwd_kernel, BCfg::SMEM, &attr_done);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     const int64_t warps = (int64_t)p.b * p.hq * p.n_ranks * p.lpad;
     if (warps == 0) return cudaSuccess;
@@ -792,6 +824,7 @@ cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream)
         attn_bwd_kernel<<<(unsigned)items, NTHREADS, BCfg::SMEM, stream>>>(p, tq, tk, tv, tdo, tdq);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    if (p.accumulate) return cudaSuccess;  // dq_acc is the caller's output
     const int64_t threads = (int64_t)p.b * p.n_ranks * p.q_len * p.hq * (HD / 8);
     attn_bwd_post_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(p, q_rows);
     return cudaGetLastError();

@@ -185,12 +185,10 @@ __global__ void __launch_bounds__(RM) attn_simt_kernel(const __grid_constant__ A
 template <int D>
 cudaError_t launch_simt_d(const AttnParams &p, cudaStream_t stream)
 {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(attn_simt_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             SimtCfg<D>::SMEM);
+    static unsigned long long attr_done = 0;
+    {
+        cudaError_t e = set_smem_per_device((const void *)attn_simt_kernel<D>, SimtCfg<D>::SMEM, &attr_done);
         if (e != cudaSuccess) return e;
-        attr = true;
     }
     const int64_t items = (int64_t)p.n_ranks * p.n_qt * p.b * p.hq;
     if (items == 0) return cudaSuccess;

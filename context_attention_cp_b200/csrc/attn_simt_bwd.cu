@@ -303,24 +303,18 @@ __global__ void __launch_bounds__(SRM) simt_bwd_dkv_kernel(const __grid_constant
     }
 }
 
-template <typename K>
-cudaError_t set_smem(K kernel, int bytes)
-{
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-}
 
 template <typename T, int D>
 cudaError_t launch_simt_bwd_t(const BwdParams &p, cudaStream_t st)
 {
     using C = SbCfg<D>;
-    static bool attr = false;
+    static unsigned long long done_dq = 0, done_dv = 0, done_dk = 0;
     cudaError_t e;
-    if (!attr) {
-        if ((e = set_smem(simt_bwd_dq_kernel<T, D>, C::SMEM)) != cudaSuccess) return e;
-        if ((e = set_smem(simt_bwd_dkv_kernel<T, D, false>, C::SMEM)) != cudaSuccess) return e;
-        if ((e = set_smem(simt_bwd_dkv_kernel<T, D, true>, C::SMEM)) != cudaSuccess) return e;
-        attr = true;
-    }
+    if ((e = set_smem_per_device((const void *)simt_bwd_dq_kernel<T, D>, C::SMEM, &done_dq)) != cudaSuccess) return e;
+    if ((e = set_smem_per_device((const void *)simt_bwd_dkv_kernel<T, D, false>, C::SMEM, &done_dv)) != cudaSuccess)
+        return e;
+    if ((e = set_smem_per_device((const void *)simt_bwd_dkv_kernel<T, D, true>, C::SMEM, &done_dk)) != cudaSuccess)
+        return e;
     const int64_t rows = (int64_t)p.b * p.hq * p.n_ranks * p.q_len;
     if (rows == 0) return cudaSuccess;
     simt_bwd_stats_kernel<T, D><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(p);

@@ -24,7 +24,10 @@
 // the softmax overwrites columns [0, 64) of S_j with bf16 probabilities P_j, which
 // the PV MMA reads as its A operand; O_j = [256 + d j, 256 + d (j + 1)).
 // The MMA warp interleaves the two tiles (PV_0(n), S_0(n+1), PV_1(n), S_1(n+1), ...)
-// so the tensor core works on one tile while the other tile's softmax runs.
+// so the tensor core works on one tile while the other tile's softmax runs.  P is
+// handed over in two halves of 64 keys, each with its own barrier, so the first
+// half of PV runs while the softmax computes the second half of P; S_j(n+1) can
+// only follow PV_j(n), because it overwrites the columns that hold P_j(n).
 //
 // Softmax details: scores are handled in the log2 domain (scale * log2 e folded
 // into one FMA); the max used in the exponent is raised only when a row's max
@@ -33,6 +36,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
+
+#include <algorithm>
 
 #include "kernels.h"
 #include "ptx.cuh"
@@ -53,8 +58,12 @@ constexpr int NQ = 2;    // query tiles per CTA
 constexpr int NSK = CP_ATTN_NSK;  // K stages
 constexpr int NSV = CP_ATTN_NSV;  // V stages
 constexpr int NTHREADS = 384;
-constexpr int REGS_SOFTMAX = 208;
-constexpr int REGS_OTHER = 88;
+#ifndef CP_ATTN_REGS_SOFTMAX
+#define CP_ATTN_REGS_SOFTMAX 208
+#endif
+constexpr int REGS_SOFTMAX = CP_ATTN_REGS_SOFTMAX;
+constexpr int REGS_OTHER = (NTHREADS * 168 - 2 * 128 * REGS_SOFTMAX) / 128;  // the rest of the launch's registers
+static_assert(REGS_OTHER >= 24 && REGS_OTHER % 8 == 0, "register split");
 constexpr int WARP_LOAD = 8;
 constexpr int WARP_MMA = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -65,6 +74,35 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define CP_EXP2_EMU_MOD 0
 #endif
 constexpr int kEmuMod = CP_EXP2_EMU_MOD;
+// P handed to the MMA warp in two halves of 64 keys (1) or whole (0).
+#ifndef CP_ATTN_SPLIT_P
+#define CP_ATTN_SPLIT_P 0
+#endif
+constexpr bool kSplitP = CP_ATTN_SPLIT_P != 0;
+// The two softmax warpgroups take turns for their exponential phases (1) or run
+// freely (0).  Turns are handed over on named barriers kTurn0 / kTurn1 (the
+// teardown uses barrier 1).
+#ifndef CP_ATTN_PINGPONG
+#define CP_ATTN_PINGPONG 0
+#endif
+constexpr bool kPingPong = CP_ATTN_PINGPONG != 0;
+constexpr int kTurn0 = 2, kTurn1 = 3;
+// Persistent grids (one CTA per SM walking the work items) for the document-mask
+// instantiation and for the ring's.
+#ifndef CP_ATTN_DOC_PERSIST
+#define CP_ATTN_DOC_PERSIST 1
+#endif
+#ifndef CP_ATTN_RING_PERSIST
+#define CP_ATTN_RING_PERSIST 0
+#endif
+constexpr bool kDocPersist = CP_ATTN_DOC_PERSIST != 0;
+constexpr bool kRingPersist = CP_ATTN_RING_PERSIST != 0;
+// A turn starts before the S load (0) or after the row max (1: the loads and row
+// maxima of the two tiles overlap, at the cost of more live registers).
+#ifndef CP_ATTN_TURN_LATE
+#define CP_ATTN_TURN_LATE 0
+#endif
+constexpr bool kTurnLate = CP_ATTN_TURN_LATE != 0;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
@@ -83,9 +121,12 @@ struct Cfg {
         B_VF = B_KE + NSK,
         B_VE = B_VF + NSV,
         B_SF = B_VE + NSV,  // per query tile
-        B_PF = B_SF + NQ,
-        B_PV = B_PF + NQ,
-        B_DONE = B_PV + NQ,
+        B_PF = B_SF + NQ,   // P of keys [0, 64) of the tile stored (per query tile)
+        B_PH = B_PF + NQ,   // P of keys [64, 128) stored
+        B_PV = B_PH + NQ,
+        B_OF = B_PV + NQ,   // O of query tile j read out by its epilogue (per query tile)
+        B_QE = B_OF + NQ,   // Q buffer free: the work item's last S products are done
+        B_DONE = B_QE + 1,
         NBAR = B_DONE + 1
     };
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -97,26 +138,22 @@ struct Cfg {
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
 };
 
-// Document start of position pos: the last entry of the sorted starts <= pos.
-__device__ __forceinline__ int64_t doc_start_of(const int *starts, int n, int64_t pos)
+// Document start of position pos (one load from the per-position table).
+__device__ __forceinline__ int doc_start_of(const AttnParams &p, int pos)
 {
-    int lo = 0, hi = n;  // first start > pos
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if ((int64_t)__ldg(starts + mid) <= pos) lo = mid + 1; else hi = mid;
-    }
-    return lo > 0 ? (int64_t)__ldg(starts + lo - 1) : 0;
+    if (!bounds_ok(pos >= 0 && pos < p.seq_len, p.status, 104)) return 0;
+    return __ldg(p.doc_pos_start + pos);
 }
 
 // First key tile t of a block (kv_len keys, ranges k, tiles of BN) whose key at
 // index min(t * BN + off, kv_len - 1) has a position >= x.
-__device__ __forceinline__ int first_tile_from(const Range &k, int64_t kv_len, int off, int64_t x)
+__device__ __forceinline__ int first_tile_from(const Range32 &k, int kv_len, int off, int x)
 {
     const int n_kt = (int)((kv_len + BN - 1) / BN);
     int lo = 0, hi = n_kt;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        int64_t t = (int64_t)mid * BN + off;
+        int t = mid * BN + off;
         if (t > kv_len - 1) t = kv_len - 1;
         if (range_pos(k, t) < x) lo = mid + 1; else hi = mid;
     }
@@ -134,18 +171,18 @@ __device__ __forceinline__ int first_tile_from(const Range &k, int64_t kv_len, i
 template <bool DOC>
 struct TileSeq {
     const AttnParams *p;
-    Range qr;
+    Range32 qr;
     int rank;
     int q_lo0;
     bool q_ok1;  // query tile 1 holds rows (tile 0 always does)
     int step, kt, kt_end_all;
     int kt_full0, kt_full1, kt_end0, kt_end1;
     int kt_beg0, kt_beg1, kt_fb0, kt_fb1, kt_beg_all;
-    int64_t ds_min0, ds_max0, ds_min1, ds_max1;  // document starts of the tiles' first / last rows
+    int ds_min0, ds_max0, ds_min1, ds_max1;  // document starts of the tiles' first / last rows
     int src;
-    Range kr;
+    Range32 kr;
 
-    __device__ void init(const AttnParams &pp, const Range &q, int rk, int qlo0)
+    __device__ void init(const AttnParams &pp, const Range32 &q, int rk, int qlo0)
     {
         p = &pp;
         qr = q;
@@ -158,13 +195,12 @@ struct TileSeq {
         kt_beg0 = kt_beg1 = kt_fb0 = kt_fb1 = kt_beg_all = 0;
         ds_min0 = ds_max0 = ds_min1 = ds_max1 = 0;
         if (DOC) {
-            const int64_t last = pp.q_len - 1;
-            ds_min0 = doc_start_of(pp.doc_starts, pp.n_docs, range_pos(q, (int64_t)qlo0));
-            ds_max0 = doc_start_of(pp.doc_starts, pp.n_docs, range_pos(q, (int64_t)(qlo0 + BM - 1 < last ? qlo0 + BM - 1 : last)));
+            const int last = pp.q_len - 1;
+            ds_min0 = doc_start_of(pp, range_pos(q, qlo0));
+            ds_max0 = doc_start_of(pp, range_pos(q, qlo0 + BM - 1 < last ? qlo0 + BM - 1 : last));
             if (q_ok1) {
-                ds_min1 = doc_start_of(pp.doc_starts, pp.n_docs, range_pos(q, (int64_t)(qlo0 + BM)));
-                ds_max1 = doc_start_of(pp.doc_starts, pp.n_docs,
-                                       range_pos(q, (int64_t)(qlo0 + 2 * BM - 1 < last ? qlo0 + 2 * BM - 1 : last)));
+                ds_min1 = doc_start_of(pp, range_pos(q, qlo0 + BM));
+                ds_max1 = doc_start_of(pp, range_pos(q, qlo0 + 2 * BM - 1 < last ? qlo0 + 2 * BM - 1 : last));
             }
         }
     }
@@ -189,11 +225,12 @@ struct TileSeq {
             if (step >= p->step_end) return false;
             const int N = p->n_ranks;
             src = ((rank - step) % N + N) % N;
-            kr = (p->use_layout && !p->kv_explicit) ? layout_range(p->layout, N, p->seq_len, src) : p->kv_range;
-            kv_tile_bounds<int64_t>(qr, p->q_len, q_lo0, BM, kr, p->kv_len, BN, p->causal != 0, &kt_full0, &kt_end0);
+            kr = (p->use_layout && !p->kv_explicit) ? layout_range_t<int>(p->layout, N, (int)p->seq_len, src)
+                                                    : to_range32(p->kv_range);
+            kv_tile_bounds<int>(qr, p->q_len, q_lo0, BM, kr, p->kv_len, BN, p->causal != 0, &kt_full0, &kt_end0);
             kt_full1 = kt_end1 = 0;
             if (q_ok1)
-                kv_tile_bounds<int64_t>(qr, p->q_len, q_lo0 + BM, BM, kr, p->kv_len, BN, p->causal != 0, &kt_full1,
+                kv_tile_bounds<int>(qr, p->q_len, q_lo0 + BM, BM, kr, p->kv_len, BN, p->causal != 0, &kt_full1,
                                         &kt_end1);
             if (DOC) {
                 kt_beg0 = first_tile_from(kr, p->kv_len, BN - 1, ds_min0);
@@ -239,7 +276,7 @@ __device__ __forceinline__ void store_row_chunk(void *o, int dtype, int64_t off,
     }
 }
 
-template <int D, bool DOC>
+template <int D, bool DOC, bool PERSIST>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v)
@@ -257,23 +294,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int warp = tid >> 5;
     const int lane = tid & 31;
 
-    // ---- work item: (rank, query-tile pair) from the order table, then (batch, head)
+    // ---- work items: item = (order entry e, batch, head), e = (rank, query-tile pair)
+    // from the order table.  A CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...
+    // (one item when the grid covers them all; a persistent grid walks several, its
+    // barrier phases, K/V stages and TMEM carrying over from item to item).
     const int bh_count = p.b * p.hq;
-    const int bh = blockIdx.x % bh_count;
-    const int e = blockIdx.x / bh_count;
-    int rank, qp;
-    if (p.order_len) {
-        rank = (int)(p.order[e] >> 16);
-        qp = (int)(p.order[e] & 0xffffu);
-    } else {
-        rank = e / p.n_qt;
-        qp = e % p.n_qt;
-    }
-    const int h = bh % p.hq;
-    const int bb = bh / p.hq;
-    const int hk = h / p.group;
-    const int q_lo0 = qp * (NQ * BM);
-    const Range qr = p.use_layout ? layout_range(p.layout, p.n_ranks, p.seq_len, rank) : p.q_range;
+    const int n_items = p.n_ranks * p.n_qt * bh_count;
+    struct Item {
+        int rank, qp, h, bb, hk, q_lo0;
+        Range32 qr;
+    };
+    auto decode = [&](int item) {
+        Item it;
+        const int bh = item % bh_count;
+        const int e = item / bh_count;
+        if (p.order_len) {
+            it.rank = (int)(p.order[e] >> 16);
+            it.qp = (int)(p.order[e] & 0xffffu);
+        } else {
+            it.rank = e / p.n_qt;
+            it.qp = e % p.n_qt;
+        }
+        it.h = bh % p.hq;
+        it.bb = bh / p.hq;
+        it.hk = it.h / p.group;
+        it.q_lo0 = it.qp * (NQ * BM);
+        it.qr = p.use_layout ? layout_range_t<int>(p.layout, p.n_ranks, (int)p.seq_len, it.rank) : to_range32(p.q_range);
+        return it;
+    };
+    // tensor rows the maps and outputs cover (for the debug build's bounds checks)
+    const int64_t q_rows_all = p.q_row_step ? (int64_t)p.n_ranks * p.q_row_step : p.q_len;
+    const int64_t kv_rows_all = p.kv_row_step ? (int64_t)p.n_ranks * p.kv_row_step : p.kv_len;
+    (void)q_rows_all;
+    (void)kv_rows_all;
 
     // ---- setup: barriers, TMEM
     if (tid == 0) {
@@ -283,8 +336,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int j = 0; j < NQ; ++j) {
             mbar_init(bar(C::B_SF + j), 1);
             mbar_init(bar(C::B_PF + j), BM / 32);  // one arrival per softmax warp
+            mbar_init(bar(C::B_PH + j), BM / 32);
             mbar_init(bar(C::B_PV + j), 1);
+            mbar_init(bar(C::B_OF + j), BM / 32);
         }
+        mbar_init(bar(C::B_QE), 1);
         mbar_init(bar(C::B_DONE), 1);
         *abort_flag = 0;
         mbar_fence_init();
@@ -321,32 +377,48 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             WaitCtx w{abort_flag, p.status, 1};
-            TileSeq<DOC> seq;
-            seq.init(p, qr, rank, q_lo0);
-            int n = 0;
-            const int q_row = (int)(rank * p.q_row_step) + q_lo0;
-            while (seq.next()) {
-                if (n == 0) {
-                    const int nq = seq.q_ok1 ? 2 : 1;
-                    mbar_expect_tx(bar(C::B_Q), nq * C::TILE);
-                    for (int j = 0; j < nq; ++j)
-                        for (int kb = 0; kb < D / 64; ++kb)
-                            tma_load_4d(s_base + C::OFF_Q + j * C::TILE + kb * C::SUB, &tm_q, bar(C::B_Q), kb * 64,
-                                        h, q_row + j * BM, bb);
+            int n = 0;   // K/V tiles loaded, over all work items
+            int qi = 0;  // work items that visit key tiles (each loads its Q once)
+            bool stop = false;
+            for (int item = blockIdx.x; item < n_items && !stop; item += gridDim.x) {
+                const Item it = decode(item);
+                TileSeq<DOC> seq;
+                seq.init(p, it.qr, it.rank, it.q_lo0);
+                const int q_row = (int)(it.rank * p.q_row_step) + it.q_lo0;
+                bool first = true;
+                while (seq.next()) {
+                    if (first) {
+                        // the previous item's S products have read its Q
+                        if (!mbar_wait(bar(C::B_QE), (qi & 1) ^ 1, w)) { stop = true; break; }
+                        const int nq = seq.q_ok1 ? 2 : 1;
+                        mbar_expect_tx(bar(C::B_Q), nq * C::TILE);
+                        for (int j = 0; j < nq; ++j)
+                            for (int kb = 0; kb < D / 64; ++kb)
+                                if (bounds_ok(q_row + j * BM >= 0 && q_row + j * BM < q_rows_all && it.h < p.hq &&
+                                                  it.bb < p.b,
+                                              p.status, 101))
+                                    tma_load_4d(s_base + C::OFF_Q + j * C::TILE + kb * C::SUB, &tm_q, bar(C::B_Q),
+                                                kb * 64, it.h, q_row + j * BM, it.bb);
+                        first = false;
+                        ++qi;
+                    }
+                    const int kv_row = (int)(seq.src * p.kv_row_step) + seq.kt * BN;
+                    const int sk = n % NSK, sv = n % NSV;
+                    if (!mbar_wait(bar(C::B_KE + sk), ((n / NSK) & 1) ^ 1, w)) { stop = true; break; }
+                    mbar_expect_tx(bar(C::B_KF + sk), C::TILE);
+                    const bool kv_ok = bounds_ok(kv_row >= 0 && kv_row < kv_rows_all && it.hk < p.hkv && it.bb < p.b,
+                                                 p.status, 102);
+                    for (int kb = 0; kb < D / 64 && kv_ok; ++kb)
+                        tma_load_4d(s_base + C::OFF_K + sk * C::TILE + kb * C::SUB, &tm_k, bar(C::B_KF + sk),
+                                    kb * 64, it.hk, kv_row, it.bb);
+                    if (!mbar_wait(bar(C::B_VE + sv), ((n / NSV) & 1) ^ 1, w)) { stop = true; break; }
+                    mbar_expect_tx(bar(C::B_VF + sv), C::TILE);
+                    for (int kb = 0; kb < D / 64 && kv_ok; ++kb)
+                        tma_load_4d(s_base + C::OFF_V + sv * C::TILE + kb * C::SUB, &tm_v, bar(C::B_VF + sv),
+                                    kb * 64, it.hk, kv_row, it.bb);
+                    ++n;
                 }
-                const int kv_row = (int)(seq.src * p.kv_row_step) + seq.kt * BN;
-                const int sk = n % NSK, sv = n % NSV;
-                if (!mbar_wait(bar(C::B_KE + sk), ((n / NSK) & 1) ^ 1, w)) break;
-                mbar_expect_tx(bar(C::B_KF + sk), C::TILE);
-                for (int kb = 0; kb < D / 64; ++kb)
-                    tma_load_4d(s_base + C::OFF_K + sk * C::TILE + kb * C::SUB, &tm_k, bar(C::B_KF + sk), kb * 64,
-                                hk, kv_row, bb);
-                if (!mbar_wait(bar(C::B_VE + sv), ((n / NSV) & 1) ^ 1, w)) break;
-                mbar_expect_tx(bar(C::B_VF + sv), C::TILE);
-                for (int kb = 0; kb < D / 64; ++kb)
-                    tma_load_4d(s_base + C::OFF_V + sv * C::TILE + kb * C::SUB, &tm_v, bar(C::B_VF + sv), kb * 64,
-                                hk, kv_row, bb);
-                ++n;
+                if (!PERSIST) break;
             }
             if (*abort_flag && n > 0) {
                 // let the loads already issued land in shared memory before the CTA leaves
@@ -360,17 +432,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     while (!mbar_try_wait(bar(C::B_VF + i % NSV), (i / NSV) & 1) &&
                            global_timer_ns() - t0 < kWaitLimitNs) {}
                 }
-                const uint64_t t0 = global_timer_ns();
-                while (!mbar_try_wait(bar(C::B_Q), 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
+                if (qi > 0) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar(C::B_Q), (qi - 1) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {}
+                }
             }
         }
     } else if (warp == WARP_MMA) {
         // ================================================================ MMA issuer
         if (lane == 0) {
             WaitCtx w{abort_flag, p.status, 3};
-            TileSeq<DOC> seq;
-            seq.init(p, qr, rank, q_lo0);
-            int pc0 = 0, pc1 = 0;  // PV MMAs issued per query tile
+            int pc0 = 0, pc1 = 0;  // PV products issued per query tile, over all work items
+            int oi0 = 0, oi1 = 0;  // work items whose O of query tile j was accumulated
+            int n = 0;             // key tiles consumed, over all work items (K/V stages)
+            int qi = 0;            // work items that visit key tiles (Q loads)
             auto issue_s = [&](int j, int m) {
                 const int sk = m % NSK;
                 const uint32_t d_tmem = tbase + (uint32_t)(j * 128);
@@ -384,54 +459,84 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 tc_commit(bar(C::B_SF + j));
             };
-            bool have = seq.next();
             bool ok = true;
-            if (have) {
-                ok = mbar_wait(bar(C::B_Q), 0, w) && mbar_wait(bar(C::B_KF + 0), 0, w);
-                if (ok) {
-                    tc_fence_after();
-                    for (int j = 0; j < NQ; ++j)
-                        if (seq.need(j)) issue_s(j, 0);
-                    tc_commit(bar(C::B_KE + 0));
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+                const Item it = decode(item);
+                TileSeq<DOC> seq;
+                seq.init(p, it.qr, it.rank, it.q_lo0);
+                bool have = seq.next();
+                if (!have) {
+                    if (!PERSIST) break;
+                    continue;
                 }
-            }
-            int n = 0;
-            while (have && ok) {
-                const bool need_n0 = seq.need(0), need_n1 = seq.need(1);
-                const bool have_next = seq.next();  // seq now describes tile n + 1
-                const int sv = n % NSV;
-                if (!mbar_wait(bar(C::B_VF + sv), (n / NSV) & 1, w)) break;
-                bool k_ready = false;
-#pragma unroll
-                for (int j = 0; j < NQ; ++j) {
-                    int &pc = j ? pc1 : pc0;
-                    if (j ? need_n1 : need_n0) {
-                        if (!mbar_wait(bar(C::B_PF + j), pc & 1, w)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint32_t p_tmem = tbase + (uint32_t)(j * 128);
-                        const uint32_t vb = s_base + C::OFF_V + sv * C::TILE;
-                        const uint32_t o_tmem = tbase + C::T_O + (uint32_t)(j * D);
-#pragma unroll
-                        for (int k = 0; k < BN / 16; ++k)
-                            mma_ts(o_tmem, p_tmem + k * 8, smem_desc_sw128(vb + k * 2048, C::SUB, 1024), C::IDESC_PV,
-                                   (k > 0 || pc > 0) ? 1u : 0u);
-                        tc_commit(bar(C::B_PV + j));
-                        ++pc;
-                    }
-                    if (have_next && seq.need(j)) {
-                        if (!k_ready) {
-                            if (!mbar_wait(bar(C::B_KF + (n + 1) % NSK), ((n + 1) / NSK) & 1, w)) { ok = false; break; }
-                            tc_fence_after();
-                            k_ready = true;
-                        }
-                        issue_s(j, n + 1);
-                    }
-                }
+                ok = mbar_wait(bar(C::B_Q), qi & 1, w) && mbar_wait(bar(C::B_KF + n % NSK), (n / NSK) & 1, w);
                 if (!ok) break;
-                tc_commit(bar(C::B_VE + sv));
-                if (have_next) tc_commit(bar(C::B_KE + (n + 1) % NSK));
-                ++n;
-                have = have_next;
+                tc_fence_after();
+                for (int j = 0; j < NQ; ++j)
+                    if (seq.need(j)) issue_s(j, n);
+                tc_commit(bar(C::B_KE + n % NSK));
+                bool pv0 = false, pv1 = false;  // query tile j has a PV product in this item
+                while (have && ok) {
+                    const bool need_n0 = seq.need(0), need_n1 = seq.need(1);
+                    const bool have_next = seq.next();  // seq now describes tile n + 1
+                    if (!have_next) tc_commit(bar(C::B_QE));  // the item's last S products are issued
+                    const int sv = n % NSV;
+                    if (!mbar_wait(bar(C::B_VF + sv), (n / NSV) & 1, w)) { ok = false; break; }
+                    bool k_ready = false;
+#pragma unroll
+                    for (int j = 0; j < NQ; ++j) {
+                        int &pc = j ? pc1 : pc0;
+                        bool &pv = j ? pv1 : pv0;
+                        const int oi = j ? oi1 : oi0;
+                        if (j ? need_n1 : need_n0) {
+                            const uint32_t p_tmem = tbase + (uint32_t)(j * 128);
+                            const uint32_t vb = s_base + C::OFF_V + sv * C::TILE;
+                            const uint32_t o_tmem = tbase + C::T_O + (uint32_t)(j * D);
+                            // the first product of an item overwrites O: the previous item's
+                            // epilogue must have read it out
+                            if (!pv && oi > 0 && !mbar_wait(bar(C::B_OF + j), (oi - 1) & 1, w)) { ok = false; break; }
+                            if (kSplitP) {
+                                // PV in two halves of 64 keys: the first half runs while the
+                                // softmax still computes the probabilities of the second
+                                if (!mbar_wait(bar(C::B_PF + j), pc & 1, w)) { ok = false; break; }
+                                tc_fence_after();
+#pragma unroll
+                                for (int k = 0; k < BN / 32; ++k)
+                                    mma_ts(o_tmem, p_tmem + k * 8, smem_desc_sw128(vb + k * 2048, C::SUB, 1024),
+                                           C::IDESC_PV, (k > 0 || pv) ? 1u : 0u);
+                            }
+                            if (!mbar_wait(bar(C::B_PH + j), pc & 1, w)) { ok = false; break; }
+                            tc_fence_after();
+#pragma unroll
+                            for (int k = kSplitP ? BN / 32 : 0; k < BN / 16; ++k)
+                                mma_ts(o_tmem, p_tmem + k * 8, smem_desc_sw128(vb + k * 2048, C::SUB, 1024),
+                                       C::IDESC_PV, (k > 0 || pv) ? 1u : 0u);
+                            tc_commit(bar(C::B_PV + j));
+                            ++pc;
+                            pv = true;
+                        }
+                        if (have_next && seq.need(j)) {
+                            if (!k_ready) {
+                                if (!mbar_wait(bar(C::B_KF + (n + 1) % NSK), ((n + 1) / NSK) & 1, w)) {
+                                    ok = false;
+                                    break;
+                                }
+                                tc_fence_after();
+                                k_ready = true;
+                            }
+                            issue_s(j, n + 1);
+                        }
+                    }
+                    if (!ok) break;
+                    tc_commit(bar(C::B_VE + sv));
+                    if (have_next) tc_commit(bar(C::B_KE + (n + 1) % NSK));
+                    ++n;
+                    have = have_next;
+                }
+                if (pv0) ++oi0;
+                if (pv1) ++oi1;
+                ++qi;
+                if (!PERSIST) break;
             }
             // drain: every MMA issued above has finished before TMEM is released
             tc_commit(bar(C::B_DONE));
@@ -448,94 +553,117 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int wl = warp & 3;        // TMEM lane quadrant
         const int r_in = wl * 32 + lane;  // row within the query tile
         WaitCtx w{abort_flag, p.status, 5 + j};
-        const int row = q_lo0 + j * BM + r_in;  // local query index in the rank's block
-        const bool row_ok = row < p.q_len;
-        const int64_t pos_q = range_pos(qr, row_ok ? row : (p.q_len > 0 ? p.q_len - 1 : 0));
-        const int64_t ds_row = DOC ? doc_start_of(p.doc_starts, p.n_docs, pos_q) : 0;
         const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
         const uint32_t s_tmem = tbase + lane_off + (uint32_t)(j * 128);
         const uint32_t o_tmem = tbase + lane_off + C::T_O + (uint32_t)(j * D);
         const float sl2 = p.scale_log2;
+        int cs = 0;           // S tiles of this query tile consumed, over all work items
+        bool aborted = false;
+
+        for (int item = blockIdx.x; item < n_items && !aborted; item += gridDim.x) {
+        const Item it = decode(item);
+        const int rank = it.rank, h = it.h, bb = it.bb, q_lo0 = it.q_lo0;
+        const Range32 qr = it.qr;
+        const int row = q_lo0 + j * BM + r_in;  // local query index in the rank's block
+        const bool row_in = row < p.q_len;
+        const int pos_q = range_pos(qr, row_in ? row : (p.q_len > 0 ? p.q_len - 1 : 0));
+        const int ds_row = DOC ? doc_start_of(p, pos_q) : 0;
 
         float m = -INFINITY;  // max used in the exponent (log2 units)
         float l = 0.f;        // running sum
-        int c = 0;            // tiles processed by this query tile
-        bool aborted = false;
+        int c = 0;            // tiles processed by this query tile in this item
 
         TileSeq<DOC> seq;
         seq.init(p, qr, rank, q_lo0);
+        // Both softmax warpgroups walk the CTA's whole key-tile sequence (the union of
+        // what the two query tiles visit).  With kPingPong their exponential phases
+        // take turns (tile 0 first at every entry), so each has the MUFU pipe to
+        // itself while the tensor core runs the other tile's products; a warpgroup
+        // with nothing to do at an entry still takes and hands over its turn, and a
+        // warpgroup that gave up (bounded wait expired) keeps taking its turns
+        // without work, so the hand-overs always pair up.
+        int nseq = 0;
         while (seq.next()) {
-            if (!seq.need(j)) continue;
-            {
-                const bool okw = mbar_wait(bar(C::B_SF + j), c & 1, w);
-                if (__any_sync(0xffffffffu, !okw)) { aborted = true; break; }
+            bool mine = seq.need(j) && !aborted;
+            if (mine) {
+                const bool okw = mbar_wait(bar(C::B_SF + j), cs & 1, w);
+                if (__any_sync(0xffffffffu, !okw)) { aborted = true; mine = false; }
             }
-            tc_fence_after();
             float s[BN];
-            tmem_ld64f_nowait(s_tmem, s);
-            tmem_ld64f_nowait(s_tmem + 64, s + 64);
-            tmem_wait_ld_dep(s);
-            reg_dep64(s + 64);
-            // ---- mask (partial tiles only).  Positions increase with the local key
-            // index, so the keys this row may see form a prefix of the tile.
-            if (seq.partial(j)) {
-                const int k0 = seq.kt * BN;
-                int cnt = p.kv_len - k0;
-                if (cnt > BN) cnt = BN;
-                if (p.causal) {
-                    int lo = 0, hi = cnt;
-                    while (lo < hi) {
-                        const int mid = (lo + hi) >> 1;
-                        if (range_pos(seq.kr, k0 + mid) <= pos_q) lo = mid + 1; else hi = mid;
-                    }
-                    cnt = lo;
-                }
-                int beg = 0;  // keys before this row's document start are invisible
-                if (DOC) {
-                    int lo = 0, hi = cnt;
-                    while (lo < hi) {
-                        const int mid = (lo + hi) >> 1;
-                        if (range_pos(seq.kr, k0 + mid) < ds_row) lo = mid + 1; else hi = mid;
-                    }
-                    beg = lo;
-                }
-#pragma unroll
-                for (int cc = 0; cc < BN; ++cc)
-                    if (cc >= cnt || (DOC && cc < beg)) s[cc] = -INFINITY;
-            }
-            // ---- row max: four chains of 3-input max
-            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-            for (int cc = 4; cc < BN - 4; cc += 8) {
-                mx0 = fmax3(mx0, s[cc], s[cc + 1]);
-                mx1 = fmax3(mx1, s[cc + 2], s[cc + 3]);
-                mx2 = fmax3(mx2, s[cc + 4], s[cc + 5]);
-                mx3 = fmax3(mx3, s[cc + 6], s[cc + 7]);
-            }
-            mx0 = fmax3(mx0, s[BN - 4], s[BN - 3]);
-            mx1 = fmax3(mx1, s[BN - 2], s[BN - 1]);
-            const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
-            // Raise the exponent's max only when it grew by more than the threshold;
-            // then O and l are rescaled below (after P is out of the registers).
-            float f_rescale = 1.f;
+            float f_rescale = 1.f, mu = 0.f;
             bool rescale = false;
-            if (c == 0) {
-                m = mx;
-            } else {
-                const bool need_rescale = mx > m + kRescaleThreshold;
-                rescale = __any_sync(0xffffffffu, need_rescale);
-                if (rescale) {
-                    const float m_new = fmaxf(m, mx);
-                    f_rescale = (m_new == m) ? 1.f : ex2_approx(m - m_new);
-                    m = m_new;
-                    l *= f_rescale;
+            if (kPingPong && !kTurnLate && (j == 1 || nseq > 0)) named_bar_sync(j == 0 ? kTurn0 : kTurn1, 2 * BM);
+            if (mine) {
+                tc_fence_after();
+                tmem_ld64f_nowait(s_tmem, s);
+                tmem_ld64f_nowait(s_tmem + 64, s + 64);
+                tmem_wait_ld_dep(s);
+                reg_dep64(s + 64);
+                // ---- mask (partial tiles only).  Positions increase with the local key
+                // index, so the keys this row may see form a prefix of the tile.
+                if (seq.partial(j)) {
+                    const int k0 = seq.kt * BN;
+                    int cnt = p.kv_len - k0;
+                    if (cnt > BN) cnt = BN;
+                    if (p.causal) {
+                        int lo = 0, hi = cnt;
+                        while (lo < hi) {
+                            const int mid = (lo + hi) >> 1;
+                            if (range_pos(seq.kr, k0 + mid) <= pos_q) lo = mid + 1; else hi = mid;
+                        }
+                        cnt = lo;
+                    }
+                    int beg = 0;  // keys before this row's document start are invisible
+                    if (DOC) {
+                        int lo = 0, hi = cnt;
+                        while (lo < hi) {
+                            const int mid = (lo + hi) >> 1;
+                            if (range_pos(seq.kr, k0 + mid) < ds_row) lo = mid + 1; else hi = mid;
+                        }
+                        beg = lo;
+                    }
+#pragma unroll
+                    for (int cc = 0; cc < BN; ++cc)
+                        if (cc >= cnt || (DOC && cc < beg)) s[cc] = -INFINITY;
                 }
+                // ---- row max: four chains of 3-input max
+                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+                for (int cc = 4; cc < BN - 4; cc += 8) {
+                    mx0 = fmax3(mx0, s[cc], s[cc + 1]);
+                    mx1 = fmax3(mx1, s[cc + 2], s[cc + 3]);
+                    mx2 = fmax3(mx2, s[cc + 4], s[cc + 5]);
+                    mx3 = fmax3(mx3, s[cc + 6], s[cc + 7]);
+                }
+                mx0 = fmax3(mx0, s[BN - 4], s[BN - 3]);
+                mx1 = fmax3(mx1, s[BN - 2], s[BN - 1]);
+                const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
+                // Raise the exponent's max only when it grew by more than the threshold;
+                // then l is rescaled here and O below, before the first half of P is
+                // handed to the MMA warp.
+                if (c == 0) {
+                    m = mx;
+                } else {
+                    const bool need_rescale = mx > m + kRescaleThreshold;
+                    rescale = __any_sync(0xffffffffu, need_rescale);
+                    if (rescale) {
+                        const float m_new = fmaxf(m, mx);
+                        f_rescale = (m_new == m) ? 1.f : ex2_approx(m - m_new);
+                        m = m_new;
+                        l *= f_rescale;
+                    }
+                }
+                mu = (m == -INFINITY) ? 0.f : m;
             }
-            const float mu = (m == -INFINITY) ? 0.f : m;
-            // ---- probabilities, row sum, bf16 P into TMEM columns [0, 64) of S_j,
-            // 32 columns at a time so each chunk's scores die once packed.  The
-            // scale-subtract and the row sum run as packed fp32x2 instructions.
-            {
+            if (kPingPong && kTurnLate && (j == 1 || nseq > 0)) named_bar_sync(j == 0 ? kTurn0 : kTurn1, 2 * BM);
+            if (mine) {
+                // ---- probabilities, row sum, bf16 P into TMEM columns [0, 64) of S_j,
+                // 32 columns at a time so each chunk's scores die once packed.  The
+                // scale-subtract and the row sum run as packed fp32x2 instructions.
+                // With kSplitP, P is handed to the MMA warp in two halves (keys [0, 64),
+                // then [64, 128)); a rescale of O happens before the first half, since
+                // PV adds into O.
+                bool okr = true;
                 const uint64_t sl2x2 = f2_pack(sl2, sl2);
                 const uint64_t nmux2 = f2_pack(-mu, -mu);
                 uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = f2_pack(0.f, 0.f);
@@ -558,47 +686,66 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         pk[i] = pack_bf16x2(e0, e1);
                     }
                     tmem_st16(s_tmem + 16 * q4, pk);
+                    if (q4 == (kSplitP ? 1 : 3) && rescale) {
+                        // O must hold every earlier tile's P V before it is rescaled
+                        const bool okw = mbar_wait(bar(C::B_PV + j), (cs - 1) & 1, w);
+                        okr = !__any_sync(0xffffffffu, !okw);
+                        if (okr) {
+                            tc_fence_after();
+#pragma unroll
+                            for (int c0 = 0; c0 < D; c0 += 32) {
+                                uint32_t r[32];
+                                tmem_ld32(o_tmem + c0, r);
+#pragma unroll
+                                for (int cc = 0; cc < 32; ++cc)
+                                    r[cc] = __float_as_uint(__uint_as_float(r[cc]) * f_rescale);
+                                tmem_st32(o_tmem + c0, r);
+                            }
+                        }
+                    }
+                    if (q4 == 3 && kPingPong) named_bar_arrive(j == 0 ? kTurn1 : kTurn0, 2 * BM);
+                    if ((kSplitP && q4 == 1) || q4 == 3) {
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0 && okr) mbar_arrive(bar((kSplitP && q4 == 1) ? C::B_PF + j : C::B_PH + j));
+                    }
                 }
                 float a0, a1, a2, a3;
                 f2_unpack(acc0, a0, a1);
                 f2_unpack(acc1, a2, a3);
                 l += (a0 + a1) + (a2 + a3);
-            }
-            if (rescale) {
-                // O must hold every earlier tile's P V before it is rescaled
-                const bool okw = mbar_wait(bar(C::B_PV + j), (c - 1) & 1, w);
-                if (__any_sync(0xffffffffu, !okw)) { aborted = true; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t r[32];
-                    tmem_ld32(o_tmem + c0, r);
-#pragma unroll
-                    for (int cc = 0; cc < 32; ++cc) r[cc] = __float_as_uint(__uint_as_float(r[cc]) * f_rescale);
-                    tmem_st32(o_tmem + c0, r);
+                if (okr) {
+                    ++c;
+                    ++cs;
+                } else {
+                    aborted = true;
                 }
+            } else if (kPingPong) {
+                named_bar_arrive(j == 0 ? kTurn1 : kTurn0, 2 * BM);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_PF + j));
-            ++c;
+            ++nseq;
         }
+        // tile 0 takes the hand-over of tile 1's last turn
+        if (kPingPong && j == 0 && nseq > 0) named_bar_sync(kTurn0, 2 * BM);
         aborted = __any_sync(0xffffffffu, aborted || (*abort_flag != 0));
 
         // ================================================================ epilogue
         if (!aborted && c > 0) {
-            const bool okw = mbar_wait(bar(C::B_PV + j), (c - 1) & 1, w);
+            const bool okw = mbar_wait(bar(C::B_PV + j), (cs - 1) & 1, w);
             aborted = __any_sync(0xffffffffu, !okw);
             if (!aborted) tc_fence_after();
         }
-        if (!aborted && (c > 0 || p.epi == EPI_STORE)) {
+        if (!aborted && (c > 0 || p.epi == EPI_STORE || p.o_out != nullptr)) {
             const bool empty = !(l > 0.f);
             const float lse2 = empty ? -INFINITY : m + log2f(l);
             const float inv_l = empty ? 0.f : 1.f / l;
             const int64_t orow = (int64_t)rank * p.q_row_step + row;
             const int64_t obase = (int64_t)bb * p.o_sb + orow * p.o_ss + (int64_t)h * p.o_sh;
             float *lse_ptr = p.lse + (int64_t)bb * p.lse_sb + (int64_t)h * p.lse_sh + orow * p.lse_ss;
+            // a row outside the output tensors (debug builds record it and skip it)
+            const bool row_ok = row_in && bounds_ok(orow >= 0 && orow < q_rows_all && h < p.hq && bb < p.b,
+                                                    p.status, 103);
             if (p.epi == EPI_STORE) {
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += 32) {
@@ -611,7 +758,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 if (row_ok) *lse_ptr = lse2 * kLn2;
             } else {
-                // EPI_MERGE: (o, lse) in memory are fp32 and hold a partial; LSE-merge into them
+                // EPI_MERGE: (o, lse) in memory are fp32 and hold a partial; LSE-merge
+                // this launch's result into them.  With o_out set, the merged o goes
+                // there (in o_out's dtype) instead of back into o, also for rows this
+                // launch gave nothing (a copy of the partial in memory).
+                const bool to_out = p.o_out != nullptr;
                 const float la = row_ok ? *lse_ptr * kLog2e : -INFINITY;
                 float wa = 1.f, wb = 0.f, new_lse = la;
                 if (!empty) {
@@ -626,28 +777,43 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         wb = ex2_approx(lse2 - new_lse) * inv_l;
                     }
                 }
-                float *orow_ptr = reinterpret_cast<float *>(p.o) + obase;
+                const float *orow_ptr = reinterpret_cast<const float *>(p.o) + obase;
+                const int64_t out_base =
+                    to_out ? (int64_t)bb * p.oo_sb + orow * p.oo_ss + (int64_t)h * p.oo_sh : obase;
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     uint32_t r[32];
-                    tmem_ld32(o_tmem + c0, r);
-                    if (row_ok && !empty) {
+                    if (c > 0) tmem_ld32(o_tmem + c0, r);
+                    if (row_ok && (!empty || to_out)) {
                         float v[32];
                         const float4 *src4 = reinterpret_cast<const float4 *>(orow_ptr + c0);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const float4 a = (wa != 0.f) ? src4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-                            v[4 * i + 0] = fmaf(wa, a.x, wb * __uint_as_float(r[4 * i + 0]));
-                            v[4 * i + 1] = fmaf(wa, a.y, wb * __uint_as_float(r[4 * i + 1]));
-                            v[4 * i + 2] = fmaf(wa, a.z, wb * __uint_as_float(r[4 * i + 2]));
-                            v[4 * i + 3] = fmaf(wa, a.w, wb * __uint_as_float(r[4 * i + 3]));
+                            const float b0 = empty ? 0.f : wb * __uint_as_float(r[4 * i + 0]);
+                            const float b1 = empty ? 0.f : wb * __uint_as_float(r[4 * i + 1]);
+                            const float b2 = empty ? 0.f : wb * __uint_as_float(r[4 * i + 2]);
+                            const float b3 = empty ? 0.f : wb * __uint_as_float(r[4 * i + 3]);
+                            v[4 * i + 0] = fmaf(wa, a.x, b0);
+                            v[4 * i + 1] = fmaf(wa, a.y, b1);
+                            v[4 * i + 2] = fmaf(wa, a.z, b2);
+                            v[4 * i + 3] = fmaf(wa, a.w, b3);
                         }
-                        store_row_chunk(p.o, DT_FP32, obase + c0, v);
+                        if (to_out) store_row_chunk(p.o_out, p.o_out_dtype, out_base + c0, v);
+                        else store_row_chunk(p.o, DT_FP32, obase + c0, v);
                     }
                 }
                 if (row_ok && !empty) *lse_ptr = new_lse * kLn2;
             }
         }
+        if (!PERSIST) break;
+        if (!aborted && c > 0) {
+            // O of this tile is read out: the next item's first PV may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_OF + j));
+        }
+        }  // work items
         teardown();
     }
 }
@@ -690,20 +856,34 @@ bool make_map(CUtensorMap *m, const void *base, int64_t b, int64_t s, int64_t H,
     return r == CUDA_SUCCESS;
 }
 
-template <int D, bool DOC>
+// Streaming multiprocessors of the current device (looked up once per device).
+int sm_count()
+{
+    static int counts[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 0 || dev >= 64) return 148;
+    if (!counts[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        counts[dev] = n;
+    }
+    return counts[dev];
+}
+
+template <int D, bool DOC, bool PERSIST>
 cudaError_t launch_dd(const AttnParams &p, cudaStream_t stream, const CUtensorMap &tq, const CUtensorMap &tk,
                       const CUtensorMap &tv)
 {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e =
-            cudaFuncSetAttribute(attn_tc_kernel<D, DOC>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static unsigned long long attr_done = 0;
+    cudaError_t e = set_smem_per_device((const void *)attn_tc_kernel<D, DOC, PERSIST>, Cfg<D>::SMEM, &attr_done);
+    if (e != cudaSuccess) return e;
     const int64_t items = (int64_t)p.n_ranks * p.n_qt * p.b * p.hq;
     if (items == 0) return cudaSuccess;
-    attn_tc_kernel<D, DOC><<<(unsigned)items, NTHREADS, Cfg<D>::SMEM, stream>>>(p, tq, tk, tv);
+    if (items > INT32_MAX) return cudaErrorInvalidValue;
+    // persistent: one CTA per SM walks the items (one CTA fits an SM); otherwise one per item
+    const int64_t grid = PERSIST ? std::min<int64_t>(items, sm_count()) : items;
+    attn_tc_kernel<D, DOC, PERSIST><<<(unsigned)grid, NTHREADS, Cfg<D>::SMEM, stream>>>(p, tq, tk, tv);
     return cudaGetLastError();
 }
 
@@ -715,7 +895,10 @@ cudaError_t launch_d(const AttnParams &p, cudaStream_t stream, int64_t q_rows, i
         !make_map(&tk, p.k, p.b, kv_rows, p.hkv, D, p.k_sb, p.k_ss, p.k_sh) ||
         !make_map(&tv, p.v, p.b, kv_rows, p.hkv, D, p.v_sb, p.v_ss, p.v_sh))
         return cudaErrorInvalidValue;
-    return p.n_docs > 0 ? launch_dd<D, true>(p, stream, tq, tk, tv) : launch_dd<D, false>(p, stream, tq, tk, tv);
+    // the document mask leaves few key tiles per work item: a persistent grid keeps the
+    // per-item set-up (Q load, pipeline fill, epilogue) off the critical path
+    if (p.n_docs > 0) return launch_dd<D, true, kDocPersist>(p, stream, tq, tk, tv);
+    return launch_dd<D, false, kRingPersist>(p, stream, tq, tk, tv);
 }
 
 }  // namespace

@@ -92,8 +92,13 @@ struct BwdParams {
     int kv_explicit, n_kv_blocks;
     const int *doc_starts;
     int n_docs;
-    // accumulate = 1 (the block form, FFMA kernels only): dq, dk, dv are fp32 and this
-    // call's shares are added to them; 0: they are written in the input dtype
+    // tensor-core path: doc_pos_end[pos] = first position past the document holding
+    // position pos (INT32_MAX for the last document), from launch_doc_tables
+    const int *doc_pos_end;
+    // accumulate = 1 (the block form): dq, dk, dv are fp32 and this call's shares are
+    // added to them (the tensor-core kernel reduces dQ straight into dq_acc = dq and
+    // adds dK, dV in its epilogue; no dq conversion); 0: they are written in the
+    // input dtype
     int accumulate;
     // work order: entry e -> (key block, key tile) = (order[e] >> 16, order[e] & 0xffff);
     // head_major puts (batch, kv head) outside the order in the grid

@@ -46,6 +46,11 @@ struct AttnParams {
     int64_t o_sb, o_ss, o_sh;
     float *lse;
     int64_t lse_sb, lse_sh, lse_ss;
+    // EPI_MERGE only (tensor-core path): when o_out is set, the merged o is written
+    // there in o_out_dtype (strides oo_*) and o is left as it was; lse is updated.
+    void *o_out;
+    int o_out_dtype;
+    int64_t oo_sb, oo_ss, oo_sh;
     int *status;
     // All-Gather form: kv_explicit = 1 takes kv_range for every rank and step (one
     // gathered key block, kv_row_step = 0).  Document mask (bf16 path): doc_starts
@@ -54,6 +59,9 @@ struct AttnParams {
     int kv_explicit;
     const int *doc_starts;
     int n_docs;
+    // tensor-core path: doc_pos_start[pos] = first position of the document holding
+    // position pos (of the seq_len positions), from launch_doc_tables
+    const int *doc_pos_start;
     // work order: entry e -> (rank, row group) = (order[e] >> 16, order[e] & 0xffff);
     // a row group is the query rows one CTA covers (256 tensor-core, 128 SIMT)
     int n_qt;                  // row groups per rank
@@ -90,6 +98,19 @@ struct PermuteParams {
     void *dst;
 };
 cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream);
+
+// Raises the dynamic shared-memory limit of kernel `fn` to `bytes` on the current
+// device, once per device (the attribute belongs to the device, not the process):
+// `done` keeps one bit per device ordinal below 64; higher ordinals set it on every
+// call.  From status.cu.
+cudaError_t set_smem_per_device(const void *fn, int bytes, unsigned long long *done);
+
+// Per-position document bounds (doc_tables.cu): for every position p < seq_len,
+// doc_start[p] = the first position of the document holding p and doc_end[p] = the
+// first position past it (INT32_MAX for the last document); starts: n_docs sorted
+// document starts on the device, the first 0.
+cudaError_t launch_doc_tables(const int *starts, int n_docs, int64_t seq_len, int *doc_start, int *doc_end,
+                              cudaStream_t stream);
 
 // Device status word of the current device (2 ints), from status.cu.
 cudaError_t status_word(int **ptr);

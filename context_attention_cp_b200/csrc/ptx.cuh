@@ -9,7 +9,16 @@ namespace cpattn {
 
 // Device status word layout (see status.cu): word 0 collects error bits, word 1
 // records where the first bounded wait gave up.
-enum { STATUS_TIMEOUT = 1 };
+enum { STATUS_TIMEOUT = 1, STATUS_BOUNDS = 2 };
+
+// Debug builds (CP_DEBUG_BOUNDS=1, libcpattn_debug.so) check every TMA coordinate
+// and every global index of the tensor-core kernels before the access.  A failed
+// check records STATUS_BOUNDS and the check's tag in the status word and skips the
+// access (no trap); cp_stream_check then reports CP_ERR_BOUNDS.  Release builds
+// compile the checks away.
+#ifndef CP_DEBUG_BOUNDS
+#define CP_DEBUG_BOUNDS 0
+#endif
 
 // A bounded wait gives up after this long and reports STATUS_TIMEOUT.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
@@ -112,6 +121,38 @@ static __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t pa
 static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx &w)
 {
     return mbar_wait_limit(bar, parity, w, kWaitLimitNs);
+}
+
+// True when `ok` holds; in debug builds a false `ok` is recorded (STATUS_BOUNDS, tag).
+__device__ __forceinline__ bool bounds_ok(bool ok, int *status, int tag)
+{
+#if CP_DEBUG_BOUNDS
+    if (!ok) {
+        atomicOr(status, STATUS_BOUNDS);
+        atomicCAS(status + 1, 0, tag);
+    }
+    return ok;
+#else
+    (void)ok;
+    (void)status;
+    (void)tag;
+    return true;
+#endif
+}
+
+// ------------------------------------------------------------------ named barriers
+
+// Waits at named barrier `id` until `nthreads` threads have arrived (this warp's
+// threads included).  Warp-uniform.
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Arrives at named barrier `id` (expecting `nthreads` in all) without waiting.
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ------------------------------------------------------------------ TMA

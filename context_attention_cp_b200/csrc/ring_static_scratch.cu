@@ -21,7 +21,10 @@
 //     its whole partial before the merge reads it), so nothing has to be cleared;
 //   - the first call on a device looks up the array's device address (a host-side
 //     reference to the array is not a device address); make that first call before
-//     any stream capture on that device.
+//     any stream capture on that device;
+//   - the looked-up address is kept for the life of the process; a device reset
+//     (cudaDeviceReset) unloads the array, after which this entry point must not be
+//     called on that device.
 #include <cuda_runtime.h>
 
 #include <mutex>

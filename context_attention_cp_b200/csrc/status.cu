@@ -29,6 +29,18 @@ cudaError_t status_word(int **ptr)
     return cudaSuccess;
 }
 
+cudaError_t set_smem_per_device(const void *fn, int bytes, unsigned long long *done)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (bit && (__atomic_load_n(done, __ATOMIC_ACQUIRE) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) __atomic_fetch_or(done, bit, __ATOMIC_RELEASE);
+    return e;
+}
+
 namespace {
 
 // One warp waits on an mbarrier that nothing ever arrives at; the bounded wait runs

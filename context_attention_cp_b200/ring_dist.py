@@ -32,32 +32,58 @@ import torch.distributed as dist
 from . import _binding as B
 
 
+def _nvtx_push(t, name):
+    """An NVTX range per ring step for profilers (CUDA tensors only)."""
+    if t.is_cuda:
+        torch.cuda.nvtx.range_push(name)
+
+
+def _nvtx_pop(t):
+    if t.is_cuda:
+        torch.cuda.nvtx.range_pop()
+
+
 def block_compute(q, k, v, q_range, kv_range, causal, scale, o, lse, accumulate):
     """The default step: the tensor-core (bf16) or FFMA (fp32) block kernel."""
     B.block_attn_fwd(q, k, v, q_range, kv_range, causal, scale, o, lse, accumulate=accumulate)
 
 
-def ring_attn_fwd_dist(q, k, v, layout, causal, scale=None, group=None, compute=block_compute):
+def merge_out(o_acc, lse_acc, o_b, lse_b, o_out):
+    """The default last merge: the standalone LSE-merge kernel writing o in the
+    output dtype."""
+    B.lse_merge(o_acc, lse_acc, o_b, lse_b, o_out=o_out)
+
+
+def ring_attn_fwd_dist(q, k, v, layout, causal, scale=None, group=None, compute=block_compute, merge=merge_out):
     """This rank's share of ring attention.
 
     q [b, c, Hq, d], k / v [b, c, Hkv, d]: this rank's local blocks (its layout
     positions, in order).  Returns (o [b, c, Hq, d] in q's dtype, lse [b, Hq, c]
     fp32) for the local queries.  All ranks of `group` call it together.
+
+    Steps 0 .. N-2 keep the running (o, lse) in fp32 (the block kernel's fused
+    merge from step 1 on); the last step writes its partial and the standalone
+    merge folds it in and writes o in q's dtype.
     """
     rank = dist.get_rank(group)
     N = dist.get_world_size(group)
     b, c, Hq, d = q.shape
     if scale is None:
-        scale = d ** -0.5
+        scale = 0.0  # the library's default: 1/sqrt(d)
     S = c * N
     q_range = B.layout_range(layout, N, S, rank)
     nxt, prv = (rank + 1) % N, (rank - 1) % N
     to_global = (lambda r: dist.get_global_rank(group, r)) if group is not None else (lambda r: r)
-    o = torch.empty((b, c, Hq, d), dtype=torch.float32, device=q.device)
+    out = torch.empty((b, c, Hq, d), dtype=q.dtype, device=q.device)
     lse = torch.empty((b, Hq, c), dtype=torch.float32, device=q.device)
+    if N == 1:
+        compute(q, k, v, q_range, q_range, causal, scale, out, lse, False)
+        return out, lse
+    o = torch.empty((b, c, Hq, d), dtype=torch.float32, device=q.device)
     cur_k, cur_v = k.contiguous(), v.contiguous()
     buf_k, buf_v = torch.empty_like(cur_k), torch.empty_like(cur_v)
     for r in range(N):
+        _nvtx_push(q, "ring step %d of %d" % (r, N))
         src = (rank - r) % N                      # the block this rank holds at step r
         reqs = []
         if r + 1 < N:                             # pass the block on, take the next one
@@ -66,13 +92,21 @@ def ring_attn_fwd_dist(q, k, v, layout, causal, scale=None, group=None, compute=
                    dist.P2POp(dist.irecv, buf_k, to_global(prv), group),
                    dist.P2POp(dist.irecv, buf_v, to_global(prv), group)]
             reqs = dist.batch_isend_irecv(ops)
-        compute(q, cur_k, cur_v, q_range, B.layout_range(layout, N, S, src), causal, scale, o, lse, r > 0)
+        kv_range = B.layout_range(layout, N, S, src)
+        if r + 1 < N:
+            compute(q, cur_k, cur_v, q_range, kv_range, causal, scale, o, lse, r > 0)
+        else:
+            o_b = torch.empty_like(out)
+            lse_b = torch.empty_like(lse)
+            compute(q, cur_k, cur_v, q_range, kv_range, causal, scale, o_b, lse_b, False)
+            merge(o, lse, o_b, lse_b, out)
         for req in reqs:
             req.wait()
         if r + 1 < N:
             cur_k, buf_k = buf_k, cur_k
             cur_v, buf_v = buf_v, cur_v
-    return o.to(q.dtype), lse
+        _nvtx_pop(q)
+    return out, lse
 
 
 def block_bwd_compute(q, k, v, o, lse, do, q_range, kv_range, causal, scale, dq_acc, dk_acc, dv_acc):
@@ -93,7 +127,7 @@ def ring_attn_bwd_dist(q, k, v, o, lse, do, layout, causal, scale=None, group=No
     N = dist.get_world_size(group)
     b, c, Hq, d = q.shape
     if scale is None:
-        scale = d ** -0.5
+        scale = 0.0  # the library's default: 1/sqrt(d)
     S = c * N
     q_range = B.layout_range(layout, N, S, rank)
     nxt, prv = (rank + 1) % N, (rank - 1) % N
@@ -104,13 +138,15 @@ def ring_attn_bwd_dist(q, k, v, o, lse, do, layout, causal, scale=None, group=No
         ops += [dist.P2POp(dist.irecv, t, to_global(prv), group) for t in recv]
         return dist.batch_isend_irecv(ops)
 
-    f32 = dict(dtype=torch.float32, device=q.device)
-    dq = torch.zeros(q.shape, **f32)
+    dq = torch.zeros(q.shape, dtype=torch.float32, device=q.device)
     cur_k, cur_v = k.contiguous(), v.contiguous()
     buf_k, buf_v = torch.empty_like(cur_k), torch.empty_like(cur_v)
+    # the travelling accumulators live where the travelling block does
+    f32 = dict(dtype=torch.float32, device=k.device)
     cur_dk, cur_dv = torch.zeros(k.shape, **f32), torch.zeros(v.shape, **f32)
     buf_dk, buf_dv = torch.empty_like(cur_dk), torch.empty_like(cur_dv)
     for r in range(N):
+        _nvtx_push(q, "ring backward step %d of %d" % (r, N))
         src = (rank - r) % N                      # the block this rank holds at step r
         kv_reqs = exchange([cur_k, cur_v], [buf_k, buf_v]) if r + 1 < N else []
         compute(q, cur_k, cur_v, o, lse, do, q_range, B.layout_range(layout, N, S, src), causal, scale, dq,
@@ -125,4 +161,5 @@ def ring_attn_bwd_dist(q, k, v, o, lse, do, layout, causal, scale=None, group=No
             if r + 1 < N:
                 cur_k, buf_k = buf_k, cur_k
                 cur_v, buf_v = buf_v, cur_v
+        _nvtx_pop(q)
     return dq.to(q.dtype), cur_dk.to(k.dtype), cur_dv.to(v.dtype)

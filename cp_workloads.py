@@ -76,9 +76,12 @@ WORKLOADS = [
     Workload("noncausal_s64k_contig32", 5, "bf16", 1, 16, 16, 128, 65536, False, "contiguous", 32),
     Workload("llama3_8b_s8k_zigzag4_docs8", 6, "bf16", 1, 32, 8, 128, 8192, True, "zigzag", 4, n_docs=8,
              notes="All-Gather CP with a document mask"),
+    Workload("llama3_8b_s8k_zigzag4_docs32", 7, "bf16", 1, 32, 8, 128, 8192, True, "zigzag", 4, n_docs=32,
+             notes="All-Gather CP with a document mask, short documents"),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
-BENCH_WORKLOAD = "llama3_8b_s8k_zigzag4"
+# the largest workload that fits one GPU: the Llama-3-70B head shape at S = 131072
+BENCH_WORKLOAD = "llama3_70b_s128k_zigzag8"
 
 
 def torch_dtype(name):

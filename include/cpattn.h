@@ -51,7 +51,10 @@ typedef enum {
     CP_ERR_UNSUPPORTED = 2, /* valid request the library does not implement (e.g. d) */
     CP_ERR_SHAPE = 3,       /* inconsistent or indivisible sizes */
     CP_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
-    CP_ERR_TIMEOUT = 5      /* a device-side bounded wait expired (see cp_stream_check) */
+    CP_ERR_TIMEOUT = 5,     /* a device-side bounded wait expired (see cp_stream_check) */
+    CP_ERR_BOUNDS = 6       /* debug build (libcpattn_debug.so) only: a kernel's bounds check
+                               of a TMA coordinate or global index failed; the access was
+                               skipped (see cp_stream_check) */
 } cp_status;
 
 typedef enum { CP_BF16 = 0, CP_FP32 = 1 } cp_dtype;
@@ -66,14 +69,21 @@ typedef enum { CP_MASK_NONE = 0, CP_MASK_CAUSAL = 1 } cp_mask_mode;
  *   STRIPED   : rank i holds positions i, i+N, i+2N, ... (token p on rank p mod N) */
 typedef enum { CP_LAYOUT_CONTIGUOUS = 0, CP_LAYOUT_ZIGZAG = 1, CP_LAYOUT_STRIPED = 2 } cp_layout;
 
-/* How cp_ring_attn_fwd runs the N steps:
- *   FUSED   : one launch; each CTA owns a 128-row query tile of one rank and walks
- *             the ring steps in order, keeping each step's partial (o_b, lse_b) and
- *             the running (o, lse) on chip and merging them with the LSE formula.
- *   STEPWISE: N launches of the block kernel (all ranks per launch) writing
- *             (o_b, lse_b) to the workspace, each followed by a standalone merge
- *             launch; the last merge writes the output.  Needs a workspace. */
-typedef enum { CP_RING_FUSED = 0, CP_RING_STEPWISE = 1 } cp_ring_mode;
+/* How cp_ring_attn_fwd runs the N steps (section Ring Attention):
+ *   FUSED        : one launch; each CTA owns two 128-row query tiles of one rank and
+ *                  walks the ring steps in order, keeping each step's partial
+ *                  (o_b, lse_b) and the running (o, lse) on chip and merging them
+ *                  with the LSE formula.
+ *   STEPWISE     : the page's loop as written: N launches of the block kernel (all
+ *                  ranks per launch) writing (o_b, lse_b) to the workspace, each
+ *                  followed by a standalone merge launch; the last merge writes the
+ *                  output.  Needs a workspace.
+ *   STEPWISE_EPI : N launches of the block kernel, one ring step each; from step 1
+ *                  on the block kernel merges its partial into the running fp32
+ *                  (o, lse) in its epilogue (no o_b in memory, no merge launch); the
+ *                  last step writes o in the output dtype.  Needs a workspace for a
+ *                  bf16 output (the fp32 running o), none for fp32. */
+typedef enum { CP_RING_FUSED = 0, CP_RING_STEPWISE = 1, CP_RING_STEPWISE_EPI = 2 } cp_ring_mode;
 
 /* A strided 4-D view.  Token tensors: [b, s, H, d]; lse tensors: [b, H, s, 1]
  * (shape[3] = 1).  dtype is a cp_dtype.  Strides in elements; stride[3] must be 1. */
@@ -103,7 +113,9 @@ typedef struct {
  *     Hq % Hkv == 0, query head h reads KV head h / (Hq/Hkv); d in {64, 128}.
  *   q_range / kv_range: original positions of the sq query / sk key rows
  *     (len[0] + len[1] must equal sq / sk).  Used only when mask_mode is causal.
- *   softmax_scale: multiplies q.k (1/sqrt(d) for standard attention); > 0.
+ *   softmax_scale: multiplies q.k; 0 selects the standard 1/sqrt(d) (section
+ *     分块注意力: x_j = q.k_j / sqrt(d_h)), any other value must be finite and > 0.
+ *     The same holds for every entry point below that takes softmax_scale.
  *   accumulate == 0: writes o_b into o ([b, sq, Hq, d], dtype = q's dtype or
  *     CP_FP32) and lse_b into lse ([b, Hq, sq, 1] fp32).  Rows that see no key get
  *     o = 0, lse = -inf.
@@ -141,8 +153,12 @@ cp_status cp_ring_attn_fwd(int32_t layout, int32_t N, int32_t causal, const cp_t
                            cp_tensor *o, cp_tensor *lse, int32_t mode, void *workspace,
                            size_t workspace_bytes, void *stream);
 
-/* Workspace bytes cp_ring_attn_fwd needs for this problem (0 for CP_RING_FUSED).
- * Returns 0 as well for invalid arguments (cp_ring_attn_fwd then reports them). */
+/* Workspace bytes cp_ring_attn_fwd needs for this problem (section Ring Attention:
+ * the running (o, lse) the loop keeps and, in the stepwise loop, each step's
+ * partial (o_b, lse_b)): 0 for CP_RING_FUSED; the fp32 running o for
+ * CP_RING_STEPWISE_EPI with bf16 (0 with fp32); the fp32 running o, o_b in dtype
+ * and lse_b fp32 for CP_RING_STEPWISE.  Returns 0 as well for invalid arguments
+ * (cp_ring_attn_fwd then reports them). */
 size_t cp_ring_workspace_bytes(int32_t layout, int32_t N, int32_t mode, int32_t dtype, int64_t b,
                                int64_t S, int64_t Hq, int64_t d);
 
@@ -325,15 +341,18 @@ cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_t
  *   shares are added to (the caller zeroes them once).
  *   workspace: cp_block_bwd_workspace_bytes(b, sq, Hq) bytes, 256-byte aligned (the
  *   rows' lse and D).
- * Runs the FFMA backward kernels (fp32 arithmetic).  Rows whose lse is -inf add
- * nothing.  Argument errors return synchronously. */
+ * bf16 with d = 128 runs the tensor-core backward kernel (P and dS rounded to bf16
+ * for the tensor cores, fp32 accumulation; dK, dV added in its epilogue, dQ added
+ * with fp32 atomic reductions, so dq_acc's rounding can vary from run to run);
+ * fp32 and bf16 with d = 64 run the FFMA backward kernels (fp32 arithmetic).  Rows
+ * whose lse is -inf add nothing.  Argument errors return synchronously. */
 cp_status cp_block_attn_bwd(const cp_tensor *q, const cp_tensor *k, const cp_tensor *v,
                             const cp_tensor *o, const cp_tensor *lse, const cp_tensor *dout,
                             const cp_range *q_range, const cp_range *kv_range, int32_t mask_mode,
                             float softmax_scale, cp_tensor *dq_acc, cp_tensor *dk_acc, cp_tensor *dv_acc,
                             void *workspace, size_t workspace_bytes, void *stream);
 
-/* Workspace bytes cp_block_attn_bwd needs. */
+/* Workspace bytes cp_block_attn_bwd needs (the (lse, D) table, rows padded to 64). */
 size_t cp_block_bwd_workspace_bytes(int64_t b, int64_t sq, int64_t Hq);
 
 /* Workspace bytes cp_ring_attn_bwd needs (0 for invalid arguments). */
@@ -350,10 +369,16 @@ size_t cp_ring_bwd_workspace_bytes(int32_t layout, int32_t N, int32_t dtype, int
 cp_status cp_layout_permute(int32_t layout, int32_t N, int32_t seq_axis, const cp_tensor *x,
                             cp_tensor *x_ranked, int32_t inverse, void *stream);
 
-/* Host only: the cp_range of rank `rank` for a sequence of S tokens. */
+/* Host only: the cp_range of rank `rank` for a sequence of S tokens split over N
+ * ranks in `layout` (sections 因果掩码带来的负载不均 for the contiguous split, Zig-zag
+ * for 2N chunks with rank i holding chunks i and 2N-1-i, Striped for token p on rank
+ * p mod N).  Requires S % N == 0 (S % 2N == 0 for zig-zag) and 0 <= rank < N. */
 cp_status cp_layout_range(int32_t layout, int32_t N, int64_t S, int32_t rank, cp_range *out);
 
-/* Host only: the tile classes the kernels use for a (query block, key block) pair.
+/* Host only: the tile classes the kernels use for a (query block, key block) pair
+ * (caption of the ring figure in section Ring Attention: blocks the causal mask
+ * hides completely are skipped whole; section Zig-zag: the steps j != i of the
+ * zig-zag layout are unmasked rectangles).
  * out[qt * n_kt + kt] = 0 (skip: no visible pair), 1 (full: every pair visible),
  * 2 (partial: masked element by element), for tiles of tile_q x tile_k local
  * rows; n_qt = ceil(q_len / tile_q), n_kt = ceil(kv_len / tile_k).  Rows past
@@ -363,8 +388,9 @@ cp_status cp_tile_classes(const cp_range *q_range, int64_t q_len, const cp_range
                           int8_t *out);
 
 /* Synchronises `stream`, then reports (and clears) the device status word of the
- * current device: CP_ERR_TIMEOUT if a kernel's bounded wait expired since the last
- * check, CP_ERR_CUDA if the stream reported an error, else CP_OK. */
+ * current device: CP_ERR_BOUNDS if a bounds check of the debug build failed,
+ * CP_ERR_TIMEOUT if a kernel's bounded wait expired since the last check,
+ * CP_ERR_CUDA if the stream reported an error, else CP_OK. */
 cp_status cp_stream_check(void *stream);
 
 /* Failure-detection self-test: launches on `stream` a one-warp kernel that waits on
@@ -402,7 +428,10 @@ int32_t cp_abi_version(void);
  *   All calls on a device share the array and it keeps the last call's contents
  *   (the ring writes everything it reads, so nothing needs clearing); calls whose
  *   work overlaps on the GPU race on it.  The first call on each device looks up
- *   the array's device address; make that first call before any stream capture. */
+ *   the array's device address; make that first call before any stream capture.
+ *   The address is kept for the life of the process: after a reset of the device
+ *   (cudaDeviceReset) the array is gone and this entry point must not be called on
+ *   that device again. */
 cp_status cp_ring_attn_fwd_static_scratch(int32_t layout, int32_t N, int32_t causal, const cp_tensor *q,
                                           const cp_tensor *k, const cp_tensor *v, float softmax_scale,
                                           cp_tensor *o, cp_tensor *lse, void *stream);

@@ -38,9 +38,19 @@ def test_every_declared_symbol_is_exported(cp):
     assert cp.lib().cp_abi_version() == 1
 
 
+def test_debug_library_exports_the_same_symbols(cp):
+    """The bounds-checking build (libcpattn_debug.so) is the same ABI."""
+    from context_attention_cp_b200 import build
+    path = build.build(debug_bounds=True)
+    handle = ctypes.CDLL(path)
+    for n in _declared_symbols():
+        assert hasattr(handle, n), n
+
+
 def test_status_strings(cp):
-    for code in range(6):
+    for code in range(7):
         assert cp.lib().cp_status_string(code)
+    assert b"bounds" in cp.lib().cp_status_string(6)
     assert cp.lib().cp_status_string(99) == b"unknown status"
 
 

@@ -80,3 +80,61 @@ def test_reference_arm_line_on_rank_zero(monkeypatch, capsys):
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def _dist_worker(rank, world, port, out):
+    """bench.run_dist on gloo ranks with the oracle as the block and merge steps."""
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK="0")
+    import contextlib
+    import io
+
+    import numpy as np
+    import torch
+
+    import bench
+    import oracle
+    from test_ring_dist import _oracle_merge, _positions
+
+    def step(qq, kk, vv, q_range, kv_range, causal, scale, o, lse, accumulate):
+        scale = scale or qq.shape[-1] ** -0.5
+        ob, lb = oracle.attention(qq.double().numpy(), kk.double().numpy(), vv.double().numpy(), causal, scale,
+                                  pos_q=_positions(q_range), pos_k=_positions(kv_range), nthreads=1)
+        if accumulate:
+            om, lm = oracle.lse_merge(o.double().numpy().transpose(0, 2, 1, 3), lse.double().numpy(),
+                                      ob.transpose(0, 2, 1, 3), lb)
+            ob, lb = om.transpose(0, 2, 1, 3), lm
+        o.copy_(torch.from_numpy(np.ascontiguousarray(ob)))
+        lse.copy_(torch.from_numpy(np.ascontiguousarray(lb)))
+
+    class A:
+        workload = "fp32_s256_contig2"
+        warmup = 3
+        steps = 2
+
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        rc = bench.run_dist(A(), ring_kw={"compute": step, "merge": _oracle_merge}, device=torch.device("cpu"),
+                            backend="gloo")
+    out[rank] = (rc, buf.getvalue())
+
+
+def test_run_dist_line_over_two_gloo_ranks():
+    """The --gpus N path of bench.py: every rank runs the real-rank ring on its block,
+    the time is the max over ranks, and rank 0 alone prints one JSON line with the
+    whole workload's throughput (strong scaling)."""
+    import json
+    port = 29550 + os.getpid() % 400
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_dist_worker, args=(2, port, out), nprocs=2, start_method="spawn", join=True)
+    assert out[0][0] == 0 and out[1][0] == 0
+    assert out[1][1].strip() == ""
+    lines = [ln for ln in out[0][1].splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["scaling"] == "strong" and d["value"] > 0
+    assert d["config"]["workload"] == "fp32_s256_contig2" and d["config"]["N"] == 2
+    assert d["e2e"]["h2d_bytes_per_step"] > 0 and d["e2e"]["value"] > 0

@@ -188,7 +188,7 @@ RING_CASES = [
 ]
 
 
-@pytest.mark.parametrize("mode", ["fused", "stepwise"])
+@pytest.mark.parametrize("mode", ["fused", "stepwise", "stepwise_epi"])
 @pytest.mark.parametrize("case", RING_CASES, ids=lambda c: "-".join(map(str, c)))
 def test_ring_matches_oracle(cp, case, mode):
     layout, N, S, causal, hq, hkv, d, dt = case
@@ -204,7 +204,7 @@ def test_fp32_workload_full(cp):
     """The fp32 S=256 contiguous N=2 workload, every output element."""
     w = W.BY_NAME["fp32_s256_contig2"]
     q, k, v = W.make_inputs(w)
-    for mode in ("fused", "stepwise"):
+    for mode in ("fused", "stepwise", "stepwise_epi"):
         o, lse = _ring_on_gpu(cp, q, k, v, w.layout, w.N, w.causal, mode)
         ro, rl = oracle.ring_attention(np64(q), np64(k), np64(v), w.layout, w.N, w.causal, w.scale)
         assert_close_lse(np64(lse), rl, 1e-5, mode)

@@ -24,6 +24,16 @@ def _positions(rng_tuple):
     return np.array(out, dtype=np.int64)
 
 
+def _oracle_merge(o_acc, lse_acc, o_b, lse_b, o_out):
+    """The last step's merge of the driver, done by the oracle: (o_acc, lse_acc) and
+    (o_b, lse_b) merged, o written to o_out, lse_acc updated."""
+    import oracle
+    om, lm = oracle.lse_merge(o_acc.numpy().transpose(0, 2, 1, 3), lse_acc.numpy(),
+                              o_b.numpy().transpose(0, 2, 1, 3), lse_b.numpy())
+    o_out.copy_(torch.from_numpy(np.ascontiguousarray(om.transpose(0, 2, 1, 3))))
+    lse_acc.copy_(torch.from_numpy(np.ascontiguousarray(lm)))
+
+
 def _worker(rank, world, port, layout, S, out):
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -54,7 +64,8 @@ def _worker(rank, world, port, layout, S, out):
             o.copy_(torch.from_numpy(np.ascontiguousarray(ob)))
             lse.copy_(torch.from_numpy(np.ascontiguousarray(lb)))
 
-        o, lse = ring_dist.ring_attn_fwd_dist(ql, kl, vl, layout, True, 0.35, compute=oracle_step)
+        o, lse = ring_dist.ring_attn_fwd_dist(ql, kl, vl, layout, True, 0.35, compute=oracle_step,
+                                              merge=_oracle_merge)
         want_o, want_l = oracle.ring_attention(q, k, v, layout, world, True, 0.35, nthreads=1)
         out[rank] = (float(np.max(np.abs(o.numpy() - want_o[:, pos]))),
                      float(np.max(np.abs(lse.numpy() - want_l[:, :, pos]))),
@@ -179,7 +190,7 @@ def _group_worker(rank, world, port, out):
                 dv += torch.from_numpy(bv)
 
             o, lse = ring_dist.ring_attn_fwd_dist(loc(q), loc(k), loc(v), layout, True, 0.5, group=sub,
-                                                  compute=fwd_step)
+                                                  compute=fwd_step, merge=_oracle_merge)
             grads = ring_dist.ring_attn_bwd_dist(loc(q), loc(k), loc(v), o, lse, loc(do), layout, True, 0.5,
                                                  group=sub, compute=bwd_step)
             wo, wl = oracle.attention(q, k, v, True, 0.5, nthreads=1)
