@@ -90,7 +90,7 @@ constexpr int kTurn0 = 2, kTurn1 = 3;
 // Persistent grids (one CTA per SM walking the work items) for the document-mask
 // instantiation and for the ring's.
 #ifndef CP_ATTN_DOC_PERSIST
-#define CP_ATTN_DOC_PERSIST 1
+#define CP_ATTN_DOC_PERSIST 0
 #endif
 #ifndef CP_ATTN_RING_PERSIST
 #define CP_ATTN_RING_PERSIST 0
@@ -170,7 +170,6 @@ __device__ __forceinline__ int first_tile_from(const Range32 &k, int kv_len, int
 // local index, so both are runs of whole tiles).
 template <bool DOC>
 struct TileSeq {
-    const AttnParams *p;
     Range32 qr;
     int rank;
     int q_lo0;
@@ -184,7 +183,6 @@ struct TileSeq {
 
     __device__ void init(const AttnParams &pp, const Range32 &q, int rk, int qlo0)
     {
-        p = &pp;
         qr = q;
         rank = rk;
         q_lo0 = qlo0;
@@ -216,27 +214,27 @@ struct TileSeq {
         if (q_ok1 && kt < kt_beg1 && kt_beg1 < kt_end1 && kt_beg1 < nk) nk = kt_beg1;
         kt = nk;
     }
-    __device__ bool next()
+    __device__ bool next(const AttnParams &p)
     {
         ++kt;
         skip_gap();
         while (kt >= kt_end_all) {
             ++step;
-            if (step >= p->step_end) return false;
-            const int N = p->n_ranks;
+            if (step >= p.step_end) return false;
+            const int N = p.n_ranks;
             src = ((rank - step) % N + N) % N;
-            kr = (p->use_layout && !p->kv_explicit) ? layout_range_t<int>(p->layout, N, (int)p->seq_len, src)
-                                                    : to_range32(p->kv_range);
-            kv_tile_bounds<int>(qr, p->q_len, q_lo0, BM, kr, p->kv_len, BN, p->causal != 0, &kt_full0, &kt_end0);
+            kr = (p.use_layout && !p.kv_explicit) ? layout_range_t<int>(p.layout, N, (int)p.seq_len, src)
+                                                    : to_range32(p.kv_range);
+            kv_tile_bounds<int>(qr, p.q_len, q_lo0, BM, kr, p.kv_len, BN, p.causal != 0, &kt_full0, &kt_end0);
             kt_full1 = kt_end1 = 0;
             if (q_ok1)
-                kv_tile_bounds<int>(qr, p->q_len, q_lo0 + BM, BM, kr, p->kv_len, BN, p->causal != 0, &kt_full1,
+                kv_tile_bounds<int>(qr, p.q_len, q_lo0 + BM, BM, kr, p.kv_len, BN, p.causal != 0, &kt_full1,
                                         &kt_end1);
             if (DOC) {
-                kt_beg0 = first_tile_from(kr, p->kv_len, BN - 1, ds_min0);
-                kt_fb0 = first_tile_from(kr, p->kv_len, 0, ds_max0);
-                kt_beg1 = q_ok1 ? first_tile_from(kr, p->kv_len, BN - 1, ds_min1) : kt_end1;
-                kt_fb1 = q_ok1 ? first_tile_from(kr, p->kv_len, 0, ds_max1) : kt_end1;
+                kt_beg0 = first_tile_from(kr, p.kv_len, BN - 1, ds_min0);
+                kt_fb0 = first_tile_from(kr, p.kv_len, 0, ds_max0);
+                kt_beg1 = q_ok1 ? first_tile_from(kr, p.kv_len, BN - 1, ds_min1) : kt_end1;
+                kt_fb1 = q_ok1 ? first_tile_from(kr, p.kv_len, 0, ds_max1) : kt_end1;
                 kt_beg_all = kt_beg0 < kt_beg1 ? kt_beg0 : kt_beg1;
             }
             kt_end_all = kt_end0 > kt_end1 ? kt_end0 : kt_end1;
@@ -386,7 +384,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 seq.init(p, it.qr, it.rank, it.q_lo0);
                 const int q_row = (int)(it.rank * p.q_row_step) + it.q_lo0;
                 bool first = true;
-                while (seq.next()) {
+                while (seq.next(p)) {
                     if (first) {
                         // the previous item's S products have read its Q
                         if (!mbar_wait(bar(C::B_QE), (qi & 1) ^ 1, w)) { stop = true; break; }
@@ -464,7 +462,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const Item it = decode(item);
                 TileSeq<DOC> seq;
                 seq.init(p, it.qr, it.rank, it.q_lo0);
-                bool have = seq.next();
+                bool have = seq.next(p);
                 if (!have) {
                     if (!PERSIST) break;
                     continue;
@@ -478,7 +476,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 bool pv0 = false, pv1 = false;  // query tile j has a PV product in this item
                 while (have && ok) {
                     const bool need_n0 = seq.need(0), need_n1 = seq.need(1);
-                    const bool have_next = seq.next();  // seq now describes tile n + 1
+                    const bool have_next = seq.next(p);  // seq now describes tile n + 1
                     if (!have_next) tc_commit(bar(C::B_QE));  // the item's last S products are issued
                     const int sv = n % NSV;
                     if (!mbar_wait(bar(C::B_VF + sv), (n / NSV) & 1, w)) { ok = false; break; }
@@ -560,7 +558,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int cs = 0;           // S tiles of this query tile consumed, over all work items
         bool aborted = false;
 
-        for (int item = blockIdx.x; item < n_items && !aborted; item += gridDim.x) {
+        // one work item: its tiles' softmax and its epilogue
+        auto run_item = [&](int item) {
         const Item it = decode(item);
         const int rank = it.rank, h = it.h, bb = it.bb, q_lo0 = it.q_lo0;
         const Range32 qr = it.qr;
@@ -583,7 +582,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // warpgroup that gave up (bounded wait expired) keeps taking its turns
         // without work, so the hand-overs always pair up.
         int nseq = 0;
-        while (seq.next()) {
+        while (seq.next(p)) {
             bool mine = seq.need(j) && !aborted;
             if (mine) {
                 const bool okw = mbar_wait(bar(C::B_SF + j), cs & 1, w);
@@ -806,14 +805,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (row_ok && !empty) *lse_ptr = new_lse * kLn2;
             }
         }
-        if (!PERSIST) break;
-        if (!aborted && c > 0) {
+        if (PERSIST && !aborted && c > 0) {
             // O of this tile is read out: the next item's first PV may overwrite it
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::B_OF + j));
         }
-        }  // work items
+        };
+        if (PERSIST) {
+            for (int item = blockIdx.x; item < n_items && !aborted; item += gridDim.x) run_item(item);
+        } else {
+            run_item(blockIdx.x);
+        }
         teardown();
     }
 }

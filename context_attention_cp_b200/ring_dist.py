@@ -80,13 +80,16 @@ def ring_attn_fwd_dist(q, k, v, layout, causal, scale=None, group=None, compute=
         compute(q, k, v, q_range, q_range, causal, scale, out, lse, False)
         return out, lse
     o = torch.empty((b, c, Hq, d), dtype=torch.float32, device=q.device)
+    # the caller's k, v are only read (step 0); received blocks alternate between two
+    # buffers of the driver's own
     cur_k, cur_v = k.contiguous(), v.contiguous()
-    buf_k, buf_v = torch.empty_like(cur_k), torch.empty_like(cur_v)
+    bufs = [(torch.empty_like(cur_k), torch.empty_like(cur_v)) for _ in range(min(2, N - 1))]
     for r in range(N):
         _nvtx_push(q, "ring step %d of %d" % (r, N))
         src = (rank - r) % N                      # the block this rank holds at step r
         reqs = []
         if r + 1 < N:                             # pass the block on, take the next one
+            buf_k, buf_v = bufs[r % 2]
             ops = [dist.P2POp(dist.isend, cur_k, to_global(nxt), group),
                    dist.P2POp(dist.isend, cur_v, to_global(nxt), group),
                    dist.P2POp(dist.irecv, buf_k, to_global(prv), group),
@@ -103,8 +106,7 @@ def ring_attn_fwd_dist(q, k, v, layout, causal, scale=None, group=None, compute=
         for req in reqs:
             req.wait()
         if r + 1 < N:
-            cur_k, buf_k = buf_k, cur_k
-            cur_v, buf_v = buf_v, cur_v
+            cur_k, cur_v = buf_k, buf_v
         _nvtx_pop(q)
     return out, lse
 
@@ -139,8 +141,10 @@ def ring_attn_bwd_dist(q, k, v, o, lse, do, layout, causal, scale=None, group=No
         return dist.batch_isend_irecv(ops)
 
     dq = torch.zeros(q.shape, dtype=torch.float32, device=q.device)
+    # the caller's k, v are only read (step 0); received blocks alternate between two
+    # buffers of the driver's own
     cur_k, cur_v = k.contiguous(), v.contiguous()
-    buf_k, buf_v = torch.empty_like(cur_k), torch.empty_like(cur_v)
+    bufs = [(torch.empty_like(cur_k), torch.empty_like(cur_v)) for _ in range(min(2, N - 1))]
     # the travelling accumulators live where the travelling block does
     f32 = dict(dtype=torch.float32, device=k.device)
     cur_dk, cur_dv = torch.zeros(k.shape, **f32), torch.zeros(v.shape, **f32)
@@ -148,6 +152,8 @@ def ring_attn_bwd_dist(q, k, v, o, lse, do, layout, causal, scale=None, group=No
     for r in range(N):
         _nvtx_push(q, "ring backward step %d of %d" % (r, N))
         src = (rank - r) % N                      # the block this rank holds at step r
+        if r + 1 < N:
+            buf_k, buf_v = bufs[r % 2]
         kv_reqs = exchange([cur_k, cur_v], [buf_k, buf_v]) if r + 1 < N else []
         compute(q, cur_k, cur_v, o, lse, do, q_range, B.layout_range(layout, N, S, src), causal, scale, dq,
                 cur_dk, cur_dv)
@@ -159,7 +165,6 @@ def ring_attn_bwd_dist(q, k, v, o, lse, do, layout, causal, scale=None, group=No
             cur_dk, buf_dk = buf_dk, cur_dk
             cur_dv, buf_dv = buf_dv, cur_dv
             if r + 1 < N:
-                cur_k, buf_k = buf_k, cur_k
-                cur_v, buf_v = buf_v, cur_v
+                cur_k, cur_v = buf_k, buf_v
         _nvtx_pop(q)
     return dq.to(q.dtype), cur_dk.to(k.dtype), cur_dv.to(v.dtype)

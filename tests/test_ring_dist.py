@@ -64,8 +64,11 @@ def _worker(rank, world, port, layout, S, out):
             o.copy_(torch.from_numpy(np.ascontiguousarray(ob)))
             lse.copy_(torch.from_numpy(np.ascontiguousarray(lb)))
 
+        k_before, v_before = kl.clone(), vl.clone()
         o, lse = ring_dist.ring_attn_fwd_dist(ql, kl, vl, layout, True, 0.35, compute=oracle_step,
                                               merge=_oracle_merge)
+        # the caller's blocks are read, never written (they feed the backward next)
+        assert torch.equal(kl, k_before) and torch.equal(vl, v_before)
         want_o, want_l = oracle.ring_attention(q, k, v, layout, world, True, 0.35, nthreads=1)
         out[rank] = (float(np.max(np.abs(o.numpy() - want_o[:, pos]))),
                      float(np.max(np.abs(lse.numpy() - want_l[:, :, pos]))),
@@ -123,7 +126,9 @@ def _bwd_worker(rank, world, port, layout, S, causal, out):
             dk += torch.from_numpy(bk)
             dv += torch.from_numpy(bv)
 
+        k_before, v_before = kl.clone(), vl.clone()
         dq, dk, dv = ring_dist.ring_attn_bwd_dist(ql, kl, vl, ol, lsel, dol, layout, causal, 0.35, compute=oracle_step)
+        assert torch.equal(kl, k_before) and torch.equal(vl, v_before)
         want = oracle.attention_bwd(q, k, v, do, causal, 0.35, nthreads=1)[:3]
         errs = [float(np.max(np.abs(g.numpy() - w[:, pos]))) for g, w in zip((dq, dk, dv), want)]
         out[rank] = (errs, seen,
