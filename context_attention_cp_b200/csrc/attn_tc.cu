@@ -96,6 +96,17 @@ constexpr int kTurn0 = 2, kTurn1 = 3;
 #define CP_ATTN_RING_PERSIST 0
 #endif
 constexpr bool kDocPersist = CP_ATTN_DOC_PERSIST != 0;
+// S computed in two halves of 64 keys into a two-slot ring per query tile (1): the
+// next key tile's first half only waits for the PV of this tile's first half, so a
+// softmax warpgroup always has the other half's scores ready; or S whole (0).
+#ifndef CP_ATTN_HALF_S
+#define CP_ATTN_HALF_S 0
+#endif
+constexpr bool kHalfS = CP_ATTN_HALF_S != 0;
+constexpr int NH = kHalfS ? 2 : 1;  // S parts per key tile
+constexpr int HW = BN / NH;         // keys per S part
+static_assert(!(kHalfS && CP_ATTN_SPLIT_P), "split P hand-over applies to whole S only");
+static_assert(!(kHalfS && CP_ATTN_PINGPONG), "turn-taking is written for whole S");
 constexpr bool kRingPersist = CP_ATTN_RING_PERSIST != 0;
 // A turn starts before the S load (0) or after the row max (1: the loads and row
 // maxima of the two tiles overlap, at the cost of more live registers).
@@ -120,11 +131,13 @@ struct Cfg {
         B_KE = B_KF + NSK,
         B_VF = B_KE + NSK,
         B_VE = B_VF + NSV,
-        B_SF = B_VE + NSV,  // per query tile
-        B_PF = B_SF + NQ,   // P of keys [0, 64) of the tile stored (per query tile)
-        B_PH = B_PF + NQ,   // P of keys [64, 128) stored
-        B_PV = B_PH + NQ,
-        B_OF = B_PV + NQ,   // O of query tile j read out by its epilogue (per query tile)
+        B_SF = B_VE + NSV,  // per query tile and S part: index 2 j + part
+        B_PF = B_SF + 2 * NQ,  // P of keys [0, 64) of the tile stored (per query tile)
+        B_PH = B_PF + NQ,   // P stored: whole S, keys [64, 128) with the split hand-over, or S
+                            // part h (index 2 j + h; one barrier per part, so the softmax
+                            // never runs two phases ahead of the MMA warp on one barrier)
+        B_PV = B_PH + 2 * NQ,  // PV of S part h done (index 2 j + h), one barrier per part
+        B_OF = B_PV + 2 * NQ,   // O of query tile j read out by its epilogue (per query tile)
         B_QE = B_OF + NQ,   // Q buffer free: the work item's last S products are done
         B_DONE = B_QE + 1,
         NBAR = B_DONE + 1
@@ -134,7 +147,7 @@ struct Cfg {
     static_assert(SMEM <= 232448, "shared memory per CTA exceeds 227 KB");
     static constexpr int T_O = 256;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false);
+    static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, HW, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
 };
 
@@ -181,7 +194,7 @@ struct TileSeq {
     int src;
     Range32 kr;
 
-    __device__ void init(const AttnParams &pp, const Range32 &q, int rk, int qlo0)
+    __device__ __forceinline__ void init(const AttnParams &pp, const Range32 &q, int rk, int qlo0)
     {
         qr = q;
         rank = rk;
@@ -206,7 +219,7 @@ struct TileSeq {
     // layout) can need two disjoint runs of key tiles; tiles in between, needed by
     // neither, are skipped, so every tile of the sequence has a reader (the K/V stage
     // bookkeeping of the producer and the MMA warp relies on it).
-    __device__ void skip_gap()
+    __device__ __forceinline__ void skip_gap()
     {
         if (!DOC || need(0) || need(1)) return;
         int nk = kt_end_all;
@@ -214,7 +227,7 @@ struct TileSeq {
         if (q_ok1 && kt < kt_beg1 && kt_beg1 < kt_end1 && kt_beg1 < nk) nk = kt_beg1;
         kt = nk;
     }
-    __device__ bool next(const AttnParams &p)
+    __device__ __forceinline__ bool next(const AttnParams &p)
     {
         ++kt;
         skip_gap();
@@ -243,11 +256,11 @@ struct TileSeq {
         }
         return true;
     }
-    __device__ bool need(int j) const
+    __device__ __forceinline__ bool need(int j) const
     {
         return kt < (j ? kt_end1 : kt_end0) && (!DOC || kt >= (j ? kt_beg1 : kt_beg0));
     }
-    __device__ bool partial(int j) const
+    __device__ __forceinline__ bool partial(int j) const
     {
         return kt >= (j ? kt_full1 : kt_full0) || (DOC && kt < (j ? kt_fb1 : kt_fb0));
     }
@@ -332,10 +345,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int i = 0; i < NSK; ++i) { mbar_init(bar(C::B_KF + i), 1); mbar_init(bar(C::B_KE + i), 1); }
         for (int i = 0; i < NSV; ++i) { mbar_init(bar(C::B_VF + i), 1); mbar_init(bar(C::B_VE + i), 1); }
         for (int j = 0; j < NQ; ++j) {
-            mbar_init(bar(C::B_SF + j), 1);
+            mbar_init(bar(C::B_SF + 2 * j), 1);
+            mbar_init(bar(C::B_SF + 2 * j + 1), 1);
             mbar_init(bar(C::B_PF + j), BM / 32);  // one arrival per softmax warp
-            mbar_init(bar(C::B_PH + j), BM / 32);
-            mbar_init(bar(C::B_PV + j), 1);
+            mbar_init(bar(C::B_PH + 2 * j), BM / 32);
+            mbar_init(bar(C::B_PH + 2 * j + 1), BM / 32);
+            mbar_init(bar(C::B_PV + 2 * j), 1);
+            mbar_init(bar(C::B_PV + 2 * j + 1), 1);
             mbar_init(bar(C::B_OF + j), BM / 32);
         }
         mbar_init(bar(C::B_QE), 1);
@@ -444,18 +460,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int oi0 = 0, oi1 = 0;  // work items whose O of query tile j was accumulated
             int n = 0;             // key tiles consumed, over all work items (K/V stages)
             int qi = 0;            // work items that visit key tiles (Q loads)
-            auto issue_s = [&](int j, int m) {
+            // S of query tile j against keys [HW h, HW (h + 1)) of key tile m, into the
+            // tile's S columns for part h
+            auto issue_s = [&](int j, int m, int h) {
                 const int sk = m % NSK;
-                const uint32_t d_tmem = tbase + (uint32_t)(j * 128);
+                const uint32_t d_tmem = tbase + (uint32_t)(j * 128 + h * HW);
                 const uint32_t qa = s_base + C::OFF_Q + j * C::TILE;
-                const uint32_t kb_ = s_base + C::OFF_K + sk * C::TILE;
+                const uint32_t kb_ = s_base + C::OFF_K + sk * C::TILE + (uint32_t)(h * HW * 128);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * C::SUB + (k & 3) * 32;
                     mma_ss(d_tmem, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb_ + off, 16, 1024),
                            C::IDESC_QK, k > 0 ? 1u : 0u);
                 }
-                tc_commit(bar(C::B_SF + j));
+                tc_commit(bar(C::B_SF + 2 * j + h));
             };
             bool ok = true;
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -470,8 +488,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 ok = mbar_wait(bar(C::B_Q), qi & 1, w) && mbar_wait(bar(C::B_KF + n % NSK), (n / NSK) & 1, w);
                 if (!ok) break;
                 tc_fence_after();
-                for (int j = 0; j < NQ; ++j)
-                    if (seq.need(j)) issue_s(j, n);
+                for (int h = 0; h < NH; ++h)
+                    for (int j = 0; j < NQ; ++j)
+                        if (seq.need(j)) issue_s(j, n, h);
                 tc_commit(bar(C::B_KE + n % NSK));
                 bool pv0 = false, pv1 = false;  // query tile j has a PV product in this item
                 while (have && ok) {
@@ -482,12 +501,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!mbar_wait(bar(C::B_VF + sv), (n / NSV) & 1, w)) { ok = false; break; }
                     bool k_ready = false;
 #pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+#pragma unroll
                     for (int j = 0; j < NQ; ++j) {
                         int &pc = j ? pc1 : pc0;
                         bool &pv = j ? pv1 : pv0;
                         const int oi = j ? oi1 : oi0;
                         if (j ? need_n1 : need_n0) {
-                            const uint32_t p_tmem = tbase + (uint32_t)(j * 128);
+                            const uint32_t p_tmem = tbase + (uint32_t)(j * 128 + h * HW);
                             const uint32_t vb = s_base + C::OFF_V + sv * C::TILE;
                             const uint32_t o_tmem = tbase + C::T_O + (uint32_t)(j * D);
                             // the first product of an item overwrites O: the previous item's
@@ -503,13 +524,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                     mma_ts(o_tmem, p_tmem + k * 8, smem_desc_sw128(vb + k * 2048, C::SUB, 1024),
                                            C::IDESC_PV, (k > 0 || pv) ? 1u : 0u);
                             }
-                            if (!mbar_wait(bar(C::B_PH + j), pc & 1, w)) { ok = false; break; }
+                            // part h of every key tile has its own barrier: phase = tiles so far
+                            if (!mbar_wait(bar(C::B_PH + 2 * j + h), (pc / NH) & 1, w)) { ok = false; break; }
                             tc_fence_after();
+                            // keys [HW h, HW (h + 1)) of the tile: P columns from the part's
+                            // first, V rows from 16-key step HW h / 16 on
 #pragma unroll
-                            for (int k = kSplitP ? BN / 32 : 0; k < BN / 16; ++k)
-                                mma_ts(o_tmem, p_tmem + k * 8, smem_desc_sw128(vb + k * 2048, C::SUB, 1024),
-                                       C::IDESC_PV, (k > 0 || pv) ? 1u : 0u);
-                            tc_commit(bar(C::B_PV + j));
+                            for (int k = kSplitP ? BN / 32 : 0; k < HW / 16; ++k)
+                                mma_ts(o_tmem, p_tmem + k * 8,
+                                       smem_desc_sw128(vb + (h * (HW / 16) + k) * 2048, C::SUB, 1024), C::IDESC_PV,
+                                       (k > 0 || pv) ? 1u : 0u);
+                            tc_commit(bar(C::B_PV + 2 * j + h));
                             ++pc;
                             pv = true;
                         }
@@ -522,8 +547,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                 tc_fence_after();
                                 k_ready = true;
                             }
-                            issue_s(j, n + 1);
+                            issue_s(j, n + 1, h);
                         }
+                    }
+                    if (!ok) break;
                     }
                     if (!ok) break;
                     tc_commit(bar(C::B_VE + sv));
@@ -582,10 +609,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // warpgroup that gave up (bounded wait expired) keeps taking its turns
         // without work, so the hand-overs always pair up.
         int nseq = 0;
+        if (!kHalfS) {
         while (seq.next(p)) {
             bool mine = seq.need(j) && !aborted;
             if (mine) {
-                const bool okw = mbar_wait(bar(C::B_SF + j), cs & 1, w);
+                const bool okw = mbar_wait(bar(C::B_SF + 2 * j), cs & 1, w);
                 if (__any_sync(0xffffffffu, !okw)) { aborted = true; mine = false; }
             }
             float s[BN];
@@ -687,7 +715,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tmem_st16(s_tmem + 16 * q4, pk);
                     if (q4 == (kSplitP ? 1 : 3) && rescale) {
                         // O must hold every earlier tile's P V before it is rescaled
-                        const bool okw = mbar_wait(bar(C::B_PV + j), (cs - 1) & 1, w);
+                        const bool okw = mbar_wait(bar(C::B_PV + 2 * j), (cs - 1) & 1, w);
                         okr = !__any_sync(0xffffffffu, !okw);
                         if (okr) {
                             tc_fence_after();
@@ -707,7 +735,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         tmem_wait_st();
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0 && okr) mbar_arrive(bar((kSplitP && q4 == 1) ? C::B_PF + j : C::B_PH + j));
+                        if (lane == 0 && okr) mbar_arrive(bar((kSplitP && q4 == 1) ? C::B_PF + j : C::B_PH + 2 * j));
                     }
                 }
                 float a0, a1, a2, a3;
@@ -725,13 +753,174 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             ++nseq;
         }
+        } else {
+        while (seq.next(p)) {
+            bool mine = seq.need(j) && !aborted;
+            if (kPingPong && !kTurnLate && (j == 1 || nseq > 0)) named_bar_sync(j == 0 ? kTurn0 : kTurn1, 2 * BM);
+            // the tile's S parts (one, or two halves of 64 keys), each: scores out of
+            // TMEM, mask, row max, probabilities and row sum, bf16 P back into TMEM
+#pragma unroll
+            for (int hp = 0; hp < NH; ++hp) {
+            if (mine) {
+                const bool okw = mbar_wait(bar(C::B_SF + 2 * j + hp), cs & 1, w);
+                if (__any_sync(0xffffffffu, !okw)) { aborted = true; mine = false; }
+            }
+            float s[HW];
+            float f_rescale = 1.f, mu = 0.f;
+            bool rescale = false;
+            const uint32_t sp_tmem = s_tmem + (uint32_t)(hp * HW);  // this part's S / P columns
+            if (mine) {
+                tc_fence_after();
+                tmem_ld64f_nowait(sp_tmem, s);
+                if (HW == 128) tmem_ld64f_nowait(sp_tmem + 64, s + (HW == 128 ? 64 : 0));
+                tmem_wait_ld_dep(s);
+                if (HW == 128) reg_dep64(s + (HW == 128 ? 64 : 0));
+                // ---- mask (partial tiles only).  Positions increase with the local key
+                // index, so the keys this row may see form a prefix of the tile.
+                if (seq.partial(j)) {
+                    const int k0 = seq.kt * BN + hp * HW;
+                    int cnt = p.kv_len - k0;
+                    if (cnt > HW) cnt = HW;
+                    if (cnt < 0) cnt = 0;
+                    if (p.causal) {
+                        int lo = 0, hi = cnt;
+                        while (lo < hi) {
+                            const int mid = (lo + hi) >> 1;
+                            if (range_pos(seq.kr, k0 + mid) <= pos_q) lo = mid + 1; else hi = mid;
+                        }
+                        cnt = lo;
+                    }
+                    int beg = 0;  // keys before this row's document start are invisible
+                    if (DOC) {
+                        int lo = 0, hi = cnt;
+                        while (lo < hi) {
+                            const int mid = (lo + hi) >> 1;
+                            if (range_pos(seq.kr, k0 + mid) < ds_row) lo = mid + 1; else hi = mid;
+                        }
+                        beg = lo;
+                    }
+#pragma unroll
+                    for (int cc = 0; cc < HW; ++cc)
+                        if (cc >= cnt || (DOC && cc < beg)) s[cc] = -INFINITY;
+                }
+                // ---- row max: four chains of 3-input max
+                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+                for (int cc = 4; cc < HW - 4; cc += 8) {
+                    mx0 = fmax3(mx0, s[cc], s[cc + 1]);
+                    mx1 = fmax3(mx1, s[cc + 2], s[cc + 3]);
+                    mx2 = fmax3(mx2, s[cc + 4], s[cc + 5]);
+                    mx3 = fmax3(mx3, s[cc + 6], s[cc + 7]);
+                }
+                mx0 = fmax3(mx0, s[HW - 4], s[HW - 3]);
+                mx1 = fmax3(mx1, s[HW - 2], s[HW - 1]);
+                const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
+                // Raise the exponent's max only when it grew by more than the threshold;
+                // then l is rescaled here and O below, before the part's P is handed to
+                // the MMA warp.
+                if (c == 0 && hp == 0) {
+                    m = mx;
+                } else {
+                    const bool need_rescale = mx > m + kRescaleThreshold;
+                    rescale = __any_sync(0xffffffffu, need_rescale);
+                    if (rescale) {
+                        const float m_new = fmaxf(m, mx);
+                        f_rescale = (m_new == m) ? 1.f : ex2_approx(m - m_new);
+                        m = m_new;
+                        l *= f_rescale;
+                    }
+                }
+                mu = (m == -INFINITY) ? 0.f : m;
+            }
+            if (kPingPong && kTurnLate && (j == 1 || nseq > 0)) named_bar_sync(j == 0 ? kTurn0 : kTurn1, 2 * BM);
+            if (mine) {
+                // ---- probabilities, row sum, bf16 P into the part's first HW / 2 TMEM
+                // columns, 32 scores at a time so each chunk's scores die once packed.
+                // The scale-subtract and the row sum run as packed fp32x2 instructions.
+                // With kSplitP (whole S), P is handed to the MMA warp in two halves
+                // (keys [0, 64), then [64, 128)); a rescale of O happens before the
+                // first P of the part is handed over, since PV adds into O.
+                bool okr = true;
+                const uint64_t sl2x2 = f2_pack(sl2, sl2);
+                const uint64_t nmux2 = f2_pack(-mu, -mu);
+                uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = f2_pack(0.f, 0.f);
+                const bool emu = kEmuMod > 0 && !seq.partial(j);
+                constexpr int NC = HW / 32;  // chunks of 32 scores
+#pragma unroll
+                for (int q4 = 0; q4 < NC; ++q4) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float e0, e1;
+                        f2_unpack(f2_fma(f2_pack(s[32 * q4 + 2 * i], s[32 * q4 + 2 * i + 1]), sl2x2, nmux2), e0, e1);
+                        if (kEmuMod > 0 && (i % (kEmuMod > 0 ? kEmuMod : 1)) == kEmuMod - 1 && emu) {
+                            exp2_fma2(e0, e1);
+                        } else {
+                            e0 = ex2_approx(e0);
+                            e1 = ex2_approx(e1);
+                        }
+                        const uint64_t e01 = f2_pack(e0, e1);
+                        if (i & 1) acc1 = f2_add(acc1, e01); else acc0 = f2_add(acc0, e01);
+                        pk[i] = pack_bf16x2(e0, e1);
+                    }
+                    tmem_st16(sp_tmem + 16 * q4, pk);
+                    if (q4 == (kSplitP ? 1 : NC - 1) && rescale) {
+                        // O must hold every earlier part's P V before it is rescaled
+                        // every earlier part's PV: this tile's part 0 (hp = 1), or the
+                        // previous tile's last part (hp = 0; its part 0 finished before this
+                        // tile's S part 0 did)
+                        const bool okw = hp == 1 ? mbar_wait(bar(C::B_PV + 2 * j), cs & 1, w)
+                                                : mbar_wait(bar(C::B_PV + 2 * j + NH - 1), (cs - 1) & 1, w);
+                        okr = !__any_sync(0xffffffffu, !okw);
+                        if (okr) {
+                            tc_fence_after();
+#pragma unroll
+                            for (int c0 = 0; c0 < D; c0 += 32) {
+                                uint32_t r[32];
+                                tmem_ld32(o_tmem + c0, r);
+#pragma unroll
+                                for (int cc = 0; cc < 32; ++cc)
+                                    r[cc] = __float_as_uint(__uint_as_float(r[cc]) * f_rescale);
+                                tmem_st32(o_tmem + c0, r);
+                            }
+                        }
+                    }
+                    if (q4 == NC - 1 && kPingPong) named_bar_arrive(j == 0 ? kTurn1 : kTurn0, 2 * BM);
+                    if ((kSplitP && q4 == 1) || q4 == NC - 1) {
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0 && okr) mbar_arrive(bar((kSplitP && q4 == 1) ? C::B_PF + j : C::B_PH + 2 * j + hp));
+                    }
+                }
+                float a0, a1, a2, a3;
+                f2_unpack(acc0, a0, a1);
+                f2_unpack(acc1, a2, a3);
+                l += (a0 + a1) + (a2 + a3);
+                if (!okr) {
+                    aborted = true;
+                    mine = false;
+                }
+            } else if (kPingPong) {
+                named_bar_arrive(j == 0 ? kTurn1 : kTurn0, 2 * BM);
+            }
+            }  // S parts
+            if (mine) {
+                ++c;
+                ++cs;
+            }
+            ++nseq;
+        }
+        }
         // tile 0 takes the hand-over of tile 1's last turn
         if (kPingPong && j == 0 && nseq > 0) named_bar_sync(kTurn0, 2 * BM);
         aborted = __any_sync(0xffffffffu, aborted || (*abort_flag != 0));
 
         // ================================================================ epilogue
         if (!aborted && c > 0) {
-            const bool okw = mbar_wait(bar(C::B_PV + j), (cs - 1) & 1, w);
+            // the last tile's PV of every part (each part's barrier completes once per tile)
+            bool okw = true;
+            for (int hp = 0; hp < NH; ++hp) okw = okw && mbar_wait(bar(C::B_PV + 2 * j + hp), (cs - 1) & 1, w);
             aborted = __any_sync(0xffffffffu, !okw);
             if (!aborted) tc_fence_after();
         }
