@@ -21,6 +21,14 @@
 
 using namespace cpattn;
 
+// The backward's grid is head-major (the CTAs resident at one time share a few heads'
+// Q, dO and dQ rows in L2) once one head's work items fill a wave of the device, or
+// always with CP_BWD_HEAD_MAJOR=1.
+#ifndef CP_BWD_HEAD_MAJOR
+#define CP_BWD_HEAD_MAJOR 0
+#endif
+constexpr bool kBwdHeadMajor = CP_BWD_HEAD_MAJOR != 0;
+
 namespace {
 
 // NVTX range for profilers (a no-op unless a tool is attached): the entry points and,
@@ -831,12 +839,9 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     // the gather of K and V into original order (as in the forward)
     if ((s = cp_layout_permute(layout, N, 1, &kg, const_cast<cp_tensor *>(k), 1, stream)) != CP_OK) return s;
     if ((s = cp_layout_permute(layout, N, 1, &vg, const_cast<cp_tensor *>(v), 1, stream)) != CP_OK) return s;
-    std::vector<int32_t> docs_h((size_t)n_docs);
-    for (int32_t i = 0; i < n_docs; ++i) docs_h[i] = (int32_t)doc_starts[i];
-    cudaError_t e = cudaMemcpyAsync(docs_dev, docs_h.data(), sizeof(int32_t) * (size_t)n_docs, cudaMemcpyHostToDevice, st);
-    if (e != cudaSuccess) return cuda_fail(e, "document table copy");
-    if (n_docs > 1 && tc_path) {
-        e = launch_doc_tables(docs_dev, n_docs, S, doc_pos_start, doc_pos_end, st);
+    cudaError_t e = cudaSuccess;
+    if (n_docs > 1) {  // device starts for the FFMA kernels, per-position bounds for the tensor-core one
+        e = launch_doc_tables(doc_starts, n_docs, S, docs_dev, doc_pos_start, doc_pos_end, st);
         if (e != cudaSuccess) return cuda_fail(e, "document bounds launch");
     }
 
@@ -931,7 +936,7 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "device query");
-    p.head_major = n_kt >= (int64_t)sms;
+    p.head_major = kBwdHeadMajor || n_kt >= (int64_t)sms;
     e = launch_attn_bwd(p, st);
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     // the reduce-scatter: the summed dK, dV of the gathered block back to each rank
@@ -1127,21 +1132,10 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
     int *docs_dev = reinterpret_cast<int *>(ws + 2 * kv_bytes);
     if ((s = cp_layout_permute(layout, N, 1, &kg, const_cast<cp_tensor *>(k), 1, stream)) != CP_OK) return s;
     if ((s = cp_layout_permute(layout, N, 1, &vg, const_cast<cp_tensor *>(v), 1, stream)) != CP_OK) return s;
-    int32_t docs32[1024];
-    std::vector<int32_t> docs_big;
-    int32_t *docs_h = docs32;
-    if (n_docs > 1024) {
-        docs_big.resize((size_t)n_docs);
-        docs_h = docs_big.data();
-    }
-    for (int32_t i = 0; i < n_docs; ++i) docs_h[i] = (int32_t)doc_starts[i];
-    // pageable source: the copy is staged before the call returns
-    cudaError_t e = cudaMemcpyAsync(docs_dev, docs_h, sizeof(int32_t) * (size_t)n_docs, cudaMemcpyHostToDevice, st);
-    if (e != cudaSuccess) return cuda_fail(e, "document table copy");
     int *doc_pos_start = reinterpret_cast<int *>(ws + 2 * kv_bytes + up((int64_t)n_docs * 4));
     int *doc_pos_end = doc_pos_start + up(S * 4) / 4;
-    if (n_docs > 1 && q->dtype == CP_BF16) {
-        e = launch_doc_tables(docs_dev, n_docs, S, doc_pos_start, doc_pos_end, st);
+    if (n_docs > 1) {  // device starts for the FFMA kernel, per-position bounds for the tensor-core one
+        const cudaError_t e = launch_doc_tables(doc_starts, n_docs, S, docs_dev, doc_pos_start, doc_pos_end, st);
         if (e != cudaSuccess) return cuda_fail(e, "document bounds launch");
     }
 
@@ -1177,10 +1171,8 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
     {
         std::vector<std::pair<int64_t, uint32_t>> work;
         const int n_groups = (int)((c + rows - 1) / rows);
-        auto doc_start = [&](int64_t pos) {
-            int64_t ds = 0;
-            for (int32_t i2 = 0; i2 < n_docs && doc_starts[i2] <= pos; ++i2) ds = doc_starts[i2];
-            return ds;
+        auto doc_start = [&](int64_t pos) {  // the last start <= pos
+            return *(std::upper_bound(doc_starts, doc_starts + n_docs, pos) - 1);
         };
         for (int i2 = 0; i2 < N; ++i2) {
             const Range qr = layout_range(layout, N, S, i2);
@@ -1420,7 +1412,7 @@ cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "device query");
-    p.head_major = (int64_t)N * n_kt >= (int64_t)sms;
+    p.head_major = kBwdHeadMajor || (int64_t)N * n_kt >= (int64_t)sms;
     e = launch_attn_bwd(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return CP_OK;

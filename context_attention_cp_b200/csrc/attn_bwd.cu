@@ -117,27 +117,6 @@ __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap *map, uint32
         "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// Makes this thread's generic-proxy shared-memory writes visible to the async proxy
-// (tensor cores, bulk copies).
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-// OR of `pred` over the `nthreads` threads of named barrier `id` (all must call).
-__device__ __forceinline__ bool bar_any(uint32_t id, uint32_t nthreads, bool pred)
-{
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "barrier.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}\n"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
-        : "memory");
-    return r != 0;
-}
 
 // Query-tile sequence of one CTA: (query head of the group, ring step, query tile)
 // with the tile seeing at least one key of the CTA's key tile.  Every role walks it.
@@ -689,43 +668,74 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 // Per query row: (lse log2 e, D = do . o) into the statistics table (padding rows
 // get (+inf, 0), which makes their probabilities 0), and a zeroed dQ accumulator row.
-// One warp per (batch, head, rank, padded row).
+// Sixteen threads per (batch, head, rank, padded row), each with 16-byte slices of
+// o and dout (8 bf16) and 32 bytes of the accumulator, two rows in flight per thread.
+constexpr int kPreRowsPerThread = 2;
 __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __grid_constant__ BwdParams p, int64_t acc_rows)
 {
-    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
+    constexpr int TPR = HD / 8;  // threads per row
+    const int part = threadIdx.x % TPR;
     const int64_t total = (int64_t)p.b * p.hq * p.n_ranks * p.lpad;
-    if (gw >= total) return;
-    const int t = (int)(gw % p.lpad);
-    int64_t rest = gw / p.lpad;
-    const int i = (int)(rest % p.n_ranks);
-    rest /= p.n_ranks;
-    const int h = (int)(rest % p.hq);
-    const int bb = (int)(rest / p.hq);
-    float2 st = make_float2(INFINITY, 0.f);
-    if (t < p.q_len) {
-        const int64_t row = (int64_t)i * p.q_row_step + t;
-        const uint2 ov = *reinterpret_cast<const uint2 *>(reinterpret_cast<const uint16_t *>(p.o) + bb * p.o_sb +
-                                                          row * p.o_ss + h * p.o_sh + lane * 4);
-        const uint2 gv = *reinterpret_cast<const uint2 *>(reinterpret_cast<const uint16_t *>(p.dout) + bb * p.do_sb +
-                                                          row * p.do_ss + h * p.do_sh + lane * 4);
-        auto lo = [](uint32_t x) { return __uint_as_float(x << 16); };
-        auto hi = [](uint32_t x) { return __uint_as_float(x & 0xffff0000u); };
-        float acc = lo(ov.x) * lo(gv.x);
-        acc = fmaf(hi(ov.x), hi(gv.x), acc);
-        acc = fmaf(lo(ov.y), lo(gv.y), acc);
-        acc = fmaf(hi(ov.y), hi(gv.y), acc);
+    const int64_t row_slot = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / TPR;  // first row of this thread
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x / TPR;
+    auto lo = [](uint32_t x) { return __uint_as_float(x << 16); };
+    auto hi = [](uint32_t x) { return __uint_as_float(x & 0xffff0000u); };
+    for (int64_t g0 = row_slot; g0 < total; g0 += stride * kPreRowsPerThread) {
+        uint4 ov[kPreRowsPerThread], gv[kPreRowsPerThread];
+        int64_t gw[kPreRowsPerThread], qrow[kPreRowsPerThread];
+        int hh[kPreRowsPerThread], bq[kPreRowsPerThread];
+        bool live[kPreRowsPerThread];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        const float lse = p.lse[bb * p.lse_sb + h * p.lse_sh + row * p.lse_ss];
-        st.x = (lse == -INFINITY) ? INFINITY : lse * kLog2eB;
-        st.y = acc;
-        if (!p.accumulate) {  // the block form adds into the caller's accumulator instead
-            float4 *dq = reinterpret_cast<float4 *>(p.dq_acc + (((int64_t)bb * acc_rows + row) * p.hq + h) * HD) + lane;
-            *dq = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < kPreRowsPerThread; ++u) {
+            gw[u] = g0 + u * stride;
+            const int64_t g = gw[u] < total ? gw[u] : total - 1;
+            const int t = (int)(g % p.lpad);
+            int64_t rest = g / p.lpad;
+            const int i = (int)(rest % p.n_ranks);
+            rest /= p.n_ranks;
+            hh[u] = (int)(rest % p.hq);
+            bq[u] = (int)(rest / p.hq);
+            live[u] = gw[u] < total && t < p.q_len;
+            qrow[u] = (int64_t)i * p.q_row_step + t;
+            if (live[u]) {
+                ov[u] = *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(p.o) + bq[u] * p.o_sb +
+                                                         qrow[u] * p.o_ss + hh[u] * p.o_sh + part * 8);
+                gv[u] = *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(p.dout) + bq[u] * p.do_sb +
+                                                         qrow[u] * p.do_ss + hh[u] * p.do_sh + part * 8);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kPreRowsPerThread; ++u) {
+            float acc = 0.f;
+            if (live[u]) {
+                acc = lo(ov[u].x) * lo(gv[u].x);
+                acc = fmaf(hi(ov[u].x), hi(gv[u].x), acc);
+                acc = fmaf(lo(ov[u].y), lo(gv[u].y), acc);
+                acc = fmaf(hi(ov[u].y), hi(gv[u].y), acc);
+                acc = fmaf(lo(ov[u].z), lo(gv[u].z), acc);
+                acc = fmaf(hi(ov[u].z), hi(gv[u].z), acc);
+                acc = fmaf(lo(ov[u].w), lo(gv[u].w), acc);
+                acc = fmaf(hi(ov[u].w), hi(gv[u].w), acc);
+            }
+            // the TPR threads of a row are consecutive lanes of one warp
+#pragma unroll
+            for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, TPR);
+            if (gw[u] >= total) continue;
+            float2 st = make_float2(INFINITY, 0.f);
+            if (live[u]) {
+                const float lse = p.lse[bq[u] * p.lse_sb + hh[u] * p.lse_sh + qrow[u] * p.lse_ss];
+                st.x = (lse == -INFINITY) ? INFINITY : lse * kLog2eB;
+                st.y = acc;
+                if (!p.accumulate) {  // the block form adds into the caller's accumulator instead
+                    float4 *dq = reinterpret_cast<float4 *>(p.dq_acc + (((int64_t)bq[u] * acc_rows + qrow[u]) * p.hq + hh[u]) * HD) +
+                                 part * 2;
+                    dq[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    dq[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            if (part == 0) p.stats[gw[u]] = st;
         }
     }
-    if (lane == 0) p.stats[gw] = st;
 }
 
 // dq = dq_acc (already scaled) in bf16; 8 values per thread.
@@ -814,9 +824,14 @@ cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream)
         cudaError_t e = set_smem_per_device((const void *)attn_bwd_kernel, BCfg::SMEM, &attr_done);
         if (e != cudaSuccess) return e;
     }
-    const int64_t warps = (int64_t)p.b * p.hq * p.n_ranks * p.lpad;
-    if (warps == 0) return cudaSuccess;
-    attn_bwd_pre_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, stream>>>(p, q_rows);
+    const int64_t rows = (int64_t)p.b * p.hq * p.n_ranks * p.lpad;
+    if (rows == 0) return cudaSuccess;
+    {
+        // 16 threads per row, two rows each; at most 8 resident CTAs of 256 threads per SM
+        const int64_t want = (rows * (HD / 8) / kPreRowsPerThread + 255) / 256;
+        const int64_t cap = (int64_t)sm_count() * 8;
+        attn_bwd_pre_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, stream>>>(p, q_rows);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int64_t items = (int64_t)(p.order_len ? p.order_len : p.n_kv_blocks * p.n_kt) * p.b * p.hkv;

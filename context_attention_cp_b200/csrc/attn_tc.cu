@@ -114,6 +114,28 @@ constexpr bool kRingPersist = CP_ATTN_RING_PERSIST != 0;
 #define CP_ATTN_TURN_LATE 0
 #endif
 constexpr bool kTurnLate = CP_ATTN_TURN_LATE != 0;
+// One-item CTAs (the grid covers every work item):
+//   CP_ATTN_EARLY_Q   the producer starts the Q load right after the barrier set-up,
+//                     before the tile walk is worked out;
+//   CP_ATTN_PREFETCH_Q the item one wave later gets its Q prefetched into L2;
+//   CP_ATTN_STAGGER   query tile 1 starts its first key tile after tile 0's first P;
+//   CP_ATTN_TMA_O     bf16 output tiles leave through shared memory and a TMA store.
+#ifndef CP_ATTN_EARLY_Q
+#define CP_ATTN_EARLY_Q 1
+#endif
+#ifndef CP_ATTN_PREFETCH_Q
+#define CP_ATTN_PREFETCH_Q 1
+#endif
+#ifndef CP_ATTN_STAGGER
+#define CP_ATTN_STAGGER 1
+#endif
+#ifndef CP_ATTN_TMA_O
+#define CP_ATTN_TMA_O 1
+#endif
+constexpr bool kEarlyQ = CP_ATTN_EARLY_Q != 0;
+constexpr bool kPrefetchQ = CP_ATTN_PREFETCH_Q != 0;
+constexpr bool kStagger = CP_ATTN_STAGGER != 0;
+constexpr bool kTmaO = CP_ATTN_TMA_O != 0;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
@@ -139,7 +161,8 @@ struct Cfg {
         B_PV = B_PH + 2 * NQ,  // PV of S part h done (index 2 j + h), one barrier per part
         B_OF = B_PV + 2 * NQ,   // O of query tile j read out by its epilogue (per query tile)
         B_QE = B_OF + NQ,   // Q buffer free: the work item's last S products are done
-        B_DONE = B_QE + 1,
+        B_STAG = B_QE + 1,  // query tile 0's first P is stored (tile 1 starts after it)
+        B_DONE = B_STAG + 1,
         NBAR = B_DONE + 1
     };
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -290,7 +313,8 @@ __device__ __forceinline__ void store_row_chunk(void *o, int dtype, int64_t off,
 template <int D, bool DOC, bool PERSIST>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tm_q,
-                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v)
+                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_o, int o_tma, int next_stride)
 {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -339,8 +363,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     (void)q_rows_all;
     (void)kv_rows_all;
 
-    // ---- setup: barriers, TMEM
-    if (tid == 0) {
+    // Q tiles of an item into the Q buffer (both tiles when the second holds rows)
+    auto issue_q = [&](const Item &it) {
+        const int q_row = (int)(it.rank * p.q_row_step) + it.q_lo0;
+        const int nq = it.q_lo0 + BM < p.q_len ? 2 : 1;
+        mbar_expect_tx(bar(C::B_Q), nq * C::TILE);
+        for (int j = 0; j < nq; ++j)
+            for (int kb = 0; kb < D / 64; ++kb)
+                if (bounds_ok(q_row + j * BM >= 0 && q_row + j * BM < q_rows_all && it.h < p.hq && it.bb < p.b,
+                              p.status, 101))
+                    tma_load_4d(s_base + C::OFF_Q + j * C::TILE + kb * C::SUB, &tm_q, bar(C::B_Q), kb * 64, it.h,
+                                q_row + j * BM, it.bb);
+    };
+
+    // ---- setup: barriers (by the producer thread, which then starts the Q load of a
+    // one-item CTA at once, before the tile walk is worked out), TMEM
+    if (warp == WARP_LOAD && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
         mbar_init(bar(C::B_Q), 1);
         for (int i = 0; i < NSK; ++i) { mbar_init(bar(C::B_KF + i), 1); mbar_init(bar(C::B_KE + i), 1); }
         for (int i = 0; i < NSV; ++i) { mbar_init(bar(C::B_VF + i), 1); mbar_init(bar(C::B_VE + i), 1); }
@@ -355,9 +396,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(bar(C::B_OF + j), BM / 32);
         }
         mbar_init(bar(C::B_QE), 1);
+        mbar_init(bar(C::B_STAG), BM / 32);
         mbar_init(bar(C::B_DONE), 1);
         *abort_flag = 0;
         mbar_fence_init();
+        if (!PERSIST && kEarlyQ) issue_q(decode(blockIdx.x));
     }
     if (warp == WARP_MMA) {
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -387,32 +430,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp == WARP_LOAD) {
         // ================================================================ producer
         if (lane == 0) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
             WaitCtx w{abort_flag, p.status, 1};
             int n = 0;   // K/V tiles loaded, over all work items
-            int qi = 0;  // work items that visit key tiles (each loads its Q once)
+            int qi = (PERSIST || !kEarlyQ) ? 0 : 1;  // Q loads issued (early: at set-up)
             bool stop = false;
             for (int item = blockIdx.x; item < n_items && !stop; item += gridDim.x) {
                 const Item it = decode(item);
                 TileSeq<DOC> seq;
                 seq.init(p, it.qr, it.rank, it.q_lo0);
-                const int q_row = (int)(it.rank * p.q_row_step) + it.q_lo0;
-                bool first = true;
+                bool first = PERSIST || !kEarlyQ;
                 while (seq.next(p)) {
                     if (first) {
                         // the previous item's S products have read its Q
                         if (!mbar_wait(bar(C::B_QE), (qi & 1) ^ 1, w)) { stop = true; break; }
-                        const int nq = seq.q_ok1 ? 2 : 1;
-                        mbar_expect_tx(bar(C::B_Q), nq * C::TILE);
-                        for (int j = 0; j < nq; ++j)
-                            for (int kb = 0; kb < D / 64; ++kb)
-                                if (bounds_ok(q_row + j * BM >= 0 && q_row + j * BM < q_rows_all && it.h < p.hq &&
-                                                  it.bb < p.b,
-                                              p.status, 101))
-                                    tma_load_4d(s_base + C::OFF_Q + j * C::TILE + kb * C::SUB, &tm_q, bar(C::B_Q),
-                                                kb * 64, it.h, q_row + j * BM, it.bb);
+                        issue_q(it);
                         first = false;
                         ++qi;
                     }
@@ -431,8 +462,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         tma_load_4d(s_base + C::OFF_V + sv * C::TILE + kb * C::SUB, &tm_v, bar(C::B_VF + sv),
                                     kb * 64, it.hk, kv_row, it.bb);
                     ++n;
+                    if (!PERSIST && kPrefetchQ && n == 1 && next_stride > 0 && blockIdx.x + next_stride < n_items) {
+                        // the item about to start on the SM that frees up next: its Q into L2
+                        const Item nx = decode(blockIdx.x + next_stride);
+                        const int nq_row = (int)(nx.rank * p.q_row_step) + nx.q_lo0;
+                        for (int j = 0; j < (nx.q_lo0 + BM < p.q_len ? 2 : 1); ++j)
+                            for (int kb = 0; kb < D / 64; ++kb)
+                                if (nq_row + j * BM < q_rows_all)
+                                    tma_prefetch_l2_4d(&tm_q, kb * 64, nx.h, nq_row + j * BM, nx.bb);
+                    }
                 }
-                if (!PERSIST) break;
+                if (!PERSIST) {
+                    // an item without key tiles never consumes its Q: let the load land
+                    if (n == 0 && kEarlyQ) {
+                        const uint64_t t0 = global_timer_ns();
+                        while (!mbar_try_wait(bar(C::B_Q), 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
+                    }
+                    break;
+                }
             }
             if (*abort_flag && n > 0) {
                 // let the loads already issued land in shared memory before the CTA leaves
@@ -612,6 +659,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!kHalfS) {
         while (seq.next(p)) {
             bool mine = seq.need(j) && !aborted;
+            // a one-item CTA: when both query tiles start on the first key tile, tile 1
+            // begins after tile 0's first P is stored, so the two exponential phases
+            // alternate from the start instead of sharing the MUFU pipe
+            const bool stagger = kStagger && !PERSIST && nseq == 0 && seq.need(0);
+            if (stagger && j == 1 && mine) {
+                const bool okw = mbar_wait(bar(C::B_STAG), 0, w);
+                if (__any_sync(0xffffffffu, !okw)) { aborted = true; mine = false; }
+            }
             if (mine) {
                 const bool okw = mbar_wait(bar(C::B_SF + 2 * j), cs & 1, w);
                 if (__any_sync(0xffffffffu, !okw)) { aborted = true; mine = false; }
@@ -736,6 +791,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0 && okr) mbar_arrive(bar((kSplitP && q4 == 1) ? C::B_PF + j : C::B_PH + 2 * j));
+                        if (q4 == 3 && stagger && j == 0 && lane == 0) mbar_arrive(bar(C::B_STAG));
                     }
                 }
                 float a0, a1, a2, a3;
@@ -924,6 +980,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             aborted = __any_sync(0xffffffffu, !okw);
             if (!aborted) tc_fence_after();
         }
+        // a one-item CTA's tile epilogue may meet at a named barrier (the TMA store):
+        // the four warps of the tile agree on going ahead (no wait that can expire
+        // comes after this point)
+        if (!PERSIST) aborted = bar_any(4 + j, BM, aborted || (*abort_flag != 0));
         if (!aborted && (c > 0 || p.epi == EPI_STORE || p.o_out != nullptr)) {
             const bool empty = !(l > 0.f);
             const float lse2 = empty ? -INFINITY : m + log2f(l);
@@ -934,7 +994,45 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // a row outside the output tensors (debug builds record it and skip it)
             const bool row_ok = row_in && bounds_ok(orow >= 0 && orow < q_rows_all && h < p.hq && bb < p.b,
                                                     p.status, 103);
-            if (p.epi == EPI_STORE) {
+            // bf16 tiles that lie wholly inside the block leave through shared memory and
+            // one TMA store: a thread owns a row, so direct stores would touch 32 rows
+            // per warp instruction.  The staging buffer is this tile's Q buffer, free
+            // since the last PV product (issued after the tile's last S) completed.
+            const int rt = (threadIdx.x & (BM - 1));  // row within the tile (= r_in)
+            const int tile_row0 = row - rt;           // the tile's first local row
+            const bool tma_o = kTmaO && !PERSIST && o_tma && p.epi == EPI_STORE && tile_row0 + BM <= p.q_len &&
+                               bounds_ok(orow - rt + BM <= q_rows_all, p.status, 105);
+            if (tma_o) {
+                uint8_t *stile = smem + C::OFF_Q + j * C::TILE;
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t r[32];
+                    if (c > 0) tmem_ld32(o_tmem + c0, r);
+                    uint32_t w16[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        w16[i] = (c > 0) ? pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l)
+                                         : 0u;
+                    // columns [c0, c0 + 32): 64-column box c0 / 64, 16-byte chunks from
+                    // (c0 % 64) / 8, 128-byte swizzle (chunk index ^ row % 8)
+                    uint8_t *rowp = stile + (c0 / 64) * C::SUB + rt * 128;
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const int ch = (((c0 % 64) / 8) + t) ^ (rt & 7);
+                        *reinterpret_cast<uint4 *>(rowp + ch * 16) =
+                            make_uint4(w16[4 * t], w16[4 * t + 1], w16[4 * t + 2], w16[4 * t + 3]);
+                    }
+                }
+                fence_async_smem();
+                named_bar_sync(4 + j, BM);
+                if (rt == 0) {
+                    for (int kb = 0; kb < D / 64; ++kb)
+                        tma_store_4d(&tm_o, s_base + C::OFF_Q + j * C::TILE + kb * C::SUB, kb * 64, h, (int)orow, bb);
+                    bulk_commit();
+                    bulk_wait_read_all();  // the CTA may leave once the box is read out
+                }
+                if (row_ok) *lse_ptr = lse2 * kLn2;
+            } else if (p.epi == EPI_STORE) {
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     uint32_t r[32];
@@ -1048,24 +1146,9 @@ bool make_map(CUtensorMap *m, const void *base, int64_t b, int64_t s, int64_t H,
     return r == CUDA_SUCCESS;
 }
 
-// Streaming multiprocessors of the current device (looked up once per device).
-int sm_count()
-{
-    static int counts[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    if (dev < 0 || dev >= 64) return 148;
-    if (!counts[dev]) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        counts[dev] = n;
-    }
-    return counts[dev];
-}
-
 template <int D, bool DOC, bool PERSIST>
 cudaError_t launch_dd(const AttnParams &p, cudaStream_t stream, const CUtensorMap &tq, const CUtensorMap &tk,
-                      const CUtensorMap &tv)
+                      const CUtensorMap &tv, const CUtensorMap &to, int o_tma)
 {
     static unsigned long long attr_done = 0;
     cudaError_t e = set_smem_per_device((const void *)attn_tc_kernel<D, DOC, PERSIST>, Cfg<D>::SMEM, &attr_done);
@@ -1075,7 +1158,10 @@ cudaError_t launch_dd(const AttnParams &p, cudaStream_t stream, const CUtensorMa
     if (items > INT32_MAX) return cudaErrorInvalidValue;
     // persistent: one CTA per SM walks the items (one CTA fits an SM); otherwise one per item
     const int64_t grid = PERSIST ? std::min<int64_t>(items, sm_count()) : items;
-    attn_tc_kernel<D, DOC, PERSIST><<<(unsigned)grid, NTHREADS, Cfg<D>::SMEM, stream>>>(p, tq, tk, tv);
+    // one CTA per item: the item one wave later (one resident CTA per SM) prefetches its Q
+    const int next_stride = PERSIST ? 0 : sm_count();
+    attn_tc_kernel<D, DOC, PERSIST><<<(unsigned)grid, NTHREADS, Cfg<D>::SMEM, stream>>>(p, tq, tk, tv, to, o_tma,
+                                                                                       next_stride);
     return cudaGetLastError();
 }
 
@@ -1089,8 +1175,15 @@ cudaError_t launch_d(const AttnParams &p, cudaStream_t stream, int64_t q_rows, i
         return cudaErrorInvalidValue;
     // the document mask leaves few key tiles per work item: a persistent grid keeps the
     // per-item set-up (Q load, pipeline fill, epilogue) off the critical path
-    if (p.n_docs > 0) return launch_dd<D, true, kDocPersist>(p, stream, tq, tk, tv);
-    return launch_dd<D, false, kRingPersist>(p, stream, tq, tk, tv);
+    // bf16 output written by TMA stores from the epilogue (when its strides allow a map)
+    CUtensorMap to = tq;
+    int o_tma = 0;
+    if (p.epi == EPI_STORE && p.o_dtype == DT_BF16 && make_map(&to, p.o, p.b, q_rows, p.hq, D, p.o_sb, p.o_ss, p.o_sh))
+        o_tma = 1;
+    else
+        to = tq;
+    if (p.n_docs > 0) return launch_dd<D, true, kDocPersist>(p, stream, tq, tk, tv, to, o_tma);
+    return launch_dd<D, false, kRingPersist>(p, stream, tq, tk, tv, to, o_tma);
 }
 
 }  // namespace

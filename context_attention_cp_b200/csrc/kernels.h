@@ -107,10 +107,16 @@ cudaError_t set_smem_per_device(const void *fn, int bytes, unsigned long long *d
 
 // Per-position document bounds (doc_tables.cu): for every position p < seq_len,
 // doc_start[p] = the first position of the document holding p and doc_end[p] = the
-// first position past it (INT32_MAX for the last document); starts: n_docs sorted
-// document starts on the device, the first 0.
-cudaError_t launch_doc_tables(const int *starts, int n_docs, int64_t seq_len, int *doc_start, int *doc_end,
-                              cudaStream_t stream);
+// first position past it (INT32_MAX for the last document); starts: the n_docs
+// sorted document starts in HOST memory, the first 0 (they reach the kernel as
+// launch parameters, so nothing is copied from pageable memory), also written to
+// starts_dev [n_docs] for the FFMA kernels.
+cudaError_t launch_doc_tables(const int64_t *starts, int n_docs, int64_t seq_len, int *starts_dev, int *doc_start,
+                              int *doc_end, cudaStream_t stream);
+
+// Streaming multiprocessors of the current device (looked up once per device), from
+// status.cu.
+int sm_count();
 
 // Device status word of the current device (2 ints), from status.cu.
 cudaError_t status_word(int **ptr);

@@ -74,4 +74,19 @@ cudaError_t launch_wait_timeout_selftest(uint64_t limit_ns, cudaStream_t stream)
     return cudaGetLastError();
 }
 
+// Streaming multiprocessors of the current device (looked up once per device).
+int sm_count()
+{
+    static int counts[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 0 || dev >= 64) return 148;
+    if (!counts[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        counts[dev] = n;
+    }
+    return counts[dev];
+}
+
 }  // namespace cpattn
