@@ -124,10 +124,10 @@ constexpr bool kTurnLate = CP_ATTN_TURN_LATE != 0;
 #define CP_ATTN_EARLY_Q 1
 #endif
 #ifndef CP_ATTN_PREFETCH_Q
-#define CP_ATTN_PREFETCH_Q 1
+#define CP_ATTN_PREFETCH_Q 0
 #endif
 #ifndef CP_ATTN_STAGGER
-#define CP_ATTN_STAGGER 1
+#define CP_ATTN_STAGGER 0
 #endif
 #ifndef CP_ATTN_TMA_O
 #define CP_ATTN_TMA_O 1
@@ -136,6 +136,14 @@ constexpr bool kEarlyQ = CP_ATTN_EARLY_Q != 0;
 constexpr bool kPrefetchQ = CP_ATTN_PREFETCH_Q != 0;
 constexpr bool kStagger = CP_ATTN_STAGGER != 0;
 constexpr bool kTmaO = CP_ATTN_TMA_O != 0;
+// Key tiles after a query tile's first in a work item start their exponentials on
+// the first 32 score columns while the other 96 are still being read out of TMEM
+// (1), instead of after the whole row's max (0).  Written for whole P hand-over,
+// free-running warpgroups and exponentials on the MUFU pipe only.
+#ifndef CP_ATTN_CHUNKED_EXP
+#define CP_ATTN_CHUNKED_EXP 0
+#endif
+constexpr bool kChunkedExp = CP_ATTN_CHUNKED_EXP != 0 && !kSplitP && !kPingPong && kEmuMod == 0;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
@@ -655,6 +663,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // with nothing to do at an entry still takes and hands over its turn, and a
         // warpgroup that gave up (bounded wait expired) keeps taking its turns
         // without work, so the hand-overs always pair up.
+        // ---- mask of a partial tile: keys [beg, cnt) of the tile are visible to this row
+        // (positions increase with the local key index, so the visible keys form an
+        // interval: up to the row's position, from its document's start)
+        auto mask_bounds = [&](const TileSeq<DOC> &sq, int &cnt, int &beg) {
+            const int k0 = sq.kt * BN;
+            cnt = p.kv_len - k0;
+            if (cnt > BN) cnt = BN;
+            if (p.causal) {
+                int lo = 0, hi = cnt;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (range_pos(sq.kr, k0 + mid) <= pos_q) lo = mid + 1; else hi = mid;
+                }
+                cnt = lo;
+            }
+            beg = 0;
+            if (DOC) {
+                int lo = 0, hi = cnt;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (range_pos(sq.kr, k0 + mid) < ds_row) lo = mid + 1; else hi = mid;
+                }
+                beg = lo;
+            }
+        };
         int nseq = 0;
         if (!kHalfS) {
         while (seq.next(p)) {
@@ -674,8 +707,136 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             float s[BN];
             float f_rescale = 1.f, mu = 0.f;
             bool rescale = false;
+            const bool chunked = kChunkedExp && mine && c > 0;
+            if (chunked) {
+                // ---- a tile after the first: the exponent's max m is known before the
+                // scores arrive, so the exponentials of columns [0, 32) start while
+                // columns [32, 128) are still in flight from TMEM.  A chunk whose max
+                // exceeds m by more than the threshold (rare once the running max has
+                // settled) raises m to the max of the chunks from it on (no earlier chunk
+                // can exceed that), then rescales the probabilities already stored, the
+                // row sums, and O before P is handed over.
+                tc_fence_after();
+                tmem_ld32f_nowait(s_tmem, s);
+                tmem_wait_ld_dep32(s);
+                tmem_ld32f_nowait(s_tmem + 32, s + 32);
+                tmem_ld64f_nowait(s_tmem + 64, s + 64);
+                const bool part = seq.partial(j);
+                int cnt = BN, beg = 0;
+                if (part) {
+                    mask_bounds(seq, cnt, beg);
+#pragma unroll
+                    for (int cc = 0; cc < 32; ++cc)
+                        if (cc >= cnt || (DOC && cc < beg)) s[cc] = -INFINITY;
+                }
+                bool rest = false;  // columns [32, 128) arrived (and masked)
+                auto take_rest = [&]() {
+                    tmem_wait_ld_dep32(s + 32);
+                    reg_dep64(s + 64);
+                    if (part) {
+#pragma unroll
+                        for (int cc = 32; cc < BN; ++cc)
+                            if (cc >= cnt || (DOC && cc < beg)) s[cc] = -INFINITY;
+                    }
+                    rest = true;
+                };
+                mu = (m == -INFINITY) ? 0.f : m;
+                bool okr = true;
+                const uint64_t sl2x2 = f2_pack(sl2, sl2);
+                uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = f2_pack(0.f, 0.f);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    if (q4 == 1 && !rest) take_rest();
+                    // max of this chunk: two chains of 3-input max
+                    float c0m = s[32 * q4], c1m = s[32 * q4 + 1];
+#pragma unroll
+                    for (int cc = 2; cc < 30; cc += 4) {
+                        c0m = fmax3(c0m, s[32 * q4 + cc], s[32 * q4 + cc + 1]);
+                        c1m = fmax3(c1m, s[32 * q4 + cc + 2], s[32 * q4 + cc + 3]);
+                    }
+                    const float cmx = fmax3(c0m, c1m, fmaxf(s[32 * q4 + 30], s[32 * q4 + 31])) * sl2;
+                    if (__any_sync(0xffffffffu, cmx > m + kRescaleThreshold)) {
+                        if (!rest) take_rest();
+                        float r0 = cmx, r1 = -INFINITY;
+#pragma unroll
+                        for (int cc = 32 * (q4 + 1); cc < BN; cc += 2) {
+                            r0 = fmaxf(r0, s[cc] * sl2);
+                            r1 = fmaxf(r1, s[cc + 1] * sl2);
+                        }
+                        const float m_new = fmaxf(m, fmaxf(r0, r1));
+                        const float f = (m_new == m) ? 1.f : ex2_approx(m - m_new);
+                        if (q4 > 0) {
+                            // probabilities of columns [0, 32 q4) are in TMEM (bf16): scale them
+                            tmem_wait_st();
+#pragma unroll
+                            for (int qq = 0; qq < q4; ++qq) {
+                                uint32_t pr[16];
+                                tmem_ld16(s_tmem + 16 * qq, pr);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i)
+                                    pr[i] = pack_bf16x2(__uint_as_float(pr[i] << 16) * f,
+                                                        __uint_as_float(pr[i] & 0xffff0000u) * f);
+                                tmem_st16(s_tmem + 16 * qq, pr);
+                            }
+                        }
+                        acc0 = f2_fma(acc0, f2_pack(f, f), f2_pack(0.f, 0.f));
+                        acc1 = f2_fma(acc1, f2_pack(f, f), f2_pack(0.f, 0.f));
+                        l *= f;
+                        f_rescale = f;
+                        m = m_new;
+                        mu = (m == -INFINITY) ? 0.f : m;
+                        rescale = true;
+                    }
+                    const uint64_t nmux2 = f2_pack(-mu, -mu);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float e0, e1;
+                        f2_unpack(f2_fma(f2_pack(s[32 * q4 + 2 * i], s[32 * q4 + 2 * i + 1]), sl2x2, nmux2), e0, e1);
+                        e0 = ex2_approx(e0);
+                        e1 = ex2_approx(e1);
+                        const uint64_t e01 = f2_pack(e0, e1);
+                        if (i & 1) acc1 = f2_add(acc1, e01); else acc0 = f2_add(acc0, e01);
+                        pk[i] = pack_bf16x2(e0, e1);
+                    }
+                    tmem_st16(s_tmem + 16 * q4, pk);
+                    if (q4 == 3 && rescale) {
+                        // O must hold every earlier tile's P V before it is rescaled
+                        const bool okw = mbar_wait(bar(C::B_PV + 2 * j), (cs - 1) & 1, w);
+                        okr = !__any_sync(0xffffffffu, !okw);
+                        if (okr) {
+                            tc_fence_after();
+#pragma unroll
+                            for (int c0 = 0; c0 < D; c0 += 32) {
+                                uint32_t r[32];
+                                tmem_ld32(o_tmem + c0, r);
+#pragma unroll
+                                for (int cc = 0; cc < 32; ++cc)
+                                    r[cc] = __float_as_uint(__uint_as_float(r[cc]) * f_rescale);
+                                tmem_st32(o_tmem + c0, r);
+                            }
+                        }
+                    }
+                    if (q4 == 3) {
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0 && okr) mbar_arrive(bar(C::B_PH + 2 * j));
+                    }
+                }
+                float a0, a1, a2, a3;
+                f2_unpack(acc0, a0, a1);
+                f2_unpack(acc1, a2, a3);
+                l += (a0 + a1) + (a2 + a3);
+                if (okr) {
+                    ++c;
+                    ++cs;
+                } else {
+                    aborted = true;
+                }
+            }
             if (kPingPong && !kTurnLate && (j == 1 || nseq > 0)) named_bar_sync(j == 0 ? kTurn0 : kTurn1, 2 * BM);
-            if (mine) {
+            if (mine && !chunked) {
                 tc_fence_after();
                 tmem_ld64f_nowait(s_tmem, s);
                 tmem_ld64f_nowait(s_tmem + 64, s + 64);
@@ -684,26 +845,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // ---- mask (partial tiles only).  Positions increase with the local key
                 // index, so the keys this row may see form a prefix of the tile.
                 if (seq.partial(j)) {
-                    const int k0 = seq.kt * BN;
-                    int cnt = p.kv_len - k0;
-                    if (cnt > BN) cnt = BN;
-                    if (p.causal) {
-                        int lo = 0, hi = cnt;
-                        while (lo < hi) {
-                            const int mid = (lo + hi) >> 1;
-                            if (range_pos(seq.kr, k0 + mid) <= pos_q) lo = mid + 1; else hi = mid;
-                        }
-                        cnt = lo;
-                    }
-                    int beg = 0;  // keys before this row's document start are invisible
-                    if (DOC) {
-                        int lo = 0, hi = cnt;
-                        while (lo < hi) {
-                            const int mid = (lo + hi) >> 1;
-                            if (range_pos(seq.kr, k0 + mid) < ds_row) lo = mid + 1; else hi = mid;
-                        }
-                        beg = lo;
-                    }
+                    int cnt, beg;
+                    mask_bounds(seq, cnt, beg);
 #pragma unroll
                     for (int cc = 0; cc < BN; ++cc)
                         if (cc >= cnt || (DOC && cc < beg)) s[cc] = -INFINITY;
@@ -738,7 +881,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 mu = (m == -INFINITY) ? 0.f : m;
             }
             if (kPingPong && kTurnLate && (j == 1 || nseq > 0)) named_bar_sync(j == 0 ? kTurn0 : kTurn1, 2 * BM);
-            if (mine) {
+            if (mine && !chunked) {
                 // ---- probabilities, row sum, bf16 P into TMEM columns [0, 64) of S_j,
                 // 32 columns at a time so each chunk's scores die once packed.  The
                 // scale-subtract and the row sum run as packed fp32x2 instructions.

@@ -401,6 +401,40 @@ __device__ __forceinline__ void tmem_wait_ld_dep(float *v)
                  :
                  : "memory");
 }
+// 32 columns (fp32) without waiting; see tmem_ld64f_nowait.
+#define CP_F8B(b) "=f"(v[b + 0]), "=f"(v[b + 1]), "=f"(v[b + 2]), "=f"(v[b + 3]), \
+                  "=f"(v[b + 4]), "=f"(v[b + 5]), "=f"(v[b + 6]), "=f"(v[b + 7])
+__device__ __forceinline__ void tmem_ld32f_nowait(uint32_t taddr, float *v)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : CP_F8B(0), CP_F8B(8), CP_F8B(16), CP_F8B(24)
+        : "r"(taddr)
+        : "memory");
+}
+#undef CP_F8B
+// As tmem_wait_ld_dep for 32 registers.
+__device__ __forceinline__ void tmem_wait_ld_dep32(float *v)
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : CP_D8(0), CP_D8(8), CP_D8(16), CP_D8(24)
+                 :
+                 : "memory");
+}
+// 16 columns of 32 bit, then wait.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
 // Compiler-only dependency on 64 more registers (after a tmem_wait_ld_dep()).
 __device__ __forceinline__ void reg_dep64(float *v)
 {
