@@ -144,6 +144,16 @@ constexpr bool kTmaO = CP_ATTN_TMA_O != 0;
 #define CP_ATTN_CHUNKED_EXP 0
 #endif
 constexpr bool kChunkedExp = CP_ATTN_CHUNKED_EXP != 0 && !kSplitP && !kPingPong && kEmuMod == 0;
+// Grid order of the ring instantiation: (batch, kv head) outermost, the order table's
+// entries within it and the query heads of the kv head's group innermost (1), so the
+// CTAs resident at one time read one kv head's K/V blocks and these stay in L2; or
+// the order table outermost with every (batch, query head) innermost (0).  The
+// document instantiation keeps the latter: its gathered K/V fits in L2 anyway and
+// its very unequal items balance better heaviest first across all heads.
+#ifndef CP_ATTN_KV_MAJOR
+#define CP_ATTN_KV_MAJOR 1
+#endif
+constexpr bool kKvMajor = CP_ATTN_KV_MAJOR != 0;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
@@ -347,10 +357,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int rank, qp, h, bb, hk, q_lo0;
         Range32 qr;
     };
+    const int n_entries = p.n_ranks * p.n_qt;
     auto decode = [&](int item) {
         Item it;
-        const int bh = item % bh_count;
-        const int e = item / bh_count;
+        int bh, e;
+        if (kKvMajor && !DOC) {
+            // item = ((bb * hkv + hk) * n_entries + e) * group + g, query head hk * group + g
+            const int g = item % p.group;
+            const int rest = item / p.group;
+            e = rest % n_entries;
+            const int bkv = rest / n_entries;
+            bh = (bkv / p.hkv) * p.hq + (bkv % p.hkv) * p.group + g;
+        } else {
+            bh = item % bh_count;
+            e = item / bh_count;
+        }
         if (p.order_len) {
             it.rank = (int)(p.order[e] >> 16);
             it.qp = (int)(p.order[e] & 0xffffu);
