@@ -130,44 +130,52 @@ __device__ __forceinline__ int64_t doc_end_of(const BwdParams &p, int64_t pos)
 
 // First query tile (of BQ rows, q_len rows, ranges q) whose row at offset off
 // (clamped to the block) has a position >= x.
-__device__ __forceinline__ int first_qtile_from(const Range &q, int q_len, int off, int64_t x)
+__device__ __forceinline__ int first_qtile_from(const Range32 &q, int q_len, int off, int x)
 {
     const int n_qt = (q_len + BQ - 1) / BQ;
     int lo = 0, hi = n_qt;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        int64_t r = (int64_t)mid * BQ + off;
+        int r = mid * BQ + off;
         if (r > q_len - 1) r = q_len - 1;
         if (range_pos(q, r) < x) lo = mid + 1; else hi = mid;
     }
     return lo;
 }
 
-// With the head-major grid, the steps of a head start at a rotation that depends on
-// the key tile, so CTAs of one key block reduce into different dQ rows at any one
-// time.
+// With the head-major grid the CTAs of one key block must not all reduce into the
+// same dQ rows at once.  Either the ring steps of a head start at a rotation that
+// depends on the key tile (p.tile_rotation = 0: concurrent CTAs spread over every
+// query rank of the group's heads), or every CTA walks the steps in order and starts
+// each step's query tiles at an offset that depends on the key tile, wrapping
+// around (1: concurrent CTAs spread over the tiles of one or two query ranks).  The
+// host picks 1 when the group's dQ rows are too many for L2 to hold.
 struct QSeq {
     const BwdParams *p;
-    int j, k_lo, h0, n_qt, nsteps, rot;
-    Range kr;
-    int hi, sc, r, qt, qt_full, i, h;
+    // positions stay below 2^30 (the ABI checks it), so the ranges are 32-bit
+    int j, k_lo, h0, n_qt, nsteps, rot, qrot;
+    int qb_cur, left;              // first query tile of the current step, tiles left in it
+    Range32 kr;
+    int hi, sc, qt, qt_full, i, h;
     int qt_stop, qt_fend;          // query tiles [qt_stop, ...) see nothing; [qt_full, qt_fend) are full
-    int64_t de_first, de_last;     // document ends of the tile's first / last key (document mask)
-    Range qr;
+    int de_first, de_last;         // document ends of the tile's first / last key (document mask)
+    Range32 qr;
 
     __device__ void init(const BwdParams &pp, int jj, int kt, const Range &k, int hq0)
     {
         p = &pp;
         j = jj;
         k_lo = kt * BK;
-        kr = k;
+        kr = to_range32(k);
         h0 = hq0;
         n_qt = (pp.q_len + BQ - 1) / BQ;
         nsteps = pp.step_end - pp.step_begin;
-        rot = (nsteps > 0 && pp.head_major) ? kt % nsteps : 0;
+        rot = (nsteps > 0 && pp.head_major && !pp.tile_rotation) ? kt % nsteps : 0;
+        qrot = (pp.head_major && pp.tile_rotation) ? kt : 0;
+        qb_cur = 0;
+        left = 0;
         hi = 0;
         sc = -1;
-        r = pp.step_begin;
         qt = n_qt - 1;
         qt_full = 0;
         qt_stop = n_qt;
@@ -175,8 +183,8 @@ struct QSeq {
         de_first = de_last = INT32_MAX;
         if (pp.n_docs > 0 && pp.kv_len > 0) {
             const int64_t k_hi = k_lo + BK - 1 < pp.kv_len - 1 ? k_lo + BK - 1 : pp.kv_len - 1;
-            de_first = doc_end_of(pp, range_pos(k, (int64_t)k_lo));
-            de_last = doc_end_of(pp, range_pos(k, k_hi));
+            de_first = (int)doc_end_of(pp, range_pos(k, (int64_t)k_lo));
+            de_last = (int)doc_end_of(pp, range_pos(k, k_hi));
         }
         i = 0;
         h = hq0;
@@ -184,35 +192,54 @@ struct QSeq {
     __device__ bool next()
     {
         if (nsteps <= 0) return false;
-        ++qt;
-        while (qt >= qt_stop) {
-            if (++sc >= nsteps) {
-                sc = 0;
-                if (++hi >= p->group) return false;
+        if (!p->tile_rotation) {
+            ++qt;
+            while (qt >= qt_stop) {
+                if (!next_step()) return false;
+                qt = qb_cur;
             }
-            r = p->step_begin + (sc + rot) % nsteps;
-            const int N = p->n_ranks;
-            i = (j + r) % N;
-            qr = p->use_layout ? layout_range(p->layout, N, p->seq_len, i) : p->q_range;
-            if (p->n_docs > 0 && p->kv_len > 0 && p->q_len > 0 &&
-                range_pos(qr, (int64_t)0) >= de_last) {  // the whole rank lies after the tile's documents
-                qt = n_qt;
-                qt_stop = n_qt;
-                continue;
-            }
-            int qb;
-            q_tile_bounds<int64_t>(qr, p->q_len, BQ, kr, p->kv_len, k_lo, BK, p->causal != 0, &qb, &qt_full);
-            qt_stop = n_qt;
-            qt_fend = n_qt;
-            if (p->n_docs > 0) {
-                // rows at or past the end of the last key's document see none of the
-                // tile; rows must end before the first key's document ends to see all
-                qt_stop = first_qtile_from(qr, p->q_len, 0, de_last);
-                qt_fend = first_qtile_from(qr, p->q_len, BQ - 1, de_first);
-            }
-            qt = qb;
+            return true;
         }
+        if (left > 1) {  // the next query tile of this step, wrapping past the last
+            --left;
+            if (++qt >= qt_stop) qt = qb_cur;
+            return true;
+        }
+        do {
+            if (!next_step()) return false;
+        } while (qb_cur >= qt_stop);
+        left = qt_stop - qb_cur;
+        qt = qb_cur + qrot % left;
+        return true;
+    }
+    // Moves to the next (query head, ring step) and works out its query tiles:
+    // [qb_cur, qt_stop) see the key tile (qb_cur >= qt_stop: none).
+    __device__ bool next_step()
+    {
+        if (++sc >= nsteps) {
+            sc = 0;
+            if (++hi >= p->group) return false;
+        }
+        const int r = p->step_begin + (sc + rot) % nsteps;
+        const int N = p->n_ranks;
+        i = (j + r) % N;
+        qr = p->use_layout ? layout_range_t<int>(p->layout, N, (int)p->seq_len, i) : to_range32(p->q_range);
         h = h0 + hi;
+        if (p->n_docs > 0 && p->kv_len > 0 && p->q_len > 0 &&
+            range_pos(qr, 0) >= de_last) {  // the whole rank lies after the tile's documents
+            qb_cur = n_qt;
+            qt_stop = n_qt;
+            return true;
+        }
+        q_tile_bounds<int>(qr, p->q_len, BQ, kr, p->kv_len, k_lo, BK, p->causal != 0, &qb_cur, &qt_full);
+        qt_stop = n_qt;
+        qt_fend = n_qt;
+        if (p->n_docs > 0) {
+            // rows at or past the end of the last key's document see none of the
+            // tile; rows must end before the first key's document ends to see all
+            qt_stop = first_qtile_from(qr, p->q_len, 0, de_last);
+            qt_fend = first_qtile_from(qr, p->q_len, BQ - 1, de_first);
+        }
         return true;
     }
     __device__ bool partial() const { return qt < qt_full || qt >= qt_fend; }
@@ -511,7 +538,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     while (lo < hi) {
                         const int mid = (lo + hi) >> 1;
                         const int64_t row = row0 + mid < last ? row0 + mid : last;
-                        if (range_pos(seq.qr, row) < pk) lo = mid + 1; else hi = mid;
+                        if (range_pos(seq.qr, (int)row) < pk) lo = mid + 1; else hi = mid;
                     }
                     c_first = lo;
                 }
@@ -522,7 +549,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     while (lo < hi) {
                         const int mid = (lo + hi) >> 1;
                         const int64_t row = row0 + mid < last ? row0 + mid : last;
-                        if (range_pos(seq.qr, row) < de_key) lo = mid + 1; else hi = mid;
+                        if (range_pos(seq.qr, (int)row) < de_key) lo = mid + 1; else hi = mid;
                     }
                     c_last = lo;
                 }

@@ -103,6 +103,10 @@ struct BwdParams {
     // work order: entry e -> (key block, key tile) = (order[e] >> 16, order[e] & 0xffff);
     // head_major puts (batch, kv head) outside the order in the grid
     int head_major;
+    // with head_major: 1 = each CTA starts every ring step's query tiles at an offset
+    // set by its key tile (wrapping around); 0 = it starts its ring steps at such an
+    // offset (see QSeq in attn_bwd.cu)
+    int tile_rotation;
     int n_kt;
     int order_len;
     uint32_t order[kMaxOrder];
