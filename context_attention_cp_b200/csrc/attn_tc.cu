@@ -204,6 +204,15 @@ __device__ __forceinline__ int doc_start_of(const AttnParams &p, int pos)
 __device__ __forceinline__ int first_tile_from(const Range32 &k, int kv_len, int off, int x)
 {
     const int n_kt = (int)((kv_len + BN - 1) / BN);
+    if (k.len1 == 0 && k.stride > 0) {
+        // one segment, positions start0 + i stride: the first index i* at or past x; a
+        // tile qualifies once its probe index (clamped to kv_len - 1) reaches i*
+        const int istar = x <= k.start0 ? 0 : (x - k.start0 + k.stride - 1) / k.stride;
+        if (istar > kv_len - 1) return n_kt;
+        const int t1 = istar - off <= 0 ? 0 : (istar - off + BN - 1) / BN;
+        const int tc = kv_len - off <= 0 ? 0 : (kv_len - off + BN - 1) / BN;
+        return min(min(t1, tc), n_kt);
+    }
     int lo = 0, hi = n_kt;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
@@ -691,6 +700,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int k0 = sq.kt * BN;
             cnt = p.kv_len - k0;
             if (cnt > BN) cnt = BN;
+            const Range32 &kr = sq.kr;
+            const bool seg0 = kr.len1 == 0 || k0 + cnt - 1 < kr.len0;
+            if (kr.stride > 0 && (seg0 || k0 >= kr.len0)) {
+                // the tile's keys lie in one segment: positions base + i stride
+                const int base = seg0 ? kr.start0 : kr.start1 - kr.len0 * kr.stride;
+                if (p.causal) {
+                    const int ilast = pos_q < base ? -1 : (pos_q - base) / kr.stride;
+                    cnt = min(max(ilast - k0 + 1, 0), cnt);
+                }
+                beg = 0;
+                if (DOC) {
+                    const int istar = ds_row <= base ? 0 : (ds_row - base + kr.stride - 1) / kr.stride;
+                    beg = min(max(istar - k0, 0), cnt);
+                }
+                return;
+            }
             if (p.causal) {
                 int lo = 0, hi = cnt;
                 while (lo < hi) {
