@@ -207,7 +207,7 @@ __device__ __forceinline__ int first_tile_from(const Range32 &k, int kv_len, int
     if (k.len1 == 0 && k.stride > 0) {
         // one segment, positions start0 + i stride: the first index i* at or past x; a
         // tile qualifies once its probe index (clamped to kv_len - 1) reaches i*
-        const int istar = x <= k.start0 ? 0 : (x - k.start0 + k.stride - 1) / k.stride;
+        const int istar = x <= k.start0 ? 0 : k.stride == 1 ? x - k.start0 : (x - k.start0 + k.stride - 1) / k.stride;
         if (istar > kv_len - 1) return n_kt;
         const int t1 = istar - off <= 0 ? 0 : (istar - off + BN - 1) / BN;
         const int tc = kv_len - off <= 0 ? 0 : (kv_len - off + BN - 1) / BN;
@@ -706,12 +706,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // the tile's keys lie in one segment: positions base + i stride
                 const int base = seg0 ? kr.start0 : kr.start1 - kr.len0 * kr.stride;
                 if (p.causal) {
-                    const int ilast = pos_q < base ? -1 : (pos_q - base) / kr.stride;
+                    const int ilast = pos_q < base ? -1 : kr.stride == 1 ? pos_q - base : (pos_q - base) / kr.stride;
                     cnt = min(max(ilast - k0 + 1, 0), cnt);
                 }
                 beg = 0;
                 if (DOC) {
-                    const int istar = ds_row <= base ? 0 : (ds_row - base + kr.stride - 1) / kr.stride;
+                    const int istar = ds_row <= base     ? 0
+                                      : kr.stride == 1 ? ds_row - base
+                                                       : (ds_row - base + kr.stride - 1) / kr.stride;
                     beg = min(max(istar - k0, 0), cnt);
                 }
                 return;
