@@ -213,7 +213,10 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
         "scaling": "strong" if args.gpus > 1 else "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "ms_per_step": None,
+        # a whole step (every query row) is never run: the time one would take at the
+        # sampled rate
+        "ms_per_step": w.effective_flops() / (value * 1e12) * 1e3 if value > 0 else None,
+        "ms_per_step_how": "extrapolated: the workload's effective FLOPs / the sampled rate",
         "config": {"workload": w.name, "b": w.b, "S": w.S, "hq": w.hq, "hkv": w.hkv, "d": w.d,
                    "layout": w.layout, "N": w.N, "causal": w.causal},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
