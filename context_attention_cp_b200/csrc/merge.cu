@@ -56,7 +56,10 @@ __device__ __forceinline__ void store8(void *base, int dtype, int64_t off, const
     }
 }
 
-constexpr int MT = 256;  // threads per CTA
+#ifndef CP_MERGE_THREADS
+#define CP_MERGE_THREADS 256
+#endif
+constexpr int MT = CP_MERGE_THREADS;  // threads per CTA
 #ifndef CP_MERGE_TS
 #define CP_MERGE_TS 8
 #endif
