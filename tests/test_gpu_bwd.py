@@ -64,6 +64,7 @@ BWD_CASES = [
     ("contiguous", 1, 320, True, 2, 2, 1),
     ("contiguous", 3, 96, True, 1, 2, 2),    # c = 32, less than one query tile
     ("zigzag", 8, 2048, True, 1, 8, 2),
+    ("zigzag", 4, 1024, True, 2, 8, 2),      # two batch entries, groups of four query heads
 ]
 
 

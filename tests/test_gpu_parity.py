@@ -200,6 +200,21 @@ def test_ring_matches_oracle(cp, case, mode):
     assert_close_o(np64(o), ro, tol_o)
 
 
+@pytest.mark.parametrize("mode", ["fused", "stepwise", "stepwise_epi"])
+@pytest.mark.parametrize("layout,N,S", [("zigzag", 4, 1024), ("striped", 2, 512)])
+def test_ring_batched_gqa_matches_oracle(cp, layout, N, S, mode):
+    """Two batch entries and groups of four query heads per kv head, every output
+    element: the kernel's grid runs (batch, kv head) outermost and the query heads of
+    a group innermost, so every decoded (batch, kv head, rank, query head) must land
+    on its own rows."""
+    q, k, v = W.random_qkv(2, S, 8, 2, 128, "bf16", seed=S + 7 * N)
+    o, lse = _ring_on_gpu(cp, q, k, v, layout, N, True, mode)
+    ro, rl = oracle.ring_attention(np64(q), np64(k), np64(v), layout, N, True, 128 ** -0.5)
+    tol_o, tol_l = TOL["bf16"]
+    assert_close_lse(np64(lse), rl, tol_l)
+    assert_close_o(np64(o), ro, tol_o)
+
+
 def test_fp32_workload_full(cp):
     """The fp32 S=256 contiguous N=2 workload, every output element."""
     w = W.BY_NAME["fp32_s256_contig2"]
