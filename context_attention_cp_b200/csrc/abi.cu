@@ -22,12 +22,13 @@
 using namespace cpattn;
 
 // The backward's grid is head-major (the CTAs resident at one time share a few heads'
-// Q, dO and dQ rows in L2) once one head's work items fill a wave of the device, or
-// always with CP_BWD_HEAD_MAJOR=1.
+// Q, dO and dQ rows in L2) once one head's work items fill a wave of the device;
+// CP_BWD_HEAD_MAJOR=1 makes it always head-major, -1 never.
 #ifndef CP_BWD_HEAD_MAJOR
 #define CP_BWD_HEAD_MAJOR 0
 #endif
-constexpr bool kBwdHeadMajor = CP_BWD_HEAD_MAJOR != 0;
+constexpr bool kBwdHeadMajor = CP_BWD_HEAD_MAJOR > 0;
+constexpr bool kBwdNeverHeadMajor = CP_BWD_HEAD_MAJOR < 0;
 
 // Head-major backward: the resident CTAs of one kv head reduce into its group's dQ
 // rows.  When those rows (group x rows x d fp32) fit in L2, the CTAs start their ring
@@ -954,7 +955,7 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "device query");
-    p.head_major = kBwdHeadMajor || n_kt >= (int64_t)sms;
+    p.head_major = !kBwdNeverHeadMajor && (kBwdHeadMajor || n_kt >= (int64_t)sms);
     p.tile_rotation = p.head_major && bwd_tile_rotation(p.group, S, p.d, dev);
     e = launch_attn_bwd(p, st);
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
@@ -1431,7 +1432,7 @@ cp_status cp_ring_attn_bwd(int32_t layout, int32_t N, int32_t causal, const cp_t
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "device query");
-    p.head_major = kBwdHeadMajor || (int64_t)N * n_kt >= (int64_t)sms;
+    p.head_major = !kBwdNeverHeadMajor && (kBwdHeadMajor || (int64_t)N * n_kt >= (int64_t)sms);
     p.tile_rotation = p.head_major && bwd_tile_rotation(p.group, S, p.d, dev);
     e = launch_attn_bwd(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
