@@ -31,6 +31,10 @@ def _allgather(cp, q, k, v, layout, N, causal, docs):
     return o, lse
 
 
+# More document starts than one launch of the table kernel takes (2048 per launch):
+# 2500 documents of a few tokens each over 8192 positions.
+MANY_DOCS = [0] + sorted(int(x) for x in np.random.default_rng(5).choice(np.arange(1, 8192), 2499, replace=False))
+
 CASES = [
     # layout, N, S, b, hq, hkv, document starts
     ("zigzag", 4, 1024, 1, 4, 2, [0, 100, 101, 400, 777]),
@@ -40,6 +44,7 @@ CASES = [
     ("contiguous", 1, 640, 1, 2, 2, [0, 64, 320]),
     ("zigzag", 8, 2048, 1, 8, 2, list(range(0, 2048, 97))),   # many short documents
     ("zigzag", 4, 1024, 1, 4, 2, [0]),                        # no mask: plain causal attention
+    ("zigzag", 4, 8192, 1, 2, 1, MANY_DOCS),                  # two launches of the table kernel
 ]
 
 
@@ -148,6 +153,7 @@ BWD_CASES = [
     ("contiguous", 3, 390, 1, 2, 1, [0, 129, 130, 389]),
     ("zigzag", 8, 2048, 1, 8, 2, list(range(0, 2048, 97))),
     ("zigzag", 4, 1024, 1, 4, 2, [0]),
+    ("zigzag", 4, 8192, 1, 2, 1, MANY_DOCS),
 ]
 
 
