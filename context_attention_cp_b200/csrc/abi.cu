@@ -855,9 +855,16 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     int *doc_pos_start = reinterpret_cast<int *>(ws + 4 * kb + up((int64_t)n_docs * 4));
     int *doc_pos_end = reinterpret_cast<int *>(ws + 4 * kb + up((int64_t)n_docs * 4) + up(S * 4));
     char *ws_q = ws + 4 * kb + up((int64_t)n_docs * 4) + 2 * up(S * 4);
-    // the gather of K and V into original order (as in the forward)
-    if ((s = cp_layout_permute(layout, N, 1, &kg, const_cast<cp_tensor *>(k), 1, stream)) != CP_OK) return s;
-    if ((s = cp_layout_permute(layout, N, 1, &vg, const_cast<cp_tensor *>(v), 1, stream)) != CP_OK) return s;
+    // the gather of K and V into original order (as in the forward), unless the
+    // tensor-core kernel reads K, V and writes dK, dV in place (same rule as the forward)
+    const int64_t kv_map_h = (tc_path && layout == CP_LAYOUT_ZIGZAG && (c / 2) % kBwdKeyTile == 0) ? c / 2 : 0;
+    const bool kv_in_place = tc_path && (layout == CP_LAYOUT_CONTIGUOUS || kv_map_h > 0);
+    if (!kv_in_place) {
+        if ((s = cp_layout_permute(layout, N, 1, &kg, const_cast<cp_tensor *>(k), 1, stream)) != CP_OK) return s;
+        if ((s = cp_layout_permute(layout, N, 1, &vg, const_cast<cp_tensor *>(v), 1, stream)) != CP_OK) return s;
+    }
+    const cp_tensor &kx = kv_in_place ? *k : kg, &vx = kv_in_place ? *v : vg;
+    const cp_tensor &dkx = kv_in_place ? *dk : dkg, &dvx = kv_in_place ? *dv : dvg;
     cudaError_t e = cudaSuccess;
     if (n_docs > 1) {  // device starts for the FFMA kernels, per-position bounds for the tensor-core one
         e = launch_doc_tables(doc_starts, n_docs, S, docs_dev, doc_pos_start, doc_pos_end, st);
@@ -887,10 +894,10 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     p.kv_row_step = 0;
     p.scale = softmax_scale;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
-    p.q = q->data; p.k = kg.data; p.v = vg.data; p.o = o->data; p.dout = dout->data;
+    p.q = q->data; p.k = kx.data; p.v = vx.data; p.o = o->data; p.dout = dout->data;
     p.q_sb = q->stride[0]; p.q_ss = q->stride[1]; p.q_sh = q->stride[2];
-    p.k_sb = kg.stride[0]; p.k_ss = kg.stride[1]; p.k_sh = kg.stride[2];
-    p.v_sb = vg.stride[0]; p.v_ss = vg.stride[1]; p.v_sh = vg.stride[2];
+    p.k_sb = kx.stride[0]; p.k_ss = kx.stride[1]; p.k_sh = kx.stride[2];
+    p.v_sb = vx.stride[0]; p.v_ss = vx.stride[1]; p.v_sh = vx.stride[2];
     p.o_sb = o->stride[0]; p.o_ss = o->stride[1]; p.o_sh = o->stride[2];
     p.do_sb = dout->stride[0]; p.do_ss = dout->stride[1]; p.do_sh = dout->stride[2];
     p.lse = static_cast<const float *>(lse->data);
@@ -899,10 +906,11 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     p.stats = reinterpret_cast<float2 *>(ws_q);
     p.lpad = (int)w.lpad;
     p.dq_acc = reinterpret_cast<float *>(ws_q + w.stats_bytes);
-    p.dq = dq->data; p.dk = dkg.data; p.dv = dvg.data;
+    p.dq = dq->data; p.dk = dkx.data; p.dv = dvx.data;
     p.dq_sb = dq->stride[0]; p.dq_ss = dq->stride[1]; p.dq_sh = dq->stride[2];
-    p.dk_sb = dkg.stride[0]; p.dk_ss = dkg.stride[1]; p.dk_sh = dkg.stride[2];
-    p.dv_sb = dvg.stride[0]; p.dv_ss = dvg.stride[1]; p.dv_sh = dvg.stride[2];
+    p.dk_sb = dkx.stride[0]; p.dk_ss = dkx.stride[1]; p.dk_sh = dkx.stride[2];
+    p.dv_sb = dvx.stride[0]; p.dv_ss = dvx.stride[1]; p.dv_sh = dvx.stride[2];
+    p.kv_map_h = (int)kv_map_h;
     p.doc_starts = n_docs > 1 ? docs_dev : nullptr;
     p.n_docs = n_docs > 1 ? n_docs : 0;
     p.doc_pos_end = doc_pos_end;
@@ -959,6 +967,7 @@ cp_status cp_allgather_attn_bwd(int32_t layout, int32_t N, int32_t causal, const
     p.tile_rotation = p.head_major && bwd_tile_rotation(p.group, S, p.d, dev);
     e = launch_attn_bwd(p, st);
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    if (kv_in_place) return CP_OK;  // dK, dV were written to the ranks' blocks directly
     // the reduce-scatter: the summed dK, dV of the gathered block back to each rank
     if ((s = cp_layout_permute(layout, N, 1, &dkg, dk, 0, stream)) != CP_OK) return s;
     if ((s = cp_layout_permute(layout, N, 1, &dvg, dv, 0, stream)) != CP_OK) return s;
@@ -1143,15 +1152,24 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     NvtxRange call_range("cp_allgather_attn_fwd");
 
-    // the all-gather: every rank's K/V block back into one original-order copy
+    // the all-gather: every rank's K/V block back into one original-order copy.  The
+    // tensor-core kernel reads the ranks' blocks in place instead when every key tile
+    // of the original order is a run of consecutive rank-major rows: the contiguous
+    // layout (rank-major order is the original order), or zig-zag chunks that are a
+    // whole number of key tiles (rows through zigzag_row)
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
     char *ws = static_cast<char *>(workspace);
     const int64_t kv_bytes = up(b * S * Hkv * d * elem_size(q->dtype));
     cp_tensor kg{ws, q->dtype, 0, {b, S, Hkv, d}, {S * Hkv * d, Hkv * d, d, 1}};
     cp_tensor vg{ws + kv_bytes, q->dtype, 0, {b, S, Hkv, d}, {S * Hkv * d, Hkv * d, d, 1}};
     int *docs_dev = reinterpret_cast<int *>(ws + 2 * kv_bytes);
-    if ((s = cp_layout_permute(layout, N, 1, &kg, const_cast<cp_tensor *>(k), 1, stream)) != CP_OK) return s;
-    if ((s = cp_layout_permute(layout, N, 1, &vg, const_cast<cp_tensor *>(v), 1, stream)) != CP_OK) return s;
+    const bool tc_fwd = q->dtype == CP_BF16;
+    const int64_t kv_map_h = (tc_fwd && layout == CP_LAYOUT_ZIGZAG && (c / 2) % 128 == 0) ? c / 2 : 0;
+    const bool kv_in_place = tc_fwd && (layout == CP_LAYOUT_CONTIGUOUS || kv_map_h > 0);
+    if (!kv_in_place) {
+        if ((s = cp_layout_permute(layout, N, 1, &kg, const_cast<cp_tensor *>(k), 1, stream)) != CP_OK) return s;
+        if ((s = cp_layout_permute(layout, N, 1, &vg, const_cast<cp_tensor *>(v), 1, stream)) != CP_OK) return s;
+    }
     int *doc_pos_start = reinterpret_cast<int *>(ws + 2 * kv_bytes + up((int64_t)n_docs * 4));
     int *doc_pos_end = doc_pos_start + up(S * 4) / 4;
     if (n_docs > 1) {  // device starts for the FFMA kernel, per-position bounds for the tensor-core one
@@ -1216,7 +1234,8 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
             for (size_t e2 = 0; e2 < work.size(); ++e2) p.order[e2] = work[e2].second;
         }
     }
-    fill_inputs(p, q, &kg, &vg);
+    p.kv_map_h = (int)kv_map_h;
+    fill_inputs(p, q, kv_in_place ? k : &kg, kv_in_place ? v : &vg);
     fill_outputs(p, EPI_STORE, o, lse);
     set_status_ptr(p);
     return launch_attn(p, q->dtype, st);

@@ -353,7 +353,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_do);
             WaitCtx w{abort_flag, p.status, 41};
-            const int kv_row = (int)(j * p.kv_row_step) + k_lo;
+            int kv_row = (int)(j * p.kv_row_step) + k_lo;
+            if (p.kv_map_h > 0) kv_row = zigzag_row<int>(kv_row, p.kv_map_h, p.n_ranks);
             mbar_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
             const bool kv_ok = bounds_ok(kv_row >= 0 && kv_row < kv_rows_all && hk < p.hkv && bb < p.b, p.status, 201);
             for (int kb = 0; kb < 2 && kv_ok; ++kb) {
@@ -644,7 +645,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             void *out = half == 0 ? p.dk : p.dv;
             const int64_t sb = half == 0 ? p.dk_sb : p.dv_sb, ss = half == 0 ? p.dk_ss : p.dv_ss,
                           sh = half == 0 ? p.dk_sh : p.dv_sh;
-            const int64_t orow = (int64_t)j * p.kv_row_step + key;
+            // the tile's keys are consecutive rows of the key tensor (also in place)
+            int64_t orow = (int64_t)j * p.kv_row_step + k_lo;
+            if (p.kv_map_h > 0) orow = zigzag_row<int64_t>(orow, p.kv_map_h, p.n_ranks);
+            orow += krow;
             const bool key_in = key_ok && bounds_ok(orow >= 0 && orow < kv_rows_all, p.status, 205);
             if (p.accumulate) {
                 // block form: add this call's share into the caller's fp32 accumulator

@@ -485,7 +485,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         first = false;
                         ++qi;
                     }
-                    const int kv_row = (int)(seq.src * p.kv_row_step) + seq.kt * BN;
+                    int kv_row = (int)(seq.src * p.kv_row_step) + seq.kt * BN;
+                    if (p.kv_map_h > 0) kv_row = zigzag_row<int>(kv_row, p.kv_map_h, p.n_ranks);
                     const int sk = n % NSK, sv = n % NSV;
                     if (!mbar_wait(bar(C::B_KE + sk), ((n / NSK) & 1) ^ 1, w)) { stop = true; break; }
                     mbar_expect_tx(bar(C::B_KF + sk), C::TILE);

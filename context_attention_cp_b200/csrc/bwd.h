@@ -95,6 +95,9 @@ struct BwdParams {
     // tensor-core path: doc_pos_end[pos] = first position past the document holding
     // position pos (INT32_MAX for the last document), from launch_doc_tables
     const int *doc_pos_end;
+    // as AttnParams::kv_map_h: the key block read (K, V) and written (dK, dV) in place
+    // in zig-zag rank-major order, chunks of kv_map_h positions (0: rows = positions)
+    int kv_map_h;
     // accumulate = 1 (the block form): dq, dk, dv are fp32 and this call's shares are
     // added to them (the tensor-core kernel reduces dQ straight into dq_acc = dq and
     // adds dK, dV in its epilogue; no dq conversion); 0: they are written in the

@@ -62,6 +62,10 @@ struct AttnParams {
     // tensor-core path: doc_pos_start[pos] = first position of the document holding
     // position pos (of the seq_len positions), from launch_doc_tables
     const int *doc_pos_start;
+    // kv_explicit with a zig-zag rank-major K/V (the All-Gather entry reading the
+    // ranks' blocks in place): the chunk length h > 0, a multiple of the key tile, and
+    // key tile rows map through zigzag_row(position, h, n_ranks); 0: rows = positions
+    int kv_map_h;
     // work order: entry e -> (rank, row group) = (order[e] >> 16, order[e] & 0xffff);
     // a row group is the query rows one CTA covers (256 tensor-core, 128 SIMT)
     int n_qt;                  // row groups per rank

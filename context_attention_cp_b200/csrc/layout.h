@@ -93,6 +93,15 @@ CP_HD RangeT<I> layout_range_t(int layout, int N, I S, int rank)
 
 CP_HD Range layout_range(int layout, int N, int64_t S, int rank) { return layout_range_t<int64_t>(layout, N, S, rank); }
 
+// Row of original position pos in a zig-zag rank-major sequence (chunks of h
+// positions, N ranks of 2h rows): rank i holds chunk i, then chunk 2N - 1 - i.
+template <typename I>
+CP_HD I zigzag_row(I pos, I h, int N)
+{
+    const I ch = pos / h;
+    return ch < (I)N ? ch * 2 * h + (pos - ch * h) : ((I)(2 * N - 1) - ch) * 2 * h + h + (pos - ch * h);
+}
+
 // For query tile [q_lo, q_lo + tile_q) of a block of q_len rows (ranges q) against a
 // key block of kv_len rows (ranges k) cut into tiles of tile_k: key tiles
 // [0, *kt_full) are FULL, [*kt_full, *kt_end) PARTIAL, [*kt_end, n_kt) SKIP.
