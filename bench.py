@@ -368,11 +368,18 @@ def run_legs(cp, torch, dev, w, qd, kd, vd, o, lse, timer, peaks, peak_src, args
             t, _ = timer(lambda: cp.allgather_attn_fwd(qa, ka, va, wd.layout, wd.N, wd.causal, docs, None, oa, la,
                                                        wsa), steps)
             cp.stream_check()
+            # the library reads the ranks' K/V blocks in place when every key tile is a run
+            # of consecutive rank-major rows (contiguous; zig-zag chunks of whole tiles)
+            c = wd.S // wd.N
+            in_place = wd.dtype == "bf16" and (wd.layout == "contiguous" or
+                                               (wd.layout == "zigzag" and (c // 2) % 128 == 0))
+            gather = "" if in_place else "K and V gather + "
             e = {"n_docs": len(docs),
-                 "forward": tflops_entry(wd.effective_flops(), t, peak_tf, peak_src, launches_per_step=4,
+                 "forward": tflops_entry(wd.effective_flops(), t, peak_tf, peak_src,
+                                         launches_per_step=2 if in_place else 4,
                                          kernel="attn_tc_kernel (document variant)",
-                                         timed="whole call: K and V gather + document tables + document-masked"
-                                               " attention")}
+                                         timed="whole call: " + gather + "document tables + document-masked"
+                                               " attention" + (" (K/V read in place)" if in_place else ""))}
             doa = cp.layout_permute(W.make_do(wd).to(dev), wd.layout, wd.N)
             gq, gk, gv = torch.empty_like(qa), torch.empty_like(ka), torch.empty_like(va)
             wsb = torch.empty(cp.lib().cp_allgather_bwd_workspace_bytes(wd.N, 0, wd.b, wd.S, wd.hq, wd.hkv, wd.d,
@@ -380,9 +387,10 @@ def run_legs(cp, torch, dev, w, qd, kd, vd, o, lse, timer, peaks, peak_src, args
             tb, _ = timer(lambda: cp.allgather_attn_bwd(qa, ka, va, oa, la, doa, wd.layout, wd.N, wd.causal, docs,
                                                         None, gq, gk, gv, wsb), steps)
             cp.stream_check()
-            e["backward"] = tflops_entry(2.5 * wd.effective_flops(), tb, peak_tf, peak_src, launches_per_step=8,
-                                         timed="K, V gather + document tables + statistics + backward kernel"
-                                               " + dq conversion + dK, dV scatter")
+            e["backward"] = tflops_entry(2.5 * wd.effective_flops(), tb, peak_tf, peak_src,
+                                         launches_per_step=4 if in_place else 8,
+                                         timed="whole call: " + gather + "document tables + statistics + backward"
+                                               " kernel + dq conversion" + ("" if in_place else " + dK, dV scatter"))
             ag[name] = e
             del qa, ka, va, oa, la, wsa, doa, gq, gk, gv, wsb
             torch.cuda.empty_cache()
