@@ -15,7 +15,8 @@ L2 flushed before every timed call):
               the ring (block launches + standalone merges, the page's loop as
               written; block launches merging in their epilogue) on the 8B and the
               non-causal 64K workloads, with the standalone merge's share;
-  merge     : the standalone LSE merge's HBM bandwidth at two partial sizes;
+  merge     : the standalone LSE merge's HBM bandwidth at two partial sizes, and
+              the layout permute's on this workload's q, k and lse;
   backward  : cp_ring_attn_bwd on the headline workload and the 8B one;
   allgather : All-Gather CP with a document mask (8 and 32 documents), forward and
               backward;
@@ -278,9 +279,24 @@ def run_legs(cp, torch, dev, w, qd, kd, vd, o, lse, timer, peaks, peak_src, args
         return {"shape": [b, S, H, d], "gbs": gbs, "frac_of_measured_hbm": gbs / hbm, "frac_of_8tbs": gbs / 8000.0,
                 "bytes_per_launch": mbytes, "ms_per_launch": t}
 
+    def permute_gbs(x, seq_axis=1, inverse=False):
+        y = torch.empty_like(x)
+        t, ms = timer(lambda: cp.layout_permute(x, w.layout, w.N, seq_axis=seq_axis, inverse=inverse, out=y), steps)
+        nbytes = 2 * x.numel() * x.element_size()
+        gbs = nbytes / (t * 1e-3) / 1e9
+        del y
+        torch.cuda.empty_cache()
+        return {"shape": list(x.shape), "seq_axis": seq_axis, "inverse": inverse, "gbs": gbs,
+                "frac_of_measured_hbm": gbs / hbm, "bytes_per_launch": nbytes, "ms_per_launch": t,
+                "ms_median": statistics.median(ms)}
+
     if "merge" in legs:
         w2, w5 = W.BY_NAME["llama3_8b_s8k_zigzag4"], W.BY_NAME["noncausal_s64k_contig32"]
         out["merge"] = {w2.name: merge_gbs(w2.b, w2.S, w2.hq, w2.d), w5.name: merge_gbs(w5.b, w5.S, w5.hq, w5.d)}
+        # the layout permute on this workload's tensors: bytes = read + write of the tensor
+        out["permute"] = {"layout": w.layout, "n_ranks": w.N,
+                          "q": permute_gbs(qd), "o_inverse": permute_gbs(qd, inverse=True),
+                          "k": permute_gbs(kd), "lse_inverse": permute_gbs(lse, seq_axis=2, inverse=True)}
 
     if "configs" in legs:
         cfgs = {}

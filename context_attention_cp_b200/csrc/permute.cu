@@ -6,8 +6,12 @@
 // (and the outputs put back).  Row i*c + t of the ranked tensor is the token at
 // original position pos(i, t) of the layout (see layout.h).
 //
-// The tensor is viewed as [outer, seq, inner] bytes; each thread moves one 16-,
-// 4- or 1-byte piece, consecutive threads covering consecutive bytes of a row.
+// The tensor is viewed as [outer, seq, inner] bytes and copied in 16-, 4- or
+// 1-byte pieces.  A row of at least one piece per lane of a warp goes to one warp:
+// the row's source and destination are worked out once, and the lanes stream the
+// row with several loads in flight each.  4-byte rows (the LSE) go four to a thread
+// with 16-byte accesses where the positions allow; other short rows take one piece
+// per thread.
 //
 // The same file holds the Ulysses all-to-all (section DeepSpeed-Ulysses: the
 // sequence-sharded [s/P, n_h, d_h] blocks become head-sharded [s, n_h/P, d_h] ones
@@ -17,8 +21,109 @@
 #include "kernels.h"
 #include "ulysses.h"
 
+// 1: rows (chunks) of at least 32 pieces go one per warp and 4-byte rows four per
+// thread; 0: one piece per thread everywhere (measured against each other).
+#ifndef CP_PERMUTE_ROWS
+#define CP_PERMUTE_ROWS 1
+#endif
+
 namespace cpattn {
 namespace {
+
+constexpr int kRowUnroll = 4;  // loads in flight per lane in a row copy
+
+template <typename T>
+__device__ __forceinline__ void copy_row(const T *__restrict__ s, T *__restrict__ d, int64_t n, int lane)
+{
+    // every load of a pass is issued before its stores, a ragged last pass included
+    for (int64_t e = lane; e < n; e += 32 * kRowUnroll) {
+        T r[kRowUnroll];
+#pragma unroll
+        for (int u = 0; u < kRowUnroll; ++u)
+            if (e + 32 * u < n) r[u] = s[e + 32 * u];
+#pragma unroll
+        for (int u = 0; u < kRowUnroll; ++u)
+            if (e + 32 * u < n) d[e + 32 * u] = r[u];
+    }
+}
+
+// Ranked row rr of a sequence in the layout -> original position.
+__device__ __forceinline__ int64_t ranked_to_pos(const PermuteParams &p, int64_t c, int64_t rr)
+{
+    const int rank = (int)(rr / c);
+    const Range r = layout_range(p.layout, p.n_ranks, p.seq, rank);
+    return range_pos(r, rr - (int64_t)rank * c);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) permute_rows_kernel(const __grid_constant__ PermuteParams p)
+{
+    const int64_t per_row = p.inner_bytes / (int64_t)sizeof(T);
+    const int64_t rows = p.outer * p.seq;
+    const int64_t c = p.seq / p.n_ranks;
+    const int lane = threadIdx.x & 31;
+    const T *src = reinterpret_cast<const T *>(p.src);
+    T *dst = reinterpret_cast<T *>(p.dst);
+    const int64_t n_warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows; row += n_warps) {
+        const int64_t o = row / p.seq, rr = row - o * p.seq;
+        const int64_t pos = ranked_to_pos(p, c, rr);
+        const int64_t from = p.inverse ? rr : pos;
+        const int64_t to = p.inverse ? pos : rr;
+        copy_row(src + (o * p.seq + from) * per_row, dst + (o * p.seq + to) * per_row, per_row, lane);
+    }
+}
+
+// 4-byte rows (the fp32 LSE, sequence last): each thread takes 4 consecutive ranked
+// rows, one 16-byte access on the ranked side; on the original side one 16-byte
+// access when the 4 positions are consecutive and aligned (contiguous and zig-zag
+// chunks), else 4 word accesses (striped).  Needs seq % 4 == 0 and 16-byte bases.
+template <typename I>
+__global__ void __launch_bounds__(256) permute_words_kernel(const __grid_constant__ PermuteParams p)
+{
+    // I: int32_t when outer * seq fits (fewer instructions per group), else int64_t
+    const I seq = (I)p.seq;
+    const I groups_per_seq = seq / 4;
+    const I groups = (I)p.outer * groups_per_seq;
+    const I c = seq / p.n_ranks;
+    const uint32_t *src = static_cast<const uint32_t *>(p.src);
+    uint32_t *dst = static_cast<uint32_t *>(p.dst);
+    for (I g = (I)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += (I)gridDim.x * blockDim.x) {
+        const I o = g / groups_per_seq;
+        const I rr = (g - o * groups_per_seq) * 4;
+        I pos[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int rank = (int)((rr + u) / c);
+            const RangeT<I> r = layout_range_t<I>(p.layout, p.n_ranks, seq, rank);
+            pos[u] = range_pos(r, rr + u - (I)rank * c);
+        }
+        const bool vec = pos[0] % 4 == 0 && pos[1] == pos[0] + 1 && pos[2] == pos[0] + 2 && pos[3] == pos[0] + 3;
+        const int64_t base = (int64_t)o * seq;
+        if (!p.inverse) {
+            uint4 v;
+            if (vec) {
+                v = *reinterpret_cast<const uint4 *>(src + base + pos[0]);
+            } else {
+                v.x = src[base + pos[0]];
+                v.y = src[base + pos[1]];
+                v.z = src[base + pos[2]];
+                v.w = src[base + pos[3]];
+            }
+            *reinterpret_cast<uint4 *>(dst + base + rr) = v;
+        } else {
+            const uint4 v = *reinterpret_cast<const uint4 *>(src + base + rr);
+            if (vec) {
+                *reinterpret_cast<uint4 *>(dst + base + pos[0]) = v;
+            } else {
+                dst[base + pos[0]] = v.x;
+                dst[base + pos[1]] = v.y;
+                dst[base + pos[2]] = v.z;
+                dst[base + pos[3]] = v.w;
+            }
+        }
+    }
+}
 
 template <typename T>
 __global__ void __launch_bounds__(256) permute_kernel(const __grid_constant__ PermuteParams p)
@@ -33,9 +138,7 @@ __global__ void __launch_bounds__(256) permute_kernel(const __grid_constant__ Pe
         const int64_t piece = idx % per_row;
         const int64_t rr = (idx / per_row) % p.seq;  // ranked row
         const int64_t o = idx / (per_row * p.seq);
-        const int rank = (int)(rr / c);
-        const Range r = layout_range(p.layout, p.n_ranks, p.seq, rank);
-        const int64_t pos = range_pos(r, rr - (int64_t)rank * c);
+        const int64_t pos = ranked_to_pos(p, c, rr);
         const int64_t from = p.inverse ? rr : pos;
         const int64_t to = p.inverse ? pos : rr;
         dst[(o * p.seq + to) * per_row + piece] = src[(o * p.seq + from) * per_row + piece];
@@ -65,20 +168,50 @@ __global__ void __launch_bounds__(256) shard_transpose_kernel(const __grid_const
     }
 }
 
+// The same with one warp per chunk (chunks of at least 32 pieces).
+template <typename T>
+__global__ void __launch_bounds__(256) shard_transpose_rows_kernel(const __grid_constant__ ShardParams p)
+{
+    const int64_t per = p.chunk_bytes / (int64_t)sizeof(T);
+    const int64_t n_chunks = p.P * p.b * p.rows;
+    const int lane = threadIdx.x & 31;
+    const T *src = reinterpret_cast<const T *>(p.src);
+    T *dst = reinterpret_cast<T *>(p.dst);
+    const int64_t n_warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t ch = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); ch < n_chunks; ch += n_warps) {
+        // ch walks y in order: y[r][bb][i]
+        const int64_t i = ch % p.rows;
+        const int64_t rest = ch / p.rows;
+        const int64_t bb = rest % p.b;
+        const int64_t r = rest / p.b;
+        const int64_t xo = ((bb * p.rows + i) * p.P + r) * per;
+        const int64_t yo = ch * per;
+        if (p.inverse) copy_row(src + yo, dst + xo, per, lane);
+        else copy_row(src + xo, dst + yo, per, lane);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_shard_transpose(const ShardParams &p, cudaStream_t stream)
 {
     const int64_t rows = p.P * p.b * p.rows;
     if (rows == 0 || p.chunk_bytes == 0) return cudaSuccess;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = sm_count();
     const uintptr_t al = reinterpret_cast<uintptr_t>(p.src) | reinterpret_cast<uintptr_t>(p.dst);
     int width = 1;
     if (p.chunk_bytes % 16 == 0 && al % 16 == 0) width = 16;
     else if (p.chunk_bytes % 4 == 0 && al % 4 == 0) width = 4;
-    const int64_t total = rows * (p.chunk_bytes / width);
+    const int64_t per = p.chunk_bytes / width;
+    if (CP_PERMUTE_ROWS && per >= 32) {  // one warp per chunk, 8 per block
+        int64_t blocks = (rows + 7) / 8;
+        if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+        if (width == 16) shard_transpose_rows_kernel<uint4><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        else if (width == 4) shard_transpose_rows_kernel<uint32_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        else shard_transpose_rows_kernel<uint8_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        return cudaGetLastError();
+    }
+    const int64_t total = rows * per;
     int64_t blocks = (total + 255) / 256;
     if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
     if (width == 16) shard_transpose_kernel<uint4><<<(unsigned)blocks, 256, 0, stream>>>(p);
@@ -91,14 +224,28 @@ cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream)
 {
     const int64_t rows = p.outer * p.seq;
     if (rows == 0 || p.inner_bytes == 0) return cudaSuccess;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = sm_count();
     const uintptr_t al = reinterpret_cast<uintptr_t>(p.src) | reinterpret_cast<uintptr_t>(p.dst);
     int width = 1;
     if (p.inner_bytes % 16 == 0 && al % 16 == 0) width = 16;
     else if (p.inner_bytes % 4 == 0 && al % 4 == 0) width = 4;
-    const int64_t total = rows * (p.inner_bytes / width);
+    const int64_t per = p.inner_bytes / width;
+    if (CP_PERMUTE_ROWS && per >= 32) {  // one warp per row, 8 per block
+        int64_t blocks = (rows + 7) / 8;
+        if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+        if (width == 16) permute_rows_kernel<uint4><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        else if (width == 4) permute_rows_kernel<uint32_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        else permute_rows_kernel<uint8_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        return cudaGetLastError();
+    }
+    if (CP_PERMUTE_ROWS && p.inner_bytes == 4 && p.seq % 4 == 0 && al % 16 == 0) {
+        int64_t blocks = (rows / 4 + 255) / 256;
+        if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+        if (rows + (int64_t)sms * 16 * 256 <= INT32_MAX) permute_words_kernel<int32_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        else permute_words_kernel<int64_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        return cudaGetLastError();
+    }
+    const int64_t total = rows * per;
     int64_t blocks = (total + 255) / 256;
     if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
     if (width == 16) permute_kernel<uint4><<<(unsigned)blocks, 256, 0, stream>>>(p);

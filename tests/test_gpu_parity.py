@@ -162,6 +162,35 @@ def test_permute_is_bit_exact(cp, layout, N, S):
                           L.permute(lse.view(torch.int32).numpy(), layout, N, axis=2))
 
 
+@pytest.mark.parametrize("layout,N,S", [("zigzag", 4, 1024), ("striped", 3, 96), ("contiguous", 8, 1024)])
+@pytest.mark.parametrize("H,d,dt", [(9, 128, "bf16"), (1, 37, "fp32"), (1, 33, "bf16"), (2, 160, "fp32")])
+def test_permute_long_rows_bit_exact(cp, layout, N, S, H, d, dt):
+    """Rows of at least 32 copy pieces (16-, 4- and 1-byte pieces, ragged passes)."""
+    g = torch.Generator().manual_seed(S + N + d)
+    x = torch.randn((2, S, H, d), generator=g).to(W.torch_dtype(dt))
+    bits = torch.int16 if dt == "bf16" else torch.int32
+    xr = cp.layout_permute(x.cuda(), layout, N)
+    assert np.array_equal(xr.cpu().view(bits).numpy(), L.permute(x.view(bits).numpy(), layout, N, axis=1))
+    back = cp.layout_permute(xr, layout, N, inverse=True)
+    assert torch.equal(back.cpu().view(bits), x.view(bits))
+
+
+@pytest.mark.parametrize("layout", L.LAYOUTS)
+@pytest.mark.parametrize("N,S", [(4, 24), (3, 18), (8, 4096), (2, 8)])
+def test_permute_lse_rows_bit_exact(cp, layout, N, S):
+    """4-byte rows, sequence last, both directions: groups of 4 that straddle a
+    zig-zag chunk or a rank (S = 24 over 4 ranks: chunks of 3), S % 4 != 0."""
+    if layout == "zigzag" and S % (2 * N):
+        pytest.skip("zig-zag needs S % 2N == 0")
+    g = torch.Generator().manual_seed(7 * S + N)
+    lse = torch.randn((3, 5, S), generator=g)
+    want = L.permute(lse.view(torch.int32).numpy(), layout, N, axis=2)
+    lr = cp.layout_permute(lse.cuda(), layout, N, seq_axis=2)
+    assert np.array_equal(lr.cpu().view(torch.int32).numpy(), want)
+    back = cp.layout_permute(lr, layout, N, seq_axis=2, inverse=True)
+    assert torch.equal(back.cpu().view(torch.int32), lse.view(torch.int32))
+
+
 # ------------------------------------------------------------------ ring
 
 def _ring_on_gpu(cp, q, k, v, layout, N, causal, mode):

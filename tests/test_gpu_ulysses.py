@@ -22,7 +22,10 @@ def cp():
 
 
 @pytest.mark.parametrize("P,b,S,H,d,dt", [(4, 2, 64, 8, 128, "bf16"), (2, 1, 48, 6, 64, "fp32"), (8, 1, 8192, 32, 128, "bf16"),
-                                        (1, 1, 16, 4, 128, "bf16")])
+                                        (1, 1, 16, 4, 128, "bf16"),
+                                        # chunks of 2 16-byte pieces (one piece per thread) and of
+                                        # 37 4-byte pieces (one warp per chunk, ragged last pass)
+                                        (4, 1, 64, 4, 8, "fp32"), (2, 1, 32, 2, 37, "fp32")])
 def test_all_to_all_is_bit_exact(cp, P, b, S, H, d, dt):
     x = torch.randn((b, S, H, d), generator=torch.Generator().manual_seed(S + P)).to(W.torch_dtype(dt))
     y = cp.ulysses_all_to_all(x.cuda(), P)
