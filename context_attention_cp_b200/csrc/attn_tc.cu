@@ -55,11 +55,15 @@ constexpr int NQ = 2;    // query tiles per CTA
 #ifndef CP_ATTN_NSV
 #define CP_ATTN_NSV 2
 #endif
+// P through shared memory (below): the two P buffers take the second V stage's room.
+#ifndef CP_ATTN_P_SMEM
+#define CP_ATTN_P_SMEM 0
+#endif
 constexpr int NSK = CP_ATTN_NSK;  // K stages
-constexpr int NSV = CP_ATTN_NSV;  // V stages
+constexpr int NSV = CP_ATTN_P_SMEM ? 1 : CP_ATTN_NSV;  // V stages
 constexpr int NTHREADS = 384;
 #ifndef CP_ATTN_REGS_SOFTMAX
-#define CP_ATTN_REGS_SOFTMAX 208
+#define CP_ATTN_REGS_SOFTMAX (CP_ATTN_P_SMEM ? 200 : 208)
 #endif
 constexpr int REGS_SOFTMAX = CP_ATTN_REGS_SOFTMAX;
 constexpr int REGS_OTHER = (NTHREADS * 168 - 2 * 128 * REGS_SOFTMAX) / 128;  // the rest of the launch's registers
@@ -136,6 +140,16 @@ constexpr bool kEarlyQ = CP_ATTN_EARLY_Q != 0;
 constexpr bool kPrefetchQ = CP_ATTN_PREFETCH_Q != 0;
 constexpr bool kStagger = CP_ATTN_STAGGER != 0;
 constexpr bool kTmaO = CP_ATTN_TMA_O != 0;
+// Where P (the bf16 probabilities) goes.  0: over the tile's own S columns in TMEM,
+// PV a TS product, two V stages; the next S waits for this tile's PV.  1: a
+// shared-memory buffer per query tile (a write waits for the tile's previous PV), PV
+// an SS product, one V stage; the scores' TMEM columns are free once the softmax has
+// read them, so the next key tile's S is issued then, while this tile's exponentials
+// still run.  Measured slower: an SS product at full rate reads 128 bytes per clock,
+// all of shared memory's bandwidth, and the softmax's P stores wait behind it.
+constexpr bool kPSmem = CP_ATTN_P_SMEM != 0;
+static_assert(!kPSmem || (!kHalfS && !kSplitP && !kPingPong && !kStagger && !kDocPersist && !kRingPersist),
+              "the shared-memory P hand-over is written for whole S, free-running warpgroups and one-item CTAs");
 // Key tiles after a query tile's first in a work item start their exponentials on
 // the first 32 score columns while the other 96 are still being read out of TMEM
 // (1), instead of after the whole row's max (0).  Written for whole P hand-over,
@@ -143,7 +157,7 @@ constexpr bool kTmaO = CP_ATTN_TMA_O != 0;
 #ifndef CP_ATTN_CHUNKED_EXP
 #define CP_ATTN_CHUNKED_EXP 0
 #endif
-constexpr bool kChunkedExp = CP_ATTN_CHUNKED_EXP != 0 && !kSplitP && !kPingPong && kEmuMod == 0;
+constexpr bool kChunkedExp = CP_ATTN_CHUNKED_EXP != 0 && !kSplitP && !kPingPong && kEmuMod == 0 && !kPSmem;
 // Grid order of the ring instantiation: (batch, kv head) outermost, the order table's
 // entries within it and the query heads of the kv head's group innermost (1), so the
 // CTAs resident at one time read one kv head's K/V blocks and these stay in L2; or
@@ -164,7 +178,9 @@ struct Cfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + NQ * TILE;
     static constexpr int OFF_V = OFF_K + NSK * TILE;
-    static constexpr int OFF_BAR = OFF_V + NSV * TILE;
+    static constexpr int PTILE = BM * BN * 2;         // P of one query tile (kPSmem)
+    static constexpr int OFF_P = OFF_V + NSV * TILE;
+    static constexpr int OFF_BAR = OFF_P + (kPSmem ? NQ * PTILE : 0);
     enum {
         B_Q = 0,
         B_KF = 1,
@@ -180,7 +196,8 @@ struct Cfg {
         B_OF = B_PV + 2 * NQ,   // O of query tile j read out by its epilogue (per query tile)
         B_QE = B_OF + NQ,   // Q buffer free: the work item's last S products are done
         B_STAG = B_QE + 1,  // query tile 0's first P is stored (tile 1 starts after it)
-        B_DONE = B_STAG + 1,
+        B_SC = B_STAG + 1,  // kPSmem: query tile j's scores are read out of TMEM (per tile)
+        B_DONE = B_SC + NQ,
         NBAR = B_DONE + 1
     };
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -435,6 +452,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         mbar_init(bar(C::B_QE), 1);
         mbar_init(bar(C::B_STAG), BM / 32);
+        for (int j = 0; j < NQ; ++j) {
+            mbar_init(bar(C::B_SC + j), BM / 32);
+        }
         mbar_init(bar(C::B_DONE), 1);
         *abort_flag = 0;
         mbar_fence_init();
@@ -562,6 +582,77 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc_commit(bar(C::B_SF + 2 * j + h));
             };
             bool ok = true;
+            if constexpr (kPSmem) {
+                // ---- P through shared memory (one work item per CTA).  Per key tile n:
+                // the S products of tile n + 1 go out first, each once its query tile's
+                // softmax has read the previous scores; then the PV products of tile n,
+                // each once its P is stored.
+                const int item = blockIdx.x;
+                TileSeq<DOC> seq;
+                bool have = false;
+                if (item < n_items) {
+                    const Item it = decode(item);
+                    seq.init(p, it.qr, it.rank, it.q_lo0);
+                    have = seq.next(p);
+                }
+                if (have) {
+                    ok = mbar_wait(bar(C::B_Q), 0, w) && mbar_wait(bar(C::B_KF), 0, w);
+                    if (ok) {
+                        tc_fence_after();
+                        int si0 = 0, si1 = 0;  // S products issued per query tile
+                        int pc0 = 0, pc1 = 0;  // PV products issued per query tile
+                        for (int j = 0; j < NQ; ++j)
+                            if (seq.need(j)) {
+                                issue_s(j, 0, 0);
+                                ++(j ? si1 : si0);
+                            }
+                        tc_commit(bar(C::B_KE));
+                        while (have && ok) {
+                            const bool need_n0 = seq.need(0), need_n1 = seq.need(1);
+                            const bool have_next = seq.next(p);  // seq now describes tile n + 1
+                            if (!have_next) tc_commit(bar(C::B_QE));  // the item's last S products are issued
+                            if (have_next) {
+                                if (!mbar_wait(bar(C::B_KF + (n + 1) % NSK), ((n + 1) / NSK) & 1, w)) { ok = false; break; }
+                                for (int j = 0; j < NQ && ok; ++j) {
+                                    if (!seq.need(j)) continue;
+                                    int &si = j ? si1 : si0;
+                                    // the softmax has read this tile's previous scores
+                                    if (si > 0 && !mbar_wait(bar(C::B_SC + j), (si - 1) & 1, w)) { ok = false; break; }
+                                    tc_fence_after();
+                                    issue_s(j, n + 1, 0);
+                                    ++si;
+                                }
+                                if (!ok) break;
+                                tc_commit(bar(C::B_KE + (n + 1) % NSK));
+                            }
+                            const int sv = n % NSV;
+                            if (!mbar_wait(bar(C::B_VF + sv), (n / NSV) & 1, w)) { ok = false; break; }
+                            const uint32_t vb = s_base + C::OFF_V + sv * C::TILE;
+                            for (int j = 0; j < NQ && ok; ++j) {
+                                if (!(j ? need_n1 : need_n0)) continue;
+                                int &pc = j ? pc1 : pc0;
+                                if (!mbar_wait(bar(C::B_PH + 2 * j), pc & 1, w)) { ok = false; break; }
+                                tc_fence_after();
+                                const uint32_t o_tmem = tbase + C::T_O + (uint32_t)(j * D);
+                                const uint32_t pa = s_base + C::OFF_P + j * C::PTILE;
+#pragma unroll
+                                for (int k = 0; k < BN / 16; ++k) {
+                                    const uint32_t off = (k >> 2) * C::SUB + (k & 3) * 32;
+                                    mma_ss(o_tmem, smem_desc_sw128(pa + off, 16, 1024),
+                                           smem_desc_sw128(vb + k * 2048, C::SUB, 1024), C::IDESC_PV,
+                                           (k > 0 || pc > 0) ? 1u : 0u);
+                                }
+                                tc_commit(bar(C::B_PV + 2 * j));
+                                ++pc;
+                            }
+                            if (!ok) break;
+                            tc_commit(bar(C::B_VE + sv));
+                            ++n;
+                            have = have_next;
+                        }
+                    }
+                }
+            } else {
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 const Item it = decode(item);
                 TileSeq<DOC> seq;
@@ -649,6 +740,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 ++qi;
                 if (!PERSIST) break;
             }
+            }
             // drain: every MMA issued above has finished before TMEM is released
             tc_commit(bar(C::B_DONE));
             const uint64_t t0 = global_timer_ns();
@@ -667,6 +759,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
         const uint32_t s_tmem = tbase + lane_off + (uint32_t)(j * 128);
         const uint32_t o_tmem = tbase + lane_off + C::T_O + (uint32_t)(j * D);
+        // this row's P in the shared buffer (kPSmem): 8-row atoms of 1024 bytes
+        const uint32_t p_row = s_base + C::OFF_P + (uint32_t)(j * C::PTILE + (r_in >> 3) * 1024 + (r_in & 7) * 128);
+        (void)p_row;
         const float sl2 = p.scale_log2;
         int cs = 0;           // S tiles of this query tile consumed, over all work items
         bool aborted = false;
@@ -891,6 +986,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tmem_ld64f_nowait(s_tmem + 64, s + 64);
                 tmem_wait_ld_dep(s);
                 reg_dep64(s + 64);
+                if (kPSmem) {  // the scores are in registers: the tile's next S may overwrite them
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(C::B_SC + j));
+                }
                 // ---- mask (partial tiles only).  Positions increase with the local key
                 // index, so the keys this row may see form a prefix of the tile.
                 if (seq.partial(j)) {
@@ -959,11 +1059,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         if (i & 1) acc1 = f2_add(acc1, e01); else acc0 = f2_add(acc0, e01);
                         pk[i] = pack_bf16x2(e0, e1);
                     }
-                    tmem_st16(s_tmem + 16 * q4, pk);
+                    if (kPSmem) {
+                        // the buffer is free once the tile's previous PV is done
+                        if (q4 == 0 && cs > 0) {
+                            const bool okw = mbar_wait(bar(C::B_PV + 2 * j), (cs - 1) & 1, w);
+                            okr = !__any_sync(0xffffffffu, !okw);
+                        }
+                        if (okr) {
+                            // row r_in, keys [32 q4, 32 q4 + 32): 16-byte chunks c = 4 q4 + i
+                            // of the 128-byte-swizzled K-major layout (64-key blocks)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int cc = 4 * q4 + i;
+                                st_shared_v4(p_row + (uint32_t)((cc >> 3) * C::SUB + (((cc & 7) ^ (r_in & 7)) << 4)),
+                                             pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                            }
+                        }
+                    } else {
+                        tmem_st16(s_tmem + 16 * q4, pk);
+                    }
                     if (q4 == (kSplitP ? 1 : 3) && rescale) {
                         // O must hold every earlier tile's P V before it is rescaled
                         const bool okw = mbar_wait(bar(C::B_PV + 2 * j), (cs - 1) & 1, w);
-                        okr = !__any_sync(0xffffffffu, !okw);
+                        okr = okr && !__any_sync(0xffffffffu, !okw);
                         if (okr) {
                             tc_fence_after();
 #pragma unroll
@@ -979,6 +1097,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     if (q4 == 3 && kPingPong) named_bar_arrive(j == 0 ? kTurn1 : kTurn0, 2 * BM);
                     if ((kSplitP && q4 == 1) || q4 == 3) {
+                        if (kPSmem) fence_async_smem();  // P stores visible to the tensor core
                         tmem_wait_st();
                         tc_fence_before();
                         __syncwarp();
