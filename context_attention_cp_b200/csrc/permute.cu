@@ -7,9 +7,9 @@
 // original position pos(i, t) of the layout (see layout.h).
 //
 // The tensor is viewed as [outer, seq, inner] bytes and copied in 16-, 4- or
-// 1-byte pieces.  A row of at least one piece per lane of a warp goes to one warp:
-// the row's source and destination are worked out once, and the lanes stream the
-// row with several loads in flight each.  4-byte rows (the LSE) go four to a thread
+// 1-byte pieces.  A row of at least one piece per lane of a warp goes to one warp
+// (a long row in 8 KB segments, a warp each): the row's source and destination are
+// worked out once, and the lanes stream the row with several loads in flight each.  4-byte rows (the LSE) go four to a thread
 // with 16-byte accesses where the positions allow; other short rows take one piece
 // per thread.
 //
@@ -55,22 +55,29 @@ __device__ __forceinline__ int64_t ranked_to_pos(const PermuteParams &p, int64_t
     return range_pos(r, rr - (int64_t)rank * c);
 }
 
+// A row (chunk) of more than kSegPieces pieces is cut into segments of kSegPieces, a
+// warp per segment, so a few long rows still spread over the whole grid.
+constexpr int64_t kSegPieces = 512;
+
 template <typename T>
-__global__ void __launch_bounds__(256) permute_rows_kernel(const __grid_constant__ PermuteParams p)
+__global__ void __launch_bounds__(256) permute_rows_kernel(const __grid_constant__ PermuteParams p, int64_t n_seg)
 {
     const int64_t per_row = p.inner_bytes / (int64_t)sizeof(T);
-    const int64_t rows = p.outer * p.seq;
+    const int64_t units = p.outer * p.seq * n_seg;
     const int64_t c = p.seq / p.n_ranks;
     const int lane = threadIdx.x & 31;
     const T *src = reinterpret_cast<const T *>(p.src);
     T *dst = reinterpret_cast<T *>(p.dst);
     const int64_t n_warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows; row += n_warps) {
+    for (int64_t u = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < units; u += n_warps) {
+        const int64_t row = n_seg == 1 ? u : u / n_seg;
+        const int64_t e0 = n_seg == 1 ? 0 : (u - row * n_seg) * kSegPieces;
+        const int64_t n = per_row - e0 < kSegPieces || n_seg == 1 ? per_row - e0 : kSegPieces;
         const int64_t o = row / p.seq, rr = row - o * p.seq;
         const int64_t pos = ranked_to_pos(p, c, rr);
         const int64_t from = p.inverse ? rr : pos;
         const int64_t to = p.inverse ? pos : rr;
-        copy_row(src + (o * p.seq + from) * per_row, dst + (o * p.seq + to) * per_row, per_row, lane);
+        copy_row(src + (o * p.seq + from) * per_row + e0, dst + (o * p.seq + to) * per_row + e0, n, lane);
     }
 }
 
@@ -168,26 +175,29 @@ __global__ void __launch_bounds__(256) shard_transpose_kernel(const __grid_const
     }
 }
 
-// The same with one warp per chunk (chunks of at least 32 pieces).
+// The same with one warp per chunk (chunks of at least 32 pieces; longer ones in
+// segments of kSegPieces).
 template <typename T>
-__global__ void __launch_bounds__(256) shard_transpose_rows_kernel(const __grid_constant__ ShardParams p)
+__global__ void __launch_bounds__(256) shard_transpose_rows_kernel(const __grid_constant__ ShardParams p, int64_t n_seg)
 {
     const int64_t per = p.chunk_bytes / (int64_t)sizeof(T);
-    const int64_t n_chunks = p.P * p.b * p.rows;
+    const int64_t units = p.P * p.b * p.rows * n_seg;
     const int lane = threadIdx.x & 31;
     const T *src = reinterpret_cast<const T *>(p.src);
     T *dst = reinterpret_cast<T *>(p.dst);
     const int64_t n_warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t ch = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); ch < n_chunks; ch += n_warps) {
-        // ch walks y in order: y[r][bb][i]
+    for (int64_t u = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < units; u += n_warps) {
+        const int64_t ch = n_seg == 1 ? u : u / n_seg;  // ch walks y in order: y[r][bb][i]
+        const int64_t e0 = n_seg == 1 ? 0 : (u - ch * n_seg) * kSegPieces;
+        const int64_t n = per - e0 < kSegPieces || n_seg == 1 ? per - e0 : kSegPieces;
         const int64_t i = ch % p.rows;
         const int64_t rest = ch / p.rows;
         const int64_t bb = rest % p.b;
         const int64_t r = rest / p.b;
-        const int64_t xo = ((bb * p.rows + i) * p.P + r) * per;
-        const int64_t yo = ch * per;
-        if (p.inverse) copy_row(src + yo, dst + xo, per, lane);
-        else copy_row(src + xo, dst + yo, per, lane);
+        const int64_t xo = ((bb * p.rows + i) * p.P + r) * per + e0;
+        const int64_t yo = ch * per + e0;
+        if (p.inverse) copy_row(src + yo, dst + xo, n, lane);
+        else copy_row(src + xo, dst + yo, n, lane);
     }
 }
 
@@ -203,12 +213,13 @@ cudaError_t launch_shard_transpose(const ShardParams &p, cudaStream_t stream)
     if (p.chunk_bytes % 16 == 0 && al % 16 == 0) width = 16;
     else if (p.chunk_bytes % 4 == 0 && al % 4 == 0) width = 4;
     const int64_t per = p.chunk_bytes / width;
-    if (CP_PERMUTE_ROWS && per >= 32) {  // one warp per chunk, 8 per block
-        int64_t blocks = (rows + 7) / 8;
+    if (CP_PERMUTE_ROWS && per >= 32) {  // one warp per chunk (segment), 8 per block
+        const int64_t n_seg = per > 2 * kSegPieces ? (per + kSegPieces - 1) / kSegPieces : 1;
+        int64_t blocks = (rows * n_seg + 7) / 8;
         if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-        if (width == 16) shard_transpose_rows_kernel<uint4><<<(unsigned)blocks, 256, 0, stream>>>(p);
-        else if (width == 4) shard_transpose_rows_kernel<uint32_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
-        else shard_transpose_rows_kernel<uint8_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        if (width == 16) shard_transpose_rows_kernel<uint4><<<(unsigned)blocks, 256, 0, stream>>>(p, n_seg);
+        else if (width == 4) shard_transpose_rows_kernel<uint32_t><<<(unsigned)blocks, 256, 0, stream>>>(p, n_seg);
+        else shard_transpose_rows_kernel<uint8_t><<<(unsigned)blocks, 256, 0, stream>>>(p, n_seg);
         return cudaGetLastError();
     }
     const int64_t total = rows * per;
@@ -230,12 +241,13 @@ cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream)
     if (p.inner_bytes % 16 == 0 && al % 16 == 0) width = 16;
     else if (p.inner_bytes % 4 == 0 && al % 4 == 0) width = 4;
     const int64_t per = p.inner_bytes / width;
-    if (CP_PERMUTE_ROWS && per >= 32) {  // one warp per row, 8 per block
-        int64_t blocks = (rows + 7) / 8;
+    if (CP_PERMUTE_ROWS && per >= 32) {  // one warp per row (segment), 8 per block
+        const int64_t n_seg = per > 2 * kSegPieces ? (per + kSegPieces - 1) / kSegPieces : 1;
+        int64_t blocks = (rows * n_seg + 7) / 8;
         if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-        if (width == 16) permute_rows_kernel<uint4><<<(unsigned)blocks, 256, 0, stream>>>(p);
-        else if (width == 4) permute_rows_kernel<uint32_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
-        else permute_rows_kernel<uint8_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        if (width == 16) permute_rows_kernel<uint4><<<(unsigned)blocks, 256, 0, stream>>>(p, n_seg);
+        else if (width == 4) permute_rows_kernel<uint32_t><<<(unsigned)blocks, 256, 0, stream>>>(p, n_seg);
+        else permute_rows_kernel<uint8_t><<<(unsigned)blocks, 256, 0, stream>>>(p, n_seg);
         return cudaGetLastError();
     }
     if (CP_PERMUTE_ROWS && p.inner_bytes == 4 && p.seq % 4 == 0 && al % 16 == 0) {

@@ -163,9 +163,11 @@ def test_permute_is_bit_exact(cp, layout, N, S):
 
 
 @pytest.mark.parametrize("layout,N,S", [("zigzag", 4, 1024), ("striped", 3, 96), ("contiguous", 8, 1024)])
-@pytest.mark.parametrize("H,d,dt", [(9, 128, "bf16"), (1, 37, "fp32"), (1, 33, "bf16"), (2, 160, "fp32")])
+@pytest.mark.parametrize("H,d,dt", [(9, 128, "bf16"), (1, 37, "fp32"), (1, 33, "bf16"), (2, 160, "fp32"),
+                                    (72, 130, "bf16")])
 def test_permute_long_rows_bit_exact(cp, layout, N, S, H, d, dt):
-    """Rows of at least 32 copy pieces (16-, 4- and 1-byte pieces, ragged passes)."""
+    """Rows of at least 32 copy pieces (16-, 4- and 1-byte pieces, ragged passes);
+    rows of 18720 bytes go in segments of 8 KB with a ragged last one."""
     g = torch.Generator().manual_seed(S + N + d)
     x = torch.randn((2, S, H, d), generator=g).to(W.torch_dtype(dt))
     bits = torch.int16 if dt == "bf16" else torch.int32

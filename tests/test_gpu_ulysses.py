@@ -25,7 +25,9 @@ def cp():
                                         (1, 1, 16, 4, 128, "bf16"),
                                         # chunks of 2 16-byte pieces (one piece per thread) and of
                                         # 37 4-byte pieces (one warp per chunk, ragged last pass)
-                                        (4, 1, 64, 4, 8, "fp32"), (2, 1, 32, 2, 37, "fp32")])
+                                        (4, 1, 64, 4, 8, "fp32"), (2, 1, 32, 2, 37, "fp32"),
+                                        # chunks of 20800 bytes: 8 KB segments, ragged last one
+                                        (2, 1, 16, 4, 2600, "fp32")])
 def test_all_to_all_is_bit_exact(cp, P, b, S, H, d, dt):
     x = torch.randn((b, S, H, d), generator=torch.Generator().manual_seed(S + P)).to(W.torch_dtype(dt))
     y = cp.ulysses_all_to_all(x.cuda(), P)
