@@ -243,7 +243,7 @@ const std::vector<uint32_t> &ring_order_locked(int layout, int N, int64_t S, int
     return g_order_cache.emplace(key, std::move(out)).first->second;
 }
 
-int rows_per_cta(int32_t dtype) { return dtype == CP_BF16 ? attn_tc_rows_per_cta() : 128; }
+int rows_per_cta(int32_t dtype, bool doc = false) { return dtype == CP_BF16 ? attn_tc_rows_per_cta(doc) : 128; }
 
 // Work order of the backward: (key rank, key tile) entries sorted by the number of
 // query tiles that see the key tile over all steps, heaviest first.
@@ -1146,7 +1146,7 @@ cp_status cp_allgather_attn_fwd(int32_t layout, int32_t N, int32_t causal, const
     if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     const int64_t c = S / N;
     if (b == 0 || S == 0) return CP_OK;
-    const int rows = rows_per_cta(q->dtype);
+    const int rows = rows_per_cta(q->dtype, n_docs > 1);  // the document instantiation's CTA
     const int n_qt = (int)((c + rows - 1) / rows);
     if (n_qt > 65535) return fail(CP_ERR_SHAPE, "too many query tiles per rank");
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -68,8 +68,6 @@ constexpr int NTHREADS = 384;
 constexpr int REGS_SOFTMAX = CP_ATTN_REGS_SOFTMAX;
 constexpr int REGS_OTHER = (NTHREADS * 168 - 2 * 128 * REGS_SOFTMAX) / 128;  // the rest of the launch's registers
 static_assert(REGS_OTHER >= 24 && REGS_OTHER % 8 == 0, "register split");
-constexpr int WARP_LOAD = 8;
-constexpr int WARP_MMA = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // In tiles without masking, pair i of every 16 probability pairs is computed on
 // the FMA pipe (exp2_fma) when i % kEmuMod == kEmuMod - 1, the rest on the MUFU
@@ -100,6 +98,18 @@ constexpr int kTurn0 = 2, kTurn1 = 3;
 #define CP_ATTN_RING_PERSIST 0
 #endif
 constexpr bool kDocPersist = CP_ATTN_DOC_PERSIST != 0;
+// Query tiles per CTA of the document-mask instantiation: 1 (two CTAs per SM) or 2
+// (the ring's CTA).  The persistent grid is written for two.
+#ifndef CP_ATTN_DOC_NQ
+#define CP_ATTN_DOC_NQ 1
+#endif
+constexpr int kDocNQ = kDocPersist ? 2 : CP_ATTN_DOC_NQ;
+// Register split of the one-tile CTA (128 per thread at launch, two CTAs per SM): the
+// softmax warpgroup's share; the producer / MMA warpgroup gets 256 minus it (200 / 56
+// spills 40 bytes in the producer / MMA roles, the least of 176–200).
+#ifndef CP_ATTN_DOC1_REGS
+#define CP_ATTN_DOC1_REGS 200
+#endif
 // S computed in two halves of 64 keys into a two-slot ring per query tile (1): the
 // next key tile's first half only waits for the PV of this tile's first half, so a
 // softmax warpgroup always has the other half's scores ready; or S whole (0).
@@ -112,6 +122,11 @@ constexpr int HW = BN / NH;         // keys per S part
 static_assert(!(kHalfS && CP_ATTN_SPLIT_P), "split P hand-over applies to whole S only");
 static_assert(!(kHalfS && CP_ATTN_PINGPONG), "turn-taking is written for whole S");
 constexpr bool kRingPersist = CP_ATTN_RING_PERSIST != 0;
+// Query tiles per CTA of the ring instantiation (2, or 1 as the document one).
+#ifndef CP_ATTN_RING_NQ
+#define CP_ATTN_RING_NQ 2
+#endif
+constexpr int kRingNQ = kRingPersist ? 2 : CP_ATTN_RING_NQ;
 // A turn starts before the S load (0) or after the row max (1: the loads and row
 // maxima of the two tiles overlap, at the cost of more live registers).
 #ifndef CP_ATTN_TURN_LATE
@@ -171,40 +186,53 @@ constexpr bool kKvMajor = CP_ATTN_KV_MAJOR != 0;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
-template <int D>
+// Shared memory, barriers, TMEM and threads of a CTA with NQT query tiles: two (the
+// ring: the two tiles' chains interleave on the tensor pipe, one CTA per SM) or one
+// (documents: one K and one V stage, 256 TMEM columns and 256 threads, so two CTAs
+// share an SM and one's set-up, first loads and epilogue overlap the other's tiles).
+template <int D, int NQT = NQ>
 struct Cfg {
+    static constexpr int NSK_ = NQT == 1 ? 1 : NSK;
+    static constexpr int NSV_ = NQT == 1 ? 1 : NSV;
+    static constexpr int NTHR = 128 * (NQT + 1);    // softmax warpgroups + producer / MMA warpgroup
+    static constexpr int CTAS_PER_SM = NQT == 1 ? 2 : 1;
+    static constexpr int REGS_SM = NQT == 1 ? CP_ATTN_DOC1_REGS : REGS_SOFTMAX;  // softmax warpgroups
+    static constexpr int REGS_OT = NQT == 1 ? 256 - CP_ATTN_DOC1_REGS : REGS_OTHER;  // producer / MMA
+    static_assert(NQT * 128 * REGS_SM + 128 * REGS_OT <= NTHR * (65536 / (NTHR * CTAS_PER_SM) / 8 * 8),
+                  "register split exceeds the launch's registers");
     static constexpr int SUB = BM * 128;     // one 64-column swizzle block (16 KB)
     static constexpr int TILE = BM * D * 2;  // a 128 x D bf16 tile
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + NQ * TILE;
-    static constexpr int OFF_V = OFF_K + NSK * TILE;
+    static constexpr int OFF_K = OFF_Q + NQT * TILE;
+    static constexpr int OFF_V = OFF_K + NSK_ * TILE;
     static constexpr int PTILE = BM * BN * 2;         // P of one query tile (kPSmem)
-    static constexpr int OFF_P = OFF_V + NSV * TILE;
-    static constexpr int OFF_BAR = OFF_P + (kPSmem ? NQ * PTILE : 0);
+    static constexpr int OFF_P = OFF_V + NSV_ * TILE;
+    static constexpr int OFF_BAR = OFF_P + (kPSmem ? NQT * PTILE : 0);
     enum {
         B_Q = 0,
         B_KF = 1,
-        B_KE = B_KF + NSK,
-        B_VF = B_KE + NSK,
-        B_VE = B_VF + NSV,
-        B_SF = B_VE + NSV,  // per query tile and S part: index 2 j + part
-        B_PF = B_SF + 2 * NQ,  // P of keys [0, 64) of the tile stored (per query tile)
-        B_PH = B_PF + NQ,   // P stored: whole S, keys [64, 128) with the split hand-over, or S
-                            // part h (index 2 j + h; one barrier per part, so the softmax
-                            // never runs two phases ahead of the MMA warp on one barrier)
-        B_PV = B_PH + 2 * NQ,  // PV of S part h done (index 2 j + h), one barrier per part
-        B_OF = B_PV + 2 * NQ,   // O of query tile j read out by its epilogue (per query tile)
-        B_QE = B_OF + NQ,   // Q buffer free: the work item's last S products are done
-        B_STAG = B_QE + 1,  // query tile 0's first P is stored (tile 1 starts after it)
-        B_SC = B_STAG + 1,  // kPSmem: query tile j's scores are read out of TMEM (per tile)
-        B_DONE = B_SC + NQ,
+        B_KE = B_KF + NSK_,
+        B_VF = B_KE + NSK_,
+        B_VE = B_VF + NSV_,
+        B_SF = B_VE + NSV_,  // per query tile and S part: index 2 j + part
+        B_PF = B_SF + 2 * NQT,  // P of keys [0, 64) of the tile stored (per query tile)
+        B_PH = B_PF + NQT,   // P stored: whole S, keys [64, 128) with the split hand-over, or S
+                             // part h (index 2 j + h; one barrier per part, so the softmax
+                             // never runs two phases ahead of the MMA warp on one barrier)
+        B_PV = B_PH + 2 * NQT,  // PV of S part h done (index 2 j + h), one barrier per part
+        B_OF = B_PV + 2 * NQT,   // O of query tile j read out by its epilogue (per query tile)
+        B_QE = B_OF + NQT,   // Q buffer free: the work item's last S products are done
+        B_STAG = B_QE + 1,   // query tile 0's first P is stored (tile 1 starts after it)
+        B_SC = B_STAG + 1,   // kPSmem: query tile j's scores are read out of TMEM (per tile)
+        B_DONE = B_SC + NQT,
         NBAR = B_DONE + 1
     };
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 64 + 1024;  // + alignment slack
     static_assert(SMEM <= 232448, "shared memory per CTA exceeds 227 KB");
-    static constexpr int T_O = 256;
-    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(CTAS_PER_SM == 1 || CTAS_PER_SM * (SMEM + 1024) <= 233472, "two CTAs do not fit an SM");
+    static constexpr int T_O = 128 * NQT;                // O columns after the S columns
+    static constexpr uint32_t TMEM_COLS = NQT == 1 ? 256 : 512;
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, HW, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
 };
@@ -248,7 +276,7 @@ __device__ __forceinline__ int first_tile_from(const Range32 &k, int kv_len, int
 // start of its first row to its last row, and every row sees the keys from the
 // document start of its last row to its first row (positions increase with the
 // local index, so both are runs of whole tiles).
-template <bool DOC>
+template <bool DOC, int NQT = NQ>
 struct TileSeq {
     Range32 qr;
     int rank;
@@ -266,7 +294,7 @@ struct TileSeq {
         qr = q;
         rank = rk;
         q_lo0 = qlo0;
-        q_ok1 = qlo0 + BM < pp.q_len;
+        q_ok1 = NQT > 1 && qlo0 + BM < pp.q_len;
         step = pp.step_begin - 1;
         kt = 0;
         kt_end_all = 0;
@@ -354,13 +382,17 @@ __device__ __forceinline__ void store_row_chunk(void *o, int dtype, int64_t off,
     }
 }
 
-template <int D, bool DOC, bool PERSIST>
-__global__ void __launch_bounds__(NTHREADS, 1)
+template <int D, bool DOC, bool PERSIST, int NQT>
+__global__ void __launch_bounds__(128 * (NQT + 1), NQT == 1 ? 2 : 1)
     attn_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ CUtensorMap tm_o, int o_tma, int next_stride)
 {
-    using C = Cfg<D>;
+    using C = Cfg<D, NQT>;
+    // this instantiation's shape (the namespace-level names are the two-tile CTA's)
+    constexpr int NQ = NQT, NSK = C::NSK_, NSV = C::NSV_, NTHREADS = C::NTHR;
+    constexpr int WARP_LOAD = 4 * NQT, WARP_MMA = 4 * NQT + 1;
+    constexpr int REGS_SOFTMAX = C::REGS_SM, REGS_OTHER = C::REGS_OT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t s_base = smem_u32(smem);
@@ -421,7 +453,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // Q tiles of an item into the Q buffer (both tiles when the second holds rows)
     auto issue_q = [&](const Item &it) {
         const int q_row = (int)(it.rank * p.q_row_step) + it.q_lo0;
-        const int nq = it.q_lo0 + BM < p.q_len ? 2 : 1;
+        const int nq = (NQ > 1 && it.q_lo0 + BM < p.q_len) ? 2 : 1;
         mbar_expect_tx(bar(C::B_Q), nq * C::TILE);
         for (int j = 0; j < nq; ++j)
             for (int kb = 0; kb < D / 64; ++kb)
@@ -483,7 +515,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
     };
 
-    if (warp >= 8) {
+    if (warp >= 4 * NQ) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
     if (warp == WARP_LOAD) {
         // ================================================================ producer
@@ -494,7 +526,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             bool stop = false;
             for (int item = blockIdx.x; item < n_items && !stop; item += gridDim.x) {
                 const Item it = decode(item);
-                TileSeq<DOC> seq;
+                TileSeq<DOC, NQT> seq;
                 seq.init(p, it.qr, it.rank, it.q_lo0);
                 bool first = PERSIST || !kEarlyQ;
                 while (seq.next(p)) {
@@ -525,7 +557,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         // the item about to start on the SM that frees up next: its Q into L2
                         const Item nx = decode(blockIdx.x + next_stride);
                         const int nq_row = (int)(nx.rank * p.q_row_step) + nx.q_lo0;
-                        for (int j = 0; j < (nx.q_lo0 + BM < p.q_len ? 2 : 1); ++j)
+                        for (int j = 0; j < ((NQ > 1 && nx.q_lo0 + BM < p.q_len) ? 2 : 1); ++j)
                             for (int kb = 0; kb < D / 64; ++kb)
                                 if (nq_row + j * BM < q_rows_all)
                                     tma_prefetch_l2_4d(&tm_q, kb * 64, nx.h, nq_row + j * BM, nx.bb);
@@ -588,7 +620,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // softmax has read the previous scores; then the PV products of tile n,
                 // each once its P is stored.
                 const int item = blockIdx.x;
-                TileSeq<DOC> seq;
+                TileSeq<DOC, NQT> seq;
                 bool have = false;
                 if (item < n_items) {
                     const Item it = decode(item);
@@ -655,7 +687,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             } else {
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 const Item it = decode(item);
-                TileSeq<DOC> seq;
+                TileSeq<DOC, NQT> seq;
                 seq.init(p, it.qr, it.rank, it.q_lo0);
                 bool have = seq.next(p);
                 if (!have) {
@@ -780,7 +812,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float l = 0.f;        // running sum
         int c = 0;            // tiles processed by this query tile in this item
 
-        TileSeq<DOC> seq;
+        TileSeq<DOC, NQT> seq;
         seq.init(p, qr, rank, q_lo0);
         // Both softmax warpgroups walk the CTA's whole key-tile sequence (the union of
         // what the two query tiles visit).  With kPingPong their exponential phases
@@ -792,7 +824,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // ---- mask of a partial tile: keys [beg, cnt) of the tile are visible to this row
         // (positions increase with the local key index, so the visible keys form an
         // interval: up to the row's position, from its document's start)
-        auto mask_bounds = [&](const TileSeq<DOC> &sq, int &cnt, int &beg) {
+        auto mask_bounds = [&](const TileSeq<DOC, NQT> &sq, int &cnt, int &beg) {
             const int k0 = sq.kt * BN;
             cnt = p.kv_len - k0;
             if (cnt > BN) cnt = BN;
@@ -1457,22 +1489,23 @@ bool make_map(CUtensorMap *m, const void *base, int64_t b, int64_t s, int64_t H,
     return r == CUDA_SUCCESS;
 }
 
-template <int D, bool DOC, bool PERSIST>
+template <int D, bool DOC, bool PERSIST, int NQT>
 cudaError_t launch_dd(const AttnParams &p, cudaStream_t stream, const CUtensorMap &tq, const CUtensorMap &tk,
                       const CUtensorMap &tv, const CUtensorMap &to, int o_tma)
 {
+    using C = Cfg<D, NQT>;
     static unsigned long long attr_done = 0;
-    cudaError_t e = set_smem_per_device((const void *)attn_tc_kernel<D, DOC, PERSIST>, Cfg<D>::SMEM, &attr_done);
+    cudaError_t e = set_smem_per_device((const void *)attn_tc_kernel<D, DOC, PERSIST, NQT>, C::SMEM, &attr_done);
     if (e != cudaSuccess) return e;
     const int64_t items = (int64_t)p.n_ranks * p.n_qt * p.b * p.hq;
     if (items == 0) return cudaSuccess;
     if (items > INT32_MAX) return cudaErrorInvalidValue;
     // persistent: one CTA per SM walks the items (one CTA fits an SM); otherwise one per item
     const int64_t grid = PERSIST ? std::min<int64_t>(items, sm_count()) : items;
-    // one CTA per item: the item one wave later (one resident CTA per SM) prefetches its Q
-    const int next_stride = PERSIST ? 0 : sm_count();
-    attn_tc_kernel<D, DOC, PERSIST><<<(unsigned)grid, NTHREADS, Cfg<D>::SMEM, stream>>>(p, tq, tk, tv, to, o_tma,
-                                                                                       next_stride);
+    // one CTA per item: the item one wave later prefetches its Q
+    const int next_stride = PERSIST ? 0 : sm_count() * C::CTAS_PER_SM;
+    attn_tc_kernel<D, DOC, PERSIST, NQT><<<(unsigned)grid, C::NTHR, C::SMEM, stream>>>(p, tq, tk, tv, to, o_tma,
+                                                                                     next_stride);
     return cudaGetLastError();
 }
 
@@ -1493,14 +1526,14 @@ cudaError_t launch_d(const AttnParams &p, cudaStream_t stream, int64_t q_rows, i
         o_tma = 1;
     else
         to = tq;
-    if (p.n_docs > 0) return launch_dd<D, true, kDocPersist>(p, stream, tq, tk, tv, to, o_tma);
-    return launch_dd<D, false, kRingPersist>(p, stream, tq, tk, tv, to, o_tma);
+    if (p.n_docs > 0) return launch_dd<D, true, kDocPersist, kDocNQ>(p, stream, tq, tk, tv, to, o_tma);
+    return launch_dd<D, false, kRingPersist, kRingNQ>(p, stream, tq, tk, tv, to, o_tma);
 }
 
 }  // namespace
 
 // Query rows per CTA of the tensor-core kernel (the work-order table counts these).
-int attn_tc_rows_per_cta() { return NQ * BM; }
+int attn_tc_rows_per_cta(bool doc) { return (doc ? kDocNQ : kRingNQ) * BM; }
 
 cudaError_t launch_attn_tc(const AttnParams &p, cudaStream_t stream)
 {

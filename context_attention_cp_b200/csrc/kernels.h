@@ -79,8 +79,9 @@ struct TensorMaps;  // defined in attn_tc.cu
 // used to build TMA tensor maps.  Returns a cudaError_t.
 cudaError_t launch_attn_tc(const AttnParams &p, cudaStream_t stream);
 
-// Query rows one CTA of the tensor-core kernel covers (the unit of the work order).
-int attn_tc_rows_per_cta();
+// Query rows one CTA of the tensor-core kernel covers (the unit of the work order);
+// doc: the document-mask instantiation.
+int attn_tc_rows_per_cta(bool doc);
 
 // fp32 SIMT path (d in {64, 128}); one CTA covers 128 query rows.
 cudaError_t launch_attn_simt(const AttnParams &p, cudaStream_t stream);
