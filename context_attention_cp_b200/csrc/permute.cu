@@ -81,52 +81,73 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const __grid_constant
     }
 }
 
-// 4-byte rows (the fp32 LSE, sequence last): each thread takes 4 consecutive ranked
-// rows, one 16-byte access on the ranked side; on the original side one 16-byte
-// access when the 4 positions are consecutive and aligned (contiguous and zig-zag
-// chunks), else 4 word accesses (striped).  Needs seq % 4 == 0 and 16-byte bases.
+// 4-byte rows (the fp32 LSE, sequence last): a thread moves groups of 4 consecutive
+// ranked rows, one 16-byte access on the ranked side.  The launcher sends only
+// sequences whose rank length c and zig-zag chunk length c / 2 are multiples of 4, so
+// a group never straddles a rank or a chunk and its positions are pos0 + u * stride,
+// worked out once per group.  On the original side that is one 16-byte access when
+// stride == 1 (contiguous, zig-zag; pos0 is then a multiple of 4) and 4 word accesses
+// when striped.  kWordUnroll groups, a grid-stride apart, are loaded before any of
+// them is stored.
+constexpr int kWordUnroll = 4;
+
 template <typename I>
 __global__ void __launch_bounds__(256) permute_words_kernel(const __grid_constant__ PermuteParams p)
 {
-    // I: int32_t when outer * seq fits (fewer instructions per group), else int64_t
+    // I: int32_t when the group indices with the unrolled strides fit, else int64_t
     const I seq = (I)p.seq;
     const I groups_per_seq = seq / 4;
     const I groups = (I)p.outer * groups_per_seq;
     const I c = seq / p.n_ranks;
+    const I threads = (I)gridDim.x * blockDim.x;
     const uint32_t *src = static_cast<const uint32_t *>(p.src);
     uint32_t *dst = static_cast<uint32_t *>(p.dst);
-    for (I g = (I)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += (I)gridDim.x * blockDim.x) {
-        const I o = g / groups_per_seq;
-        const I rr = (g - o * groups_per_seq) * 4;
-        I pos[4];
+    for (I g0 = (I)blockIdx.x * blockDim.x + threadIdx.x; g0 < groups; g0 += threads * kWordUnroll) {
+        int64_t ranked[kWordUnroll], orig[kWordUnroll];  // word offsets of the group's first row
+        I stride[kWordUnroll];
+        uint4 v[kWordUnroll];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int rank = (int)((rr + u) / c);
+        for (int u = 0; u < kWordUnroll; ++u) {
+            const I g = g0 + (I)u * threads;
+            stride[u] = 0;  // 0: no group here
+            if (g >= groups) continue;
+            const I o = g / groups_per_seq;
+            const I rr = (g - o * groups_per_seq) * 4;
+            const int rank = (int)(rr / c);
             const RangeT<I> r = layout_range_t<I>(p.layout, p.n_ranks, seq, rank);
-            pos[u] = range_pos(r, rr + u - (I)rank * c);
+            const int64_t base = (int64_t)o * seq;
+            ranked[u] = base + rr;
+            orig[u] = base + range_pos(r, rr - (I)rank * c);
+            stride[u] = r.stride;
         }
-        const bool vec = pos[0] % 4 == 0 && pos[1] == pos[0] + 1 && pos[2] == pos[0] + 2 && pos[3] == pos[0] + 3;
-        const int64_t base = (int64_t)o * seq;
-        if (!p.inverse) {
-            uint4 v;
-            if (vec) {
-                v = *reinterpret_cast<const uint4 *>(src + base + pos[0]);
+#pragma unroll
+        for (int u = 0; u < kWordUnroll; ++u) {
+            if (stride[u] == 0) continue;
+            if (p.inverse) {
+                v[u] = *reinterpret_cast<const uint4 *>(src + ranked[u]);
+            } else if (stride[u] == 1) {
+                v[u] = *reinterpret_cast<const uint4 *>(src + orig[u]);
             } else {
-                v.x = src[base + pos[0]];
-                v.y = src[base + pos[1]];
-                v.z = src[base + pos[2]];
-                v.w = src[base + pos[3]];
+                const int64_t s1 = stride[u];
+                v[u].x = src[orig[u]];
+                v[u].y = src[orig[u] + s1];
+                v[u].z = src[orig[u] + 2 * s1];
+                v[u].w = src[orig[u] + 3 * s1];
             }
-            *reinterpret_cast<uint4 *>(dst + base + rr) = v;
-        } else {
-            const uint4 v = *reinterpret_cast<const uint4 *>(src + base + rr);
-            if (vec) {
-                *reinterpret_cast<uint4 *>(dst + base + pos[0]) = v;
+        }
+#pragma unroll
+        for (int u = 0; u < kWordUnroll; ++u) {
+            if (stride[u] == 0) continue;
+            if (!p.inverse) {
+                *reinterpret_cast<uint4 *>(dst + ranked[u]) = v[u];
+            } else if (stride[u] == 1) {
+                *reinterpret_cast<uint4 *>(dst + orig[u]) = v[u];
             } else {
-                dst[base + pos[0]] = v.x;
-                dst[base + pos[1]] = v.y;
-                dst[base + pos[2]] = v.z;
-                dst[base + pos[3]] = v.w;
+                const int64_t s1 = stride[u];
+                dst[orig[u]] = v[u].x;
+                dst[orig[u] + s1] = v[u].y;
+                dst[orig[u] + 2 * s1] = v[u].z;
+                dst[orig[u] + 3 * s1] = v[u].w;
             }
         }
     }
@@ -250,11 +271,17 @@ cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream)
         else permute_rows_kernel<uint8_t><<<(unsigned)blocks, 256, 0, stream>>>(p, n_seg);
         return cudaGetLastError();
     }
-    if (CP_PERMUTE_ROWS && p.inner_bytes == 4 && p.seq % 4 == 0 && al % 16 == 0) {
-        int64_t blocks = (rows / 4 + 255) / 256;
+    const int64_t c_rank = p.n_ranks > 0 ? p.seq / p.n_ranks : 0;
+    const bool groups_aligned = c_rank % 4 == 0 && (p.layout != LAYOUT_ZIGZAG || (c_rank / 2) % 4 == 0);
+    if (CP_PERMUTE_ROWS && p.inner_bytes == 4 && p.seq % 4 == 0 && groups_aligned && al % 16 == 0) {
+        const int64_t groups = rows / 4;
+        int64_t blocks = (groups + 256 * kWordUnroll - 1) / (256 * kWordUnroll);
         if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
-        if (rows + (int64_t)sms * 16 * 256 <= INT32_MAX) permute_words_kernel<int32_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
-        else permute_words_kernel<int64_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        // group indices reach groups + kWordUnroll * (threads in the grid)
+        if (groups + (int64_t)kWordUnroll * blocks * 256 <= INT32_MAX)
+            permute_words_kernel<int32_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        else
+            permute_words_kernel<int64_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
         return cudaGetLastError();
     }
     const int64_t total = rows * per;
