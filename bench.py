@@ -29,8 +29,10 @@ L2 flushed before every timed call):
 With --gpus N > 1 (torchrun, one process per GPU) the ring runs across the N real
 ranks instead (context_attention_cp_b200.ring_dist): each rank holds its layout
 block of the workload (c = S / N tokens) and passes K/V blocks to its neighbour
-with NCCL point-to-point transfers while its block kernel runs.  The total work is
-the workload's, whatever N (strong scaling); the time is the max over ranks.
+with NCCL point-to-point transfers while its block kernel runs; with --ring peer
+the blocks stay where they are and each step's block kernel reads the other rank's
+K/V from its memory (ring_dist.ring_attn_fwd_peer).  The total work is the
+workload's, whatever N (strong scaling); the time is the max over ranks.
 Rank 0 prints one JSON line.
 """
 import argparse
@@ -674,8 +676,17 @@ def run_dist(args, ring_kw=None, device=None, backend="nccl"):
     peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     q, k, v = dist_inputs(w, rank, world, device, torch)
     kw = dict(ring_kw or {})
+    ring = getattr(args, "ring", "nccl")
+    kv = None
+    if ring == "peer":
+        # every rank maps the others' K/V blocks once; the block kernels read them in place
+        kv = ring_dist.PeerBlocks([k.shape, v.shape], k.dtype, device)
+        kv.local[0].copy_(k)
+        kv.local[1].copy_(v)
 
     def step():
+        if kv is not None:
+            return ring_dist.ring_attn_fwd_peer(q, kv, w.layout, w.causal, **kw)
         return ring_dist.ring_attn_fwd_dist(q, k, v, w.layout, w.causal, **kw)
 
     for _ in range(args.warmup):
@@ -719,8 +730,14 @@ def run_dist(args, ring_kw=None, device=None, backend="nccl"):
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record()
     for _ in range(e_steps):
-        qx, kx, vx = (t.to(device, non_blocking=True) for t in (qh, kh, vh))
-        ox, lx = ring_dist.ring_attn_fwd_dist(qx, kx, vx, w.layout, w.causal, **kw)
+        qx = qh.to(device, non_blocking=True)
+        if kv is not None:
+            kv.local[0].copy_(kh, non_blocking=True)
+            kv.local[1].copy_(vh, non_blocking=True)
+            ox, lx = ring_dist.ring_attn_fwd_peer(qx, kv, w.layout, w.causal, **kw)
+        else:
+            kx, vx = (t.to(device, non_blocking=True) for t in (kh, vh))
+            ox, lx = ring_dist.ring_attn_fwd_dist(qx, kx, vx, w.layout, w.causal, **kw)
         ox.cpu(), lx.cpu()
     if cuda:
         f1.record()
@@ -729,6 +746,8 @@ def run_dist(args, ring_kw=None, device=None, backend="nccl"):
     else:
         e_my = (time.perf_counter() - t1) * 1e3
     e_ms = reduce_max(e_my, world, device)
+    if kv is not None:
+        kv.close()
     es = 2 if w.dtype == "bf16" else 4
     h2d = world * (q.numel() + k.numel() + v.numel()) * es
     d2h = world * (q.numel() * es + w.b * w.hq * (w.S // world) * 4)
@@ -742,7 +761,11 @@ def run_dist(args, ring_kw=None, device=None, backend="nccl"):
             "config": {"workload": w.name, "b": w.b, "S": w.S, "hq": w.hq, "hkv": w.hkv, "d": w.d,
                        "layout": w.layout, "N": world, "causal": w.causal,
                        "l2": "inputs exceed L2 (no flush between steps)",
-                       "parallelism": "ring over %d real ranks (K/V blocks passed with NCCL point-to-point)" % world},
+                       "ring": ring,
+                       "parallelism": ("ring over %d real ranks (K/V blocks read in place from the other ranks'"
+                                       " memory by the block kernel)" % world) if ring == "peer" else
+                                      ("ring over %d real ranks (K/V blocks passed with NCCL point-to-point)"
+                                       % world)},
             "pct_bf16_peak": per_gpu / peak_tf,
             "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (block form, one launch per ring step)",
                          "achieved": per_gpu, "peak": peak_tf, "unit": "TFLOP/s", "frac": per_gpu / peak_tf,
@@ -780,6 +803,9 @@ def main():
                     help="comma list of merge,configs,backward,allgather,ulysses; 'all' or 'none'")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=12.0)
+    ap.add_argument("--ring", default="nccl", choices=["nccl", "peer"],
+                    help="with --gpus N > 1: pass the K/V blocks with NCCL (nccl) or read them in place from the"
+                         " other ranks' memory (peer)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":

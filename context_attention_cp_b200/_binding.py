@@ -32,6 +32,10 @@ class CpRange(ctypes.Structure):
                 ("len", ctypes.c_int64 * 2), ("stride", ctypes.c_int64)]
 
 
+class CpPeerHandle(ctypes.Structure):
+    _fields_ = [("ipc", ctypes.c_uint8 * 64), ("offset", ctypes.c_uint64), ("bytes", ctypes.c_uint64)]
+
+
 _T = ctypes.POINTER(CpTensor)
 _R = ctypes.POINTER(CpRange)
 _i32, _i64, _vp, _f32, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
@@ -66,6 +70,9 @@ _SIGNATURES = {
     "cp_stream_check": (_i32, [_vp]),
     "cp_selftest_wait_timeout": (_i32, [ctypes.c_uint64, _vp]),
     "cp_ring_attn_fwd_static_scratch": (_i32, [_i32, _i32, _i32, _T, _T, _T, _f32, _T, _T, _vp]),
+    "cp_peer_export": (_i32, [_vp, ctypes.POINTER(CpPeerHandle)]),
+    "cp_peer_import": (_i32, [ctypes.POINTER(CpPeerHandle), ctypes.POINTER(ctypes.c_void_p)]),
+    "cp_peer_close": (_i32, [ctypes.POINTER(CpPeerHandle)]),
     "cp_status_string": (ctypes.c_char_p, [_i32]),
     "cp_last_error": (ctypes.c_char_p, []),
     "cp_abi_version": (_i32, []),
@@ -431,3 +438,49 @@ def selftest_wait_timeout(limit_ns=20_000_000):
 def stream_check():
     """Synchronise the current stream and raise if a kernel reported a device-side error."""
     _check(lib().cp_stream_check(_stream()))
+
+
+# ------------------------------------------------------------ other ranks' blocks
+
+def peer_export(t):
+    """The handle of CUDA tensor t's memory for other processes, as bytes
+    (cp_peer_export); t must stay allocated while any peer has it mapped."""
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("peer blocks must be contiguous CUDA tensors")
+    h = CpPeerHandle()
+    _check(lib().cp_peer_export(ctypes.c_void_p(t.data_ptr()), ctypes.byref(h)))
+    return bytes(h)
+
+
+class _DeviceArray:
+    """A device address seen through the CUDA array interface (zero copy)."""
+
+    def __init__(self, ptr, shape, typestr):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (ptr, False),
+                                         "version": 3, "strides": None}
+
+
+def peer_import(handle, shape, dtype):
+    """Maps another process's block (handle bytes from peer_export) on the current
+    device (cp_peer_import) and returns a contiguous tensor of `shape` and `dtype`
+    over it, without a copy."""
+    import torch
+    if dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("unsupported dtype %s" % dtype)
+    h = CpPeerHandle.from_buffer_copy(handle)
+    nbytes = torch.Size(shape).numel() * torch.empty((), dtype=dtype).element_size()
+    if nbytes > h.bytes:
+        raise ValueError("the peer block holds %d bytes, %d asked for" % (h.bytes, nbytes))
+    ptr = ctypes.c_void_p()
+    _check(lib().cp_peer_import(ctypes.byref(h), ctypes.byref(ptr)))
+    # no device argument: the tensor stays on the device that holds the memory (a
+    # device argument naming another one would copy)
+    if dtype == torch.bfloat16:
+        return torch.as_tensor(_DeviceArray(ptr.value, shape, "<i2")).view(torch.bfloat16)
+    return torch.as_tensor(_DeviceArray(ptr.value, shape, "<f4"))
+
+
+def peer_close(handle):
+    """Drops one mapping made by peer_import (cp_peer_close)."""
+    h = CpPeerHandle.from_buffer_copy(handle)
+    _check(lib().cp_peer_close(ctypes.byref(h)))

@@ -23,6 +23,15 @@ block is posted before the compute; the accumulators can only leave after it.
 After the last step every accumulator is one hop from its owner, and one more
 exchange brings it home.
 
+ring_attn_fwd_peer runs the same forward schedule without moving any block: the
+ranks of one node map each other's K/V blocks into their own address space once
+(PeerBlocks, CUDA IPC through the library's cp_peer_* calls), and the block kernel
+of step r reads rank (i - r) mod N's K/V straight from that rank's memory with its
+own tile loads -- over NVLink when the rank is another GPU -- so the transfer runs
+inside the kernel, overlapped with the math, and no copy or collective sits on the
+data path.  At each step the N ranks read N different blocks (a permutation), so
+every link carries one block's traffic.
+
 The compute steps can be replaced (`compute=`), which is how the schedules are
 tested on CPU ranks (gloo) without a GPU.
 """
@@ -168,3 +177,116 @@ def ring_attn_bwd_dist(q, k, v, o, lse, do, layout, causal, scale=None, group=No
                 cur_k, cur_v = buf_k, buf_v
         _nvtx_pop(q)
     return dq.to(q.dtype), cur_dk.to(k.dtype), cur_dv.to(v.dtype)
+
+
+class PeerBlocks:
+    """Per-rank device blocks that the kernels of every rank of `group` read in place.
+
+    shapes, dtype, device: this rank's blocks (for the ring: K and V, [b, c, Hkv, d]
+    each).  `local[t]` is this rank's block t, for the caller to write (copy_, or as
+    the output of the step producing K and V); `views[t][j]` is rank j's block t as a
+    tensor of this process (rank j's memory, mapped; this rank's own tensor for
+    j == rank).  Every rank of the group constructs it together.
+
+    Order of use, every rank alike: write `local`, publish() (the writes are finished
+    everywhere), run the kernels that read `views`, release() (those reads are
+    finished everywhere) before `local` is written again; close() at the end.  The
+    ring functions below call publish() and release() themselves.
+
+    CUDA blocks must come from cudaMalloc'd memory (torch's default caching allocator);
+    they are mapped once, here.  CPU blocks (the gloo tests) are gathered by
+    publish() instead of being mapped: the copies stand in for reading the peer."""
+
+    def __init__(self, shapes, dtype, device, group=None):
+        self.group = group
+        self.rank, self.N = dist.get_rank(group), dist.get_world_size(group)
+        self.device = torch.device(device)
+        self.local = [torch.empty(tuple(sh), dtype=dtype, device=self.device) for sh in shapes]
+        self._handles = []
+        if self.device.type != "cuda":
+            self.views = [[t if j == self.rank else torch.empty_like(t) for j in range(self.N)] for t in self.local]
+            return
+        mine = [B.peer_export(t) for t in self.local]
+        everyone = [None] * self.N
+        dist.all_gather_object(everyone, mine, group=group)
+        self.views = [[None] * self.N for _ in self.local]
+        for j, handles in enumerate(everyone):
+            for t, (h, sh) in enumerate(zip(handles, shapes)):
+                if j == self.rank:
+                    self.views[t][j] = self.local[t]
+                else:
+                    self.views[t][j] = B.peer_import(h, tuple(sh), dtype)
+                    self._handles.append(h)
+
+    def publish(self):
+        """Every rank's blocks are written: this rank's queued writes finish, then the
+        ranks meet on the host."""
+        if self.device.type == "cuda":
+            torch.cuda.current_stream(self.device).synchronize()
+        else:
+            for t, row in zip(self.local, self.views):
+                got = [torch.empty_like(t) for _ in range(self.N)]
+                dist.all_gather(got, t, group=self.group)
+                for j in range(self.N):
+                    if j != self.rank:
+                        row[j].copy_(got[j])
+        dist.barrier(group=self.group)
+
+    def release(self):
+        """Every rank's kernels that read the blocks have finished: this rank's queued
+        work finishes, then the ranks meet on the host."""
+        if self.device.type == "cuda":
+            torch.cuda.current_stream(self.device).synchronize()
+        dist.barrier(group=self.group)
+
+    def close(self):
+        """release(), then every rank drops its mappings of the others' blocks before
+        any block is freed."""
+        self.release()
+        for h in self._handles:
+            B.peer_close(h)
+        self._handles = []
+        self.views = None
+        dist.barrier(group=self.group)
+
+
+def ring_attn_fwd_peer(q, kv, layout, causal, scale=None, compute=block_compute, merge=merge_out):
+    """This rank's share of ring attention with the K/V blocks read in place.
+
+    q [b, c, Hq, d]: this rank's local queries (its layout positions, in order);
+    kv: a PeerBlocks over the group whose local blocks 0 and 1 hold this rank's K and
+    V [b, c, Hkv, d], already written.  Returns (o [b, c, Hq, d] in q's dtype, lse
+    [b, Hq, c] fp32) for the local queries.  All ranks of the group call it
+    together.  Step r runs the block kernel on rank (i - r) mod N's blocks where they
+    lie; steps 0 .. N-2 keep the running (o, lse) in fp32 (the block kernel's fused
+    merge from step 1 on), and the last step's partial is folded in by the
+    standalone merge, which writes o in q's dtype.
+    """
+    rank, N = kv.rank, kv.N
+    ks, vs = kv.views[0], kv.views[1]
+    b, c, Hq, d = q.shape
+    if scale is None:
+        scale = 0.0  # the library's default: 1/sqrt(d)
+    S = c * N
+    q_range = B.layout_range(layout, N, S, rank)
+    out = torch.empty((b, c, Hq, d), dtype=q.dtype, device=q.device)
+    lse = torch.empty((b, Hq, c), dtype=torch.float32, device=q.device)
+    kv.publish()
+    if N == 1:
+        compute(q, ks[0], vs[0], q_range, q_range, causal, scale, out, lse, False)
+    else:
+        o = torch.empty((b, c, Hq, d), dtype=torch.float32, device=q.device)
+        for r in range(N):
+            _nvtx_push(q, "peer ring step %d of %d" % (r, N))
+            src = (rank - r) % N                  # the block step r attends to, read where it lies
+            kv_range = B.layout_range(layout, N, S, src)
+            if r + 1 < N:
+                compute(q, ks[src], vs[src], q_range, kv_range, causal, scale, o, lse, r > 0)
+            else:
+                o_b = torch.empty_like(out)
+                lse_b = torch.empty_like(lse)
+                compute(q, ks[src], vs[src], q_range, kv_range, causal, scale, o_b, lse_b, False)
+                merge(o, lse, o_b, lse_b, out)
+            _nvtx_pop(q)
+    kv.release()
+    return out, lse

@@ -411,6 +411,48 @@ const char *cp_last_error(void);
 /* ABI version, bumped on incompatible changes. */
 int32_t cp_abi_version(void);
 
+/* ---- Blocks of other ranks on one node (real ranks, one process per GPU) ----
+ * Section Ring Attention: at ring step r rank i attends its Q to the K/V block that
+ * rank (i - r) mod N started with, and the block travels from rank to rank.  Between
+ * the processes of one node the blocks can stay where they are instead: every rank
+ * maps the other ranks' K/V blocks into its own address space with these calls and
+ * passes the mapped addresses to cp_block_attn_fwd, whose tile loads (plain TMA
+ * loads, no multicast) then read the peer's memory directly -- over NVLink when it
+ * lives on another GPU -- so the transfer overlaps the math inside the kernel and no
+ * copy or collective sits on the data path.
+ *
+ * cp_peer_handle: `ipc` is the CUDA IPC handle of the device allocation holding a
+ * block, `offset` the block's byte offset inside that allocation, `bytes` the bytes
+ * from the block's start to the allocation's end (an upper bound on what may be read
+ * through the mapping).  It is plain bytes: send it to the other processes by any
+ * host channel. */
+typedef struct {
+    uint8_t ipc[64];
+    uint64_t offset;
+    uint64_t bytes;
+} cp_peer_handle;
+
+/* Describes the block at `ptr`: device memory this process allocated with cudaMalloc
+ * (a caching allocator's block inside such an allocation qualifies; memory from
+ * stream-ordered pools or virtual-memory mappings does not and gives CP_ERR_CUDA).
+ * Host-only.  The caller keeps the memory allocated while any peer has it mapped.
+ * Errors: CP_ERR_INVALID_ARG for NULL arguments or a pointer that is not device
+ * memory of this process. */
+cp_status cp_peer_export(const void *ptr, cp_peer_handle *out);
+
+/* Maps the block described by `h`, exported by ANOTHER process, on the current device
+ * and returns its address there in *ptr.  Mappings are counted per (device,
+ * allocation), so several blocks of one allocation map it once.  When the memory
+ * lives on another GPU, peer access from the current device is enabled as needed.
+ * Host-only.  Errors: CP_ERR_CUDA when the driver refuses (a handle exported by this
+ * same process, no peer path between the GPUs, an allocation already freed). */
+cp_status cp_peer_import(const cp_peer_handle *h, void **ptr);
+
+/* Drops one import of `h` on the current device; the allocation is unmapped when its
+ * last import is closed.  The caller makes sure that no queued kernel still reads it.
+ * Errors: CP_ERR_INVALID_ARG when `h` is not mapped on the current device. */
+cp_status cp_peer_close(const cp_peer_handle *h);
+
 /* Bytes of device scratch the library reserves for cp_ring_attn_fwd_static_scratch. */
 #define CP_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
 

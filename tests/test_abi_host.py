@@ -385,3 +385,17 @@ def test_block_bwd_argument_errors_are_synchronous(cp):
     assert call(wsb=8) == 1                                    # workspace too small
     assert call(ws=0x100008) == 1                              # workspace alignment
     assert call(kr_=_range(((0,), (95,), 1))) != 0             # range length differs from the key block
+
+
+def test_peer_calls_reject_null_arguments(cp):
+    """cp_peer_export / cp_peer_import / cp_peer_close refuse NULL arguments before
+    any CUDA call; the handle struct has the layout the header declares."""
+    from context_attention_cp_b200._binding import CpPeerHandle
+    assert ctypes.sizeof(CpPeerHandle) == 64 + 8 + 8
+    h = CpPeerHandle()
+    assert cp.lib().cp_peer_export(None, ctypes.byref(h)) == 1
+    assert cp.lib().cp_peer_export(ctypes.c_void_p(0x1000), None) == 1
+    assert cp.lib().cp_peer_import(None, ctypes.byref(ctypes.c_void_p())) == 1
+    assert cp.lib().cp_peer_import(ctypes.byref(h), None) == 1
+    assert cp.lib().cp_peer_close(None) == 1
+    assert b"NULL" in cp.lib().cp_last_error()

@@ -82,7 +82,7 @@ def test_reference_arm_line_on_rank_zero(monkeypatch, capsys):
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
-def _dist_worker(rank, world, port, out):
+def _dist_worker(rank, world, port, out, ring="nccl"):
     """bench.run_dist on gloo ranks with the oracle as the block and merge steps."""
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -114,6 +114,7 @@ def _dist_worker(rank, world, port, out):
         warmup = 3
         steps = 2
 
+    A.ring = ring
     buf = io.StringIO()
     with contextlib.redirect_stdout(buf):
         rc = bench.run_dist(A(), ring_kw={"compute": step, "merge": _oracle_merge}, device=torch.device("cpu"),
@@ -121,15 +122,17 @@ def _dist_worker(rank, world, port, out):
     out[rank] = (rc, buf.getvalue())
 
 
-def test_run_dist_line_over_two_gloo_ranks():
-    """The --gpus N path of bench.py: every rank runs the real-rank ring on its block,
-    the time is the max over ranks, and rank 0 alone prints one JSON line with the
-    whole workload's throughput (strong scaling)."""
+@pytest.mark.parametrize("ring", ["nccl", "peer"])
+def test_run_dist_line_over_two_gloo_ranks(ring):
+    """The --gpus N path of bench.py: every rank runs the real-rank ring on its block
+    (blocks passed around, or read in place with --ring peer), the time is the max
+    over ranks, and rank 0 alone prints one JSON line with the whole workload's
+    throughput (strong scaling)."""
     import json
-    port = 29550 + os.getpid() % 400
+    port = 29550 + (os.getpid() + 3 * len(ring)) % 400
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.start_processes(_dist_worker, args=(2, port, out), nprocs=2, start_method="spawn", join=True)
+    mp.start_processes(_dist_worker, args=(2, port, out, ring), nprocs=2, start_method="spawn", join=True)
     assert out[0][0] == 0 and out[1][0] == 0
     assert out[1][1].strip() == ""
     lines = [ln for ln in out[0][1].splitlines() if ln.startswith("{")]
@@ -138,3 +141,4 @@ def test_run_dist_line_over_two_gloo_ranks():
     assert d["n_gpus"] == 2 and d["scaling"] == "strong" and d["value"] > 0
     assert d["config"]["workload"] == "fp32_s256_contig2" and d["config"]["N"] == 2
     assert d["e2e"]["h2d_bytes_per_step"] > 0 and d["e2e"]["value"] > 0
+    assert d["config"]["ring"] == ring

@@ -90,3 +90,68 @@ def test_ring_dist_processes_share_one_gpu(layout, world, S):
     for rank, e in errs.items():
         assert e["o"] <= 2e-2 and e["lse"] <= 1e-3, errs          # the bf16 forward bar
         assert max(e["dq"], e["dk"], e["dv"]) <= 2e-2, errs       # the tensor-core backward bar
+
+
+def _peer_worker(rank, world, port, layout, S, out):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import torch.distributed as dist
+
+    import cp_workloads as W
+    import oracle
+    from context_attention_cp_b200 import _binding as B
+    from context_attention_cp_b200 import ring_dist
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        hq, hkv, d = 4, 1, 128
+        q, k, v = W.random_qkv(1, S, hq, hkv, d, "bf16", seed=S + world + 1)
+        pos = torch.tensor(oracle.layout.rank_positions(layout, world, S, rank))
+        ql, kl, vl = (t[:, pos].contiguous() for t in (q, k, v))
+        kv = ring_dist.PeerBlocks([kl.shape, vl.shape], torch.bfloat16, "cuda")
+        # every other rank's block is a mapping of that process's memory, not a copy
+        mapped = all(kv.views[t][j].data_ptr() != kv.local[t].data_ptr()
+                     for t in range(2) for j in range(world) if j != rank)
+        p = pos.numpy()
+        errs = []
+        for k_scale in (1.0, 2.0):  # the blocks rewritten between two calls (x2 is exact in bf16)
+            kv.local[0].copy_((kl * k_scale).cuda())
+            kv.local[1].copy_(vl.cuda())
+            o, lse = ring_dist.ring_attn_fwd_peer(ql.cuda(), kv, layout, True)
+            B.stream_check()
+            want_o, want_l = oracle.attention(q.double().numpy(), k.double().numpy() * k_scale, v.double().numpy(),
+                                              True, d ** -0.5)
+            f = lambda t: t.detach().double().cpu().numpy()  # noqa: E731
+            errs.append((float(np.max(np.abs(f(o) - want_o[:, p]))), float(np.max(np.abs(f(lse) - want_l[:, :, p])))))
+        kv.close()
+        out[rank] = (errs, mapped)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 1024), ("striped", 4, 1024), ("zigzag", 4, 2048)])
+def test_peer_ring_processes_share_one_gpu(layout, world, S):
+    """The in-place ring (ring_dist.ring_attn_fwd_peer): each process maps the other
+    processes' K/V blocks (cp_peer_export / cp_peer_import, CUDA IPC) and its block
+    kernel reads them where they lie; no block is copied or sent.  The processes
+    share cuda:0, so the mapped memory is the same GPU's: this checks the mapping,
+    the schedule and the kernels, not NVLink.  No kernel waits on another process:
+    the ranks meet only on the host (publish / release)."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import torch.multiprocessing as mp
+    port = 29300 + (os.getpid() + world * 13 + S) % 250
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_peer_worker, args=(world, port, layout, S, out), nprocs=world, start_method="spawn",
+                       join=True)
+    assert sorted(out.keys()) == list(range(world))
+    res = dict(out)
+    for rank, (errs, mapped) in res.items():
+        assert mapped, res
+        for err_o, err_l in errs:
+            assert err_o <= 2e-2 and err_l <= 1e-3, res   # the bf16 forward bar

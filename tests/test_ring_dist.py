@@ -216,3 +216,70 @@ def test_ring_in_a_sub_group():
     assert sorted(out.keys()) == [1, 3]
     for rank, errs in out.items():
         assert max(errs) <= 1e-6, (rank, errs)
+
+
+def _peer_worker(rank, world, port, layout, S, out):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import oracle
+    from context_attention_cp_b200 import ring_dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        r = np.random.default_rng(5)
+        b, hq, hkv, d = 1, 4, 2, 8
+        q = r.standard_normal((b, S, hq, d))
+        k = r.standard_normal((b, S, hkv, d))
+        v = r.standard_normal((b, S, hkv, d))
+        pos = np.array(oracle.layout.rank_positions(layout, world, S, rank))
+        ql, kl, vl = (torch.from_numpy(np.ascontiguousarray(t[:, pos])) for t in (q, k, v))
+        seen = []
+
+        def oracle_step(qq, kk, vv, q_range, kv_range, causal, scale, o, lse, accumulate):
+            pk = _positions(kv_range)
+            seen.append(int(pk[0]))
+            ob, lb = oracle.attention(qq.numpy(), kk.numpy(), vv.numpy(), causal, scale,
+                                      pos_q=_positions(q_range), pos_k=pk, nthreads=1)
+            if accumulate:
+                om, lm = oracle.lse_merge(o.numpy().transpose(0, 2, 1, 3), lse.numpy(), ob.transpose(0, 2, 1, 3), lb)
+                ob, lb = om.transpose(0, 2, 1, 3), lm
+            o.copy_(torch.from_numpy(np.ascontiguousarray(ob)))
+            lse.copy_(torch.from_numpy(np.ascontiguousarray(lb)))
+
+        kv = ring_dist.PeerBlocks([kl.shape, vl.shape], kl.dtype, "cpu")
+        errs = []
+        for scale in (0.35, 0.2):             # two calls over the same blocks, rewritten between them
+            kv.local[0].copy_(kl * (scale / 0.35))
+            kv.local[1].copy_(vl)
+            seen.clear()
+            o, lse = ring_dist.ring_attn_fwd_peer(ql, kv, layout, True, 0.35, compute=oracle_step,
+                                                  merge=_oracle_merge)
+            want_o, want_l = oracle.ring_attention(q, k * (scale / 0.35), v, layout, world, True, 0.35, nthreads=1)
+            errs.append((float(np.max(np.abs(o.numpy() - want_o[:, pos]))),
+                         float(np.max(np.abs(lse.numpy() - want_l[:, :, pos])))))
+        kv.close()
+        out[rank] = (errs, seen,
+                     [int(oracle.layout.rank_positions(layout, world, S, (rank - s) % world)[0]) for s in range(world)])
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 32), ("striped", 3, 24), ("zigzag", 4, 64)])
+def test_peer_ring_over_gloo_ranks(layout, world, S):
+    """The in-place ring (ring_attn_fwd_peer): no block moves between steps; step r
+    reads rank (i - r) mod N's K/V block where it lies (on CPU ranks the blocks are
+    gathered by PeerBlocks.publish, standing in for the mapping), twice over blocks
+    rewritten between the calls."""
+    port = 29550 + (os.getpid() + world * 5 + S) % 900
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_peer_worker, args=(world, port, layout, S, out), nprocs=world, start_method="spawn",
+                       join=True)
+    assert sorted(out.keys()) == list(range(world))
+    for rank, (errs, seen, want_seen) in out.items():
+        for err_o, err_l in errs:
+            assert err_o <= 1e-6 and err_l <= 1e-6, (rank, errs)
+        assert seen == want_seen, (rank, seen, want_seen)
