@@ -21,7 +21,9 @@ Entry points mirror include/cpattn.h:
   tile_classes(q_range, q_len, kv_range, kv_len, causal, tile_q, tile_k)
   stream_check()
 The real-rank ring (one process per GPU, K/V passed with torch.distributed
-point-to-point transfers) lives in context_attention_cp_b200.ring_dist.
+point-to-point transfers, or read in place from the other ranks' memory with
+PeerBlocks / ring_attn_fwd_peer) lives in context_attention_cp_b200.ring_dist;
+peer_export / peer_import / peer_close map another process's device block.
 Tensors are torch tensors on the current CUDA device; token tensors are
 [b, s, H, d] with d contiguous, lse tensors [b, H, s] fp32.
 """
@@ -30,5 +32,5 @@ from ._binding import (  # noqa: F401
     layout_range, lib, lib_path,
     lse_merge, ring_attn_bwd, ring_attn_fwd, ring_attn_fwd_static_scratch, ring_bwd_workspace_bytes,
     ring_workspace_bytes, selftest_wait_timeout, stream_check, tile_classes, ulysses_all_to_all, ulysses_attn_bwd, ulysses_attn_fwd,
-    ulysses_workspace_bytes, usp_attn_bwd, usp_attn_fwd, usp_workspace_bytes,
+    ulysses_workspace_bytes, usp_attn_bwd, usp_attn_fwd, usp_workspace_bytes, peer_close, peer_export, peer_import,
 )
