@@ -30,7 +30,10 @@ of step r reads rank (i - r) mod N's K/V straight from that rank's memory with i
 own tile loads -- over NVLink when the rank is another GPU -- so the transfer runs
 inside the kernel, overlapped with the math, and no copy or collective sits on the
 data path.  At each step the N ranks read N different blocks (a permutation), so
-every link carries one block's traffic.
+every link carries one block's traffic.  ring_attn_bwd_peer does the same for the
+backward: step r adds rank i's shares for block (i - r) mod N into that block
+owner's fp32 dK, dV accumulators where they lie, with a host barrier between steps
+so that each accumulator has one writer at a time.
 
 The compute steps can be replaced (`compute=`), which is how the schedules are
 tested on CPU ranks (gloo) without a GPU.
@@ -180,64 +183,80 @@ def ring_attn_bwd_dist(q, k, v, o, lse, do, layout, causal, scale=None, group=No
 
 
 class PeerBlocks:
-    """Per-rank device blocks that the kernels of every rank of `group` read in place.
+    """Per-rank blocks that the kernels of every rank of `group` read and write in place.
 
     shapes, dtype, device: this rank's blocks (for the ring: K and V, [b, c, Hkv, d]
-    each).  `local[t]` is this rank's block t, for the caller to write (copy_, or as
-    the output of the step producing K and V); `views[t][j]` is rank j's block t as a
-    tensor of this process (rank j's memory, mapped; this rank's own tensor for
-    j == rank).  Every rank of the group constructs it together.
+    each; or the fp32 dK, dV accumulators).  `local[t]` is this rank's block t, for
+    the caller to write (copy_, or as the output of the step producing it);
+    `views[t][j]` is rank j's block t as a tensor of this process -- rank j's memory,
+    mapped, not a copy (this rank's own tensor for j == rank).  Every rank of the
+    group constructs it together.
 
     Order of use, every rank alike: write `local`, publish() (the writes are finished
-    everywhere), run the kernels that read `views`, release() (those reads are
-    finished everywhere) before `local` is written again; close() at the end.  The
-    ring functions below call publish() and release() themselves.
+    everywhere), run the kernels that use `views`, release() (that work is finished
+    everywhere) before a block is written again; close() at the end.  The ring
+    functions below call publish() and release() themselves.
 
-    CUDA blocks must come from cudaMalloc'd memory (torch's default caching allocator);
-    they are mapped once, here.  CPU blocks (the gloo tests) are gathered by
-    publish() instead of being mapped: the copies stand in for reading the peer."""
+    CUDA blocks come from torch's caching allocator (cudaMalloc'd memory) and are
+    mapped with cp_peer_export / cp_peer_import, once, here.  CPU blocks (the gloo
+    tests) live in POSIX shared memory opened by every rank, so a peer's view is the
+    same memory there too."""
 
     def __init__(self, shapes, dtype, device, group=None):
         self.group = group
         self.rank, self.N = dist.get_rank(group), dist.get_world_size(group)
         self.device = torch.device(device)
-        self.local = [torch.empty(tuple(sh), dtype=dtype, device=self.device) for sh in shapes]
-        self._handles = []
-        if self.device.type != "cuda":
-            self.views = [[t if j == self.rank else torch.empty_like(t) for j in range(self.N)] for t in self.local]
-            return
-        mine = [B.peer_export(t) for t in self.local]
+        self._handles, self._shm = [], []
+        shapes = [tuple(sh) for sh in shapes]
+        if self.device.type == "cuda":
+            self.local = [torch.empty(sh, dtype=dtype, device=self.device) for sh in shapes]
+            mine = [B.peer_export(t) for t in self.local]
+        else:
+            self.local, mine = [], []
+            for sh in shapes:
+                t, name = self._shared_cpu(sh, dtype, None)
+                self.local.append(t)
+                mine.append(name)
         everyone = [None] * self.N
         dist.all_gather_object(everyone, mine, group=group)
-        self.views = [[None] * self.N for _ in self.local]
+        self.views = [[None] * self.N for _ in shapes]
         for j, handles in enumerate(everyone):
             for t, (h, sh) in enumerate(zip(handles, shapes)):
                 if j == self.rank:
                     self.views[t][j] = self.local[t]
-                else:
-                    self.views[t][j] = B.peer_import(h, tuple(sh), dtype)
+                elif self.device.type == "cuda":
+                    self.views[t][j] = B.peer_import(h, sh, dtype)
                     self._handles.append(h)
+                else:
+                    self.views[t][j] = self._shared_cpu(sh, dtype, h)[0]
+
+    def _shared_cpu(self, shape, dtype, name):
+        """A CPU tensor in POSIX shared memory: a new segment (name None) or the
+        segment another rank made."""
+        from multiprocessing import resource_tracker, shared_memory
+        nbytes = max(1, torch.Size(shape).numel() * torch.empty((), dtype=dtype).element_size())
+        if name is None:
+            shm = shared_memory.SharedMemory(create=True, size=nbytes)
+        else:
+            shm = shared_memory.SharedMemory(name=name)
+            resource_tracker.unregister(shm._name, "shared_memory")  # the creating rank unlinks it
+        self._shm.append((shm, name is None))
+        return torch.frombuffer(shm.buf, dtype=dtype, count=torch.Size(shape).numel()).view(shape), shm.name
+
+    def _sync(self):
+        if self.device.type == "cuda":
+            torch.cuda.current_stream(self.device).synchronize()
+        dist.barrier(group=self.group)
 
     def publish(self):
-        """Every rank's blocks are written: this rank's queued writes finish, then the
+        """Every rank's blocks are written: this rank's queued work finishes, then the
         ranks meet on the host."""
-        if self.device.type == "cuda":
-            torch.cuda.current_stream(self.device).synchronize()
-        else:
-            for t, row in zip(self.local, self.views):
-                got = [torch.empty_like(t) for _ in range(self.N)]
-                dist.all_gather(got, t, group=self.group)
-                for j in range(self.N):
-                    if j != self.rank:
-                        row[j].copy_(got[j])
-        dist.barrier(group=self.group)
+        self._sync()
 
     def release(self):
-        """Every rank's kernels that read the blocks have finished: this rank's queued
-        work finishes, then the ranks meet on the host."""
-        if self.device.type == "cuda":
-            torch.cuda.current_stream(self.device).synchronize()
-        dist.barrier(group=self.group)
+        """Every rank's work on the blocks is finished: this rank's queued work
+        finishes, then the ranks meet on the host."""
+        self._sync()
 
     def close(self):
         """release(), then every rank drops its mappings of the others' blocks before
@@ -247,7 +266,16 @@ class PeerBlocks:
             B.peer_close(h)
         self._handles = []
         self.views = None
+        self.local = None
         dist.barrier(group=self.group)
+        for shm, owner in self._shm:
+            try:
+                shm.close()
+            except BufferError:  # a caller still holds a view; the mapping goes at exit
+                pass
+            if owner:
+                shm.unlink()
+        self._shm = []
 
 
 def ring_attn_fwd_peer(q, kv, layout, causal, scale=None, compute=block_compute, merge=merge_out):
@@ -290,3 +318,47 @@ def ring_attn_fwd_peer(q, kv, layout, causal, scale=None, compute=block_compute,
             _nvtx_pop(q)
     kv.release()
     return out, lse
+
+
+def ring_attn_bwd_peer(q, kv, o, lse, do, layout, causal, scale=None, acc=None, compute=block_bwd_compute):
+    """This rank's gradients of ring attention with every block left in place.
+
+    q, o, do [b, c, Hq, d]: this rank's local blocks; o and lse [b, Hq, c] are this
+    rank's results of the whole-sequence forward (for example ring_attn_fwd_peer);
+    kv: the PeerBlocks holding every rank's K and V (blocks 0 and 1), already
+    written; acc: a PeerBlocks of two blocks shaped like K and V in the accumulation
+    dtype (fp32 for the kernels) over the same group, reused across calls (made and
+    closed here when None).  Returns (dq, dk, dv) in q's / k's dtype for this
+    rank's blocks.  All ranks of the group call it together.
+
+    Step r: rank i adds its queries' shares for block j = (i - r) mod N into its own
+    dQ and into rank j's dK, dV accumulators, in rank j's memory (the block backward
+    adds with plain fp32 loads and stores).  The ranks meet on the host after every
+    step, so at every step each accumulator has exactly one writer, and the
+    accumulators never travel."""
+    rank, N = kv.rank, kv.N
+    ks, vs = kv.views[0], kv.views[1]
+    b, c, Hq, d = q.shape
+    if scale is None:
+        scale = 0.0  # the library's default: 1/sqrt(d)
+    S = c * N
+    q_range = B.layout_range(layout, N, S, rank)
+    own_acc = acc is None
+    if own_acc:
+        acc = PeerBlocks([ks[rank].shape, vs[rank].shape], torch.float32, q.device, kv.group)
+    acc.local[0].zero_()
+    acc.local[1].zero_()
+    dq = torch.zeros(q.shape, dtype=acc.local[0].dtype, device=q.device)
+    kv.publish()                                  # K, V written and the accumulators zeroed everywhere
+    for r in range(N):
+        _nvtx_push(q, "peer ring backward step %d of %d" % (r, N))
+        src = (rank - r) % N                      # the block step r works on, where it lies
+        compute(q, ks[src], vs[src], o, lse, do, q_range, B.layout_range(layout, N, S, src), causal, scale, dq,
+                acc.views[0][src], acc.views[1][src])
+        acc.release()                             # this step's adds are finished everywhere
+        _nvtx_pop(q)
+    dk = acc.local[0].to(ks[rank].dtype, copy=True)  # a copy: the accumulators stay with `acc`
+    dv = acc.local[1].to(vs[rank].dtype, copy=True)
+    if own_acc:
+        acc.close()
+    return dq.to(q.dtype), dk, dv

@@ -109,25 +109,34 @@ def _peer_worker(rank, world, port, layout, S, out):
     try:
         hq, hkv, d = 4, 1, 128
         q, k, v = W.random_qkv(1, S, hq, hkv, d, "bf16", seed=S + world + 1)
+        do = W.random_do(1, S, hq, d, "bf16", seed=S + world + 1)
         pos = torch.tensor(oracle.layout.rank_positions(layout, world, S, rank))
-        ql, kl, vl = (t[:, pos].contiguous() for t in (q, k, v))
+        ql, kl, vl, dol = (t[:, pos].contiguous() for t in (q, k, v, do))
         kv = ring_dist.PeerBlocks([kl.shape, vl.shape], torch.bfloat16, "cuda")
+        acc = ring_dist.PeerBlocks([kl.shape, vl.shape], torch.float32, "cuda")
         # every other rank's block is a mapping of that process's memory, not a copy
         mapped = all(kv.views[t][j].data_ptr() != kv.local[t].data_ptr()
                      for t in range(2) for j in range(world) if j != rank)
         p = pos.numpy()
-        errs = []
+        errs, gerrs = [], []
+        f = lambda t: t.detach().double().cpu().numpy()  # noqa: E731
         for k_scale in (1.0, 2.0):  # the blocks rewritten between two calls (x2 is exact in bf16)
             kv.local[0].copy_((kl * k_scale).cuda())
             kv.local[1].copy_(vl.cuda())
             o, lse = ring_dist.ring_attn_fwd_peer(ql.cuda(), kv, layout, True)
             B.stream_check()
-            want_o, want_l = oracle.attention(q.double().numpy(), k.double().numpy() * k_scale, v.double().numpy(),
-                                              True, d ** -0.5)
-            f = lambda t: t.detach().double().cpu().numpy()  # noqa: E731
+            k64 = k.double().numpy() * k_scale
+            want_o, want_l = oracle.attention(q.double().numpy(), k64, v.double().numpy(), True, d ** -0.5)
             errs.append((float(np.max(np.abs(f(o) - want_o[:, p]))), float(np.max(np.abs(f(lse) - want_l[:, :, p])))))
+            # the backward adds into the owners' dK, dV accumulators where they lie
+            dq, dk, dv = ring_dist.ring_attn_bwd_peer(ql.cuda(), kv, o, lse, dol.cuda(), layout, True, acc=acc)
+            B.stream_check()
+            wg = oracle.attention_bwd(q.double().numpy(), k64, v.double().numpy(), do.double().numpy(), True,
+                                      d ** -0.5)[:3]
+            gerrs.append([float(np.max(np.abs(f(g) - w[:, p])) / np.max(np.abs(w))) for g, w in zip((dq, dk, dv), wg)])
+        acc.close()
         kv.close()
-        out[rank] = (errs, mapped)
+        out[rank] = (errs, gerrs, mapped)
         dist.barrier()
     finally:
         dist.destroy_process_group()
@@ -135,9 +144,10 @@ def _peer_worker(rank, world, port, layout, S, out):
 
 @pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 1024), ("striped", 4, 1024), ("zigzag", 4, 2048)])
 def test_peer_ring_processes_share_one_gpu(layout, world, S):
-    """The in-place ring (ring_dist.ring_attn_fwd_peer): each process maps the other
-    processes' K/V blocks (cp_peer_export / cp_peer_import, CUDA IPC) and its block
-    kernel reads them where they lie; no block is copied or sent.  The processes
+    """The in-place ring (ring_dist.ring_attn_fwd_peer, ring_attn_bwd_peer): each
+    process maps the other processes' K/V blocks and dK/dV accumulators
+    (cp_peer_export / cp_peer_import, CUDA IPC); its block kernels read the K/V and
+    add into the accumulators where they lie; no block is copied or sent.  The processes
     share cuda:0, so the mapped memory is the same GPU's: this checks the mapping,
     the schedule and the kernels, not NVLink.  No kernel waits on another process:
     the ranks meet only on the host (publish / release)."""
@@ -151,7 +161,9 @@ def test_peer_ring_processes_share_one_gpu(layout, world, S):
                        join=True)
     assert sorted(out.keys()) == list(range(world))
     res = dict(out)
-    for rank, (errs, mapped) in res.items():
+    for rank, (errs, gerrs, mapped) in res.items():
         assert mapped, res
         for err_o, err_l in errs:
             assert err_o <= 2e-2 and err_l <= 1e-3, res   # the bf16 forward bar
+        for g in gerrs:
+            assert max(g) <= 2e-2, res                    # the tensor-core backward bar

@@ -270,9 +270,9 @@ def _peer_worker(rank, world, port, layout, S, out):
 @pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 32), ("striped", 3, 24), ("zigzag", 4, 64)])
 def test_peer_ring_over_gloo_ranks(layout, world, S):
     """The in-place ring (ring_attn_fwd_peer): no block moves between steps; step r
-    reads rank (i - r) mod N's K/V block where it lies (on CPU ranks the blocks are
-    gathered by PeerBlocks.publish, standing in for the mapping), twice over blocks
-    rewritten between the calls."""
+    reads rank (i - r) mod N's K/V block where it lies (on CPU ranks the blocks live
+    in shared memory that every rank opens, standing in for the device mapping),
+    twice over blocks rewritten between the calls."""
     port = 29550 + (os.getpid() + world * 5 + S) % 900
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
@@ -282,4 +282,77 @@ def test_peer_ring_over_gloo_ranks(layout, world, S):
     for rank, (errs, seen, want_seen) in out.items():
         for err_o, err_l in errs:
             assert err_o <= 1e-6 and err_l <= 1e-6, (rank, errs)
+        assert seen == want_seen, (rank, seen, want_seen)
+
+
+def _peer_bwd_worker(rank, world, port, layout, S, causal, out):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import oracle
+    from context_attention_cp_b200 import ring_dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        r = np.random.default_rng(13)
+        b, hq, hkv, d = 1, 4, 2, 8
+        q = r.standard_normal((b, S, hq, d))
+        k = r.standard_normal((b, S, hkv, d))
+        v = r.standard_normal((b, S, hkv, d))
+        do = r.standard_normal((b, S, hq, d))
+        o_full, lse_full = oracle.attention(q, k, v, causal, 0.35, nthreads=1)
+        pos = np.array(oracle.layout.rank_positions(layout, world, S, rank))
+        loc = lambda t: torch.from_numpy(np.ascontiguousarray(t[:, pos]))  # noqa: E731
+        ql, kl, vl, dol, ol = (loc(t) for t in (q, k, v, do, o_full))
+        lsel = torch.from_numpy(np.ascontiguousarray(lse_full[:, :, pos]))
+        seen = []
+
+        def oracle_step(qq, kk, vv, oo, ll, gg, q_range, kv_range, causal, scale, dq, dk, dv):
+            pk = _positions(kv_range)
+            seen.append(int(pk[0]))
+            delta = np.einsum("bshd,bshd->bhs", gg.numpy(), oo.numpy())
+            a, bk, bv, _, _ = oracle.attention_bwd(qq.numpy(), kk.numpy(), vv.numpy(), gg.numpy(), causal, scale,
+                                                   pos_q=_positions(q_range), pos_k=pk, lse=ll.numpy(), delta=delta,
+                                                   nthreads=1)
+            dq += torch.from_numpy(a)
+            dk += torch.from_numpy(bk)   # the owner's accumulator, in shared memory
+            dv += torch.from_numpy(bv)
+
+        kv = ring_dist.PeerBlocks([kl.shape, vl.shape], kl.dtype, "cpu")
+        acc = ring_dist.PeerBlocks([kl.shape, vl.shape], torch.float64, "cpu")
+        kv.local[0].copy_(kl)
+        kv.local[1].copy_(vl)
+        want = oracle.attention_bwd(q, k, v, do, causal, 0.35, nthreads=1)[:3]
+        errs = []
+        for _ in range(2):                       # the accumulators reused by a second call
+            seen.clear()
+            dq, dk, dv = ring_dist.ring_attn_bwd_peer(ql, kv, ol, lsel, dol, layout, causal, 0.35, acc=acc,
+                                                      compute=oracle_step)
+            errs.append([float(np.max(np.abs(g.numpy() - w[:, pos]))) for g, w in zip((dq, dk, dv), want)])
+        acc.close()
+        kv.close()
+        out[rank] = (errs, seen,
+                     [int(oracle.layout.rank_positions(layout, world, S, (rank - s) % world)[0]) for s in range(world)])
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("layout,world,S,causal", [("zigzag", 2, 32, True), ("striped", 3, 24, True),
+                                                   ("zigzag", 4, 64, True), ("contiguous", 3, 24, False)])
+def test_peer_ring_backward_over_gloo_ranks(layout, world, S, causal):
+    """The in-place backward (ring_attn_bwd_peer): step r adds rank i's shares for
+    block (i - r) mod N into that block owner's dK, dV accumulators where they lie
+    (shared memory on CPU ranks); the gradients of every rank equal the oracle's
+    whole-sequence gradients, twice with the accumulators reused."""
+    port = 29450 + (os.getpid() + world * 17 + S + int(causal)) % 900
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_peer_bwd_worker, args=(world, port, layout, S, causal, out), nprocs=world,
+                       start_method="spawn", join=True)
+    assert sorted(out.keys()) == list(range(world))
+    for rank, (errs, seen, want_seen) in out.items():
+        for e in errs:
+            assert max(e) <= 1e-9, (rank, errs)
         assert seen == want_seen, (rank, seen, want_seen)
