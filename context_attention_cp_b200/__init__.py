@@ -23,7 +23,8 @@ Entry points mirror include/cpattn.h:
 The real-rank ring (one process per GPU, K/V passed with torch.distributed
 point-to-point transfers, or read in place from the other ranks' memory with
 PeerBlocks / ring_attn_fwd_peer) lives in context_attention_cp_b200.ring_dist;
-peer_export / peer_import / peer_close map another process's device block.
+peer_export / peer_import / peer_close map another process's device block, peer_copy
+pulls one into local memory.
 Tensors are torch tensors on the current CUDA device; token tensors are
 [b, s, H, d] with d contiguous, lse tensors [b, H, s] fp32.
 """
@@ -32,5 +33,5 @@ from ._binding import (  # noqa: F401
     layout_range, lib, lib_path,
     lse_merge, ring_attn_bwd, ring_attn_fwd, ring_attn_fwd_static_scratch, ring_bwd_workspace_bytes,
     ring_workspace_bytes, selftest_wait_timeout, stream_check, tile_classes, ulysses_all_to_all, ulysses_attn_bwd, ulysses_attn_fwd,
-    ulysses_workspace_bytes, usp_attn_bwd, usp_attn_fwd, usp_workspace_bytes, peer_close, peer_export, peer_import,
+    ulysses_workspace_bytes, usp_attn_bwd, usp_attn_fwd, usp_workspace_bytes, peer_close, peer_copy, peer_export, peer_import,
 )

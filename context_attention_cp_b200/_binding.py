@@ -73,6 +73,7 @@ _SIGNATURES = {
     "cp_peer_export": (_i32, [_vp, ctypes.POINTER(CpPeerHandle)]),
     "cp_peer_import": (_i32, [ctypes.POINTER(CpPeerHandle), ctypes.POINTER(ctypes.c_void_p)]),
     "cp_peer_close": (_i32, [ctypes.POINTER(CpPeerHandle)]),
+    "cp_peer_copy": (_i32, [_vp, _vp, _sz, _vp]),
     "cp_status_string": (ctypes.c_char_p, [_i32]),
     "cp_last_error": (ctypes.c_char_p, []),
     "cp_abi_version": (_i32, []),
@@ -484,3 +485,13 @@ def peer_close(handle):
     """Drops one mapping made by peer_import (cp_peer_close)."""
     h = CpPeerHandle.from_buffer_copy(handle)
     _check(lib().cp_peer_close(ctypes.byref(h)))
+
+
+def peer_copy(dst, src):
+    """Copies contiguous tensor src (for example a block from peer_import) into dst, on
+    the current stream, with the copy engines (cp_peer_copy)."""
+    if not (dst.is_contiguous() and src.is_contiguous()) or dst.dtype != src.dtype or dst.shape != src.shape:
+        raise ValueError("peer_copy needs contiguous tensors of one shape and dtype")
+    nbytes = dst.numel() * dst.element_size()
+    _check(lib().cp_peer_copy(ctypes.c_void_p(dst.data_ptr()), ctypes.c_void_p(src.data_ptr()), nbytes, _stream()))
+    return dst

@@ -2,11 +2,13 @@
 //
 // "上下文并行与 Ring Attention" (hs-black.github.io), section Ring Attention: at
 // step r rank i attends its Q to the K/V block that rank (i - r) mod N started
-// with.  Between the processes of one node the blocks need not travel: every rank
-// maps the others' blocks into its own address space once, and the block kernel
-// of step r reads rank (i - r) mod N's K/V straight from that rank's memory with
-// its ordinary (non-multicast) TMA tile loads, so the transfer over NVLink happens
-// inside the kernel, tile by tile, overlapped with the math.
+// with.  Between the processes of one node nobody needs to send: every rank maps
+// the others' blocks into its own address space once; at step r it pulls rank
+// (i - r) mod N's block across the link (the forward copies it one step ahead
+// into a local buffer with the copy engines, so it crosses once however many CTAs
+// read it), or works on it where it lies (the backward's key-tile CTAs read each
+// K/V tile once and add their dK, dV shares into the owner's accumulator with
+// plain loads and stores).  No load anywhere uses cluster multicast.
 //
 // cp_peer_export describes a block (the IPC handle of the allocation holding it and
 // the block's offset in that allocation); the handle bytes go to the other ranks
@@ -14,6 +16,9 @@
 // (lazily enabling peer access when it lives on another GPU) and returns the
 // block's address there; cp_peer_close drops the mapping.  Mappings are counted
 // per (device, allocation), so blocks that share an allocation map it once.
+// cp_peer_copy pulls a mapped block into this GPU's memory with the copy engines,
+// for readers that would otherwise cross the link many times (every query-tile CTA
+// of the forward reads every K/V tile of the block).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -125,5 +130,14 @@ extern "C" cp_status cp_peer_close(const cp_peer_handle *h)
     g_peer_maps.erase(it);
     if (e != cudaSuccess)
         return cpattn::report_error(CP_ERR_CUDA, "cudaIpcCloseMemHandle: %s", cudaGetErrorString(e));
+    return CP_OK;
+}
+
+extern "C" cp_status cp_peer_copy(void *dst, const void *src, size_t bytes, void *stream)
+{
+    if (bytes == 0) return CP_OK;
+    if (!dst || !src) return cpattn::report_error(CP_ERR_INVALID_ARG, "dst or src is NULL");
+    cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cpattn::report_error(CP_ERR_CUDA, "cudaMemcpyAsync: %s", cudaGetErrorString(e));
     return CP_OK;
 }

@@ -23,14 +23,13 @@ block is posted before the compute; the accumulators can only leave after it.
 After the last step every accumulator is one hop from its owner, and one more
 exchange brings it home.
 
-ring_attn_fwd_peer runs the same forward schedule without moving any block: the
-ranks of one node map each other's K/V blocks into their own address space once
-(PeerBlocks, CUDA IPC through the library's cp_peer_* calls), and the block kernel
-of step r reads rank (i - r) mod N's K/V straight from that rank's memory with its
-own tile loads -- over NVLink when the rank is another GPU -- so the transfer runs
-inside the kernel, overlapped with the math, and no copy or collective sits on the
-data path.  At each step the N ranks read N different blocks (a permutation), so
-every link carries one block's traffic.  ring_attn_bwd_peer does the same for the
+ring_attn_fwd_peer runs the same forward schedule with no rank sending: the ranks
+of one node map each other's K/V blocks into their own address space once
+(PeerBlocks, CUDA IPC through the library's cp_peer_* calls), and step r pulls rank
+(i - r) mod N's block into a local buffer one step ahead with the copy engines,
+overlapped with the step before (or, with stage=False, the block kernel reads it
+where it lies).  No collective sits on the data path.  At each step the N ranks
+pull N different blocks (a permutation), so every link carries one block.  ring_attn_bwd_peer does the same for the
 backward: step r adds rank i's shares for block (i - r) mod N into that block
 owner's fp32 dK, dV accumulators where they lie, with a host barrier between steps
 so that each accumulator has one writer at a time.
@@ -278,17 +277,24 @@ class PeerBlocks:
         self._shm = []
 
 
-def ring_attn_fwd_peer(q, kv, layout, causal, scale=None, compute=block_compute, merge=merge_out):
-    """This rank's share of ring attention with the K/V blocks read in place.
+def ring_attn_fwd_peer(q, kv, layout, causal, scale=None, stage=True, compute=block_compute, merge=merge_out):
+    """This rank's share of ring attention over blocks that no rank sends.
 
     q [b, c, Hq, d]: this rank's local queries (its layout positions, in order);
     kv: a PeerBlocks over the group whose local blocks 0 and 1 hold this rank's K and
     V [b, c, Hkv, d], already written.  Returns (o [b, c, Hq, d] in q's dtype, lse
     [b, Hq, c] fp32) for the local queries.  All ranks of the group call it
-    together.  Step r runs the block kernel on rank (i - r) mod N's blocks where they
-    lie; steps 0 .. N-2 keep the running (o, lse) in fp32 (the block kernel's fused
-    merge from step 1 on), and the last step's partial is folded in by the
-    standalone merge, which writes o in q's dtype.
+    together.
+
+    Step r attends to rank (i - r) mod N's block.  stage=True pulls that block into
+    one of two local buffers one step ahead, on a copy stream with the copy engines
+    (cp_peer_copy), while the block kernel of the step before runs: every CTA of the
+    forward reads every K/V tile of the block, so reading the peer in place would
+    carry each tile across the link once per reading CTA.  stage=False runs the block
+    kernel on the peer's memory directly (the same GPU's memory when the ranks share
+    one, as in the tests).  Steps 0 .. N-2 keep the running (o, lse) in fp32 (the
+    block kernel's fused merge from step 1 on), and the last step's partial is
+    folded in by the standalone merge, which writes o in q's dtype.
     """
     rank, N = kv.rank, kv.N
     ks, vs = kv.views[0], kv.views[1]
@@ -302,20 +308,61 @@ def ring_attn_fwd_peer(q, kv, layout, causal, scale=None, compute=block_compute,
     kv.publish()
     if N == 1:
         compute(q, ks[0], vs[0], q_range, q_range, causal, scale, out, lse, False)
-    else:
-        o = torch.empty((b, c, Hq, d), dtype=torch.float32, device=q.device)
-        for r in range(N):
-            _nvtx_push(q, "peer ring step %d of %d" % (r, N))
-            src = (rank - r) % N                  # the block step r attends to, read where it lies
-            kv_range = B.layout_range(layout, N, S, src)
+        kv.release()
+        return out, lse
+    cuda = q.is_cuda
+    if stage:
+        # steps 1 .. N-1 read block (rank - r) mod N from buffer (r - 1) % n_buf
+        n_buf = min(2, N - 1)
+        bufs = [(torch.empty_like(ks[rank]), torch.empty_like(vs[rank])) for _ in range(n_buf)]
+        if cuda:
+            main, side = torch.cuda.current_stream(), torch.cuda.Stream()
+            fetched = [torch.cuda.Event() for _ in range(n_buf)]
+            used = [torch.cuda.Event() for _ in range(n_buf)]
+
+    def fetch(r):
+        """Pull block (rank - r) mod N into its buffer, after the step that last read
+        that buffer (step r - n_buf) is done with it."""
+        src, slot = (rank - r) % N, (r - 1) % n_buf
+        if not cuda:
+            bufs[slot][0].copy_(ks[src])
+            bufs[slot][1].copy_(vs[src])
+            return
+        with torch.cuda.stream(side):
+            if r - n_buf >= 1:
+                side.wait_event(used[slot])
+            B.peer_copy(bufs[slot][0], ks[src])
+            B.peer_copy(bufs[slot][1], vs[src])
+            fetched[slot].record(side)
+
+    o = torch.empty((b, c, Hq, d), dtype=torch.float32, device=q.device)
+    if stage:
+        fetch(1)
+    for r in range(N):
+        _nvtx_push(q, "peer ring step %d of %d" % (r, N))
+        src = (rank - r) % N                      # the block step r attends to
+        kv_range = B.layout_range(layout, N, S, src)
+        if r == 0 or not stage:
+            kk, vv = ks[src], vs[src]             # the local block, or the peer's where it lies
+        else:
+            slot = (r - 1) % n_buf
+            if cuda:
+                main.wait_event(fetched[slot])
+            kk, vv = bufs[slot]
             if r + 1 < N:
-                compute(q, ks[src], vs[src], q_range, kv_range, causal, scale, o, lse, r > 0)
-            else:
-                o_b = torch.empty_like(out)
-                lse_b = torch.empty_like(lse)
-                compute(q, ks[src], vs[src], q_range, kv_range, causal, scale, o_b, lse_b, False)
-                merge(o, lse, o_b, lse_b, out)
-            _nvtx_pop(q)
+                fetch(r + 1)                      # the next block comes in while this step runs
+        if r + 1 < N:
+            compute(q, kk, vv, q_range, kv_range, causal, scale, o, lse, r > 0)
+        else:
+            o_b = torch.empty_like(out)
+            lse_b = torch.empty_like(lse)
+            compute(q, kk, vv, q_range, kv_range, causal, scale, o_b, lse_b, False)
+            merge(o, lse, o_b, lse_b, out)
+        if stage and cuda and r >= 1:
+            used[(r - 1) % n_buf].record(main)
+        _nvtx_pop(q)
+    if stage and cuda:
+        main.wait_stream(side)
     kv.release()
     return out, lse
 

@@ -453,6 +453,13 @@ cp_status cp_peer_import(const cp_peer_handle *h, void **ptr);
  * Errors: CP_ERR_INVALID_ARG when `h` is not mapped on the current device. */
 cp_status cp_peer_close(const cp_peer_handle *h);
 
+/* Queues on `stream` a copy of `bytes` from `src` (typically a block mapped with
+ * cp_peer_import) to `dst` (device memory of the current device), done by the copy
+ * engines (cudaMemcpyAsync, device to device), so a block read by many CTAs crosses
+ * the link between GPUs once.  Errors: CP_ERR_INVALID_ARG for NULL pointers with
+ * bytes > 0; CP_ERR_CUDA when the copy cannot be queued. */
+cp_status cp_peer_copy(void *dst, const void *src, size_t bytes, void *stream);
+
 /* Bytes of device scratch the library reserves for cp_ring_attn_fwd_static_scratch. */
 #define CP_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
 

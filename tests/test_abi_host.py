@@ -388,8 +388,9 @@ def test_block_bwd_argument_errors_are_synchronous(cp):
 
 
 def test_peer_calls_reject_null_arguments(cp):
-    """cp_peer_export / cp_peer_import / cp_peer_close refuse NULL arguments before
-    any CUDA call; the handle struct has the layout the header declares."""
+    """cp_peer_export / cp_peer_import / cp_peer_close / cp_peer_copy refuse NULL
+    arguments before any CUDA call; the handle struct has the layout the header
+    declares."""
     from context_attention_cp_b200._binding import CpPeerHandle
     assert ctypes.sizeof(CpPeerHandle) == 64 + 8 + 8
     h = CpPeerHandle()
@@ -399,3 +400,5 @@ def test_peer_calls_reject_null_arguments(cp):
     assert cp.lib().cp_peer_import(ctypes.byref(h), None) == 1
     assert cp.lib().cp_peer_close(None) == 1
     assert b"NULL" in cp.lib().cp_last_error()
+    assert cp.lib().cp_peer_copy(None, ctypes.c_void_p(0x1000), 16, None) == 1
+    assert cp.lib().cp_peer_copy(None, None, 0, None) == 0   # nothing to copy: no CUDA call

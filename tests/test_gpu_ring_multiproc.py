@@ -120,10 +120,13 @@ def _peer_worker(rank, world, port, layout, S, out):
         p = pos.numpy()
         errs, gerrs = [], []
         f = lambda t: t.detach().double().cpu().numpy()  # noqa: E731
-        for k_scale in (1.0, 2.0):  # the blocks rewritten between two calls (x2 is exact in bf16)
+        # the blocks rewritten between two calls (x2 is exact in bf16); the first call
+        # pulls each peer block into a local buffer one step ahead, the second reads it
+        # in place
+        for k_scale, stage in ((1.0, True), (2.0, False)):
             kv.local[0].copy_((kl * k_scale).cuda())
             kv.local[1].copy_(vl.cuda())
-            o, lse = ring_dist.ring_attn_fwd_peer(ql.cuda(), kv, layout, True)
+            o, lse = ring_dist.ring_attn_fwd_peer(ql.cuda(), kv, layout, True, stage=stage)
             B.stream_check()
             k64 = k.double().numpy() * k_scale
             want_o, want_l = oracle.attention(q.double().numpy(), k64, v.double().numpy(), True, d ** -0.5)
@@ -142,12 +145,15 @@ def _peer_worker(rank, world, port, layout, S, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 1024), ("striped", 4, 1024), ("zigzag", 4, 2048)])
+@pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 1024), ("striped", 4, 1024), ("zigzag", 4, 2048),
+                                            ("contiguous", 3, 1536)])
 def test_peer_ring_processes_share_one_gpu(layout, world, S):
     """The in-place ring (ring_dist.ring_attn_fwd_peer, ring_attn_bwd_peer): each
     process maps the other processes' K/V blocks and dK/dV accumulators
-    (cp_peer_export / cp_peer_import, CUDA IPC); its block kernels read the K/V and
-    add into the accumulators where they lie; no block is copied or sent.  The processes
+    (cp_peer_export / cp_peer_import, CUDA IPC); the forward pulls each peer block
+    into a local double buffer one step ahead (cp_peer_copy on a copy stream) or
+    reads it in place, and the backward's kernels read the K/V and add into the
+    accumulators where they lie; no rank sends anything.  The processes
     share cuda:0, so the mapped memory is the same GPU's: this checks the mapping,
     the schedule and the kernels, not NVLink.  No kernel waits on another process:
     the ranks meet only on the host (publish / release)."""

@@ -250,11 +250,13 @@ def _peer_worker(rank, world, port, layout, S, out):
 
         kv = ring_dist.PeerBlocks([kl.shape, vl.shape], kl.dtype, "cpu")
         errs = []
-        for scale in (0.35, 0.2):             # two calls over the same blocks, rewritten between them
+        # two calls over the same blocks, rewritten between them: the first pulls each
+        # peer block into a local buffer one step ahead, the second reads it in place
+        for scale, stage in ((0.35, True), (0.2, False)):
             kv.local[0].copy_(kl * (scale / 0.35))
             kv.local[1].copy_(vl)
             seen.clear()
-            o, lse = ring_dist.ring_attn_fwd_peer(ql, kv, layout, True, 0.35, compute=oracle_step,
+            o, lse = ring_dist.ring_attn_fwd_peer(ql, kv, layout, True, 0.35, stage=stage, compute=oracle_step,
                                                   merge=_oracle_merge)
             want_o, want_l = oracle.ring_attention(q, k * (scale / 0.35), v, layout, world, True, 0.35, nthreads=1)
             errs.append((float(np.max(np.abs(o.numpy() - want_o[:, pos]))),
@@ -267,12 +269,14 @@ def _peer_worker(rank, world, port, layout, S, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 32), ("striped", 3, 24), ("zigzag", 4, 64)])
+@pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 32), ("striped", 3, 24), ("zigzag", 4, 64),
+                                            ("contiguous", 5, 40)])
 def test_peer_ring_over_gloo_ranks(layout, world, S):
     """The in-place ring (ring_attn_fwd_peer): no block moves between steps; step r
-    reads rank (i - r) mod N's K/V block where it lies (on CPU ranks the blocks live
-    in shared memory that every rank opens, standing in for the device mapping),
-    twice over blocks rewritten between the calls."""
+    attends to rank (i - r) mod N's K/V block, pulled into a local double buffer one
+    step ahead or read where it lies (on CPU ranks the blocks live in shared memory
+    that every rank opens, standing in for the device mapping), twice over blocks
+    rewritten between the calls; 5 ranks cycle the two buffers twice."""
     port = 29550 + (os.getpid() + world * 5 + S) % 900
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
