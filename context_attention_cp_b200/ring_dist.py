@@ -259,7 +259,8 @@ class PeerBlocks:
 
     def close(self):
         """release(), then every rank drops its mappings of the others' blocks before
-        any block is freed."""
+        any block is freed.  Tensors taken from `views` or `local` must not be used
+        after close(): the memory behind them is unmapped or freed."""
         self.release()
         for h in self._handles:
             B.peer_close(h)
