@@ -402,3 +402,17 @@ def test_peer_calls_reject_null_arguments(cp):
     assert b"NULL" in cp.lib().cp_last_error()
     assert cp.lib().cp_peer_copy(None, ctypes.c_void_p(0x1000), 16, None) == 1
     assert cp.lib().cp_peer_copy(None, None, 0, None) == 0   # nothing to copy: no CUDA call
+
+
+def test_peer_import_checks_size_and_dtype_before_mapping(cp):
+    """peer_import refuses a view larger than the exported block and an unsupported
+    dtype before it maps anything (no CUDA call)."""
+    import torch
+
+    from context_attention_cp_b200._binding import CpPeerHandle
+    h = CpPeerHandle()
+    h.offset, h.bytes = 0, 64
+    with pytest.raises(ValueError):
+        cp.peer_import(bytes(h), (1, 16, 1, 2), torch.float32)      # 128 bytes asked, 64 held
+    with pytest.raises(TypeError):
+        cp.peer_import(bytes(h), (1, 4, 1, 2), torch.float16)
