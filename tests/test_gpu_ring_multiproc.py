@@ -92,7 +92,7 @@ def test_ring_dist_processes_share_one_gpu(layout, world, S):
         assert max(e["dq"], e["dk"], e["dv"]) <= 2e-2, errs       # the tensor-core backward bar
 
 
-def _peer_worker(rank, world, port, layout, S, out):
+def _peer_worker(rank, world, port, layout, S, causal, out):
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
@@ -120,55 +120,61 @@ def _peer_worker(rank, world, port, layout, S, out):
         p = pos.numpy()
         errs, gerrs = [], []
         f = lambda t: t.detach().double().cpu().numpy()  # noqa: E731
-        # the blocks rewritten between two calls (x2 is exact in bf16); the first call
-        # pulls each peer block into a local buffer one step ahead, the second reads it
-        # in place
-        for k_scale, stage in ((1.0, True), (2.0, False)):
+        # the blocks rewritten between two calls (x2 is exact in bf16); each forward runs
+        # twice, pulling the peer blocks into local buffers one step ahead and reading
+        # them in place: the same kernels on the same bytes, so the results must agree
+        # bit for bit
+        same = True
+        for k_scale in (1.0, 2.0):
             kv.local[0].copy_((kl * k_scale).cuda())
             kv.local[1].copy_(vl.cuda())
-            o, lse = ring_dist.ring_attn_fwd_peer(ql.cuda(), kv, layout, True, stage=stage)
+            o, lse = ring_dist.ring_attn_fwd_peer(ql.cuda(), kv, layout, causal, stage=True)
+            o2, lse2 = ring_dist.ring_attn_fwd_peer(ql.cuda(), kv, layout, causal, stage=False)
             B.stream_check()
+            same = same and torch.equal(o, o2) and torch.equal(lse, lse2)
             k64 = k.double().numpy() * k_scale
-            want_o, want_l = oracle.attention(q.double().numpy(), k64, v.double().numpy(), True, d ** -0.5)
+            want_o, want_l = oracle.attention(q.double().numpy(), k64, v.double().numpy(), causal, d ** -0.5)
             errs.append((float(np.max(np.abs(f(o) - want_o[:, p]))), float(np.max(np.abs(f(lse) - want_l[:, :, p])))))
             # the backward adds into the owners' dK, dV accumulators where they lie
-            dq, dk, dv = ring_dist.ring_attn_bwd_peer(ql.cuda(), kv, o, lse, dol.cuda(), layout, True, acc=acc)
+            dq, dk, dv = ring_dist.ring_attn_bwd_peer(ql.cuda(), kv, o, lse, dol.cuda(), layout, causal, acc=acc)
             B.stream_check()
-            wg = oracle.attention_bwd(q.double().numpy(), k64, v.double().numpy(), do.double().numpy(), True,
+            wg = oracle.attention_bwd(q.double().numpy(), k64, v.double().numpy(), do.double().numpy(), causal,
                                       d ** -0.5)[:3]
             gerrs.append([float(np.max(np.abs(f(g) - w[:, p])) / np.max(np.abs(w))) for g, w in zip((dq, dk, dv), wg)])
         acc.close()
         kv.close()
-        out[rank] = (errs, gerrs, mapped)
+        out[rank] = (errs, gerrs, mapped, same)
         dist.barrier()
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 1024), ("striped", 4, 1024), ("zigzag", 4, 2048),
-                                            ("contiguous", 3, 1536)])
-def test_peer_ring_processes_share_one_gpu(layout, world, S):
+@pytest.mark.parametrize("layout,world,S,causal", [("zigzag", 2, 1024, True), ("striped", 4, 1024, True),
+                                                   ("zigzag", 4, 2048, True), ("contiguous", 3, 1536, True),
+                                                   ("contiguous", 2, 1024, False)])
+def test_peer_ring_processes_share_one_gpu(layout, world, S, causal):
     """The in-place ring (ring_dist.ring_attn_fwd_peer, ring_attn_bwd_peer): each
     process maps the other processes' K/V blocks and dK/dV accumulators
     (cp_peer_export / cp_peer_import, CUDA IPC); the forward pulls each peer block
     into a local double buffer one step ahead (cp_peer_copy on a copy stream) or
-    reads it in place, and the backward's kernels read the K/V and add into the
-    accumulators where they lie; no rank sends anything.  The processes
+    reads it in place -- bit for bit the same result -- and the backward's kernels
+    read the K/V and add into the accumulators where they lie; no rank sends
+    anything.  The processes
     share cuda:0, so the mapped memory is the same GPU's: this checks the mapping,
     the schedule and the kernels, not NVLink.  No kernel waits on another process:
     the ranks meet only on the host (publish / release)."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     import torch.multiprocessing as mp
-    port = 29300 + (os.getpid() + world * 13 + S) % 250
+    port = 29300 + (os.getpid() + world * 13 + S + int(causal)) % 250
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.start_processes(_peer_worker, args=(world, port, layout, S, out), nprocs=world, start_method="spawn",
+    mp.start_processes(_peer_worker, args=(world, port, layout, S, causal, out), nprocs=world, start_method="spawn",
                        join=True)
     assert sorted(out.keys()) == list(range(world))
     res = dict(out)
-    for rank, (errs, gerrs, mapped) in res.items():
-        assert mapped, res
+    for rank, (errs, gerrs, mapped, same) in res.items():
+        assert mapped and same, res
         for err_o, err_l in errs:
             assert err_o <= 2e-2 and err_l <= 1e-3, res   # the bf16 forward bar
         for g in gerrs:
