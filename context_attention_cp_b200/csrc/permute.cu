@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const __grid_constant
     }
 }
 
-// 4-byte rows (the fp32 LSE, sequence last): a thread moves groups of 4 consecutive
+// 4-byte rows (the fp32 LSE, sequence last) in general: a thread moves groups of 4 consecutive
 // ranked rows, one 16-byte access on the ranked side.  The launcher sends only
 // sequences whose rank length c and zig-zag chunk length c / 2 are multiples of 4, so
 // a group never straddles a rank or a chunk and its positions are pos0 + u * stride,
@@ -148,6 +148,66 @@ __global__ void __launch_bounds__(256) permute_words_kernel(const __grid_constan
                 dst[orig[u] + s1] = v[u].y;
                 dst[orig[u] + 2 * s1] = v[u].z;
                 dst[orig[u] + 3 * s1] = v[u].w;
+            }
+        }
+    }
+}
+
+// The same copy when every segment of every rank (c rows; c / 2 for zig-zag) is a
+// multiple of kSpanRows: a CTA takes a span of kSpanRows consecutive ranked rows,
+// which then lies inside one segment of one rank, so the span's first position is
+// decoded once per thread and its rows sit at pos0 + x * stride; each thread moves
+// kWordUnroll groups of 4 rows, all loaded before any is stored.
+constexpr int kSpanRows = 256 * 4 * kWordUnroll;
+
+template <typename I>
+__global__ void __launch_bounds__(256) permute_words_span_kernel(const __grid_constant__ PermuteParams p)
+{
+    // I: int32_t when outer * seq fits, else int64_t
+    const I seq = (I)p.seq;
+    const I c = seq / p.n_ranks;
+    const I spans_per_seq = seq / kSpanRows;
+    const I n_spans = (I)p.outer * spans_per_seq;
+    const uint32_t *src = static_cast<const uint32_t *>(p.src);
+    uint32_t *dst = static_cast<uint32_t *>(p.dst);
+    for (I sp = (I)blockIdx.x; sp < n_spans; sp += (I)gridDim.x) {
+        const I o = sp / spans_per_seq;
+        const I rr0 = (sp - o * spans_per_seq) * kSpanRows;
+        const int rank = (int)(rr0 / c);
+        const RangeT<I> r = layout_range_t<I>(p.layout, p.n_ranks, seq, rank);
+        const int64_t base = (int64_t)o * seq;
+        const int64_t ranked0 = base + rr0;
+        const int64_t orig0 = base + range_pos(r, rr0 - (I)rank * c);
+        const int64_t st = r.stride;
+        uint4 v[kWordUnroll];
+#pragma unroll
+        for (int u = 0; u < kWordUnroll; ++u) {
+            const int64_t x = 4 * ((int64_t)u * 256 + threadIdx.x);  // row offset inside the span
+            if (p.inverse) {
+                v[u] = *reinterpret_cast<const uint4 *>(src + ranked0 + x);
+            } else if (st == 1) {
+                v[u] = *reinterpret_cast<const uint4 *>(src + orig0 + x);
+            } else {
+                const int64_t a = orig0 + x * st;
+                v[u].x = src[a];
+                v[u].y = src[a + st];
+                v[u].z = src[a + 2 * st];
+                v[u].w = src[a + 3 * st];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kWordUnroll; ++u) {
+            const int64_t x = 4 * ((int64_t)u * 256 + threadIdx.x);
+            if (!p.inverse) {
+                *reinterpret_cast<uint4 *>(dst + ranked0 + x) = v[u];
+            } else if (st == 1) {
+                *reinterpret_cast<uint4 *>(dst + orig0 + x) = v[u];
+            } else {
+                const int64_t a = orig0 + x * st;
+                dst[a] = v[u].x;
+                dst[a + st] = v[u].y;
+                dst[a + 2 * st] = v[u].z;
+                dst[a + 3 * st] = v[u].w;
             }
         }
     }
@@ -273,6 +333,16 @@ cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream)
     }
     const int64_t c_rank = p.n_ranks > 0 ? p.seq / p.n_ranks : 0;
     const bool groups_aligned = c_rank % 4 == 0 && (p.layout != LAYOUT_ZIGZAG || (c_rank / 2) % 4 == 0);
+    const int64_t seg = p.layout == LAYOUT_ZIGZAG ? c_rank / 2 : c_rank;
+    if (CP_PERMUTE_ROWS && p.inner_bytes == 4 && seg > 0 && seg % kSpanRows == 0 && al % 16 == 0) {
+        const int64_t spans = rows / kSpanRows;
+        const int64_t blocks = spans < (int64_t)sms * 16 ? spans : (int64_t)sms * 16;
+        if (rows + (int64_t)sms * 16 * kSpanRows <= INT32_MAX)
+            permute_words_span_kernel<int32_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        else
+            permute_words_span_kernel<int64_t><<<(unsigned)blocks, 256, 0, stream>>>(p);
+        return cudaGetLastError();
+    }
     if (CP_PERMUTE_ROWS && p.inner_bytes == 4 && p.seq % 4 == 0 && groups_aligned && al % 16 == 0) {
         const int64_t groups = rows / 4;
         int64_t blocks = (groups + 256 * kWordUnroll - 1) / (256 * kWordUnroll);

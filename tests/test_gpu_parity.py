@@ -178,14 +178,16 @@ def test_permute_long_rows_bit_exact(cp, layout, N, S, H, d, dt):
 
 
 @pytest.mark.parametrize("layout", L.LAYOUTS)
-@pytest.mark.parametrize("N,S", [(4, 24), (3, 18), (8, 4096), (2, 8)])
-def test_permute_lse_rows_bit_exact(cp, layout, N, S):
+@pytest.mark.parametrize("N,S,H", [(4, 24, 5), (3, 18, 5), (8, 4096, 5), (2, 8, 5), (2, 16384, 5), (4, 65536, 40)])
+def test_permute_lse_rows_bit_exact(cp, layout, N, S, H):
     """4-byte rows, sequence last, both directions: groups of 4 that straddle a
-    zig-zag chunk or a rank (S = 24 over 4 ranks: chunks of 3), S % 4 != 0."""
+    zig-zag chunk or a rank (S = 24 over 4 ranks: chunks of 3), S % 4 != 0; rank
+    chunks that hold whole 4096-row spans (S = 16384 over 2 ranks, and 65536 over 4
+    with 3 x 40 rows: more spans than the grid has CTAs)."""
     if layout == "zigzag" and S % (2 * N):
         pytest.skip("zig-zag needs S % 2N == 0")
     g = torch.Generator().manual_seed(7 * S + N)
-    lse = torch.randn((3, 5, S), generator=g)
+    lse = torch.randn((3, H, S), generator=g)
     want = L.permute(lse.view(torch.int32).numpy(), layout, N, axis=2)
     lr = cp.layout_permute(lse.cuda(), layout, N, seq_axis=2)
     assert np.array_equal(lr.cpu().view(torch.int32).numpy(), want)
