@@ -414,12 +414,13 @@ int32_t cp_abi_version(void);
 /* ---- Blocks of other ranks on one node (real ranks, one process per GPU) ----
  * Section Ring Attention: at ring step r rank i attends its Q to the K/V block that
  * rank (i - r) mod N started with, and the block travels from rank to rank.  Between
- * the processes of one node the blocks can stay where they are instead: every rank
- * maps the other ranks' K/V blocks into its own address space with these calls and
- * passes the mapped addresses to cp_block_attn_fwd, whose tile loads (plain TMA
- * loads, no multicast) then read the peer's memory directly -- over NVLink when it
- * lives on another GPU -- so the transfer overlaps the math inside the kernel and no
- * copy or collective sits on the data path.
+ * the processes of one node no rank needs to send: every rank maps the other ranks'
+ * blocks into its own address space with these calls, then either pulls the block of
+ * the next step into a local buffer (cp_peer_copy, copy engines, overlapped with the
+ * current step's kernel) or passes the mapped addresses to the block kernels
+ * directly (cp_block_attn_fwd / cp_block_attn_bwd: plain TMA tile loads, no
+ * multicast, and plain stores into a peer's dK, dV accumulators).  No collective
+ * sits on the data path.
  *
  * cp_peer_handle: `ipc` is the CUDA IPC handle of the device allocation holding a
  * block, `offset` the block's byte offset inside that allocation, `bytes` the bytes
