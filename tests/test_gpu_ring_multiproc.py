@@ -153,7 +153,7 @@ def _peer_worker(rank, world, port, layout, S, causal, out):
                                                    ("zigzag", 4, 2048, True), ("contiguous", 3, 1536, True),
                                                    ("contiguous", 2, 1024, False)])
 def test_peer_ring_processes_share_one_gpu(layout, world, S, causal):
-    """The in-place ring (ring_dist.ring_attn_fwd_peer, ring_attn_bwd_peer): each
+    """The ring without sends (ring_dist.ring_attn_fwd_peer, ring_attn_bwd_peer): each
     process maps the other processes' K/V blocks and dK/dV accumulators
     (cp_peer_export / cp_peer_import, CUDA IPC); the forward pulls each peer block
     into a local double buffer one step ahead (cp_peer_copy on a copy stream) or

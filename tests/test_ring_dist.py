@@ -272,7 +272,7 @@ def _peer_worker(rank, world, port, layout, S, out):
 @pytest.mark.parametrize("layout,world,S", [("zigzag", 2, 32), ("striped", 3, 24), ("zigzag", 4, 64),
                                             ("contiguous", 5, 40)])
 def test_peer_ring_over_gloo_ranks(layout, world, S):
-    """The in-place ring (ring_attn_fwd_peer): no block moves between steps; step r
+    """The ring without sends (ring_attn_fwd_peer): no rank sends a block; step r
     attends to rank (i - r) mod N's K/V block, pulled into a local double buffer one
     step ahead or read where it lies (on CPU ranks the blocks live in shared memory
     that every rank opens, standing in for the device mapping), twice over blocks
@@ -346,7 +346,7 @@ def _peer_bwd_worker(rank, world, port, layout, S, causal, out):
 @pytest.mark.parametrize("layout,world,S,causal", [("zigzag", 2, 32, True), ("striped", 3, 24, True),
                                                    ("zigzag", 4, 64, True), ("contiguous", 3, 24, False)])
 def test_peer_ring_backward_over_gloo_ranks(layout, world, S, causal):
-    """The in-place backward (ring_attn_bwd_peer): step r adds rank i's shares for
+    """The backward without sends (ring_attn_bwd_peer): step r adds rank i's shares for
     block (i - r) mod N into that block owner's dK, dV accumulators where they lie
     (shared memory on CPU ranks); the gradients of every rank equal the oracle's
     whole-sequence gradients, twice with the accumulators reused."""
