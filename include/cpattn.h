@@ -26,14 +26,17 @@
  *     [b, H, s] fp32 holding natural-log values.  Strides are in elements.
  *   - Ownership: the caller owns every buffer and the stream.  No entry point
  *     allocates device memory; no pointer is kept after return, apart from work
- *     already queued on `stream`.
+ *     already queued on `stream` and the mappings cp_peer_import makes (kept until
+ *     cp_peer_close).
  *   - Errors: argument problems are reported synchronously through the return
  *     value (and a message from cp_last_error()).  Device-side problems (a
  *     bounded wait that ran out, a CUDA launch error) are reported by
  *     cp_stream_check() or by the next call's return value.  Nothing throws.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
- *   - Thread-compatible: no global mutable state besides the per-device status
- *     word read by cp_stream_check() and the per-thread last-error message.
+ *   - Thread-compatible: the global state is the per-device status word read by
+ *     cp_stream_check(), the per-thread last-error message, and caches guarded by
+ *     locks (work orders per shape, the peer mappings of cp_peer_import, the static
+ *     scratch address per device).
  */
 #ifndef CPATTN_H
 #define CPATTN_H
