@@ -62,6 +62,17 @@ L2_FLUSH_BYTES = 256 << 20
 HOLD_CYCLES = 400_000
 
 
+def emit(line, args):
+    """Prints the JSON line; with --jsonl PATH also appends it to PATH (one record per
+    line, for keeping results across runs)."""
+    text = json.dumps(line)
+    print(text, flush=True)
+    path = getattr(args, "jsonl", None)
+    if path:
+        with open(path, "a") as f:
+            f.write(text + "\n")
+
+
 class L2Flush:
     """Empties the L2 of the timed call's data before each timed call.
 
@@ -251,7 +262,7 @@ def run_reference(args):
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    print(json.dumps(line), flush=True)
+    emit(line, args)
     return 0
 
 
@@ -629,7 +640,7 @@ def run_one_gpu(args):
         "clocks": clk,
     }
     line.update(extra)
-    print(json.dumps(line), flush=True)
+    emit(line, args)
     return 0
 
 
@@ -777,7 +788,7 @@ def run_dist(args, ring_kw=None, device=None, backend="nccl"):
             "gpu_launches": world * args.steps * (w_launches_dist(world)),
             "clocks": clk,
         }
-        print(json.dumps(line), flush=True)
+        emit(line, args)
     dist.barrier()
     dist.destroy_process_group()
     return 0
@@ -803,6 +814,7 @@ def main():
                     help="comma list of merge,configs,backward,allgather,ulysses; 'all' or 'none'")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=12.0)
+    ap.add_argument("--jsonl", default=None, help="also append the JSON line to this file")
     ap.add_argument("--ring", default="nccl", choices=["nccl", "peer"],
                     help="with --gpus N > 1: pass the K/V blocks with NCCL (nccl) or read them in place from the"
                          " other ranks' memory (peer)")

@@ -82,6 +82,30 @@ def test_reference_arm_line_on_rank_zero(monkeypatch, capsys):
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
+def test_reference_arm_appends_jsonl(monkeypatch, capsys, tmp_path):
+    """--jsonl PATH appends the printed line to PATH, one record per run."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "0")
+    path = tmp_path / "results.jsonl"
+
+    class A:
+        workload = "fp32_s256_contig2"
+        warmup = 3
+        steps = 1
+        gpus = 1
+        ref_seconds = 0.1
+        jsonl = str(path)
+
+    assert bench.run_reference(A()) == 0
+    assert bench.run_reference(A()) == 0
+    printed = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    stored = path.read_text().splitlines()
+    assert len(stored) == 2 and stored == printed
+    assert all(json.loads(ln)["impl"] == "reference" for ln in stored)
+
+
 def _dist_worker(rank, world, port, out, ring="nccl"):
     """bench.run_dist on gloo ranks with the oracle as the block and merge steps."""
     sys.path.insert(0, ROOT)
