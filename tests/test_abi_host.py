@@ -110,6 +110,42 @@ def test_tile_classes_match_brute_force(cp, layout, N, S, tile, causal):
             assert got == want, (i, j)
 
 
+def _random_range(draw_int, nseg):
+    """An increasing position map of one or two segments (the ABI's requirement)."""
+    stride = draw_int(1, 4)
+    len0, start0 = draw_int(1, 70), draw_int(0, 200)
+    if nseg == 1:
+        return (start0,), (len0,), stride
+    len1, gap = draw_int(1, 70), draw_int(1, 100)
+    return (start0, start0 + (len0 - 1) * stride + gap), (len0, len1), stride
+
+
+def _range_positions(r):
+    starts, lens, stride = r
+    return [s0 + t * stride for s0, n in zip(starts, lens) for t in range(n)]
+
+
+def test_tile_classes_of_random_ranges_match_brute_force(cp):
+    """The tile classifier the kernels walk with (FULL prefix, PARTIAL band, SKIP
+    rest), on random increasing position maps of one or two segments, strides 1-4,
+    ragged lengths and unequal query / key tile sizes, causal or not, against a
+    pair-by-pair brute force."""
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=300, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+    @given(data=st.data(), nq=st.integers(1, 2), nk=st.integers(1, 2), causal=st.booleans(),
+           tq=st.sampled_from([16, 32, 64, 128]), tk=st.sampled_from([16, 32, 64, 128]))
+    def check(data, nq, nk, causal, tq, tk):
+        draw_int = lambda lo, hi: data.draw(st.integers(lo, hi))  # noqa: E731
+        qr, kr = _random_range(draw_int, nq), _random_range(draw_int, nk)
+        pq, pk = _range_positions(qr), _range_positions(kr)
+        got = cp.tile_classes(qr, len(pq), kr, len(pk), causal, tq, tk)
+        assert got == _brute_classes(pq, pk, causal, tq, tk), (qr, kr, causal, tq, tk)
+
+    check()
+
+
 def test_tile_classes_zigzag_rectangles(cp):
     """Off-diagonal zig-zag steps need no mask: with tiles that divide c/2, no tile is
     partial unless j == i (section Zig-zag, the remark after the case table)."""
