@@ -65,6 +65,27 @@ def test_layout_range_matches_oracle(cp, layout, N, S):
         assert pos == L.rank_positions(layout, N, S, rank)
 
 
+def test_layout_range_random_sizes_match_oracle(cp):
+    """cp_layout_range against the oracle's integer maps for random rank counts
+    (1-16) and sequence lengths (multiples of N, of 2N for zig-zag); together the
+    ranks' positions are a permutation of 0 .. S-1."""
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=200, deadline=None)
+    @given(layout=st.sampled_from(L.LAYOUTS), N=st.integers(1, 16), m=st.integers(1, 40))
+    def check(layout, N, m):
+        S = m * N * (2 if layout == "zigzag" else 1)
+        seen = []
+        for rank in range(N):
+            got = _range_positions(cp.layout_range(layout, N, S, rank))
+            assert got == L.rank_positions(layout, N, S, rank), (layout, N, S, rank)
+            seen.extend(got)
+        assert sorted(seen) == list(range(S))
+
+    check()
+
+
 def test_layout_range_rejects(cp):
     with pytest.raises(cp.CPError) as e:
         cp.layout_range("contiguous", 3, 10, 0)
