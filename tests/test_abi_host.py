@@ -473,3 +473,25 @@ def test_peer_import_checks_size_and_dtype_before_mapping(cp):
         cp.peer_import(bytes(h), (1, 16, 1, 2), torch.float32)      # 128 bytes asked, 64 held
     with pytest.raises(TypeError):
         cp.peer_import(bytes(h), (1, 4, 1, 2), torch.float16)
+
+
+def test_allgather_workspace_holds_the_pages_full_kv_bytes(cp):
+    """The gathered K/V term of cp_allgather_workspace_bytes equals the page's full
+    K/V size (512 MiB for the 70B heads at 128K, 64 MiB with one KV head).  The rest
+    of the workspace (document tables) does not depend on n_kv, so the K/V term of
+    n_kv heads is (ws(n_kv) - ws(1)) * n_kv / (n_kv - 1) and that of one head
+    ws(n_kv) - ws(1) over n_kv - 1."""
+    rows = []
+    with open(os.path.join(ROOT, "tests", "golden", "allgather_kv_bytes.txt")) as f:
+        for ln in f:
+            if ln.strip() and not ln.startswith("#"):
+                rows.append([int(x) for x in ln.split()])
+    assert len(rows) == 2
+    (b, S, hkv, d, want8), (_, _, one, _, want1) = rows
+    assert one == 1
+    ws = {h: cp.allgather_workspace_bytes(8, 0, b, S, h, d, 1) for h in (1, hkv)}
+    per_head = (ws[hkv] - ws[1]) // (hkv - 1)
+    assert (ws[hkv] - ws[1]) % (hkv - 1) == 0
+    assert per_head * hkv == want8 == 2 * 2 * b * S * hkv * d
+    assert per_head == want1
+
