@@ -166,3 +166,15 @@ def test_run_dist_line_over_two_gloo_ranks(ring):
     assert d["config"]["workload"] == "fp32_s256_contig2" and d["config"]["N"] == 2
     assert d["e2e"]["h2d_bytes_per_step"] > 0 and d["e2e"]["value"] > 0
     assert d["config"]["ring"] == ring
+
+
+def test_headline_traffic_comes_from_a_capture_of_the_current_kernel():
+    """The bench line's roofline.traffic for the headline workload is read from the
+    committed ncu summary, and only while the forward kernel's sources hash to the
+    value recorded with the capture: a kernel change without a new capture reports
+    null, and this test flags that the summary needs refreshing."""
+    sys.path.insert(0, ROOT)
+    import bench
+    t = bench.profiled_traffic("llama3_70b_s128k_zigzag8")
+    assert t is not None and t > 4.8e9      # at least Q + K + V + O once
+    assert bench.profiled_traffic("no_such_workload") is None
