@@ -474,11 +474,15 @@ def peer_import(handle, shape, dtype):
         raise ValueError("the peer block holds %d bytes, %d asked for" % (h.bytes, nbytes))
     ptr = ctypes.c_void_p()
     _check(lib().cp_peer_import(ctypes.byref(h), ctypes.byref(ptr)))
-    # no device argument: the tensor stays on the device that holds the memory (a
-    # device argument naming another one would copy)
-    if dtype == torch.bfloat16:
-        return torch.as_tensor(_DeviceArray(ptr.value, shape, "<i2")).view(torch.bfloat16)
-    return torch.as_tensor(_DeviceArray(ptr.value, shape, "<f4"))
+    try:
+        # no device argument: the tensor stays on the device that holds the memory (a
+        # device argument naming another one would copy)
+        if dtype == torch.bfloat16:
+            return torch.as_tensor(_DeviceArray(ptr.value, shape, "<i2")).view(torch.bfloat16)
+        return torch.as_tensor(_DeviceArray(ptr.value, shape, "<f4"))
+    except Exception:
+        lib().cp_peer_close(ctypes.byref(h))  # the mapping made above is not handed out
+        raise
 
 
 def peer_close(handle):
