@@ -208,6 +208,41 @@ def test_eight_keys_every_two_block_split():
             assert abs(lse[0] - math.log(math.exp(la) + math.exp(lb))) <= 1e-12
 
 
+def test_many_block_splits_merged_in_any_order():
+    """The ring folds N partials one after the other, in its own step order.  For
+    random partitions of up to 64 keys into up to 8 nonempty blocks (some empty
+    blocks too, lse = -inf), merging the blocks' partials one by one in a random
+    order, starting from the empty accumulator (0, -inf), gives one-shot softmax
+    (section 分块注意力: the split result equals the unsplit one, for any split)."""
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=150, deadline=None)
+    @given(n=st.integers(1, 64), nb=st.integers(1, 8), seed=st.integers(0, 2 ** 31 - 1))
+    def check(n, nb, seed):
+        r = np.random.default_rng(seed)
+        d = 3
+        qv = r.standard_normal(d) * 2.0
+        keys = r.standard_normal((n, d)) * 2.0
+        vals = r.standard_normal((n, d))
+        scale = 1 / math.sqrt(d)
+        full_o, full_lse = _partial(qv, keys, vals, list(range(n)), scale)
+        owner = r.integers(0, nb, n)           # block of each key; a block may stay empty
+        order = r.permutation(nb)
+        acc_o, acc_l = np.zeros((1, d)), np.array([-np.inf])
+        for blk in order:
+            idx = [t for t in range(n) if owner[t] == blk]
+            if idx:
+                ob, lb = _partial(qv, keys, vals, idx, scale)
+            else:
+                ob, lb = np.zeros(d), -np.inf
+            acc_o, acc_l = oracle.lse_merge(acc_o, acc_l, ob[None], np.array([lb]))
+        assert np.max(np.abs(acc_o[0] - full_o)) <= 1e-12
+        assert abs(acc_l[0] - full_lse) <= 1e-12
+
+    check()
+
+
 def test_merge_weights_sum_to_one():
     """o_1 = o_2 = 1 returns e^{lse_1-lse} + e^{lse_2-lse}, which must be 1; o_1 = 1,
     o_2 = 0 returns the first weight, e^{lse_1} / (e^{lse_1} + e^{lse_2})."""
